@@ -1,0 +1,135 @@
+/*
+ * kdn.h -- C ABI of the B200 (sm_100a) Diagonal Kalman Delta Network memory recurrence.
+ *
+ * The method (Kalman Delta Networks explainer, sections "把记忆问题重新想成一个滤波问题"
+ * and "对角近似"; aifromscratch "Kalman Delta Networks", "Approximation 1: Diagonal KDN";
+ * delta-rule tutorial "Память с поправкой"; KDA article "معماری KDA", per-channel decay):
+ * per head, with a memory S (d_k x d_v, read as S^T k), a per-channel key-space
+ * uncertainty P (d_k), and for every token t
+ *
+ *     P^-_t = alpha_t^2 * P_{t-1} + sigma_t                        (predict; diagonal stays diagonal)
+ *     g_t   = P^-_t * k_t / (r_t + sum_i P^-_{t,i} k_{t,i}^2)      (Kalman gain)
+ *     W     = diag(alpha_t) S_{t-1};  u_t = v_t - W^T k_t;  S_t = W + g_t u_t^T   (decayed delta write)
+ *     o_t   = S_t^T q_t                                            (readout after the write)
+ *     P_t   = P^-_t / (1 + mu * P^-_t * k_t^2 / r_t)               (mean-field projection, scaled by mu)
+ *
+ * Products and divisions of vectors are elementwise.  alpha in [0,1], sigma >= 0 and
+ * r > 0 are variances; mu > 0 scales the precision increment (1 = plain mean-field).
+ *
+ * Conventions shared by every entry point
+ *  - Memory: the caller owns every buffer; the library never allocates.  Pointers
+ *    marked "device" must be device memory of the current CUDA device; buffers must
+ *    not overlap unless stated.
+ *  - Layout: contiguous row-major.  Token tensors are [B, T, H, d] (dense batch) or
+ *    [1, T_total, H, d] with cu_seqlens (packed varlen); r is [B, T, H].  States are
+ *    per sequence: S [N, H, d_k, d_v] fp32, P [N, H, d_k] fp32, N = B or num_seqs.
+ *  - Types: token inputs and o are all fp32 or all bf16 (kdn_dtype_t); states fp32.
+ *  - Sizes: d_k in {32, 64, 128}, d_v in {32, 64, 128, 256}; other sizes return
+ *    KDN_ERR_UNSUPPORTED.  Empty problems (T == 0 or B == 0) are a no-op.
+ *  - Streams: every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream).  Argument validation is synchronous and returns an
+ *    error before anything is launched.  A failed launch returns KDN_ERR_CUDA.
+ *  - Device-side conditions (a bounded wait that gave up, an input outside the
+ *    tensor-core path's range) are recorded in a device error word and reported,
+ *    after a stream synchronisation, by kdn_last_device_error().
+ *  - Thread safety: calls may come from several host threads on different streams.
+ *    Calls that share output or state buffers must be ordered by the caller.
+ */
+#ifndef KDN_H_
+#define KDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDN_OK = 0,
+    KDN_ERR_INVALID_ARG = 1,   /* null pointer, bad size, non-monotone cu_seqlens (host copy), mu <= 0 */
+    KDN_ERR_UNSUPPORTED = 2,   /* d_k / d_v / chunk / dtype combination not built */
+    KDN_ERR_CUDA = 3,          /* a CUDA runtime call or a launch failed */
+    KDN_ERR_TIMEOUT = 4,       /* a bounded device wait gave up (kernel returned early) */
+    KDN_ERR_RANGE = 5,         /* a chunk's cumulative decay left the tensor-core path's range */
+    KDN_ERR_WORKSPACE = 6      /* workspace missing or smaller than kdn_workspace_size() */
+} kdn_status_t;
+
+typedef enum { KDN_DTYPE_F32 = 0, KDN_DTYPE_BF16 = 1 } kdn_dtype_t;
+
+/* Execution paths of kdn_forward_chunkwise (the `chunk` field):
+ *  0        token-serial fused recurrence (any dtype; exact fp32 arithmetic);
+ *  16/32/64 chunkwise: for bf16 inputs and chunk 64 the tcgen05 tensor-core kernel,
+ *           otherwise the fp32 CUDA-core chunk kernel (same algebra, fp32 FMA). */
+typedef struct {
+    int B, T, H, d_k, d_v;          /* varlen: B == 1 and T = total tokens */
+    const int32_t *cu_seqlens;      /* device int32 [num_seqs + 1], cu[0] = 0, cu[num_seqs] = T; NULL = dense batch */
+    int num_seqs;                   /* number of packed sequences; ignored (taken as B) when cu_seqlens == NULL */
+    kdn_dtype_t in_dtype;           /* dtype of q, k, v, alpha, sigma, r and o */
+    float mu;                       /* information scaling, > 0 */
+    int chunk;                      /* execution path, see above */
+} kdn_problem_t;
+
+/* Bytes of device workspace kdn_forward_chunkwise() and kdn_gain_scan() need for `p`
+ * (0 is possible).  Host-only; no CUDA call. */
+kdn_status_t kdn_workspace_size(const kdn_problem_t *p, size_t *bytes);
+
+/* Prefill / training forward over whole sequences (KDA article, "chunkwise" regime;
+ * explainer, "对角近似").
+ *  q, k, alpha, sigma : device [B, T, H, d_k]        (in_dtype)
+ *  v                  : device [B, T, H, d_v]        (in_dtype)
+ *  r                  : device [B, T, H]             (in_dtype)
+ *  S0, P0             : device fp32 [N, H, d_k, d_v], [N, H, d_k]; NULL -> S0 = 0, P0 = 1
+ *  o                  : device [B, T, H, d_v]        (in_dtype), written for every token
+ *  S_out, P_out       : device fp32, final states per sequence; either may be NULL.
+ *                       They may not alias S0 / P0.
+ *  workspace          : device, >= kdn_workspace_size() bytes, 256-byte aligned; its
+ *                       contents on entry do not matter.
+ * Every sequence starts from its own S0/P0 (chunks restart at sequence starts). */
+kdn_status_t kdn_forward_chunkwise(const kdn_problem_t *p,
+                                   const void *q, const void *k, const void *v,
+                                   const void *alpha, const void *sigma, const void *r,
+                                   const float *S0, const float *P0,
+                                   void *o, float *S_out, float *P_out,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* One autoregressive step for N independent sequences (KDA article, "fused
+ * recurrent kernel" regime): predict, gain, write, readout and uncertainty update
+ * of one token, with the state read from and written back to HBM in place.
+ *  q, k, alpha, sigma : device [N, H, d_k] (in_dtype);  v : device [N, H, d_v];  r : device [N, H]
+ *  S                  : device fp32 [N, H, d_k, d_v], updated in place
+ *  P                  : device fp32 [N, H, d_k], updated in place
+ *  o                  : device [N, H, d_v] (in_dtype) */
+kdn_status_t kdn_decode_step(int N, int H, int d_k, int d_v, kdn_dtype_t in_dtype, float mu,
+                             const void *q, const void *k, const void *v,
+                             const void *alpha, const void *sigma, const void *r,
+                             float *S, float *P, void *o, void *stream);
+
+/* The uncertainty / gain scan on its own (explainer, closing paragraph of "各向同性近似":
+ * the uncertainty recursion is a Moebius map whose 2x2 matrices compose, so it runs
+ * as an associative scan).  Independent of the memory S.
+ *  k, alpha, sigma : device [B, T, H, d_k];  r : device [B, T, H]   (in_dtype)
+ *  P0              : device fp32 [N, H, d_k] or NULL (ones)
+ *  g               : device fp32 [B, T, H, d_k], the gain of every token, or NULL
+ *  beta_eff        : device fp32 [B, T, H], k_t^T g_t (the effective write strength), or NULL
+ *  P_out           : device fp32 [N, H, d_k], uncertainty after the last token, or NULL
+ *  workspace       : as for kdn_forward_chunkwise (same size rule). */
+kdn_status_t kdn_gain_scan(const kdn_problem_t *p,
+                           const void *k, const void *alpha, const void *sigma, const void *r,
+                           const float *P0, float *g, float *beta_eff, float *P_out,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/* Synchronises `stream`, then returns and clears the device error word
+ * (KDN_ERR_TIMEOUT or KDN_ERR_RANGE if a kernel recorded one, else KDN_OK). */
+kdn_status_t kdn_last_device_error(void *stream);
+
+/* Static description of a status code. */
+const char *kdn_status_string(kdn_status_t s);
+
+/* Library version, e.g. "kdn-b200 0.1 sm_100a". */
+const char *kdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KDN_H_ */

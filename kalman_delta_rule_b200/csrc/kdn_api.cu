@@ -1,0 +1,163 @@
+// C ABI of libkdn.so: argument validation, workspace sizing, dispatch to the kernels,
+// and the device error word.  Declarations and the contract are in include/kdn.h.
+#include <math.h>
+#include <mutex>
+
+#include "kdn_common.cuh"
+#include "kdn_launch.h"
+
+namespace {
+
+__device__ unsigned g_kdn_err;  // bits kdn::ERR_*; one copy per device
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+unsigned *g_err_ptr[kMaxDevices];
+
+unsigned *err_word() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_err_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_kdn_err) != cudaSuccess) return nullptr;
+        g_err_ptr[dev] = static_cast<unsigned *>(p);
+    }
+    return g_err_ptr[dev];
+}
+
+bool dk_ok(int d) { return d == 32 || d == 64 || d == 128; }
+bool dv_ok(int d) { return d == 32 || d == 64 || d == 128 || d == 256; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Resolved {
+    long long ntok;
+    int nseq;
+    bool bf16;
+};
+
+kdn_status_t check_problem(const kdn_problem_t *p, Resolved *out) {
+    if (!p) return KDN_ERR_INVALID_ARG;
+    if (p->B < 0 || p->T < 0 || p->H <= 0) return KDN_ERR_INVALID_ARG;
+    if (!(p->mu > 0.f) || !isfinite(p->mu)) return KDN_ERR_INVALID_ARG;
+    if (p->in_dtype != KDN_DTYPE_F32 && p->in_dtype != KDN_DTYPE_BF16) return KDN_ERR_INVALID_ARG;
+    if (!dk_ok(p->d_k) || !dv_ok(p->d_v)) return KDN_ERR_UNSUPPORTED;
+    if (p->chunk != 0 && p->chunk != 16 && p->chunk != 32 && p->chunk != 64) return KDN_ERR_UNSUPPORTED;
+    if (p->cu_seqlens) {
+        if (p->B != 1 || p->num_seqs < 0) return KDN_ERR_INVALID_ARG;
+        out->nseq = p->num_seqs;
+    } else {
+        out->nseq = p->B;
+    }
+    out->ntok = (long long)p->B * p->T;
+    out->bf16 = p->in_dtype == KDN_DTYPE_BF16;
+    if (out->ntok > (1ll << 31) / 2) return KDN_ERR_UNSUPPORTED;
+    return KDN_OK;
+}
+
+kdn_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? KDN_OK : KDN_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *kdn_status_string(kdn_status_t s) {
+    switch (s) {
+        case KDN_OK: return "ok";
+        case KDN_ERR_INVALID_ARG: return "invalid argument";
+        case KDN_ERR_UNSUPPORTED: return "unsupported size, dtype or chunk";
+        case KDN_ERR_CUDA: return "CUDA runtime or launch error";
+        case KDN_ERR_TIMEOUT: return "a bounded device wait gave up";
+        case KDN_ERR_RANGE: return "chunk decay outside the tensor-core path's range";
+        case KDN_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+const char *kdn_version(void) { return "kdn-b200 0.1 sm_100a"; }
+
+kdn_status_t kdn_workspace_size(const kdn_problem_t *p, size_t *bytes) {
+    Resolved rv;
+    kdn_status_t st = check_problem(p, &rv);
+    if (st != KDN_OK) return st;
+    if (!bytes) return KDN_ERR_INVALID_ARG;
+    *bytes = 0;
+    return KDN_OK;
+}
+
+kdn_status_t kdn_forward_chunkwise(const kdn_problem_t *p, const void *q, const void *k, const void *v,
+                                   const void *alpha, const void *sigma, const void *r, const float *S0,
+                                   const float *P0, void *o, float *S_out, float *P_out, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
+    Resolved rv;
+    kdn_status_t st = check_problem(p, &rv);
+    if (st != KDN_OK) return st;
+    size_t need = 0;
+    kdn_workspace_size(p, &need);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return KDN_ERR_WORKSPACE;
+    if (rv.nseq == 0 || (rv.ntok == 0 && !S_out && !P_out)) return KDN_OK;
+    if (rv.ntok > 0 && (!q || !k || !v || !alpha || !sigma || !r || !o)) return KDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, alpha, sigma, r, o, S0, P0, S_out, P_out};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KDN_ERR_INVALID_ARG;
+    if ((S_out && S_out == S0) || (P_out && P_out == P0)) return KDN_ERR_INVALID_ARG;
+    if (!p->cu_seqlens && rv.nseq > 0 && p->T == 0 && !S_out && !P_out) return KDN_OK;
+
+    kdn::TokenArgs a{};
+    a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.sigma = sigma; a.r = r; a.o = o;
+    a.S0 = S0; a.P0 = P0; a.S_out = S_out; a.P_out = P_out;
+    a.cu = p->cu_seqlens; a.T = p->T; a.nseq = rv.nseq; a.H = p->H; a.dk = p->d_k; a.dv = p->d_v;
+    a.mu = p->mu; a.err = err_word();
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+
+    if (p->chunk == 0) {
+        const int dvt = p->d_v < 64 ? p->d_v : 64;
+        return cuda_status(kdn::launch_recurrent(a, rv.bf16, dvt, cs));
+    }
+    return cuda_status(kdn::launch_chunk_simt(a, rv.bf16, p->chunk, cs));
+}
+
+kdn_status_t kdn_decode_step(int N, int H, int d_k, int d_v, kdn_dtype_t in_dtype, float mu, const void *q,
+                             const void *k, const void *v, const void *alpha, const void *sigma, const void *r,
+                             float *S, float *P, void *o, void *stream) {
+    if (N < 0 || H <= 0 || !(mu > 0.f) || !isfinite(mu)) return KDN_ERR_INVALID_ARG;
+    if (in_dtype != KDN_DTYPE_F32 && in_dtype != KDN_DTYPE_BF16) return KDN_ERR_INVALID_ARG;
+    if (!dk_ok(d_k) || !dv_ok(d_v)) return KDN_ERR_UNSUPPORTED;
+    if (N == 0) return KDN_OK;
+    const void *ptrs[] = {q, k, v, alpha, sigma, r, S, P, o};
+    for (const void *ptr : ptrs)
+        if (!ptr || !aligned16(ptr)) return KDN_ERR_INVALID_ARG;
+    kdn::TokenArgs a{};
+    a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.sigma = sigma; a.r = r; a.o = o;
+    a.S0 = S; a.P0 = P; a.S_out = S; a.P_out = P;
+    a.cu = nullptr; a.T = 1; a.nseq = N; a.H = H; a.dk = d_k; a.dv = d_v; a.mu = mu; a.err = err_word();
+    // one tile per head: the in-place uncertainty is read and written by one CTA
+    return cuda_status(kdn::launch_recurrent(a, in_dtype == KDN_DTYPE_BF16, d_v, static_cast<cudaStream_t>(stream)));
+}
+
+kdn_status_t kdn_gain_scan(const kdn_problem_t *p, const void *k, const void *alpha, const void *sigma,
+                           const void *r, const float *P0, float *g, float *beta_eff, float *P_out,
+                           void *workspace, size_t workspace_bytes, void *stream) {
+    Resolved rv;
+    kdn_status_t st = check_problem(p, &rv);
+    if (st != KDN_OK) return st;
+    (void)k; (void)alpha; (void)sigma; (void)r; (void)P0; (void)g; (void)beta_eff; (void)P_out;
+    (void)workspace; (void)workspace_bytes; (void)stream;
+    return KDN_ERR_UNSUPPORTED;
+}
+
+kdn_status_t kdn_last_device_error(void *stream) {
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(cs) != cudaSuccess) return KDN_ERR_CUDA;
+    unsigned *ew = err_word();
+    if (!ew) return KDN_ERR_CUDA;
+    unsigned bits = 0;
+    if (cudaMemcpyAsync(&bits, ew, sizeof(bits), cudaMemcpyDeviceToHost, cs) != cudaSuccess) return KDN_ERR_CUDA;
+    if (cudaMemsetAsync(ew, 0, sizeof(unsigned), cs) != cudaSuccess) return KDN_ERR_CUDA;
+    if (cudaStreamSynchronize(cs) != cudaSuccess) return KDN_ERR_CUDA;
+    if (bits & kdn::ERR_TIMEOUT) return KDN_ERR_TIMEOUT;
+    if (bits & kdn::ERR_RANGE) return KDN_ERR_RANGE;
+    return KDN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,17 @@
+// Host-side launchers of the KDN kernels (internal to libkdn.so).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "kdn_common.cuh"
+
+namespace kdn {
+
+// token-serial fused recurrence; dvt = d_v tile per CTA (32/64/128/256, divides d_v)
+cudaError_t launch_recurrent(const TokenArgs &a, bool bf16_in, int dvt, cudaStream_t st);
+
+// chunkwise forward on CUDA cores in fp32 (chunk C <= 64); any dtype
+cudaError_t launch_chunk_simt(const TokenArgs &a, bool bf16_in, int C, cudaStream_t st);
+
+}  // namespace kdn

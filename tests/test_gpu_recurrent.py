@@ -1,0 +1,113 @@
+"""GPU parity of the fused recurrent kernel (prefill path chunk=0) and the decode step
+against the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+
+import oracle
+from kalman_delta_rule_b200 import inputs
+from tests.kdn_testutil import dense_shape, max_rel_err, oracle_chains, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32, TOL_BF16 = 1e-4, 2e-2
+
+
+def run_forward(kdn, w, chunk, mu=1.0, S0=None, P0=None):
+    import torch
+    args = [to_dev(dense_shape(w, getattr(w, n))) for n in ("q", "k", "v", "alpha", "sigma")]
+    r = to_dev(dense_shape(w, w.r))
+    cu = to_dev(w.cu_seqlens) if w.B == 1 and w.num_seqs > 1 else None
+    o, S, P = kdn.forward(*args, r, cu_seqlens=cu, S0=to_dev(S0), P0=to_dev(P0), mu=mu, chunk=chunk)
+    torch.cuda.synchronize()
+    kdn.last_device_error()
+    return to_host(o).reshape((-1,) + o.shape[2:]), to_host(S), to_host(P)
+
+
+@pytest.mark.parametrize("mu", [1.0, 32.0])
+def test_tiny_fp32_recurrent_matches_oracle(kdn, mu):
+    w = inputs.tiny_fp32()
+    ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens, mu=mu)
+    o, S, P = run_forward(kdn, w, chunk=0, mu=mu)
+    assert max_rel_err(o, ref["o"]) <= TOL_F32
+    assert max_rel_err(S, ref["S"]) <= TOL_F32
+    assert max_rel_err(P, ref["P"]) <= TOL_F32
+
+
+def ragged(seed, lens, H, dk, dv, bf16):
+    tok = inputs.draw_tokens(seed, int(sum(lens)), H, dk, dv, bf16)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return inputs.Workload(name="ragged", H=H, dk=dk, dv=dv, cu_seqlens=cu, bf16=bf16, B=1, T=int(sum(lens)), **tok)
+
+
+@pytest.mark.parametrize("dk,dv", [(32, 32), (64, 128), (128, 256), (128, 32)])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_ragged_varlen_recurrent(kdn, dk, dv, bf16):
+    w = ragged(100 + dk + dv, [1, 63, 64, 65, 130], 3, dk, dv, bf16)
+    rng = np.random.default_rng(1)
+    S0 = (0.1 * rng.standard_normal((w.num_seqs, w.H, dk, dv))).astype(np.float32)
+    P0 = rng.uniform(0.3, 2.0, (w.num_seqs, w.H, dk)).astype(np.float32)
+    ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens, S0=S0, P0=P0, mu=2.0)
+    o, S, P = run_forward(kdn, w, chunk=0, mu=2.0, S0=S0, P0=P0)
+    tol = TOL_BF16 if bf16 else TOL_F32
+    assert max_rel_err(o, ref["o"]) <= tol
+    assert max_rel_err(S, ref["S"]) <= tol
+    assert max_rel_err(P, ref["P"]) <= tol
+
+
+def test_empty_sequences_and_zero_tokens(kdn):
+    w = ragged(7, [5, 0, 3], 2, 32, 32, True)  # an empty sequence in the middle
+    S0 = np.random.default_rng(2).standard_normal((3, 2, 32, 32)).astype(np.float32)
+    ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens, S0=S0)
+    o, S, P = run_forward(kdn, w, chunk=0, S0=S0)
+    assert max_rel_err(o, ref["o"]) <= TOL_BF16
+    np.testing.assert_array_equal(S[1], S0[1])  # the empty sequence passes its state through
+    np.testing.assert_array_equal(P[1], 1.0)
+    assert max_rel_err(S, ref["S"]) <= TOL_BF16
+
+
+def decode_run(kdn, S0, P0, steps, bf16=True, mu=1.0):
+    import torch
+    S = to_dev(S0).clone()
+    P = to_dev(P0).clone()
+    outs = []
+    for st in steps:
+        o = kdn.decode_step(*[to_dev(st[n]) for n in ("q", "k", "v", "alpha", "sigma", "r")], S, P, mu=mu)
+        outs.append(to_host(o))
+    torch.cuda.synchronize()
+    kdn.last_device_error()
+    return np.stack(outs), to_host(S), to_host(P)
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 256), (32, 64)])
+@pytest.mark.parametrize("bf16", [True, False])
+def test_decode_small_matches_oracle(kdn, dk, dv, bf16):
+    N, H, n = 5, 3, 12
+    rng = np.random.default_rng(dk + dv)
+    S0 = (0.1 * rng.standard_normal((N, H, dk, dv))).astype(np.float32)
+    P0 = np.logaddexp(0, rng.standard_normal((N, H, dk))).astype(np.float32)
+    steps = [inputs.draw_tokens((9, s), N, H, dk, dv, bf16) for s in range(n)]
+    o, S, P = decode_run(kdn, S0, P0, steps, bf16, mu=1.5)
+    ref = oracle.run_decode(S0, P0, steps, mu=1.5)
+    tol = TOL_BF16 if bf16 else TOL_F32
+    assert max_rel_err(o, ref["o"]) <= tol
+    assert max_rel_err(S, ref["S"]) <= tol
+    assert max_rel_err(P, ref["P"]) <= tol
+
+
+def test_decode_full_size_sampled(kdn):
+    """The decode workload's launch configuration (256 sequences x 32 heads, d = 128,
+    fp32 state, bf16 inputs) for 16 steps; sampled (sequence, head) chains are checked
+    against the oracle element by element."""
+    w = inputs.decode_256x32()
+    n = 16
+    steps = [w.step(s) for s in range(n)]
+    o, S, P = decode_run(kdn, w.S0, w.P0, steps)
+    rng = np.random.default_rng(0)
+    picks = [(int(a), int(b)) for a, b in zip(rng.integers(0, w.N, 12), rng.integers(0, w.H, 12))]
+    picks += [(0, 0), (w.N - 1, w.H - 1)]
+    for (ns, h) in picks:
+        sub = [{nm: a[ns:ns + 1, h:h + 1] for nm, a in st.items()} for st in steps]
+        ref = oracle.run_decode(w.S0[ns:ns + 1, h:h + 1], w.P0[ns:ns + 1, h:h + 1], sub)
+        assert max_rel_err(o[:, ns, h], ref["o"][:, 0, 0]) <= TOL_BF16
+        assert max_rel_err(S[ns, h], ref["S"][0, 0]) <= TOL_BF16
+        assert max_rel_err(P[ns, h], ref["P"][0, 0]) <= TOL_BF16
