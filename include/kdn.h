@@ -119,6 +119,11 @@ kdn_status_t kdn_gain_scan(const kdn_problem_t *p,
                            const float *P0, float *g, float *beta_eff, float *P_out,
                            void *workspace, size_t workspace_bytes, void *stream);
 
+/* Which execution path kdn_forward_chunkwise() takes for `p` (host-only; no CUDA call
+ * besides resolving the driver's tensor-map encoder once): 0 token-serial recurrence,
+ * 1 fp32 CUDA-core chunk kernel, 2 tcgen05 tensor-core chunk kernel; -1 if `p` is invalid. */
+int kdn_execution_path(const kdn_problem_t *p);
+
 /* Synchronises `stream`, then returns and clears the device error word
  * (KDN_ERR_TIMEOUT or KDN_ERR_RANGE if a kernel recorded one, else KDN_OK). */
 kdn_status_t kdn_last_device_error(void *stream);

@@ -47,6 +47,7 @@ _SIGS = {
     "kdn_last_device_error": (_i, [_vp]),
     "kdn_status_string": (ctypes.c_char_p, [_i]),
     "kdn_version": (ctypes.c_char_p, []),
+    "kdn_execution_path": (_i, [_PP]),
 }
 
 
@@ -91,6 +92,10 @@ def kdn_gain_scan(problem, k, alpha, sigma, r, P0, g, beta_eff, P_out, workspace
 
 def kdn_last_device_error(stream=None) -> int:
     return load().kdn_last_device_error(stream)
+
+
+def kdn_execution_path(problem) -> int:
+    return load().kdn_execution_path(ctypes.byref(problem))
 
 
 def kdn_status_string(code: int) -> str:
@@ -204,6 +209,14 @@ def gain_scan(k, alpha, sigma, r, cu_seqlens=None, P0=None, mu: float = 1.0, chu
                        _ptr(workspace), wbytes, _stream_handle(stream))
     _check(st, "kdn_gain_scan")
     return g, be, P_out
+
+
+PATH_NAMES = {0: "recurrent", 1: "chunk_fp32", 2: "chunk_tcgen05"}
+
+
+def execution_path(q, v, cu_seqlens=None, mu: float = 1.0, chunk: int = 64) -> str:
+    """Name of the kernel path kdn_forward_chunkwise takes for these tensors."""
+    return PATH_NAMES.get(kdn_execution_path(make_problem(q, v, cu_seqlens=cu_seqlens, mu=mu, chunk=chunk)), "invalid")
 
 
 def last_device_error(stream=None):

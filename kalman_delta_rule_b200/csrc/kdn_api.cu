@@ -114,6 +114,11 @@ kdn_status_t kdn_forward_chunkwise(const kdn_problem_t *p, const void *q, const 
         const int dvt = p->d_v < 64 ? p->d_v : 64;
         return cuda_status(kdn::launch_recurrent(a, rv.bf16, dvt, cs));
     }
+    if (kdn::chunk_tc_supported(p->d_k, p->d_v, rv.bf16, p->chunk, rv.ntok)) {
+        const long long ctas128 = (long long)rv.nseq * p->H * (p->d_v / 128);
+        const int dvt = (p->d_v == 64 || ctas128 < 148) ? 64 : 128;
+        return cuda_status(kdn::launch_chunk_tc(a, rv.ntok, dvt, cs));
+    }
     return cuda_status(kdn::launch_chunk_simt(a, rv.bf16, p->chunk, cs));
 }
 
@@ -144,6 +149,13 @@ kdn_status_t kdn_gain_scan(const kdn_problem_t *p, const void *k, const void *al
     (void)k; (void)alpha; (void)sigma; (void)r; (void)P0; (void)g; (void)beta_eff; (void)P_out;
     (void)workspace; (void)workspace_bytes; (void)stream;
     return KDN_ERR_UNSUPPORTED;
+}
+
+int kdn_execution_path(const kdn_problem_t *p) {
+    Resolved rv;
+    if (check_problem(p, &rv) != KDN_OK) return -1;
+    if (p->chunk == 0) return 0;
+    return kdn::chunk_tc_supported(p->d_k, p->d_v, rv.bf16, p->chunk, rv.ntok) ? 2 : 1;
 }
 
 kdn_status_t kdn_last_device_error(void *stream) {

@@ -14,4 +14,8 @@ cudaError_t launch_recurrent(const TokenArgs &a, bool bf16_in, int dvt, cudaStre
 // chunkwise forward on CUDA cores in fp32 (chunk C <= 64); any dtype
 cudaError_t launch_chunk_simt(const TokenArgs &a, bool bf16_in, int C, cudaStream_t st);
 
+// chunkwise forward on tcgen05 tensor cores (bf16 inputs, d_k = 128, chunk 64)
+bool chunk_tc_supported(int dk, int dv, bool bf16_in, int chunk, long long ntok);
+cudaError_t launch_chunk_tc(const TokenArgs &a, long long ntok, int dvt, cudaStream_t st);
+
 }  // namespace kdn

@@ -1,0 +1,81 @@
+"""GPU parity of the tcgen05 tensor-core chunk kernel (bf16 inputs, d_k = 128,
+chunk 64) against the fp64 oracle: ragged tails, varlen, every d_v tile width,
+initial states, and the full-size workloads on sampled (sequence, head) chains."""
+import numpy as np
+import pytest
+
+import oracle
+from kalman_delta_rule_b200 import inputs
+from tests.kdn_testutil import dense_shape, max_rel_err, oracle_chains, to_dev, to_host
+from tests.test_gpu_recurrent import TOL_BF16, ragged, run_forward
+
+pytestmark = pytest.mark.gpu
+
+
+def path_of(kdn, w, chunk=64):
+    p = kdn.kdn_problem_t()
+    p.B = w.B or 1
+    p.T, p.H, p.d_k, p.d_v = w.ntok // p.B, w.H, w.dk, w.dv
+    p.cu_seqlens, p.num_seqs = None, p.B
+    p.in_dtype, p.mu, p.chunk = (1 if w.bf16 else 0), 1.0, chunk
+    return kdn.PATH_NAMES[kdn.kdn_execution_path(p)]
+
+
+@pytest.mark.parametrize("dv", [64, 128, 256])
+def test_tc_dense_ragged_tail(kdn, dv):
+    w = inputs.dense("tc_dense", 300 + dv, 2, 3, 200, 128, dv, bf16=True)   # 200 = 3 chunks + a tail of 8
+    assert path_of(kdn, w) == "chunk_tcgen05"
+    ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens)
+    o, S, P = run_forward(kdn, w, chunk=64)
+    assert max_rel_err(o, ref["o"]) <= TOL_BF16
+    assert max_rel_err(S, ref["S"]) <= TOL_BF16
+    assert max_rel_err(P, ref["P"]) <= TOL_BF16
+
+
+@pytest.mark.parametrize("mu", [1.0, 128.0])
+def test_tc_varlen_with_initial_state(kdn, mu):
+    w = ragged(77, [1, 63, 64, 65, 200, 130, 7], 2, 128, 128, True)
+    rng = np.random.default_rng(8)
+    S0 = (0.1 * rng.standard_normal((w.num_seqs, w.H, 128, 128))).astype(np.float32)
+    P0 = rng.uniform(0.3, 2.0, (w.num_seqs, w.H, 128)).astype(np.float32)
+    ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens, S0=S0, P0=P0, mu=mu)
+    o, S, P = run_forward(kdn, w, chunk=64, mu=mu, S0=S0, P0=P0)
+    assert max_rel_err(o, ref["o"]) <= TOL_BF16
+    assert max_rel_err(S, ref["S"]) <= TOL_BF16
+    assert max_rel_err(P, ref["P"]) <= TOL_BF16
+
+
+def sampled_check(kdn, w, picks, tol=TOL_BF16):
+    o, S, P = run_forward(kdn, w, chunk=64)
+    ref = oracle_chains(w, picks)
+    cu = w.cu_seqlens
+    for (s, h), rr in ref.items():
+        sl = slice(int(cu[s]), int(cu[s + 1]))
+        assert max_rel_err(o[sl, h], rr["o"]) <= tol, (s, h)
+        assert max_rel_err(S[s, h], rr["S"]) <= tol, (s, h)
+        assert max_rel_err(P[s, h], rr["P"]) <= tol, (s, h)
+
+
+def test_prefill_4x4096_full_size_sampled(kdn):
+    """B=4, H=16, T=4096, d=128, bf16, chunk 64 -- the benchmark's launch configuration."""
+    w = inputs.prefill_4x4096()
+    assert path_of(kdn, w) == "chunk_tcgen05"
+    rng = np.random.default_rng(1)
+    picks = [(0, 0), (3, 15)] + [(int(a), int(b)) for a, b in zip(rng.integers(0, 4, 6), rng.integers(0, 16, 6))]
+    sampled_check(kdn, w, sorted(set(picks)))
+
+
+def test_long_context_65536_full_size_sampled(kdn):
+    """B=1, H=32, T=65536 with repeated-key segments; two whole heads checked."""
+    w = inputs.long_context_65536()
+    sampled_check(kdn, w, [(0, 0), (0, 31)])
+
+
+def test_varlen_262144_full_size_sampled(kdn):
+    """262144 packed tokens, lengths U{512..16384}, H=16, d_k=128, d_v=256."""
+    w = inputs.varlen_262144()
+    lens = np.diff(w.cu_seqlens)
+    longest = int(np.argmax(lens))
+    shortest = int(np.argmin(lens))
+    picks = [(longest, 3), (shortest, 0), (w.num_seqs - 1, 15), (0, 7)]
+    sampled_check(kdn, w, picks)
