@@ -1,0 +1,452 @@
+#!/usr/bin/env python
+"""Benchmark of the Diagonal KDN memory recurrence on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill|long|varlen] [--no-cpu-baseline]
+
+Primary metric: prefill tokens/s of kdn_forward_chunkwise on the chunkwise-prefill
+workload (B=4, H=16, T=4096, d_k=d_v=128, bf16 inputs, fp32 state, chunk 64); a step
+is one forward over the whole batch (uncertainty/gain, chunk algebra, state carry and
+readout -- every step of the hot path), timed with CUDA events on the launching stream.
+The JSON line also carries the decode rate (steps/s on 256 sequences x 32 heads,
+d = 128, fp32 state, 1024 steps), each with its roofline fraction against the measured
+HBM copy bandwidth, the end-to-end rate through the C ABI with host buffers, and the
+fp64 oracle timed on the host cores.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own independent batch
+(weak scaling, no data-path collective); timings are the max over ranks.
+
+--impl reference times the fp64 CPU oracle (rank 0 only) on a bounded sample of the
+same workload per step.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def workload(name, seed_offset=0):
+    from kalman_delta_rule_b200 import inputs
+    if name == "prefill":
+        w = inputs.prefill_4x4096(seed=1 if not seed_offset else (1, seed_offset))
+    elif name == "long":
+        w = inputs.long_context_65536(seed=3 if not seed_offset else (3, seed_offset))
+    elif name == "varlen":
+        w = inputs.varlen_262144(seed=4 if not seed_offset else (4, seed_offset))
+    else:
+        raise ValueError(name)
+    return w
+
+
+def algorithmic_bytes(w, state_out=True):
+    """Bytes a forward must move at least: every input once, o once, final S and P."""
+    esz = 2 if w.bf16 else 4
+    per_tok_head = (4 * w.dk + 2 * w.dv) * esz + esz       # q, k, alpha, sigma, v, o, r
+    n = w.ntok * w.H * per_tok_head
+    if state_out:
+        n += w.num_seqs * w.H * (w.dk * w.dv + w.dk) * 4
+    return n
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the GPU is loaded."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        top = sorted(sm)[len(sm) // 4:] or sm   # under load: drop the idle tail
+        return {"sm_mhz": statistics.median(top), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    import torch
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ our arm
+def to_dev(a, dev):
+    import torch
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    if a.dtype == np.int32:
+        return torch.from_numpy(a).to(dev)
+    return torch.from_numpy(a.astype(np.float32)).to(dev)
+
+
+def bench_prefill(args, world, rank, dev, kdn):
+    import torch
+    w = workload(args.workload, seed_offset=rank)
+    B = w.B if w.B else 1
+    shp = lambda x: x.reshape((B, w.ntok // B) + x.shape[1:])
+    names = ("q", "k", "v", "alpha", "sigma", "r")
+    host = {n: shp(getattr(w, n)) for n in names}
+    d = {n: to_dev(host[n], dev) for n in names}
+    cu = to_dev(w.cu_seqlens, dev) if (w.B == 1 and w.num_seqs > 1) else None
+    o = torch.empty(d["q"].shape[:3] + (w.dv,), dtype=d["q"].dtype, device=dev)
+    S_out = torch.empty((w.num_seqs, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+    P_out = torch.empty((w.num_seqs, w.H, w.dk), dtype=torch.float32, device=dev)
+    prob = kdn.make_problem(d["q"], d["v"], cu_seqlens=cu, mu=w.mu, chunk=w.chunk)
+    ws_bytes = kdn.kdn_workspace_size(prob)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    path = kdn.PATH_NAMES[kdn.kdn_execution_path(prob)]
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kdn.forward(d["q"], d["k"], d["v"], d["alpha"], d["sigma"], d["r"], cu_seqlens=cu, mu=w.mu, chunk=w.chunk,
+                    o=o, S_out=S_out, P_out=P_out, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    kdn.last_device_error()
+    # sustained run for the clock record (same kernel, same inputs), then the timed region
+    with ClockSampler(dev.index) as clk:
+        t_end = time.time() + args.clock_seconds
+        while time.time() < t_end:
+            for _ in range(20):
+                step()
+            torch.cuda.synchronize()
+        barrier(world)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        evs[0].record(stream)
+        for i in range(args.steps):
+            step()
+            evs[i + 1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    kdn.last_device_error()
+    per_step_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
+    total_ms = evs[0].elapsed_time(evs[-1])
+    total_ms = max_over_ranks(total_ms, world)
+    ms_step = total_ms / args.steps
+    tokens = w.ntok  # per rank, all heads included
+    value = world * tokens * args.steps / (total_ms / 1e3)
+
+    # end to end through the C ABI: pinned host inputs -> device, forward, o -> host
+    pinned = {n: torch.from_numpy(np.ascontiguousarray(host[n]).view(np.int16) if host[n].dtype == np.uint16
+                                  else np.ascontiguousarray(host[n])).pin_memory() for n in names}
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = o_host.numel() * o_host.element_size()
+
+    def e2e_step():
+        for n in names:
+            dst = d[n].view(torch.int16) if d[n].dtype == torch.bfloat16 else d[n]
+            dst.copy_(pinned[n], non_blocking=True)
+        step()
+        o_host.copy_(o, non_blocking=True)
+
+    for _ in range(max(1, args.warmup // 2)):
+        e2e_step()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(3, min(args.steps, 10))
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = world * tokens * e_steps / (e2e_ms / 1e3)
+
+    nbytes = algorithmic_bytes(w)
+    return dict(w=w, value=value, ms_step=ms_step, per_step_ms=per_step_ms, clocks=clk.summary(), path=path,
+                e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
+                         steps=e_steps),
+                bytes=nbytes, launches=args.steps)
+
+
+def bench_decode(args, world, rank, dev, kdn, steps=1024, N=256, H=32, d=128):
+    """1024 decode steps on 256 sequences x 32 heads (inputs resident, drawn on the device)."""
+    import torch
+    g = torch.Generator(device=dev)
+    g.manual_seed(2_000 + rank)
+    S = 0.1 * torch.randn((N, H, d, d), generator=g, device=dev)
+    P = torch.nn.functional.softplus(torch.randn((N, H, d), generator=g, device=dev))
+    shape = (steps, N, H, d)
+    q = torch.nn.functional.normalize(torch.randn(shape, generator=g, device=dev), dim=-1).bfloat16()
+    k = torch.nn.functional.normalize(torch.randn(shape, generator=g, device=dev), dim=-1).bfloat16()
+    v = torch.randn(shape, generator=g, device=dev).bfloat16()
+    al = torch.sigmoid(torch.randn(shape, generator=g, device=dev) + 4.0).bfloat16()
+    r = (torch.nn.functional.softplus(torch.randn((steps, N, H), generator=g, device=dev)) + 1e-3).bfloat16()
+    sg = torch.nn.functional.softplus(torch.randn(shape, generator=g, device=dev) - 3.0).bfloat16()
+    o = torch.empty((N, H, d), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def run(n):
+        for s in range(n):
+            kdn.decode_step(q[s], k[s], v[s], al[s], sg[s], r[s], S, P, o=o)
+
+    run(min(steps, max(3, args.warmup)))
+    kdn.last_device_error()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run(steps)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    kdn.last_device_error()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    per_step = ms / steps
+    head_step_bytes = 2 * d * d * 4 + 2 * d * 4 + (4 * d + d) * 2 + 2 + d * 2
+    nbytes = N * H * head_step_bytes
+    return dict(value=world * steps / (ms / 1e3), ms_step=per_step, bytes=nbytes, steps=steps, N=N, H=H, d=d)
+
+
+def cpu_baseline_prefill(w, max_seconds=30.0):
+    """The fp64 oracle on the host cores over whole (sequence, head) chains of the workload."""
+    import oracle
+    cores = os.cpu_count() or 1
+    chains = [(s, h) for s in range(w.num_seqs) for h in range(w.H)]
+    # bounded sample: as many whole chains as fit ~max_seconds at ~0.5 s per chain-core
+    per_chain_tokens = w.ntok / w.num_seqs
+    est_chain_s = per_chain_tokens * 5 * w.dk * w.dv * 2 / 1.2e9
+    n = int(min(len(chains), max(cores, cores * max_seconds / max(est_chain_s, 1e-3))))
+    n = max(1, min(n, len(chains)))
+    pick = chains[:n]
+    t0 = time.perf_counter()
+    oracle.diag_chains(w, pick, threads=cores)
+    dt = time.perf_counter() - t0
+    tok = sum(int(w.cu_seqlens[s + 1] - w.cu_seqlens[s]) for s, _ in pick) / w.H
+    return {"value": tok / dt, "unit": "tokens/s", "cores": min(cores, n), "kind": "oracle",
+            "sample": f"{n} of {len(chains)} (sequence, head) chains of the workload, whole length, fp64 C oracle, "
+                      f"{dt:.1f} s wall"}
+
+
+def kernel_hash():
+    h = hashlib.sha1()
+    for fn in ("kdn_chunk_tc.cu", "kdn_tc.cuh", "kdn_common.cuh"):
+        with open(os.path.join(ROOT, "kalman_delta_rule_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic(workload_name):
+    """dram bytes per launch from the committed ncu summary, if taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    cur = kernel_hash()
+    for line in open(p):
+        parts = line.split()
+        if len(parts) >= 3 and not line.startswith("#") and parts[0] == workload_name and parts[2] == cur:
+            return float(parts[1])
+    return None
+
+
+def ours(args):
+    import torch
+    from kalman_delta_rule_b200 import binding as kdn
+    kdn.load()
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    pk, pk_kind = peaks()
+    pre = bench_prefill(args, world, rank, dev, kdn)
+    dec = bench_decode(args, world, rank, dev, kdn, steps=args.decode_steps) if not args.no_decode else None
+    w = pre["w"]
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_prefill(w)
+    if rank == 0:
+        kern_s = statistics.mean(pre["per_step_ms"]) / 1e3
+        ach = pre["bytes"] / kern_s / 1e9
+        hbm = float(pk["hbm_gbs"])
+        traffic = recorded_traffic(w.name)
+        line = {
+            "metric": "KDN prefill tokens/s + decode steps/s on 1 B200; % of HBM/tensor roofline",
+            "value": pre["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": pre["ms_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded; shapes and distributions of the workload recipe)",
+            "config": {"workload": w.name, "B": w.B, "T": w.ntok // (w.B or 1), "H": w.H, "d_k": w.dk, "d_v": w.dv,
+                       "chunk": w.chunk, "mu": w.mu, "state": "fp32", "kernel_path": pre["path"],
+                       "l2": f"inputs larger than L2 ({pre['bytes'] / 1e9:.2f} GB > 0.13 GB), no flush",
+                       "parallelism": f"replicas x{world} (independent batches, no collective)"},
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                         "traffic": traffic, "peak_kind": f"{pk_kind} copy bandwidth",
+                         "algorithmic_bytes_per_launch": pre["bytes"]},
+            "cpu_baseline": cpu,
+            "e2e": pre["e2e"],
+            "gpu_launches": pre["launches"],
+            "clocks": pre["clocks"],
+        }
+        if dec is not None:
+            dach = dec["bytes"] / (dec["ms_step"] / 1e3) / 1e9
+            line["decode"] = {"metric": "decode steps/s", "value": dec["value"], "unit": "steps/s",
+                              "ms_per_step": dec["ms_step"], "steps": dec["steps"],
+                              "workload": f"decode_N{dec['N']}_H{dec['H']}_d{dec['d']}_bf16_fp32state",
+                              "gpu_launches": dec["steps"],
+                              "roofline": {"bound": "hbm", "achieved": dach, "peak": hbm, "unit": "GB/s",
+                                           "frac": dach / hbm, "traffic": None,
+                                           "algorithmic_bytes_per_launch": dec["bytes"]}}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ reference arm (the oracle)
+def reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    w = workload(args.workload)
+    cores = os.cpu_count() or 1
+    n = max(1, min(cores, w.num_seqs * w.H, 8))
+    chains = [(s, h) for s in range(w.num_seqs) for h in range(w.H)][:n]
+    # each step: the oracle over n whole chains, cut to a bounded token count
+    max_tok = int(os.environ.get("KDN_REF_TOKENS", "1024"))
+
+    class Sub:
+        pass
+    sub = Sub()
+    for nm in ("q", "k", "v", "alpha", "sigma", "r"):
+        setattr(sub, nm, getattr(w, nm))
+    cu = np.array([0] + [min(int(w.cu_seqlens[s + 1] - w.cu_seqlens[s]), max_tok) for s in range(w.num_seqs)])
+    # rebuild a token array holding the first max_tok tokens of each sequence
+    idx = np.concatenate([np.arange(int(w.cu_seqlens[s]), int(w.cu_seqlens[s]) + cu[s + 1]) for s in range(w.num_seqs)])
+    for nm in ("q", "k", "v", "alpha", "sigma", "r"):
+        setattr(sub, nm, getattr(w, nm)[idx])
+    sub.cu_seqlens = np.concatenate([[0], np.cumsum(cu[1:])]).astype(np.int64)
+    sub.H, sub.mu = w.H, w.mu
+    for _ in range(args.warmup):
+        oracle.diag_chains(sub, chains[:1], threads=1)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.diag_chains(sub, chains, threads=cores)
+    dt = time.perf_counter() - t0
+    tok = sum(int(sub.cu_seqlens[s + 1] - sub.cu_seqlens[s]) for s, _ in chains) / w.H * args.steps
+    value = tok / dt
+    line = {"impl": "reference", "metric": "KDN prefill tokens/s + decode steps/s on 1 B200; % of HBM/tensor roofline",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic (seeded)",
+            "config": {"workload": w.name, "B": w.B, "T": w.ntok // (w.B or 1), "H": w.H, "d_k": w.dk, "d_v": w.dv,
+                       "chunk": w.chunk},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(cores, len(chains)), "kind": "oracle",
+                             "sample": f"per step: {len(chains)} (sequence, head) chains x first {max_tok} tokens"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="prefill", choices=["prefill", "long", "varlen"])
+    ap.add_argument("--clock-seconds", type=float, default=2.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=1024)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        reference(args)
+    else:
+        ours(args)
+
+
+if __name__ == "__main__":
+    main()

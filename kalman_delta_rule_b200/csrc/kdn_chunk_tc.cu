@@ -5,18 +5,18 @@
 //
 // One CTA owns one (sequence, head, d_v tile of DVT columns); d_k = 128, chunk C = 64.
 // Per chunk (local tokens t, s in [0, L)), with Gam_t = prod_{j<=t} alpha_j per channel
-// and the chunk's geometric-middle reference rho = Gam_{L-1}^{-1/2}:
+// (decay referenced to the chunk start) and den_t = r_t + sum_i P^-_{t,i} k_{t,i}^2:
 //   prep (independent of the memory S):
-//     uncertainty recursion and gain g_t (CUDA cores, thread = key channel)
-//     K~ = k Gam rho,  Q~ = q Gam rho,  G~ = g / (Gam rho),  G' = G~ Gam_{L-1}^{1/2}
-//     MMA1   [A; Aq] = [K~; Q~] G~^T                 -> A (s < t), Aq (s <= t)
+//     uncertainty recursion in four token quarters joined by the Moebius composites of
+//     the quarters' 2x2 maps (CUDA cores, thread = key-channel pair x quarter)
+//     K~ = k Gam,  Q~ = q Gam,  G^ = P^- k / Gam   (the gain is G^ Gam / den)
+//     MMA1   [A; Aq] = [K~; Q~] G^^T, columns scaled by 1/den  -> A (s < t), Aq (s <= t)
 //     T = (I + A)^{-1}                               (CUDA cores, blocked 16x16)
 //     MMA_X  X = Aq T                                (M = 64)
 //     MMA2   [w; X K~] = [T; X] K~ ,  Q' = Q~ - X K~
 //   serial (carries S in TMEM, fp32):
-//     S0' = Gam_{L-1}^{1/2} S (bf16 operand),  TMEM S <- Gam_{L-1} S
-//     MMA4   [U; O] = [-w; Q'] S0' + [T; X] V        (K = 128 + 64)
-//     MMA5   S += G'^T U
+//     MMA4   [U; O] = [-w; Q'] S + [T; X] V          (K = 128 + 64)
+//     MMA5   S += G^^T (U / den) ;  then S <- Gam_{L-1} S (rows)
 // which is the serial recurrence unrolled exactly: U = (I + A)^{-1}(V - K S0),
 // O = Q S0 + Aq U, S_next = Gam_{L-1} S0 + sum_s (Gam_{L-1}/Gam_s) g_s u_s^T.
 // The factored decay needs Gam_{L-1} >= 1e-30 per channel; a chunk outside that range
@@ -34,19 +34,18 @@ constexpr int C = 64, DK = 128, NT = 256;
 
 template <int DVT>
 struct TcSmem {
-    static constexpr uint32_t Q = 0;                        // q tile (TMA) 16 KB; later T fp32 [64][64]
-    static constexpr uint32_t K = Q + 16384;                // k tile (TMA) 16 KB; later A fp32 [64][64]
-    static constexpr uint32_t V = K + 16384;                // v tile (TMA) DVT*128 B
+    static constexpr uint32_t Q = 0;                        // q tile (TMA)
+    static constexpr uint32_t K = Q + 16384;                // k tile (TMA); then A fp32 [64][64]
+    static constexpr uint32_t AL = K + 16384;               // alpha tile (TMA); then Aq bf16 64 x 64
+    static constexpr uint32_t SG = AL + 16384;              // sigma tile (TMA); then T fp32 [64][64]
+    static constexpr uint32_t V = SG + 16384;               // v tile (TMA), DVT*128 B
     static constexpr uint32_t KQ = V + DVT * 128;           // [K~; Q~] bf16, K-major, 2 atoms of 128 rows
-    static constexpr uint32_t G = KQ + 32768;               // G~ bf16, 64 token rows x 128 ch
-    static constexpr uint32_t GP = G + 16384;               // alpha tile (TMA), turned into G' in place
-    static constexpr uint32_t AQ = GP + 16384;              // Aq bf16, 64 x 64
-    static constexpr uint32_t Y = AQ + 8192;                // [T; X] bf16, 128 x 64
-    static constexpr uint32_t A4 = Y + 16384;               // [-w; Q'] bf16 128 x 128; pass A: g numerators fp32
-    static constexpr uint32_t S = A4 + 32768;               // S0' bf16, 128 channel rows x DVT (MN-major)
-    static constexpr uint32_t U = S + DVT * 256;            // U bf16, 64 token rows x DVT (MN-major)
-    static constexpr uint32_t SIG = (DVT >= 128) ? U : U + DVT * 128;   // sigma tile (TMA) 16 KB
-    static constexpr uint32_t MISC = SIG + 16384;
+    static constexpr uint32_t G = KQ + 32768;               // G^ bf16, 64 token rows x 128 ch
+    static constexpr uint32_t Y = G + 16384;                // [T; X] bf16, 128 x 64
+    static constexpr uint32_t A4 = Y + 16384;               // [-w; Q'] bf16 128 x 128; prep: P^- k^2 fp32 [64][128]
+    static constexpr uint32_t S = A4 + 32768;               // S bf16, 128 channel rows x DVT (MN-major)
+    static constexpr uint32_t U = S + DVT * 256;            // U / den bf16, 64 token rows x DVT (MN-major)
+    static constexpr uint32_t MISC = U + DVT * 128;
     static constexpr uint32_t MISC_BYTES = 2048;
     static constexpr uint32_t total = MISC + MISC_BYTES;
     static constexpr uint32_t TMA_BYTES = 4 * 16384 + DVT * 128;
@@ -64,49 +63,79 @@ __device__ __forceinline__ void st_bf16(uint8_t *base, uint32_t off, float v) {
     *reinterpret_cast<__nv_bfloat16 *>(base + off) = __float2bfloat16_rn(v);
 }
 
-// T = (I + A)^{-1} for a strictly lower 64x64 fp32 A (row-major), blocked by 16.
+// fp32 64x64 tiles in shared memory: 4-float groups of a row are XOR-permuted by the row
+// index, so that column reads across rows and float4 row accesses are bank-conflict free.
+__device__ __forceinline__ int fsw(int r, int c) { return r * 64 + ((((c >> 2) ^ r) & 15) << 2) + (c & 3); }
+
+// T = (I + A)^{-1} for a strictly lower 64x64 fp32 A (fsw layout), blocked by 16:
+// the four 16x16 diagonal blocks by forward substitution, then block levels
+// T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj, each thread producing a 1x4 strip.
 // T's strictly-upper blocks are used as scratch; readers mask them out.
 __device__ void tri_inverse64(const float *A, float *T, int tid) {
-    if (tid < 64) {
+    if (tid < 64) {   // diagonal blocks: thread = (block, column), forward substitution
         const int o = (tid >> 4) * 16, j = tid & 15;
         float x[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
         for (int r = 1; r < 16; ++r) {
-            if (r > j) {
-                float acc = 0.f;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int s = 0; s < r; ++s)
-                    if (s >= j) acc = fmaf(A[(o + r) * 64 + o + s], x[s], acc);
-                x[r] = -acc;
-            }
+            for (int s = 0; s < r; ++s) acc[s & 3] = fmaf(A[fsw(o + r, o + s)], x[s], acc[s & 3]);
+            if (r > j) x[r] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) T[(o + r) * 64 + o + j] = x[r];
+        for (int r = 0; r < 16; ++r) T[fsw(o + r, o + j)] = x[r];
     }
     __syncthreads();
+    // block levels: T_ij = -T_ii M_ij, M_ij = sum_{k=j}^{i-1} A_ik T_kj.  An item is a 1x4 strip;
+    // its dot products are split over `ks` adjacent lanes and reduced with shuffles.
     for (int lvl = 1; lvl < 4; ++lvl) {
-        const int nblk = 4 - lvl;
-        for (int e = tid; e < nblk * 256; e += NT) {
-            const int bj = e >> 8, bi = bj + lvl, rr = (e >> 4) & 15, cc = e & 15;
-            float acc = 0.f;
-            for (int kb = bj; kb < bi; ++kb)
-#pragma unroll
-                for (int s = 0; s < 16; ++s)
-                    acc = fmaf(A[(bi * 16 + rr) * 64 + kb * 16 + s], T[(kb * 16 + s) * 64 + bj * 16 + cc], acc);
-            T[(bj * 16 + rr) * 64 + bi * 16 + cc] = acc;   // M_ij parked in the upper block (bj, bi)
+        const int items = (4 - lvl) * 64, ks = 256 / items >= 4 ? 4 : (256 / items >= 2 ? 2 : 1);
+        const int item = tid / ks, kp = tid % ks;
+        const bool live = item < items;
+        const int bj = item >> 6, bi = bj + lvl, rr = (item >> 2) & 15, c4 = (item & 3) * 4;
+        const int row = bi * 16 + rr;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (live)
+            for (int kk = bj * 16 + kp; kk < bi * 16; kk += ks) {
+                const float av = A[fsw(row, kk)];
+                const float4 tv = *reinterpret_cast<const float4 *>(T + fsw(kk, bj * 16 + c4));
+                acc.x = fmaf(av, tv.x, acc.x); acc.y = fmaf(av, tv.y, acc.y);
+                acc.z = fmaf(av, tv.z, acc.z); acc.w = fmaf(av, tv.w, acc.w);
+            }
+        for (int off = 1; off < ks; off <<= 1) {
+            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off); acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
+            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off); acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
         }
+        if (live && kp == 0) *reinterpret_cast<float4 *>(T + fsw(bj * 16 + rr, bi * 16 + c4)) = acc;   // parked in (bj, bi)
         __syncthreads();
-        for (int e = tid; e < nblk * 256; e += NT) {
-            const int bj = e >> 8, bi = bj + lvl, rr = (e >> 4) & 15, cc = e & 15;
-            float acc = 0.f;
-            for (int u = 0; u <= rr; ++u)
-                acc = fmaf(T[(bi * 16 + rr) * 64 + bi * 16 + u], T[(bj * 16 + u) * 64 + bi * 16 + cc], acc);
-            T[(bi * 16 + rr) * 64 + bj * 16 + cc] = -acc;
+        acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (live)
+            for (int u = kp; u <= rr; u += ks) {
+                const float tv = T[fsw(row, bi * 16 + u)];
+                const float4 mv = *reinterpret_cast<const float4 *>(T + fsw(bj * 16 + u, bi * 16 + c4));
+                acc.x = fmaf(tv, mv.x, acc.x); acc.y = fmaf(tv, mv.y, acc.y);
+                acc.z = fmaf(tv, mv.z, acc.z); acc.w = fmaf(tv, mv.w, acc.w);
+            }
+        for (int off = 1; off < ks; off <<= 1) {
+            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off); acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
+            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off); acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
         }
+        if (live && kp == 0)
+            *reinterpret_cast<float4 *>(T + fsw(row, bj * 16 + c4)) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
         __syncthreads();
     }
+}
+
+// pack 8 floats (scaled) into one 16-byte bf16 chunk
+__device__ __forceinline__ uint4 pack8(const float *v, float sc = 1.f) {
+    uint4 w;
+    w.x = tc::pack_bf16x2(v[0] * sc, v[1] * sc);
+    w.y = tc::pack_bf16x2(v[2] * sc, v[3] * sc);
+    w.z = tc::pack_bf16x2(v[4] * sc, v[5] * sc);
+    w.w = tc::pack_bf16x2(v[6] * sc, v[7] * sc);
+    return w;
 }
 }  // namespace
 
@@ -115,17 +144,19 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
 {
     using L_ = TcSmem<DVT>;
     using namespace tc;
+    constexpr int HV = DVT / 2;   // d_v columns per warp in the epilogues (two warps share a lane quadrant)
     extern __shared__ uint8_t smraw[];
     const uint32_t raw_u32 = smem_u32(smraw);
     const uint32_t sb = (raw_u32 + 1023u) & ~1023u;     // 1024-B aligned base (swizzle atoms)
     uint8_t *sm = smraw + (sb - raw_u32);
 
     float *misc = reinterpret_cast<float *>(sm + L_::MISC);
-    float *r_s = misc;              // [64]
-    float *invden = misc + 64;      // [64]
-    float *gamc = misc + 128;       // [128] chunk decay Gam_{L-1}
-    float *gam31 = misc + 256;      // [128] Gam_31 (start of the second half of the chunk)
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(misc + 384);
+    float *r_s = misc;              // [64] r_t
+    float *mur = misc + 64;         // [64] mu / r_t
+    float *invden = misc + 128;     // [64] 1 / den_t (0 past the chunk end)
+    float *gamc = misc + 192;       // [128] chunk decay Gam_{L-1}
+    float *pst = misc + 320;        // [128] uncertainty at the chunk start
+    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(misc + 448);
     uint64_t *bar_mma = bar_tma + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_mma + 1);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
@@ -140,6 +171,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     int t0, t1;
     seq_range(a, sq_, t0, t1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, whalf = warp >> 2;     // TMEM lane quadrant, column half
     const int H = a.H, dv = a.dv;
     const float mu = a.mu;
 
@@ -157,14 +189,14 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t T_PREP = tmem, T_D4 = tmem + 128, T_S = tmem + 256;
-    const uint32_t lane_off = ((uint32_t)(warp & 3) * 32u) << 16;
+    const uint32_t lane_off = ((uint32_t)quad * 32u) << 16;
 
-    // ---- initial memory tile -> TMEM (lane = key channel), uncertainty -> registers
+    // ---- initial memory tile -> TMEM (lane = key channel) and its bf16 operand copy
     const size_t sbase = (size_t)sh * DK * dv + (size_t)tile * DVT;
-    if (warp < 4) {
-        const int i = tid;
+    {
+        const int i = quad * 32 + lane;
 #pragma unroll 1
-        for (int cb = 0; cb < DVT; cb += 32) {
+        for (int cb = whalf * HV; cb < whalf * HV + HV; cb += 32) {
             float v[32];
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
@@ -173,10 +205,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 v[j] = x.x; v[j + 1] = x.y; v[j + 2] = x.z; v[j + 3] = x.w;
             }
             tmem_st32(T_S + lane_off + cb, v);
+            const uint32_t atom = (uint32_t)(cb >> 6) * 16384u;
+#pragma unroll
+            for (int chn = 0; chn < 4; ++chn)
+                *reinterpret_cast<uint4 *>(sm + L_::S + atom + swz(i, (((cb & 63) >> 3) + chn) * 16)) = pack8(v + chn * 8);
         }
     }
-    float P = 1.f;
-    if (tid < DK && a.P0) P = a.P0[(size_t)sh * DK + tid];
+    if (tid < DK) pst[tid] = a.P0 ? a.P0[(size_t)sh * DK + tid] : 1.f;
 
     const int nchunks = (t1 - t0 + C - 1) / C;
     uint32_t tma_phase = 0, mma_phase = 0;
@@ -185,11 +220,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         for (int b = 0; b < 2; ++b) {
             tma_load_3d(sm + L_::Q + b * 8192, &prm.tq, b * 64, h, t0, bar_tma);
             tma_load_3d(sm + L_::K + b * 8192, &prm.tk, b * 64, h, t0, bar_tma);
-            tma_load_3d(sm + L_::GP + b * 8192, &prm.tal, b * 64, h, t0, bar_tma);
-            tma_load_3d(sm + L_::SIG + b * 8192, &prm.tsg, b * 64, h, t0, bar_tma);
+            tma_load_3d(sm + L_::AL + b * 8192, &prm.tal, b * 64, h, t0, bar_tma);
+            tma_load_3d(sm + L_::SG + b * 8192, &prm.tsg, b * 64, h, t0, bar_tma);
         }
         for (int b = 0; b < DVT / 64; ++b) tma_load_3d(sm + L_::V + b * 8192, &prm.tv, tile * DVT + b * 64, h, t0, bar_tma);
     }
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -209,84 +245,167 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     for (int c = 0; c < nchunks; ++c) {
         const int c0 = t0 + c * C;
         const int L = min(C, t1 - c0);
-        if (tid < C) r_s[tid] = (tid < L) ? ldf(rin + (size_t)(c0 + tid) * H + h) : 1.f;
+        const int nxt = c0 + C;
+        const bool more = c + 1 < nchunks;
+        if (tid < C) {
+            const float rr = (tid < L) ? ldf(rin + (size_t)(c0 + tid) * H + h) : 1.f;
+            r_s[tid] = rr;
+            mur[tid] = mu / rr;
+        }
         if (!mbar_wait(bar_tma, tma_phase)) atomicExch(abort_flag, 1);
         tma_phase ^= 1u;
         __syncthreads();
         if (*abort_flag) break;
 
-        // ---- pass A: uncertainty recursion and gain numerators (thread = key channel)
+        // ---- uncertainty recursion (thread = channel pair cp x token quarter qt).  Each quarter
+        //      first composes the 2x2 maps of its 16 tokens (predict [[a, s],[0,1]] then update
+        //      [[1,0],[c,1]]); a quarter then starts from the composites of the quarters before it.
+        //      Output: P^- per (token, channel) and the decay Gam before every 4th token.
         {
-            float *gnum = reinterpret_cast<float *>(sm + L_::A4);
-            if (tid < DK) {
-                const int i = tid;
-                const uint32_t coff = (uint32_t)(i >> 6) * 8192u, cb = (uint32_t)(i & 63) * 2u;
-                float gam = 1.f;
-                for (int t = 0; t < L; ++t) {
+            float *pmv = reinterpret_cast<float *>(sm + L_::A4);                  // [64][128] P^-
+            float *comp = reinterpret_cast<float *>(sm + L_::Y);                  // [3][128][5]
+            float *gst = reinterpret_cast<float *>(sm + L_::Y + 7680);            // [16][128] Gam before token 4g
+            const int cp = tid & 63, qt = tid >> 6, ch = cp * 2;
+            const uint32_t coff = (uint32_t)(ch >> 6) * 8192u, cb = (uint32_t)(ch & 63) * 2u;
+            const float p0a = pst[ch], p0b = pst[ch + 1];
+            const int tb = qt * 16, te = min(L, tb + 16);
+            if (qt < 3 && te > tb) {
+                float a00 = 1.f, a01 = 0.f, a10 = 0.f, a11 = 1.f, ga = 1.f;
+                float b00 = 1.f, b01 = 0.f, b10 = 0.f, b11 = 1.f, gb = 1.f;
+                for (int t = tb; t < te; ++t) {
                     const uint32_t off = coff + swz(t, cb);
-                    const float al = bf16_at(sm + L_::GP, off), sg = bf16_at(sm + L_::SIG, off);
-                    const float kk = bf16_at(sm + L_::K, off);
-                    const float mr = mu / r_s[t];
-                    const float pm = fmaf(al * al, P, sg);
-                    const float gn = pm * kk;
-                    gnum[t * 128 + i] = gn;
-                    P = __fdividef(pm, fmaf(mr * kk, gn, 1.f));
-                    gam *= al;
-                    if (t == 31) gam31[i] = gam;
+                    const uint32_t aw = *reinterpret_cast<const uint32_t *>(sm + L_::AL + off);
+                    const uint32_t sw = *reinterpret_cast<const uint32_t *>(sm + L_::SG + off);
+                    const uint32_t kw = *reinterpret_cast<const uint32_t *>(sm + L_::K + off);
+                    const float mr = mur[t];
+                    {
+                        const float al = bf16_lo(aw), sg = bf16_lo(sw), kk = bf16_lo(kw);
+                        const float aa = al * al, cc = mr * kk * kk;
+                        const float y00 = fmaf(aa, a00, sg * a10), y01 = fmaf(aa, a01, sg * a11);
+                        a10 = fmaf(cc, y00, a10); a11 = fmaf(cc, y01, a11); a00 = y00; a01 = y01; ga *= al;
+                    }
+                    {
+                        const float al = bf16_hi(aw), sg = bf16_hi(sw), kk = bf16_hi(kw);
+                        const float aa = al * al, cc = mr * kk * kk;
+                        const float y00 = fmaf(aa, b00, sg * b10), y01 = fmaf(aa, b01, sg * b11);
+                        b10 = fmaf(cc, y00, b10); b11 = fmaf(cc, y01, b11); b00 = y00; b01 = y01; gb *= al;
+                    }
+                    if ((t & 7) == 7) {
+                        const float sa = 1.f / a11, sb2 = 1.f / b11;
+                        a00 *= sa; a01 *= sa; a10 *= sa; a11 = 1.f;
+                        b00 *= sb2; b01 *= sb2; b10 *= sb2; b11 = 1.f;
+                    }
                 }
-                gamc[i] = gam;
+                float *ca = comp + (qt * 128 + ch) * 5;
+                ca[0] = a00; ca[1] = a01; ca[2] = a10; ca[3] = a11; ca[4] = ga;
+                ca[5] = b00; ca[6] = b01; ca[7] = b10; ca[8] = b11; ca[9] = gb;
             }
             __syncthreads();
-            // gain denominators r_t + sum_i P^-_i k_i^2 (4 threads per token)
+            float Pa = p0a, Pb = p0b, gama = 1.f, gamb = 1.f;
+            for (int q2 = 0; q2 < qt; ++q2) {
+                const float *ca = comp + (q2 * 128 + ch) * 5;
+                Pa = fmaf(ca[0], Pa, ca[1]) / fmaf(ca[2], Pa, ca[3]);
+                Pb = fmaf(ca[5], Pb, ca[6]) / fmaf(ca[7], Pb, ca[8]);
+                gama *= ca[4];
+                gamb *= ca[9];
+            }
+#pragma unroll 4
+            for (int t = tb; t < tb + 16; ++t) {
+                if ((t & 3) == 0) *reinterpret_cast<float2 *>(gst + (t >> 2) * 128 + ch) = make_float2(gama, gamb);
+                if (t < te) {
+                    const uint32_t off = coff + swz(t, cb);
+                    const uint32_t aw = *reinterpret_cast<const uint32_t *>(sm + L_::AL + off);
+                    const uint32_t sw = *reinterpret_cast<const uint32_t *>(sm + L_::SG + off);
+                    const uint32_t kw = *reinterpret_cast<const uint32_t *>(sm + L_::K + off);
+                    const float mr = mur[t];
+                    const float ala = bf16_lo(aw), alb = bf16_hi(aw), ka = bf16_lo(kw), kb = bf16_hi(kw);
+                    const float pma = fmaf(ala * ala, Pa, bf16_lo(sw)), pmb = fmaf(alb * alb, Pb, bf16_hi(sw));
+                    *reinterpret_cast<float2 *>(pmv + t * 128 + ch) = make_float2(pma, pmb);
+                    Pa = __fdividef(pma, fmaf(mr * ka * ka, pma, 1.f));
+                    Pb = __fdividef(pmb, fmaf(mr * kb * kb, pmb, 1.f));
+                    gama *= ala;
+                    gamb *= alb;
+                }
+            }
+            if (te == L && tb < L) {     // this thread processed the chunk's last token
+                pst[ch] = Pa;
+                pst[ch + 1] = Pb;
+                gamc[ch] = gama;
+                gamc[ch + 1] = gamb;
+                if (!(gama >= 1e-30f) || !(gamb >= 1e-30f)) raise_error(a.err, ERR_RANGE);
+            }
+        }
+        __syncthreads();
+        // ---- elementwise pass (thread = 8 channels x 4 tokens, 16-byte accesses):
+        //      K~ = k Gam, Q~ = q Gam, G^ = P^- k / Gam, and den_t = r_t + sum_i P^-_i k_i^2
+        {
+            const float *pmv = reinterpret_cast<const float *>(sm + L_::A4);
+            const float *gst = reinterpret_cast<const float *>(sm + L_::Y + 7680);
+            const int o = tid & 15, g = tid >> 4, c8 = o * 8;
+            const uint32_t atom8 = (uint32_t)(o >> 3) * 8192u, atom16 = (uint32_t)(o >> 3) * 16384u;
+            const uint32_t chunkb = (uint32_t)(o & 7) * 16u;
+            float gam[8];
             {
-                const int t = tid >> 2, part = tid & 3;
-                float acc = 0.f;
+                const float4 g0 = *reinterpret_cast<const float4 *>(gst + g * 128 + c8);
+                const float4 g1 = *reinterpret_cast<const float4 *>(gst + g * 128 + c8 + 4);
+                gam[0] = g0.x; gam[1] = g0.y; gam[2] = g0.z; gam[3] = g0.w;
+                gam[4] = g1.x; gam[5] = g1.y; gam[6] = g1.z; gam[7] = g1.w;
+            }
+#pragma unroll 1
+            for (int j = 0; j < 4; ++j) {
+                const int t = g * 4 + j;
+                const uint32_t off = swz(t, chunkb);
+                float xsum = 0.f;
+                uint4 kq = make_uint4(0u, 0u, 0u, 0u), qq = kq, gg = kq;
                 if (t < L) {
-#pragma unroll 8
-                    for (int j = 0; j < 32; ++j) {
-                        const int ch = part * 32 + j;
-                        acc = fmaf(gnum[t * 128 + ch], bf16_at(sm + L_::K, (uint32_t)(ch >> 6) * 8192u + swz(t, (ch & 63) * 2)), acc);
+                    const uint4 aw = *reinterpret_cast<const uint4 *>(sm + L_::AL + atom8 + off);
+                    const uint4 kw = *reinterpret_cast<const uint4 *>(sm + L_::K + atom8 + off);
+                    const uint4 qw = *reinterpret_cast<const uint4 *>(sm + L_::Q + atom8 + off);
+                    const float4 p0 = *reinterpret_cast<const float4 *>(pmv + t * 128 + c8);
+                    const float4 p1 = *reinterpret_cast<const float4 *>(pmv + t * 128 + c8 + 4);
+                    const uint32_t *ap = reinterpret_cast<const uint32_t *>(&aw);
+                    const uint32_t *kp = reinterpret_cast<const uint32_t *>(&kw);
+                    const uint32_t *qp = reinterpret_cast<const uint32_t *>(&qw);
+                    const float pm[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                    uint32_t *kqp = reinterpret_cast<uint32_t *>(&kq);
+                    uint32_t *qqp = reinterpret_cast<uint32_t *>(&qq);
+                    uint32_t *ggp = reinterpret_cast<uint32_t *>(&gg);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float al0 = bf16_lo(ap[e]), al1 = bf16_hi(ap[e]);
+                        const float k0 = bf16_lo(kp[e]), k1 = bf16_hi(kp[e]);
+                        gam[2 * e] *= al0;
+                        gam[2 * e + 1] *= al1;
+                        const float pk0 = pm[2 * e] * k0, pk1 = pm[2 * e + 1] * k1;
+                        xsum = fmaf(pk0, k0, xsum);
+                        xsum = fmaf(pk1, k1, xsum);
+                        kqp[e] = pack_bf16x2(k0 * gam[2 * e], k1 * gam[2 * e + 1]);
+                        qqp[e] = pack_bf16x2(bf16_lo(qp[e]) * gam[2 * e], bf16_hi(qp[e]) * gam[2 * e + 1]);
+                        ggp[e] = pack_bf16x2(__fdividef(pk0, gam[2 * e]), __fdividef(pk1, gam[2 * e + 1]));
                     }
                 }
-                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                if (part == 0) invden[t] = (t < L) ? 1.f / (r_s[t] + acc) : 0.f;
+                *reinterpret_cast<uint4 *>(sm + L_::KQ + atom16 + swz(t, chunkb)) = kq;
+                *reinterpret_cast<uint4 *>(sm + L_::KQ + atom16 + swz(64 + t, chunkb)) = qq;
+                *reinterpret_cast<uint4 *>(sm + L_::G + atom8 + off) = gg;
+                // den over the 16 lanes that share this token
+                xsum += __shfl_xor_sync(0xffffffffu, xsum, 8);
+                xsum += __shfl_xor_sync(0xffffffffu, xsum, 4);
+                xsum += __shfl_xor_sync(0xffffffffu, xsum, 2);
+                xsum += __shfl_xor_sync(0xffffffffu, xsum, 1);
+                if (o == 0) invden[t] = (t < L) ? 1.f / (r_s[t] + xsum) : 0.f;
             }
-            __syncthreads();
-            // ---- pass B: decayed operands (thread = channel x half of the chunk)
-            {
-                const int i = tid & 127, half = tid >> 7;
-                const float gC = gamc[i];
-                if (half == 0 && L > 0 && !(gC >= 1e-30f)) raise_error(a.err, ERR_RANGE);
-                const float rho = rsqrtf(gC), sqg = sqrtf(gC);
-                const uint32_t coff = (uint32_t)(i >> 6) * 8192u, cb = (uint32_t)(i & 63) * 2u;
-                const uint32_t kqoff = (uint32_t)(i >> 6) * 16384u;
-                float gam = half ? gam31[i] : 1.f;
-                for (int t = half * 32; t < half * 32 + 32; ++t) {
-                    const uint32_t off = coff + swz(t, cb);
-                    float kt = 0.f, qt = 0.f, gt = 0.f, gp = 0.f;
-                    if (t < L) {
-                        const float al = bf16_at(sm + L_::GP, off);
-                        gam *= al;
-                        const float gr = gam * rho;
-                        const float g = gnum[t * 128 + i] * invden[t];
-                        kt = bf16_at(sm + L_::K, off) * gr;
-                        qt = bf16_at(sm + L_::Q, off) * gr;
-                        gt = __fdividef(g, gr);
-                        gp = gt * sqg;
-                    }
-                    st_bf16(sm + L_::KQ, kqoff + swz(t, cb), kt);
-                    st_bf16(sm + L_::KQ, kqoff + swz(64 + t, cb), qt);
-                    st_bf16(sm + L_::G, off, gt);
-                    st_bf16(sm + L_::GP, off, gp);
-                }
-            }
+        }
+        __syncthreads();
+        // q tile of the next chunk (its space is free now)
+        if (tid == 0 && more) {
+            mbar_expect_tx(bar_tma, L_::TMA_BYTES);
+            for (int b = 0; b < 2; ++b) tma_load_3d(sm + L_::Q + b * 8192, &prm.tq, b * 64, h, nxt, bar_tma);
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
 
-        // ---- MMA1: [A; Aq] = [K~; Q~] G~^T   (M=128, N=64, K=128)
+        // ---- MMA1: [A; Aq] = [K~; Q~] G^^T   (M=128, N=64, K=128)
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
@@ -298,32 +417,32 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             mma_commit(bar_mma);
         }
         wait_mma();
-        // rows 0..63 -> A (fp32, strictly lower); rows 64..127 -> Aq (bf16, lower incl. diagonal)
+        // rows 0..63 -> A (fp32, strictly lower) ; rows 64..127 -> Aq (bf16, lower incl. diagonal); columns / den
         float *Af = reinterpret_cast<float *>(sm + L_::K);
-        float *Tf = reinterpret_cast<float *>(sm + L_::Q);
-        if (warp < 4) {
-            const int row = warp * 32 + lane;
-#pragma unroll 1
-            for (int hb = 0; hb < 2; ++hb) {
-                float v[32];
-                tmem_ld32(T_PREP + lane_off + hb * 32, v);
-                if (row < 64) {
+        float *Tf = reinterpret_cast<float *>(sm + L_::SG);
+        {
+            const int row = quad * 32 + lane, s0 = whalf * 32;
+            float v[32];
+            tmem_ld32(T_PREP + lane_off + s0, v);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) Af[row * 64 + hb * 32 + j] = (hb * 32 + j < row) ? v[j] : 0.f;
-                } else {
-                    const int t = row - 64;
+            for (int j = 0; j < 32; j += 4) {
+                const float4 d4 = *reinterpret_cast<const float4 *>(invden + s0 + j);
+                v[j] *= d4.x; v[j + 1] *= d4.y; v[j + 2] *= d4.z; v[j + 3] *= d4.w;
+            }
+            if (row < 64) {
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint4 w4;
-                        uint32_t *wp = reinterpret_cast<uint32_t *>(&w4);
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4 *>(Af + fsw(row, s0 + j)) =
+                        make_float4(s0 + j < row ? v[j] : 0.f, s0 + j + 1 < row ? v[j + 1] : 0.f,
+                                    s0 + j + 2 < row ? v[j + 2] : 0.f, s0 + j + 3 < row ? v[j + 3] : 0.f);
+            } else {
+                const int t = row - 64;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int s0 = hb * 32 + ch * 8 + 2 * e;
-                            wp[e] = pack_bf16x2(s0 <= t ? v[ch * 8 + 2 * e] : 0.f, s0 + 1 <= t ? v[ch * 8 + 2 * e + 1] : 0.f);
-                        }
-                        *reinterpret_cast<uint4 *>(sm + L_::AQ + swz(t, (hb * 4 + ch) * 16)) = w4;
-                    }
-                }
+                for (int j = 0; j < 32; ++j)
+                    if (s0 + j > t) v[j] = 0.f;
+#pragma unroll
+                for (int chn = 0; chn < 4; ++chn)
+                    *reinterpret_cast<uint4 *>(sm + L_::AL + swz(t, (whalf * 4 + chn) * 16)) = pack8(v + chn * 8);
             }
         }
         tc_fence_before();
@@ -335,14 +454,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
                 const int chn = q4 * 2 + m;
-                uint4 w4;
-                uint32_t *wp = reinterpret_cast<uint32_t *>(&w4);
+                float v[8];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int s0 = chn * 8 + 2 * e;
-                    wp[e] = pack_bf16x2(s0 <= t ? Tf[t * 64 + s0] : 0.f, s0 + 1 <= t ? Tf[t * 64 + s0 + 1] : 0.f);
-                }
-                *reinterpret_cast<uint4 *>(sm + L_::Y + swz(t, chn * 16)) = w4;
+                for (int e = 0; e < 8; ++e) v[e] = (chn * 8 + e <= t) ? Tf[fsw(t, chn * 8 + e)] : 0.f;
+                *reinterpret_cast<uint4 *>(sm + L_::Y + swz(t, chn * 16)) = pack8(v);
             }
         }
         fence_async_smem();
@@ -354,39 +469,27 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(T_PREP + 64, sdesc(sb + L_::AQ + ks * 32u, 16, 1024), sdesc(sb + L_::Y + ks * 2048u, 8192, 1024),
+                mma_bf16(T_PREP + 64, sdesc(sb + L_::AL + ks * 32u, 16, 1024), sdesc(sb + L_::Y + ks * 2048u, 8192, 1024),
                          ID_M64_N64_KM, ks > 0);
             mma_commit(bar_mma);
-            if (c + 1 < nchunks) {   // q and k tiles of the next chunk (their space is free now)
-                const int n0 = c0 + C;
-                mbar_expect_tx(bar_tma, L_::TMA_BYTES);
+            if (more)   // k and sigma tiles of the next chunk (A and T fp32 are consumed)
                 for (int b = 0; b < 2; ++b) {
-                    tma_load_3d(sm + L_::Q + b * 8192, &prm.tq, b * 64, h, n0, bar_tma);
-                    tma_load_3d(sm + L_::K + b * 8192, &prm.tk, b * 64, h, n0, bar_tma);
+                    tma_load_3d(sm + L_::K + b * 8192, &prm.tk, b * 64, h, nxt, bar_tma);
+                    tma_load_3d(sm + L_::SG + b * 8192, &prm.tsg, b * 64, h, nxt, bar_tma);
                 }
-            }
         }
         wait_mma();
+        if (tid == 0 && more)   // alpha tile of the next chunk (Aq consumed)
+            for (int b = 0; b < 2; ++b) tma_load_3d(sm + L_::AL + b * 8192, &prm.tal, b * 64, h, nxt, bar_tma);
         // X -> bf16, rows 64..127 of Y.  M=64 accumulator: row m sits in lane (m%16) + 32*(m/16).
-        if (warp < 4) {
-            float v[32], v2[32];
-            tmem_ld32(T_PREP + 64 + lane_off, v);
-            tmem_ld32(T_PREP + 64 + lane_off + 32, v2);
+        {
+            float v[32];
+            tmem_ld32(T_PREP + 64 + lane_off + whalf * 32, v);
             if (lane < 16) {
-                const int t = warp * 16 + lane;
+                const int t = quad * 16 + lane;
 #pragma unroll
-                for (int chn = 0; chn < 8; ++chn) {
-                    uint4 w4;
-                    uint32_t *wp = reinterpret_cast<uint32_t *>(&w4);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int s0 = chn * 8 + 2 * e;
-                        const float x0 = s0 < 32 ? v[s0] : v2[s0 - 32];
-                        const float x1 = s0 + 1 < 32 ? v[s0 + 1] : v2[s0 + 1 - 32];
-                        wp[e] = pack_bf16x2(x0, x1);
-                    }
-                    *reinterpret_cast<uint4 *>(sm + L_::Y + swz(64 + t, chn * 16)) = w4;
-                }
+                for (int chn = 0; chn < 4; ++chn)
+                    *reinterpret_cast<uint4 *>(sm + L_::Y + swz(64 + t, (whalf * 4 + chn) * 16)) = pack8(v + chn * 8);
             }
         }
         fence_async_smem();
@@ -404,57 +507,37 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         }
         wait_mma();
         // rows 0..63 -> -w ; rows 64..127 -> Q' = Q~ - X K~   (bf16 into A4)
-        if (warp < 4) {
-            const int row = warp * 32 + lane;
+        {
+            const int row = quad * 32 + lane;
 #pragma unroll 1
-            for (int cb = 0; cb < 4; ++cb) {
+            for (int cb = whalf * 2; cb < whalf * 2 + 2; ++cb) {
                 float v[32];
                 tmem_ld32(T_PREP + lane_off + cb * 32, v);
                 const uint32_t atom = (uint32_t)(cb >> 1) * 16384u;
 #pragma unroll
                 for (int chn = 0; chn < 4; ++chn) {
                     const uint32_t boff = swz(row, ((cb & 1) * 4 + chn) * 16);
-                    uint4 w4;
-                    uint32_t *wp = reinterpret_cast<uint32_t *>(&w4);
                     if (row < 64) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) wp[e] = pack_bf16x2(-v[chn * 8 + 2 * e], -v[chn * 8 + 2 * e + 1]);
+                        *reinterpret_cast<uint4 *>(sm + L_::A4 + atom + boff) = pack8(v + chn * 8, -1.f);
                     } else {
                         const uint4 q4 = *reinterpret_cast<const uint4 *>(sm + L_::KQ + atom + boff);
                         const uint32_t *qp = reinterpret_cast<const uint32_t *>(&q4);
+                        float w8[8];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            wp[e] = pack_bf16x2(bf16_lo(qp[e]) - v[chn * 8 + 2 * e], bf16_hi(qp[e]) - v[chn * 8 + 2 * e + 1]);
+                        for (int e = 0; e < 4; ++e) {
+                            w8[2 * e] = bf16_lo(qp[e]) - v[chn * 8 + 2 * e];
+                            w8[2 * e + 1] = bf16_hi(qp[e]) - v[chn * 8 + 2 * e + 1];
+                        }
+                        *reinterpret_cast<uint4 *>(sm + L_::A4 + atom + boff) = pack8(w8);
                     }
-                    *reinterpret_cast<uint4 *>(sm + L_::A4 + atom + boff) = w4;
                 }
-            }
-            // ---- memory tile: S0' = Gam^{1/2} S (bf16 operand), TMEM S <- Gam S
-            const int i = row;
-            const float gC = gamc[i], sqg = sqrtf(gC);
-#pragma unroll 1
-            for (int cb = 0; cb < DVT / 32; ++cb) {
-                float v[32];
-                tmem_ld32(T_S + lane_off + cb * 32, v);
-                const uint32_t atom = (uint32_t)(cb >> 1) * 16384u;
-#pragma unroll
-                for (int chn = 0; chn < 4; ++chn) {
-                    uint4 w4;
-                    uint32_t *wp = reinterpret_cast<uint32_t *>(&w4);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) wp[e] = pack_bf16x2(sqg * v[chn * 8 + 2 * e], sqg * v[chn * 8 + 2 * e + 1]);
-                    *reinterpret_cast<uint4 *>(sm + L_::S + atom + swz(i, ((cb & 1) * 4 + chn) * 16)) = w4;
-                }
-#pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] *= gC;
-                tmem_st32(T_S + lane_off + cb * 32, v);
             }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
 
-        // ---- MMA4: [U; O] = [-w; Q'] S0' + [T; X] V   (M=128, N=DVT, K=128+64)
+        // ---- MMA4: [U; O] = [-w; Q'] S + [T; X] V   (M=128, N=DVT, K=128+64)
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
@@ -470,38 +553,27 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             mma_commit(bar_mma);
         }
         wait_mma();
-        if (tid == 0 && c + 1 < nchunks)
+        if (tid == 0 && more)
             for (int b = 0; b < DVT / 64; ++b)
-                tma_load_3d(sm + L_::V + b * 8192, &prm.tv, tile * DVT + b * 64, h, c0 + C, bar_tma);
-        // rows 0..63 -> U (bf16, zero past the chunk end); rows 64..127 -> o (global)
-        if (warp < 4) {
-            const int row = warp * 32 + lane;
+                tma_load_3d(sm + L_::V + b * 8192, &prm.tv, tile * DVT + b * 64, h, nxt, bar_tma);
+        // rows 0..63 -> U / den (bf16, zero past the chunk end); rows 64..127 -> o (global)
+        {
+            const int row = quad * 32 + lane;
+            const float sc = row < 64 ? invden[row] : 1.f;
 #pragma unroll 1
-            for (int cb = 0; cb < DVT / 32; ++cb) {
+            for (int cb = whalf * HV; cb < whalf * HV + HV; cb += 32) {
                 float v[32];
-                tmem_ld32(T_D4 + lane_off + cb * 32, v);
+                tmem_ld32(T_D4 + lane_off + cb, v);
                 if (row < 64) {
-                    const bool live = row < L;
-                    const uint32_t blk = (uint32_t)(cb >> 1) * 8192u;
+                    const uint32_t blk = (uint32_t)(cb >> 6) * 8192u;
 #pragma unroll
-                    for (int chn = 0; chn < 4; ++chn) {
-                        uint4 w4;
-                        uint32_t *wp = reinterpret_cast<uint32_t *>(&w4);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            wp[e] = live ? pack_bf16x2(v[chn * 8 + 2 * e], v[chn * 8 + 2 * e + 1]) : 0u;
-                        *reinterpret_cast<uint4 *>(sm + L_::U + blk + swz(row, ((cb & 1) * 4 + chn) * 16)) = w4;
-                    }
+                    for (int chn = 0; chn < 4; ++chn)
+                        *reinterpret_cast<uint4 *>(sm + L_::U + blk + swz(row, (((cb & 63) >> 3) + chn) * 16)) =
+                            pack8(v + chn * 8, sc);
                 } else if (row - 64 < L) {
-                    bf16 *dst = out + ((size_t)(c0 + row - 64) * H + h) * dv + tile * DVT + cb * 32;
+                    bf16 *dst = out + ((size_t)(c0 + row - 64) * H + h) * dv + tile * DVT + cb;
 #pragma unroll
-                    for (int chn = 0; chn < 4; ++chn) {
-                        uint4 w4;
-                        uint32_t *wp = reinterpret_cast<uint32_t *>(&w4);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) wp[e] = pack_bf16x2(v[chn * 8 + 2 * e], v[chn * 8 + 2 * e + 1]);
-                        *reinterpret_cast<uint4 *>(dst + chn * 8) = w4;
-                    }
+                    for (int chn = 0; chn < 4; ++chn) *reinterpret_cast<uint4 *>(dst + chn * 8) = pack8(v + chn * 8);
                 }
             }
         }
@@ -509,31 +581,46 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         tc_fence_before();
         __syncthreads();
 
-        // ---- MMA5: S += G'^T U   (M=128 channels, N=DVT, K=64 tokens; both operands MN-major)
+        // ---- MMA5: S += G^^T (U / den)   (M=128 channels, N=DVT, K=64 tokens; both operands MN-major)
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(T_S, sdesc(sb + L_::GP + ks * 2048u, 8192, 1024), sdesc(sb + L_::U + ks * 2048u, 8192, 1024),
+                mma_bf16(T_S, sdesc(sb + L_::G + ks * 2048u, 8192, 1024), sdesc(sb + L_::U + ks * 2048u, 8192, 1024),
                          ID_M128_NV_MM, 1);
             mma_commit(bar_mma);
         }
         wait_mma();
-        if (tid == 0 && c + 1 < nchunks)
-            for (int b = 0; b < 2; ++b) {
-                tma_load_3d(sm + L_::GP + b * 8192, &prm.tal, b * 64, h, c0 + C, bar_tma);
-                tma_load_3d(sm + L_::SIG + b * 8192, &prm.tsg, b * 64, h, c0 + C, bar_tma);
+        // ---- decay the rows by the chunk's Gam_{L-1}; refresh the bf16 operand copy
+        {
+            const int i = quad * 32 + lane;
+            const float gC = gamc[i];
+#pragma unroll 1
+            for (int cb = whalf * HV; cb < whalf * HV + HV; cb += 32) {
+                float v[32];
+                tmem_ld32(T_S + lane_off + cb, v);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] *= gC;
+                tmem_st32(T_S + lane_off + cb, v);
+                const uint32_t atom = (uint32_t)(cb >> 6) * 16384u;
+#pragma unroll
+                for (int chn = 0; chn < 4; ++chn)
+                    *reinterpret_cast<uint4 *>(sm + L_::S + atom + swz(i, (((cb & 63) >> 3) + chn) * 16)) = pack8(v + chn * 8);
             }
+        }
+        fence_async_smem();
+        tc_fence_before();
         __syncthreads();
+        tc_fence_after();
         if (*abort_flag) break;
     }
 
     // ---- final state
     if (!*abort_flag) {
-        if (warp < 4 && a.S_out) {
-            const int i = tid;
+        if (a.S_out) {
+            const int i = quad * 32 + lane;
 #pragma unroll 1
-            for (int cb = 0; cb < DVT; cb += 32) {
+            for (int cb = whalf * HV; cb < whalf * HV + HV; cb += 32) {
                 float v[32];
                 tmem_ld32(T_S + lane_off + cb, v);
 #pragma unroll
@@ -542,7 +629,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                         make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
             }
         }
-        if (a.P_out && tid < DK && tile == 0) a.P_out[(size_t)sh * DK + tid] = P;
+        if (a.P_out && tid < DK && tile == 0) a.P_out[(size_t)sh * DK + tid] = pst[tid];
     } else {
         raise_error(a.err, ERR_TIMEOUT);
     }

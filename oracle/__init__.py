@@ -180,6 +180,30 @@ def delta_forward(q, k, v, alpha, beta, cu_seqlens=None, S0=None, threads: Optio
     return dict(o=o, S=S)
 
 
+def diag_chains(w, chains, mu=None, S0=None, P0=None, threads: Optional[int] = None):
+    """Diagonal KDN on selected (sequence, head) chains of a workload ``w`` (any object
+    with q, k, v, alpha, sigma, r as [ntok, H, d], cu_seqlens and mu).
+
+    The chains are packed as the sequences of a one-head problem and run in one call
+    (one thread per chain).  Returns {(s, h): dict(o [len, dv], S [dk, dv], P [dk])}."""
+    mu = w.mu if mu is None else mu
+    cu = w.cu_seqlens
+    pieces = [((s, h), (slice(int(cu[s]), int(cu[s + 1])), slice(h, h + 1))) for s, h in chains]
+
+    def cat(name):
+        return np.concatenate([getattr(w, name)[sl] for _, sl in pieces], axis=0)
+    lens = [sl[0].stop - sl[0].start for _, sl in pieces]
+    cu2 = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    S0s = None if S0 is None else np.stack([S0[s, h] for (s, h), _ in pieces])[:, None]
+    P0s = None if P0 is None else np.stack([P0[s, h] for (s, h), _ in pieces])[:, None]
+    res = diag_forward(cat("q"), cat("k"), cat("v"), cat("alpha"), cat("sigma"), cat("r"),
+                       cu_seqlens=cu2, S0=S0s, P0=P0s, mu=mu, threads=threads)
+    out = {}
+    for i, ((s, h), _) in enumerate(pieces):
+        out[(s, h)] = dict(o=res["o"][cu2[i]:cu2[i + 1], 0], S=res["S"][i, 0], P=res["P"][i, 0])
+    return out
+
+
 def mobius_matrix(alpha, sigma, k, r, mu: float = 1.0):
     """2x2 matrix of one token's map P -> P_new on one key channel.
 

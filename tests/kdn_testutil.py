@@ -41,26 +41,6 @@ def dense_shape(w, x):
 
 
 def oracle_chains(w, chains, mu=None, S0=None, P0=None, threads=None):
-    """Oracle on the listed (seq, head) chains of workload ``w``.
-
-    Returns {(s, h): dict(o [len, dv], S [dk, dv], P [dk])}."""
-    mu = w.mu if mu is None else mu
-    out = {}
-    cu = w.cu_seqlens
-    pieces = []
-    for s, h in chains:
-        t0, t1 = int(cu[s]), int(cu[s + 1])
-        sl = (slice(t0, t1), slice(h, h + 1))
-        pieces.append(((s, h), sl))
-    # one oracle call over all chains: pack them as sequences of a 1-head problem
-    def cat(name):
-        return np.concatenate([getattr(w, name)[sl] for _, sl in pieces], axis=0)
-    lens = [sl[0].stop - sl[0].start for _, sl in pieces]
-    cu2 = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
-    S0s = None if S0 is None else np.stack([S0[s, h] for (s, h), _ in pieces])[:, None]
-    P0s = None if P0 is None else np.stack([P0[s, h] for (s, h), _ in pieces])[:, None]
-    res = oracle.diag_forward(cat("q"), cat("k"), cat("v"), cat("alpha"), cat("sigma"), cat("r"),
-                              cu_seqlens=cu2, S0=S0s, P0=P0s, mu=mu, threads=threads)
-    for i, ((s, h), _) in enumerate(pieces):
-        out[(s, h)] = dict(o=res["o"][cu2[i]:cu2[i + 1], 0], S=res["S"][i, 0], P=res["P"][i, 0])
-    return out
+    """Oracle on the listed (seq, head) chains of workload ``w``:
+    {(s, h): dict(o [len, dv], S [dk, dv], P [dk])}."""
+    return oracle.diag_chains(w, chains, mu=mu, S0=S0, P0=P0, threads=threads)
