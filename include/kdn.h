@@ -68,10 +68,14 @@ typedef struct {
     kdn_dtype_t in_dtype;           /* dtype of q, k, v, alpha, sigma, r and o */
     float mu;                       /* information scaling, > 0 */
     int chunk;                      /* execution path, see above */
+    int max_seqlen;                 /* varlen: upper bound on every sequence length (0 = unknown, taken as T);
+                                       sizes the gain scan's work list.  A sequence longer than it makes
+                                       kdn_gain_scan record KDN_ERR_INVALID_ARG in the device error word. */
 } kdn_problem_t;
 
-/* Bytes of device workspace kdn_forward_chunkwise() and kdn_gain_scan() need for `p`
- * (0 is possible).  Host-only; no CUDA call. */
+/* Bytes of device workspace needed for `p`: the larger of what kdn_gain_scan() and
+ * kdn_forward_chunkwise() use (the forward paths currently use none, so the forward
+ * also accepts workspace = NULL).  Host-only; no CUDA call. */
 kdn_status_t kdn_workspace_size(const kdn_problem_t *p, size_t *bytes);
 
 /* Prefill / training forward over whole sequences (KDA article, "chunkwise" regime;
@@ -113,7 +117,12 @@ kdn_status_t kdn_decode_step(int N, int H, int d_k, int d_v, kdn_dtype_t in_dtyp
  *  g               : device fp32 [B, T, H, d_k], the gain of every token, or NULL
  *  beta_eff        : device fp32 [B, T, H], k_t^T g_t (the effective write strength), or NULL
  *  P_out           : device fp32 [N, H, d_k], uncertainty after the last token, or NULL
- *  workspace       : as for kdn_forward_chunkwise (same size rule). */
+ *  workspace       : device, >= kdn_workspace_size() bytes, 256-byte aligned; its contents
+ *                    on entry do not matter (the call resets what it uses).
+ * Single pass: every 64-token chunk composes its tokens' maps, publishes the composite,
+ * and takes its starting uncertainty from its predecessors by decoupled look-back
+ * (bounded waits; a wait that gives up records KDN_ERR_TIMEOUT).  Concurrent calls
+ * must use distinct workspaces. */
 kdn_status_t kdn_gain_scan(const kdn_problem_t *p,
                            const void *k, const void *alpha, const void *sigma, const void *r,
                            const float *P0, float *g, float *beta_eff, float *P_out,
@@ -125,7 +134,7 @@ kdn_status_t kdn_gain_scan(const kdn_problem_t *p,
 int kdn_execution_path(const kdn_problem_t *p);
 
 /* Synchronises `stream`, then returns and clears the device error word
- * (KDN_ERR_TIMEOUT or KDN_ERR_RANGE if a kernel recorded one, else KDN_OK). */
+ * (KDN_ERR_TIMEOUT, KDN_ERR_RANGE or KDN_ERR_INVALID_ARG if a kernel recorded one, else KDN_OK). */
 kdn_status_t kdn_last_device_error(void *stream);
 
 /* Static description of a status code. */

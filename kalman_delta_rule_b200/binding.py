@@ -31,7 +31,8 @@ class KdnError(RuntimeError):
 class kdn_problem_t(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("d_k", ctypes.c_int),
                 ("d_v", ctypes.c_int), ("cu_seqlens", ctypes.c_void_p), ("num_seqs", ctypes.c_int),
-                ("in_dtype", ctypes.c_int), ("mu", ctypes.c_float), ("chunk", ctypes.c_int)]
+                ("in_dtype", ctypes.c_int), ("mu", ctypes.c_float), ("chunk", ctypes.c_int),
+                ("max_seqlen", ctypes.c_int)]
 
 
 _lib = None
@@ -142,7 +143,7 @@ def _check(st: int, where: str):
         raise KdnError(st, where)
 
 
-def make_problem(q, v, H=None, cu_seqlens=None, mu: float = 1.0, chunk: int = 64) -> kdn_problem_t:
+def make_problem(q, v, H=None, cu_seqlens=None, mu: float = 1.0, chunk: int = 64, max_seqlen: int = 0) -> kdn_problem_t:
     B, T, H_, dk = q.shape
     p = kdn_problem_t()
     p.B, p.T, p.H, p.d_k, p.d_v = B, T, H_, dk, v.shape[-1]
@@ -151,6 +152,7 @@ def make_problem(q, v, H=None, cu_seqlens=None, mu: float = 1.0, chunk: int = 64
     p.in_dtype = _dtype_code(q)
     p.mu = float(mu)
     p.chunk = int(chunk)
+    p.max_seqlen = int(max_seqlen)
     return p
 
 
@@ -193,10 +195,10 @@ def decode_step(q, k, v, alpha, sigma, r, S, P, mu: float = 1.0, o=None, stream=
 
 
 def gain_scan(k, alpha, sigma, r, cu_seqlens=None, P0=None, mu: float = 1.0, chunk: int = 64,
-              want_g: bool = True, want_beta: bool = True, workspace=None, stream=None):
+              want_g: bool = True, want_beta: bool = True, workspace=None, stream=None, max_seqlen: int = 0):
     """Run kdn_gain_scan; returns (g [B,T,H,dk] fp32 or None, beta_eff [B,T,H] or None, P_out [N,H,dk])."""
     torch = _torch()
-    p = make_problem(k, k, cu_seqlens=cu_seqlens, mu=mu, chunk=chunk)
+    p = make_problem(k, k, cu_seqlens=cu_seqlens, mu=mu, chunk=chunk, max_seqlen=max_seqlen)
     dev = k.device
     g = torch.empty(k.shape, dtype=torch.float32, device=dev) if want_g else None
     be = torch.empty(k.shape[:3], dtype=torch.float32, device=dev) if want_beta else None

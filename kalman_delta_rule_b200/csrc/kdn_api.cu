@@ -34,6 +34,7 @@ struct Resolved {
     long long ntok;
     int nseq;
     bool bf16;
+    long long nchunks_max;   // gain scan work list (chunks of 64 per sequence, upper bound)
 };
 
 kdn_status_t check_problem(const kdn_problem_t *p, Resolved *out) {
@@ -51,6 +52,9 @@ kdn_status_t check_problem(const kdn_problem_t *p, Resolved *out) {
     }
     out->ntok = (long long)p->B * p->T;
     out->bf16 = p->in_dtype == KDN_DTYPE_BF16;
+    if (p->max_seqlen < 0) return KDN_ERR_INVALID_ARG;
+    const long long ml = (p->max_seqlen > 0 && p->max_seqlen < p->T) ? p->max_seqlen : p->T;
+    out->nchunks_max = (ml + 63) / 64;
     if (out->ntok > (1ll << 31) / 2) return KDN_ERR_UNSUPPORTED;
     return KDN_OK;
 }
@@ -81,7 +85,7 @@ kdn_status_t kdn_workspace_size(const kdn_problem_t *p, size_t *bytes) {
     kdn_status_t st = check_problem(p, &rv);
     if (st != KDN_OK) return st;
     if (!bytes) return KDN_ERR_INVALID_ARG;
-    *bytes = 0;
+    *bytes = kdn::scan_workspace_bytes((long long)rv.nseq * p->H, rv.nchunks_max, p->d_k);
     return KDN_OK;
 }
 
@@ -92,9 +96,7 @@ kdn_status_t kdn_forward_chunkwise(const kdn_problem_t *p, const void *q, const 
     Resolved rv;
     kdn_status_t st = check_problem(p, &rv);
     if (st != KDN_OK) return st;
-    size_t need = 0;
-    kdn_workspace_size(p, &need);
-    if (need > 0 && (!workspace || workspace_bytes < need)) return KDN_ERR_WORKSPACE;
+    (void)workspace; (void)workspace_bytes;   // the forward paths use no workspace
     if (rv.nseq == 0 || (rv.ntok == 0 && !S_out && !P_out)) return KDN_OK;
     if (rv.ntok > 0 && (!q || !k || !v || !alpha || !sigma || !r || !o)) return KDN_ERR_INVALID_ARG;
     const void *ptrs[] = {q, k, v, alpha, sigma, r, o, S0, P0, S_out, P_out};
@@ -146,9 +148,19 @@ kdn_status_t kdn_gain_scan(const kdn_problem_t *p, const void *k, const void *al
     Resolved rv;
     kdn_status_t st = check_problem(p, &rv);
     if (st != KDN_OK) return st;
-    (void)k; (void)alpha; (void)sigma; (void)r; (void)P0; (void)g; (void)beta_eff; (void)P_out;
-    (void)workspace; (void)workspace_bytes; (void)stream;
-    return KDN_ERR_UNSUPPORTED;
+    if (rv.nseq == 0 || rv.ntok == 0) return KDN_OK;
+    if (!k || !alpha || !sigma || !r) return KDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {k, alpha, sigma, r, P0, g, beta_eff, P_out};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KDN_ERR_INVALID_ARG;
+    const size_t need = kdn::scan_workspace_bytes((long long)rv.nseq * p->H, rv.nchunks_max, p->d_k);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return KDN_ERR_WORKSPACE;
+    kdn::ScanArgs a{};
+    a.k = k; a.alpha = alpha; a.sigma = sigma; a.r = r; a.P0 = P0;
+    a.g = g; a.beta = beta_eff; a.P_out = P_out;
+    a.cu = p->cu_seqlens; a.T = p->T; a.nseq = rv.nseq; a.H = p->H; a.dk = p->d_k; a.mu = p->mu;
+    a.nchunks_max = (int)rv.nchunks_max; a.nchains = rv.nseq * p->H; a.err = err_word();
+    return cuda_status(kdn::launch_gain_scan(a, rv.bf16, workspace, static_cast<cudaStream_t>(stream)));
 }
 
 int kdn_execution_path(const kdn_problem_t *p) {
@@ -169,6 +181,7 @@ kdn_status_t kdn_last_device_error(void *stream) {
     if (cudaStreamSynchronize(cs) != cudaSuccess) return KDN_ERR_CUDA;
     if (bits & kdn::ERR_TIMEOUT) return KDN_ERR_TIMEOUT;
     if (bits & kdn::ERR_RANGE) return KDN_ERR_RANGE;
+    if (bits & kdn::ERR_ARG) return KDN_ERR_INVALID_ARG;
     return KDN_OK;
 }
 

@@ -11,7 +11,7 @@
 namespace kdn {
 
 // bits of the device error word (reported by kdn_last_device_error)
-enum : unsigned { ERR_TIMEOUT = 1u, ERR_RANGE = 2u };
+enum : unsigned { ERR_TIMEOUT = 1u, ERR_RANGE = 2u, ERR_ARG = 4u };
 
 __device__ __forceinline__ void raise_error(unsigned *err, unsigned bit) {
     if (err) atomicOr(err, bit);
@@ -61,6 +61,20 @@ struct TokenArgs {
     int T;                                       // dense sequence length (ignored with cu)
     int nseq, H, dk, dv;
     float mu;
+    unsigned *err;
+};
+
+struct ScanArgs {
+    const void *k, *alpha, *sigma, *r;          // [ntok, H, dk] / [ntok, H]
+    const float *P0;                            // [N, H, dk] or NULL (ones)
+    float *g, *beta, *P_out;                    // [ntok, H, dk], [ntok, H], [N, H, dk]; each may be NULL
+    const int32_t *cu;                          // device [N+1] or NULL
+    int T, nseq, H, dk;
+    float mu;
+    int nchunks_max, nchains;                   // chunk-major work list: nchunks_max x (nseq * H)
+    unsigned *counter;                          // workspace: ticket counter
+    int *flags;                                 // workspace: per (chunk, chain) publication flag
+    float *desc;                                // workspace: per (chunk, chain) [4][dk] aggregate + end value
     unsigned *err;
 };
 

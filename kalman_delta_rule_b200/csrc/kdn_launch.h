@@ -18,4 +18,8 @@ cudaError_t launch_chunk_simt(const TokenArgs &a, bool bf16_in, int C, cudaStrea
 bool chunk_tc_supported(int dk, int dv, bool bf16_in, int chunk, long long ntok);
 cudaError_t launch_chunk_tc(const TokenArgs &a, long long ntok, int dvt, cudaStream_t st);
 
+// single-pass Moebius scan of the uncertainty with decoupled look-back (workspace-backed)
+size_t scan_workspace_bytes(long long nchains, long long nchunks_max, int dk);
+cudaError_t launch_gain_scan(ScanArgs a, bool bf16_in, void *workspace, cudaStream_t st);
+
 }  // namespace kdn

@@ -180,7 +180,7 @@ def delta_forward(q, k, v, alpha, beta, cu_seqlens=None, S0=None, threads: Optio
     return dict(o=o, S=S)
 
 
-def diag_chains(w, chains, mu=None, S0=None, P0=None, threads: Optional[int] = None):
+def diag_chains(w, chains, mu=None, S0=None, P0=None, threads: Optional[int] = None, trace: bool = False):
     """Diagonal KDN on selected (sequence, head) chains of a workload ``w`` (any object
     with q, k, v, alpha, sigma, r as [ntok, H, d], cu_seqlens and mu).
 
@@ -197,10 +197,14 @@ def diag_chains(w, chains, mu=None, S0=None, P0=None, threads: Optional[int] = N
     S0s = None if S0 is None else np.stack([S0[s, h] for (s, h), _ in pieces])[:, None]
     P0s = None if P0 is None else np.stack([P0[s, h] for (s, h), _ in pieces])[:, None]
     res = diag_forward(cat("q"), cat("k"), cat("v"), cat("alpha"), cat("sigma"), cat("r"),
-                       cu_seqlens=cu2, S0=S0s, P0=P0s, mu=mu, threads=threads)
+                       cu_seqlens=cu2, S0=S0s, P0=P0s, mu=mu, threads=threads, trace=trace)
     out = {}
     for i, ((s, h), _) in enumerate(pieces):
-        out[(s, h)] = dict(o=res["o"][cu2[i]:cu2[i + 1], 0], S=res["S"][i, 0], P=res["P"][i, 0])
+        sl = slice(cu2[i], cu2[i + 1])
+        out[(s, h)] = dict(o=res["o"][sl, 0], S=res["S"][i, 0], P=res["P"][i, 0])
+        if trace:
+            out[(s, h)].update(g=res["trace_g"][sl, 0], beta_eff=res["trace_beta_eff"][sl, 0],
+                               Pm=res["trace_Pm"][sl, 0])
     return out
 
 

@@ -52,6 +52,7 @@ def problem(**kw):
     p = B.kdn_problem_t()
     p.B, p.T, p.H, p.d_k, p.d_v = 2, 128, 4, 128, 128
     p.cu_seqlens, p.num_seqs, p.in_dtype, p.mu, p.chunk = None, 0, B.KDN_DTYPE_BF16, 1.0, 64
+    p.max_seqlen = 0
     for k, v in kw.items():
         setattr(p, k, v)
     return p
@@ -67,6 +68,7 @@ def problem(**kw):
     (dict(B=-1), B.KDN_ERR_INVALID_ARG),
     (dict(in_dtype=7), B.KDN_ERR_INVALID_ARG),
     (dict(cu_seqlens=FAKE, B=2, num_seqs=3), B.KDN_ERR_INVALID_ARG),
+    (dict(max_seqlen=-1), B.KDN_ERR_INVALID_ARG),
 ])
 def test_problem_validation(lib, kw, code):
     p = problem(**kw)
@@ -81,6 +83,10 @@ def test_workspace_size_is_host_only_and_sane(lib):
         for dt in (B.KDN_DTYPE_F32, B.KDN_DTYPE_BF16):
             n = B.kdn_workspace_size(problem(chunk=chunk, in_dtype=dt))
             assert 0 <= n < (1 << 34)
+    # a tighter max_seqlen shrinks the gain scan's work list
+    full = B.kdn_workspace_size(problem(B=1, T=4096))
+    tight = B.kdn_workspace_size(problem(B=1, T=4096, max_seqlen=512))
+    assert tight < full
     assert lib.kdn_workspace_size(None, None) == B.KDN_ERR_INVALID_ARG
 
 
@@ -95,10 +101,15 @@ def test_forward_rejects_bad_pointers(lib):
     # final state aliasing the initial state
     assert B.kdn_forward_chunkwise(p, *ptrs, FAKE + 4096, None, FAKE, FAKE + 4096, None, None, 0, None) == B.KDN_ERR_INVALID_ARG
     assert B.kdn_forward_chunkwise(p, *ptrs, None, FAKE + 4096, FAKE, None, FAKE + 4096, None, 0, None) == B.KDN_ERR_INVALID_ARG
-    # chunked paths that need a workspace reject a missing one
+    # the gain scan rejects a missing, short or misaligned workspace before any CUDA call
     p64 = problem(chunk=64)
-    if B.kdn_workspace_size(p64) > 0:
-        assert B.kdn_forward_chunkwise(p64, *ptrs, None, None, FAKE, None, None, None, 0, None) == B.KDN_ERR_WORKSPACE
+    need = B.kdn_workspace_size(p64)
+    assert need > 0
+    k_a_s_r = [FAKE] * 4
+    assert B.kdn_gain_scan(p64, *k_a_s_r, None, FAKE, None, None, None, 0, None) == B.KDN_ERR_WORKSPACE
+    assert B.kdn_gain_scan(p64, *k_a_s_r, None, FAKE, None, None, FAKE + 4096, need - 1, None) == B.KDN_ERR_WORKSPACE
+    assert B.kdn_gain_scan(p64, *k_a_s_r, None, FAKE, None, None, FAKE + 16, need, None) == B.KDN_ERR_WORKSPACE
+    assert B.kdn_gain_scan(p64, None, *k_a_s_r[1:], None, FAKE, None, None, FAKE, need, None) == B.KDN_ERR_INVALID_ARG
 
 
 def test_decode_rejects_bad_arguments(lib):
