@@ -128,6 +128,27 @@ kdn_status_t kdn_gain_scan(const kdn_problem_t *p,
                            const float *P0, float *g, float *beta_eff, float *P_out,
                            void *workspace, size_t workspace_bytes, void *stream);
 
+/* kdn_gain_scan() for callers that cannot allocate device memory at call time -- for
+ * example a plugin hosted by a framework that owns every device buffer and exposes no
+ * allocator, or a serving loop that bans cudaMalloc/cudaFree after start-up (cudaFree
+ * synchronises the device).  The paper has no counterpart: this entry point only changes
+ * where the scan keeps its scratch.
+ *  Arguments: as kdn_gain_scan() without the workspace; inputs and outputs stay the
+ *  caller's.  Scratch: a fixed 16 MiB device array inside the library, one per GPU that
+ *  loads it, held until the process exits.  A problem whose scan needs more (more than
+ *  about 8000 (chunk of 64 tokens, sequence x head) pairs at d_k = 128) returns
+ *  KDN_ERR_UNSUPPORTED before anything runs.
+ *  Set-up: the first call on a device looks up that device's array address (with the
+ *  device current); make that first call before any stream capture.  No cudaMalloc,
+ *  cudaFree or allocating library routine is called.
+ *  Sharing: every call uses the same array and leaves its last contents there (each call
+ *  clears the part that must start at zero).  Calls that overlap on the GPU -- on
+ *  different streams, or from different host threads -- race on the array and must be
+ *  ordered by the caller. */
+kdn_status_t kdn_gain_scan_noalloc(const kdn_problem_t *p,
+                                   const void *k, const void *alpha, const void *sigma, const void *r,
+                                   const float *P0, float *g, float *beta_eff, float *P_out, void *stream);
+
 /* Which execution path kdn_forward_chunkwise() takes for `p` (host-only; no CUDA call
  * besides resolving the driver's tensor-map encoder once): 0 token-serial recurrence,
  * 1 fp32 CUDA-core chunk kernel, 2 tcgen05 tensor-core chunk kernel; -1 if `p` is invalid. */

@@ -49,6 +49,7 @@ _SIGS = {
     "kdn_status_string": (ctypes.c_char_p, [_i]),
     "kdn_version": (ctypes.c_char_p, []),
     "kdn_execution_path": (_i, [_PP]),
+    "kdn_gain_scan_noalloc": (_i, [_PP] + [_vp] * 4 + [_vp] + [_vp] * 3 + [_vp]),
 }
 
 
@@ -89,6 +90,12 @@ def kdn_decode_step(N, H, d_k, d_v, in_dtype, mu, q, k, v, alpha, sigma, r, S, P
 def kdn_gain_scan(problem, k, alpha, sigma, r, P0, g, beta_eff, P_out, workspace, workspace_bytes, stream):
     return load().kdn_gain_scan(ctypes.byref(problem), k, alpha, sigma, r, P0, g, beta_eff, P_out,
                                 workspace, workspace_bytes, stream)
+
+
+def kdn_gain_scan_noalloc(problem, k, alpha, sigma, r, P0, g, beta_eff, P_out, stream):
+    """The gain scan on the library's fixed scratch array: for callers that cannot
+    allocate device memory when they call (no workspace argument)."""
+    return load().kdn_gain_scan_noalloc(ctypes.byref(problem), k, alpha, sigma, r, P0, g, beta_eff, P_out, stream)
 
 
 def kdn_last_device_error(stream=None) -> int:

@@ -142,25 +142,51 @@ kdn_status_t kdn_decode_step(int N, int H, int d_k, int d_v, kdn_dtype_t in_dtyp
     return cuda_status(kdn::launch_recurrent(a, in_dtype == KDN_DTYPE_BF16, d_v, static_cast<cudaStream_t>(stream)));
 }
 
-kdn_status_t kdn_gain_scan(const kdn_problem_t *p, const void *k, const void *alpha, const void *sigma,
-                           const void *r, const float *P0, float *g, float *beta_eff, float *P_out,
-                           void *workspace, size_t workspace_bytes, void *stream) {
-    Resolved rv;
-    kdn_status_t st = check_problem(p, &rv);
+static kdn_status_t scan_args(const kdn_problem_t *p, const void *k, const void *alpha, const void *sigma,
+                              const void *r, const float *P0, float *g, float *beta_eff, float *P_out,
+                              kdn::ScanArgs *a, Resolved *rv, bool *empty) {
+    kdn_status_t st = check_problem(p, rv);
     if (st != KDN_OK) return st;
-    if (rv.nseq == 0 || rv.ntok == 0) return KDN_OK;
+    *empty = rv->nseq == 0 || rv->ntok == 0;
+    if (*empty) return KDN_OK;
     if (!k || !alpha || !sigma || !r) return KDN_ERR_INVALID_ARG;
     const void *ptrs[] = {k, alpha, sigma, r, P0, g, beta_eff, P_out};
     for (const void *ptr : ptrs)
         if (ptr && !aligned16(ptr)) return KDN_ERR_INVALID_ARG;
+    *a = kdn::ScanArgs{};
+    a->k = k; a->alpha = alpha; a->sigma = sigma; a->r = r; a->P0 = P0;
+    a->g = g; a->beta = beta_eff; a->P_out = P_out;
+    a->cu = p->cu_seqlens; a->T = p->T; a->nseq = rv->nseq; a->H = p->H; a->dk = p->d_k; a->mu = p->mu;
+    a->nchunks_max = (int)rv->nchunks_max; a->nchains = rv->nseq * p->H;
+    return KDN_OK;
+}
+
+kdn_status_t kdn_gain_scan(const kdn_problem_t *p, const void *k, const void *alpha, const void *sigma,
+                           const void *r, const float *P0, float *g, float *beta_eff, float *P_out,
+                           void *workspace, size_t workspace_bytes, void *stream) {
+    Resolved rv;
+    kdn::ScanArgs a;
+    bool empty = false;
+    kdn_status_t st = scan_args(p, k, alpha, sigma, r, P0, g, beta_eff, P_out, &a, &rv, &empty);
+    if (st != KDN_OK || empty) return st;
     const size_t need = kdn::scan_workspace_bytes((long long)rv.nseq * p->H, rv.nchunks_max, p->d_k);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return KDN_ERR_WORKSPACE;
-    kdn::ScanArgs a{};
-    a.k = k; a.alpha = alpha; a.sigma = sigma; a.r = r; a.P0 = P0;
-    a.g = g; a.beta = beta_eff; a.P_out = P_out;
-    a.cu = p->cu_seqlens; a.T = p->T; a.nseq = rv.nseq; a.H = p->H; a.dk = p->d_k; a.mu = p->mu;
-    a.nchunks_max = (int)rv.nchunks_max; a.nchains = rv.nseq * p->H; a.err = err_word();
+    a.err = err_word();
     return cuda_status(kdn::launch_gain_scan(a, rv.bf16, workspace, static_cast<cudaStream_t>(stream)));
+}
+
+kdn_status_t kdn_gain_scan_noalloc(const kdn_problem_t *p, const void *k, const void *alpha, const void *sigma,
+                                   const void *r, const float *P0, float *g, float *beta_eff, float *P_out,
+                                   void *stream) {
+    Resolved rv;
+    kdn::ScanArgs a;
+    bool empty = false;
+    kdn_status_t st = scan_args(p, k, alpha, sigma, r, P0, g, beta_eff, P_out, &a, &rv, &empty);
+    if (st != KDN_OK || empty) return st;
+    if (kdn::scan_workspace_bytes((long long)rv.nseq * p->H, rv.nchunks_max, p->d_k) > kdn::noalloc_scratch_bytes())
+        return KDN_ERR_UNSUPPORTED;
+    a.err = err_word();
+    return cuda_status(kdn::launch_gain_scan_noalloc(a, rv.bf16, static_cast<cudaStream_t>(stream)));
 }
 
 int kdn_execution_path(const kdn_problem_t *p) {

@@ -21,5 +21,8 @@ cudaError_t launch_chunk_tc(const TokenArgs &a, long long ntok, int dvt, cudaStr
 // single-pass Moebius scan of the uncertainty with decoupled look-back (workspace-backed)
 size_t scan_workspace_bytes(long long nchains, long long nchunks_max, int dk);
 cudaError_t launch_gain_scan(ScanArgs a, bool bf16_in, void *workspace, cudaStream_t st);
+// the same scan on the library's fixed scratch array (no allocation, no caller workspace)
+size_t noalloc_scratch_bytes();
+cudaError_t launch_gain_scan_noalloc(const ScanArgs &a, bool bf16_in, cudaStream_t st);
 
 }  // namespace kdn

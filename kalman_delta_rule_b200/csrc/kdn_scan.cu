@@ -16,6 +16,8 @@
 //      den_t = r_t + sum_i P^-_i k_i^2, the gain g_t = P^- k / den_t and k^T g.
 // Work is handed out by a ticket counter in chunk-major order, so every predecessor of
 // a chunk was taken by a CTA that is already running; waits are bounded.
+#include <mutex>
+
 #include "kdn_common.cuh"
 #include "kdn_launch.h"
 
@@ -300,6 +302,46 @@ cudaError_t launch_gain_scan(ScanArgs a, bool bf16_in, void *workspace, cudaStre
         case 257: return launch_scan_t<128, bf16>(a, st);
     }
     return cudaErrorInvalidValue;
+}
+
+// ---------------------------------------------------------------- allocation-free variant
+// Scratch of kdn_gain_scan_noalloc: a fixed device array (one copy on every GPU that loads
+// the library, held until the process exits) used instead of a caller-provided workspace.
+constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;
+static __device__ __align__(256) unsigned char g_scan_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mu;
+void *g_scratch_addr[kMaxScratchDevices];
+}  // namespace
+
+// Device address of the current GPU's scratch array.  In host code the array's name only
+// stands for the symbol, so the address is looked up once per device (with that device
+// current) and cached.
+static cudaError_t scratch_address(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_scan_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return cudaSuccess;
+}
+
+size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+cudaError_t launch_gain_scan_noalloc(const ScanArgs &a, bool bf16_in, cudaStream_t st) {
+    void *ws = nullptr;
+    cudaError_t e = scratch_address(&ws);
+    if (e != cudaSuccess) return e;
+    return launch_gain_scan(a, bf16_in, ws, st);   // clears the ticket counter and flags it uses
 }
 
 }  // namespace kdn
