@@ -245,8 +245,42 @@ def bench_prefill(args, world, rank, dev, kdn):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     e2e_value = world * tokens * e_steps / (e2e_ms / 1e3)
 
+    # the uncertainty / gain scan on its own, over the same inputs (g fp32, k^T g, final P)
+    scan = None
+    if not args.no_scan:
+        ws_scan = torch.empty(max(kdn.kdn_workspace_size(prob), 1), dtype=torch.uint8, device=dev)
+        g_out = torch.empty(d["k"].shape, dtype=torch.float32, device=dev)
+        b_out = torch.empty(d["k"].shape[:3], dtype=torch.float32, device=dev)
+        p_out = torch.empty((w.num_seqs, w.H, w.dk), dtype=torch.float32, device=dev)
+        sp = kdn.make_problem(d["k"], d["k"], cu_seqlens=cu, mu=w.mu, chunk=w.chunk)
+        sargs = [d[n].data_ptr() for n in ("k", "alpha", "sigma", "r")]
+        sh = stream.cuda_stream or None
+
+        def scan_step():
+            st = kdn.kdn_gain_scan(sp, *sargs, None, g_out.data_ptr(), b_out.data_ptr(), p_out.data_ptr(),
+                                   ws_scan.data_ptr(), ws_scan.numel(), sh)
+            if st != kdn.KDN_OK:
+                raise kdn.KdnError(st, "kdn_gain_scan")
+
+        for _ in range(args.warmup):
+            scan_step()
+        kdn.last_device_error()
+        barrier(world)
+        sev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        sev[0].record(stream)
+        for i in range(args.steps):
+            scan_step()
+            sev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        kdn.last_device_error()
+        s_ms = max_over_ranks(sev[0].elapsed_time(sev[-1]), world) / args.steps
+        esz = 2 if w.bf16 else 4
+        s_bytes = w.ntok * w.H * (3 * w.dk * esz + esz + w.dk * 4 + 4) + w.num_seqs * w.H * w.dk * 4
+        scan = dict(value=world * w.ntok / (s_ms / 1e3), ms_step=s_ms, bytes=s_bytes, launches=args.steps)
+
     nbytes = algorithmic_bytes(w)
-    return dict(w=w, value=value, ms_step=ms_step, per_step_ms=per_step_ms, clocks=clk.summary(), path=path,
+    return dict(w=w, value=value, ms_step=ms_step, per_step_ms=per_step_ms, clocks=clk.summary(), path=path, scan=scan,
                 e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                          steps=e_steps),
                 bytes=nbytes, launches=args.steps)
@@ -290,24 +324,23 @@ def bench_decode(args, world, rank, dev, kdn, steps=1024, N=256, H=32, d=128):
     return dict(value=world * steps / (ms / 1e3), ms_step=per_step, bytes=nbytes, steps=steps, N=N, H=H, d=d)
 
 
-def cpu_baseline_prefill(w, max_seconds=30.0):
-    """The fp64 oracle on the host cores over whole (sequence, head) chains of the workload."""
+def cpu_baseline_prefill(w, min_seconds=10.0, max_reps=50):
+    """The fp64 oracle on the host cores over the whole workload (every (sequence, head)
+    chain, full length), repeated until about `min_seconds` of wall time have passed."""
     import oracle
     cores = os.cpu_count() or 1
     chains = [(s, h) for s in range(w.num_seqs) for h in range(w.H)]
-    # bounded sample: as many whole chains as fit ~max_seconds at ~0.5 s per chain-core
-    per_chain_tokens = w.ntok / w.num_seqs
-    est_chain_s = per_chain_tokens * 5 * w.dk * w.dv * 2 / 1.2e9
-    n = int(min(len(chains), max(cores, cores * max_seconds / max(est_chain_s, 1e-3))))
-    n = max(1, min(n, len(chains)))
-    pick = chains[:n]
-    t0 = time.perf_counter()
-    oracle.diag_chains(w, pick, threads=cores)
-    dt = time.perf_counter() - t0
-    tok = sum(int(w.cu_seqlens[s + 1] - w.cu_seqlens[s]) for s, _ in pick) / w.H
-    return {"value": tok / dt, "unit": "tokens/s", "cores": min(cores, n), "kind": "oracle",
-            "sample": f"{n} of {len(chains)} (sequence, head) chains of the workload, whole length, fp64 C oracle, "
-                      f"{dt:.1f} s wall"}
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.diag_chains(w, chains, threads=cores)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_seconds or reps >= max_reps:
+            break
+    tok = reps * w.ntok
+    return {"value": tok / dt, "unit": "tokens/s", "cores": min(cores, len(chains)), "kind": "oracle",
+            "sample": f"the whole workload ({len(chains)} (sequence, head) chains x full length) run {reps} times "
+                      f"by the fp64 C oracle, {dt:.1f} s wall"}
 
 
 def kernel_hash():
@@ -366,6 +399,14 @@ def ours(args):
             "gpu_launches": pre["launches"],
             "clocks": pre["clocks"],
         }
+        if pre["scan"] is not None:
+            sc = pre["scan"]
+            sach = sc["bytes"] / (sc["ms_step"] / 1e3) / 1e9
+            line["gain_scan"] = {"metric": "gain scan tokens/s (P^-, gain, k^T g, final P)", "value": sc["value"],
+                                 "unit": "tokens/s", "ms_per_step": sc["ms_step"], "gpu_launches": sc["launches"],
+                                 "roofline": {"bound": "hbm", "achieved": sach, "peak": hbm, "unit": "GB/s",
+                                              "frac": sach / hbm, "traffic": None,
+                                              "algorithmic_bytes_per_launch": sc["bytes"]}}
         if dec is not None:
             dach = dec["bytes"] / (dec["ms_step"] / 1e3) / 1e9
             line["decode"] = {"metric": "decode steps/s", "value": dec["value"], "unit": "steps/s",
@@ -438,6 +479,7 @@ def main():
     ap.add_argument("--clock-seconds", type=float, default=2.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-scan", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=1024)
     args = ap.parse_args()
     if args.warmup < 3:

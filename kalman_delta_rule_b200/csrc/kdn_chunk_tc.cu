@@ -7,8 +7,8 @@
 // Per chunk (local tokens t, s in [0, L)), with Gam_t = prod_{j<=t} alpha_j per channel
 // (decay referenced to the chunk start) and den_t = r_t + sum_i P^-_{t,i} k_{t,i}^2:
 //   prep (independent of the memory S):
-//     uncertainty recursion in four token quarters joined by the Moebius composites of
-//     the quarters' 2x2 maps (CUDA cores, thread = key-channel pair x quarter)
+//     uncertainty recursion in eight 8-token segments joined by the Moebius composites
+//     of the segments' 2x2 maps (CUDA cores, thread = key-channel pair x segment)
 //     K~ = k Gam,  Q~ = q Gam,  G^ = P^- k / Gam   (the gain is G^ Gam / den)
 //     MMA1   [A; Aq] = [K~; Q~] G^^T, columns scaled by 1/den  -> A (s < t), Aq (s <= t)
 //     T = (I + A)^{-1}                               (CUDA cores, blocked 16x16)
@@ -30,25 +30,29 @@
 namespace kdn {
 
 namespace {
-constexpr int C = 64, DK = 128, NT = 256;
+constexpr int C = 64, DK = 128, NT = 512, LDA = 68;   // LDA: padded fp32 row stride of A and T
 
 template <int DVT>
 struct TcSmem {
-    static constexpr uint32_t Q = 0;                        // q tile (TMA)
-    static constexpr uint32_t K = Q + 16384;                // k tile (TMA); then A fp32 [64][64]
-    static constexpr uint32_t AL = K + 16384;               // alpha tile (TMA); then Aq bf16 64 x 64
-    static constexpr uint32_t SG = AL + 16384;              // sigma tile (TMA); then T fp32 [64][64]
+    static constexpr uint32_t Q = 0;                        // q tile (TMA); then T fp32 [64][LDA]
+    static constexpr uint32_t K = Q + 16384;                // k tile (TMA); then A fp32 [64][LDA] at K + 1024
+    static constexpr uint32_t AL = K + 16384;               // alpha tile (TMA); then Aq bf16 64 x 64 at AL + 8192
+    static constexpr uint32_t SG = AL + 16384;              // sigma tile (TMA)
     static constexpr uint32_t V = SG + 16384;               // v tile (TMA), DVT*128 B
     static constexpr uint32_t KQ = V + DVT * 128;           // [K~; Q~] bf16, K-major, 2 atoms of 128 rows
     static constexpr uint32_t G = KQ + 32768;               // G^ bf16, 64 token rows x 128 ch
-    static constexpr uint32_t Y = G + 16384;                // [T; X] bf16, 128 x 64
-    static constexpr uint32_t A4 = Y + 16384;               // [-w; Q'] bf16 128 x 128; prep: P^- k^2 fp32 [64][128]
+    static constexpr uint32_t Y = G + 16384;                // [T; X] bf16 128 x 64; prep: segment composites
+    static constexpr uint32_t A4 = Y + 16384;               // [-w; Q'] bf16 128 x 128; prep: P^- fp32 [64][128]
     static constexpr uint32_t S = A4 + 32768;               // S bf16, 128 channel rows x DVT (MN-major)
-    static constexpr uint32_t U = S + DVT * 256;            // U / den bf16, 64 token rows x DVT (MN-major)
+    static constexpr uint32_t U = S + DVT * 256;            // U / den bf16 64 x DVT; prep: Gam every 4 tokens
     static constexpr uint32_t MISC = U + DVT * 128;
     static constexpr uint32_t MISC_BYTES = 2048;
     static constexpr uint32_t total = MISC + MISC_BYTES;
     static constexpr uint32_t TMA_BYTES = 4 * 16384 + DVT * 128;
+    static constexpr uint32_t AF = K + 1024, TF = Q, AQ = AL + 8192;
+    static_assert(TF + 64 * LDA * 4 <= AF, "T and A fp32 tiles overlap");
+    static_assert(AF + 64 * LDA * 4 <= AQ, "A fp32 tile overlaps Aq");
+    static_assert(DVT * 128 >= 16 * 128 * 4, "U must hold the decay table");
 };
 
 struct TcParams {
@@ -56,74 +60,66 @@ struct TcParams {
     CUtensorMap tq, tk, tv, tal, tsg;
 };
 
-__device__ __forceinline__ float bf16_at(const uint8_t *base, uint32_t off) {
-    return __uint_as_float(((uint32_t) * reinterpret_cast<const unsigned short *>(base + off)) << 16);
-}
-__device__ __forceinline__ void st_bf16(uint8_t *base, uint32_t off, float v) {
-    *reinterpret_cast<__nv_bfloat16 *>(base + off) = __float2bfloat16_rn(v);
-}
-
-// fp32 64x64 tiles in shared memory: 4-float groups of a row are XOR-permuted by the row
-// index, so that column reads across rows and float4 row accesses are bank-conflict free.
-__device__ __forceinline__ int fsw(int r, int c) { return r * 64 + ((((c >> 2) ^ r) & 15) << 2) + (c & 3); }
-
-// T = (I + A)^{-1} for a strictly lower 64x64 fp32 A (fsw layout), blocked by 16:
+// T = (I + A)^{-1} for a strictly lower 64x64 fp32 A (row stride LDA), blocked by 16:
 // the four 16x16 diagonal blocks by forward substitution, then block levels
-// T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj, each thread producing a 1x4 strip.
-// T's strictly-upper blocks are used as scratch; readers mask them out.
+// T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj with 1x4 output strips whose dot products are
+// split over `ks` adjacent lanes.  T's strictly-upper blocks are used as scratch.
 __device__ void tri_inverse64(const float *A, float *T, int tid) {
-    if (tid < 64) {   // diagonal blocks: thread = (block, column), forward substitution
+    if (tid < 64) {
         const int o = (tid >> 4) * 16, j = tid & 15;
         float x[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
         for (int r = 1; r < 16; ++r) {
+            const float *arow = A + (o + r) * LDA + o;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int s = 0; s < r; ++s) acc[s & 3] = fmaf(A[fsw(o + r, o + s)], x[s], acc[s & 3]);
+            for (int s = 0; s < r; ++s) acc[s & 3] = fmaf(arow[s], x[s], acc[s & 3]);
             if (r > j) x[r] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) T[fsw(o + r, o + j)] = x[r];
+        for (int r = 0; r < 16; ++r) T[(o + r) * LDA + o + j] = x[r];
     }
     __syncthreads();
-    // block levels: T_ij = -T_ii M_ij, M_ij = sum_{k=j}^{i-1} A_ik T_kj.  An item is a 1x4 strip;
-    // its dot products are split over `ks` adjacent lanes and reduced with shuffles.
     for (int lvl = 1; lvl < 4; ++lvl) {
-        const int items = (4 - lvl) * 64, ks = 256 / items >= 4 ? 4 : (256 / items >= 2 ? 2 : 1);
+        const int items = (4 - lvl) * 64, ks = lvl == 1 ? 2 : (lvl == 2 ? 4 : 8);
         const int item = tid / ks, kp = tid % ks;
         const bool live = item < items;
         const int bj = item >> 6, bi = bj + lvl, rr = (item >> 2) & 15, c4 = (item & 3) * 4;
         const int row = bi * 16 + rr;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (live)
+        if (live) {
+            const float *arow = A + row * LDA;
             for (int kk = bj * 16 + kp; kk < bi * 16; kk += ks) {
-                const float av = A[fsw(row, kk)];
-                const float4 tv = *reinterpret_cast<const float4 *>(T + fsw(kk, bj * 16 + c4));
+                const float av = arow[kk];
+                const float4 tv = *reinterpret_cast<const float4 *>(T + kk * LDA + bj * 16 + c4);
                 acc.x = fmaf(av, tv.x, acc.x); acc.y = fmaf(av, tv.y, acc.y);
                 acc.z = fmaf(av, tv.z, acc.z); acc.w = fmaf(av, tv.w, acc.w);
             }
+        }
         for (int off = 1; off < ks; off <<= 1) {
             acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off); acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
             acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off); acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
         }
-        if (live && kp == 0) *reinterpret_cast<float4 *>(T + fsw(bj * 16 + rr, bi * 16 + c4)) = acc;   // parked in (bj, bi)
+        if (live && kp == 0) *reinterpret_cast<float4 *>(T + (bj * 16 + rr) * LDA + bi * 16 + c4) = acc;   // parked
         __syncthreads();
         acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (live)
-            for (int u = kp; u <= rr; u += ks) {
-                const float tv = T[fsw(row, bi * 16 + u)];
-                const float4 mv = *reinterpret_cast<const float4 *>(T + fsw(bj * 16 + u, bi * 16 + c4));
+        if (live) {
+            const float *trow = T + row * LDA + bi * 16;
+            for (int uu = kp; uu <= rr; uu += ks) {
+                const float tv = trow[uu];
+                const float4 mv = *reinterpret_cast<const float4 *>(T + (bj * 16 + uu) * LDA + bi * 16 + c4);
                 acc.x = fmaf(tv, mv.x, acc.x); acc.y = fmaf(tv, mv.y, acc.y);
                 acc.z = fmaf(tv, mv.z, acc.z); acc.w = fmaf(tv, mv.w, acc.w);
             }
+        }
         for (int off = 1; off < ks; off <<= 1) {
             acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off); acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
             acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off); acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
         }
         if (live && kp == 0)
-            *reinterpret_cast<float4 *>(T + fsw(row, bj * 16 + c4)) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+            *reinterpret_cast<float4 *>(T + row * LDA + bj * 16 + c4) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
         __syncthreads();
     }
 }
@@ -144,7 +140,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
 {
     using L_ = TcSmem<DVT>;
     using namespace tc;
-    constexpr int HV = DVT / 2;   // d_v columns per warp in the epilogues (two warps share a lane quadrant)
+    constexpr int NC = DVT / 4;   // d_v columns per warp in the epilogues (four warps share a lane quadrant)
     extern __shared__ uint8_t smraw[];
     const uint32_t raw_u32 = smem_u32(smraw);
     const uint32_t sb = (raw_u32 + 1023u) & ~1023u;     // 1024-B aligned base (swizzle atoms)
@@ -171,7 +167,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     int t0, t1;
     seq_range(a, sq_, t0, t1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, whalf = warp >> 2;     // TMEM lane quadrant, column half
+    const int quad = warp & 3, cg = warp >> 2;     // TMEM lane quadrant, column group
     const int H = a.H, dv = a.dv;
     const float mu = a.mu;
 
@@ -190,26 +186,24 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     const uint32_t tmem = *tmem_slot;
     const uint32_t T_PREP = tmem, T_D4 = tmem + 128, T_S = tmem + 256;
     const uint32_t lane_off = ((uint32_t)quad * 32u) << 16;
+    const int row = quad * 32 + lane;   // TMEM lane this thread reads in M=128 epilogues
+    const int cb0 = cg * NC;            // first d_v column of this thread's epilogue slice
 
     // ---- initial memory tile -> TMEM (lane = key channel) and its bf16 operand copy
     const size_t sbase = (size_t)sh * DK * dv + (size_t)tile * DVT;
     {
-        const int i = quad * 32 + lane;
-#pragma unroll 1
-        for (int cb = whalf * HV; cb < whalf * HV + HV; cb += 32) {
-            float v[32];
+        float v[NC];
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-                float4 x = a.S0 ? *reinterpret_cast<const float4 *>(a.S0 + sbase + (size_t)i * dv + cb + j)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-                v[j] = x.x; v[j + 1] = x.y; v[j + 2] = x.z; v[j + 3] = x.w;
-            }
-            tmem_st32(T_S + lane_off + cb, v);
-            const uint32_t atom = (uint32_t)(cb >> 6) * 16384u;
-#pragma unroll
-            for (int chn = 0; chn < 4; ++chn)
-                *reinterpret_cast<uint4 *>(sm + L_::S + atom + swz(i, (((cb & 63) >> 3) + chn) * 16)) = pack8(v + chn * 8);
+        for (int j = 0; j < NC; j += 4) {
+            float4 x = a.S0 ? *reinterpret_cast<const float4 *>(a.S0 + sbase + (size_t)row * dv + cb0 + j)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[j] = x.x; v[j + 1] = x.y; v[j + 2] = x.z; v[j + 3] = x.w;
         }
+        tmem_st<NC>(T_S + lane_off + cb0, v);
+        const uint32_t atom = (uint32_t)(cb0 >> 6) * 16384u;
+#pragma unroll
+        for (int chn = 0; chn < NC / 8; ++chn)
+            *reinterpret_cast<uint4 *>(sm + L_::S + atom + swz(row, (((cb0 & 63) >> 3) + chn) * 16)) = pack8(v + chn * 8);
     }
     if (tid < DK) pst[tid] = a.P0 ? a.P0[(size_t)sh * DK + tid] : 1.f;
 
@@ -257,19 +251,19 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         __syncthreads();
         if (*abort_flag) break;
 
-        // ---- uncertainty recursion (thread = channel pair cp x token quarter qt).  Each quarter
-        //      first composes the 2x2 maps of its 16 tokens (predict [[a, s],[0,1]] then update
-        //      [[1,0],[c,1]]); a quarter then starts from the composites of the quarters before it.
+        // ---- uncertainty recursion (thread = channel pair cp x 8-token segment sgi).  Each
+        //      segment first composes the 2x2 maps of its tokens (predict [[a, s],[0,1]] then
+        //      update [[1,0],[c,1]]); a segment then starts from the composites before it.
         //      Output: P^- per (token, channel) and the decay Gam before every 4th token.
         {
             float *pmv = reinterpret_cast<float *>(sm + L_::A4);                  // [64][128] P^-
-            float *comp = reinterpret_cast<float *>(sm + L_::Y);                  // [3][128][5]
-            float *gst = reinterpret_cast<float *>(sm + L_::Y + 7680);            // [16][128] Gam before token 4g
-            const int cp = tid & 63, qt = tid >> 6, ch = cp * 2;
+            float *comp = reinterpret_cast<float *>(sm + L_::Y);                  // [7][128][4]
+            float *gst = reinterpret_cast<float *>(sm + L_::U);                   // [16][128]
+            const int cp = tid & 63, sgi = tid >> 6, ch = cp * 2;
             const uint32_t coff = (uint32_t)(ch >> 6) * 8192u, cb = (uint32_t)(ch & 63) * 2u;
             const float p0a = pst[ch], p0b = pst[ch + 1];
-            const int tb = qt * 16, te = min(L, tb + 16);
-            if (qt < 3 && te > tb) {
+            const int tb = sgi * 8, te = min(L, tb + 8);
+            if (sgi < 7 && te > tb) {
                 float a00 = 1.f, a01 = 0.f, a10 = 0.f, a11 = 1.f, ga = 1.f;
                 float b00 = 1.f, b01 = 0.f, b10 = 0.f, b11 = 1.f, gb = 1.f;
                 for (int t = tb; t < te; ++t) {
@@ -290,27 +284,23 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                         const float y00 = fmaf(aa, b00, sg * b10), y01 = fmaf(aa, b01, sg * b11);
                         b10 = fmaf(cc, y00, b10); b11 = fmaf(cc, y01, b11); b00 = y00; b01 = y01; gb *= al;
                     }
-                    if ((t & 7) == 7) {
-                        const float sa = 1.f / a11, sb2 = 1.f / b11;
-                        a00 *= sa; a01 *= sa; a10 *= sa; a11 = 1.f;
-                        b00 *= sb2; b01 *= sb2; b10 *= sb2; b11 = 1.f;
-                    }
                 }
-                float *ca = comp + (qt * 128 + ch) * 5;
-                ca[0] = a00; ca[1] = a01; ca[2] = a10; ca[3] = a11; ca[4] = ga;
-                ca[5] = b00; ca[6] = b01; ca[7] = b10; ca[8] = b11; ca[9] = gb;
+                const float sa = 1.f / a11, sb2 = 1.f / b11;
+                *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch) * 4) = make_float4(a00 * sa, a01 * sa, a10 * sa, ga);
+                *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch + 1) * 4) = make_float4(b00 * sb2, b01 * sb2, b10 * sb2, gb);
             }
             __syncthreads();
             float Pa = p0a, Pb = p0b, gama = 1.f, gamb = 1.f;
-            for (int q2 = 0; q2 < qt; ++q2) {
-                const float *ca = comp + (q2 * 128 + ch) * 5;
-                Pa = fmaf(ca[0], Pa, ca[1]) / fmaf(ca[2], Pa, ca[3]);
-                Pb = fmaf(ca[5], Pb, ca[6]) / fmaf(ca[7], Pb, ca[8]);
-                gama *= ca[4];
-                gamb *= ca[9];
+            for (int q2 = 0; q2 < sgi; ++q2) {
+                const float4 ca = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch) * 4);
+                const float4 cb4 = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch + 1) * 4);
+                Pa = fmaf(ca.x, Pa, ca.y) / fmaf(ca.z, Pa, 1.f);
+                Pb = fmaf(cb4.x, Pb, cb4.y) / fmaf(cb4.z, Pb, 1.f);
+                gama *= ca.w;
+                gamb *= cb4.w;
             }
-#pragma unroll 4
-            for (int t = tb; t < tb + 16; ++t) {
+#pragma unroll
+            for (int t = tb; t < tb + 8; ++t) {
                 if ((t & 3) == 0) *reinterpret_cast<float2 *>(gst + (t >> 2) * 128 + ch) = make_float2(gama, gamb);
                 if (t < te) {
                     const uint32_t off = coff + swz(t, cb);
@@ -336,70 +326,43 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             }
         }
         __syncthreads();
-        // ---- elementwise pass (thread = 8 channels x 4 tokens, 16-byte accesses):
+        // ---- elementwise pass (warp = 4 tokens, lane = 4 channels; 8-byte accesses):
         //      K~ = k Gam, Q~ = q Gam, G^ = P^- k / Gam, and den_t = r_t + sum_i P^-_i k_i^2
         {
             const float *pmv = reinterpret_cast<const float *>(sm + L_::A4);
-            const float *gst = reinterpret_cast<const float *>(sm + L_::Y + 7680);
-            const int o = tid & 15, g = tid >> 4, c8 = o * 8;
-            const uint32_t atom8 = (uint32_t)(o >> 3) * 8192u, atom16 = (uint32_t)(o >> 3) * 16384u;
-            const uint32_t chunkb = (uint32_t)(o & 7) * 16u;
-            float gam[8];
-            {
-                const float4 g0 = *reinterpret_cast<const float4 *>(gst + g * 128 + c8);
-                const float4 g1 = *reinterpret_cast<const float4 *>(gst + g * 128 + c8 + 4);
-                gam[0] = g0.x; gam[1] = g0.y; gam[2] = g0.z; gam[3] = g0.w;
-                gam[4] = g1.x; gam[5] = g1.y; gam[6] = g1.z; gam[7] = g1.w;
-            }
+            const float *gst = reinterpret_cast<const float *>(sm + L_::U);
+            const int cq = lane, g = warp, c4 = cq * 4;
+            const uint32_t atom8 = (uint32_t)(cq >> 4) * 8192u, atom16 = (uint32_t)(cq >> 4) * 16384u;
+            const uint32_t bir = (uint32_t)(cq & 15) * 8u;
+            float4 gam = *reinterpret_cast<const float4 *>(gst + g * 128 + c4);
 #pragma unroll 1
             for (int j = 0; j < 4; ++j) {
                 const int t = g * 4 + j;
-                const uint32_t off = swz(t, chunkb);
+                const uint32_t off = swz(t, bir);
                 float xsum = 0.f;
-                uint4 kq = make_uint4(0u, 0u, 0u, 0u), qq = kq, gg = kq;
+                uint2 kq = make_uint2(0u, 0u), qq = kq, gg = kq;
                 if (t < L) {
-                    const uint4 aw = *reinterpret_cast<const uint4 *>(sm + L_::AL + atom8 + off);
-                    const uint4 kw = *reinterpret_cast<const uint4 *>(sm + L_::K + atom8 + off);
-                    const uint4 qw = *reinterpret_cast<const uint4 *>(sm + L_::Q + atom8 + off);
-                    const float4 p0 = *reinterpret_cast<const float4 *>(pmv + t * 128 + c8);
-                    const float4 p1 = *reinterpret_cast<const float4 *>(pmv + t * 128 + c8 + 4);
-                    const uint32_t *ap = reinterpret_cast<const uint32_t *>(&aw);
-                    const uint32_t *kp = reinterpret_cast<const uint32_t *>(&kw);
-                    const uint32_t *qp = reinterpret_cast<const uint32_t *>(&qw);
-                    const float pm[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-                    uint32_t *kqp = reinterpret_cast<uint32_t *>(&kq);
-                    uint32_t *qqp = reinterpret_cast<uint32_t *>(&qq);
-                    uint32_t *ggp = reinterpret_cast<uint32_t *>(&gg);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float al0 = bf16_lo(ap[e]), al1 = bf16_hi(ap[e]);
-                        const float k0 = bf16_lo(kp[e]), k1 = bf16_hi(kp[e]);
-                        gam[2 * e] *= al0;
-                        gam[2 * e + 1] *= al1;
-                        const float pk0 = pm[2 * e] * k0, pk1 = pm[2 * e + 1] * k1;
-                        xsum = fmaf(pk0, k0, xsum);
-                        xsum = fmaf(pk1, k1, xsum);
-                        kqp[e] = pack_bf16x2(k0 * gam[2 * e], k1 * gam[2 * e + 1]);
-                        qqp[e] = pack_bf16x2(bf16_lo(qp[e]) * gam[2 * e], bf16_hi(qp[e]) * gam[2 * e + 1]);
-                        ggp[e] = pack_bf16x2(__fdividef(pk0, gam[2 * e]), __fdividef(pk1, gam[2 * e + 1]));
-                    }
+                    const uint2 aw = *reinterpret_cast<const uint2 *>(sm + L_::AL + atom8 + off);
+                    const uint2 kw = *reinterpret_cast<const uint2 *>(sm + L_::K + atom8 + off);
+                    const uint2 qw = *reinterpret_cast<const uint2 *>(sm + L_::Q + atom8 + off);
+                    const float4 pm = *reinterpret_cast<const float4 *>(pmv + t * 128 + c4);
+                    gam.x *= bf16_lo(aw.x); gam.y *= bf16_hi(aw.x); gam.z *= bf16_lo(aw.y); gam.w *= bf16_hi(aw.y);
+                    const float k0 = bf16_lo(kw.x), k1 = bf16_hi(kw.x), k2 = bf16_lo(kw.y), k3 = bf16_hi(kw.y);
+                    const float p0 = pm.x * k0, p1 = pm.y * k1, p2 = pm.z * k2, p3 = pm.w * k3;
+                    xsum = fmaf(p0, k0, fmaf(p1, k1, fmaf(p2, k2, p3 * k3)));
+                    kq.x = pack_bf16x2(k0 * gam.x, k1 * gam.y);
+                    kq.y = pack_bf16x2(k2 * gam.z, k3 * gam.w);
+                    qq.x = pack_bf16x2(bf16_lo(qw.x) * gam.x, bf16_hi(qw.x) * gam.y);
+                    qq.y = pack_bf16x2(bf16_lo(qw.y) * gam.z, bf16_hi(qw.y) * gam.w);
+                    gg.x = pack_bf16x2(__fdividef(p0, gam.x), __fdividef(p1, gam.y));
+                    gg.y = pack_bf16x2(__fdividef(p2, gam.z), __fdividef(p3, gam.w));
                 }
-                *reinterpret_cast<uint4 *>(sm + L_::KQ + atom16 + swz(t, chunkb)) = kq;
-                *reinterpret_cast<uint4 *>(sm + L_::KQ + atom16 + swz(64 + t, chunkb)) = qq;
-                *reinterpret_cast<uint4 *>(sm + L_::G + atom8 + off) = gg;
-                // den over the 16 lanes that share this token
-                xsum += __shfl_xor_sync(0xffffffffu, xsum, 8);
-                xsum += __shfl_xor_sync(0xffffffffu, xsum, 4);
-                xsum += __shfl_xor_sync(0xffffffffu, xsum, 2);
-                xsum += __shfl_xor_sync(0xffffffffu, xsum, 1);
-                if (o == 0) invden[t] = (t < L) ? 1.f / (r_s[t] + xsum) : 0.f;
+                *reinterpret_cast<uint2 *>(sm + L_::KQ + atom16 + swz(t, bir)) = kq;
+                *reinterpret_cast<uint2 *>(sm + L_::KQ + atom16 + swz(64 + t, bir)) = qq;
+                *reinterpret_cast<uint2 *>(sm + L_::G + atom8 + off) = gg;
+                xsum = warp_sum(xsum);
+                if (lane == 0) invden[t] = (t < L) ? 1.f / (r_s[t] + xsum) : 0.f;
             }
-        }
-        __syncthreads();
-        // q tile of the next chunk (its space is free now)
-        if (tid == 0 && more) {
-            mbar_expect_tx(bar_tma, L_::TMA_BYTES);
-            for (int b = 0; b < 2; ++b) tma_load_3d(sm + L_::Q + b * 8192, &prm.tq, b * 64, h, nxt, bar_tma);
         }
         fence_async_smem();
         tc_fence_before();
@@ -418,31 +381,31 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         }
         wait_mma();
         // rows 0..63 -> A (fp32, strictly lower) ; rows 64..127 -> Aq (bf16, lower incl. diagonal); columns / den
-        float *Af = reinterpret_cast<float *>(sm + L_::K);
-        float *Tf = reinterpret_cast<float *>(sm + L_::SG);
+        float *Af = reinterpret_cast<float *>(sm + L_::AF);
+        float *Tf = reinterpret_cast<float *>(sm + L_::TF);
         {
-            const int row = quad * 32 + lane, s0 = whalf * 32;
-            float v[32];
-            tmem_ld32(T_PREP + lane_off + s0, v);
+            const int s0 = cg * 16;
+            float v[16];
+            tmem_ld16(T_PREP + lane_off + s0, v);
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
+            for (int j = 0; j < 16; j += 4) {
                 const float4 d4 = *reinterpret_cast<const float4 *>(invden + s0 + j);
                 v[j] *= d4.x; v[j + 1] *= d4.y; v[j + 2] *= d4.z; v[j + 3] *= d4.w;
             }
             if (row < 64) {
 #pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4 *>(Af + fsw(row, s0 + j)) =
+                for (int j = 0; j < 16; j += 4)
+                    *reinterpret_cast<float4 *>(Af + row * LDA + s0 + j) =
                         make_float4(s0 + j < row ? v[j] : 0.f, s0 + j + 1 < row ? v[j + 1] : 0.f,
                                     s0 + j + 2 < row ? v[j + 2] : 0.f, s0 + j + 3 < row ? v[j + 3] : 0.f);
             } else {
                 const int t = row - 64;
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
+                for (int j = 0; j < 16; ++j)
                     if (s0 + j > t) v[j] = 0.f;
 #pragma unroll
-                for (int chn = 0; chn < 4; ++chn)
-                    *reinterpret_cast<uint4 *>(sm + L_::AL + swz(t, (whalf * 4 + chn) * 16)) = pack8(v + chn * 8);
+                for (int chn = 0; chn < 2; ++chn)
+                    *reinterpret_cast<uint4 *>(sm + L_::AQ + swz(t, (cg * 2 + chn) * 16)) = pack8(v + chn * 8);
             }
         }
         tc_fence_before();
@@ -450,15 +413,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         tri_inverse64(Af, Tf, tid);
         // T -> bf16, rows 0..63 of Y (row t, column s; zero above the diagonal)
         {
-            const int t = tid >> 2, q4 = tid & 3;
+            const int t = tid >> 3, chn = tid & 7;
+            float v[8];
 #pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                const int chn = q4 * 2 + m;
-                float v[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = (chn * 8 + e <= t) ? Tf[fsw(t, chn * 8 + e)] : 0.f;
-                *reinterpret_cast<uint4 *>(sm + L_::Y + swz(t, chn * 16)) = pack8(v);
-            }
+            for (int e = 0; e < 8; ++e) v[e] = (chn * 8 + e <= t) ? Tf[t * LDA + chn * 8 + e] : 0.f;
+            *reinterpret_cast<uint4 *>(sm + L_::Y + swz(t, chn * 16)) = pack8(v);
         }
         fence_async_smem();
         tc_fence_before();
@@ -469,27 +428,30 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(T_PREP + 64, sdesc(sb + L_::AL + ks * 32u, 16, 1024), sdesc(sb + L_::Y + ks * 2048u, 8192, 1024),
+                mma_bf16(T_PREP + 64, sdesc(sb + L_::AQ + ks * 32u, 16, 1024), sdesc(sb + L_::Y + ks * 2048u, 8192, 1024),
                          ID_M64_N64_KM, ks > 0);
             mma_commit(bar_mma);
-            if (more)   // k and sigma tiles of the next chunk (A and T fp32 are consumed)
+            if (more) {   // q, k and sigma tiles of the next chunk (T and A fp32 are consumed)
+                mbar_expect_tx(bar_tma, L_::TMA_BYTES);
                 for (int b = 0; b < 2; ++b) {
+                    tma_load_3d(sm + L_::Q + b * 8192, &prm.tq, b * 64, h, nxt, bar_tma);
                     tma_load_3d(sm + L_::K + b * 8192, &prm.tk, b * 64, h, nxt, bar_tma);
                     tma_load_3d(sm + L_::SG + b * 8192, &prm.tsg, b * 64, h, nxt, bar_tma);
                 }
+            }
         }
         wait_mma();
         if (tid == 0 && more)   // alpha tile of the next chunk (Aq consumed)
             for (int b = 0; b < 2; ++b) tma_load_3d(sm + L_::AL + b * 8192, &prm.tal, b * 64, h, nxt, bar_tma);
         // X -> bf16, rows 64..127 of Y.  M=64 accumulator: row m sits in lane (m%16) + 32*(m/16).
         {
-            float v[32];
-            tmem_ld32(T_PREP + 64 + lane_off + whalf * 32, v);
+            float v[16];
+            tmem_ld16(T_PREP + 64 + lane_off + cg * 16, v);
             if (lane < 16) {
                 const int t = quad * 16 + lane;
 #pragma unroll
-                for (int chn = 0; chn < 4; ++chn)
-                    *reinterpret_cast<uint4 *>(sm + L_::Y + swz(64 + t, (whalf * 4 + chn) * 16)) = pack8(v + chn * 8);
+                for (int chn = 0; chn < 2; ++chn)
+                    *reinterpret_cast<uint4 *>(sm + L_::Y + swz(64 + t, (cg * 2 + chn) * 16)) = pack8(v + chn * 8);
             }
         }
         fence_async_smem();
@@ -508,28 +470,24 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         wait_mma();
         // rows 0..63 -> -w ; rows 64..127 -> Q' = Q~ - X K~   (bf16 into A4)
         {
-            const int row = quad * 32 + lane;
-#pragma unroll 1
-            for (int cb = whalf * 2; cb < whalf * 2 + 2; ++cb) {
-                float v[32];
-                tmem_ld32(T_PREP + lane_off + cb * 32, v);
-                const uint32_t atom = (uint32_t)(cb >> 1) * 16384u;
+            float v[32];
+            tmem_ld32(T_PREP + lane_off + cg * 32, v);
+            const uint32_t atom = (uint32_t)(cg >> 1) * 16384u;
 #pragma unroll
-                for (int chn = 0; chn < 4; ++chn) {
-                    const uint32_t boff = swz(row, ((cb & 1) * 4 + chn) * 16);
-                    if (row < 64) {
-                        *reinterpret_cast<uint4 *>(sm + L_::A4 + atom + boff) = pack8(v + chn * 8, -1.f);
-                    } else {
-                        const uint4 q4 = *reinterpret_cast<const uint4 *>(sm + L_::KQ + atom + boff);
-                        const uint32_t *qp = reinterpret_cast<const uint32_t *>(&q4);
-                        float w8[8];
+            for (int chn = 0; chn < 4; ++chn) {
+                const uint32_t boff = swz(row, ((cg & 1) * 4 + chn) * 16);
+                if (row < 64) {
+                    *reinterpret_cast<uint4 *>(sm + L_::A4 + atom + boff) = pack8(v + chn * 8, -1.f);
+                } else {
+                    const uint4 q4 = *reinterpret_cast<const uint4 *>(sm + L_::KQ + atom + boff);
+                    const uint32_t *qp = reinterpret_cast<const uint32_t *>(&q4);
+                    float w8[8];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            w8[2 * e] = bf16_lo(qp[e]) - v[chn * 8 + 2 * e];
-                            w8[2 * e + 1] = bf16_hi(qp[e]) - v[chn * 8 + 2 * e + 1];
-                        }
-                        *reinterpret_cast<uint4 *>(sm + L_::A4 + atom + boff) = pack8(w8);
+                    for (int e = 0; e < 4; ++e) {
+                        w8[2 * e] = bf16_lo(qp[e]) - v[chn * 8 + 2 * e];
+                        w8[2 * e + 1] = bf16_hi(qp[e]) - v[chn * 8 + 2 * e + 1];
                     }
+                    *reinterpret_cast<uint4 *>(sm + L_::A4 + atom + boff) = pack8(w8);
                 }
             }
         }
@@ -558,23 +516,19 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 tma_load_3d(sm + L_::V + b * 8192, &prm.tv, tile * DVT + b * 64, h, nxt, bar_tma);
         // rows 0..63 -> U / den (bf16, zero past the chunk end); rows 64..127 -> o (global)
         {
-            const int row = quad * 32 + lane;
-            const float sc = row < 64 ? invden[row] : 1.f;
-#pragma unroll 1
-            for (int cb = whalf * HV; cb < whalf * HV + HV; cb += 32) {
-                float v[32];
-                tmem_ld32(T_D4 + lane_off + cb, v);
-                if (row < 64) {
-                    const uint32_t blk = (uint32_t)(cb >> 6) * 8192u;
+            float v[NC];
+            tmem_ld<NC>(T_D4 + lane_off + cb0, v);
+            if (row < 64) {
+                const float sc = invden[row];
+                const uint32_t blk = (uint32_t)(cb0 >> 6) * 8192u;
 #pragma unroll
-                    for (int chn = 0; chn < 4; ++chn)
-                        *reinterpret_cast<uint4 *>(sm + L_::U + blk + swz(row, (((cb & 63) >> 3) + chn) * 16)) =
-                            pack8(v + chn * 8, sc);
-                } else if (row - 64 < L) {
-                    bf16 *dst = out + ((size_t)(c0 + row - 64) * H + h) * dv + tile * DVT + cb;
+                for (int chn = 0; chn < NC / 8; ++chn)
+                    *reinterpret_cast<uint4 *>(sm + L_::U + blk + swz(row, (((cb0 & 63) >> 3) + chn) * 16)) =
+                        pack8(v + chn * 8, sc);
+            } else if (row - 64 < L) {
+                bf16 *dst = out + ((size_t)(c0 + row - 64) * H + h) * dv + tile * DVT + cb0;
 #pragma unroll
-                    for (int chn = 0; chn < 4; ++chn) *reinterpret_cast<uint4 *>(dst + chn * 8) = pack8(v + chn * 8);
-                }
+                for (int chn = 0; chn < NC / 8; ++chn) *reinterpret_cast<uint4 *>(dst + chn * 8) = pack8(v + chn * 8);
             }
         }
         fence_async_smem();
@@ -593,20 +547,16 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         wait_mma();
         // ---- decay the rows by the chunk's Gam_{L-1}; refresh the bf16 operand copy
         {
-            const int i = quad * 32 + lane;
-            const float gC = gamc[i];
-#pragma unroll 1
-            for (int cb = whalf * HV; cb < whalf * HV + HV; cb += 32) {
-                float v[32];
-                tmem_ld32(T_S + lane_off + cb, v);
+            const float gC = gamc[row];
+            float v[NC];
+            tmem_ld<NC>(T_S + lane_off + cb0, v);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] *= gC;
-                tmem_st32(T_S + lane_off + cb, v);
-                const uint32_t atom = (uint32_t)(cb >> 6) * 16384u;
+            for (int j = 0; j < NC; ++j) v[j] *= gC;
+            tmem_st<NC>(T_S + lane_off + cb0, v);
+            const uint32_t atom = (uint32_t)(cb0 >> 6) * 16384u;
 #pragma unroll
-                for (int chn = 0; chn < 4; ++chn)
-                    *reinterpret_cast<uint4 *>(sm + L_::S + atom + swz(i, (((cb & 63) >> 3) + chn) * 16)) = pack8(v + chn * 8);
-            }
+            for (int chn = 0; chn < NC / 8; ++chn)
+                *reinterpret_cast<uint4 *>(sm + L_::S + atom + swz(row, (((cb0 & 63) >> 3) + chn) * 16)) = pack8(v + chn * 8);
         }
         fence_async_smem();
         tc_fence_before();
@@ -618,16 +568,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     // ---- final state
     if (!*abort_flag) {
         if (a.S_out) {
-            const int i = quad * 32 + lane;
-#pragma unroll 1
-            for (int cb = whalf * HV; cb < whalf * HV + HV; cb += 32) {
-                float v[32];
-                tmem_ld32(T_S + lane_off + cb, v);
+            float v[NC];
+            tmem_ld<NC>(T_S + lane_off + cb0, v);
 #pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4 *>(a.S_out + sbase + (size_t)i * dv + cb + j) =
-                        make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-            }
+            for (int j = 0; j < NC; j += 4)
+                *reinterpret_cast<float4 *>(a.S_out + sbase + (size_t)row * dv + cb0 + j) =
+                    make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         }
         if (a.P_out && tid < DK && tile == 0) a.P_out[(size_t)sh * DK + tid] = pst[tid];
     } else {
