@@ -11,7 +11,8 @@
 //     of the segments' 2x2 maps (CUDA cores, thread = key-channel pair x segment)
 //     K~ = k Gam,  Q~ = q Gam,  G^ = P^- k / Gam   (the gain is G^ Gam / den)
 //     MMA1   [A; Aq] = [K~; Q~] G^^T, columns scaled by 1/den  -> A (s < t), Aq (s <= t)
-//     T = (I + A)^{-1}                               (CUDA cores, blocked 16x16)
+//     T = (I + A)^{-1} = (I - N + N^2 - N^3) D with D the 16x16 diagonal-block inverses
+//     (CUDA cores) and N = D L (L: A below the block diagonal), on the tensor cores (M = 64)
 //     MMA_X  X = Aq T                                (M = 64)
 //     MMA2   [w; X K~] = [T; X] K~ ,  Q' = Q~ - X K~
 //   serial (carries S in TMEM, fp32):
@@ -30,14 +31,14 @@
 namespace kdn {
 
 namespace {
-constexpr int C = 64, DK = 128, NT = 512, LDA = 68;   // LDA: padded fp32 row stride of A and T
+constexpr int C = 64, DK = 128, NT = 512, LDA = 68;   // LDA: padded fp32 row stride of A
 
 template <int DVT>
 struct TcSmem {
-    static constexpr uint32_t Q = 0;                        // q tile (TMA); then T fp32 [64][LDA]
+    static constexpr uint32_t Q = 0;                        // q tile (TMA); then bf16 D and L of the inverse
     static constexpr uint32_t K = Q + 16384;                // k tile (TMA); then A fp32 [64][LDA] at K + 1024
     static constexpr uint32_t AL = K + 16384;               // alpha tile (TMA); then Aq bf16 64 x 64 at AL + 8192
-    static constexpr uint32_t SG = AL + 16384;              // sigma tile (TMA)
+    static constexpr uint32_t SG = AL + 16384;              // sigma tile (TMA); then bf16 N and N^2
     static constexpr uint32_t V = SG + 16384;               // v tile (TMA), DVT*128 B
     static constexpr uint32_t KQ = V + DVT * 128;           // [K~; Q~] bf16, K-major, 2 atoms of 128 rows
     static constexpr uint32_t G = KQ + 32768;               // G^ bf16, 64 token rows x 128 ch
@@ -49,8 +50,9 @@ struct TcSmem {
     static constexpr uint32_t MISC_BYTES = 2048;
     static constexpr uint32_t total = MISC + MISC_BYTES;
     static constexpr uint32_t TMA_BYTES = 4 * 16384 + DVT * 128;
-    static constexpr uint32_t AF = K + 1024, TF = Q, AQ = AL + 8192;
-    static_assert(TF + 64 * LDA * 4 <= AF, "T and A fp32 tiles overlap");
+    static constexpr uint32_t AF = K + 1024, AQ = AL + 8192;
+    // bf16 64x64 operands of the tensor-core triangular inverse (rows of 128 B)
+    static constexpr uint32_t DB = Q, LB = Q + 8192, NB = SG, N2B = SG + 8192, RB = K + 1024;
     static_assert(AF + 64 * LDA * 4 <= AQ, "A fp32 tile overlaps Aq");
     static_assert(DVT * 128 >= 16 * 128 * 4, "U must hold the decay table");
 };
@@ -64,66 +66,6 @@ struct TcParams {
 // the four 16x16 diagonal blocks by forward substitution, then block levels
 // T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj with 1x4 output strips whose dot products are
 // split over `ks` adjacent lanes.  T's strictly-upper blocks are used as scratch.
-__device__ void tri_inverse64(const float *A, float *T, int tid) {
-    if (tid < 64) {
-        const int o = (tid >> 4) * 16, j = tid & 15;
-        float x[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
-#pragma unroll
-        for (int r = 1; r < 16; ++r) {
-            const float *arow = A + (o + r) * LDA + o;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int s = 0; s < r; ++s) acc[s & 3] = fmaf(arow[s], x[s], acc[s & 3]);
-            if (r > j) x[r] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) T[(o + r) * LDA + o + j] = x[r];
-    }
-    __syncthreads();
-    for (int lvl = 1; lvl < 4; ++lvl) {
-        const int items = (4 - lvl) * 64, ks = lvl == 1 ? 2 : (lvl == 2 ? 4 : 8);
-        const int item = tid / ks, kp = tid % ks;
-        const bool live = item < items;
-        const int bj = item >> 6, bi = bj + lvl, rr = (item >> 2) & 15, c4 = (item & 3) * 4;
-        const int row = bi * 16 + rr;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (live) {
-            const float *arow = A + row * LDA;
-            for (int kk = bj * 16 + kp; kk < bi * 16; kk += ks) {
-                const float av = arow[kk];
-                const float4 tv = *reinterpret_cast<const float4 *>(T + kk * LDA + bj * 16 + c4);
-                acc.x = fmaf(av, tv.x, acc.x); acc.y = fmaf(av, tv.y, acc.y);
-                acc.z = fmaf(av, tv.z, acc.z); acc.w = fmaf(av, tv.w, acc.w);
-            }
-        }
-        for (int off = 1; off < ks; off <<= 1) {
-            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off); acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
-            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off); acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
-        }
-        if (live && kp == 0) *reinterpret_cast<float4 *>(T + (bj * 16 + rr) * LDA + bi * 16 + c4) = acc;   // parked
-        __syncthreads();
-        acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (live) {
-            const float *trow = T + row * LDA + bi * 16;
-            for (int uu = kp; uu <= rr; uu += ks) {
-                const float tv = trow[uu];
-                const float4 mv = *reinterpret_cast<const float4 *>(T + (bj * 16 + uu) * LDA + bi * 16 + c4);
-                acc.x = fmaf(tv, mv.x, acc.x); acc.y = fmaf(tv, mv.y, acc.y);
-                acc.z = fmaf(tv, mv.z, acc.z); acc.w = fmaf(tv, mv.w, acc.w);
-            }
-        }
-        for (int off = 1; off < ks; off <<= 1) {
-            acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off); acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
-            acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off); acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
-        }
-        if (live && kp == 0)
-            *reinterpret_cast<float4 *>(T + row * LDA + bj * 16 + c4) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-        __syncthreads();
-    }
-}
-
 // pack 8 floats (scaled) into one 16-byte bf16 chunk
 __device__ __forceinline__ uint4 pack8(const float *v, float sc = 1.f) {
     uint4 w;
@@ -263,26 +205,35 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             const uint32_t coff = (uint32_t)(ch >> 6) * 8192u, cb = (uint32_t)(ch & 63) * 2u;
             const float p0a = pst[ch], p0b = pst[ch + 1];
             const int tb = sgi * 8, te = min(L, tb + 8);
+            // this thread's 8 tokens of alpha, sigma, k (2 channels each) and mu / r, loaded up front
+            uint32_t aw8[8], sw8[8], kw8[8];
+            float mr8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t off = coff + swz(tb + j, cb);
+                aw8[j] = *reinterpret_cast<const uint32_t *>(sm + L_::AL + off);
+                sw8[j] = *reinterpret_cast<const uint32_t *>(sm + L_::SG + off);
+                kw8[j] = *reinterpret_cast<const uint32_t *>(sm + L_::K + off);
+                mr8[j] = mur[tb + j];
+            }
             if (sgi < 7 && te > tb) {
                 float a00 = 1.f, a01 = 0.f, a10 = 0.f, a11 = 1.f, ga = 1.f;
                 float b00 = 1.f, b01 = 0.f, b10 = 0.f, b11 = 1.f, gb = 1.f;
-                for (int t = tb; t < te; ++t) {
-                    const uint32_t off = coff + swz(t, cb);
-                    const uint32_t aw = *reinterpret_cast<const uint32_t *>(sm + L_::AL + off);
-                    const uint32_t sw = *reinterpret_cast<const uint32_t *>(sm + L_::SG + off);
-                    const uint32_t kw = *reinterpret_cast<const uint32_t *>(sm + L_::K + off);
-                    const float mr = mur[t];
-                    {
-                        const float al = bf16_lo(aw), sg = bf16_lo(sw), kk = bf16_lo(kw);
-                        const float aa = al * al, cc = mr * kk * kk;
-                        const float y00 = fmaf(aa, a00, sg * a10), y01 = fmaf(aa, a01, sg * a11);
-                        a10 = fmaf(cc, y00, a10); a11 = fmaf(cc, y01, a11); a00 = y00; a01 = y01; ga *= al;
-                    }
-                    {
-                        const float al = bf16_hi(aw), sg = bf16_hi(sw), kk = bf16_hi(kw);
-                        const float aa = al * al, cc = mr * kk * kk;
-                        const float y00 = fmaf(aa, b00, sg * b10), y01 = fmaf(aa, b01, sg * b11);
-                        b10 = fmaf(cc, y00, b10); b11 = fmaf(cc, y01, b11); b00 = y00; b01 = y01; gb *= al;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (tb + j < te) {
+                        {
+                            const float al = bf16_lo(aw8[j]), sg = bf16_lo(sw8[j]), kk = bf16_lo(kw8[j]);
+                            const float aa = al * al, cc = mr8[j] * kk * kk;
+                            const float y00 = fmaf(aa, a00, sg * a10), y01 = fmaf(aa, a01, sg * a11);
+                            a10 = fmaf(cc, y00, a10); a11 = fmaf(cc, y01, a11); a00 = y00; a01 = y01; ga *= al;
+                        }
+                        {
+                            const float al = bf16_hi(aw8[j]), sg = bf16_hi(sw8[j]), kk = bf16_hi(kw8[j]);
+                            const float aa = al * al, cc = mr8[j] * kk * kk;
+                            const float y00 = fmaf(aa, b00, sg * b10), y01 = fmaf(aa, b01, sg * b11);
+                            b10 = fmaf(cc, y00, b10); b11 = fmaf(cc, y01, b11); b00 = y00; b01 = y01; gb *= al;
+                        }
                     }
                 }
                 const float sa = 1.f / a11, sb2 = 1.f / b11;
@@ -299,24 +250,27 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 gama *= ca.w;
                 gamb *= cb4.w;
             }
+            float pma8[8], pmb8[8];
 #pragma unroll
-            for (int t = tb; t < tb + 8; ++t) {
+            for (int j = 0; j < 8; ++j) {
+                const int t = tb + j;
                 if ((t & 3) == 0) *reinterpret_cast<float2 *>(gst + (t >> 2) * 128 + ch) = make_float2(gama, gamb);
+                pma8[j] = 0.f;
+                pmb8[j] = 0.f;
                 if (t < te) {
-                    const uint32_t off = coff + swz(t, cb);
-                    const uint32_t aw = *reinterpret_cast<const uint32_t *>(sm + L_::AL + off);
-                    const uint32_t sw = *reinterpret_cast<const uint32_t *>(sm + L_::SG + off);
-                    const uint32_t kw = *reinterpret_cast<const uint32_t *>(sm + L_::K + off);
-                    const float mr = mur[t];
-                    const float ala = bf16_lo(aw), alb = bf16_hi(aw), ka = bf16_lo(kw), kb = bf16_hi(kw);
-                    const float pma = fmaf(ala * ala, Pa, bf16_lo(sw)), pmb = fmaf(alb * alb, Pb, bf16_hi(sw));
-                    *reinterpret_cast<float2 *>(pmv + t * 128 + ch) = make_float2(pma, pmb);
-                    Pa = __fdividef(pma, fmaf(mr * ka * ka, pma, 1.f));
-                    Pb = __fdividef(pmb, fmaf(mr * kb * kb, pmb, 1.f));
+                    const float ala = bf16_lo(aw8[j]), alb = bf16_hi(aw8[j]), ka = bf16_lo(kw8[j]), kb = bf16_hi(kw8[j]);
+                    const float pma = fmaf(ala * ala, Pa, bf16_lo(sw8[j])), pmb = fmaf(alb * alb, Pb, bf16_hi(sw8[j]));
+                    pma8[j] = pma;
+                    pmb8[j] = pmb;
+                    Pa = __fdividef(pma, fmaf(mr8[j] * ka * ka, pma, 1.f));
+                    Pb = __fdividef(pmb, fmaf(mr8[j] * kb * kb, pmb, 1.f));
                     gama *= ala;
                     gamb *= alb;
                 }
             }
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (tb + j < te) *reinterpret_cast<float2 *>(pmv + (tb + j) * 128 + ch) = make_float2(pma8[j], pmb8[j]);
             if (te == L && tb < L) {     // this thread processed the chunk's last token
                 pst[ch] = Pa;
                 pst[ch + 1] = Pb;
@@ -335,33 +289,52 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             const uint32_t atom8 = (uint32_t)(cq >> 4) * 8192u, atom16 = (uint32_t)(cq >> 4) * 16384u;
             const uint32_t bir = (uint32_t)(cq & 15) * 8u;
             float4 gam = *reinterpret_cast<const float4 *>(gst + g * 128 + c4);
-#pragma unroll 1
+            uint2 aw[4], kw[4], qw[4];
+            float4 pm[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {   // loads for the warp's four tokens first
+                const int t = g * 4 + j;
+                const uint32_t off = swz(t, bir);
+                aw[j] = *reinterpret_cast<const uint2 *>(sm + L_::AL + atom8 + off);
+                kw[j] = *reinterpret_cast<const uint2 *>(sm + L_::K + atom8 + off);
+                qw[j] = *reinterpret_cast<const uint2 *>(sm + L_::Q + atom8 + off);
+                pm[j] = *reinterpret_cast<const float4 *>(pmv + t * 128 + c4);
+            }
+            float xs[4];
+            uint2 kq[4], qq[4], gg[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int t = g * 4 + j;
+                kq[j] = make_uint2(0u, 0u); qq[j] = kq[j]; gg[j] = kq[j]; xs[j] = 0.f;
+                if (t < L) {
+                    gam.x *= bf16_lo(aw[j].x); gam.y *= bf16_hi(aw[j].x); gam.z *= bf16_lo(aw[j].y); gam.w *= bf16_hi(aw[j].y);
+                    const float k0 = bf16_lo(kw[j].x), k1 = bf16_hi(kw[j].x), k2 = bf16_lo(kw[j].y), k3 = bf16_hi(kw[j].y);
+                    const float p0 = pm[j].x * k0, p1 = pm[j].y * k1, p2 = pm[j].z * k2, p3 = pm[j].w * k3;
+                    xs[j] = fmaf(p0, k0, fmaf(p1, k1, fmaf(p2, k2, p3 * k3)));
+                    kq[j].x = pack_bf16x2(k0 * gam.x, k1 * gam.y);
+                    kq[j].y = pack_bf16x2(k2 * gam.z, k3 * gam.w);
+                    qq[j].x = pack_bf16x2(bf16_lo(qw[j].x) * gam.x, bf16_hi(qw[j].x) * gam.y);
+                    qq[j].y = pack_bf16x2(bf16_lo(qw[j].y) * gam.z, bf16_hi(qw[j].y) * gam.w);
+                    gg[j].x = pack_bf16x2(__fdividef(p0, gam.x), __fdividef(p1, gam.y));
+                    gg[j].y = pack_bf16x2(__fdividef(p2, gam.z), __fdividef(p3, gam.w));
+                }
+            }
+#pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int t = g * 4 + j;
                 const uint32_t off = swz(t, bir);
-                float xsum = 0.f;
-                uint2 kq = make_uint2(0u, 0u), qq = kq, gg = kq;
-                if (t < L) {
-                    const uint2 aw = *reinterpret_cast<const uint2 *>(sm + L_::AL + atom8 + off);
-                    const uint2 kw = *reinterpret_cast<const uint2 *>(sm + L_::K + atom8 + off);
-                    const uint2 qw = *reinterpret_cast<const uint2 *>(sm + L_::Q + atom8 + off);
-                    const float4 pm = *reinterpret_cast<const float4 *>(pmv + t * 128 + c4);
-                    gam.x *= bf16_lo(aw.x); gam.y *= bf16_hi(aw.x); gam.z *= bf16_lo(aw.y); gam.w *= bf16_hi(aw.y);
-                    const float k0 = bf16_lo(kw.x), k1 = bf16_hi(kw.x), k2 = bf16_lo(kw.y), k3 = bf16_hi(kw.y);
-                    const float p0 = pm.x * k0, p1 = pm.y * k1, p2 = pm.z * k2, p3 = pm.w * k3;
-                    xsum = fmaf(p0, k0, fmaf(p1, k1, fmaf(p2, k2, p3 * k3)));
-                    kq.x = pack_bf16x2(k0 * gam.x, k1 * gam.y);
-                    kq.y = pack_bf16x2(k2 * gam.z, k3 * gam.w);
-                    qq.x = pack_bf16x2(bf16_lo(qw.x) * gam.x, bf16_hi(qw.x) * gam.y);
-                    qq.y = pack_bf16x2(bf16_lo(qw.y) * gam.z, bf16_hi(qw.y) * gam.w);
-                    gg.x = pack_bf16x2(__fdividef(p0, gam.x), __fdividef(p1, gam.y));
-                    gg.y = pack_bf16x2(__fdividef(p2, gam.z), __fdividef(p3, gam.w));
-                }
-                *reinterpret_cast<uint2 *>(sm + L_::KQ + atom16 + swz(t, bir)) = kq;
-                *reinterpret_cast<uint2 *>(sm + L_::KQ + atom16 + swz(64 + t, bir)) = qq;
-                *reinterpret_cast<uint2 *>(sm + L_::G + atom8 + off) = gg;
-                xsum = warp_sum(xsum);
-                if (lane == 0) invden[t] = (t < L) ? 1.f / (r_s[t] + xsum) : 0.f;
+                *reinterpret_cast<uint2 *>(sm + L_::KQ + atom16 + off) = kq[j];
+                *reinterpret_cast<uint2 *>(sm + L_::KQ + atom16 + swz(64 + t, bir)) = qq[j];
+                *reinterpret_cast<uint2 *>(sm + L_::G + atom8 + off) = gg[j];
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) xs[j] += __shfl_xor_sync(0xffffffffu, xs[j], off);
+            if (lane < 4) {
+                const int t = g * 4 + lane;
+                const float xv = lane == 0 ? xs[0] : (lane == 1 ? xs[1] : (lane == 2 ? xs[2] : xs[3]));
+                invden[t] = (t < L) ? __fdividef(1.f, r_s[t] + xv) : 0.f;
             }
         }
         fence_async_smem();
@@ -382,7 +355,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         wait_mma();
         // rows 0..63 -> A (fp32, strictly lower) ; rows 64..127 -> Aq (bf16, lower incl. diagonal); columns / den
         float *Af = reinterpret_cast<float *>(sm + L_::AF);
-        float *Tf = reinterpret_cast<float *>(sm + L_::TF);
         {
             const int s0 = cg * 16;
             float v[16];
@@ -410,14 +382,96 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         }
         tc_fence_before();
         __syncthreads();
-        tri_inverse64(Af, Tf, tid);
-        // T -> bf16, rows 0..63 of Y (row t, column s; zero above the diagonal)
+        // ---- T = (I + A)^{-1} on the tensor cores.  With D the four 16x16 diagonal-block inverses
+        //      (CUDA cores) and L the blocks of A below the block diagonal, N = D L is nilpotent
+        //      (N^4 = 0) and T = (I + D L)^{-1} D = (I - N + N^2 - N^3) D.
         {
-            const int t = tid >> 3, chn = tid & 7;
-            float v[8];
+            float *Db4 = reinterpret_cast<float *>(sm + L_::Y);   // [4][16][16] fp32 diagonal blocks of D
+            if (tid < 64) {
+                const int o = (tid >> 4) * 16, j = tid & 15;
+                float x[16];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = (chn * 8 + e <= t) ? Tf[t * LDA + chn * 8 + e] : 0.f;
-            *reinterpret_cast<uint4 *>(sm + L_::Y + swz(t, chn * 16)) = pack8(v);
+                for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
+#pragma unroll
+                for (int r = 1; r < 16; ++r) {
+                    const float *arow = Af + (o + r) * LDA + o;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int c = 0; c < r; ++c) acc[c & 3] = fmaf(arow[c], x[c], acc[c & 3]);
+                    if (r > j) x[r] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
+                }
+#pragma unroll
+                for (int r = 0; r < 16; ++r) Db4[(o + r) * 16 + j] = x[r];
+            }
+            __syncthreads();
+            {   // bf16 D (block diagonal) and L (below the block diagonal): one 16-byte chunk per thread each
+                const int r = tid >> 3, cc = tid & 7, b = r >> 4, cb = cc >> 1;
+                float dv8[8], lv8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int c = cc * 8 + e;
+                    dv8[e] = (cb == b) ? Db4[r * 16 + (c & 15)] : 0.f;
+                    lv8[e] = (cb < b) ? Af[r * LDA + c] : 0.f;
+                }
+                *reinterpret_cast<uint4 *>(sm + L_::DB + swz(r, cc * 16)) = pack8(dv8);
+                *reinterpret_cast<uint4 *>(sm + L_::LB + swz(r, cc * 16)) = pack8(lv8);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            // M=64 x N=64 x K=64 product: A operand K-major (rows of 128 B), B operand MN-major
+            auto mma64 = [&](uint32_t dcol, uint32_t aoff, uint32_t boff) {
+                if (tid == 0) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16(dcol, sdesc(sb + aoff + ks * 32u, 16, 1024), sdesc(sb + boff + ks * 2048u, 8192, 1024),
+                                 ID_M64_N64_KM, ks > 0);
+                    mma_commit(bar_mma);
+                }
+                wait_mma();
+            };
+            // M=64 accumulator rows: row m sits in lane (m%16) + 32*(m/16); this warp reads
+            // columns cg*16 .. cg*16+15 of rows quad*16 + lane (lanes < 16)
+            const int m64 = quad * 16 + lane;
+            auto store64 = [&](uint32_t dst, float (&v)[16]) {
+                if (lane < 16) {
+#pragma unroll
+                    for (int chn = 0; chn < 2; ++chn)
+                        *reinterpret_cast<uint4 *>(sm + dst + swz(m64, (cg * 2 + chn) * 16)) = pack8(v + chn * 8);
+                }
+            };
+            auto sync_tc = [&]() {
+                fence_async_smem();
+                tc_fence_before();
+                __syncthreads();
+            };
+            mma64(T_PREP, L_::DB, L_::LB);                        // N = D L
+            { float v[16]; tmem_ld16(T_PREP + lane_off + cg * 16, v); store64(L_::NB, v); }
+            sync_tc();
+            mma64(T_PREP + 64, L_::NB, L_::NB);                   // N^2
+            { float v[16]; tmem_ld16(T_PREP + 64 + lane_off + cg * 16, v); store64(L_::N2B, v); }
+            sync_tc();
+            mma64(T_D4, L_::N2B, L_::NB);                         // N^3 (the state-update columns are free here)
+            {   // R = I - N + N^2 - N^3
+                float n1[16], n2[16], n3[16];
+                tmem_ld16(T_PREP + lane_off + cg * 16, n1);
+                tmem_ld16(T_PREP + 64 + lane_off + cg * 16, n2);
+                tmem_ld16(T_D4 + lane_off + cg * 16, n3);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) n1[j] = (cg * 16 + j == m64 ? 1.f : 0.f) - n1[j] + n2[j] - n3[j];
+                store64(L_::RB, n1);
+            }
+            sync_tc();
+            mma64(T_PREP, L_::RB, L_::DB);                        // T = R D
+            {   // T -> bf16, rows 0..63 of Y (zero above the diagonal)
+                float v[16];
+                tmem_ld16(T_PREP + lane_off + cg * 16, v);
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    if (cg * 16 + j > m64) v[j] = 0.f;
+                store64(L_::Y, v);
+            }
         }
         fence_async_smem();
         tc_fence_before();
@@ -431,7 +485,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 mma_bf16(T_PREP + 64, sdesc(sb + L_::AQ + ks * 32u, 16, 1024), sdesc(sb + L_::Y + ks * 2048u, 8192, 1024),
                          ID_M64_N64_KM, ks > 0);
             mma_commit(bar_mma);
-            if (more) {   // q, k and sigma tiles of the next chunk (T and A fp32 are consumed)
+            if (more) {   // q, k and sigma tiles of the next chunk (the inverse's operands are consumed)
                 mbar_expect_tx(bar_tma, L_::TMA_BYTES);
                 for (int b = 0; b < 2; ++b) {
                     tma_load_3d(sm + L_::Q + b * 8192, &prm.tq, b * 64, h, nxt, bar_tma);
