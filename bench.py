@@ -148,14 +148,23 @@ def barrier(world):
         torch.cuda.synchronize()
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """The largest of the ranks' values (each rank's device-timed duration); one scalar
+    all-reduce, the only collective of the benchmark."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank_per_step, steps, local_ms, world, device="cuda"):
+    """Weak scaling: every rank processes its own batch; the job's rate is all ranks' units
+    divided by the slowest rank's time.  Returns (rate per second, max ms)."""
+    ms = max_over_ranks(local_ms, world, device)
+    return world * units_per_rank_per_step * steps / (ms / 1e3), ms
 
 
 # ------------------------------------------------------------------ our arm
@@ -211,11 +220,9 @@ def bench_prefill(args, world, rank, dev, kdn):
         barrier(world)
     kdn.last_device_error()
     per_step_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
-    total_ms = evs[0].elapsed_time(evs[-1])
-    total_ms = max_over_ranks(total_ms, world)
-    ms_step = total_ms / args.steps
     tokens = w.ntok  # per rank, all heads included
-    value = world * tokens * args.steps / (total_ms / 1e3)
+    value, total_ms = whole_job_rate(tokens, args.steps, evs[0].elapsed_time(evs[-1]), world)
+    ms_step = total_ms / args.steps
 
     # end to end through the C ABI: pinned host inputs -> device, forward, o -> host
     pinned = {n: torch.from_numpy(np.ascontiguousarray(host[n]).view(np.int16) if host[n].dtype == np.uint16
@@ -242,8 +249,7 @@ def bench_prefill(args, world, rank, dev, kdn):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = world * tokens * e_steps / (e2e_ms / 1e3)
+    e2e_value, e2e_ms = whole_job_rate(tokens, e_steps, e0.elapsed_time(e1), world)
 
     # the uncertainty / gain scan on its own, over the same inputs (g fp32, k^T g, final P)
     scan = None
