@@ -324,10 +324,35 @@ def bench_decode(args, world, rank, dev, kdn, steps=1024, N=256, H=32, d=128):
     barrier(world)
     kdn.last_device_error()
     ms = max_over_ranks(e0.elapsed_time(e1), world)
+    # the same tokens four per launch (multi-token decode: one state read/write per 4 tokens)
+    multi = None
+    if steps % 4 == 0:
+        q4, k4, v4, a4, s4, r4 = [x.view((steps // 4, 4) + x.shape[1:]).transpose(0, 1) for x in (q, k, v, al, sg, r)]
+        groups = [tuple(t[:, j].transpose(0, 1).contiguous() for t in (q4, k4, v4, a4, s4, r4)) for j in range(steps // 4)]
+        o4 = torch.empty((N, 4, H, d), dtype=torch.bfloat16, device=dev)
+
+        def run4(n):
+            for j in range(n):
+                kdn.decode_tokens(*groups[j], S, P, o=o4)
+        run4(min(len(groups), 3))
+        barrier(world)
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        m0.record(stream)
+        run4(len(groups))
+        m1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        kdn.last_device_error()
+        mms = max_over_ranks(m0.elapsed_time(m1), world)
+        # per launch: S and P read and written once, four tokens' inputs and outputs
+        b4 = N * H * (2 * d * d * 4 + 2 * d * 4 + 4 * ((4 * d + d) * 2 + 2 + d * 2))
+        multi = dict(value=world * steps / (mms / 1e3), ms_per_launch=mms / len(groups), launches=len(groups),
+                     bytes=b4)
     per_step = ms / steps
     head_step_bytes = 2 * d * d * 4 + 2 * d * 4 + (4 * d + d) * 2 + 2 + d * 2
     nbytes = N * H * head_step_bytes
-    return dict(value=world * steps / (ms / 1e3), ms_step=per_step, bytes=nbytes, steps=steps, N=N, H=H, d=d)
+    return dict(value=world * steps / (ms / 1e3), ms_step=per_step, bytes=nbytes, steps=steps, N=N, H=H, d=d,
+                multi=multi)
 
 
 def cpu_baseline_prefill(w, min_seconds=10.0, max_reps=50):
@@ -422,6 +447,15 @@ def ours(args):
                               "roofline": {"bound": "hbm", "achieved": dach, "peak": hbm, "unit": "GB/s",
                                            "frac": dach / hbm, "traffic": None,
                                            "algorithmic_bytes_per_launch": dec["bytes"]}}
+            if dec["multi"] is not None:
+                line["decode"]["four_tokens_per_launch"] = {
+                    "metric": "decode steps/s, 4 tokens per launch", "value": dec["multi"]["value"], "unit": "steps/s",
+                    "ms_per_launch": dec["multi"]["ms_per_launch"], "gpu_launches": dec["multi"]["launches"]}
+                m = dec["multi"]
+                mach = m["bytes"] / (m["ms_per_launch"] / 1e3) / 1e9
+                line["decode"]["four_tokens_per_launch"]["roofline"] = {
+                    "bound": "hbm", "achieved": mach, "peak": hbm, "unit": "GB/s", "frac": mach / hbm,
+                    "traffic": None, "algorithmic_bytes_per_launch": m["bytes"]}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -109,6 +109,20 @@ kdn_status_t kdn_decode_step(int N, int H, int d_k, int d_v, kdn_dtype_t in_dtyp
                              const void *alpha, const void *sigma, const void *r,
                              float *S, float *P, void *o, void *stream);
 
+/* Several autoregressive tokens per launch for N independent sequences (multi-token /
+ * speculative decode): the n_tokens tokens of each sequence are applied in order to the
+ * state, which is read once and written back once in place -- the state traffic of one
+ * step is shared by n_tokens tokens (KDA article, fused recurrent regime; its closing
+ * remark pairs chunkwise processing with speculative decoding).
+ *  q, k, alpha, sigma : device [N, n_tokens, H, d_k] (in_dtype);  v : device [N, n_tokens, H, d_v]
+ *  r                  : device [N, n_tokens, H];  o : device [N, n_tokens, H, d_v] (in_dtype)
+ *  S, P               : device fp32 [N, H, d_k, d_v], [N, H, d_k], updated in place
+ * n_tokens == 1 is kdn_decode_step with the token axis made explicit. */
+kdn_status_t kdn_decode_tokens(int N, int n_tokens, int H, int d_k, int d_v, kdn_dtype_t in_dtype, float mu,
+                               const void *q, const void *k, const void *v,
+                               const void *alpha, const void *sigma, const void *r,
+                               float *S, float *P, void *o, void *stream);
+
 /* The uncertainty / gain scan on its own (explainer, closing paragraph of "各向同性近似":
  * the uncertainty recursion is a Moebius map whose 2x2 matrices compose, so it runs
  * as an associative scan).  Independent of the memory S.

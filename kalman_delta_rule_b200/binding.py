@@ -44,6 +44,7 @@ _SIGS = {
     "kdn_workspace_size": (_i, [_PP, ctypes.POINTER(_sz)]),
     "kdn_forward_chunkwise": (_i, [_PP] + [_vp] * 6 + [_vp] * 2 + [_vp] * 3 + [_vp, _sz, _vp]),
     "kdn_decode_step": (_i, [_i, _i, _i, _i, _i, _f] + [_vp] * 6 + [_vp] * 3 + [_vp]),
+    "kdn_decode_tokens": (_i, [_i, _i, _i, _i, _i, _i, _f] + [_vp] * 6 + [_vp] * 3 + [_vp]),
     "kdn_gain_scan": (_i, [_PP] + [_vp] * 4 + [_vp] + [_vp] * 3 + [_vp, _sz, _vp]),
     "kdn_last_device_error": (_i, [_vp]),
     "kdn_status_string": (ctypes.c_char_p, [_i]),
@@ -85,6 +86,10 @@ def kdn_forward_chunkwise(problem, q, k, v, alpha, sigma, r, S0, P0, o, S_out, P
 
 def kdn_decode_step(N, H, d_k, d_v, in_dtype, mu, q, k, v, alpha, sigma, r, S, P, o, stream):
     return load().kdn_decode_step(N, H, d_k, d_v, in_dtype, mu, q, k, v, alpha, sigma, r, S, P, o, stream)
+
+
+def kdn_decode_tokens(N, n_tokens, H, d_k, d_v, in_dtype, mu, q, k, v, alpha, sigma, r, S, P, o, stream):
+    return load().kdn_decode_tokens(N, n_tokens, H, d_k, d_v, in_dtype, mu, q, k, v, alpha, sigma, r, S, P, o, stream)
 
 
 def kdn_gain_scan(problem, k, alpha, sigma, r, P0, g, beta_eff, P_out, workspace, workspace_bytes, stream):
@@ -198,6 +203,19 @@ def decode_step(q, k, v, alpha, sigma, r, S, P, mu: float = 1.0, o=None, stream=
     st = kdn_decode_step(N, H, dk, dv, _dtype_code(q), float(mu), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
                          _ptr(sigma), _ptr(r), _ptr(S), _ptr(P), _ptr(o), _stream_handle(stream))
     _check(st, "kdn_decode_step")
+    return o
+
+
+def decode_tokens(q, k, v, alpha, sigma, r, S, P, mu: float = 1.0, o=None, stream=None):
+    """n tokens per sequence in one launch on [N, n, H, d] token tensors; S, P updated in place."""
+    torch = _torch()
+    N, n, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((N, n, H, dv), dtype=q.dtype, device=q.device)
+    st = kdn_decode_tokens(N, n, H, dk, dv, _dtype_code(q), float(mu), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                           _ptr(sigma), _ptr(r), _ptr(S), _ptr(P), _ptr(o), _stream_handle(stream))
+    _check(st, "kdn_decode_tokens")
     return o
 
 

@@ -124,22 +124,29 @@ kdn_status_t kdn_forward_chunkwise(const kdn_problem_t *p, const void *q, const 
     return cuda_status(kdn::launch_chunk_simt(a, rv.bf16, p->chunk, cs));
 }
 
-kdn_status_t kdn_decode_step(int N, int H, int d_k, int d_v, kdn_dtype_t in_dtype, float mu, const void *q,
-                             const void *k, const void *v, const void *alpha, const void *sigma, const void *r,
-                             float *S, float *P, void *o, void *stream) {
-    if (N < 0 || H <= 0 || !(mu > 0.f) || !isfinite(mu)) return KDN_ERR_INVALID_ARG;
+kdn_status_t kdn_decode_tokens(int N, int n_tokens, int H, int d_k, int d_v, kdn_dtype_t in_dtype, float mu,
+                               const void *q, const void *k, const void *v, const void *alpha, const void *sigma,
+                               const void *r, float *S, float *P, void *o, void *stream) {
+    if (N < 0 || n_tokens < 0 || H <= 0 || !(mu > 0.f) || !isfinite(mu)) return KDN_ERR_INVALID_ARG;
     if (in_dtype != KDN_DTYPE_F32 && in_dtype != KDN_DTYPE_BF16) return KDN_ERR_INVALID_ARG;
     if (!dk_ok(d_k) || !dv_ok(d_v)) return KDN_ERR_UNSUPPORTED;
-    if (N == 0) return KDN_OK;
+    if (N == 0 || n_tokens == 0) return KDN_OK;
+    if ((long long)N * n_tokens > (1ll << 30)) return KDN_ERR_UNSUPPORTED;
     const void *ptrs[] = {q, k, v, alpha, sigma, r, S, P, o};
     for (const void *ptr : ptrs)
         if (!ptr || !aligned16(ptr)) return KDN_ERR_INVALID_ARG;
     kdn::TokenArgs a{};
     a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.sigma = sigma; a.r = r; a.o = o;
     a.S0 = S; a.P0 = P; a.S_out = S; a.P_out = P;
-    a.cu = nullptr; a.T = 1; a.nseq = N; a.H = H; a.dk = d_k; a.dv = d_v; a.mu = mu; a.err = err_word();
-    // one tile per head: the in-place uncertainty is read and written by one CTA
+    a.cu = nullptr; a.T = n_tokens; a.nseq = N; a.H = H; a.dk = d_k; a.dv = d_v; a.mu = mu; a.err = err_word();
+    // one tile per head: the in-place state and uncertainty are read and written by one CTA
     return cuda_status(kdn::launch_recurrent(a, in_dtype == KDN_DTYPE_BF16, d_v, static_cast<cudaStream_t>(stream)));
+}
+
+kdn_status_t kdn_decode_step(int N, int H, int d_k, int d_v, kdn_dtype_t in_dtype, float mu, const void *q,
+                             const void *k, const void *v, const void *alpha, const void *sigma, const void *r,
+                             float *S, float *P, void *o, void *stream) {
+    return kdn_decode_tokens(N, 1, H, d_k, d_v, in_dtype, mu, q, k, v, alpha, sigma, r, S, P, o, stream);
 }
 
 static kdn_status_t scan_args(const kdn_problem_t *p, const void *k, const void *alpha, const void *sigma,

@@ -111,3 +111,29 @@ def test_decode_full_size_sampled(kdn):
         assert max_rel_err(o[:, ns, h], ref["o"][:, 0, 0]) <= TOL_BF16
         assert max_rel_err(S[ns, h], ref["S"][0, 0]) <= TOL_BF16
         assert max_rel_err(P[ns, h], ref["P"][0, 0]) <= TOL_BF16
+
+
+@pytest.mark.parametrize("n", [1, 4, 7])
+def test_decode_tokens_matches_oracle_and_single_steps(kdn, n):
+    """n tokens per launch (multi-token decode) = the oracle's n steps, and bit-identical to
+    n single-token decode steps (the same per-token arithmetic, the state kept on chip)."""
+    import torch
+    N, H, dk, dv = 6, 3, 128, 128
+    rng = np.random.default_rng(n)
+    S0 = (0.1 * rng.standard_normal((N, H, dk, dv))).astype(np.float32)
+    P0 = np.logaddexp(0, rng.standard_normal((N, H, dk))).astype(np.float32)
+    steps = [inputs.draw_tokens((11, n, s), N, H, dk, dv, True) for s in range(n)]
+    stacked = {nm: np.stack([st[nm] for st in steps], axis=1) for nm in steps[0]}   # [N, n, H, ...]
+    S, P = to_dev(S0).clone(), to_dev(P0).clone()
+    o = kdn.decode_tokens(*[to_dev(stacked[nm]) for nm in ("q", "k", "v", "alpha", "sigma", "r")], S, P, mu=2.0)
+    torch.cuda.synchronize()
+    kdn.last_device_error()
+    ref = oracle.run_decode(S0, P0, steps, mu=2.0)
+    o_h = to_host(o).transpose(1, 0, 2, 3)   # [n, N, H, dv]
+    assert max_rel_err(o_h, ref["o"]) <= TOL_BF16
+    assert max_rel_err(to_host(S), ref["S"]) <= TOL_BF16
+    assert max_rel_err(to_host(P), ref["P"]) <= TOL_BF16
+    o1, S1, P1 = decode_run(kdn, S0, P0, steps, mu=2.0)
+    np.testing.assert_array_equal(to_host(S), S1)
+    np.testing.assert_array_equal(to_host(P), P1)
+    np.testing.assert_array_equal(o_h, o1)

@@ -84,3 +84,20 @@ def test_scan_reports_a_too_small_max_seqlen(kdn):
         kdn.last_device_error()
     assert ei.value.code == kdn.KDN_ERR_INVALID_ARG
     kdn.last_device_error()   # the word was cleared
+
+
+def test_information_scaling_weakens_the_effective_write_strength(kdn):
+    """Kalman Delta Networks explainer (techwalker), information scaling: mu = d_k instead of
+    1 lowers the mean effective write strength k^T g, also with the inputs held fixed.
+    P^- is monotone in mu (every Moebius step is monotone in P) and k^T g = k^T P^- k /
+    (r + k^T P^- k) grows with P^-, so the drop holds token by token; both settings are
+    also checked against the oracle's traces on one chain."""
+    w = inputs.prefill_4x4096()
+    means = {}
+    for mu in (1.0, 128.0):
+        g, be, P = run_scan(kdn, w, mu=mu)
+        ref = oracle.diag_chains(w, [(0, 3)], mu=mu, trace=True)[(0, 3)]
+        assert max_rel_err(be[:4096, 3], ref["beta_eff"]) <= TOL[True]
+        means[mu] = be
+    assert np.all(means[128.0] <= means[1.0] * (1 + 1e-5) + 1e-7)
+    assert float(np.mean(means[128.0])) < float(np.mean(means[1.0]))
