@@ -15,6 +15,8 @@ diag_forward   -- Diagonal KDN (predict, Kalman gain, decayed delta write,
                   readout, mean-field uncertainty update with scaling mu).
 full_kf        -- the full-covariance Kalman filter on the same model (tiny sizes).
 delta_forward  -- the delta family with a given write strength beta.
+iso_forward    -- isotropic KDN (one uncertainty per head; trace-keeping predict,
+                  exact gain, precision-averaged update scaled by mu).
 mobius_matrix  -- the 2x2 matrix of one token's uncertainty map (predict then update),
                   for the associative-scan pins.
 
@@ -59,7 +61,8 @@ def _bind(path):
     lib.kdn_oracle_diag.argtypes = [i, _i64p, i, i, i] + [_dp] * 8 + [d] + [_dp] * 7 + [i]
     lib.kdn_oracle_fullkf.argtypes = [i, _i64p, i, i, i] + [_dp] * 8 + [_dp] * 4 + [i]
     lib.kdn_oracle_delta.argtypes = [i, _i64p, i, i, i] + [_dp] * 6 + [_dp] * 2 + [i]
-    for f in (lib.kdn_oracle_diag, lib.kdn_oracle_fullkf, lib.kdn_oracle_delta):
+    lib.kdn_oracle_iso.argtypes = lib.kdn_oracle_diag.argtypes
+    for f in (lib.kdn_oracle_diag, lib.kdn_oracle_fullkf, lib.kdn_oracle_delta, lib.kdn_oracle_iso):
         f.restype = ctypes.c_int
     return lib
 
@@ -141,6 +144,38 @@ def diag_forward(q, k, v, alpha, sigma, r, cu_seqlens=None, S0=None, P0=None, mu
     return out
 
 
+def iso_forward(q, k, v, alpha, sigma, r, cu_seqlens=None, S0=None, P0=None, mu: float = 1.0,
+                trace: bool = False, threads: Optional[int] = None):
+    """Isotropic KDN over tokens [ntok, H, d]; P0 and the returned P are [nseq, H].
+
+    Returns dict(o, S, P) and, with ``trace``, per-token p^- ("Pm") and p [ntok, H],
+    the gain g [ntok, H, dk] and k^T g ("beta_eff")."""
+    q, k, v, alpha, sigma, r = map(_f64, (q, k, v, alpha, sigma, r))
+    ntok, H, dk = k.shape
+    dv = v.shape[-1]
+    cu = _cu(cu_seqlens, ntok)
+    nseq = len(cu) - 1
+    S0, P0 = _f64(S0), _f64(P0)
+    o = np.zeros((ntok, H, dv))
+    S = np.zeros((nseq, H, dk, dv))
+    P = np.zeros((nseq, H))
+    tr = {}
+    if trace:
+        tr = dict(Pm=np.zeros((ntok, H)), P=np.zeros((ntok, H)), g=np.zeros((ntok, H, dk)),
+                  beta_eff=np.zeros((ntok, H)))
+    rc = _load().kdn_oracle_iso(nseq, cu.ctypes.data_as(_i64p), H, dk, dv,
+                                _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(sigma), _ptr(r),
+                                _ptr(S0), _ptr(P0), float(mu), _ptr(o), _ptr(S), _ptr(P),
+                                _ptr(tr.get("Pm")), _ptr(tr.get("P")), _ptr(tr.get("g")),
+                                _ptr(tr.get("beta_eff")), _threads(threads))
+    if rc:
+        raise RuntimeError(f"kdn_oracle_iso failed ({rc})")
+    out = dict(o=o, S=S, P=P)
+    if trace:
+        out.update({("trace_" + n): a for n, a in tr.items()})
+    return out
+
+
 def full_kf(q, k, v, alpha, sigma, r, cu_seqlens=None, S0=None, Sigma0=None, threads: Optional[int] = None):
     """Full-covariance Kalman filter; returns dict(o, S, Sigma [nseq,H,dk,dk], g)."""
     q, k, v, alpha, sigma, r = map(_f64, (q, k, v, alpha, sigma, r))
@@ -180,9 +215,11 @@ def delta_forward(q, k, v, alpha, beta, cu_seqlens=None, S0=None, threads: Optio
     return dict(o=o, S=S)
 
 
-def diag_chains(w, chains, mu=None, S0=None, P0=None, threads: Optional[int] = None, trace: bool = False):
-    """Diagonal KDN on selected (sequence, head) chains of a workload ``w`` (any object
-    with q, k, v, alpha, sigma, r as [ntok, H, d], cu_seqlens and mu).
+def diag_chains(w, chains, mu=None, S0=None, P0=None, threads: Optional[int] = None, trace: bool = False,
+                iso: bool = False):
+    """Diagonal KDN (isotropic with ``iso``) on selected (sequence, head) chains of a
+    workload ``w`` (any object with q, k, v, alpha, sigma, r as [ntok, H, d],
+    cu_seqlens and mu).
 
     The chains are packed as the sequences of a one-head problem and run in one call
     (one thread per chain).  Returns {(s, h): dict(o [len, dv], S [dk, dv], P [dk])}."""
@@ -196,8 +233,9 @@ def diag_chains(w, chains, mu=None, S0=None, P0=None, threads: Optional[int] = N
     cu2 = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
     S0s = None if S0 is None else np.stack([S0[s, h] for (s, h), _ in pieces])[:, None]
     P0s = None if P0 is None else np.stack([P0[s, h] for (s, h), _ in pieces])[:, None]
-    res = diag_forward(cat("q"), cat("k"), cat("v"), cat("alpha"), cat("sigma"), cat("r"),
-                       cu_seqlens=cu2, S0=S0s, P0=P0s, mu=mu, threads=threads, trace=trace)
+    fwd = iso_forward if iso else diag_forward
+    res = fwd(cat("q"), cat("k"), cat("v"), cat("alpha"), cat("sigma"), cat("r"),
+              cu_seqlens=cu2, S0=S0s, P0=P0s, mu=mu, threads=threads, trace=trace)
     out = {}
     for i, ((s, h), _) in enumerate(pieces):
         sl = slice(cu2[i], cu2[i + 1])
@@ -230,7 +268,7 @@ def mobius_matrix(alpha, sigma, k, r, mu: float = 1.0):
     return M
 
 
-def run_decode(S0, P0, steps, mu: float = 1.0, threads: Optional[int] = None):
+def run_decode(S0, P0, steps, mu: float = 1.0, threads: Optional[int] = None, iso: bool = False):
     """Decode over a list of per-step token dicts ([N,H,d] arrays) from states S0, P0.
 
     One decode step is one token of the recurrence with the state carried; the
@@ -244,7 +282,8 @@ def run_decode(S0, P0, steps, mu: float = 1.0, threads: Optional[int] = None):
     arrs = {nm: stack(nm) for nm in ("q", "k", "v", "alpha", "sigma", "r")}
     flat = {nm: a.reshape((N * n,) + a.shape[2:]) for nm, a in arrs.items()}
     cu = np.arange(N + 1, dtype=np.int64) * n
-    res = diag_forward(flat["q"], flat["k"], flat["v"], flat["alpha"], flat["sigma"], flat["r"],
-                       cu_seqlens=cu, S0=S0, P0=P0, mu=mu, threads=threads)
+    fwd = iso_forward if iso else diag_forward
+    res = fwd(flat["q"], flat["k"], flat["v"], flat["alpha"], flat["sigma"], flat["r"],
+              cu_seqlens=cu, S0=S0, P0=P0, mu=mu, threads=threads)
     o = res["o"].reshape((N, n) + res["o"].shape[1:]).transpose(1, 0, 2, 3)
     return dict(o=o, S=res["S"], P=res["P"])

@@ -35,7 +35,15 @@
  *    under S -> diag(alpha) S scales by alpha^2);
  *  - the mean-field projection keeps the diagonal of the posterior PRECISION:
  *    1/P = 1/P^- + mu * k^2 / r;
- *  - the readout o_t = S_t^T q_t is taken after the write, without scaling.
+ *  - the readout o_t = S_t^T q_t is taken after the write, without scaling;
+ *  - isotropic KDN (one uncertainty p per head; explainer "各向同性近似",
+ *    aifromscratch "Approximation 2: Isotropic KDN"): the predicted covariance
+ *    diag(alpha^2) p + diag(sigma) is brought back to a multiple of the identity
+ *    keeping its trace, p^- = mean(alpha^2) p + mean(sigma) (the pages require the
+ *    isotropic recursion to stay a Moebius map, which the trace keeps and the
+ *    precision average would not); the gain p^- k / (r + p^- |k|^2) is exact for an
+ *    isotropic prior; the posterior is projected like the diagonal one, by its
+ *    precision, averaged over the d_k directions: 1/p = 1/p^- + mu |k|^2 / (d_k r).
  *
  * Layout: tokens flattened as [ntok, H, d] (dense batch b,t -> b*T + t);
  * sequence s covers tokens [cu[s], cu[s+1]); states S [nseq, H, dk, dv],
@@ -84,11 +92,11 @@ static void readout(const double *S, int dk, int dv, const double *q, double *o)
 /* ---------------------------------------------------------------- work split */
 
 typedef struct {
-    int mode;                 /* 0 diagonal KDN, 1 full covariance, 2 constant beta */
+    int mode;                 /* 0 diagonal KDN, 1 full covariance, 2 constant beta, 3 isotropic KDN */
     int nseq, H, dk, dv;
     const int64_t *cu;
     const double *q, *k, *v, *alpha, *sigma, *r, *beta;
-    const double *S0, *P0;    /* P0: [nseq,H,dk] (diag) or [nseq,H,dk,dk] (full) */
+    const double *S0, *P0;    /* P0: [nseq,H,dk] (diag), [nseq,H,dk,dk] (full), [nseq,H] (isotropic) */
     double mu;
     double *o, *S_out, *P_out;
     double *Pm_trace, *P_trace, *g_trace, *beff_trace;
@@ -120,6 +128,10 @@ static void run_item(job_t *J, int item)
         if (!Sig || !Sm || !Sk) { J->status = -1; goto done; }
         if (J->P0) memcpy(Sig, J->P0 + sh * dk * dk, sizeof(double) * (size_t)dk * dk);
         else for (int i = 0; i < dk; ++i) for (int j = 0; j < dk; ++j) Sig[(size_t)i * dk + j] = (i == j);
+    } else if (J->mode == 3) {
+        P = (double *)malloc(sizeof(double));
+        if (!P) { J->status = -1; goto done; }
+        P[0] = J->P0 ? J->P0[sh] : 1.0;
     } else {
         P = (double *)malloc(sizeof(double) * (size_t)dk);
         if (!P) { J->status = -1; goto done; }
@@ -163,6 +175,15 @@ static void run_item(job_t *J, int item)
                     double m = 0.5 * (Sig[(size_t)i * dk + j] + Sig[(size_t)j * dk + i]);
                     Sig[(size_t)i * dk + j] = Sig[(size_t)j * dk + i] = m;
                 }
+        } else if (J->mode == 3) {
+            /* isotropic predict: the trace of diag(alpha^2) p + diag(sigma), per direction */
+            const double *sg = J->sigma + th * dk;
+            double a2 = 0.0, sm = 0.0, kk = 0.0;
+            for (int i = 0; i < dk; ++i) { a2 += al[i] * al[i]; sm += sg[i]; kk += k[i] * k[i]; }
+            Pm[0] = (a2 / dk) * P[0] + sm / dk;
+            /* exact gain for an isotropic prior: g = p^- k / (r + p^- |k|^2) */
+            const double den = r + Pm[0] * kk;
+            for (int i = 0; i < dk; ++i) g[i] = Pm[0] * k[i] / den;
         } else {
             /* delta family: the write key is beta * k */
             const double b = J->beta[th];
@@ -183,6 +204,13 @@ static void run_item(job_t *J, int item)
             /* mean-field update: diagonal of the posterior precision, increment scaled by mu */
             for (int i = 0; i < dk; ++i) P[i] = Pm[i] / (1.0 + J->mu * Pm[i] * k[i] * k[i] / r);
             if (J->P_trace) memcpy(J->P_trace + th * dk, P, sizeof(double) * (size_t)dk);
+        } else if (J->mode == 3) {
+            if (J->Pm_trace) J->Pm_trace[th] = Pm[0];
+            /* precision of the posterior averaged over the d_k directions, increment scaled by mu */
+            double kk = 0.0;
+            for (int i = 0; i < dk; ++i) kk += k[i] * k[i];
+            P[0] = Pm[0] / (1.0 + J->mu * Pm[0] * kk / (dk * r));
+            if (J->P_trace) J->P_trace[th] = P[0];
         }
     }
 
@@ -190,6 +218,7 @@ static void run_item(job_t *J, int item)
     if (J->P_out) {
         if (J->mode == 1) memcpy(J->P_out + sh * dk * dk, Sig, sizeof(double) * (size_t)dk * dk);
         else if (J->mode == 0) memcpy(J->P_out + sh * dk, P, sizeof(double) * (size_t)dk);
+        else if (J->mode == 3) J->P_out[sh] = P[0];
     }
 done:
     free(S); free(u); free(g); free(Pm); free(P); free(Sig); free(Sm); free(Sk);
@@ -293,5 +322,31 @@ int kdn_oracle_delta(int nseq, const int64_t *cu, int H, int dk, int dv,
     J.mode = 2; J.nseq = nseq; J.H = H; J.dk = dk; J.dv = dv; J.cu = cu;
     J.q = q; J.k = k; J.v = v; J.alpha = alpha; J.beta = beta;
     J.S0 = S0; J.o = o; J.S_out = S_out;
+    return run_job(&J, nthreads);
+}
+
+/* Isotropic KDN, per token (one uncertainty p per head):
+ *   1. p^- = mean_i(alpha_i^2) p + mean_i(sigma_i)
+ *   2. g   = p^- k / (r + p^- |k|^2)
+ *   3. W = diag(alpha) S ; u = v - W^T k ; S = W + g u^T
+ *   4. o   = S^T q
+ *   5. p   = p^- / (1 + mu p^- |k|^2 / (d_k r))
+ * S0 NULL -> zeros, P0 [nseq,H] NULL -> ones.  Traces per token: p^- and p [ntok,H],
+ * g [ntok,H,dk], k^T g [ntok,H]. */
+int kdn_oracle_iso(int nseq, const int64_t *cu, int H, int dk, int dv,
+                   const double *q, const double *k, const double *v,
+                   const double *alpha, const double *sigma, const double *r,
+                   const double *S0, const double *P0, double mu,
+                   double *o, double *S_out, double *P_out,
+                   double *Pm_trace, double *P_trace, double *g_trace, double *beff_trace,
+                   int nthreads)
+{
+    if (check_cu(nseq, cu) || H <= 0 || dk <= 0 || dv <= 0 || !q || !k || !v || !alpha || !sigma || !r || !o)
+        return -2;
+    job_t J = {0};
+    J.mode = 3; J.nseq = nseq; J.H = H; J.dk = dk; J.dv = dv; J.cu = cu;
+    J.q = q; J.k = k; J.v = v; J.alpha = alpha; J.sigma = sigma; J.r = r;
+    J.S0 = S0; J.P0 = P0; J.mu = mu; J.o = o; J.S_out = S_out; J.P_out = P_out;
+    J.Pm_trace = Pm_trace; J.P_trace = P_trace; J.g_trace = g_trace; J.beff_trace = beff_trace;
     return run_job(&J, nthreads);
 }

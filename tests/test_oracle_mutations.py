@@ -34,6 +34,14 @@ MUTATIONS = {
     "initial_uncertainty_ignored": ("P[i] = J->P0 ? J->P0[sh * dk + i] : 1.0;", "P[i] = 1.0;"),
     "head_index_dropped": ("const size_t th = (size_t)t * H + h;", "const size_t th = (size_t)t * H;"),
     "noise_indexed_by_token_only": ("const double r = J->r ? J->r[th] : 0.0;", "const double r = J->r ? J->r[t] : 0.0;"),
+    "iso_predict_mean_of_alpha_not_alpha_squared": ("a2 += al[i] * al[i];", "a2 += al[i];"),
+    "iso_predict_drops_process_noise": ("Pm[0] = (a2 / dk) * P[0] + sm / dk;", "Pm[0] = (a2 / dk) * P[0];"),
+    "iso_gain_uses_posterior": ("const double den = r + Pm[0] * kk;", "const double den = r + P[0] * kk;"),
+    "iso_update_not_averaged_over_directions": ("P[0] = Pm[0] / (1.0 + J->mu * Pm[0] * kk / (dk * r));",
+                                                "P[0] = Pm[0] / (1.0 + J->mu * Pm[0] * kk / r);"),
+    "iso_update_ignores_mu": ("P[0] = Pm[0] / (1.0 + J->mu * Pm[0] * kk / (dk * r));",
+                              "P[0] = Pm[0] / (1.0 + Pm[0] * kk / (dk * r));"),
+    "iso_initial_uncertainty_ignored": ("P[0] = J->P0 ? J->P0[sh] : 1.0;", "P[0] = 1.0;"),
 }
 
 

@@ -439,3 +439,150 @@ def test_decode_runner_equals_one_sequence():
             S, P = one["S"], one["P"]
         np.testing.assert_allclose(dec["S"][s], S[0], rtol=1e-13, atol=1e-14)
         np.testing.assert_allclose(dec["P"][s], P[0], rtol=1e-13)
+
+
+# ------------------------------------------------------------------ isotropic KDN
+def uniform_channels(rng, T, H, dk):
+    """Decay and process noise equal across the key channels of a token (the predict
+    then keeps an isotropic covariance isotropic)."""
+    a = 1.0 / (1.0 + np.exp(-rng.normal(2.0, 1.0, (T, H, 1))))
+    s = np.logaddexp(0, rng.normal(-3.0, 1.0, (T, H, 1)))
+    return np.broadcast_to(a, (T, H, dk)).copy(), np.broadcast_to(s, (T, H, dk)).copy()
+
+
+def test_iso_one_step_gain_is_exact_and_update_is_the_kl_projection():
+    """Explainer "各向同性近似" / aifromscratch "Approximation 2": one uncertainty per head.
+    From an isotropic prior the Kalman gain is exact, so one step gives the full
+    filter's mean and readout; the scalar posterior is the reverse-KL (mean-field)
+    projection of the full posterior onto multiples of the identity, found here by a
+    library minimiser of KL(N(0, p I) || N(0, Sigma)) over p."""
+    from scipy.optimize import minimize_scalar
+    rng = np.random.default_rng(30)
+    H, dk, dv = 3, 6, 4
+    q, k, v, _, _, r = rand_problem(rng, 1, H, dk, dv, unit=False)
+    alpha, sigma = uniform_channels(rng, 1, H, dk)
+    p0 = rng.uniform(0.3, 2.0, (1, H))
+    S0 = rng.standard_normal((1, H, dk, dv))
+    iso = oracle.iso_forward(q, k, v, alpha, sigma, r, S0=S0, P0=p0, mu=1.0)
+    f = oracle.full_kf(q, k, v, alpha, sigma, r, S0=S0, Sigma0=(p0[0, :, None, None] * np.eye(dk))[None])
+    np.testing.assert_allclose(iso["S"], f["S"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(iso["o"], f["o"], rtol=1e-12, atol=1e-12)
+    for h in range(H):
+        Sig = f["Sigma"][0, h]
+        prec_tr = np.trace(np.linalg.inv(Sig))
+        logdet = np.linalg.slogdet(Sig)[1]
+
+        def kl(lp):
+            p = np.exp(lp)
+            return 0.5 * (p * prec_tr - dk + logdet - dk * lp)
+        best = minimize_scalar(kl, bounds=(-12.0, 6.0), method="bounded", options={"xatol": 1e-12})
+        np.testing.assert_allclose(iso["P"][0, h], np.exp(best.x), rtol=1e-7)
+
+
+def test_iso_predict_keeps_the_trace_of_the_diagonal_predict():
+    """Reading of the isotropic predict: with no information in the token (k = 0) the
+    step is the predict alone, and p equals the mean over channels of the diagonal
+    filter's predicted variances alpha_i^2 p + sigma_i (non-uniform alpha, sigma)."""
+    rng = np.random.default_rng(31)
+    H, dk, dv = 2, 8, 3
+    q, k, v, alpha, sigma, r = rand_problem(rng, 1, H, dk, dv)
+    k[:] = 0.0
+    p0 = rng.uniform(0.3, 2.0, (1, H))
+    iso = oracle.iso_forward(q, k, v, alpha, sigma, r, P0=p0, mu=1.0)
+    dg = oracle.diag_forward(q, k, v, alpha, sigma, r, P0=np.repeat(p0[..., None], dk, axis=-1), mu=1.0)
+    np.testing.assert_allclose(iso["P"], dg["P"].mean(axis=-1), rtol=1e-14)
+
+
+def test_iso_equals_diagonal_without_information_scaling_on_uniform_channels():
+    """mu = 0 and decay / noise uniform across channels: a diagonal uncertainty that
+    starts isotropic stays isotropic, so the two approximations coincide for every
+    token (and both are gated DeltaNet with the scalar Kalman write strength)."""
+    rng = np.random.default_rng(32)
+    T, H, dk, dv = 40, 2, 8, 5
+    q, k, v, _, _, r = rand_problem(rng, T, H, dk, dv)
+    alpha, sigma = uniform_channels(rng, T, H, dk)
+    p0 = rng.uniform(0.3, 2.0, (1, H))
+    iso = oracle.iso_forward(q, k, v, alpha, sigma, r, P0=p0, mu=0.0, trace=True)
+    dg = oracle.diag_forward(q, k, v, alpha, sigma, r, P0=np.repeat(p0[..., None], dk, axis=-1), mu=0.0,
+                             trace=True)
+    np.testing.assert_allclose(iso["o"], dg["o"], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(iso["S"], dg["S"], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(iso["trace_g"], dg["trace_g"], rtol=1e-11, atol=1e-14)
+    np.testing.assert_allclose(iso["trace_Pm"], dg["trace_Pm"][..., 0], rtol=1e-12)
+
+
+@pytest.mark.parametrize("mu", [1.0, 8.0])
+def test_iso_repeated_confirmation_closed_form(mu):
+    """No decay, no process noise, constant r, unit keys in any directions: the head's
+    precision grows by mu / (d_k r) per token, 1/p_n = 1/p_0 + n mu / (d_k r)."""
+    rng = np.random.default_rng(33)
+    n, dk, dv, r0 = 30, 8, 2, 0.45
+    k = unit_rows(rng.standard_normal((n, 1, dk)))
+    p0 = np.array([[1.7]])
+    res = oracle.iso_forward(k, k, rng.standard_normal((n, 1, dv)), np.ones((n, 1, dk)), np.zeros((n, 1, dk)),
+                             np.full((n, 1), r0), P0=p0, mu=mu, trace=True)
+    t = np.arange(1, n + 1)
+    np.testing.assert_allclose(1.0 / res["trace_P"][:, 0], 1.0 / 1.7 + t * mu / (dk * r0), rtol=1e-12)
+
+
+def test_iso_fixed_point_closed_form():
+    """Constant tokens with channel-varying decay and noise: the predicted uncertainty
+    converges to the positive root of c x^2 + (1 - a - c s) x - s = 0 with
+    a = mean(alpha^2), s = mean(sigma), c = mu |k|^2 / (d_k r)."""
+    dk, T = 4, 600
+    alpha = np.array([0.9, 0.99, 0.5, 0.8])
+    sg = np.array([0.05, 0.01, 0.2, 0.0])
+    kv = np.array([0.6, 0.3, 0.74, -0.2])
+    r0, mu = 0.8, 2.0
+    k = np.broadcast_to(kv, (T, 1, dk)).copy()
+    res = oracle.iso_forward(k, k, np.zeros((T, 1, 1)), np.broadcast_to(alpha, (T, 1, dk)),
+                             np.broadcast_to(sg, (T, 1, dk)), np.full((T, 1), r0), mu=mu, trace=True)
+    a, s, c = np.mean(alpha ** 2), np.mean(sg), mu * np.sum(kv ** 2) / (dk * r0)
+    b = 1 - a - c * s
+    x = (-b + np.sqrt(b * b + 4 * c * s)) / (2 * c)
+    np.testing.assert_allclose(res["trace_Pm"][-1, 0], x, rtol=1e-10)
+
+
+def test_iso_is_kda_with_a_derived_write_strength():
+    """Explainer "各向同性近似": the isotropic KDN keeps the delta-rule form of KDA and only
+    derives the scalar write strength from the uncertainty.  The gain is parallel to
+    the key, and the KDA recurrence (delta family, per-channel decay) driven by
+    beta_t = k^T g / |k|^2 reproduces the outputs and the memory."""
+    w = inputs.tiny_fp32()
+    iso = oracle.iso_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens, mu=4.0, trace=True)
+    k = w.k.astype(np.float64)
+    kk = np.sum(k * k, axis=-1)
+    beta = iso["trace_beta_eff"] / kk
+    np.testing.assert_allclose(iso["trace_g"], beta[..., None] * k, rtol=1e-12, atol=1e-15)
+    kda = oracle.delta_forward(w.q, w.k, w.v, w.alpha, beta, cu_seqlens=w.cu_seqlens)
+    np.testing.assert_allclose(iso["o"], kda["o"], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(iso["S"], kda["S"], rtol=1e-12, atol=1e-13)
+    assert np.all(iso["trace_beta_eff"] >= 0) and np.all(iso["trace_beta_eff"] < 1)
+    assert np.all(iso["trace_P"] > 0) and np.all(iso["trace_P"] <= iso["trace_Pm"])
+
+
+def test_iso_mobius_tree_scan_and_split_with_carried_state():
+    """The scalar recursion is a Moebius map per token, [[a, s], [c a, c s + 1]]; a
+    log-depth prefix product reproduces the serial run, and carrying (S, p) across a
+    split reproduces one call."""
+    rng = np.random.default_rng(35)
+    T, dk, mu = 257, 16, 5.0
+    q, k, v, alpha, sigma, r = rand_problem(rng, T, 1, dk, 3)
+    res = oracle.iso_forward(q, k, v, alpha, sigma, r, P0=np.array([[0.6]]), mu=mu, trace=True)
+    a = np.mean(alpha[:, 0] ** 2, axis=-1)
+    s = np.mean(sigma[:, 0], axis=-1)
+    c = mu * np.sum(k[:, 0] ** 2, axis=-1) / (dk * r[:, 0])
+    M = np.stack([np.stack([a, s], -1), np.stack([c * a, c * s + 1], -1)], -2)   # [T, 2, 2]
+    pref, step = M.copy(), 1
+    while step < T:
+        new = pref.copy()
+        new[step:] = pref[step:] @ pref[:-step]
+        pref = new / np.abs(new).max(axis=(-2, -1), keepdims=True)
+        step *= 2
+    P = (pref[:, 0, 0] * 0.6 + pref[:, 0, 1]) / (pref[:, 1, 0] * 0.6 + pref[:, 1, 1])
+    np.testing.assert_allclose(P, res["trace_P"][:, 0], rtol=1e-11)
+    cut = 100
+    x = oracle.iso_forward(q[:cut], k[:cut], v[:cut], alpha[:cut], sigma[:cut], r[:cut], P0=np.array([[0.6]]), mu=mu)
+    y = oracle.iso_forward(q[cut:], k[cut:], v[cut:], alpha[cut:], sigma[cut:], r[cut:], S0=x["S"], P0=x["P"], mu=mu)
+    np.testing.assert_allclose(np.concatenate([x["o"], y["o"]]), res["o"], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(y["P"], res["P"], rtol=1e-12)
