@@ -16,6 +16,15 @@
  * Products and divisions of vectors are elementwise.  alpha in [0,1], sigma >= 0 and
  * r > 0 are variances; mu > 0 scales the precision increment (1 = plain mean-field).
  *
+ * Isotropic variant (explainer "各向同性近似"; aifromscratch "Approximation 2: Isotropic
+ * KDN"): one uncertainty p per head instead of P (d_k), with the same memory update and
+ *
+ *     p^-_t = mean_i(alpha_{t,i}^2) p_{t-1} + mean_i(sigma_{t,i})  (trace-keeping predict)
+ *     g_t   = p^-_t k_t / (r_t + p^-_t |k_t|^2)                   (exact for an isotropic prior)
+ *     p_t   = p^-_t / (1 + mu p^-_t |k_t|^2 / (d_k r_t))          (precision averaged over d_k)
+ *
+ * Its uncertainty states are [N, H] where the diagonal ones are [N, H, d_k].
+ *
  * Conventions shared by every entry point
  *  - Memory: the caller owns every buffer; the library never allocates.  Pointers
  *    marked "device" must be device memory of the current CUDA device; buffers must
@@ -57,6 +66,9 @@ typedef enum {
 
 typedef enum { KDN_DTYPE_F32 = 0, KDN_DTYPE_BF16 = 1 } kdn_dtype_t;
 
+/* Which uncertainty the recurrence tracks (the `variant` field of kdn_problem_t). */
+typedef enum { KDN_VARIANT_DIAGONAL = 0, KDN_VARIANT_ISOTROPIC = 1 } kdn_variant_t;
+
 /* Execution paths of kdn_forward_chunkwise (the `chunk` field):
  *  0        token-serial fused recurrence (any dtype; exact fp32 arithmetic);
  *  16/32/64 chunkwise: for bf16 inputs and chunk 64 the tcgen05 tensor-core kernel,
@@ -71,6 +83,7 @@ typedef struct {
     int max_seqlen;                 /* varlen: upper bound on every sequence length (0 = unknown, taken as T);
                                        sizes the gain scan's work list.  A sequence longer than it makes
                                        kdn_gain_scan record KDN_ERR_INVALID_ARG in the device error word. */
+    int variant;                    /* kdn_variant_t; 0 (zero-initialised struct) = diagonal */
 } kdn_problem_t;
 
 /* Bytes of device workspace needed for `p`: the larger of what kdn_gain_scan() and
@@ -83,9 +96,9 @@ kdn_status_t kdn_workspace_size(const kdn_problem_t *p, size_t *bytes);
  *  q, k, alpha, sigma : device [B, T, H, d_k]        (in_dtype)
  *  v                  : device [B, T, H, d_v]        (in_dtype)
  *  r                  : device [B, T, H]             (in_dtype)
- *  S0, P0             : device fp32 [N, H, d_k, d_v], [N, H, d_k]; NULL -> S0 = 0, P0 = 1
+ *  S0, P0             : device fp32 [N, H, d_k, d_v], [N, H, d_k] ([N, H] isotropic); NULL -> S0 = 0, P0 = 1
  *  o                  : device [B, T, H, d_v]        (in_dtype), written for every token
- *  S_out, P_out       : device fp32, final states per sequence; either may be NULL.
+ *  S_out, P_out       : device fp32, final states per sequence (shapes as S0, P0); either may be NULL.
  *                       They may not alias S0 / P0.
  *  workspace          : device, >= kdn_workspace_size() bytes, 256-byte aligned; its
  *                       contents on entry do not matter.
@@ -123,6 +136,13 @@ kdn_status_t kdn_decode_tokens(int N, int n_tokens, int H, int d_k, int d_v, kdn
                                const void *alpha, const void *sigma, const void *r,
                                float *S, float *P, void *o, void *stream);
 
+/* kdn_decode_tokens() for the isotropic variant: P is device fp32 [N, H] (one
+ * uncertainty per head), updated in place; everything else as kdn_decode_tokens(). */
+kdn_status_t kdn_decode_tokens_iso(int N, int n_tokens, int H, int d_k, int d_v, kdn_dtype_t in_dtype, float mu,
+                                   const void *q, const void *k, const void *v,
+                                   const void *alpha, const void *sigma, const void *r,
+                                   float *S, float *P, void *o, void *stream);
+
 /* The uncertainty / gain scan on its own (explainer, closing paragraph of "各向同性近似":
  * the uncertainty recursion is a Moebius map whose 2x2 matrices compose, so it runs
  * as an associative scan).  Independent of the memory S.
@@ -136,7 +156,7 @@ kdn_status_t kdn_decode_tokens(int N, int n_tokens, int H, int d_k, int d_v, kdn
  * Single pass: every 64-token chunk composes its tokens' maps, publishes the composite,
  * and takes its starting uncertainty from its predecessors by decoupled look-back
  * (bounded waits; a wait that gives up records KDN_ERR_TIMEOUT).  Concurrent calls
- * must use distinct workspaces. */
+ * must use distinct workspaces.  Diagonal variant only (isotropic: KDN_ERR_UNSUPPORTED). */
 kdn_status_t kdn_gain_scan(const kdn_problem_t *p,
                            const void *k, const void *alpha, const void *sigma, const void *r,
                            const float *P0, float *g, float *beta_eff, float *P_out,

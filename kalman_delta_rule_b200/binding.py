@@ -32,7 +32,7 @@ class kdn_problem_t(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("d_k", ctypes.c_int),
                 ("d_v", ctypes.c_int), ("cu_seqlens", ctypes.c_void_p), ("num_seqs", ctypes.c_int),
                 ("in_dtype", ctypes.c_int), ("mu", ctypes.c_float), ("chunk", ctypes.c_int),
-                ("max_seqlen", ctypes.c_int)]
+                ("max_seqlen", ctypes.c_int), ("variant", ctypes.c_int)]
 
 
 _lib = None
@@ -45,6 +45,7 @@ _SIGS = {
     "kdn_forward_chunkwise": (_i, [_PP] + [_vp] * 6 + [_vp] * 2 + [_vp] * 3 + [_vp, _sz, _vp]),
     "kdn_decode_step": (_i, [_i, _i, _i, _i, _i, _f] + [_vp] * 6 + [_vp] * 3 + [_vp]),
     "kdn_decode_tokens": (_i, [_i, _i, _i, _i, _i, _i, _f] + [_vp] * 6 + [_vp] * 3 + [_vp]),
+    "kdn_decode_tokens_iso": (_i, [_i, _i, _i, _i, _i, _i, _f] + [_vp] * 6 + [_vp] * 3 + [_vp]),
     "kdn_gain_scan": (_i, [_PP] + [_vp] * 4 + [_vp] + [_vp] * 3 + [_vp, _sz, _vp]),
     "kdn_last_device_error": (_i, [_vp]),
     "kdn_status_string": (ctypes.c_char_p, [_i]),
@@ -90,6 +91,11 @@ def kdn_decode_step(N, H, d_k, d_v, in_dtype, mu, q, k, v, alpha, sigma, r, S, P
 
 def kdn_decode_tokens(N, n_tokens, H, d_k, d_v, in_dtype, mu, q, k, v, alpha, sigma, r, S, P, o, stream):
     return load().kdn_decode_tokens(N, n_tokens, H, d_k, d_v, in_dtype, mu, q, k, v, alpha, sigma, r, S, P, o, stream)
+
+
+def kdn_decode_tokens_iso(N, n_tokens, H, d_k, d_v, in_dtype, mu, q, k, v, alpha, sigma, r, S, P, o, stream):
+    return load().kdn_decode_tokens_iso(N, n_tokens, H, d_k, d_v, in_dtype, mu, q, k, v, alpha, sigma, r, S, P, o,
+                                        stream)
 
 
 def kdn_gain_scan(problem, k, alpha, sigma, r, P0, g, beta_eff, P_out, workspace, workspace_bytes, stream):
@@ -155,7 +161,11 @@ def _check(st: int, where: str):
         raise KdnError(st, where)
 
 
-def make_problem(q, v, H=None, cu_seqlens=None, mu: float = 1.0, chunk: int = 64, max_seqlen: int = 0) -> kdn_problem_t:
+VARIANTS = {"diagonal": 0, "isotropic": 1}
+
+
+def make_problem(q, v, H=None, cu_seqlens=None, mu: float = 1.0, chunk: int = 64, max_seqlen: int = 0,
+                 variant: str = "diagonal") -> kdn_problem_t:
     B, T, H_, dk = q.shape
     p = kdn_problem_t()
     p.B, p.T, p.H, p.d_k, p.d_v = B, T, H_, dk, v.shape[-1]
@@ -165,16 +175,19 @@ def make_problem(q, v, H=None, cu_seqlens=None, mu: float = 1.0, chunk: int = 64
     p.mu = float(mu)
     p.chunk = int(chunk)
     p.max_seqlen = int(max_seqlen)
+    p.variant = VARIANTS[variant]
     return p
 
 
 def forward(q, k, v, alpha, sigma, r, cu_seqlens=None, S0=None, P0=None, mu: float = 1.0, chunk: int = 64,
-            o=None, S_out=None, P_out=None, workspace=None, want_state: bool = True, stream=None):
+            o=None, S_out=None, P_out=None, workspace=None, want_state: bool = True, stream=None,
+            variant: str = "diagonal"):
     """Run kdn_forward_chunkwise on torch tensors ([B,T,H,d]; varlen: B = 1 with int32 cu_seqlens).
 
-    Returns (o, S_out, P_out).  Outputs and workspace are allocated when not given."""
+    Returns (o, S_out, P_out); P is [N,H,dk] (diagonal) or [N,H] (isotropic).  Outputs and
+    workspace are allocated when not given."""
     torch = _torch()
-    p = make_problem(q, v, cu_seqlens=cu_seqlens, mu=mu, chunk=chunk)
+    p = make_problem(q, v, cu_seqlens=cu_seqlens, mu=mu, chunk=chunk, variant=variant)
     N = p.num_seqs
     dev = q.device
     if o is None:
@@ -182,7 +195,7 @@ def forward(q, k, v, alpha, sigma, r, cu_seqlens=None, S0=None, P0=None, mu: flo
     if want_state and S_out is None:
         S_out = torch.empty((N, p.H, p.d_k, p.d_v), dtype=torch.float32, device=dev)
     if want_state and P_out is None:
-        P_out = torch.empty((N, p.H, p.d_k), dtype=torch.float32, device=dev)
+        P_out = torch.empty((N, p.H) + ((p.d_k,) if p.variant == 0 else ()), dtype=torch.float32, device=dev)
     need = kdn_workspace_size(p)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
@@ -193,9 +206,14 @@ def forward(q, k, v, alpha, sigma, r, cu_seqlens=None, S0=None, P0=None, mu: flo
     return o, S_out, P_out
 
 
-def decode_step(q, k, v, alpha, sigma, r, S, P, mu: float = 1.0, o=None, stream=None):
-    """One decode step on [N,H,d] token tensors; S [N,H,dk,dv] and P [N,H,dk] updated in place."""
+def decode_step(q, k, v, alpha, sigma, r, S, P, mu: float = 1.0, o=None, stream=None, variant: str = "diagonal"):
+    """One decode step on [N,H,d] token tensors; S [N,H,dk,dv] and P [N,H,dk] ([N,H] isotropic)
+    updated in place."""
     torch = _torch()
+    if VARIANTS[variant] == 1:
+        o4 = None if o is None else o.unsqueeze(1)
+        return decode_tokens(*(x.unsqueeze(1) for x in (q, k, v, alpha, sigma, r)), S, P, mu=mu, o=o4,
+                             stream=stream, variant=variant).squeeze(1)
     N, H, dk = q.shape
     dv = v.shape[-1]
     if o is None:
@@ -206,14 +224,17 @@ def decode_step(q, k, v, alpha, sigma, r, S, P, mu: float = 1.0, o=None, stream=
     return o
 
 
-def decode_tokens(q, k, v, alpha, sigma, r, S, P, mu: float = 1.0, o=None, stream=None):
-    """n tokens per sequence in one launch on [N, n, H, d] token tensors; S, P updated in place."""
+def decode_tokens(q, k, v, alpha, sigma, r, S, P, mu: float = 1.0, o=None, stream=None,
+                  variant: str = "diagonal"):
+    """n tokens per sequence in one launch on [N, n, H, d] token tensors; S, P updated in place
+    (P [N,H,dk] diagonal, [N,H] isotropic)."""
     torch = _torch()
     N, n, H, dk = q.shape
     dv = v.shape[-1]
     if o is None:
         o = torch.empty((N, n, H, dv), dtype=q.dtype, device=q.device)
-    st = kdn_decode_tokens(N, n, H, dk, dv, _dtype_code(q), float(mu), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+    fn = kdn_decode_tokens_iso if VARIANTS[variant] == 1 else kdn_decode_tokens
+    st = fn(N, n, H, dk, dv, _dtype_code(q), float(mu), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
                            _ptr(sigma), _ptr(r), _ptr(S), _ptr(P), _ptr(o), _stream_handle(stream))
     _check(st, "kdn_decode_tokens")
     return o
@@ -241,9 +262,10 @@ def gain_scan(k, alpha, sigma, r, cu_seqlens=None, P0=None, mu: float = 1.0, chu
 PATH_NAMES = {0: "recurrent", 1: "chunk_fp32", 2: "chunk_tcgen05"}
 
 
-def execution_path(q, v, cu_seqlens=None, mu: float = 1.0, chunk: int = 64) -> str:
+def execution_path(q, v, cu_seqlens=None, mu: float = 1.0, chunk: int = 64, variant: str = "diagonal") -> str:
     """Name of the kernel path kdn_forward_chunkwise takes for these tensors."""
-    return PATH_NAMES.get(kdn_execution_path(make_problem(q, v, cu_seqlens=cu_seqlens, mu=mu, chunk=chunk)), "invalid")
+    p = make_problem(q, v, cu_seqlens=cu_seqlens, mu=mu, chunk=chunk, variant=variant)
+    return PATH_NAMES.get(kdn_execution_path(p), "invalid")
 
 
 def last_device_error(stream=None):

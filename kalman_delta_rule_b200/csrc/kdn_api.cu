@@ -42,6 +42,7 @@ kdn_status_t check_problem(const kdn_problem_t *p, Resolved *out) {
     if (p->B < 0 || p->T < 0 || p->H <= 0) return KDN_ERR_INVALID_ARG;
     if (!(p->mu > 0.f) || !isfinite(p->mu)) return KDN_ERR_INVALID_ARG;
     if (p->in_dtype != KDN_DTYPE_F32 && p->in_dtype != KDN_DTYPE_BF16) return KDN_ERR_INVALID_ARG;
+    if (p->variant != KDN_VARIANT_DIAGONAL && p->variant != KDN_VARIANT_ISOTROPIC) return KDN_ERR_INVALID_ARG;
     if (!dk_ok(p->d_k) || !dv_ok(p->d_v)) return KDN_ERR_UNSUPPORTED;
     if (p->chunk != 0 && p->chunk != 16 && p->chunk != 32 && p->chunk != 64) return KDN_ERR_UNSUPPORTED;
     if (p->cu_seqlens) {
@@ -109,7 +110,7 @@ kdn_status_t kdn_forward_chunkwise(const kdn_problem_t *p, const void *q, const 
     a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.sigma = sigma; a.r = r; a.o = o;
     a.S0 = S0; a.P0 = P0; a.S_out = S_out; a.P_out = P_out;
     a.cu = p->cu_seqlens; a.T = p->T; a.nseq = rv.nseq; a.H = p->H; a.dk = p->d_k; a.dv = p->d_v;
-    a.mu = p->mu; a.err = err_word();
+    a.mu = p->mu; a.iso = p->variant == KDN_VARIANT_ISOTROPIC; a.err = err_word();
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
 
     if (p->chunk == 0) {
@@ -124,9 +125,9 @@ kdn_status_t kdn_forward_chunkwise(const kdn_problem_t *p, const void *q, const 
     return cuda_status(kdn::launch_chunk_simt(a, rv.bf16, p->chunk, cs));
 }
 
-kdn_status_t kdn_decode_tokens(int N, int n_tokens, int H, int d_k, int d_v, kdn_dtype_t in_dtype, float mu,
-                               const void *q, const void *k, const void *v, const void *alpha, const void *sigma,
-                               const void *r, float *S, float *P, void *o, void *stream) {
+static kdn_status_t decode_impl(int N, int n_tokens, int H, int d_k, int d_v, kdn_dtype_t in_dtype, float mu,
+                                const void *q, const void *k, const void *v, const void *alpha, const void *sigma,
+                                const void *r, float *S, float *P, void *o, void *stream, bool iso) {
     if (N < 0 || n_tokens < 0 || H <= 0 || !(mu > 0.f) || !isfinite(mu)) return KDN_ERR_INVALID_ARG;
     if (in_dtype != KDN_DTYPE_F32 && in_dtype != KDN_DTYPE_BF16) return KDN_ERR_INVALID_ARG;
     if (!dk_ok(d_k) || !dv_ok(d_v)) return KDN_ERR_UNSUPPORTED;
@@ -139,8 +140,21 @@ kdn_status_t kdn_decode_tokens(int N, int n_tokens, int H, int d_k, int d_v, kdn
     a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.sigma = sigma; a.r = r; a.o = o;
     a.S0 = S; a.P0 = P; a.S_out = S; a.P_out = P;
     a.cu = nullptr; a.T = n_tokens; a.nseq = N; a.H = H; a.dk = d_k; a.dv = d_v; a.mu = mu; a.err = err_word();
+    a.iso = iso;
     // one tile per head: the in-place state and uncertainty are read and written by one CTA
     return cuda_status(kdn::launch_recurrent(a, in_dtype == KDN_DTYPE_BF16, d_v, static_cast<cudaStream_t>(stream)));
+}
+
+kdn_status_t kdn_decode_tokens(int N, int n_tokens, int H, int d_k, int d_v, kdn_dtype_t in_dtype, float mu,
+                               const void *q, const void *k, const void *v, const void *alpha, const void *sigma,
+                               const void *r, float *S, float *P, void *o, void *stream) {
+    return decode_impl(N, n_tokens, H, d_k, d_v, in_dtype, mu, q, k, v, alpha, sigma, r, S, P, o, stream, false);
+}
+
+kdn_status_t kdn_decode_tokens_iso(int N, int n_tokens, int H, int d_k, int d_v, kdn_dtype_t in_dtype, float mu,
+                                   const void *q, const void *k, const void *v, const void *alpha, const void *sigma,
+                                   const void *r, float *S, float *P, void *o, void *stream) {
+    return decode_impl(N, n_tokens, H, d_k, d_v, in_dtype, mu, q, k, v, alpha, sigma, r, S, P, o, stream, true);
 }
 
 kdn_status_t kdn_decode_step(int N, int H, int d_k, int d_v, kdn_dtype_t in_dtype, float mu, const void *q,
@@ -154,6 +168,7 @@ static kdn_status_t scan_args(const kdn_problem_t *p, const void *k, const void 
                               kdn::ScanArgs *a, Resolved *rv, bool *empty) {
     kdn_status_t st = check_problem(p, rv);
     if (st != KDN_OK) return st;
+    if (p->variant != KDN_VARIANT_DIAGONAL) return KDN_ERR_UNSUPPORTED;
     *empty = rv->nseq == 0 || rv->ntok == 0;
     if (*empty) return KDN_OK;
     if (!k || !alpha || !sigma || !r) return KDN_ERR_INVALID_ARG;

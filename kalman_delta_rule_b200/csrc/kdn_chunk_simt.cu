@@ -16,6 +16,10 @@
 // (one thread per key channel), with the chunk's per-token gain denominators reduced
 // across channels.  This kernel is the fp32-exact path; the bf16 throughput path is
 // the tensor-core kernel.
+//
+// Isotropic KDN (explainer "各向同性近似"): the head's single uncertainty runs first,
+// from per-token channel sums (thread = token), p^- = mean(alpha^2) p + mean(sigma),
+// p = p^- / (1 + mu p^- |k|^2 / (d_k r)); the gain numerators are then p^-_t k_t.
 #include "kdn_common.cuh"
 #include "kdn_launch.h"
 
@@ -77,14 +81,44 @@ __global__ void __launch_bounds__(NT, 1) chunk_simt_kernel(TokenArgs a, int C)
         const int i = e / DVT, j = e % DVT;
         Ss[e] = a.S0 ? a.S0[sbase + (size_t)i * dv + j] : 0.f;
     }
-    float P = 1.f;
-    if (tid < DK && a.P0) P = a.P0[(size_t)sh * DK + tid];
+    float P = 1.f;   // diagonal: channel tid; isotropic: the head's (thread 0 carries it)
+    if (a.iso) {
+        if (a.P0) P = a.P0[sh];
+    } else if (tid < DK && a.P0) {
+        P = a.P0[(size_t)sh * DK + tid];
+    }
     __syncthreads();
 
     for (int c0 = t0; c0 < t1; c0 += C) {
         const int L = min(C, t1 - c0);
         if (tid < L) Rs[tid] = ldf(r + (size_t)(c0 + tid) * H + h);
         __syncthreads();
+        if (a.iso) {
+            // channel sums of alpha^2, sigma, k^2 per token (A's rows are free until A is formed)
+            if (tid < L) {
+                float sa = 0.f, ss = 0.f, sk = 0.f;
+                for (int i = 0; i < DK; ++i) {
+                    const size_t e = ((size_t)(c0 + tid) * H + h) * DK + i;
+                    const float al = ldf(alpha + e), kk = ldf(k + e);
+                    sa = fmaf(al, al, sa);
+                    ss += ldf(sigma + e);
+                    sk = fmaf(kk, kk, sk);
+                }
+                As[tid * LDC + 0] = sa;
+                As[tid * LDC + 1] = ss;
+                As[tid * LDC + 2] = sk;
+            }
+            __syncthreads();
+            if (tid == 0) {
+                constexpr float inv_dk = 1.f / DK;
+                for (int t = 0; t < L; ++t) {
+                    const float pm = fmaf(As[t * LDC] * inv_dk, P, As[t * LDC + 1] * inv_dk);
+                    As[t * LDC + 3] = pm;
+                    P = pm / fmaf(mu * As[t * LDC + 2] * inv_dk / Rs[t], pm, 1.f);
+                }
+            }
+            __syncthreads();
+        }
         // ---- uncertainty recursion, gain numerators, cumulative log decay (thread = key channel)
         if (tid < DK) {
             float b = 0.f;
@@ -92,12 +126,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_simt_kernel(TokenArgs a, int C)
                 const size_t e = ((size_t)(c0 + t) * H + h) * DK + tid;
                 const float al = ldf(alpha + e), sg = ldf(sigma + e), kk = ldf(k + e);
                 b += fmaxf(logf(al), -80.f);
-                const float pm = fmaf(al * al, P, sg);
+                const float pm = a.iso ? As[t * LDC + 3] : fmaf(al * al, P, sg);
                 Ks[tid * LDC + t] = kk;
                 Qs[tid * LDC + t] = ldf(q + e);
                 Gs[tid * LDC + t] = pm * kk;
                 Bs[tid * LDC + t] = b;
-                P = pm / fmaf(mu * kk * kk / Rs[t], pm, 1.f);
+                if (!a.iso) P = pm / fmaf(mu * kk * kk / Rs[t], pm, 1.f);
             }
         }
         __syncthreads();
@@ -219,7 +253,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_simt_kernel(TokenArgs a, int C)
             const int i = e / DVT, j = e % DVT;
             a.S_out[sbase + (size_t)i * dv + j] = Ss[e];
         }
-    if (a.P_out && tid < DK && tile == 0) a.P_out[(size_t)sh * DK + tid] = P;
+    if (a.P_out && tile == 0) {
+        if (a.iso) {
+            if (tid == 0) a.P_out[sh] = P;
+        } else if (tid < DK) {
+            a.P_out[(size_t)sh * DK + tid] = P;
+        }
+    }
 }
 
 template <int DK, int DVT, typename Tin>

@@ -22,6 +22,11 @@
 // O = Q S0 + Aq U, S_next = Gam_{L-1} S0 + sum_s (Gam_{L-1}/Gam_s) g_s u_s^T.
 // The factored decay needs Gam_{L-1} >= 1e-30 per channel; a chunk outside that range
 // sets KDN_ERR_RANGE in the device error word (the fp32 CUDA-core path has no limit).
+//
+// Isotropic KDN (explainer "各向同性近似"; aifromscratch "Approximation 2"): the prep
+// replaces the per-channel recursion by per-token channel sums (alpha^2, sigma, k^2),
+// and one warp runs the head's scalar uncertainty as a warp-wide scan of the tokens'
+// 2x2 maps; P^- of every channel is then the head's p^-, and the rest is unchanged.
 #include <mutex>
 
 #include "kdn_common.cuh"
@@ -77,7 +82,7 @@ __device__ __forceinline__ uint4 pack8(const float *v, float sc = 1.f) {
 }
 }  // namespace
 
-template <int DVT>
+template <int DVT, bool ISO>
 __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__ TcParams prm)
 {
     using L_ = TcSmem<DVT>;
@@ -93,7 +98,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     float *mur = misc + 64;         // [64] mu / r_t
     float *invden = misc + 128;     // [64] 1 / den_t (0 past the chunk end)
     float *gamc = misc + 192;       // [128] chunk decay Gam_{L-1}
-    float *pst = misc + 320;        // [128] uncertainty at the chunk start
+    float *pst = misc + 320;        // [128] uncertainty at the chunk start (isotropic: pst[0])
     uint64_t *bar_tma = reinterpret_cast<uint64_t *>(misc + 448);
     uint64_t *bar_mma = bar_tma + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_mma + 1);
@@ -147,7 +152,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         for (int chn = 0; chn < NC / 8; ++chn)
             *reinterpret_cast<uint4 *>(sm + L_::S + atom + swz(row, (((cb0 & 63) >> 3) + chn) * 16)) = pack8(v + chn * 8);
     }
-    if (tid < DK) pst[tid] = a.P0 ? a.P0[(size_t)sh * DK + tid] : 1.f;
+    if (ISO) {
+        if (tid == 0) pst[0] = a.P0 ? a.P0[sh] : 1.f;
+    } else if (tid < DK) {
+        pst[tid] = a.P0 ? a.P0[(size_t)sh * DK + tid] : 1.f;
+    }
 
     const int nchunks = (t1 - t0 + C - 1) / C;
     uint32_t tma_phase = 0, mma_phase = 0;
@@ -193,6 +202,123 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         __syncthreads();
         if (*abort_flag) break;
 
+        if constexpr (ISO) {
+            // ---- isotropic: per-token channel sums, the decay table, then the head's
+            //      uncertainty by a warp scan of the tokens' maps [[a, s], [c a, c s + 1]]
+            //      with a = mean alpha^2, s = mean sigma, c = mu |k|^2 / (d_k r)
+            float *tsum = reinterpret_cast<float *>(sm + L_::Y);                  // [64][4]
+            float *segp = tsum + 256;                                             // [8][128]
+            float *pms = reinterpret_cast<float *>(sm + L_::A4);                  // [64] p^-
+            float *gst = reinterpret_cast<float *>(sm + L_::U);                   // [16][128]
+            {
+                const uint32_t atom8 = (uint32_t)(lane >> 4) * 8192u, bir = (uint32_t)(lane & 15) * 8u;
+                float xa[4], xs[4], xk[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t off = atom8 + swz(warp * 4 + j, bir);
+                    const uint2 aw = *reinterpret_cast<const uint2 *>(sm + L_::AL + off);
+                    const uint2 sw = *reinterpret_cast<const uint2 *>(sm + L_::SG + off);
+                    const uint2 kw = *reinterpret_cast<const uint2 *>(sm + L_::K + off);
+                    const float a0 = bf16_lo(aw.x), a1 = bf16_hi(aw.x), a2 = bf16_lo(aw.y), a3 = bf16_hi(aw.y);
+                    const float k0 = bf16_lo(kw.x), k1 = bf16_hi(kw.x), k2 = bf16_lo(kw.y), k3 = bf16_hi(kw.y);
+                    xa[j] = fmaf(a0, a0, fmaf(a1, a1, fmaf(a2, a2, a3 * a3)));
+                    xs[j] = (bf16_lo(sw.x) + bf16_hi(sw.x)) + (bf16_lo(sw.y) + bf16_hi(sw.y));
+                    xk[j] = fmaf(k0, k0, fmaf(k1, k1, fmaf(k2, k2, k3 * k3)));
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        xa[j] += __shfl_xor_sync(0xffffffffu, xa[j], off);
+                        xs[j] += __shfl_xor_sync(0xffffffffu, xs[j], off);
+                        xk[j] += __shfl_xor_sync(0xffffffffu, xk[j], off);
+                    }
+                if (lane < 4) {
+                    const float va = lane == 0 ? xa[0] : (lane == 1 ? xa[1] : (lane == 2 ? xa[2] : xa[3]));
+                    const float vs = lane == 0 ? xs[0] : (lane == 1 ? xs[1] : (lane == 2 ? xs[2] : xs[3]));
+                    const float vk = lane == 0 ? xk[0] : (lane == 1 ? xk[1] : (lane == 2 ? xk[2] : xk[3]));
+                    *reinterpret_cast<float4 *>(tsum + (warp * 4 + lane) * 4) = make_float4(va, vs, vk, 0.f);
+                }
+            }
+            const int cp = tid & 63, sgi = tid >> 6, ch = cp * 2;
+            const uint32_t coff = (uint32_t)(ch >> 6) * 8192u, cb = (uint32_t)(ch & 63) * 2u;
+            const int tb = sgi * 8, te = min(L, tb + 8);
+            uint32_t aw8[8];
+            float ga = 1.f, gb = 1.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                aw8[j] = *reinterpret_cast<const uint32_t *>(sm + L_::AL + coff + swz(tb + j, cb));
+                if (tb + j < te) { ga *= bf16_lo(aw8[j]); gb *= bf16_hi(aw8[j]); }
+            }
+            *reinterpret_cast<float2 *>(segp + sgi * 128 + ch) = make_float2(ga, gb);
+            __syncthreads();
+            float gama = 1.f, gamb = 1.f;
+            for (int q2 = 0; q2 < sgi; ++q2) {
+                const float2 x = *reinterpret_cast<const float2 *>(segp + q2 * 128 + ch);
+                gama *= x.x;
+                gamb *= x.y;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int t = tb + j;
+                if ((t & 3) == 0) *reinterpret_cast<float2 *>(gst + (t >> 2) * 128 + ch) = make_float2(gama, gamb);
+                if (t < te) { gama *= bf16_lo(aw8[j]); gamb *= bf16_hi(aw8[j]); }
+            }
+            if (te == L && tb < L) {
+                gamc[ch] = gama;
+                gamc[ch + 1] = gamb;
+                if (!(gama >= 1e-30f) || !(gamb >= 1e-30f)) raise_error(a.err, ERR_RANGE);
+            }
+            if (warp == 0) {
+                constexpr float inv_dk = 1.f / DK;
+                const float p0 = pst[0];
+                float ta[2], ts[2], tc[2];
+                float m00 = 1.f, m01 = 0.f, m10 = 0.f, m11 = 1.f;   // this lane's two tokens composed
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int t = 2 * lane + u;
+                    ta[u] = 1.f; ts[u] = 0.f; tc[u] = 0.f;
+                    if (t < L) {
+                        const float4 x = *reinterpret_cast<const float4 *>(tsum + t * 4);
+                        ta[u] = x.x * inv_dk;
+                        ts[u] = x.y * inv_dk;
+                        tc[u] = mur[t] * x.z * inv_dk;
+                    }
+                    // [[a, s], [c a, c s + 1]] applied after the composite so far
+                    const float y00 = ta[u] * m00 + ts[u] * m10, y01 = ta[u] * m01 + ts[u] * m11;
+                    m10 = fmaf(tc[u], y00, m10);
+                    m11 = fmaf(tc[u], y01, m11);
+                    m00 = y00;
+                    m01 = y01;
+                }
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {   // inclusive scan: lane's maps after the earlier lanes'
+                    const float n00 = __shfl_up_sync(0xffffffffu, m00, off), n01 = __shfl_up_sync(0xffffffffu, m01, off);
+                    const float n10 = __shfl_up_sync(0xffffffffu, m10, off), n11 = __shfl_up_sync(0xffffffffu, m11, off);
+                    if (lane >= off) {
+                        const float y00 = fmaf(m00, n00, m01 * n10), y01 = fmaf(m00, n01, m01 * n11);
+                        const float y10 = fmaf(m10, n00, m11 * n10), y11 = fmaf(m10, n01, m11 * n11);
+                        const float sc = 1.f / y11;
+                        m00 = y00 * sc; m01 = y01 * sc; m10 = y10 * sc; m11 = 1.f;
+                    }
+                }
+                float e00 = __shfl_up_sync(0xffffffffu, m00, 1), e01 = __shfl_up_sync(0xffffffffu, m01, 1);
+                float e10 = __shfl_up_sync(0xffffffffu, m10, 1), e11 = __shfl_up_sync(0xffffffffu, m11, 1);
+                if (lane == 0) { e00 = 1.f; e01 = 0.f; e10 = 0.f; e11 = 1.f; }
+                float p = fmaf(e00, p0, e01) / fmaf(e10, p0, e11);
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int t = 2 * lane + u;
+                    if (t < L) {
+                        const float pm = fmaf(ta[u], p, ts[u]);
+                        pms[t] = pm;
+                        p = __fdividef(pm, fmaf(tc[u], pm, 1.f));
+                    }
+                }
+                __syncwarp();
+                if (lane == (L - 1) >> 1) pst[0] = p;
+            }
+        } else {
         // ---- uncertainty recursion (thread = channel pair cp x 8-token segment sgi).  Each
         //      segment first composes the 2x2 maps of its tokens (predict [[a, s],[0,1]] then
         //      update [[1,0],[c,1]]); a segment then starts from the composites before it.
@@ -279,6 +405,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 if (!(gama >= 1e-30f) || !(gamb >= 1e-30f)) raise_error(a.err, ERR_RANGE);
             }
         }
+        }
         __syncthreads();
         // ---- elementwise pass (warp = 4 tokens, lane = 4 channels; 8-byte accesses):
         //      K~ = k Gam, Q~ = q Gam, G^ = P^- k / Gam, and den_t = r_t + sum_i P^-_i k_i^2
@@ -298,7 +425,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 aw[j] = *reinterpret_cast<const uint2 *>(sm + L_::AL + atom8 + off);
                 kw[j] = *reinterpret_cast<const uint2 *>(sm + L_::K + atom8 + off);
                 qw[j] = *reinterpret_cast<const uint2 *>(sm + L_::Q + atom8 + off);
-                pm[j] = *reinterpret_cast<const float4 *>(pmv + t * 128 + c4);
+                if constexpr (ISO) {
+                    const float x = pmv[t];
+                    pm[j] = make_float4(x, x, x, x);
+                } else {
+                    pm[j] = *reinterpret_cast<const float4 *>(pmv + t * 128 + c4);
+                }
             }
             float xs[4];
             uint2 kq[4], qq[4], gg[4];
@@ -629,7 +761,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 *reinterpret_cast<float4 *>(a.S_out + sbase + (size_t)row * dv + cb0 + j) =
                     make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         }
-        if (a.P_out && tid < DK && tile == 0) a.P_out[(size_t)sh * DK + tid] = pst[tid];
+        if (a.P_out && tile == 0) {
+            if (ISO) {
+                if (tid == 0) a.P_out[sh] = pst[0];
+            } else if (tid < DK) {
+                a.P_out[(size_t)sh * DK + tid] = pst[tid];
+            }
+        }
     } else {
         raise_error(a.err, ERR_TIMEOUT);
     }
@@ -669,10 +807,10 @@ static bool make_map(CUtensorMap *m, const void *base, int d, int H, long long n
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DVT>
+template <int DVT, bool ISO>
 static cudaError_t launch_tc(const TcParams &prm, cudaStream_t st) {
     constexpr size_t smem = TcSmem<DVT>::total + 1024;
-    auto kern = chunk_tc_kernel<DVT>;
+    auto kern = chunk_tc_kernel<DVT, ISO>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((size_t)prm.a.nseq * prm.a.H * (prm.a.dv / DVT));
@@ -692,8 +830,8 @@ cudaError_t launch_chunk_tc(const TokenArgs &a, long long ntok, int dvt, cudaStr
         !make_map(&prm.tv, a.v, a.dv, a.H, ntok) || !make_map(&prm.tal, a.alpha, DK, a.H, ntok) ||
         !make_map(&prm.tsg, a.sigma, DK, a.H, ntok))
         return cudaErrorInvalidValue;
-    if (dvt == 128) return launch_tc<128>(prm, st);
-    if (dvt == 64) return launch_tc<64>(prm, st);
+    if (dvt == 128) return a.iso ? launch_tc<128, true>(prm, st) : launch_tc<128, false>(prm, st);
+    if (dvt == 64) return a.iso ? launch_tc<64, true>(prm, st) : launch_tc<64, false>(prm, st);
     return cudaErrorInvalidValue;
 }
 

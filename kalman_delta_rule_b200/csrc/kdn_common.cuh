@@ -55,12 +55,13 @@ __device__ __forceinline__ float warp_sum(float x) {
 struct TokenArgs {
     const void *q, *k, *v, *alpha, *sigma, *r;  // [ntok, H, d] / [ntok, H]
     void *o;                                     // [ntok, H, dv]
-    const float *S0, *P0;                        // [N, H, dk, dv], [N, H, dk] (NULL -> 0 / 1)
+    const float *S0, *P0;                        // [N, H, dk, dv], [N, H, dk] ([N, H] isotropic) (NULL -> 0 / 1)
     float *S_out, *P_out;                        // may be NULL
     const int32_t *cu;                           // device [N+1] or NULL (dense: seq s = [s*T, (s+1)*T))
     int T;                                       // dense sequence length (ignored with cu)
     int nseq, H, dk, dv;
     float mu;
+    int iso;                                     // 1: isotropic KDN (one uncertainty per head)
     unsigned *err;
 };
 

@@ -10,6 +10,11 @@
 //   P = P^- / (1 + mu P^- k^2 / r)
 // o_t = S_t^T q_t expands to (D S)^T q + (q.g) u, so S is read once and written once.
 //
+// Isotropic KDN (explainer "各向同性近似"; aifromscratch "Approximation 2"): one
+// uncertainty p per head, held by every thread; per token the channel sums of alpha^2,
+// sigma, k^2 and q k give p^- = mean(alpha^2) p + mean(sigma), g = p^- k / (r + p^- |k|^2)
+// and p = p^- / (1 + mu p^- |k|^2 / (d_k r)).
+//
 // Decode is the same kernel on one token per sequence with the state in HBM updated
 // in place (one tile per head so the uncertainty read and write stay in one CTA).
 #include "kdn_common.cuh"
@@ -31,7 +36,7 @@ struct RecShape {
     static_assert(NT >= DK, "one thread per key channel");
 };
 
-template <int DK, int DVT, typename Tin>
+template <int DK, int DVT, typename Tin, bool ISO>
 __global__ void __launch_bounds__(RecShape<DK, DVT>::NT)
 recurrent_kernel(TokenArgs a, int write_p_all_tiles)
 {
@@ -61,7 +66,7 @@ recurrent_kernel(TokenArgs a, int write_p_all_tiles)
     __shared__ float g_s[DK];
     __shared__ float redA[RPP][DVT], redB[RPP][DVT];
     __shared__ float u_s[DVT];
-    __shared__ float wsum[2][NW];
+    __shared__ float wsum[ISO ? 4 : 2][NW];
 
     // memory tile -> registers
     float4 S[NPASS];
@@ -72,23 +77,34 @@ recurrent_kernel(TokenArgs a, int write_p_all_tiles)
         S[p] = a.S0 ? __ldcs(reinterpret_cast<const float4 *>(a.S0 + sbase + (size_t)row * a.dv + col0))
                     : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    float P = 1.f;
-    if (tid < DK && a.P0) P = a.P0[(size_t)sh * DK + tid];
+    float P = 1.f;   // diagonal: channel tid's uncertainty; isotropic: the head's (every thread)
+    if (ISO) {
+        if (a.P0) P = a.P0[sh];
+    } else if (tid < DK && a.P0) {
+        P = a.P0[(size_t)sh * DK + tid];
+    }
 
     const float mu = a.mu;
     for (int t = t0; t < t1; ++t) {
         const int buf = t & 1;
         const size_t th = (size_t)t * a.H + h;
         // ---- per key channel: predict and the two gain reductions
-        float pm = 0.f, kk = 0.f, x1 = 0.f, x2 = 0.f;
+        float pm = 0.f, kk = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f, x4 = 0.f;
         if (tid < DK) {
             const size_t e = th * DK + tid;
             const float al = ldf(alpha + e), sg = ldf(sigma + e), qq = ldf(q + e);
             kk = ldf(k + e);
-            pm = fmaf(al * al, P, sg);
-            const float pk = pm * kk;
-            x1 = pk * kk;
-            x2 = qq * pk;
+            if (ISO) {
+                x1 = kk * kk;
+                x2 = qq * kk;
+                x3 = al * al;
+                x4 = sg;
+            } else {
+                pm = fmaf(al * al, P, sg);
+                const float pk = pm * kk;
+                x1 = pk * kk;
+                x2 = qq * pk;
+            }
             ak_s[buf][tid] = al * kk;
             aq_s[buf][tid] = al * qq;
             al_s[buf][tid] = al;
@@ -98,16 +114,38 @@ recurrent_kernel(TokenArgs a, int write_p_all_tiles)
         const float rr = ldf(r + th);
         x1 = warp_sum(x1);
         x2 = warp_sum(x2);
-        if (lane == 0) { wsum[0][warp] = x1; wsum[1][warp] = x2; }
+        if (ISO) {
+            x3 = warp_sum(x3);
+            x4 = warp_sum(x4);
+        }
+        if (lane == 0) {
+            wsum[0][warp] = x1;
+            wsum[1][warp] = x2;
+            if constexpr (ISO) { wsum[2][warp] = x3; wsum[3][warp] = x4; }
+        }
         __syncthreads();
-        float sx1 = 0.f, sx2 = 0.f;
+        float sx1 = 0.f, sx2 = 0.f, sx3 = 0.f, sx4 = 0.f;
 #pragma unroll
-        for (int w = 0; w < NW; ++w) { sx1 += wsum[0][w]; sx2 += wsum[1][w]; }
-        const float den = rr + sx1;
-        const float qg = sx2 / den;
-        if (tid < DK) {
-            g_s[tid] = pm * kk / den;
-            P = pm / fmaf(mu * kk * kk / rr, pm, 1.f);
+        for (int w = 0; w < NW; ++w) {
+            sx1 += wsum[0][w];
+            sx2 += wsum[1][w];
+            if constexpr (ISO) { sx3 += wsum[2][w]; sx4 += wsum[3][w]; }
+        }
+        float den, qg;
+        if (ISO) {
+            constexpr float inv_dk = 1.f / DK;
+            pm = fmaf(sx3 * inv_dk, P, sx4 * inv_dk);
+            den = fmaf(pm, sx1, rr);
+            qg = pm * sx2 / den;
+            if (tid < DK) g_s[tid] = pm * kk / den;
+            P = pm / fmaf(mu * sx1 * inv_dk / rr, pm, 1.f);
+        } else {
+            den = rr + sx1;
+            qg = sx2 / den;
+            if (tid < DK) {
+                g_s[tid] = pm * kk / den;
+                P = pm / fmaf(mu * kk * kk / rr, pm, 1.f);
+            }
         }
         // ---- column partial sums of (alpha*k)^T S and (alpha*q)^T S over this thread's rows
         float4 A = make_float4(0.f, 0.f, 0.f, 0.f), B = A;
@@ -152,13 +190,20 @@ recurrent_kernel(TokenArgs a, int write_p_all_tiles)
             __stcs(reinterpret_cast<float4 *>(a.S_out + sbase + (size_t)row * a.dv + col0), S[p]);
         }
     }
-    if (a.P_out && tid < DK && (tile == 0 || write_p_all_tiles)) a.P_out[(size_t)sh * DK + tid] = P;
+    if (a.P_out && (tile == 0 || write_p_all_tiles)) {
+        if (ISO) {
+            if (tid == 0) a.P_out[sh] = P;
+        } else if (tid < DK) {
+            a.P_out[(size_t)sh * DK + tid] = P;
+        }
+    }
 }
 
 template <int DK, int DVT, typename Tin>
 static cudaError_t launch_rec(const TokenArgs &a, cudaStream_t st) {
     const unsigned grid = (unsigned)((size_t)a.nseq * a.H * (a.dv / DVT));
-    recurrent_kernel<DK, DVT, Tin><<<grid, RecShape<DK, DVT>::NT, 0, st>>>(a, 0);
+    if (a.iso) recurrent_kernel<DK, DVT, Tin, true><<<grid, RecShape<DK, DVT>::NT, 0, st>>>(a, 0);
+    else recurrent_kernel<DK, DVT, Tin, false><<<grid, RecShape<DK, DVT>::NT, 0, st>>>(a, 0);
     return cudaGetLastError();
 }
 

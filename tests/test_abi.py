@@ -69,6 +69,7 @@ def problem(**kw):
     (dict(in_dtype=7), B.KDN_ERR_INVALID_ARG),
     (dict(cu_seqlens=FAKE, B=2, num_seqs=3), B.KDN_ERR_INVALID_ARG),
     (dict(max_seqlen=-1), B.KDN_ERR_INVALID_ARG),
+    (dict(variant=2), B.KDN_ERR_INVALID_ARG),
 ])
 def test_problem_validation(lib, kw, code):
     p = problem(**kw)
@@ -110,6 +111,10 @@ def test_forward_rejects_bad_pointers(lib):
     assert B.kdn_gain_scan(p64, *k_a_s_r, None, FAKE, None, None, FAKE + 4096, need - 1, None) == B.KDN_ERR_WORKSPACE
     assert B.kdn_gain_scan(p64, *k_a_s_r, None, FAKE, None, None, FAKE + 16, need, None) == B.KDN_ERR_WORKSPACE
     assert B.kdn_gain_scan(p64, None, *k_a_s_r[1:], None, FAKE, None, None, FAKE, need, None) == B.KDN_ERR_INVALID_ARG
+    # the scan is built for the diagonal uncertainty only
+    piso = problem(chunk=64, variant=1)
+    assert B.kdn_gain_scan(piso, *k_a_s_r, None, FAKE, None, None, FAKE, need, None) == B.KDN_ERR_UNSUPPORTED
+    assert B.kdn_gain_scan_noalloc(piso, *k_a_s_r, None, FAKE, None, None, None) == B.KDN_ERR_UNSUPPORTED
 
 
 def test_decode_rejects_bad_arguments(lib):
@@ -122,6 +127,9 @@ def test_decode_rejects_bad_arguments(lib):
     bad = list(ptrs); bad[0] = FAKE + 8
     assert B.kdn_decode_step(4, 2, 64, 64, B.KDN_DTYPE_F32, 1.0, *bad, None) == B.KDN_ERR_INVALID_ARG
     assert B.kdn_decode_step(0, 2, 64, 64, B.KDN_DTYPE_F32, 1.0, *ptrs, None) == B.KDN_OK  # empty: no-op
+    assert B.kdn_decode_tokens_iso(4, 2, 2, 48, 64, B.KDN_DTYPE_BF16, 1.0, *ptrs, None) == B.KDN_ERR_UNSUPPORTED
+    assert B.kdn_decode_tokens_iso(4, -1, 2, 64, 64, B.KDN_DTYPE_BF16, 1.0, *ptrs, None) == B.KDN_ERR_INVALID_ARG
+    assert B.kdn_decode_tokens_iso(4, 2, 2, 64, 64, B.KDN_DTYPE_BF16, 1.0, *bad, None) == B.KDN_ERR_INVALID_ARG
 
 
 def test_product_path_fails_loudly_without_library(tmp_path):
