@@ -190,15 +190,17 @@ def bench_prefill(args, world, rank, dev, kdn):
     o = torch.empty(d["q"].shape[:3] + (w.dv,), dtype=d["q"].dtype, device=dev)
     S_out = torch.empty((w.num_seqs, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
     P_out = torch.empty((w.num_seqs, w.H, w.dk), dtype=torch.float32, device=dev)
-    prob = kdn.make_problem(d["q"], d["v"], cu_seqlens=cu, mu=w.mu, chunk=w.chunk)
+    max_seqlen = int(np.diff(w.cu_seqlens).max()) if cu is not None else 0
+    prob = kdn.make_problem(d["q"], d["v"], cu_seqlens=cu, mu=w.mu, chunk=w.chunk, max_seqlen=max_seqlen)
     ws_bytes = kdn.kdn_workspace_size(prob)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     path = kdn.PATH_NAMES[kdn.kdn_execution_path(prob)]
+    launches_per_step = 2 if path == "chunk_tcgen05_two_phase" else 1
     stream = torch.cuda.current_stream()
 
     def step():
         kdn.forward(d["q"], d["k"], d["v"], d["alpha"], d["sigma"], d["r"], cu_seqlens=cu, mu=w.mu, chunk=w.chunk,
-                    o=o, S_out=S_out, P_out=P_out, workspace=ws)
+                    o=o, S_out=S_out, P_out=P_out, workspace=ws, max_seqlen=max_seqlen)
 
     for _ in range(args.warmup):
         step()
@@ -258,7 +260,7 @@ def bench_prefill(args, world, rank, dev, kdn):
         g_out = torch.empty(d["k"].shape, dtype=torch.float32, device=dev)
         b_out = torch.empty(d["k"].shape[:3], dtype=torch.float32, device=dev)
         p_out = torch.empty((w.num_seqs, w.H, w.dk), dtype=torch.float32, device=dev)
-        sp = kdn.make_problem(d["k"], d["k"], cu_seqlens=cu, mu=w.mu, chunk=w.chunk)
+        sp = kdn.make_problem(d["k"], d["k"], cu_seqlens=cu, mu=w.mu, chunk=w.chunk, max_seqlen=max_seqlen)
         sargs = [d[n].data_ptr() for n in ("k", "alpha", "sigma", "r")]
         sh = stream.cuda_stream or None
 
@@ -289,7 +291,7 @@ def bench_prefill(args, world, rank, dev, kdn):
     return dict(w=w, value=value, ms_step=ms_step, per_step_ms=per_step_ms, clocks=clk.summary(), path=path, scan=scan,
                 e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                          steps=e_steps),
-                bytes=nbytes, launches=args.steps)
+                bytes=nbytes, launches=args.steps * launches_per_step)
 
 
 def bench_decode(args, world, rank, dev, kdn, steps=1024, N=256, H=32, d=128):

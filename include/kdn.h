@@ -71,8 +71,11 @@ typedef enum { KDN_VARIANT_DIAGONAL = 0, KDN_VARIANT_ISOTROPIC = 1 } kdn_variant
 
 /* Execution paths of kdn_forward_chunkwise (the `chunk` field):
  *  0        token-serial fused recurrence (any dtype; exact fp32 arithmetic);
- *  16/32/64 chunkwise: for bf16 inputs and chunk 64 the tcgen05 tensor-core kernel,
- *           otherwise the fp32 CUDA-core chunk kernel (same algebra, fp32 FMA). */
+ *  16/32/64 chunkwise: for bf16 inputs, d_k = 128 and chunk 64 the tcgen05 tensor cores --
+ *           in two launches (a chunk-parallel prep kernel, then the chunk-serial state
+ *           kernel) when the call gets a workspace of kdn_workspace_size() bytes and the
+ *           uncertainty is diagonal, else in one fused kernel; otherwise the fp32
+ *           CUDA-core chunk kernel (same algebra, fp32 FMA). */
 typedef struct {
     int B, T, H, d_k, d_v;          /* varlen: B == 1 and T = total tokens */
     const int32_t *cu_seqlens;      /* device int32 [num_seqs + 1], cu[0] = 0, cu[num_seqs] = T; NULL = dense batch */
@@ -86,9 +89,10 @@ typedef struct {
     int variant;                    /* kdn_variant_t; 0 (zero-initialised struct) = diagonal */
 } kdn_problem_t;
 
-/* Bytes of device workspace needed for `p`: the larger of what kdn_gain_scan() and
- * kdn_forward_chunkwise() use (the forward paths currently use none, so the forward
- * also accepts workspace = NULL).  Host-only; no CUDA call. */
+/* Bytes of device workspace for `p`: the larger of what kdn_gain_scan() and the two-launch
+ * tensor-core forward use (about 68 KB per 64-token chunk and head: per-chunk operand
+ * records and look-back state; `max_seqlen` bounds it for packed sequences).  The forward
+ * also accepts workspace = NULL and then runs the single-kernel paths.  Host-only. */
 kdn_status_t kdn_workspace_size(const kdn_problem_t *p, size_t *bytes);
 
 /* Prefill / training forward over whole sequences (KDA article, "chunkwise" regime;
@@ -100,8 +104,10 @@ kdn_status_t kdn_workspace_size(const kdn_problem_t *p, size_t *bytes);
  *  o                  : device [B, T, H, d_v]        (in_dtype), written for every token
  *  S_out, P_out       : device fp32, final states per sequence (shapes as S0, P0); either may be NULL.
  *                       They may not alias S0 / P0.
- *  workspace          : device, >= kdn_workspace_size() bytes, 256-byte aligned; its
- *                       contents on entry do not matter.
+ *  workspace          : device, 256-byte aligned, or NULL.  With >= kdn_workspace_size()
+ *                       bytes the tensor-core path runs in two launches (faster); with less
+ *                       or NULL it runs as one kernel.  Contents on entry do not matter;
+ *                       concurrent calls must use distinct workspaces.
  * Every sequence starts from its own S0/P0 (chunks restart at sequence starts). */
 kdn_status_t kdn_forward_chunkwise(const kdn_problem_t *p,
                                    const void *q, const void *k, const void *v,
@@ -185,7 +191,9 @@ kdn_status_t kdn_gain_scan_noalloc(const kdn_problem_t *p,
 
 /* Which execution path kdn_forward_chunkwise() takes for `p` (host-only; no CUDA call
  * besides resolving the driver's tensor-map encoder once): 0 token-serial recurrence,
- * 1 fp32 CUDA-core chunk kernel, 2 tcgen05 tensor-core chunk kernel; -1 if `p` is invalid. */
+ * 1 fp32 CUDA-core chunk kernel, 2 tcgen05 tensor-core chunk kernel, 3 the tcgen05 path in
+ * two launches (taken when the call also gets a workspace of kdn_workspace_size() bytes;
+ * without one such a problem runs path 2); -1 if `p` is invalid. */
 int kdn_execution_path(const kdn_problem_t *p);
 
 /* Synchronises `stream`, then returns and clears the device error word

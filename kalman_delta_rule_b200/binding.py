@@ -181,13 +181,14 @@ def make_problem(q, v, H=None, cu_seqlens=None, mu: float = 1.0, chunk: int = 64
 
 def forward(q, k, v, alpha, sigma, r, cu_seqlens=None, S0=None, P0=None, mu: float = 1.0, chunk: int = 64,
             o=None, S_out=None, P_out=None, workspace=None, want_state: bool = True, stream=None,
-            variant: str = "diagonal"):
+            variant: str = "diagonal", max_seqlen: int = 0):
     """Run kdn_forward_chunkwise on torch tensors ([B,T,H,d]; varlen: B = 1 with int32 cu_seqlens).
 
-    Returns (o, S_out, P_out); P is [N,H,dk] (diagonal) or [N,H] (isotropic).  Outputs and
-    workspace are allocated when not given."""
+    Returns (o, S_out, P_out); P is [N,H,dk] (diagonal) or [N,H] (isotropic).  Outputs are
+    allocated when not given; so is the workspace when ``workspace`` is None (``False``
+    passes none, which selects the single-kernel paths)."""
     torch = _torch()
-    p = make_problem(q, v, cu_seqlens=cu_seqlens, mu=mu, chunk=chunk, variant=variant)
+    p = make_problem(q, v, cu_seqlens=cu_seqlens, mu=mu, chunk=chunk, variant=variant, max_seqlen=max_seqlen)
     N = p.num_seqs
     dev = q.device
     if o is None:
@@ -196,9 +197,11 @@ def forward(q, k, v, alpha, sigma, r, cu_seqlens=None, S0=None, P0=None, mu: flo
         S_out = torch.empty((N, p.H, p.d_k, p.d_v), dtype=torch.float32, device=dev)
     if want_state and P_out is None:
         P_out = torch.empty((N, p.H) + ((p.d_k,) if p.variant == 0 else ()), dtype=torch.float32, device=dev)
-    need = kdn_workspace_size(p)
-    if workspace is None and need:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace is False:
+        workspace = None
+    elif workspace is None:
+        need = kdn_workspace_size(p)
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev) if need else None
     wbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     st = kdn_forward_chunkwise(p, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(sigma), _ptr(r), _ptr(S0), _ptr(P0),
                                _ptr(o), _ptr(S_out), _ptr(P_out), _ptr(workspace), wbytes, _stream_handle(stream))
@@ -259,13 +262,18 @@ def gain_scan(k, alpha, sigma, r, cu_seqlens=None, P0=None, mu: float = 1.0, chu
     return g, be, P_out
 
 
-PATH_NAMES = {0: "recurrent", 1: "chunk_fp32", 2: "chunk_tcgen05"}
+PATH_NAMES = {0: "recurrent", 1: "chunk_fp32", 2: "chunk_tcgen05", 3: "chunk_tcgen05_two_phase"}
 
 
-def execution_path(q, v, cu_seqlens=None, mu: float = 1.0, chunk: int = 64, variant: str = "diagonal") -> str:
-    """Name of the kernel path kdn_forward_chunkwise takes for these tensors."""
+def execution_path(q, v, cu_seqlens=None, mu: float = 1.0, chunk: int = 64, variant: str = "diagonal",
+                   workspace: bool = True) -> str:
+    """Name of the kernel path kdn_forward_chunkwise takes for these tensors (``workspace``:
+    whether the call gets a workspace of kdn_workspace_size() bytes)."""
     p = make_problem(q, v, cu_seqlens=cu_seqlens, mu=mu, chunk=chunk, variant=variant)
-    return PATH_NAMES.get(kdn_execution_path(p), "invalid")
+    code = kdn_execution_path(p)
+    if code == 3 and not workspace:
+        code = 2
+    return PATH_NAMES.get(code, "invalid")
 
 
 def last_device_error(stream=None):

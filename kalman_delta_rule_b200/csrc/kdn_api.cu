@@ -29,6 +29,7 @@ unsigned *err_word() {
 bool dk_ok(int d) { return d == 32 || d == 64 || d == 128; }
 bool dv_ok(int d) { return d == 32 || d == 64 || d == 128 || d == 256; }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
 
 struct Resolved {
     long long ntok;
@@ -62,6 +63,19 @@ kdn_status_t check_problem(const kdn_problem_t *p, Resolved *out) {
 
 kdn_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? KDN_OK : KDN_ERR_CUDA; }
 
+// the tensor-core chunk kernels serve this problem (bf16, d_k = 128, chunk 64)
+bool tc_path(const kdn_problem_t *p, const Resolved &rv) {
+    return kdn::chunk_tc_supported(p->d_k, p->d_v, rv.bf16, p->chunk, rv.ntok);
+}
+// ... and the two-launch form applies (diagonal uncertainty, work list within 2^31 units)
+bool two_phase_path(const kdn_problem_t *p, const Resolved &rv) {
+    return tc_path(p, rv) && p->variant == KDN_VARIANT_DIAGONAL &&
+           (long long)rv.nseq * p->H * rv.nchunks_max < (1ll << 31);
+}
+size_t two_phase_bytes(const kdn_problem_t *p, const Resolved &rv) {
+    return kdn::two_phase_workspace_bytes((long long)rv.nseq * p->H, rv.nchunks_max);
+}
+
 }  // namespace
 
 extern "C" {
@@ -86,7 +100,12 @@ kdn_status_t kdn_workspace_size(const kdn_problem_t *p, size_t *bytes) {
     kdn_status_t st = check_problem(p, &rv);
     if (st != KDN_OK) return st;
     if (!bytes) return KDN_ERR_INVALID_ARG;
-    *bytes = kdn::scan_workspace_bytes((long long)rv.nseq * p->H, rv.nchunks_max, p->d_k);
+    size_t n = kdn::scan_workspace_bytes((long long)rv.nseq * p->H, rv.nchunks_max, p->d_k);
+    if (two_phase_path(p, rv)) {
+        const size_t m = two_phase_bytes(p, rv);
+        if (m > n) n = m;
+    }
+    *bytes = n;
     return KDN_OK;
 }
 
@@ -97,7 +116,6 @@ kdn_status_t kdn_forward_chunkwise(const kdn_problem_t *p, const void *q, const 
     Resolved rv;
     kdn_status_t st = check_problem(p, &rv);
     if (st != KDN_OK) return st;
-    (void)workspace; (void)workspace_bytes;   // the forward paths use no workspace
     if (rv.nseq == 0 || (rv.ntok == 0 && !S_out && !P_out)) return KDN_OK;
     if (rv.ntok > 0 && (!q || !k || !v || !alpha || !sigma || !r || !o)) return KDN_ERR_INVALID_ARG;
     const void *ptrs[] = {q, k, v, alpha, sigma, r, o, S0, P0, S_out, P_out};
@@ -117,7 +135,9 @@ kdn_status_t kdn_forward_chunkwise(const kdn_problem_t *p, const void *q, const 
         const int dvt = p->d_v < 64 ? p->d_v : 64;
         return cuda_status(kdn::launch_recurrent(a, rv.bf16, dvt, cs));
     }
-    if (kdn::chunk_tc_supported(p->d_k, p->d_v, rv.bf16, p->chunk, rv.ntok)) {
+    if (two_phase_path(p, rv) && workspace && aligned256(workspace) && workspace_bytes >= two_phase_bytes(p, rv))
+        return cuda_status(kdn::launch_chunk_two_phase(a, rv.ntok, rv.nchunks_max, workspace, cs));
+    if (tc_path(p, rv)) {
         const long long ctas128 = (long long)rv.nseq * p->H * (p->d_v / 128);
         const int dvt = (p->d_v == 64 || ctas128 < 148) ? 64 : 128;
         return cuda_status(kdn::launch_chunk_tc(a, rv.ntok, dvt, cs));
@@ -215,7 +235,8 @@ int kdn_execution_path(const kdn_problem_t *p) {
     Resolved rv;
     if (check_problem(p, &rv) != KDN_OK) return -1;
     if (p->chunk == 0) return 0;
-    return kdn::chunk_tc_supported(p->d_k, p->d_v, rv.bf16, p->chunk, rv.ntok) ? 2 : 1;
+    if (two_phase_path(p, rv)) return 3;
+    return tc_path(p, rv) ? 2 : 1;
 }
 
 kdn_status_t kdn_last_device_error(void *stream) {

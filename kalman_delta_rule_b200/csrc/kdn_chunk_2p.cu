@@ -1,0 +1,865 @@
+// Chunkwise Diagonal-KDN forward in two launches on the tcgen05 tensor cores (KDA article,
+// "chunkwise" regime; explainer "对角近似" for the diagonal uncertainty and, closing
+// paragraph of "各向同性近似", the Moebius form of its recursion).
+//
+// Everything of a chunk that does not involve the memory S is independent across chunks
+// once the uncertainty at the chunk start is known, and that uncertainty comes from an
+// associative (Moebius) scan.  So the work splits into
+//
+//   prep  (one unit = one 64-token chunk of one (sequence, head); every unit in parallel):
+//         compose the chunk's 2x2 uncertainty maps, take the starting uncertainty from the
+//         chunk's predecessors by decoupled look-back, re-expand P^- per token, form
+//         K~ = k Gam, Q~ = q Gam, G^ = P^- k / Gam and 1/den, then on the tensor cores
+//         [A; Aq] = [K~; Q~] G^^T, T = (I + A)^{-1}, X = Aq T, [w; X K~] = [T; X] K~, and
+//         write one record per unit: [-w; Q'] (Q' = Q~ - X K~), [T; X], G^, 1/den, Gam_{L-1};
+//   state (one CTA per (sequence, head, d_v tile); chunks in order):
+//         [U; O] = [-w; Q'] S + [T; X] V,   S <- Gam_{L-1} (S + G^^T (U / den)).
+//
+// Records are stored exactly in the state kernel's shared-memory operand layout (128-byte
+// swizzled atoms), so the state kernel fetches each with one bulk copy, double-buffered,
+// and its per-chunk critical path is two MMAs and two TMEM epilogues.
+//
+// The prep kernel runs two 256-thread CTAs per SM; work is handed out by a ticket counter
+// in chunk-major order, so every predecessor of a unit belongs to a CTA that is already
+// running, and every wait is bounded (a wait that gives up records KDN_ERR_TIMEOUT).
+#include "kdn_common.cuh"
+#include "kdn_launch.h"
+#include "kdn_tc.cuh"
+
+namespace kdn {
+
+namespace {
+constexpr int C = 64, DK = 128, PNT = 256, SNT = 256;
+enum : int { FLAG_NONE = 0, FLAG_AGG = 1, FLAG_INCL = 2 };
+
+// one unit's record; each part in the state kernel's operand layout
+struct Rec {
+    static constexpr uint32_t A4 = 0;          // [-w; Q'] bf16: 2 channel atoms x 128 rows x 128 B
+    static constexpr uint32_t Y = 32768;       // [T; X] bf16: 128 rows x 64 tokens
+    static constexpr uint32_t G = 49152;       // G^ bf16: 2 channel atoms x 64 token rows
+    static constexpr uint32_t MISC = 65536;    // 1/den [64] fp32, then Gam_{L-1} [128] fp32
+    static constexpr uint32_t BYTES = MISC + 768;
+};
+
+struct PrepSmem {
+    static constexpr uint32_t KQ = 0;                  // [K~; Q~] bf16, 2 channel atoms x 128 rows
+    static constexpr uint32_t G = 32768;               // G^ bf16 (record part)
+    static constexpr uint32_t W = 49152;               // work region, reused phase by phase:
+    static constexpr uint32_t COMP = W;                //   segment composites fp32 [4][128][4]
+    static constexpr uint32_t AQ = W;                  //   Aq bf16 64 x 64
+    static constexpr uint32_t DB = W + 8192;           //   D bf16 64 x 64
+    static constexpr uint32_t LB = W + 16384;          //   L, then R = I - N + N^2 - N^3
+    static constexpr uint32_t NB = W + 24576;          //   N
+    static constexpr uint32_t N2B = W + 32768;         //   N^2
+    static constexpr uint32_t ADG = W + 40960;         //   fp32 [4][16][16]: A's diagonal blocks, then D's
+    static constexpr uint32_t A4 = W;                  //   [-w; Q'] (record part), once the inverse is done
+    static constexpr uint32_t Y = W + 45056;           //   [T; X] (record part)
+    static constexpr uint32_t MISC = W + 61440;        // 1/den [64], Gam_{L-1} [128] (record tail)
+    static constexpr uint32_t RS = MISC + 768;         // r [64]
+    static constexpr uint32_t MUR = RS + 256;          // mu / r [64]
+    static constexpr uint32_t PST = MUR + 256;         // uncertainty at the chunk start [128]
+    static constexpr uint32_t DSUM = PST + 512;        // sum_i P^- k^2 per token [64]
+    static constexpr uint32_t CTL = DSUM + 256;        // mbarrier, ticket, TMEM slot, look-back flag, abort
+    static constexpr uint32_t total = CTL + 64;
+    static_assert(COMP + 4 * 128 * 16 <= DB, "composites overlap D");
+    static_assert(ADG + 4096 <= Y && Y + 16384 <= MISC, "work region");
+};
+
+template <int DVT>
+struct StateSmem {
+    static constexpr uint32_t STAGE = 67584;               // a record, rounded up to 1 KB
+    static constexpr uint32_t V0 = 2 * STAGE;              // two v tiles, DVT * 128 B each
+    static constexpr uint32_t S = V0 + 2 * DVT * 128;      // S bf16, 128 channel rows x DVT (MN-major)
+    static constexpr uint32_t U = S + DVT * 256;           // U / den bf16, 64 token rows x DVT
+    static constexpr uint32_t CTL = U + DVT * 128;         // 3 mbarriers, TMEM slot
+    static constexpr uint32_t total = CTL + 64;
+    static constexpr uint32_t V_BYTES = DVT * 128;
+};
+
+struct PrepArgs {
+    TokenArgs a;
+    long long nchunks_max;
+    int nchains;
+    unsigned *counter;
+    int *flags;
+    float *desc;      // per unit [4][128]: aggregate map (m00, m01, m10) and end-of-chunk P
+    uint8_t *rec;     // per unit Rec::BYTES
+};
+
+struct StateArgs {
+    TokenArgs a;
+    CUtensorMap tv;
+    const uint8_t *rec;
+    long long nchunks_max;
+    int nchains;
+};
+
+__device__ __forceinline__ float mob(float m00, float m01, float m10, float m11, float x) {
+    return fmaf(m00, x, m01) / fmaf(m10, x, m11);
+}
+
+__device__ __forceinline__ uint4 pack8(const float *v, float sc = 1.f) {
+    uint4 w;
+    w.x = tc::pack_bf16x2(v[0] * sc, v[1] * sc);
+    w.y = tc::pack_bf16x2(v[2] * sc, v[3] * sc);
+    w.z = tc::pack_bf16x2(v[4] * sc, v[5] * sc);
+    w.w = tc::pack_bf16x2(v[6] * sc, v[7] * sc);
+    return w;
+}
+
+__device__ __forceinline__ uint32_t ldg_u32(const bf16 *p) { return __ldg(reinterpret_cast<const unsigned *>(p)); }
+
+// Sums 16 per-lane values over the 32 lanes of a warp with 16 shuffles (each step exchanges
+// half of the remaining values).  Lanes 2m and 2m+1 end with the total of value `which`.
+__device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane, int &which) {
+    const unsigned FULL = 0xffffffffu;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const bool up = lane & 16;
+        const float send = up ? v[i] : v[i + 8], keep = up ? v[i + 8] : v[i];
+        v[i] = keep + __shfl_xor_sync(FULL, send, 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const bool up = lane & 8;
+        const float send = up ? v[i] : v[i + 4], keep = up ? v[i + 4] : v[i];
+        v[i] = keep + __shfl_xor_sync(FULL, send, 8);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const bool up = lane & 4;
+        const float send = up ? v[i] : v[i + 2], keep = up ? v[i + 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(FULL, send, 4);
+    }
+    {
+        const bool up = lane & 2;
+        const float send = up ? v[0] : v[1], keep = up ? v[1] : v[0];
+        v[0] = keep + __shfl_xor_sync(FULL, send, 2);
+    }
+    v[0] += __shfl_xor_sync(FULL, v[0], 1);
+    which = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+    return v[0];
+}
+}  // namespace
+
+// ================================================================= prep
+__global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constant__ PrepArgs pa)
+{
+    using L_ = PrepSmem;
+    using namespace tc;
+    extern __shared__ uint8_t smraw[];
+    const uint32_t raw_u32 = smem_u32(smraw);
+    const uint32_t sb = (raw_u32 + 1023u) & ~1023u;
+    uint8_t *sm = smraw + (sb - raw_u32);
+
+    float *invden = reinterpret_cast<float *>(sm + L_::MISC);
+    float *gamc = invden + 64;
+    float *r_s = reinterpret_cast<float *>(sm + L_::RS);
+    float *mur = reinterpret_cast<float *>(sm + L_::MUR);
+    float *pst = reinterpret_cast<float *>(sm + L_::PST);
+    float *dsum = reinterpret_cast<float *>(sm + L_::DSUM);
+    float *comp = reinterpret_cast<float *>(sm + L_::COMP);
+    float *adg = reinterpret_cast<float *>(sm + L_::ADG);
+    uint64_t *bar_mma = reinterpret_cast<uint64_t *>(sm + L_::CTL);
+    long long *ticket = reinterpret_cast<long long *>(sm + L_::CTL + 8);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L_::CTL + 16);
+    int *ctl = reinterpret_cast<int *>(sm + L_::CTL + 20);   // [0] look-back flag, [1] abort
+
+    const TokenArgs &a = pa.a;
+    const bf16 *__restrict__ qin = static_cast<const bf16 *>(a.q);
+    const bf16 *__restrict__ kin = static_cast<const bf16 *>(a.k);
+    const bf16 *__restrict__ ain = static_cast<const bf16 *>(a.alpha);
+    const bf16 *__restrict__ sin_ = static_cast<const bf16 *>(a.sigma);
+    const bf16 *__restrict__ rin = static_cast<const bf16 *>(a.r);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, cg = warp >> 2;     // TMEM lane quadrant, column half
+    const int H = a.H;
+    const long long units = pa.nchunks_max * pa.nchains;
+
+    if (tid == 0) {
+        mbar_init(bar_mma, 1);
+        mbar_fence_init();
+        ctl[1] = 0;
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, 256);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t T_A = *tmem_slot;
+    const uint32_t lane_off = ((uint32_t)quad * 32u) << 16;
+    const int row = quad * 32 + lane;     // TMEM lane of this thread in M=128 epilogues
+    const int m64 = quad * 16 + lane;     // row of an M=64 accumulator (lanes < 16)
+    uint32_t mma_phase = 0;
+
+    constexpr uint32_t ID_M128_N64_KK = idesc_bf16(128, 64, false, false);
+    constexpr uint32_t ID_M64_N64_KM = idesc_bf16(64, 64, false, true);
+    constexpr uint32_t ID_M128_N128_KM = idesc_bf16(128, 128, false, true);
+
+    auto wait_mma = [&]() {
+        if (!mbar_wait(bar_mma, mma_phase)) atomicExch(&ctl[1], 1);
+        mma_phase ^= 1u;
+        tc_fence_after();
+    };
+    auto sync_tc = [&]() {
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+    };
+    // M=64 x N=64 x K=64 product: A operand K-major (rows of 128 B), B operand MN-major
+    auto mma64 = [&](uint32_t dcol, uint32_t aoff, uint32_t boff) {
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(dcol, sdesc(sb + aoff + ks * 32u, 16, 1024), sdesc(sb + boff + ks * 2048u, 8192, 1024),
+                         ID_M64_N64_KM, ks > 0);
+            mma_commit(bar_mma);
+        }
+        wait_mma();
+    };
+    // 64 x 64 bf16 tile from an M=64 accumulator: row m sits in lane (m % 16) + 32 (m / 16)
+    auto store64 = [&](uint32_t dst, int row0, const float (&v)[32]) {
+        if (lane < 16) {
+#pragma unroll
+            for (int chn = 0; chn < 4; ++chn)
+                *reinterpret_cast<uint4 *>(sm + dst + swz(row0 + m64, (cg * 4 + chn) * 16)) = pack8(v + chn * 8);
+        }
+    };
+
+    for (;;) {
+        if (tid == 0) *ticket = (long long)atomicAdd(pa.counter, 1u);
+        __syncthreads();
+        const long long u = *ticket;
+        if (u >= units || ctl[1]) break;
+        const int c = (int)(u / pa.nchains), chain = (int)(u % pa.nchains);
+        const int s = chain / H, h = chain % H;
+        int t0, t1;
+        seq_range(a, s, t0, t1);
+        const int nch = (t1 - t0 + C - 1) / C;
+        if (c == 0 && tid == 0 && nch > pa.nchunks_max) raise_error(a.err, ERR_ARG);
+        if (c >= nch) {
+            __syncthreads();   // every thread has read the ticket before it is replaced
+            continue;
+        }
+        const int c0 = t0 + c * C, L = min(C, t1 - c0);
+
+        if (tid < C) {
+            const float rr = tid < L ? ldf(rin + (size_t)(c0 + tid) * H + h) : 1.f;
+            r_s[tid] = rr;
+            mur[tid] = a.mu / rr;
+            dsum[tid] = 0.f;
+        }
+        // thread = key-channel pair cp x 16-token segment sgi; alpha, sigma, k of its tokens
+        const int cp = (warp & 1) * 32 + lane, sgi = warp >> 1, ch = cp * 2, tb = sgi * 16;
+        uint32_t aw[16], sw[16], kw[16], qw[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            aw[j] = 0u; sw[j] = 0u; kw[j] = 0u;
+            if (tb + j < L) {
+                const size_t e = ((size_t)(c0 + tb + j) * H + h) * DK + ch;
+                aw[j] = ldg_u32(ain + e);
+                sw[j] = ldg_u32(sin_ + e);
+                kw[j] = ldg_u32(kin + e);
+            }
+        }
+        if (tid == 0) bulk_wait_read0();   // the previous record's bulk stores have read shared memory
+        __syncthreads();
+
+        // ---- segment composites of the uncertainty maps (predict [[a, s],[0,1]], update [[1,0],[c,1]])
+        {
+            float a00 = 1.f, a01 = 0.f, a10 = 0.f, a11 = 1.f, ga = 1.f;
+            float b00 = 1.f, b01 = 0.f, b10 = 0.f, b11 = 1.f, gb = 1.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                if (tb + j < L) {
+                    const float mr = mur[tb + j];
+                    {
+                        const float al = bf16_lo(aw[j]), sg = bf16_lo(sw[j]), kk = bf16_lo(kw[j]);
+                        const float aa = al * al, cc = mr * kk * kk;
+                        const float y00 = fmaf(aa, a00, sg * a10), y01 = fmaf(aa, a01, sg * a11);
+                        a10 = fmaf(cc, y00, a10); a11 = fmaf(cc, y01, a11); a00 = y00; a01 = y01; ga *= al;
+                    }
+                    {
+                        const float al = bf16_hi(aw[j]), sg = bf16_hi(sw[j]), kk = bf16_hi(kw[j]);
+                        const float aa = al * al, cc = mr * kk * kk;
+                        const float y00 = fmaf(aa, b00, sg * b10), y01 = fmaf(aa, b01, sg * b11);
+                        b10 = fmaf(cc, y00, b10); b11 = fmaf(cc, y01, b11); b00 = y00; b01 = y01; gb *= al;
+                    }
+                }
+            }
+            const float sa = 1.f / a11, sbb = 1.f / b11;
+            *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch) * 4) = make_float4(a00 * sa, a01 * sa, a10 * sa, ga);
+            *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch + 1) * 4) = make_float4(b00 * sbb, b01 * sbb, b10 * sbb, gb);
+        }
+        // q of the thread's tokens (consumed after the look-back)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            qw[j] = 0u;
+            if (tb + j < L) qw[j] = ldg_u32(qin + ((size_t)(c0 + tb + j) * H + h) * DK + ch);
+        }
+        __syncthreads();
+
+        // ---- chunk aggregate (thread = channel), publication and decoupled look-back
+        float g00 = 1.f, g01 = 0.f, g10 = 0.f, g11 = 1.f;
+        float *desc = pa.desc + (size_t)u * 4 * DK;
+        if (tid < DK) {
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+                const float4 cm = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + tid) * 4);
+                const float n00 = fmaf(cm.x, g00, cm.y * g10), n01 = fmaf(cm.x, g01, cm.y * g11);
+                const float n10 = fmaf(cm.z, g00, g10), n11 = fmaf(cm.z, g01, g11);
+                const float sc = 1.f / n11;
+                g00 = n00 * sc; g01 = n01 * sc; g10 = n10 * sc; g11 = 1.f;
+            }
+            if (c > 0) {
+                __stcg(desc + 0 * DK + tid, g00);
+                __stcg(desc + 1 * DK + tid, g01);
+                __stcg(desc + 2 * DK + tid, g10);
+            }
+        }
+        if (c > 0) {
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) atomicExch(pa.flags + u, FLAG_AGG);
+        }
+        if (c == 0) {
+            if (tid < DK) pst[tid] = a.P0 ? a.P0[(size_t)chain * DK + tid] : 1.f;
+        } else {
+            float r00 = 1.f, r01 = 0.f, r10 = 0.f, r11 = 1.f;   // composite of the chunks walked over
+            int j = c - 1;
+            for (;;) {
+                const long long uj = (long long)j * pa.nchains + chain;
+                if (tid == 0) {
+                    volatile int *fp = pa.flags + uj;
+                    int f = *fp;
+                    const long long ts = clock64();
+                    while (f == FLAG_NONE) {
+                        if (clock64() - ts > 2000000000ll) break;
+                        __nanosleep(64);
+                        f = *fp;
+                    }
+                    if (f == FLAG_NONE) { raise_error(a.err, ERR_TIMEOUT); f = -1; }
+                    ctl[0] = f;
+                }
+                __syncthreads();
+                const int f = ctl[0];
+                __threadfence();
+                const float *dj = pa.desc + (size_t)uj * 4 * DK;
+                if (f == FLAG_INCL || f < 0) {
+                    if (tid < DK) {
+                        const float pe = f < 0 ? 1.f : __ldcg(dj + 3 * DK + tid);
+                        pst[tid] = mob(r00, r01, r10, r11, pe);
+                    }
+                    __syncthreads();
+                    break;
+                }
+                if (tid < DK) {   // R <- R * A_j (A_j acts first)
+                    const float m00 = __ldcg(dj + tid), m01 = __ldcg(dj + DK + tid), m10 = __ldcg(dj + 2 * DK + tid);
+                    const float n00 = fmaf(r00, m00, r01 * m10), n01 = fmaf(r00, m01, r01);
+                    const float n10 = fmaf(r10, m00, r11 * m10), n11 = fmaf(r10, m01, r11);
+                    const float sc = 1.f / n11;
+                    r00 = n00 * sc; r01 = n01 * sc; r10 = n10 * sc; r11 = 1.f;
+                }
+                __syncthreads();
+                --j;
+            }
+        }
+        __syncthreads();
+        if (tid < DK) {
+            const float pe = mob(g00, g01, g10, g11, pst[tid]);
+            __stcg(desc + 3 * DK + tid, pe);
+            if (c == nch - 1 && a.P_out) a.P_out[(size_t)chain * DK + tid] = pe;
+        }
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) atomicExch(pa.flags + u, FLAG_INCL);
+
+        // ---- re-expansion fused with the chunk operands: P^- per token, Gam (inclusive decay
+        //      from the chunk start), K~ = k Gam, Q~ = q Gam, G^ = P^- k / Gam, den partial sums
+        {
+            float Pa = pst[ch], Pb = pst[ch + 1], gama = 1.f, gamb = 1.f;
+            for (int q2 = 0; q2 < sgi; ++q2) {
+                const float4 ca = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch) * 4);
+                const float4 cb = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch + 1) * 4);
+                Pa = mob(ca.x, ca.y, ca.z, 1.f, Pa);
+                Pb = mob(cb.x, cb.y, cb.z, 1.f, Pb);
+                gama *= ca.w;
+                gamb *= cb.w;
+            }
+            const uint32_t atom16 = (uint32_t)(ch >> 6) * 16384u, atom8 = (uint32_t)(ch >> 6) * 8192u;
+            const uint32_t bch = (uint32_t)(ch & 63) * 2u;
+            float xs[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int t = tb + j;
+                uint32_t kq = 0u, qq = 0u, gg = 0u;
+                xs[j] = 0.f;
+                if (t < L) {
+                    const float ala = bf16_lo(aw[j]), alb = bf16_hi(aw[j]);
+                    const float ka = bf16_lo(kw[j]), kb = bf16_hi(kw[j]);
+                    const float pma = fmaf(ala * ala, Pa, bf16_lo(sw[j])), pmb = fmaf(alb * alb, Pb, bf16_hi(sw[j]));
+                    const float mr = mur[t];
+                    Pa = __fdividef(pma, fmaf(mr * ka * ka, pma, 1.f));
+                    Pb = __fdividef(pmb, fmaf(mr * kb * kb, pmb, 1.f));
+                    gama *= ala;
+                    gamb *= alb;
+                    const float pka = pma * ka, pkb = pmb * kb;
+                    kq = pack_bf16x2(ka * gama, kb * gamb);
+                    qq = pack_bf16x2(bf16_lo(qw[j]) * gama, bf16_hi(qw[j]) * gamb);
+                    gg = pack_bf16x2(__fdividef(pka, gama), __fdividef(pkb, gamb));
+                    xs[j] = fmaf(pka, ka, pkb * kb);
+                }
+                *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(t, bch)) = kq;
+                *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(64 + t, bch)) = qq;
+                *reinterpret_cast<uint32_t *>(sm + L_::G + atom8 + swz(t, bch)) = gg;
+            }
+            if (tb < L && tb + 16 >= L) {   // this segment holds the chunk's last token
+                gamc[ch] = gama;
+                gamc[ch + 1] = gamb;
+                if (!(gama >= 1e-30f) || !(gamb >= 1e-30f)) raise_error(a.err, ERR_RANGE);
+            }
+            int which;
+            const float tot = warp_reduce16(xs, lane, which);
+            if ((lane & 1) == 0 && tb + which < L) atomicAdd(dsum + tb + which, tot);
+        }
+        __syncthreads();
+        if (tid < C) invden[tid] = tid < L ? __fdividef(1.f, r_s[tid] + dsum[tid]) : 0.f;
+        sync_tc();
+
+        // ---- MMA1: [A; Aq] = [K~; Q~] G^^T   (M=128, N=64 tokens, K=128 channels)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t ka = (uint32_t)(ks >> 2), ko = (uint32_t)(ks & 3) * 32u;
+                mma_bf16(T_A, sdesc(sb + L_::KQ + ka * 16384u + ko, 16, 1024), sdesc(sb + L_::G + ka * 8192u + ko, 16, 1024),
+                         ID_M128_N64_KK, ks > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        wait_mma();
+        // rows 0..63: A (strictly lower) -> L (bf16, below the 16x16 block diagonal) and the
+        // diagonal blocks (fp32); rows 64..127: Aq (lower incl. diagonal, bf16); columns / den
+        {
+            const int s0 = cg * 32;
+            float v[32];
+            tmem_ld32(T_A + lane_off + s0, v);
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                const float4 d4 = *reinterpret_cast<const float4 *>(invden + s0 + j);
+                v[j] *= d4.x; v[j + 1] *= d4.y; v[j + 2] *= d4.z; v[j + 3] *= d4.w;
+            }
+            if (row < 64) {
+                const int t = row, b = t >> 4, tr = t & 15;
+                float l[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) l[j] = (s0 + j < 16 * b) ? v[j] : 0.f;
+#pragma unroll
+                for (int chn = 0; chn < 4; ++chn)
+                    *reinterpret_cast<uint4 *>(sm + L_::LB + swz(t, (cg * 4 + chn) * 16)) = pack8(l + chn * 8);
+                if ((b >> 1) == cg) {
+                    const bool hi = b & 1;
+                    float *dst = adg + (b * 16 + tr) * 16;
+#pragma unroll
+                    for (int jj = 0; jj < 16; jj += 4) {
+                        float4 x;
+                        x.x = jj + 0 < tr ? (hi ? v[16 + jj + 0] : v[jj + 0]) : 0.f;
+                        x.y = jj + 1 < tr ? (hi ? v[16 + jj + 1] : v[jj + 1]) : 0.f;
+                        x.z = jj + 2 < tr ? (hi ? v[16 + jj + 2] : v[jj + 2]) : 0.f;
+                        x.w = jj + 3 < tr ? (hi ? v[16 + jj + 3] : v[jj + 3]) : 0.f;
+                        *reinterpret_cast<float4 *>(dst + jj) = x;
+                    }
+                }
+            } else {
+                const int t = row - 64;
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (s0 + j > t) v[j] = 0.f;
+#pragma unroll
+                for (int chn = 0; chn < 4; ++chn)
+                    *reinterpret_cast<uint4 *>(sm + L_::AQ + swz(t, (cg * 4 + chn) * 16)) = pack8(v + chn * 8);
+            }
+        }
+        __syncthreads();
+        // ---- T = (I + A)^{-1}: D = the 16x16 diagonal-block inverses (forward substitution,
+        //      thread = one column of one block), N = D L nilpotent, T = (I - N + N^2 - N^3) D
+        {
+            float x[16];
+            const int b = tid >> 4, j = tid & 15;
+            if (tid < 64) {
+#pragma unroll
+                for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
+#pragma unroll
+                for (int r = 1; r < 16; ++r) {
+                    const float *arow = adg + (b * 16 + r) * 16;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int cc = 0; cc < r; ++cc) acc[cc & 3] = fmaf(arow[cc], x[cc], acc[cc & 3]);
+                    if (r > j) x[r] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
+                }
+            }
+            __syncthreads();
+            if (tid < 64) {
+#pragma unroll
+                for (int r = 0; r < 16; ++r) adg[(b * 16 + r) * 16 + j] = x[r];
+            }
+            __syncthreads();
+            // bf16 D: 64 rows x 8 chunks of 16 B, two chunks per thread
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int r = tid >> 2, cc = (tid & 3) * 2 + half, rb = r >> 4, cb = cc >> 1;
+                float d8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) d8[e] = (cb == rb) ? adg[(rb * 16 + (r & 15)) * 16 + (cc & 1) * 8 + e] : 0.f;
+                *reinterpret_cast<uint4 *>(sm + L_::DB + swz(r, cc * 16)) = pack8(d8);
+            }
+        }
+        sync_tc();
+        mma64(T_A, L_::DB, L_::LB);                           // N = D L
+        { float v[32]; tmem_ld32(T_A + lane_off + cg * 32, v); store64(L_::NB, 0, v); }
+        sync_tc();
+        mma64(T_A + 64, L_::NB, L_::NB);                      // N^2
+        { float v[32]; tmem_ld32(T_A + 64 + lane_off + cg * 32, v); store64(L_::N2B, 0, v); }
+        sync_tc();
+        mma64(T_A + 128, L_::N2B, L_::NB);                    // N^3
+        {   // R = I - N + N^2 - N^3 (over L, consumed)
+            float n1[32], n2[32];
+            tmem_ld32(T_A + lane_off + cg * 32, n1);
+            tmem_ld32(T_A + 64 + lane_off + cg * 32, n2);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) n1[j] = n2[j] - n1[j];
+            tmem_ld32(T_A + 128 + lane_off + cg * 32, n2);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) n1[j] = (cg * 32 + j == m64 ? 1.f : 0.f) + n1[j] - n2[j];
+            store64(L_::LB, 0, n1);
+        }
+        sync_tc();
+        mma64(T_A, L_::LB, L_::DB);                           // T = R D
+        {   // T -> rows 0..63 of Y (zero above the diagonal)
+            float v[32];
+            tmem_ld32(T_A + lane_off + cg * 32, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (cg * 32 + j > m64) v[j] = 0.f;
+            store64(L_::Y, 0, v);
+        }
+        sync_tc();
+        mma64(T_A + 64, L_::AQ, L_::Y);                       // X = Aq T (T as MN-major B)
+        { float v[32]; tmem_ld32(T_A + 64 + lane_off + cg * 32, v); store64(L_::Y, 64, v); }
+        sync_tc();
+
+        // ---- MMA2: [w; X K~] = [T; X] K~   (M=128, N=128 channels, K=64 tokens; K~ MN-major)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(T_A + 128, sdesc(sb + L_::Y + ks * 32u, 16, 1024), sdesc(sb + L_::KQ + ks * 2048u, 16384, 1024),
+                         ID_M128_N128_KM, ks > 0);
+            mma_commit(bar_mma);
+        }
+        wait_mma();
+        // rows 0..63 -> -w ; rows 64..127 -> Q' = Q~ - X K~   (bf16, record layout)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float v[32];
+            tmem_ld32(T_A + 128 + lane_off + cg * 64 + hh * 32, v);
+            const uint32_t atom = (uint32_t)cg * 16384u;
+#pragma unroll
+            for (int chn = 0; chn < 4; ++chn) {
+                const uint32_t boff = atom + swz(row, (hh * 4 + chn) * 16);
+                if (row < 64) {
+                    *reinterpret_cast<uint4 *>(sm + L_::A4 + boff) = pack8(v + chn * 8, -1.f);
+                } else {
+                    const uint4 q4 = *reinterpret_cast<const uint4 *>(sm + L_::KQ + boff);
+                    const uint32_t *qp = reinterpret_cast<const uint32_t *>(&q4);
+                    float w8[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        w8[2 * e] = bf16_lo(qp[e]) - v[chn * 8 + 2 * e];
+                        w8[2 * e + 1] = bf16_hi(qp[e]) - v[chn * 8 + 2 * e + 1];
+                    }
+                    *reinterpret_cast<uint4 *>(sm + L_::A4 + boff) = pack8(w8);
+                }
+            }
+        }
+        sync_tc();
+        // ---- the unit's record (bulk stores; drained before the next unit reuses the buffers)
+        if (tid == 0) {
+            uint8_t *dst = pa.rec + (size_t)u * Rec::BYTES;
+            bulk_store(dst + Rec::A4, sm + L_::A4, 32768);
+            bulk_store(dst + Rec::Y, sm + L_::Y, 16384);
+            bulk_store(dst + Rec::G, sm + L_::G, 16384);
+            bulk_store(dst + Rec::MISC, sm + L_::MISC, 768);
+            bulk_commit();
+        }
+    }
+    if (ctl[1]) raise_error(a.err, ERR_TIMEOUT);
+    if (tid == 0) bulk_wait0();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(T_A, 256);
+}
+
+// ================================================================= state
+template <int DVT>
+__global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_constant__ StateArgs sa)
+{
+    using L_ = StateSmem<DVT>;
+    using namespace tc;
+    constexpr int NC = DVT / 2;   // d_v columns per thread in the epilogues
+    extern __shared__ uint8_t smraw[];
+    const uint32_t raw_u32 = smem_u32(smraw);
+    const uint32_t sb = (raw_u32 + 1023u) & ~1023u;
+    uint8_t *sm = smraw + (sb - raw_u32);
+    uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + L_::CTL);   // [2]
+    uint64_t *bar_mma = bar_full + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar_mma + 1);
+    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+
+    const TokenArgs &a = sa.a;
+    bf16 *__restrict__ out = static_cast<bf16 *>(a.o);
+    const int ntiles = a.dv / DVT;
+    const int tile = blockIdx.x % ntiles;
+    const int chain = blockIdx.x / ntiles;
+    const int s = chain / a.H, h = chain % a.H;
+    int t0, t1;
+    seq_range(a, s, t0, t1);
+    int nch = (t1 - t0 + C - 1) / C;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, cg = warp >> 2;
+    const int H = a.H, dv = a.dv;
+    if (nch > sa.nchunks_max) {   // records exist for nchunks_max chunks only
+        if (tid == 0) raise_error(a.err, ERR_ARG);
+        nch = (int)sa.nchunks_max;
+    }
+
+    if (tid == 0) {
+        mbar_init(bar_full, 1);
+        mbar_init(bar_full + 1, 1);
+        mbar_init(bar_mma, 1);
+        mbar_fence_init();
+        *abort_flag = 0;
+        tma_prefetch_desc(&sa.tv);
+    }
+    if (warp == 0) tmem_alloc(tmem_slot, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t T_S = tmem, T_D4 = tmem + 256;
+    const uint32_t lane_off = ((uint32_t)quad * 32u) << 16;
+    const int row = quad * 32 + lane;
+    const int cb0 = cg * NC;
+
+    auto issue = [&](int c, int st) {   // record and v tile of chunk c into stage st
+        const uint8_t *src = sa.rec + (size_t)((long long)c * sa.nchains + chain) * Rec::BYTES;
+        mbar_expect_tx(bar_full + st, Rec::BYTES + L_::V_BYTES);
+        bulk_load(sm + st * L_::STAGE, src, Rec::BYTES, bar_full + st);
+        for (int b = 0; b < DVT / 64; ++b)
+            tma_load_3d(sm + L_::V0 + st * L_::V_BYTES + b * 8192, &sa.tv, tile * DVT + b * 64, h, t0 + c * C,
+                        bar_full + st);
+    };
+
+    // initial memory tile -> TMEM (lane = key channel) and its bf16 operand copy
+    const size_t sbase = (size_t)chain * DK * dv + (size_t)tile * DVT;
+#pragma unroll
+    for (int p = 0; p < NC / 32; ++p) {
+        float v[32];
+        const int col = cb0 + p * 32;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            float4 x = a.S0 ? *reinterpret_cast<const float4 *>(a.S0 + sbase + (size_t)row * dv + col + j)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[j] = x.x; v[j + 1] = x.y; v[j + 2] = x.z; v[j + 3] = x.w;
+        }
+        tmem_st32(T_S + lane_off + col, v);
+        const uint32_t atom = (uint32_t)(col >> 6) * 16384u;
+#pragma unroll
+        for (int chn = 0; chn < 4; ++chn)
+            *reinterpret_cast<uint4 *>(sm + L_::S + atom + swz(row, (((col & 63) >> 3) + chn) * 16)) = pack8(v + chn * 8);
+    }
+    if (tid == 0 && nch > 0) issue(0, 0);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    constexpr uint32_t ID_M128_NV_KM = idesc_bf16(128, DVT, false, true);
+    constexpr uint32_t ID_M128_NV_MM = idesc_bf16(128, DVT, true, true);
+    uint32_t mma_phase = 0;
+    auto wait_mma = [&]() {
+        if (!mbar_wait(bar_mma, mma_phase)) atomicExch(abort_flag, 1);
+        mma_phase ^= 1u;
+        tc_fence_after();
+    };
+
+    for (int c = 0; c < nch; ++c) {
+        const int st = c & 1;
+        const int c0 = t0 + c * C, L = min(C, t1 - c0);
+        const uint32_t stg = (uint32_t)st * L_::STAGE;
+        const float *invden = reinterpret_cast<const float *>(sm + stg + Rec::MISC);
+        const float *gamc = invden + 64;
+        if (!mbar_wait(bar_full + st, (uint32_t)((c >> 1) & 1))) atomicExch(abort_flag, 1);
+        __syncthreads();
+        if (*abort_flag) break;
+        if (tid == 0 && c + 1 < nch) issue(c + 1, st ^ 1);
+
+        // ---- MMA4: [U; O] = [-w; Q'] S + [T; X] V   (M=128, N=DVT, K=128+64)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t ka = (uint32_t)(ks >> 2), ko = (uint32_t)(ks & 3) * 32u;
+                mma_bf16(T_D4, sdesc(sb + stg + Rec::A4 + ka * 16384u + ko, 16, 1024),
+                         sdesc(sb + L_::S + ks * 2048u, 16384, 1024), ID_M128_NV_KM, ks > 0);
+            }
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(T_D4, sdesc(sb + stg + Rec::Y + ks * 32u, 16, 1024),
+                         sdesc(sb + L_::V0 + st * L_::V_BYTES + ks * 2048u, 8192, 1024), ID_M128_NV_KM, 1);
+            mma_commit(bar_mma);
+        }
+        wait_mma();
+        // rows 0..63 -> U / den (bf16); rows 64..127 -> o (global, tokens of the chunk)
+#pragma unroll
+        for (int p = 0; p < NC / 32; ++p) {
+            float v[32];
+            const int col = cb0 + p * 32;
+            tmem_ld32(T_D4 + lane_off + col, v);
+            if (row < 64) {
+                const float sc = invden[row];
+                const uint32_t blk = (uint32_t)(col >> 6) * 8192u;
+#pragma unroll
+                for (int chn = 0; chn < 4; ++chn)
+                    *reinterpret_cast<uint4 *>(sm + L_::U + blk + swz(row, (((col & 63) >> 3) + chn) * 16)) =
+                        pack8(v + chn * 8, sc);
+            } else if (row - 64 < L) {
+                bf16 *dst = out + ((size_t)(c0 + row - 64) * H + h) * dv + tile * DVT + col;
+#pragma unroll
+                for (int chn = 0; chn < 4; ++chn) *reinterpret_cast<uint4 *>(dst + chn * 8) = pack8(v + chn * 8);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // ---- MMA5: S += G^^T (U / den)   (M=128 channels, N=DVT, K=64 tokens; both MN-major)
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(T_S, sdesc(sb + stg + Rec::G + ks * 2048u, 8192, 1024), sdesc(sb + L_::U + ks * 2048u, 8192, 1024),
+                         ID_M128_NV_MM, 1);
+            mma_commit(bar_mma);
+        }
+        wait_mma();
+        // ---- rows decayed by the chunk's Gam_{L-1}; refresh the bf16 operand copy
+        {
+            const float gC = gamc[row];
+#pragma unroll
+            for (int p = 0; p < NC / 32; ++p) {
+                float v[32];
+                const int col = cb0 + p * 32;
+                tmem_ld32(T_S + lane_off + col, v);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] *= gC;
+                tmem_st32(T_S + lane_off + col, v);
+                const uint32_t atom = (uint32_t)(col >> 6) * 16384u;
+#pragma unroll
+                for (int chn = 0; chn < 4; ++chn)
+                    *reinterpret_cast<uint4 *>(sm + L_::S + atom + swz(row, (((col & 63) >> 3) + chn) * 16)) =
+                        pack8(v + chn * 8);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+
+    if (!*abort_flag) {
+        if (a.S_out) {
+#pragma unroll
+            for (int p = 0; p < NC / 32; ++p) {
+                float v[32];
+                const int col = cb0 + p * 32;
+                tmem_ld32(T_S + lane_off + col, v);
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4 *>(a.S_out + sbase + (size_t)row * dv + col + j) =
+                        make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+            }
+        }
+        // a sequence without tokens had no prep unit: its uncertainty passes through here
+        if (nch == 0 && a.P_out && tile == 0 && tid < DK) a.P_out[(size_t)chain * DK + tid] = a.P0 ? a.P0[(size_t)chain * DK + tid] : 1.f;
+    } else {
+        raise_error(a.err, ERR_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// ================================================================= host side
+size_t two_phase_workspace_bytes(long long nchains, long long nchunks_max) {
+    const long long units = nchains * nchunks_max;
+    const size_t flags = ((size_t)units * 4 + 255) / 256 * 256;
+    return 256 + flags + (size_t)units * 4 * DK * 4 + (size_t)units * Rec::BYTES;
+}
+
+template <int DVT>
+static cudaError_t launch_state(const StateArgs &sa, unsigned grid, cudaStream_t st) {
+    constexpr size_t smem = StateSmem<DVT>::total + 1024;
+    auto kern = chunk_state_kernel<DVT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, SNT, smem, st>>>(sa);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long nchunks_max, void *workspace,
+                                   cudaStream_t st) {
+    const long long nchains = (long long)a.nseq * a.H;
+    if (nchains == 0) return cudaSuccess;
+    const long long units = nchains * nchunks_max;
+    const size_t flags = ((size_t)units * 4 + 255) / 256 * 256;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+
+    PrepArgs pa;
+    pa.a = a;
+    pa.nchunks_max = nchunks_max;
+    pa.nchains = (int)nchains;
+    pa.counter = reinterpret_cast<unsigned *>(ws);
+    pa.flags = reinterpret_cast<int *>(ws + 256);
+    pa.desc = reinterpret_cast<float *>(ws + 256 + flags);
+    pa.rec = ws + 256 + flags + (size_t)units * 4 * DK * 4;
+
+    StateArgs sa;
+    sa.a = a;
+    sa.rec = pa.rec;
+    sa.nchunks_max = nchunks_max;
+    sa.nchains = (int)nchains;
+    if (!make_token_map(&sa.tv, a.v, a.dv, a.H, ntok)) return cudaErrorInvalidValue;
+
+    cudaError_t e = cudaSuccess;
+    if (units > 0) {
+        e = cudaMemsetAsync(ws, 0, 256 + flags, st);   // ticket counter and unit flags
+        if (e != cudaSuccess) return e;
+        constexpr size_t psmem = PrepSmem::total + 1024;
+        e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
+        if (e != cudaSuccess) return e;
+        int dev = 0, sms = 148, per = 1;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, chunk_prep_kernel, PNT, psmem);
+        long long grid = (long long)sms * (per > 0 ? per : 1);
+        if (grid > units) grid = units;
+        chunk_prep_kernel<<<(unsigned)grid, PNT, psmem, st>>>(pa);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    const int dvt = (a.dv == 64 || nchains * (a.dv / 128) < 148) ? 64 : 128;
+    const unsigned sgrid = (unsigned)(nchains * (a.dv / dvt));
+    return dvt == 64 ? launch_state<64>(sa, sgrid, st) : launch_state<128>(sa, sgrid, st);
+}
+
+}  // namespace kdn

@@ -795,7 +795,7 @@ static EncodeTiledFn encode_fn() {
 }
 
 // [ntok, H, d] bf16 viewed as a 3-D tensor {d, H, ntok}; box = 64 channels x 1 head x 64 tokens, 128B swizzle
-static bool make_map(CUtensorMap *m, const void *base, int d, int H, long long ntok) {
+bool make_token_map(CUtensorMap *m, const void *base, int d, int H, long long ntok) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)ntok};
@@ -826,9 +826,9 @@ cudaError_t launch_chunk_tc(const TokenArgs &a, long long ntok, int dvt, cudaStr
     if (a.nseq == 0 || a.H == 0) return cudaSuccess;
     TcParams prm;
     prm.a = a;
-    if (!make_map(&prm.tq, a.q, DK, a.H, ntok) || !make_map(&prm.tk, a.k, DK, a.H, ntok) ||
-        !make_map(&prm.tv, a.v, a.dv, a.H, ntok) || !make_map(&prm.tal, a.alpha, DK, a.H, ntok) ||
-        !make_map(&prm.tsg, a.sigma, DK, a.H, ntok))
+    if (!make_token_map(&prm.tq, a.q, DK, a.H, ntok) || !make_token_map(&prm.tk, a.k, DK, a.H, ntok) ||
+        !make_token_map(&prm.tv, a.v, a.dv, a.H, ntok) || !make_token_map(&prm.tal, a.alpha, DK, a.H, ntok) ||
+        !make_token_map(&prm.tsg, a.sigma, DK, a.H, ntok))
         return cudaErrorInvalidValue;
     if (dvt == 128) return a.iso ? launch_tc<128, true>(prm, st) : launch_tc<128, false>(prm, st);
     if (dvt == 64) return a.iso ? launch_tc<64, true>(prm, st) : launch_tc<64, false>(prm, st);

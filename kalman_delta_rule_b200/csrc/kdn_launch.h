@@ -1,6 +1,7 @@
 // Host-side launchers of the KDN kernels (internal to libkdn.so).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 
@@ -17,6 +18,15 @@ cudaError_t launch_chunk_simt(const TokenArgs &a, bool bf16_in, int C, cudaStrea
 // chunkwise forward on tcgen05 tensor cores (bf16 inputs, d_k = 128, chunk 64)
 bool chunk_tc_supported(int dk, int dv, bool bf16_in, int chunk, long long ntok);
 cudaError_t launch_chunk_tc(const TokenArgs &a, long long ntok, int dvt, cudaStream_t st);
+
+// the same algebra in two launches: a chunk-parallel prep kernel (uncertainty by decoupled
+// look-back, intra-chunk matrices, triangular inverse) writing per-chunk operand records to
+// the workspace, then the chunk-serial state kernel
+size_t two_phase_workspace_bytes(long long nchains, long long nchunks_max);
+cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long nchunks_max, void *workspace,
+                                   cudaStream_t st);
+// [ntok, H, d] bf16 as a TMA tensor map with 64 x 1 x 64 boxes and 128-byte swizzle
+bool make_token_map(CUtensorMap *m, const void *base, int d, int H, long long ntok);
 
 // single-pass Moebius scan of the uncertainty with decoupled look-back (workspace-backed)
 size_t scan_workspace_bytes(long long nchains, long long nchunks_max, int dk);

@@ -12,12 +12,16 @@ pytestmark = pytest.mark.gpu
 TOL_F32, TOL_BF16 = 1e-4, 2e-2
 
 
-def run_forward(kdn, w, chunk, mu=1.0, S0=None, P0=None):
+def run_forward(kdn, w, chunk, mu=1.0, S0=None, P0=None, workspace=None):
+    """Forward through the C ABI; ``workspace`` None allocates one of kdn_workspace_size()
+    bytes (two-launch tensor-core path where it applies), False passes none."""
     import torch
     args = [to_dev(dense_shape(w, getattr(w, n))) for n in ("q", "k", "v", "alpha", "sigma")]
     r = to_dev(dense_shape(w, w.r))
     cu = to_dev(w.cu_seqlens) if w.B == 1 and w.num_seqs > 1 else None
-    o, S, P = kdn.forward(*args, r, cu_seqlens=cu, S0=to_dev(S0), P0=to_dev(P0), mu=mu, chunk=chunk)
+    max_seqlen = int(np.diff(w.cu_seqlens).max()) if cu is not None else 0
+    o, S, P = kdn.forward(*args, r, cu_seqlens=cu, S0=to_dev(S0), P0=to_dev(P0), mu=mu, chunk=chunk,
+                          workspace=workspace, max_seqlen=max_seqlen)
     torch.cuda.synchronize()
     kdn.last_device_error()
     return to_host(o).reshape((-1,) + o.shape[2:]), to_host(S), to_host(P)

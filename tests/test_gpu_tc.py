@@ -1,6 +1,8 @@
-"""GPU parity of the tcgen05 tensor-core chunk kernel (bf16 inputs, d_k = 128,
-chunk 64) against the fp64 oracle: ragged tails, varlen, every d_v tile width,
-initial states, and the full-size workloads on sampled (sequence, head) chains."""
+"""GPU parity of the tcgen05 tensor-core chunk path (bf16 inputs, d_k = 128, chunk 64)
+in both its forms -- two launches (chunk-parallel prep, chunk-serial state; with a
+workspace) and one fused kernel (without) -- against the fp64 oracle: ragged tails,
+varlen, every d_v tile width, initial states, and the full-size workloads on sampled
+(sequence, head) chains."""
 import numpy as np
 import pytest
 
@@ -12,6 +14,9 @@ from tests.test_gpu_recurrent import TOL_BF16, ragged, run_forward
 pytestmark = pytest.mark.gpu
 
 
+FORMS = {"two_phase": None, "fused": False}   # workspace argument of run_forward
+
+
 def path_of(kdn, w, chunk=64):
     p = kdn.kdn_problem_t()
     p.B = w.B or 1
@@ -21,54 +26,61 @@ def path_of(kdn, w, chunk=64):
     return kdn.PATH_NAMES[kdn.kdn_execution_path(p)]
 
 
+@pytest.mark.parametrize("form", sorted(FORMS))
 @pytest.mark.parametrize("dv", [64, 128, 256])
-def test_tc_dense_ragged_tail(kdn, dv):
+def test_tc_dense_ragged_tail(kdn, dv, form):
     w = inputs.dense("tc_dense", 300 + dv, 2, 3, 200, 128, dv, bf16=True)   # 200 = 3 chunks + a tail of 8
-    assert path_of(kdn, w) == "chunk_tcgen05"
+    assert path_of(kdn, w) == "chunk_tcgen05_two_phase"
     ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens)
-    o, S, P = run_forward(kdn, w, chunk=64)
+    o, S, P = run_forward(kdn, w, chunk=64, workspace=FORMS[form])
     assert max_rel_err(o, ref["o"]) <= TOL_BF16
     assert max_rel_err(S, ref["S"]) <= TOL_BF16
     assert max_rel_err(P, ref["P"]) <= TOL_BF16
 
 
+@pytest.mark.parametrize("form", sorted(FORMS))
 @pytest.mark.parametrize("mu", [1.0, 128.0])
-def test_tc_varlen_with_initial_state(kdn, mu):
-    w = ragged(77, [1, 63, 64, 65, 200, 130, 7], 2, 128, 128, True)
+def test_tc_varlen_with_initial_state(kdn, mu, form):
+    """Ragged sequences, an empty one among them, carried S0/P0."""
+    w = ragged(77, [1, 63, 64, 0, 65, 200, 130, 7], 2, 128, 128, True)
     rng = np.random.default_rng(8)
     S0 = (0.1 * rng.standard_normal((w.num_seqs, w.H, 128, 128))).astype(np.float32)
     P0 = rng.uniform(0.3, 2.0, (w.num_seqs, w.H, 128)).astype(np.float32)
     ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens, S0=S0, P0=P0, mu=mu)
-    o, S, P = run_forward(kdn, w, chunk=64, mu=mu, S0=S0, P0=P0)
+    o, S, P = run_forward(kdn, w, chunk=64, mu=mu, S0=S0, P0=P0, workspace=FORMS[form])
     assert max_rel_err(o, ref["o"]) <= TOL_BF16
     assert max_rel_err(S, ref["S"]) <= TOL_BF16
     assert max_rel_err(P, ref["P"]) <= TOL_BF16
+    np.testing.assert_array_equal(S[3], S0[3])     # the empty sequence passes its state through
+    np.testing.assert_array_equal(P[3], P0[3])
 
 
-def sampled_check(kdn, w, picks, tol=TOL_BF16):
-    o, S, P = run_forward(kdn, w, chunk=64)
+def sampled_check(kdn, w, picks, tol=TOL_BF16, forms=("two_phase",)):
     ref = oracle_chains(w, picks)
     cu = w.cu_seqlens
-    for (s, h), rr in ref.items():
-        sl = slice(int(cu[s]), int(cu[s + 1]))
-        assert max_rel_err(o[sl, h], rr["o"]) <= tol, (s, h)
-        assert max_rel_err(S[s, h], rr["S"]) <= tol, (s, h)
-        assert max_rel_err(P[s, h], rr["P"]) <= tol, (s, h)
+    for form in forms:
+        o, S, P = run_forward(kdn, w, chunk=64, workspace=FORMS[form])
+        for (s, h), rr in ref.items():
+            sl = slice(int(cu[s]), int(cu[s + 1]))
+            assert max_rel_err(o[sl, h], rr["o"]) <= tol, (form, s, h)
+            assert max_rel_err(S[s, h], rr["S"]) <= tol, (form, s, h)
+            assert max_rel_err(P[s, h], rr["P"]) <= tol, (form, s, h)
 
 
 def test_prefill_4x4096_full_size_sampled(kdn):
-    """B=4, H=16, T=4096, d=128, bf16, chunk 64 -- the benchmark's launch configuration."""
+    """B=4, H=16, T=4096, d=128, bf16, chunk 64 -- the benchmark's launch configuration
+    (both forms)."""
     w = inputs.prefill_4x4096()
-    assert path_of(kdn, w) == "chunk_tcgen05"
+    assert path_of(kdn, w) == "chunk_tcgen05_two_phase"
     rng = np.random.default_rng(1)
     picks = [(0, 0), (3, 15)] + [(int(a), int(b)) for a, b in zip(rng.integers(0, 4, 6), rng.integers(0, 16, 6))]
-    sampled_check(kdn, w, sorted(set(picks)))
+    sampled_check(kdn, w, sorted(set(picks)), forms=("two_phase", "fused"))
 
 
 def test_long_context_65536_full_size_sampled(kdn):
     """B=1, H=32, T=65536 with repeated-key segments; two whole heads checked."""
     w = inputs.long_context_65536()
-    sampled_check(kdn, w, [(0, 0), (0, 31)])
+    sampled_check(kdn, w, [(0, 0), (0, 31)], forms=("two_phase", "fused"))
 
 
 def test_varlen_262144_full_size_sampled(kdn):
