@@ -47,14 +47,13 @@ struct PrepSmem {
     static constexpr uint32_t W = 49152;               // work region, reused phase by phase:
     static constexpr uint32_t COMP = W;                //   segment composites fp32 [4][128][4]
     static constexpr uint32_t AQ = W;                  //   Aq bf16 64 x 64
-    static constexpr uint32_t DB = W + 8192;           //   D bf16 64 x 64
-    static constexpr uint32_t LB = W + 16384;          //   L, then R = I - N + N^2 - N^3
-    static constexpr uint32_t NB = W + 24576;          //   N
-    static constexpr uint32_t N2B = W + 32768;         //   N^2
-    static constexpr uint32_t ADG = W + 40960;         //   fp32 [4][16][16]: A's diagonal blocks, then D's
+    static constexpr uint32_t DB = W + 8192;           //   D bf16 64 x 64 (the two 32x32 diagonal-block inverses)
+    static constexpr uint32_t LB = W + 16384;          //   L: A's lower-left 32x32 block
+    static constexpr uint32_t NB = W + 24576;          //   I - N, N = D L
+    static constexpr uint32_t ADG = W + 32768;         //   fp32 [2][32][32]: A's diagonal blocks, then D's
     static constexpr uint32_t A4 = W;                  //   [-w; Q'] (record part), once the inverse is done
-    static constexpr uint32_t Y = W + 45056;           //   [T; X] (record part)
-    static constexpr uint32_t MISC = W + 61440;        // 1/den [64], Gam_{L-1} [128] (record tail)
+    static constexpr uint32_t Y = W + 40960;           //   [T; X] (record part)
+    static constexpr uint32_t MISC = W + 57344;        // 1/den [64], Gam_{L-1} [128] (record tail)
     static constexpr uint32_t RS = MISC + 768;         // r [64]
     static constexpr uint32_t MUR = RS + 256;          // mu / r [64]
     static constexpr uint32_t PST = MUR + 256;         // uncertainty at the chunk start [128]
@@ -62,7 +61,7 @@ struct PrepSmem {
     static constexpr uint32_t CTL = DSUM + 256;        // mbarrier, ticket, TMEM slot, look-back flag, abort
     static constexpr uint32_t total = CTL + 64;
     static_assert(COMP + 4 * 128 * 16 <= DB, "composites overlap D");
-    static_assert(ADG + 4096 <= Y && Y + 16384 <= MISC, "work region");
+    static_assert(ADG + 8192 <= Y && Y + 16384 <= MISC && A4 + 32768 <= Y, "work region");
 };
 
 template <int DVT>
@@ -81,7 +80,7 @@ struct PrepArgs {
     long long nchunks_max;
     int nchains;
     unsigned *counter;
-    int *flags;
+    int *flags;       // per unit, one per 32 key channels
     float *desc;      // per unit [4][128]: aggregate map (m00, m01, m10) and end-of-chunk P
     uint8_t *rec;     // per unit Rec::BYTES
 };
@@ -299,100 +298,125 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
         }
         __syncthreads();
 
-        // ---- chunk aggregate (thread = channel), publication and decoupled look-back
-        float g00 = 1.f, g01 = 0.f, g10 = 0.f, g11 = 1.f;
-        float *desc = pa.desc + (size_t)u * 4 * DK;
-        if (tid < DK) {
+        // ---- warps 0-3 (thread = key channel): chunk aggregate, its publication and the
+        //      decoupled look-back, each warp for its 32 channels with its own flag; warps 4-7
+        //      meanwhile form K~ = k Gam and Q~ = q Gam, which do not depend on the uncertainty.
+        //      Gam: inclusive decay from the chunk start.
+        const uint32_t atom16 = (uint32_t)(ch >> 6) * 16384u, atom8 = (uint32_t)(ch >> 6) * 8192u;
+        const uint32_t bch = (uint32_t)(ch & 63) * 2u;
+        auto gamma_start = [&](float &ga, float &gb) {
+            ga = 1.f;
+            gb = 1.f;
+            for (int q2 = 0; q2 < sgi; ++q2) {
+                ga *= comp[(q2 * 128 + ch) * 4 + 3];
+                gb *= comp[(q2 * 128 + ch + 1) * 4 + 3];
+            }
+        };
+        auto form_kq = [&]() {
+            float gama, gamb;
+            gamma_start(gama, gamb);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int t = tb + j;
+                uint32_t kq = 0u, qq = 0u;
+                if (t < L) {
+                    gama *= bf16_lo(aw[j]);
+                    gamb *= bf16_hi(aw[j]);
+                    kq = pack_bf16x2(bf16_lo(kw[j]) * gama, bf16_hi(kw[j]) * gamb);
+                    qq = pack_bf16x2(bf16_lo(qw[j]) * gama, bf16_hi(qw[j]) * gamb);
+                }
+                *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(t, bch)) = kq;
+                *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(64 + t, bch)) = qq;
+            }
+            if (tb < L && tb + 16 >= L) {   // this segment holds the chunk's last token
+                gamc[ch] = gama;
+                gamc[ch + 1] = gamb;
+                if (!(gama >= 1e-30f) || !(gamb >= 1e-30f)) raise_error(a.err, ERR_RANGE);
+            }
+        };
+        if (warp < 4) {
+            const int cc = tid;   // key channel
+            float *desc = pa.desc + (size_t)u * 4 * DK;
+            float g00 = 1.f, g01 = 0.f, g10 = 0.f, g11 = 1.f;
 #pragma unroll
             for (int q2 = 0; q2 < 4; ++q2) {
-                const float4 cm = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + tid) * 4);
+                const float4 cm = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + cc) * 4);
                 const float n00 = fmaf(cm.x, g00, cm.y * g10), n01 = fmaf(cm.x, g01, cm.y * g11);
                 const float n10 = fmaf(cm.z, g00, g10), n11 = fmaf(cm.z, g01, g11);
                 const float sc = 1.f / n11;
                 g00 = n00 * sc; g01 = n01 * sc; g10 = n10 * sc; g11 = 1.f;
             }
-            if (c > 0) {
-                __stcg(desc + 0 * DK + tid, g00);
-                __stcg(desc + 1 * DK + tid, g01);
-                __stcg(desc + 2 * DK + tid, g10);
-            }
-        }
-        if (c > 0) {
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) atomicExch(pa.flags + u, FLAG_AGG);
-        }
-        if (c == 0) {
-            if (tid < DK) pst[tid] = a.P0 ? a.P0[(size_t)chain * DK + tid] : 1.f;
-        } else {
-            float r00 = 1.f, r01 = 0.f, r10 = 0.f, r11 = 1.f;   // composite of the chunks walked over
-            int j = c - 1;
-            for (;;) {
-                const long long uj = (long long)j * pa.nchains + chain;
-                if (tid == 0) {
-                    volatile int *fp = pa.flags + uj;
-                    int f = *fp;
-                    const long long ts = clock64();
-                    while (f == FLAG_NONE) {
-                        if (clock64() - ts > 2000000000ll) break;
-                        __nanosleep(64);
-                        f = *fp;
-                    }
-                    if (f == FLAG_NONE) { raise_error(a.err, ERR_TIMEOUT); f = -1; }
-                    ctl[0] = f;
-                }
-                __syncthreads();
-                const int f = ctl[0];
+            if (c > 0) {   // publish the aggregate: one flag per warp's 32 channels
+                __stcg(desc + 0 * DK + cc, g00);
+                __stcg(desc + 1 * DK + cc, g01);
+                __stcg(desc + 2 * DK + cc, g10);
                 __threadfence();
-                const float *dj = pa.desc + (size_t)uj * 4 * DK;
-                if (f == FLAG_INCL || f < 0) {
-                    if (tid < DK) {
-                        const float pe = f < 0 ? 1.f : __ldcg(dj + 3 * DK + tid);
-                        pst[tid] = mob(r00, r01, r10, r11, pe);
-                    }
-                    __syncthreads();
-                    break;
-                }
-                if (tid < DK) {   // R <- R * A_j (A_j acts first)
-                    const float m00 = __ldcg(dj + tid), m01 = __ldcg(dj + DK + tid), m10 = __ldcg(dj + 2 * DK + tid);
-                    const float n00 = fmaf(r00, m00, r01 * m10), n01 = fmaf(r00, m01, r01);
-                    const float n10 = fmaf(r10, m00, r11 * m10), n11 = fmaf(r10, m01, r11);
-                    const float sc = 1.f / n11;
-                    r00 = n00 * sc; r01 = n01 * sc; r10 = n10 * sc; r11 = 1.f;
-                }
-                __syncthreads();
-                --j;
+                __syncwarp();
+                if (lane == 0) atomicExch(pa.flags + u * 4 + warp, FLAG_AGG);
             }
+            float p0;
+            if (c == 0) {
+                p0 = a.P0 ? a.P0[(size_t)chain * DK + cc] : 1.f;
+            } else {
+                float r00 = 1.f, r01 = 0.f, r10 = 0.f;   // composite of the chunks walked over ((1,1) kept at 1)
+                for (int j = c - 1;; --j) {
+                    const long long uj = (long long)j * pa.nchains + chain;
+                    int f = 0;
+                    if (lane == 0) {
+                        volatile int *fp = pa.flags + uj * 4 + warp;
+                        f = *fp;
+                        const long long ts = clock64();
+                        while (f == FLAG_NONE) {
+                            // give up after ~1 s, or at once when another wait already gave up
+                            if (clock64() - ts > 2000000000ll || (a.err && (*(volatile unsigned *)a.err & ERR_TIMEOUT))) break;
+                            __nanosleep(32);
+                            f = *fp;
+                        }
+                        if (f == FLAG_NONE) { raise_error(a.err, ERR_TIMEOUT); f = -1; }
+                    }
+                    f = __shfl_sync(0xffffffffu, f, 0);
+                    __threadfence();
+                    const float *dj = pa.desc + (size_t)uj * 4 * DK + cc;
+                    if (f == FLAG_INCL || f < 0) {
+                        p0 = mob(r00, r01, r10, 1.f, f < 0 ? 1.f : __ldcg(dj + 3 * DK));
+                        break;
+                    }
+                    const float m00 = __ldcg(dj), m01 = __ldcg(dj + DK), m10 = __ldcg(dj + 2 * DK);
+                    const float n00 = fmaf(r00, m00, r01 * m10), n01 = fmaf(r00, m01, r01);
+                    const float n10 = fmaf(r10, m00, m10), n11 = fmaf(r10, m01, 1.f);
+                    const float sc = 1.f / n11;
+                    r00 = n00 * sc; r01 = n01 * sc; r10 = n10 * sc;
+                }
+            }
+            pst[cc] = p0;
+            const float pe = mob(g00, g01, g10, 1.f, p0);
+            __stcg(desc + 3 * DK + cc, pe);
+            if (c == nch - 1 && a.P_out) a.P_out[(size_t)chain * DK + cc] = pe;
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) atomicExch(pa.flags + u * 4 + warp, FLAG_INCL);
+        } else {
+            form_kq();
         }
         __syncthreads();
-        if (tid < DK) {
-            const float pe = mob(g00, g01, g10, g11, pst[tid]);
-            __stcg(desc + 3 * DK + tid, pe);
-            if (c == nch - 1 && a.P_out) a.P_out[(size_t)chain * DK + tid] = pe;
-        }
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) atomicExch(pa.flags + u, FLAG_INCL);
+        if (warp < 4) form_kq();
 
-        // ---- re-expansion fused with the chunk operands: P^- per token, Gam (inclusive decay
-        //      from the chunk start), K~ = k Gam, Q~ = q Gam, G^ = P^- k / Gam, den partial sums
+        // ---- re-expansion: P^- per token (from the chunk-start uncertainty through the earlier
+        //      segments' composites), G^ = P^- k / Gam and the den partial sums
         {
-            float Pa = pst[ch], Pb = pst[ch + 1], gama = 1.f, gamb = 1.f;
+            float Pa = pst[ch], Pb = pst[ch + 1], gama, gamb;
+            gamma_start(gama, gamb);
             for (int q2 = 0; q2 < sgi; ++q2) {
                 const float4 ca = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch) * 4);
                 const float4 cb = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch + 1) * 4);
                 Pa = mob(ca.x, ca.y, ca.z, 1.f, Pa);
                 Pb = mob(cb.x, cb.y, cb.z, 1.f, Pb);
-                gama *= ca.w;
-                gamb *= cb.w;
             }
-            const uint32_t atom16 = (uint32_t)(ch >> 6) * 16384u, atom8 = (uint32_t)(ch >> 6) * 8192u;
-            const uint32_t bch = (uint32_t)(ch & 63) * 2u;
             float xs[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const int t = tb + j;
-                uint32_t kq = 0u, qq = 0u, gg = 0u;
+                uint32_t gg = 0u;
                 xs[j] = 0.f;
                 if (t < L) {
                     const float ala = bf16_lo(aw[j]), alb = bf16_hi(aw[j]);
@@ -404,19 +428,10 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
                     gama *= ala;
                     gamb *= alb;
                     const float pka = pma * ka, pkb = pmb * kb;
-                    kq = pack_bf16x2(ka * gama, kb * gamb);
-                    qq = pack_bf16x2(bf16_lo(qw[j]) * gama, bf16_hi(qw[j]) * gamb);
                     gg = pack_bf16x2(__fdividef(pka, gama), __fdividef(pkb, gamb));
                     xs[j] = fmaf(pka, ka, pkb * kb);
                 }
-                *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(t, bch)) = kq;
-                *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(64 + t, bch)) = qq;
                 *reinterpret_cast<uint32_t *>(sm + L_::G + atom8 + swz(t, bch)) = gg;
-            }
-            if (tb < L && tb + 16 >= L) {   // this segment holds the chunk's last token
-                gamc[ch] = gama;
-                gamc[ch + 1] = gamb;
-                if (!(gama >= 1e-30f) || !(gamb >= 1e-30f)) raise_error(a.err, ERR_RANGE);
             }
             int which;
             const float tot = warp_reduce16(xs, lane, which);
@@ -438,7 +453,7 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
             mma_commit(bar_mma);
         }
         wait_mma();
-        // rows 0..63: A (strictly lower) -> L (bf16, below the 16x16 block diagonal) and the
+        // rows 0..63: A (strictly lower) -> its lower-left 32x32 block L (bf16) and its two
         // diagonal blocks (fp32); rows 64..127: Aq (lower incl. diagonal, bf16); columns / den
         {
             const int s0 = cg * 32;
@@ -450,25 +465,20 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
                 v[j] *= d4.x; v[j + 1] *= d4.y; v[j + 2] *= d4.z; v[j + 3] *= d4.w;
             }
             if (row < 64) {
-                const int t = row, b = t >> 4, tr = t & 15;
-                float l[32];
+                const int t = row, b = t >> 5, tr = t & 31;
+                const bool lower_left = (b == 1 && cg == 0);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) l[j] = (s0 + j < 16 * b) ? v[j] : 0.f;
+                for (int chn = 0; chn < 4; ++chn) {
+                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4 *>(sm + L_::LB + swz(t, (cg * 4 + chn) * 16)) = lower_left ? pack8(v + chn * 8) : z;
+                }
+                if (b == cg) {
+                    float *dst = adg + (b * 32 + tr) * 32;
 #pragma unroll
-                for (int chn = 0; chn < 4; ++chn)
-                    *reinterpret_cast<uint4 *>(sm + L_::LB + swz(t, (cg * 4 + chn) * 16)) = pack8(l + chn * 8);
-                if ((b >> 1) == cg) {
-                    const bool hi = b & 1;
-                    float *dst = adg + (b * 16 + tr) * 16;
-#pragma unroll
-                    for (int jj = 0; jj < 16; jj += 4) {
-                        float4 x;
-                        x.x = jj + 0 < tr ? (hi ? v[16 + jj + 0] : v[jj + 0]) : 0.f;
-                        x.y = jj + 1 < tr ? (hi ? v[16 + jj + 1] : v[jj + 1]) : 0.f;
-                        x.z = jj + 2 < tr ? (hi ? v[16 + jj + 2] : v[jj + 2]) : 0.f;
-                        x.w = jj + 3 < tr ? (hi ? v[16 + jj + 3] : v[jj + 3]) : 0.f;
-                        *reinterpret_cast<float4 *>(dst + jj) = x;
-                    }
+                    for (int jj = 0; jj < 32; jj += 4)
+                        *reinterpret_cast<float4 *>(dst + jj) =
+                            make_float4(jj < tr ? v[jj] : 0.f, jj + 1 < tr ? v[jj + 1] : 0.f, jj + 2 < tr ? v[jj + 2] : 0.f,
+                                        jj + 3 < tr ? v[jj + 3] : 0.f);
                 }
             } else {
                 const int t = row - 64;
@@ -481,71 +491,74 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
             }
         }
         __syncthreads();
-        // ---- T = (I + A)^{-1}: D = the 16x16 diagonal-block inverses (forward substitution,
-        //      thread = one column of one block), N = D L nilpotent, T = (I - N + N^2 - N^3) D
+        // ---- T = (I + A)^{-1}: D = the two 32x32 diagonal-block inverses (forward substitution,
+        //      thread = one column of one block), N = D L (N^2 = 0), T = (I - N) D
         {
-            float x[16];
-            const int b = tid >> 4, j = tid & 15;
+            float x[32];
+            const int b = tid >> 5, j = tid & 31;
             if (tid < 64) {
 #pragma unroll
-                for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
+                for (int r = 0; r < 32; ++r) x[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
-                for (int r = 1; r < 16; ++r) {
-                    const float *arow = adg + (b * 16 + r) * 16;
+                for (int r = 1; r < 32; ++r) {   // A's row r is zero from column r on
+                    const float4 *arow = reinterpret_cast<const float4 *>(adg + (b * 32 + r) * 32);
                     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int cc = 0; cc < r; ++cc) acc[cc & 3] = fmaf(arow[cc], x[cc], acc[cc & 3]);
+                    for (int q4 = 0; q4 < (r + 3) / 4; ++q4) {
+                        const float4 a4 = arow[q4];
+                        acc[0] = fmaf(a4.x, x[4 * q4], acc[0]);
+                        acc[1] = fmaf(a4.y, x[4 * q4 + 1], acc[1]);
+                        acc[2] = fmaf(a4.z, x[4 * q4 + 2], acc[2]);
+                        acc[3] = fmaf(a4.w, x[4 * q4 + 3], acc[3]);
+                    }
                     if (r > j) x[r] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
                 }
             }
             __syncthreads();
             if (tid < 64) {
 #pragma unroll
-                for (int r = 0; r < 16; ++r) adg[(b * 16 + r) * 16 + j] = x[r];
+                for (int r = 0; r < 32; ++r) adg[(b * 32 + r) * 32 + j] = x[r];
             }
             __syncthreads();
             // bf16 D: 64 rows x 8 chunks of 16 B, two chunks per thread
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                const int r = tid >> 2, cc = (tid & 3) * 2 + half, rb = r >> 4, cb = cc >> 1;
+                const int r = tid >> 2, cc = (tid & 3) * 2 + half, rb = r >> 5, cb = cc >> 2;
                 float d8[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) d8[e] = (cb == rb) ? adg[(rb * 16 + (r & 15)) * 16 + (cc & 1) * 8 + e] : 0.f;
+                for (int e = 0; e < 8; ++e) d8[e] = (cb == rb) ? adg[(rb * 32 + (r & 31)) * 32 + (cc & 3) * 8 + e] : 0.f;
                 *reinterpret_cast<uint4 *>(sm + L_::DB + swz(r, cc * 16)) = pack8(d8);
             }
         }
         sync_tc();
         mma64(T_A, L_::DB, L_::LB);                           // N = D L
-        { float v[32]; tmem_ld32(T_A + lane_off + cg * 32, v); store64(L_::NB, 0, v); }
-        sync_tc();
-        mma64(T_A + 64, L_::NB, L_::NB);                      // N^2
-        { float v[32]; tmem_ld32(T_A + 64 + lane_off + cg * 32, v); store64(L_::N2B, 0, v); }
-        sync_tc();
-        mma64(T_A + 128, L_::N2B, L_::NB);                    // N^3
-        {   // R = I - N + N^2 - N^3 (over L, consumed)
-            float n1[32], n2[32];
-            tmem_ld32(T_A + lane_off + cg * 32, n1);
-            tmem_ld32(T_A + 64 + lane_off + cg * 32, n2);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) n1[j] = n2[j] - n1[j];
-            tmem_ld32(T_A + 128 + lane_off + cg * 32, n2);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) n1[j] = (cg * 32 + j == m64 ? 1.f : 0.f) + n1[j] - n2[j];
-            store64(L_::LB, 0, n1);
-        }
-        sync_tc();
-        mma64(T_A, L_::LB, L_::DB);                           // T = R D
-        {   // T -> rows 0..63 of Y (zero above the diagonal)
+        {   // I - N (bf16; N^2 = 0, so (I + D L)^{-1} = I - N)
             float v[32];
             tmem_ld32(T_A + lane_off + cg * 32, v);
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if (cg * 32 + j > m64) v[j] = 0.f;
+            for (int j = 0; j < 32; ++j) v[j] = (cg * 32 + j == m64 ? 1.f : 0.f) - v[j];
+            store64(L_::NB, 0, v);
+        }
+        sync_tc();
+        mma64(T_A + 64, L_::NB, L_::DB);                      // T = (I - N) D
+        {   // T -> rows 0..63 of Y
+            float v[32];
+            tmem_ld32(T_A + 64 + lane_off + cg * 32, v);
             store64(L_::Y, 0, v);
         }
         sync_tc();
-        mma64(T_A + 64, L_::AQ, L_::Y);                       // X = Aq T (T as MN-major B)
-        { float v[32]; tmem_ld32(T_A + 64 + lane_off + cg * 32, v); store64(L_::Y, 64, v); }
+        mma64(T_A + 128, L_::AQ, L_::Y);                      // X = Aq T (T as MN-major B)
+        {   // X -> rows 64..127 of Y, 16 columns at a time
+            for (int hh = 0; hh < 2; ++hh) {
+                float v[16];
+                tmem_ld16(T_A + 128 + lane_off + cg * 32 + hh * 16, v);
+                if (lane < 16) {
+#pragma unroll
+                    for (int chn = 0; chn < 2; ++chn)
+                        *reinterpret_cast<uint4 *>(sm + L_::Y + swz(64 + m64, (cg * 4 + hh * 2 + chn) * 16)) = pack8(v + chn * 8);
+                }
+            }
+        }
         sync_tc();
 
         // ---- MMA2: [w; X K~] = [T; X] K~   (M=128, N=128 channels, K=64 tokens; K~ MN-major)
@@ -558,15 +571,15 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
             mma_commit(bar_mma);
         }
         wait_mma();
-        // rows 0..63 -> -w ; rows 64..127 -> Q' = Q~ - X K~   (bf16, record layout)
+        // rows 0..63 -> -w ; rows 64..127 -> Q' = Q~ - X K~   (bf16, record layout), 16 columns at a time
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            float v[32];
-            tmem_ld32(T_A + 128 + lane_off + cg * 64 + hh * 32, v);
+        for (int hh = 0; hh < 4; ++hh) {
+            float v[16];
+            tmem_ld16(T_A + 128 + lane_off + cg * 64 + hh * 16, v);
             const uint32_t atom = (uint32_t)cg * 16384u;
 #pragma unroll
-            for (int chn = 0; chn < 4; ++chn) {
-                const uint32_t boff = atom + swz(row, (hh * 4 + chn) * 16);
+            for (int chn = 0; chn < 2; ++chn) {
+                const uint32_t boff = atom + swz(row, (hh * 2 + chn) * 16);
                 if (row < 64) {
                     *reinterpret_cast<uint4 *>(sm + L_::A4 + boff) = pack8(v + chn * 8, -1.f);
                 } else {
@@ -802,7 +815,7 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
 // ================================================================= host side
 size_t two_phase_workspace_bytes(long long nchains, long long nchunks_max) {
     const long long units = nchains * nchunks_max;
-    const size_t flags = ((size_t)units * 4 + 255) / 256 * 256;
+    const size_t flags = ((size_t)units * 16 + 255) / 256 * 256;
     return 256 + flags + (size_t)units * 4 * DK * 4 + (size_t)units * Rec::BYTES;
 }
 
@@ -821,7 +834,7 @@ cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long
     const long long nchains = (long long)a.nseq * a.H;
     if (nchains == 0) return cudaSuccess;
     const long long units = nchains * nchunks_max;
-    const size_t flags = ((size_t)units * 4 + 255) / 256 * 256;
+    const size_t flags = ((size_t)units * 16 + 255) / 256 * 256;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
 
     PrepArgs pa;
@@ -847,11 +860,16 @@ cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long
         constexpr size_t psmem = PrepSmem::total + 1024;
         e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
         if (e != cudaSuccess) return e;
+        // all of the unified L1 / shared array as shared memory, so that two CTAs fit on an SM
+        e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (e != cudaSuccess) return e;
         int dev = 0, sms = 148, per = 1;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, chunk_prep_kernel, PNT, psmem);
-        long long grid = (long long)sms * (per > 0 ? per : 1);
+        // two CTAs fit on an SM (registers and shared memory); the occupancy query can report
+        // fewer.  Extra CTAs are harmless: units go out by ticket to resident CTAs only.
+        long long grid = (long long)sms * (per > 2 ? per : 2);
         if (grid > units) grid = units;
         chunk_prep_kernel<<<(unsigned)grid, PNT, psmem, st>>>(pa);
         e = cudaGetLastError();

@@ -168,7 +168,8 @@ __global__ void __launch_bounds__(SNT) gain_scan_kernel(ScanArgs a)
                     int f = *fp;
                     const long long tstart = clock64();
                     while (f == FLAG_NONE) {
-                        if (clock64() - tstart > 2000000000ll) break;
+                        // give up after ~1 s, or at once when another wait already gave up
+                        if (clock64() - tstart > 2000000000ll || (a.err && (*(volatile unsigned *)a.err & ERR_TIMEOUT))) break;
                         __nanosleep(64);
                         f = *fp;
                     }
