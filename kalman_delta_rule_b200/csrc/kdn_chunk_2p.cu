@@ -30,7 +30,7 @@ namespace kdn {
 
 namespace {
 constexpr int C = 64, DK = 128, PNT = 256, SNT = 256;
-enum : int { FLAG_NONE = 0, FLAG_AGG = 1, FLAG_INCL = 2 };
+constexpr int ADS = 36;   // padded fp32 row stride of the diagonal blocks (conflict-free row-wise float4 access)
 
 // one unit's record; each part in the state kernel's operand layout
 struct Rec {
@@ -50,10 +50,10 @@ struct PrepSmem {
     static constexpr uint32_t DB = W + 8192;           //   D bf16 64 x 64 (the two 32x32 diagonal-block inverses)
     static constexpr uint32_t LB = W + 16384;          //   L: A's lower-left 32x32 block
     static constexpr uint32_t NB = W + 24576;          //   I - N, N = D L
-    static constexpr uint32_t ADG = W + 32768;         //   fp32 [2][32][32]: A's diagonal blocks, then D's
+    static constexpr uint32_t ADG = W + 32768;         //   fp32 [2][32][ADS]: A's diagonal blocks, then D's
     static constexpr uint32_t A4 = W;                  //   [-w; Q'] (record part), once the inverse is done
-    static constexpr uint32_t Y = W + 40960;           //   [T; X] (record part)
-    static constexpr uint32_t MISC = W + 57344;        // 1/den [64], Gam_{L-1} [128] (record tail)
+    static constexpr uint32_t Y = W + 43008;           //   [T; X] (record part)
+    static constexpr uint32_t MISC = W + 59392;        // 1/den [64], Gam_{L-1} [128] (record tail)
     static constexpr uint32_t RS = MISC + 768;         // r [64]
     static constexpr uint32_t MUR = RS + 256;          // mu / r [64]
     static constexpr uint32_t PST = MUR + 256;         // uncertainty at the chunk start [128]
@@ -61,7 +61,7 @@ struct PrepSmem {
     static constexpr uint32_t CTL = DSUM + 256;        // mbarrier, ticket, TMEM slot, look-back flag, abort
     static constexpr uint32_t total = CTL + 64;
     static_assert(COMP + 4 * 128 * 16 <= DB, "composites overlap D");
-    static_assert(ADG + 8192 <= Y && Y + 16384 <= MISC && A4 + 32768 <= Y, "work region");
+    static_assert(ADG + 64 * ADS * 4 <= Y && Y + 16384 <= MISC && A4 + 32768 <= Y, "work region");
 };
 
 template <int DVT>
@@ -80,8 +80,7 @@ struct PrepArgs {
     long long nchunks_max;
     int nchains;
     unsigned *counter;
-    int *flags;       // per unit, one per 32 key channels
-    float *desc;      // per unit [4][128]: aggregate map (m00, m01, m10) and end-of-chunk P
+    unsigned long long *desc;   // per unit [4][128] tagged words: aggregate map (m00, m01, m10), end-of-chunk P
     uint8_t *rec;     // per unit Rec::BYTES
 };
 
@@ -107,6 +106,23 @@ __device__ __forceinline__ uint4 pack8(const float *v, float sc = 1.f) {
 }
 
 __device__ __forceinline__ uint32_t ldg_u32(const bf16 *p) { return __ldg(reinterpret_cast<const unsigned *>(p)); }
+
+// Look-back descriptors are 64-bit words (value, tag): each word carries its own status, so a
+// reader that sees a tag also sees that word's value, with no fence between writer and flag.
+enum : unsigned { TAG_NONE = 0, TAG_AGG = 1, TAG_INCL = 2 };
+__device__ __forceinline__ unsigned long long tagged(float x, unsigned tag) {
+    return ((unsigned long long)tag << 32) | __float_as_uint(x);
+}
+__device__ __forceinline__ unsigned tag_of(unsigned long long w) { return (unsigned)(w >> 32); }
+__device__ __forceinline__ float value_of(unsigned long long w) { return __uint_as_float((unsigned)w); }
+__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
 
 // Sums 16 per-lane values over the 32 lanes of a warp with 16 shuffles (each step exchanges
 // half of the remaining values).  Lanes 2m and 2m+1 end with the total of value `which`.
@@ -299,9 +315,7 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
         __syncthreads();
 
         // ---- warps 0-3 (thread = key channel): chunk aggregate, its publication and the
-        //      decoupled look-back, each warp for its 32 channels with its own flag; warps 4-7
-        //      meanwhile form K~ = k Gam and Q~ = q Gam, which do not depend on the uncertainty.
-        //      Gam: inclusive decay from the chunk start.
+        //      decoupled look-back, every channel on its own.
         const uint32_t atom16 = (uint32_t)(ch >> 6) * 16384u, atom8 = (uint32_t)(ch >> 6) * 8192u;
         const uint32_t bch = (uint32_t)(ch & 63) * 2u;
         auto gamma_start = [&](float &ga, float &gb) {
@@ -312,31 +326,9 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
                 gb *= comp[(q2 * 128 + ch + 1) * 4 + 3];
             }
         };
-        auto form_kq = [&]() {
-            float gama, gamb;
-            gamma_start(gama, gamb);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int t = tb + j;
-                uint32_t kq = 0u, qq = 0u;
-                if (t < L) {
-                    gama *= bf16_lo(aw[j]);
-                    gamb *= bf16_hi(aw[j]);
-                    kq = pack_bf16x2(bf16_lo(kw[j]) * gama, bf16_hi(kw[j]) * gamb);
-                    qq = pack_bf16x2(bf16_lo(qw[j]) * gama, bf16_hi(qw[j]) * gamb);
-                }
-                *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(t, bch)) = kq;
-                *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(64 + t, bch)) = qq;
-            }
-            if (tb < L && tb + 16 >= L) {   // this segment holds the chunk's last token
-                gamc[ch] = gama;
-                gamc[ch + 1] = gamb;
-                if (!(gama >= 1e-30f) || !(gamb >= 1e-30f)) raise_error(a.err, ERR_RANGE);
-            }
-        };
         if (warp < 4) {
             const int cc = tid;   // key channel
-            float *desc = pa.desc + (size_t)u * 4 * DK;
+            unsigned long long *desc = pa.desc + (size_t)u * 4 * DK + cc;
             float g00 = 1.f, g01 = 0.f, g10 = 0.f, g11 = 1.f;
 #pragma unroll
             for (int q2 = 0; q2 < 4; ++q2) {
@@ -346,42 +338,44 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
                 const float sc = 1.f / n11;
                 g00 = n00 * sc; g01 = n01 * sc; g10 = n10 * sc; g11 = 1.f;
             }
-            if (c > 0) {   // publish the aggregate: one flag per warp's 32 channels
-                __stcg(desc + 0 * DK + cc, g00);
-                __stcg(desc + 1 * DK + cc, g01);
-                __stcg(desc + 2 * DK + cc, g10);
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) atomicExch(pa.flags + u * 4 + warp, FLAG_AGG);
+            if (c > 0) {   // publish the aggregate
+                st_relaxed(desc + 0 * DK, tagged(g00, TAG_AGG));
+                st_relaxed(desc + 1 * DK, tagged(g01, TAG_AGG));
+                st_relaxed(desc + 2 * DK, tagged(g10, TAG_AGG));
             }
             float p0;
             if (c == 0) {
                 p0 = a.P0 ? a.P0[(size_t)chain * DK + cc] : 1.f;
-            } else {
+            } else {   // walk back: compose aggregates until an end-of-chunk uncertainty
                 float r00 = 1.f, r01 = 0.f, r10 = 0.f;   // composite of the chunks walked over ((1,1) kept at 1)
+                bool timed_out = false;
                 for (int j = c - 1;; --j) {
-                    const long long uj = (long long)j * pa.nchains + chain;
-                    int f = 0;
-                    if (lane == 0) {
-                        volatile int *fp = pa.flags + uj * 4 + warp;
-                        f = *fp;
-                        const long long ts = clock64();
-                        while (f == FLAG_NONE) {
-                            // give up after ~1 s, or at once when another wait already gave up
-                            if (clock64() - ts > 2000000000ll || (a.err && (*(volatile unsigned *)a.err & ERR_TIMEOUT))) break;
-                            __nanosleep(32);
-                            f = *fp;
+                    const unsigned long long *dj = pa.desc + ((size_t)j * pa.nchains + chain) * 4 * DK + cc;
+                    unsigned long long w0 = 0ull, w1 = 0ull, w2 = 0ull, w3 = ld_relaxed(dj + 3 * DK);
+                    const long long ts = clock64();
+                    while (tag_of(w3) != TAG_INCL) {
+                        w0 = ld_relaxed(dj);
+                        w1 = ld_relaxed(dj + DK);
+                        w2 = ld_relaxed(dj + 2 * DK);
+                        if (tag_of(w0) == TAG_AGG && tag_of(w1) == TAG_AGG && tag_of(w2) == TAG_AGG) break;
+                        // give up after ~1 s, or at once when another wait already gave up
+                        if (clock64() - ts > 2000000000ll || (a.err && (*(volatile unsigned *)a.err & ERR_TIMEOUT))) {
+                            timed_out = true;
+                            break;
                         }
-                        if (f == FLAG_NONE) { raise_error(a.err, ERR_TIMEOUT); f = -1; }
+                        __nanosleep(32);
+                        w3 = ld_relaxed(dj + 3 * DK);
                     }
-                    f = __shfl_sync(0xffffffffu, f, 0);
-                    __threadfence();
-                    const float *dj = pa.desc + (size_t)uj * 4 * DK + cc;
-                    if (f == FLAG_INCL || f < 0) {
-                        p0 = mob(r00, r01, r10, 1.f, f < 0 ? 1.f : __ldcg(dj + 3 * DK));
+                    if (timed_out) {
+                        raise_error(a.err, ERR_TIMEOUT);
+                        p0 = 1.f;
                         break;
                     }
-                    const float m00 = __ldcg(dj), m01 = __ldcg(dj + DK), m10 = __ldcg(dj + 2 * DK);
+                    if (tag_of(w3) == TAG_INCL) {
+                        p0 = mob(r00, r01, r10, 1.f, value_of(w3));
+                        break;
+                    }
+                    const float m00 = value_of(w0), m01 = value_of(w1), m10 = value_of(w2);
                     const float n00 = fmaf(r00, m00, r01 * m10), n01 = fmaf(r00, m01, r01);
                     const float n10 = fmaf(r10, m00, m10), n11 = fmaf(r10, m01, 1.f);
                     const float sc = 1.f / n11;
@@ -390,19 +384,14 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
             }
             pst[cc] = p0;
             const float pe = mob(g00, g01, g10, 1.f, p0);
-            __stcg(desc + 3 * DK + cc, pe);
+            st_relaxed(desc + 3 * DK, tagged(pe, TAG_INCL));
             if (c == nch - 1 && a.P_out) a.P_out[(size_t)chain * DK + cc] = pe;
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) atomicExch(pa.flags + u * 4 + warp, FLAG_INCL);
-        } else {
-            form_kq();
         }
         __syncthreads();
-        if (warp < 4) form_kq();
 
-        // ---- re-expansion: P^- per token (from the chunk-start uncertainty through the earlier
-        //      segments' composites), G^ = P^- k / Gam and the den partial sums
+        // ---- re-expansion fused with the chunk operands: P^- per token (from the chunk-start
+        //      uncertainty through the earlier segments' composites), Gam (inclusive decay from
+        //      the chunk start), K~ = k Gam, Q~ = q Gam, G^ = P^- k / Gam, den partial sums
         {
             float Pa = pst[ch], Pb = pst[ch + 1], gama, gamb;
             gamma_start(gama, gamb);
@@ -416,7 +405,7 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const int t = tb + j;
-                uint32_t gg = 0u;
+                uint32_t kq = 0u, qq = 0u, gg = 0u;
                 xs[j] = 0.f;
                 if (t < L) {
                     const float ala = bf16_lo(aw[j]), alb = bf16_hi(aw[j]);
@@ -428,10 +417,19 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
                     gama *= ala;
                     gamb *= alb;
                     const float pka = pma * ka, pkb = pmb * kb;
+                    kq = pack_bf16x2(ka * gama, kb * gamb);
+                    qq = pack_bf16x2(bf16_lo(qw[j]) * gama, bf16_hi(qw[j]) * gamb);
                     gg = pack_bf16x2(__fdividef(pka, gama), __fdividef(pkb, gamb));
                     xs[j] = fmaf(pka, ka, pkb * kb);
                 }
+                *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(t, bch)) = kq;
+                *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(64 + t, bch)) = qq;
                 *reinterpret_cast<uint32_t *>(sm + L_::G + atom8 + swz(t, bch)) = gg;
+            }
+            if (tb < L && tb + 16 >= L) {   // this segment holds the chunk's last token
+                gamc[ch] = gama;
+                gamc[ch + 1] = gamb;
+                if (!(gama >= 1e-30f) || !(gamb >= 1e-30f)) raise_error(a.err, ERR_RANGE);
             }
             int which;
             const float tot = warp_reduce16(xs, lane, which);
@@ -473,7 +471,7 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
                     *reinterpret_cast<uint4 *>(sm + L_::LB + swz(t, (cg * 4 + chn) * 16)) = lower_left ? pack8(v + chn * 8) : z;
                 }
                 if (b == cg) {
-                    float *dst = adg + (b * 32 + tr) * 32;
+                    float *dst = adg + (b * 32 + tr) * ADS;
 #pragma unroll
                     for (int jj = 0; jj < 32; jj += 4)
                         *reinterpret_cast<float4 *>(dst + jj) =
@@ -501,7 +499,7 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
                 for (int r = 0; r < 32; ++r) x[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
                 for (int r = 1; r < 32; ++r) {   // A's row r is zero from column r on
-                    const float4 *arow = reinterpret_cast<const float4 *>(adg + (b * 32 + r) * 32);
+                    const float4 *arow = reinterpret_cast<const float4 *>(adg + (b * 32 + r) * ADS);
                     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int q4 = 0; q4 < (r + 3) / 4; ++q4) {
@@ -517,7 +515,7 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
             __syncthreads();
             if (tid < 64) {
 #pragma unroll
-                for (int r = 0; r < 32; ++r) adg[(b * 32 + r) * 32 + j] = x[r];
+                for (int r = 0; r < 32; ++r) adg[(b * 32 + r) * ADS + j] = x[r];
             }
             __syncthreads();
             // bf16 D: 64 rows x 8 chunks of 16 B, two chunks per thread
@@ -526,7 +524,7 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
                 const int r = tid >> 2, cc = (tid & 3) * 2 + half, rb = r >> 5, cb = cc >> 2;
                 float d8[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) d8[e] = (cb == rb) ? adg[(rb * 32 + (r & 31)) * 32 + (cc & 3) * 8 + e] : 0.f;
+                for (int e = 0; e < 8; ++e) d8[e] = (cb == rb) ? adg[(rb * 32 + (r & 31)) * ADS + (cc & 3) * 8 + e] : 0.f;
                 *reinterpret_cast<uint4 *>(sm + L_::DB + swz(r, cc * 16)) = pack8(d8);
             }
         }
@@ -815,8 +813,7 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
 // ================================================================= host side
 size_t two_phase_workspace_bytes(long long nchains, long long nchunks_max) {
     const long long units = nchains * nchunks_max;
-    const size_t flags = ((size_t)units * 16 + 255) / 256 * 256;
-    return 256 + flags + (size_t)units * 4 * DK * 4 + (size_t)units * Rec::BYTES;
+    return 256 + (size_t)units * 4 * DK * 8 + (size_t)units * Rec::BYTES;
 }
 
 template <int DVT>
@@ -834,7 +831,7 @@ cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long
     const long long nchains = (long long)a.nseq * a.H;
     if (nchains == 0) return cudaSuccess;
     const long long units = nchains * nchunks_max;
-    const size_t flags = ((size_t)units * 16 + 255) / 256 * 256;
+    const size_t desc_bytes = (size_t)units * 4 * DK * 8;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
 
     PrepArgs pa;
@@ -842,9 +839,8 @@ cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long
     pa.nchunks_max = nchunks_max;
     pa.nchains = (int)nchains;
     pa.counter = reinterpret_cast<unsigned *>(ws);
-    pa.flags = reinterpret_cast<int *>(ws + 256);
-    pa.desc = reinterpret_cast<float *>(ws + 256 + flags);
-    pa.rec = ws + 256 + flags + (size_t)units * 4 * DK * 4;
+    pa.desc = reinterpret_cast<unsigned long long *>(ws + 256);
+    pa.rec = ws + 256 + desc_bytes;
 
     StateArgs sa;
     sa.a = a;
@@ -855,7 +851,7 @@ cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long
 
     cudaError_t e = cudaSuccess;
     if (units > 0) {
-        e = cudaMemsetAsync(ws, 0, 256 + flags, st);   // ticket counter and unit flags
+        e = cudaMemsetAsync(ws, 0, 256 + desc_bytes, st);   // ticket counter and look-back words (untagged)
         if (e != cudaSuccess) return e;
         constexpr size_t psmem = PrepSmem::total + 1024;
         e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
