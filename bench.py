@@ -226,6 +226,27 @@ def bench_prefill(args, world, rank, dev, kdn):
     value, total_ms = whole_job_rate(tokens, args.steps, evs[0].elapsed_time(evs[-1]), world)
     ms_step = total_ms / args.steps
 
+    # the same forward without a workspace (the one-kernel tensor-core path), for comparison
+    single = None
+    if path == "chunk_tcgen05_two_phase":
+        def step_single():
+            kdn.forward(d["q"], d["k"], d["v"], d["alpha"], d["sigma"], d["r"], cu_seqlens=cu, mu=w.mu,
+                        chunk=w.chunk, o=o, S_out=S_out, P_out=P_out, workspace=False, max_seqlen=max_seqlen)
+        for _ in range(2):
+            step_single()
+        barrier(world)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_single = max(3, min(args.steps, 5))
+        f0.record(stream)
+        for _ in range(n_single):
+            step_single()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        kdn.last_device_error()
+        s_value, s_ms = whole_job_rate(w.ntok, n_single, f0.elapsed_time(f1), world)
+        single = dict(value=s_value, ms_per_step=s_ms / n_single, path="chunk_tcgen05", gpu_launches=n_single)
+
     # end to end through the C ABI: pinned host inputs -> device, forward, o -> host
     pinned = {n: torch.from_numpy(np.ascontiguousarray(host[n]).view(np.int16) if host[n].dtype == np.uint16
                                   else np.ascontiguousarray(host[n])).pin_memory() for n in names}
@@ -289,6 +310,7 @@ def bench_prefill(args, world, rank, dev, kdn):
 
     nbytes = algorithmic_bytes(w)
     return dict(w=w, value=value, ms_step=ms_step, per_step_ms=per_step_ms, clocks=clk.summary(), path=path, scan=scan,
+                single=single,
                 e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                          steps=e_steps),
                 bytes=nbytes, launches=args.steps * launches_per_step)
@@ -378,14 +400,15 @@ def cpu_baseline_prefill(w, min_seconds=10.0, max_reps=50):
 
 def kernel_hash():
     h = hashlib.sha1()
-    for fn in ("kdn_chunk_tc.cu", "kdn_tc.cuh", "kdn_common.cuh"):
+    for fn in ("kdn_chunk_2p.cu", "kdn_tc.cuh", "kdn_common.cuh"):
         with open(os.path.join(ROOT, "kalman_delta_rule_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:12]
 
 
 def recorded_traffic(workload_name):
-    """dram bytes per launch from the committed ncu summary, if taken on the current kernel source."""
+    """dram bytes of one forward step (its prep and state launches) from the committed ncu
+    summary, if taken on the current kernel source."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
     if not os.path.exists(p):
         return None
@@ -425,13 +448,20 @@ def ours(args):
                        "l2": f"inputs larger than L2 ({pre['bytes'] / 1e9:.2f} GB > 0.13 GB), no flush",
                        "parallelism": f"replicas x{world} (independent batches, no collective)"},
             "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                         "traffic": traffic, "peak_kind": f"{pk_kind} copy bandwidth",
-                         "algorithmic_bytes_per_launch": pre["bytes"]},
+                         "traffic": traffic if pre["path"] == "chunk_tcgen05_two_phase" else None,
+                         "peak_kind": f"{pk_kind} copy bandwidth",
+                         "algorithmic_bytes_per_launch": pre["bytes"],
+                         "unit_of_measure": "one forward step = the prep and the state launch of the "
+                                            "two-launch tensor-core path; achieved and traffic are per step"},
             "cpu_baseline": cpu,
             "e2e": pre["e2e"],
             "gpu_launches": pre["launches"],
             "clocks": pre["clocks"],
         }
+        if pre["single"] is not None:
+            sg = pre["single"]
+            sg["roofline_frac"] = pre["bytes"] / (sg["ms_per_step"] / 1e3) / 1e9 / hbm
+            line["prefill_single_kernel"] = sg
         if pre["scan"] is not None:
             sc = pre["scan"]
             sach = sc["bytes"] / (sc["ms_step"] / 1e3) / 1e9

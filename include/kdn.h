@@ -196,6 +196,14 @@ kdn_status_t kdn_gain_scan_noalloc(const kdn_problem_t *p,
  * without one such a problem runs path 2); -1 if `p` is invalid. */
 int kdn_execution_path(const kdn_problem_t *p);
 
+/* Self-test of failure detection: launches one kernel whose two bounded waits -- a poll of a
+ * device word that nothing writes (the look-back's wait) and an mbarrier phase that nothing
+ * completes (the tensor-core kernels' wait) -- each give up after `limit_cycles` SM clock cycles
+ * (1e3 .. 4e9; 2e6 is about a millisecond) and record KDN_ERR_TIMEOUT in the device error word.
+ * Nothing faults or hangs; kdn_last_device_error() then reports KDN_ERR_TIMEOUT and clears it.
+ * The method has no counterpart on the pages: this checks the library's own error path. */
+kdn_status_t kdn_selftest_bounded_wait(long long limit_cycles, void *stream);
+
 /* Synchronises `stream`, then returns and clears the device error word
  * (KDN_ERR_TIMEOUT, KDN_ERR_RANGE or KDN_ERR_INVALID_ARG if a kernel recorded one, else KDN_OK). */
 kdn_status_t kdn_last_device_error(void *stream);

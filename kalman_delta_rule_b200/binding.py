@@ -48,6 +48,7 @@ _SIGS = {
     "kdn_decode_tokens_iso": (_i, [_i, _i, _i, _i, _i, _i, _f] + [_vp] * 6 + [_vp] * 3 + [_vp]),
     "kdn_gain_scan": (_i, [_PP] + [_vp] * 4 + [_vp] + [_vp] * 3 + [_vp, _sz, _vp]),
     "kdn_last_device_error": (_i, [_vp]),
+    "kdn_selftest_bounded_wait": (_i, [ctypes.c_longlong, _vp]),
     "kdn_status_string": (ctypes.c_char_p, [_i]),
     "kdn_version": (ctypes.c_char_p, []),
     "kdn_execution_path": (_i, [_PP]),
@@ -274,6 +275,12 @@ def execution_path(q, v, cu_seqlens=None, mu: float = 1.0, chunk: int = 64, vari
     if code == 3 and not workspace:
         code = 2
     return PATH_NAMES.get(code, "invalid")
+
+
+def selftest_bounded_wait(limit_cycles: int = 2_000_000, stream=None):
+    """Launch the failure-detection self-test (bounded waits that run out); the device error
+    word then holds KDN_ERR_TIMEOUT, which last_device_error() raises."""
+    _check(load().kdn_selftest_bounded_wait(int(limit_cycles), _stream_handle(stream)), "kdn_selftest_bounded_wait")
 
 
 def last_device_error(stream=None):

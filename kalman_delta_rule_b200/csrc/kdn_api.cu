@@ -231,6 +231,13 @@ kdn_status_t kdn_gain_scan_noalloc(const kdn_problem_t *p, const void *k, const 
     return cuda_status(kdn::launch_gain_scan_noalloc(a, rv.bf16, static_cast<cudaStream_t>(stream)));
 }
 
+kdn_status_t kdn_selftest_bounded_wait(long long limit_cycles, void *stream) {
+    if (limit_cycles < 1000 || limit_cycles > 4000000000ll) return KDN_ERR_INVALID_ARG;
+    unsigned *err = err_word();
+    if (!err) return KDN_ERR_CUDA;
+    return cuda_status(kdn::launch_bounded_wait_selftest(limit_cycles, err, static_cast<cudaStream_t>(stream)));
+}
+
 int kdn_execution_path(const kdn_problem_t *p) {
     Resolved rv;
     if (check_problem(p, &rv) != KDN_OK) return -1;

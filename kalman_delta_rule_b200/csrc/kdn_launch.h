@@ -28,6 +28,9 @@ cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long
 // [ntok, H, d] bf16 as a TMA tensor map with 64 x 1 x 64 boxes and 128-byte swizzle
 bool make_token_map(CUtensorMap *m, const void *base, int d, int H, long long ntok);
 
+// failure-detection self-test: bounded waits that run out and record ERR_TIMEOUT
+cudaError_t launch_bounded_wait_selftest(long long limit_cycles, unsigned *err, cudaStream_t st);
+
 // single-pass Moebius scan of the uncertainty with decoupled look-back (workspace-backed)
 size_t scan_workspace_bytes(long long nchains, long long nchunks_max, int dk);
 cudaError_t launch_gain_scan(ScanArgs a, bool bf16_in, void *workspace, cudaStream_t st);

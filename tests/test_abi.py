@@ -142,3 +142,8 @@ def test_product_path_fails_loudly_without_library(tmp_path):
             mod.load(str(tmp_path / "missing.so"))
     finally:
         mod._lib = saved
+
+
+def test_selftest_rejects_a_bad_wait_bound(lib):
+    assert B.load().kdn_selftest_bounded_wait(10, None) == B.KDN_ERR_INVALID_ARG
+    assert B.load().kdn_selftest_bounded_wait(1 << 40, None) == B.KDN_ERR_INVALID_ARG
