@@ -174,7 +174,7 @@ kdn_status_t kdn_gain_scan(const kdn_problem_t *p,
  * synchronises the device).  The paper has no counterpart: this entry point only changes
  * where the scan keeps its scratch.
  *  Arguments: as kdn_gain_scan() without the workspace; inputs and outputs stay the
- *  caller's.  Scratch: a fixed 16 MiB device array inside the library, one per GPU that
+ *  caller's.  Scratch: a fixed 32 MiB device array inside the library, one per GPU that
  *  loads it, held until the process exits.  A problem whose scan needs more (more than
  *  about 8000 (chunk of 64 tokens, sequence x head) pairs at d_k = 128) returns
  *  KDN_ERR_UNSUPPORTED before anything runs.

@@ -214,7 +214,7 @@ kdn_status_t kdn_gain_scan(const kdn_problem_t *p, const void *k, const void *al
     const size_t need = kdn::scan_workspace_bytes((long long)rv.nseq * p->H, rv.nchunks_max, p->d_k);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return KDN_ERR_WORKSPACE;
     a.err = err_word();
-    return cuda_status(kdn::launch_gain_scan(a, rv.bf16, workspace, static_cast<cudaStream_t>(stream)));
+    return cuda_status(kdn::launch_gain_scan(a, rv.bf16, rv.ntok, workspace, static_cast<cudaStream_t>(stream)));
 }
 
 kdn_status_t kdn_gain_scan_noalloc(const kdn_problem_t *p, const void *k, const void *alpha, const void *sigma,
@@ -228,7 +228,7 @@ kdn_status_t kdn_gain_scan_noalloc(const kdn_problem_t *p, const void *k, const 
     if (kdn::scan_workspace_bytes((long long)rv.nseq * p->H, rv.nchunks_max, p->d_k) > kdn::noalloc_scratch_bytes())
         return KDN_ERR_UNSUPPORTED;
     a.err = err_word();
-    return cuda_status(kdn::launch_gain_scan_noalloc(a, rv.bf16, static_cast<cudaStream_t>(stream)));
+    return cuda_status(kdn::launch_gain_scan_noalloc(a, rv.bf16, rv.ntok, static_cast<cudaStream_t>(stream)));
 }
 
 kdn_status_t kdn_selftest_bounded_wait(long long limit_cycles, void *stream) {

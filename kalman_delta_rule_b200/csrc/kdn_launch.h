@@ -33,9 +33,13 @@ cudaError_t launch_bounded_wait_selftest(long long limit_cycles, unsigned *err, 
 
 // single-pass Moebius scan of the uncertainty with decoupled look-back (workspace-backed)
 size_t scan_workspace_bytes(long long nchains, long long nchunks_max, int dk);
-cudaError_t launch_gain_scan(ScanArgs a, bool bf16_in, void *workspace, cudaStream_t st);
+cudaError_t launch_gain_scan(ScanArgs a, bool bf16_in, long long ntok, void *workspace, cudaStream_t st);
 // the same scan on the library's fixed scratch array (no allocation, no caller workspace)
 size_t noalloc_scratch_bytes();
-cudaError_t launch_gain_scan_noalloc(const ScanArgs &a, bool bf16_in, cudaStream_t st);
+cudaError_t launch_gain_scan_noalloc(const ScanArgs &a, bool bf16_in, long long ntok, cudaStream_t st);
+// bf16, d_k = 128: TMA-staged scan with tagged look-back words (its own workspace layout)
+bool gain_scan_tma_supported(int dk, bool bf16_in);
+size_t scan_tma_workspace_bytes(long long nchains, long long nchunks_max);
+cudaError_t launch_gain_scan_tma(const ScanArgs &a, long long ntok, void *workspace, cudaStream_t st);
 
 }  // namespace kdn

@@ -281,11 +281,14 @@ static cudaError_t launch_scan_t(const ScanArgs &a, cudaStream_t st) {
 size_t scan_workspace_bytes(long long nchains, long long nchunks_max, int dk) {
     const long long units = nchains * nchunks_max;
     const size_t flags = ((size_t)units * 4 + 255) / 256 * 256;
-    return 256 + flags + (size_t)units * 4 * dk * 4;
+    const size_t generic = 256 + flags + (size_t)units * 4 * dk * 4;
+    const size_t tma = dk == 128 ? scan_tma_workspace_bytes(nchains, nchunks_max) : 0;
+    return generic > tma ? generic : tma;
 }
 
-cudaError_t launch_gain_scan(ScanArgs a, bool bf16_in, void *workspace, cudaStream_t st) {
+cudaError_t launch_gain_scan(ScanArgs a, bool bf16_in, long long ntok, void *workspace, cudaStream_t st) {
     if (a.nchains == 0 || a.nchunks_max == 0) return cudaSuccess;
+    if (gain_scan_tma_supported(a.dk, bf16_in)) return launch_gain_scan_tma(a, ntok, workspace, st);
     const long long units = (long long)a.nchains * a.nchunks_max;
     const size_t flags = ((size_t)units * 4 + 255) / 256 * 256;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -308,7 +311,7 @@ cudaError_t launch_gain_scan(ScanArgs a, bool bf16_in, void *workspace, cudaStre
 // ---------------------------------------------------------------- allocation-free variant
 // Scratch of kdn_gain_scan_noalloc: a fixed device array (one copy on every GPU that loads
 // the library, held until the process exits) used instead of a caller-provided workspace.
-constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;
+constexpr size_t kNoAllocScratchBytes = (size_t)32 << 20;
 static __device__ __align__(256) unsigned char g_scan_scratch[kNoAllocScratchBytes];
 
 namespace {
@@ -338,11 +341,11 @@ static cudaError_t scratch_address(void **out) {
 
 size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 
-cudaError_t launch_gain_scan_noalloc(const ScanArgs &a, bool bf16_in, cudaStream_t st) {
+cudaError_t launch_gain_scan_noalloc(const ScanArgs &a, bool bf16_in, long long ntok, cudaStream_t st) {
     void *ws = nullptr;
     cudaError_t e = scratch_address(&ws);
     if (e != cudaSuccess) return e;
-    return launch_gain_scan(a, bf16_in, ws, st);   // clears the ticket counter and flags it uses
+    return launch_gain_scan(a, bf16_in, ntok, ws, st);   // clears the ticket counter and flags it uses
 }
 
 }  // namespace kdn

@@ -1,0 +1,370 @@
+// The uncertainty / gain scan for bf16 inputs with d_k = 128: the same single pass with a
+// decoupled look-back as the generic scan (explainer, closing paragraph of "各向同性近似": the
+// uncertainty recursion is a Moebius map whose 2x2 matrices compose), with
+//  - the chunk's alpha, sigma and k tiles fetched by TMA one unit ahead (two stages), so the
+//    loads of the next unit overlap the current one;
+//  - look-back words that carry their own tag (64-bit (value, tag) per key channel), so a
+//    reader never needs a fence or a flag, and every channel walks back on its own;
+//  - thread = key-channel pair x 16-token segment in the composite and re-expansion passes.
+// Outputs: g_t = P^-_t k_t / den_t (fp32), k_t^T g_t, and the uncertainty after each sequence.
+#include "kdn_common.cuh"
+#include "kdn_launch.h"
+#include "kdn_tc.cuh"
+
+namespace kdn {
+
+namespace {
+constexpr int C = 64, DK = 128, NT = 256;
+enum : unsigned { TAG_AGG = 1, TAG_INCL = 2 };
+
+struct ScanTmaSmem {
+    static constexpr uint32_t STAGE = 3 * 16384;          // alpha, sigma, k tiles of one chunk
+    static constexpr uint32_t COMP = 2 * STAGE;           // segment composites fp32 [4][128][4]
+    static constexpr uint32_t MISC = COMP + 4 * 128 * 16;  // r [64], mu / r [64], P at chunk start [128], sum P^- k^2 [64]
+    static constexpr uint32_t CTL = MISC + 1280;           // 2 mbarriers, ticket
+    static constexpr uint32_t total = CTL + 64;
+};
+
+struct ScanTmaArgs {
+    ScanArgs a;
+    CUtensorMap tal, tsg, tk;
+    unsigned long long *words;   // per unit [4][128]: aggregate (m00, m01, m10), end-of-chunk P
+};
+
+__device__ __forceinline__ float mob(float m00, float m01, float m10, float m11, float x) {
+    return fmaf(m00, x, m01) / fmaf(m10, x, m11);
+}
+__device__ __forceinline__ unsigned long long tagged(float x, unsigned tag) {
+    return ((unsigned long long)tag << 32) | __float_as_uint(x);
+}
+__device__ __forceinline__ unsigned tag_of(unsigned long long w) { return (unsigned)(w >> 32); }
+__device__ __forceinline__ float value_of(unsigned long long w) { return __uint_as_float((unsigned)w); }
+__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Sums 16 per-lane values over the 32 lanes of a warp with 16 shuffles (each step exchanges
+// half of the remaining values).  Lanes 2m and 2m+1 end with the total of value `which`.
+__device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane, int &which) {
+    const unsigned FULL = 0xffffffffu;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const bool up = lane & 16;
+        const float send = up ? v[i] : v[i + 8], keep = up ? v[i + 8] : v[i];
+        v[i] = keep + __shfl_xor_sync(FULL, send, 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const bool up = lane & 8;
+        const float send = up ? v[i] : v[i + 4], keep = up ? v[i + 4] : v[i];
+        v[i] = keep + __shfl_xor_sync(FULL, send, 8);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const bool up = lane & 4;
+        const float send = up ? v[i] : v[i + 2], keep = up ? v[i + 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(FULL, send, 4);
+    }
+    {
+        const bool up = lane & 2;
+        const float send = up ? v[0] : v[1], keep = up ? v[1] : v[0];
+        v[0] = keep + __shfl_xor_sync(FULL, send, 2);
+    }
+    v[0] += __shfl_xor_sync(FULL, v[0], 1);
+    which = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+    return v[0];
+}
+}  // namespace
+
+__global__ void __launch_bounds__(NT, 2) gain_scan_tma_kernel(const __grid_constant__ ScanTmaArgs sa)
+{
+    using L_ = ScanTmaSmem;
+    using namespace tc;
+    extern __shared__ uint8_t smraw[];
+    const uint32_t raw_u32 = smem_u32(smraw);
+    const uint32_t sb = (raw_u32 + 1023u) & ~1023u;
+    uint8_t *sm = smraw + (sb - raw_u32);
+    float *comp = reinterpret_cast<float *>(sm + L_::COMP);
+    float *r_s = reinterpret_cast<float *>(sm + L_::MISC);
+    float *mur = r_s + 64;
+    float *pst = mur + 64;
+    float *dsum = pst + 128;
+    uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + L_::CTL);   // [2]
+    long long *ticket = reinterpret_cast<long long *>(sm + L_::CTL + 16);
+
+    const ScanArgs &a = sa.a;
+    const bf16 *__restrict__ rin = static_cast<const bf16 *>(a.r);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = a.H;
+    const long long units = (long long)a.nchunks_max * a.nchains;
+    const int cp = (warp & 1) * 32 + lane, sgi = warp >> 1, ch = cp * 2, tb = sgi * 16;
+    const uint32_t catom = (uint32_t)(ch >> 6) * 8192u, bch = (uint32_t)(ch & 63) * 2u;
+
+    if (tid == 0) {
+        mbar_init(bar_full, 1);
+        mbar_init(bar_full + 1, 1);
+        mbar_fence_init();
+        tma_prefetch_desc(&sa.tal);
+        tma_prefetch_desc(&sa.tsg);
+        tma_prefetch_desc(&sa.tk);
+    }
+    __syncthreads();
+
+    struct Unit { long long u; int c, chain, h, c0, L, nch; };
+    // next unit with tokens (all threads; tickets of chunks past a sequence's end are skipped)
+    auto claim = [&]() -> Unit {
+        Unit n;
+        for (;;) {
+            if (tid == 0) *ticket = (long long)atomicAdd(a.counter, 1u);
+            __syncthreads();
+            n.u = *ticket;
+            __syncthreads();
+            if (n.u >= units) return n;
+            n.c = (int)(n.u / a.nchains);
+            n.chain = (int)(n.u % a.nchains);
+            n.h = n.chain % H;
+            int t0, t1;
+            if (a.cu) { t0 = __ldg(a.cu + n.chain / H); t1 = __ldg(a.cu + n.chain / H + 1); }
+            else { t0 = (n.chain / H) * a.T; t1 = t0 + a.T; }
+            n.nch = (t1 - t0 + C - 1) / C;
+            if (n.c == 0 && tid == 0 && n.nch > a.nchunks_max) raise_error(a.err, ERR_ARG);
+            if (n.c < n.nch) {
+                n.c0 = t0 + n.c * C;
+                n.L = min(C, t1 - n.c0);
+                return n;
+            }
+        }
+    };
+    // the unit's tiles into stage st (thread 0), its r into r_next (threads < 64)
+    float r_next = 1.f;
+    auto fetch = [&](const Unit &n, int st) {
+        if (tid == 0) {
+            mbar_expect_tx(bar_full + st, L_::STAGE);
+            uint8_t *dst = sm + st * L_::STAGE;
+            for (int b = 0; b < 2; ++b) {
+                tma_load_3d(dst + b * 8192, &sa.tal, b * 64, n.h, n.c0, bar_full + st);
+                tma_load_3d(dst + 16384 + b * 8192, &sa.tsg, b * 64, n.h, n.c0, bar_full + st);
+                tma_load_3d(dst + 32768 + b * 8192, &sa.tk, b * 64, n.h, n.c0, bar_full + st);
+            }
+        }
+        r_next = (tid < n.L) ? ldf(rin + (size_t)(n.c0 + tid) * H + n.h) : 1.f;
+    };
+
+    Unit nx = claim();
+    if (nx.u < units) fetch(nx, 0);
+    bool abort = false;
+    for (int it = 0;; ++it) {
+        const Unit cur = nx;
+        if (cur.u >= units || abort) break;
+        const int st = it & 1;
+        const long long u = cur.u;
+        const int c = cur.c, chain = cur.chain, h = cur.h, c0 = cur.c0, L = cur.L, nch = cur.nch;
+        if (tid < C) {
+            r_s[tid] = r_next;
+            mur[tid] = a.mu / r_next;
+            dsum[tid] = 0.f;
+        }
+        if (!mbar_wait(bar_full + st, (uint32_t)((it >> 1) & 1))) abort = true;   // k-th use of a stage: parity k & 1
+        // the next unit's tiles go to the other stage while this one is processed
+        nx = claim();
+        if (nx.u < units) fetch(nx, st ^ 1);
+        if (__syncthreads_or(abort)) {
+            raise_error(a.err, ERR_TIMEOUT);
+            break;
+        }
+        const uint8_t *tile = sm + st * L_::STAGE;
+
+        // ---- segment composites of the uncertainty maps (predict [[a, s],[0,1]], update [[1,0],[c,1]])
+        {
+            float a00 = 1.f, a01 = 0.f, a10 = 0.f, a11 = 1.f, ga = 1.f;
+            float b00 = 1.f, b01 = 0.f, b10 = 0.f, b11 = 1.f, gb = 1.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                if (tb + j < L) {
+                    const uint32_t off = catom + swz(tb + j, bch);
+                    const uint32_t aw = *reinterpret_cast<const uint32_t *>(tile + off);
+                    const uint32_t sw = *reinterpret_cast<const uint32_t *>(tile + 16384 + off);
+                    const uint32_t kw = *reinterpret_cast<const uint32_t *>(tile + 32768 + off);
+                    const float mr = mur[tb + j];
+                    {
+                        const float al = bf16_lo(aw), sg = bf16_lo(sw), kk = bf16_lo(kw);
+                        const float aa = al * al, cc = mr * kk * kk;
+                        const float y00 = fmaf(aa, a00, sg * a10), y01 = fmaf(aa, a01, sg * a11);
+                        a10 = fmaf(cc, y00, a10); a11 = fmaf(cc, y01, a11); a00 = y00; a01 = y01; ga *= al;
+                    }
+                    {
+                        const float al = bf16_hi(aw), sg = bf16_hi(sw), kk = bf16_hi(kw);
+                        const float aa = al * al, cc = mr * kk * kk;
+                        const float y00 = fmaf(aa, b00, sg * b10), y01 = fmaf(aa, b01, sg * b11);
+                        b10 = fmaf(cc, y00, b10); b11 = fmaf(cc, y01, b11); b00 = y00; b01 = y01; gb *= al;
+                    }
+                }
+            }
+            const float sa_ = 1.f / a11, sb_ = 1.f / b11;
+            *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch) * 4) = make_float4(a00 * sa_, a01 * sa_, a10 * sa_, ga);
+            *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch + 1) * 4) = make_float4(b00 * sb_, b01 * sb_, b10 * sb_, gb);
+        }
+        __syncthreads();
+
+        // ---- warps 0-3 (thread = key channel): aggregate, its publication, decoupled look-back
+        if (warp < 4) {
+            const int cc = tid;
+            unsigned long long *wd = sa.words + (size_t)u * 4 * DK + cc;
+            float g00 = 1.f, g01 = 0.f, g10 = 0.f, g11 = 1.f;
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+                const float4 cm = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + cc) * 4);
+                const float n00 = fmaf(cm.x, g00, cm.y * g10), n01 = fmaf(cm.x, g01, cm.y * g11);
+                const float n10 = fmaf(cm.z, g00, g10), n11 = fmaf(cm.z, g01, g11);
+                const float sc = 1.f / n11;
+                g00 = n00 * sc; g01 = n01 * sc; g10 = n10 * sc; g11 = 1.f;
+            }
+            if (c > 0) {
+                st_relaxed(wd + 0 * DK, tagged(g00, TAG_AGG));
+                st_relaxed(wd + 1 * DK, tagged(g01, TAG_AGG));
+                st_relaxed(wd + 2 * DK, tagged(g10, TAG_AGG));
+            }
+            float p0;
+            if (c == 0) {
+                p0 = a.P0 ? a.P0[(size_t)chain * DK + cc] : 1.f;
+            } else {
+                float r00 = 1.f, r01 = 0.f, r10 = 0.f;   // composite of the chunks walked over ((1,1) kept at 1)
+                bool timed_out = false;
+                for (int j = c - 1;; --j) {
+                    const unsigned long long *dj = sa.words + ((size_t)j * a.nchains + chain) * 4 * DK + cc;
+                    unsigned long long w0 = 0ull, w1 = 0ull, w2 = 0ull, w3 = ld_relaxed(dj + 3 * DK);
+                    const long long ts = clock64();
+                    while (tag_of(w3) != TAG_INCL) {
+                        w0 = ld_relaxed(dj);
+                        w1 = ld_relaxed(dj + DK);
+                        w2 = ld_relaxed(dj + 2 * DK);
+                        if (tag_of(w0) == TAG_AGG && tag_of(w1) == TAG_AGG && tag_of(w2) == TAG_AGG) break;
+                        // give up after ~1 s, or at once when another wait already gave up
+                        if (clock64() - ts > 2000000000ll || (a.err && (*(volatile unsigned *)a.err & ERR_TIMEOUT))) {
+                            timed_out = true;
+                            break;
+                        }
+                        __nanosleep(32);
+                        w3 = ld_relaxed(dj + 3 * DK);
+                    }
+                    if (timed_out) {
+                        raise_error(a.err, ERR_TIMEOUT);
+                        p0 = 1.f;
+                        break;
+                    }
+                    if (tag_of(w3) == TAG_INCL) {
+                        p0 = mob(r00, r01, r10, 1.f, value_of(w3));
+                        break;
+                    }
+                    const float m00 = value_of(w0), m01 = value_of(w1), m10 = value_of(w2);
+                    const float n00 = fmaf(r00, m00, r01 * m10), n01 = fmaf(r00, m01, r01);
+                    const float n10 = fmaf(r10, m00, m10), n11 = fmaf(r10, m01, 1.f);
+                    const float sc = 1.f / n11;
+                    r00 = n00 * sc; r01 = n01 * sc; r10 = n10 * sc;
+                }
+            }
+            pst[cc] = p0;
+            const float pe = mob(g00, g01, g10, 1.f, p0);
+            st_relaxed(wd + 3 * DK, tagged(pe, TAG_INCL));
+            if (c == nch - 1 && a.P_out) a.P_out[(size_t)chain * DK + cc] = pe;
+        }
+        __syncthreads();
+
+        // ---- re-expansion: P^- k per token and channel, the gain denominators, g and k^T g
+        float pk[32];
+        {
+            float Pa = pst[ch], Pb = pst[ch + 1];
+            for (int q2 = 0; q2 < sgi; ++q2) {
+                const float4 ca = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch) * 4);
+                const float4 cb = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch + 1) * 4);
+                Pa = mob(ca.x, ca.y, ca.z, 1.f, Pa);
+                Pb = mob(cb.x, cb.y, cb.z, 1.f, Pb);
+            }
+            float xs[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                pk[2 * j] = 0.f;
+                pk[2 * j + 1] = 0.f;
+                xs[j] = 0.f;
+                if (tb + j < L) {
+                    const uint32_t off = catom + swz(tb + j, bch);
+                    const uint32_t aw = *reinterpret_cast<const uint32_t *>(tile + off);
+                    const uint32_t sw = *reinterpret_cast<const uint32_t *>(tile + 16384 + off);
+                    const uint32_t kw = *reinterpret_cast<const uint32_t *>(tile + 32768 + off);
+                    const float ala = bf16_lo(aw), alb = bf16_hi(aw), ka = bf16_lo(kw), kb = bf16_hi(kw);
+                    const float pma = fmaf(ala * ala, Pa, bf16_lo(sw)), pmb = fmaf(alb * alb, Pb, bf16_hi(sw));
+                    const float pka = pma * ka, pkb = pmb * kb;
+                    const float mr = mur[tb + j];
+                    Pa = pma / fmaf(mr * ka, pka, 1.f);
+                    Pb = pmb / fmaf(mr * kb, pkb, 1.f);
+                    pk[2 * j] = pka;
+                    pk[2 * j + 1] = pkb;
+                    xs[j] = fmaf(pka, ka, pkb * kb);
+                }
+            }
+            int which;
+            const float tot = warp_reduce16(xs, lane, which);
+            if ((lane & 1) == 0 && tb + which < L) atomicAdd(dsum + tb + which, tot);
+        }
+        __syncthreads();
+        if (tid < C && tid < L) {
+            const float x = dsum[tid];
+            const float inv = 1.f / (r_s[tid] + x);
+            dsum[tid] = inv;
+            if (a.beta) a.beta[(size_t)(c0 + tid) * H + h] = x * inv;
+        }
+        __syncthreads();
+        if (a.g) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                if (tb + j < L) {
+                    const float inv = dsum[tb + j];
+                    *reinterpret_cast<float2 *>(a.g + ((size_t)(c0 + tb + j) * H + h) * DK + ch) =
+                        make_float2(pk[2 * j] * inv, pk[2 * j + 1] * inv);
+                }
+            }
+        }
+        __syncthreads();   // the stage, composites and sums are free for the next unit
+    }
+}
+
+size_t scan_tma_workspace_bytes(long long nchains, long long nchunks_max) {
+    return 256 + (size_t)(nchains * nchunks_max) * 4 * DK * 8;
+}
+
+bool gain_scan_tma_supported(int dk, bool bf16_in) { return bf16_in && dk == DK; }
+
+cudaError_t launch_gain_scan_tma(const ScanArgs &a, long long ntok, void *workspace, cudaStream_t st) {
+    if (a.nchains == 0 || a.nchunks_max == 0) return cudaSuccess;
+    const long long units = (long long)a.nchains * a.nchunks_max;
+    ScanTmaArgs sa;
+    sa.a = a;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    sa.a.counter = reinterpret_cast<unsigned *>(ws);
+    sa.words = reinterpret_cast<unsigned long long *>(ws + 256);
+    if (!make_token_map(&sa.tal, a.alpha, DK, a.H, ntok) || !make_token_map(&sa.tsg, a.sigma, DK, a.H, ntok) ||
+        !make_token_map(&sa.tk, a.k, DK, a.H, ntok))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(ws, 0, scan_tma_workspace_bytes(a.nchains, a.nchunks_max), st);
+    if (e != cudaSuccess) return e;
+    constexpr size_t smem = ScanTmaSmem::total + 1024;
+    e = cudaFuncSetAttribute(gain_scan_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(gain_scan_tma_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // two CTAs per SM; units go out by ticket to resident CTAs only, so extra CTAs are harmless
+    long long grid = (long long)sms * 2;
+    if (grid > units) grid = units;
+    gain_scan_tma_kernel<<<(unsigned)grid, NT, smem, st>>>(sa);
+    return cudaGetLastError();
+}
+
+}  // namespace kdn

@@ -42,7 +42,7 @@ def test_noalloc_gain_scan_matches_the_workspace_version_twice(kdn):
 
 def test_noalloc_gain_scan_rejects_a_problem_larger_than_its_scratch(kdn):
     import torch
-    # 32 heads x 1024 chunks of a 65536-token sequence need about 64 MiB of scratch
+    # 32 heads x 1024 chunks of a 65536-token sequence need about 128 MiB of scratch
     k = torch.empty((1, 65536, 32, 128), dtype=torch.bfloat16, device="cuda")
     p = kdn.make_problem(k, k)
     ptr = k.data_ptr()
