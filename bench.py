@@ -247,6 +247,31 @@ def bench_prefill(args, world, rank, dev, kdn):
         s_value, s_ms = whole_job_rate(w.ntok, n_single, f0.elapsed_time(f1), world)
         single = dict(value=s_value, ms_per_step=s_ms / n_single, path="chunk_tcgen05", gpu_launches=n_single)
 
+    # the isotropic variant (one uncertainty per head) on the same inputs and path
+    iso = None
+    if path.startswith("chunk_tcgen05"):
+        P_iso = torch.empty((w.num_seqs, w.H), dtype=torch.float32, device=dev)
+
+        def step_iso():
+            kdn.forward(d["q"], d["k"], d["v"], d["alpha"], d["sigma"], d["r"], cu_seqlens=cu, mu=w.mu,
+                        chunk=w.chunk, o=o, S_out=S_out, P_out=P_iso, workspace=ws, max_seqlen=max_seqlen,
+                        variant="isotropic")
+        for _ in range(2):
+            step_iso()
+        barrier(world)
+        i0, i1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_iso = max(3, min(args.steps, 5))
+        i0.record(stream)
+        for _ in range(n_iso):
+            step_iso()
+        i1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        kdn.last_device_error()
+        i_value, i_ms = whole_job_rate(w.ntok, n_iso, i0.elapsed_time(i1), world)
+        iso = dict(value=i_value, ms_per_step=i_ms / n_iso, gpu_launches=n_iso * launches_per_step,
+                   path=kdn.execution_path(d["q"], d["v"], cu_seqlens=cu, chunk=w.chunk, variant="isotropic"))
+
     # end to end through the C ABI: pinned host inputs -> device, forward, o -> host
     pinned = {n: torch.from_numpy(np.ascontiguousarray(host[n]).view(np.int16) if host[n].dtype == np.uint16
                                   else np.ascontiguousarray(host[n])).pin_memory() for n in names}
@@ -310,7 +335,7 @@ def bench_prefill(args, world, rank, dev, kdn):
 
     nbytes = algorithmic_bytes(w)
     return dict(w=w, value=value, ms_step=ms_step, per_step_ms=per_step_ms, clocks=clk.summary(), path=path, scan=scan,
-                single=single,
+                single=single, iso=iso,
                 e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                          steps=e_steps),
                 bytes=nbytes, launches=args.steps * launches_per_step)
@@ -458,6 +483,12 @@ def ours(args):
             "gpu_launches": pre["launches"],
             "clocks": pre["clocks"],
         }
+        if pre["iso"] is not None:
+            it = pre["iso"]
+            it["metric"] = "isotropic KDN prefill tokens/s"
+            it["unit"] = "tokens/s"
+            it["roofline_frac"] = pre["bytes"] / (it["ms_per_step"] / 1e3) / 1e9 / hbm
+            line["prefill_isotropic"] = it
         if pre["single"] is not None:
             sg = pre["single"]
             sg["roofline_frac"] = pre["bytes"] / (sg["ms_per_step"] / 1e3) / 1e9 / hbm

@@ -67,10 +67,9 @@ kdn_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? KDN_OK : KDN
 bool tc_path(const kdn_problem_t *p, const Resolved &rv) {
     return kdn::chunk_tc_supported(p->d_k, p->d_v, rv.bf16, p->chunk, rv.ntok);
 }
-// ... and the two-launch form applies (diagonal uncertainty, work list within 2^31 units)
+// ... and the two-launch form applies (work list within 2^31 units)
 bool two_phase_path(const kdn_problem_t *p, const Resolved &rv) {
-    return tc_path(p, rv) && p->variant == KDN_VARIANT_DIAGONAL &&
-           (long long)rv.nseq * p->H * rv.nchunks_max < (1ll << 31);
+    return tc_path(p, rv) && (long long)rv.nseq * p->H * rv.nchunks_max < (1ll << 31);
 }
 size_t two_phase_bytes(const kdn_problem_t *p, const Resolved &rv) {
     return kdn::two_phase_workspace_bytes((long long)rv.nseq * p->H, rv.nchunks_max);

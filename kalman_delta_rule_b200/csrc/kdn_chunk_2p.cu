@@ -19,6 +19,10 @@
 // swizzled atoms), so the state kernel fetches each with one bulk copy, double-buffered,
 // and its per-chunk critical path is two MMAs and two TMEM epilogues.
 //
+// Isotropic KDN (one uncertainty per head): the prep first sums alpha^2, sigma and k^2 over the
+// channels of every token; each channel then carries the head's map (channel means) through the
+// same composite / look-back / re-expansion machinery, and the records are the same.
+//
 // The prep kernel runs two 256-thread CTAs per SM; work is handed out by a ticket counter
 // in chunk-major order, so every predecessor of a unit belongs to a CTA that is already
 // running, and every wait is bounded (a wait that gives up records KDN_ERR_TIMEOUT).
@@ -58,7 +62,8 @@ struct PrepSmem {
     static constexpr uint32_t MUR = RS + 256;          // mu / r [64]
     static constexpr uint32_t PST = MUR + 256;         // uncertainty at the chunk start [128]
     static constexpr uint32_t DSUM = PST + 512;        // sum_i P^- k^2 per token [64]
-    static constexpr uint32_t CTL = DSUM + 256;        // mbarrier, ticket, TMEM slot, look-back flag, abort
+    static constexpr uint32_t TSUM = DSUM + 256;       // isotropic: per-token sums of alpha^2, sigma, k^2 [64][4]
+    static constexpr uint32_t CTL = TSUM + 1024;       // mbarrier, ticket, TMEM slot, look-back flag, abort
     static constexpr uint32_t total = CTL + 64;
     static_assert(COMP + 4 * 128 * 16 <= DB, "composites overlap D");
     static_assert(ADG + 64 * ADS * 4 <= Y && Y + 16384 <= MISC && A4 + 32768 <= Y, "work region");
@@ -158,6 +163,7 @@ __device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane, int &wh
 }  // namespace
 
 // ================================================================= prep
+template <bool ISO>
 __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constant__ PrepArgs pa)
 {
     using L_ = PrepSmem;
@@ -173,6 +179,7 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
     float *mur = reinterpret_cast<float *>(sm + L_::MUR);
     float *pst = reinterpret_cast<float *>(sm + L_::PST);
     float *dsum = reinterpret_cast<float *>(sm + L_::DSUM);
+    float *tsum = reinterpret_cast<float *>(sm + L_::TSUM);
     float *comp = reinterpret_cast<float *>(sm + L_::COMP);
     float *adg = reinterpret_cast<float *>(sm + L_::ADG);
     uint64_t *bar_mma = reinterpret_cast<uint64_t *>(sm + L_::CTL);
@@ -263,6 +270,7 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
             r_s[tid] = rr;
             mur[tid] = a.mu / rr;
             dsum[tid] = 0.f;
+            if (ISO) *reinterpret_cast<float4 *>(tsum + tid * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         // thread = key-channel pair cp x 16-token segment sgi; alpha, sigma, k of its tokens
         const int cp = (warp & 1) * 32 + lane, sgi = warp >> 1, ch = cp * 2, tb = sgi * 16;
@@ -280,6 +288,35 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
         if (tid == 0) bulk_wait_read0();   // the previous record's bulk stores have read shared memory
         __syncthreads();
 
+        // isotropic (explainer "各向同性近似"): every channel carries the head's uncertainty, with
+        // the maps of the channel means a = mean alpha^2, s = mean sigma, c = mu |k|^2 / (d_k r)
+        if constexpr (ISO) {
+            float xa[16], xg[16], xk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float a0 = bf16_lo(aw[j]), a1 = bf16_hi(aw[j]), k0 = bf16_lo(kw[j]), k1 = bf16_hi(kw[j]);
+                xa[j] = fmaf(a0, a0, a1 * a1);
+                xg[j] = bf16_lo(sw[j]) + bf16_hi(sw[j]);
+                xk[j] = fmaf(k0, k0, k1 * k1);
+            }
+            int which;
+            const float sa_ = warp_reduce16(xa, lane, which);
+            const float sg_ = warp_reduce16(xg, lane, which);
+            const float sk_ = warp_reduce16(xk, lane, which);
+            if ((lane & 1) == 0 && tb + which < L) {
+                atomicAdd(tsum + (tb + which) * 4 + 0, sa_);
+                atomicAdd(tsum + (tb + which) * 4 + 1, sg_);
+                atomicAdd(tsum + (tb + which) * 4 + 2, sk_);
+            }
+            __syncthreads();
+            if (tid < C) {   // the token's map parameters, in place
+                constexpr float inv_dk = 1.f / DK;
+                const float4 x = *reinterpret_cast<const float4 *>(tsum + tid * 4);
+                *reinterpret_cast<float4 *>(tsum + tid * 4) =
+                    make_float4(x.x * inv_dk, x.y * inv_dk, mur[tid] * x.z * inv_dk, 0.f);
+            }
+            __syncthreads();
+        }
         // ---- segment composites of the uncertainty maps (predict [[a, s],[0,1]], update [[1,0],[c,1]])
         {
             float a00 = 1.f, a01 = 0.f, a10 = 0.f, a11 = 1.f, ga = 1.f;
@@ -288,15 +325,19 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
             for (int j = 0; j < 16; ++j) {
                 if (tb + j < L) {
                     const float mr = mur[tb + j];
+                    float4 iso = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if constexpr (ISO) iso = *reinterpret_cast<const float4 *>(tsum + (tb + j) * 4);
                     {
-                        const float al = bf16_lo(aw[j]), sg = bf16_lo(sw[j]), kk = bf16_lo(kw[j]);
-                        const float aa = al * al, cc = mr * kk * kk;
+                        const float al = bf16_lo(aw[j]), kk = bf16_lo(kw[j]);
+                        const float aa = ISO ? iso.x : al * al, sg = ISO ? iso.y : bf16_lo(sw[j]);
+                        const float cc = ISO ? iso.z : mr * kk * kk;
                         const float y00 = fmaf(aa, a00, sg * a10), y01 = fmaf(aa, a01, sg * a11);
                         a10 = fmaf(cc, y00, a10); a11 = fmaf(cc, y01, a11); a00 = y00; a01 = y01; ga *= al;
                     }
                     {
-                        const float al = bf16_hi(aw[j]), sg = bf16_hi(sw[j]), kk = bf16_hi(kw[j]);
-                        const float aa = al * al, cc = mr * kk * kk;
+                        const float al = bf16_hi(aw[j]), kk = bf16_hi(kw[j]);
+                        const float aa = ISO ? iso.x : al * al, sg = ISO ? iso.y : bf16_hi(sw[j]);
+                        const float cc = ISO ? iso.z : mr * kk * kk;
                         const float y00 = fmaf(aa, b00, sg * b10), y01 = fmaf(aa, b01, sg * b11);
                         b10 = fmaf(cc, y00, b10); b11 = fmaf(cc, y01, b11); b00 = y00; b01 = y01; gb *= al;
                     }
@@ -345,7 +386,7 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
             }
             float p0;
             if (c == 0) {
-                p0 = a.P0 ? a.P0[(size_t)chain * DK + cc] : 1.f;
+                p0 = a.P0 ? a.P0[ISO ? (size_t)chain : (size_t)chain * DK + cc] : 1.f;
             } else {   // walk back: compose aggregates until an end-of-chunk uncertainty
                 float r00 = 1.f, r01 = 0.f, r10 = 0.f;   // composite of the chunks walked over ((1,1) kept at 1)
                 bool timed_out = false;
@@ -385,7 +426,10 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
             pst[cc] = p0;
             const float pe = mob(g00, g01, g10, 1.f, p0);
             st_relaxed(desc + 3 * DK, tagged(pe, TAG_INCL));
-            if (c == nch - 1 && a.P_out) a.P_out[(size_t)chain * DK + cc] = pe;
+            if (c == nch - 1 && a.P_out) {
+                if (!ISO) a.P_out[(size_t)chain * DK + cc] = pe;
+                else if (cc == 0) a.P_out[chain] = pe;
+            }
         }
         __syncthreads();
 
@@ -410,10 +454,20 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
                 if (t < L) {
                     const float ala = bf16_lo(aw[j]), alb = bf16_hi(aw[j]);
                     const float ka = bf16_lo(kw[j]), kb = bf16_hi(kw[j]);
-                    const float pma = fmaf(ala * ala, Pa, bf16_lo(sw[j])), pmb = fmaf(alb * alb, Pb, bf16_hi(sw[j]));
-                    const float mr = mur[t];
-                    Pa = __fdividef(pma, fmaf(mr * ka * ka, pma, 1.f));
-                    Pb = __fdividef(pmb, fmaf(mr * kb * kb, pmb, 1.f));
+                    float pma, pmb;
+                    if constexpr (ISO) {   // the head's map, the same on every channel
+                        const float4 iso = *reinterpret_cast<const float4 *>(tsum + t * 4);
+                        pma = fmaf(iso.x, Pa, iso.y);
+                        pmb = fmaf(iso.x, Pb, iso.y);
+                        Pa = __fdividef(pma, fmaf(iso.z, pma, 1.f));
+                        Pb = __fdividef(pmb, fmaf(iso.z, pmb, 1.f));
+                    } else {
+                        pma = fmaf(ala * ala, Pa, bf16_lo(sw[j]));
+                        pmb = fmaf(alb * alb, Pb, bf16_hi(sw[j]));
+                        const float mr = mur[t];
+                        Pa = __fdividef(pma, fmaf(mr * ka * ka, pma, 1.f));
+                        Pb = __fdividef(pmb, fmaf(mr * kb * kb, pmb, 1.f));
+                    }
                     gama *= ala;
                     gamb *= alb;
                     const float pka = pma * ka, pkb = pmb * kb;
@@ -801,7 +855,10 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
             }
         }
         // a sequence without tokens had no prep unit: its uncertainty passes through here
-        if (nch == 0 && a.P_out && tile == 0 && tid < DK) a.P_out[(size_t)chain * DK + tid] = a.P0 ? a.P0[(size_t)chain * DK + tid] : 1.f;
+        if (nch == 0 && a.P_out && tile == 0) {
+            if (!a.iso && tid < DK) a.P_out[(size_t)chain * DK + tid] = a.P0 ? a.P0[(size_t)chain * DK + tid] : 1.f;
+            else if (a.iso && tid == 0) a.P_out[chain] = a.P0 ? a.P0[chain] : 1.f;
+        }
     } else {
         raise_error(a.err, ERR_TIMEOUT);
     }
@@ -854,20 +911,21 @@ cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long
         e = cudaMemsetAsync(ws, 0, 256 + desc_bytes, st);   // ticket counter and look-back words (untagged)
         if (e != cudaSuccess) return e;
         constexpr size_t psmem = PrepSmem::total + 1024;
-        e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
+        auto prep = a.iso ? chunk_prep_kernel<true> : chunk_prep_kernel<false>;
+        e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
         if (e != cudaSuccess) return e;
         // all of the unified L1 / shared array as shared memory, so that two CTAs fit on an SM
-        e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        e = cudaFuncSetAttribute(prep, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (e != cudaSuccess) return e;
         int dev = 0, sms = 148, per = 1;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, chunk_prep_kernel, PNT, psmem);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, prep, PNT, psmem);
         // two CTAs fit on an SM (registers and shared memory); the occupancy query can report
         // fewer.  Extra CTAs are harmless: units go out by ticket to resident CTAs only.
         long long grid = (long long)sms * (per > 2 ? per : 2);
         if (grid > units) grid = units;
-        chunk_prep_kernel<<<(unsigned)grid, PNT, psmem, st>>>(pa);
+        prep<<<(unsigned)grid, PNT, psmem, st>>>(pa);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -300,8 +300,8 @@ __global__ void __launch_bounds__(NT, 2) gain_scan_tma_kernel(const __grid_const
                     const float pma = fmaf(ala * ala, Pa, bf16_lo(sw)), pmb = fmaf(alb * alb, Pb, bf16_hi(sw));
                     const float pka = pma * ka, pkb = pmb * kb;
                     const float mr = mur[tb + j];
-                    Pa = pma / fmaf(mr * ka, pka, 1.f);
-                    Pb = pmb / fmaf(mr * kb, pkb, 1.f);
+                    Pa = __fdividef(pma, fmaf(mr * ka, pka, 1.f));
+                    Pb = __fdividef(pmb, fmaf(mr * kb, pkb, 1.f));
                     pk[2 * j] = pka;
                     pk[2 * j + 1] = pkb;
                     xs[j] = fmaf(pka, ka, pkb * kb);

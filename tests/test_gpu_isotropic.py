@@ -14,13 +14,17 @@ pytestmark = pytest.mark.gpu
 TOL_F32, TOL_BF16 = 1e-4, 2e-2
 
 
-def run_iso(kdn, w, chunk, mu=1.0, S0=None, P0=None):
+def run_iso(kdn, w, chunk, mu=1.0, S0=None, P0=None, workspace=None):
+    """Isotropic forward; ``workspace`` None allocates one (two-launch tensor-core path where
+    it applies), False passes none (the fused tensor-core kernel)."""
     import torch
     args = [to_dev(dense_shape(w, getattr(w, n))) for n in ("q", "k", "v", "alpha", "sigma", "r")]
     cu = to_dev(w.cu_seqlens) if w.B == 1 and w.num_seqs > 1 else None
-    path = kdn.execution_path(args[0], args[2], cu_seqlens=cu, chunk=chunk, variant="isotropic")
+    max_seqlen = int(np.diff(w.cu_seqlens).max()) if cu is not None else 0
+    path = kdn.execution_path(args[0], args[2], cu_seqlens=cu, chunk=chunk, variant="isotropic",
+                              workspace=workspace is None)
     o, S, P = kdn.forward(*args, cu_seqlens=cu, S0=to_dev(S0), P0=to_dev(P0), mu=mu, chunk=chunk,
-                          variant="isotropic")
+                          variant="isotropic", workspace=workspace, max_seqlen=max_seqlen)
     torch.cuda.synchronize()
     kdn.last_device_error()
     return path, to_host(o).reshape((-1,) + o.shape[2:]), to_host(S), to_host(P)
@@ -39,19 +43,21 @@ def test_iso_tiny_fp32_every_chunk(kdn, chunk, mu):
     assert max_rel_err(P, ref["P"]) <= TOL_F32
 
 
-@pytest.mark.parametrize("dk,dv,chunk", [(128, 64, 64), (128, 128, 64), (128, 256, 64), (64, 128, 64),
-                                         (128, 128, 0), (32, 32, 32)])
-def test_iso_ragged_varlen_bf16_with_initial_state(kdn, dk, dv, chunk):
+@pytest.mark.parametrize("dk,dv,chunk,form", [(128, 64, 64, "two_phase"), (128, 128, 64, "two_phase"),
+                                              (128, 256, 64, "two_phase"), (128, 128, 64, "fused"),
+                                              (128, 256, 64, "fused"), (64, 128, 64, "two_phase"),
+                                              (128, 128, 0, "two_phase"), (32, 32, 32, "two_phase")])
+def test_iso_ragged_varlen_bf16_with_initial_state(kdn, dk, dv, chunk, form):
     """Ragged sequences (1 token, chunk-1, chunk, chunk+1, several chunks and a tail),
-    an empty sequence, carried S0 and p0, mu = 4."""
+    an empty sequence, carried S0 and p0, mu = 4; tensor-core cases in both forms."""
     w = ragged(700 + dk + dv + chunk, [1, 63, 64, 0, 65, 300], 3, dk, dv, True)
     rng = np.random.default_rng(dk + dv)
     S0 = (0.1 * rng.standard_normal((w.num_seqs, w.H, dk, dv))).astype(np.float32)
     P0 = rng.uniform(0.3, 2.0, (w.num_seqs, w.H)).astype(np.float32)
     ref = oracle.iso_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens, S0=S0, P0=P0, mu=4.0)
-    path, o, S, P = run_iso(kdn, w, chunk, mu=4.0, S0=S0, P0=P0)
+    path, o, S, P = run_iso(kdn, w, chunk, mu=4.0, S0=S0, P0=P0, workspace=None if form == "two_phase" else False)
     if chunk == 64 and dk == 128:
-        assert path == "chunk_tcgen05"
+        assert path == ("chunk_tcgen05_two_phase" if form == "two_phase" else "chunk_tcgen05")
     assert max_rel_err(o, ref["o"]) <= TOL_BF16
     assert max_rel_err(S, ref["S"]) <= TOL_BF16
     assert max_rel_err(P, ref["P"]) <= TOL_BF16
@@ -59,18 +65,19 @@ def test_iso_ragged_varlen_bf16_with_initial_state(kdn, dk, dv, chunk):
 
 
 def test_iso_prefill_full_size_sampled(kdn):
-    """The prefill workload (4 x 4096 tokens, 16 heads, d = 128, bf16) on the tcgen05
-    path; sampled chains against the oracle element by element."""
+    """The prefill workload (4 x 4096 tokens, 16 heads, d = 128, bf16) on the tcgen05 path
+    in both forms; sampled chains against the oracle element by element."""
     w = inputs.prefill_4x4096()
-    path, o, S, P = run_iso(kdn, w, 64)
-    assert path == "chunk_tcgen05"
-    o = o.reshape(w.B * w.T, w.H, -1)
     ref = oracle.diag_chains(w, [(0, 0), (2, 7), (3, 15)], iso=True)
-    for (s, h), rr in ref.items():
-        sl = slice(int(w.cu_seqlens[s]), int(w.cu_seqlens[s + 1]))
-        assert max_rel_err(o[sl, h], rr["o"]) <= TOL_BF16
-        assert max_rel_err(S[s, h], rr["S"]) <= TOL_BF16
-        assert max_rel_err(P[s, h], rr["P"]) <= TOL_BF16
+    for workspace, name in ((None, "chunk_tcgen05_two_phase"), (False, "chunk_tcgen05")):
+        path, o, S, P = run_iso(kdn, w, 64, workspace=workspace)
+        assert path == name
+        o = o.reshape(w.B * w.T, w.H, -1)
+        for (s, h), rr in ref.items():
+            sl = slice(int(w.cu_seqlens[s]), int(w.cu_seqlens[s + 1]))
+            assert max_rel_err(o[sl, h], rr["o"]) <= TOL_BF16, (name, s, h)
+            assert max_rel_err(S[s, h], rr["S"]) <= TOL_BF16, (name, s, h)
+            assert max_rel_err(P[s, h], rr["P"]) <= TOL_BF16, (name, s, h)
 
 
 @pytest.mark.parametrize("n", [1, 5])
