@@ -71,13 +71,15 @@ struct PrepSmem {
 
 template <int DVT>
 struct StateSmem {
+    // operand tiles are 64-column swizzle atoms; a 32-column tile uses half of one
+    static constexpr uint32_t W64 = DVT < 64 ? 64 : DVT;
     static constexpr uint32_t STAGE = 67584;               // a record, rounded up to 1 KB
-    static constexpr uint32_t V0 = 2 * STAGE;              // two v tiles, DVT * 128 B each
-    static constexpr uint32_t S = V0 + 2 * DVT * 128;      // S bf16, 128 channel rows x DVT (MN-major)
-    static constexpr uint32_t U = S + DVT * 256;           // U / den bf16, 64 token rows x DVT
-    static constexpr uint32_t CTL = U + DVT * 128;         // 3 mbarriers, TMEM slot
+    static constexpr uint32_t V_BYTES = W64 * 128;         // v tile (64 tokens x W64 columns)
+    static constexpr uint32_t V0 = 2 * STAGE;              // two v tiles
+    static constexpr uint32_t S = V0 + 2 * V_BYTES;        // S bf16, 128 channel rows x DVT (MN-major)
+    static constexpr uint32_t U = S + W64 * 256;           // U / den bf16, 64 token rows x DVT
+    static constexpr uint32_t CTL = U + W64 * 128;         // 3 mbarriers, TMEM slot
     static constexpr uint32_t total = CTL + 64;
-    static constexpr uint32_t V_BYTES = DVT * 128;
 };
 
 struct PrepArgs {
@@ -671,7 +673,8 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
 {
     using L_ = StateSmem<DVT>;
     using namespace tc;
-    constexpr int NC = DVT / 2;   // d_v columns per thread in the epilogues
+    constexpr int NC = DVT / 2;           // d_v columns per thread in the epilogues
+    constexpr int CW = NC < 32 ? NC : 32;  // columns per TMEM load
     extern __shared__ uint8_t smraw[];
     const uint32_t raw_u32 = smem_u32(smraw);
     const uint32_t sb = (raw_u32 + 1023u) & ~1023u;
@@ -716,31 +719,33 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
     const int row = quad * 32 + lane;
     const int cb0 = cg * NC;
 
+    // the v tile: whole 64-column boxes; a 32-column tile is one half of its box
+    const int vx0 = (tile * DVT) & ~63;
+    const uint32_t voff = (uint32_t)((tile * DVT) & 63) * 2u;
     auto issue = [&](int c, int st) {   // record and v tile of chunk c into stage st
         const uint8_t *src = sa.rec + (size_t)((long long)c * sa.nchains + chain) * Rec::BYTES;
         mbar_expect_tx(bar_full + st, Rec::BYTES + L_::V_BYTES);
         bulk_load(sm + st * L_::STAGE, src, Rec::BYTES, bar_full + st);
-        for (int b = 0; b < DVT / 64; ++b)
-            tma_load_3d(sm + L_::V0 + st * L_::V_BYTES + b * 8192, &sa.tv, tile * DVT + b * 64, h, t0 + c * C,
-                        bar_full + st);
+        for (int b = 0; b < (int)(L_::W64 / 64); ++b)
+            tma_load_3d(sm + L_::V0 + st * L_::V_BYTES + b * 8192, &sa.tv, vx0 + b * 64, h, t0 + c * C, bar_full + st);
     };
 
     // initial memory tile -> TMEM (lane = key channel) and its bf16 operand copy
     const size_t sbase = (size_t)chain * DK * dv + (size_t)tile * DVT;
 #pragma unroll
-    for (int p = 0; p < NC / 32; ++p) {
-        float v[32];
-        const int col = cb0 + p * 32;
+    for (int p = 0; p < NC / CW; ++p) {
+        float v[CW];
+        const int col = cb0 + p * CW;
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) {
+        for (int j = 0; j < CW; j += 4) {
             float4 x = a.S0 ? *reinterpret_cast<const float4 *>(a.S0 + sbase + (size_t)row * dv + col + j)
                             : make_float4(0.f, 0.f, 0.f, 0.f);
             v[j] = x.x; v[j + 1] = x.y; v[j + 2] = x.z; v[j + 3] = x.w;
         }
-        tmem_st32(T_S + lane_off + col, v);
+        tmem_st<CW>(T_S + lane_off + col, v);
         const uint32_t atom = (uint32_t)(col >> 6) * 16384u;
 #pragma unroll
-        for (int chn = 0; chn < 4; ++chn)
+        for (int chn = 0; chn < CW / 8; ++chn)
             *reinterpret_cast<uint4 *>(sm + L_::S + atom + swz(row, (((col & 63) >> 3) + chn) * 16)) = pack8(v + chn * 8);
     }
     if (tid == 0 && nch > 0) issue(0, 0);
@@ -781,27 +786,27 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma_bf16(T_D4, sdesc(sb + stg + Rec::Y + ks * 32u, 16, 1024),
-                         sdesc(sb + L_::V0 + st * L_::V_BYTES + ks * 2048u, 8192, 1024), ID_M128_NV_KM, 1);
+                         sdesc(sb + L_::V0 + st * L_::V_BYTES + ks * 2048u + voff, 8192, 1024), ID_M128_NV_KM, 1);
             mma_commit(bar_mma);
         }
         wait_mma();
         // rows 0..63 -> U / den (bf16); rows 64..127 -> o (global, tokens of the chunk)
 #pragma unroll
-        for (int p = 0; p < NC / 32; ++p) {
-            float v[32];
-            const int col = cb0 + p * 32;
-            tmem_ld32(T_D4 + lane_off + col, v);
+        for (int p = 0; p < NC / CW; ++p) {
+            float v[CW];
+            const int col = cb0 + p * CW;
+            tmem_ld<CW>(T_D4 + lane_off + col, v);
             if (row < 64) {
                 const float sc = invden[row];
                 const uint32_t blk = (uint32_t)(col >> 6) * 8192u;
 #pragma unroll
-                for (int chn = 0; chn < 4; ++chn)
+                for (int chn = 0; chn < CW / 8; ++chn)
                     *reinterpret_cast<uint4 *>(sm + L_::U + blk + swz(row, (((col & 63) >> 3) + chn) * 16)) =
                         pack8(v + chn * 8, sc);
             } else if (row - 64 < L) {
                 bf16 *dst = out + ((size_t)(c0 + row - 64) * H + h) * dv + tile * DVT + col;
 #pragma unroll
-                for (int chn = 0; chn < 4; ++chn) *reinterpret_cast<uint4 *>(dst + chn * 8) = pack8(v + chn * 8);
+                for (int chn = 0; chn < CW / 8; ++chn) *reinterpret_cast<uint4 *>(dst + chn * 8) = pack8(v + chn * 8);
             }
         }
         fence_async_smem();
@@ -821,16 +826,16 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
         {
             const float gC = gamc[row];
 #pragma unroll
-            for (int p = 0; p < NC / 32; ++p) {
-                float v[32];
-                const int col = cb0 + p * 32;
-                tmem_ld32(T_S + lane_off + col, v);
+            for (int p = 0; p < NC / CW; ++p) {
+                float v[CW];
+                const int col = cb0 + p * CW;
+                tmem_ld<CW>(T_S + lane_off + col, v);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] *= gC;
-                tmem_st32(T_S + lane_off + col, v);
+                for (int j = 0; j < CW; ++j) v[j] *= gC;
+                tmem_st<CW>(T_S + lane_off + col, v);
                 const uint32_t atom = (uint32_t)(col >> 6) * 16384u;
 #pragma unroll
-                for (int chn = 0; chn < 4; ++chn)
+                for (int chn = 0; chn < CW / 8; ++chn)
                     *reinterpret_cast<uint4 *>(sm + L_::S + atom + swz(row, (((col & 63) >> 3) + chn) * 16)) =
                         pack8(v + chn * 8);
             }
@@ -844,12 +849,12 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
     if (!*abort_flag) {
         if (a.S_out) {
 #pragma unroll
-            for (int p = 0; p < NC / 32; ++p) {
-                float v[32];
-                const int col = cb0 + p * 32;
-                tmem_ld32(T_S + lane_off + col, v);
+            for (int p = 0; p < NC / CW; ++p) {
+                float v[CW];
+                const int col = cb0 + p * CW;
+                tmem_ld<CW>(T_S + lane_off + col, v);
 #pragma unroll
-                for (int j = 0; j < 32; j += 4)
+                for (int j = 0; j < CW; j += 4)
                     *reinterpret_cast<float4 *>(a.S_out + sbase + (size_t)row * dv + col + j) =
                         make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
             }
@@ -929,8 +934,19 @@ cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    const int dvt = (a.dv == 64 || nchains * (a.dv / 128) < 148) ? 64 : 128;
+    // the narrowest d_v tile whose CTAs still fit on the SMs at one per SM (more chains in flight,
+    // shorter MMAs and epilogues); with more chains than that, the widest
+    int sms = 148;
+    {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    int dvt = a.dv < 128 ? a.dv : 128;
+    for (int w = 32; w <= dvt; w *= 2)
+        if (nchains * (a.dv / w) <= sms) { dvt = w; break; }
     const unsigned sgrid = (unsigned)(nchains * (a.dv / dvt));
+    if (dvt == 32) return launch_state<32>(sa, sgrid, st);
     return dvt == 64 ? launch_state<64>(sa, sgrid, st) : launch_state<128>(sa, sgrid, st);
 }
 

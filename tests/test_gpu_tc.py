@@ -38,6 +38,18 @@ def test_tc_dense_ragged_tail(kdn, dv, form):
     assert max_rel_err(P, ref["P"]) <= TOL_BF16
 
 
+@pytest.mark.parametrize("H", [20, 80])
+def test_tc_two_phase_wider_dv_tiles(kdn, H):
+    """Enough (sequence, head) chains that the state kernel takes 64- (H=20) and 128-column
+    (H=80) d_v tiles (the small cases above take 32), with a ragged tail."""
+    w = inputs.dense("tc_tiles", 40 + H, 2, H, 136, 128, 128, bf16=True)   # 136 = 2 chunks + 8
+    ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens, mu=2.0)
+    o, S, P = run_forward(kdn, w, chunk=64, mu=2.0)
+    assert max_rel_err(o, ref["o"]) <= TOL_BF16
+    assert max_rel_err(S, ref["S"]) <= TOL_BF16
+    assert max_rel_err(P, ref["P"]) <= TOL_BF16
+
+
 @pytest.mark.parametrize("form", sorted(FORMS))
 @pytest.mark.parametrize("mu", [1.0, 128.0])
 def test_tc_varlen_with_initial_state(kdn, mu, form):
