@@ -69,10 +69,15 @@ bool tc_path(const kdn_problem_t *p, const Resolved &rv) {
 }
 // ... and the two-launch form applies (work list within 2^31 units)
 bool two_phase_path(const kdn_problem_t *p, const Resolved &rv) {
-    return tc_path(p, rv) && (long long)rv.nseq * p->H * rv.nchunks_max < (1ll << 31);
+    const long long units = p->cu_seqlens ? (rv.ntok / 64 + rv.nseq) * p->H : (long long)rv.nseq * p->H * rv.nchunks_max;
+    return tc_path(p, rv) && units < (1ll << 31);
 }
 size_t two_phase_bytes(const kdn_problem_t *p, const Resolved &rv) {
-    return kdn::two_phase_workspace_bytes((long long)rv.nseq * p->H, rv.nchunks_max);
+    if (p->cu_seqlens) {   // packed: sum_s ceil(len_s / 64) <= T / 64 + num_seqs units per head
+        const long long units = (rv.ntok / 64 + rv.nseq) * p->H;
+        return kdn::two_phase_workspace_bytes(units, (rv.ntok + 63) / 64, rv.nseq);
+    }
+    return kdn::two_phase_workspace_bytes((long long)rv.nseq * p->H * rv.nchunks_max, 0, 0);
 }
 
 }  // namespace

@@ -82,6 +82,18 @@ struct StateSmem {
     static constexpr uint32_t total = CTL + 64;
 };
 
+// Units of packed (varlen) problems are numbered densely, chunk-major over the chunks that exist,
+// with the sequences of each chunk level in order of length (longest first):
+//     unit (c, s, h) = U[c] + pos[s] * H + h      (for c < the sequence's chunk count)
+// U[c] = H x #{(c', s) : c' < c, chunks(s) > c'}; pos = rank of s by chunk count, order = pos^-1.
+// Dense batches use unit = c * nchains + chain.
+struct UnitTable {
+    long long *U;      // [cmax + 1]; U[cmax] = number of units
+    int *order, *pos;  // [nseq]
+    int *hist, *fill;  // [cmax + 1] scratch of the table kernel
+    int cmax;          // ceil(T / 64): bounds every sequence's chunk count
+};
+
 struct PrepArgs {
     TokenArgs a;
     long long nchunks_max;
@@ -89,6 +101,9 @@ struct PrepArgs {
     unsigned *counter;
     unsigned long long *desc;   // per unit [4][128] tagged words: aggregate map (m00, m01, m10), end-of-chunk P
     uint8_t *rec;     // per unit Rec::BYTES
+    const long long *U;         // varlen unit table (NULL: dense numbering)
+    const int *order, *pos;
+    int cmax;
 };
 
 struct StateArgs {
@@ -97,6 +112,8 @@ struct StateArgs {
     const uint8_t *rec;
     long long nchunks_max;
     int nchains;
+    const long long *U;         // varlen unit table (NULL: dense numbering)
+    const int *order;
 };
 
 __device__ __forceinline__ float mob(float m00, float m01, float m10, float m11, float x) {
@@ -165,7 +182,7 @@ __device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane, int &wh
 }  // namespace
 
 // ================================================================= prep
-template <bool ISO>
+template <bool ISO, bool PACKED>
 __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constant__ PrepArgs pa)
 {
     using L_ = PrepSmem;
@@ -198,7 +215,9 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, cg = warp >> 2;     // TMEM lane quadrant, column half
     const int H = a.H;
-    const long long units = pa.nchunks_max * pa.nchains;
+    constexpr bool packed = PACKED;   // packed (varlen) unit numbering through the unit table
+    const long long units = packed ? pa.U[pa.cmax] : pa.nchunks_max * pa.nchains;
+    int level = 0;   // packed: this CTA's chunk level (its tickets only grow)
 
     if (tid == 0) {
         mbar_init(bar_mma, 1);
@@ -255,12 +274,22 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
         __syncthreads();
         const long long u = *ticket;
         if (u >= units || ctl[1]) break;
-        const int c = (int)(u / pa.nchains), chain = (int)(u % pa.nchains);
+        int c, chain, rank = 0;
+        if constexpr (PACKED) {
+            while (level < pa.cmax && pa.U[level + 1] <= u) ++level;
+            c = level;
+            const int idx = (int)(u - pa.U[c]);
+            rank = idx / H;
+            chain = pa.order[rank] * H + idx % H;
+        } else {
+            c = (int)(u / pa.nchains);
+            chain = (int)(u % pa.nchains);
+        }
         const int s = chain / H, h = chain % H;
         int t0, t1;
         seq_range(a, s, t0, t1);
         const int nch = (t1 - t0 + C - 1) / C;
-        if (c == 0 && tid == 0 && nch > pa.nchunks_max) raise_error(a.err, ERR_ARG);
+        if (!packed && c == 0 && tid == 0 && nch > pa.nchunks_max) raise_error(a.err, ERR_ARG);
         if (c >= nch) {
             __syncthreads();   // every thread has read the ticket before it is replaced
             continue;
@@ -393,7 +422,8 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
                 float r00 = 1.f, r01 = 0.f, r10 = 0.f;   // composite of the chunks walked over ((1,1) kept at 1)
                 bool timed_out = false;
                 for (int j = c - 1;; --j) {
-                    const unsigned long long *dj = pa.desc + ((size_t)j * pa.nchains + chain) * 4 * DK + cc;
+                    const long long uj = packed ? pa.U[j] + (long long)rank * H + h : (long long)j * pa.nchains + chain;
+                    const unsigned long long *dj = pa.desc + (size_t)uj * 4 * DK + cc;
                     unsigned long long w0 = 0ull, w1 = 0ull, w2 = 0ull, w3 = ld_relaxed(dj + 3 * DK);
                     const long long ts = clock64();
                     while (tag_of(w3) != TAG_INCL) {
@@ -688,7 +718,10 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
     bf16 *__restrict__ out = static_cast<bf16 *>(a.o);
     const int ntiles = a.dv / DVT;
     const int tile = blockIdx.x % ntiles;
-    const int chain = blockIdx.x / ntiles;
+    const bool packed = sa.U != nullptr;
+    // packed problems: chains in order of length, longest first (the long chains start first)
+    const int rank = packed ? (int)(blockIdx.x / ntiles) / a.H : 0;
+    const int chain = packed ? sa.order[rank] * a.H + (int)(blockIdx.x / ntiles) % a.H : (int)(blockIdx.x / ntiles);
     const int s = chain / a.H, h = chain % a.H;
     int t0, t1;
     seq_range(a, s, t0, t1);
@@ -696,7 +729,7 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, cg = warp >> 2;
     const int H = a.H, dv = a.dv;
-    if (nch > sa.nchunks_max) {   // records exist for nchunks_max chunks only
+    if (!packed && nch > sa.nchunks_max) {   // records exist for nchunks_max chunks only
         if (tid == 0) raise_error(a.err, ERR_ARG);
         nch = (int)sa.nchunks_max;
     }
@@ -723,7 +756,8 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
     const int vx0 = (tile * DVT) & ~63;
     const uint32_t voff = (uint32_t)((tile * DVT) & 63) * 2u;
     auto issue = [&](int c, int st) {   // record and v tile of chunk c into stage st
-        const uint8_t *src = sa.rec + (size_t)((long long)c * sa.nchains + chain) * Rec::BYTES;
+        const long long uc = packed ? sa.U[c] + (long long)rank * H + h : (long long)c * sa.nchains + chain;
+        const uint8_t *src = sa.rec + (size_t)uc * Rec::BYTES;
         mbar_expect_tx(bar_full + st, Rec::BYTES + L_::V_BYTES);
         bulk_load(sm + st * L_::STAGE, src, Rec::BYTES, bar_full + st);
         for (int b = 0; b < (int)(L_::W64 / 64); ++b)
@@ -872,10 +906,72 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+// ================================================================= unit table (packed problems)
+// One CTA: chunk counts of the sequences, their histogram, U by two block-wide prefix sums,
+// and the ranks of the sequences by chunk count (equal counts in any order).
+__global__ void __launch_bounds__(1024) unit_table_kernel(const int32_t *__restrict__ cu, int nseq, int H, UnitTable t)
+{
+    constexpr int NTH = 1024;
+    __shared__ long long part[NTH];
+    const int tid = threadIdx.x;
+    const int n = t.cmax + 1;
+    for (int i = tid; i < n; i += NTH) { t.hist[i] = 0; t.fill[i] = 0; }
+    __syncthreads();
+    for (int q = tid; q < nseq; q += NTH) {
+        const int nc = min((__ldg(cu + q + 1) - __ldg(cu + q) + C - 1) / C, t.cmax);
+        atomicAdd(t.hist + nc, 1);
+    }
+    __syncthreads();
+    const int per = (n + NTH - 1) / NTH, b = min(n, tid * per), e = min(n, b + per);
+    // exclusive prefix over the threads' partial sums (Hillis-Steele in shared memory)
+    auto block_exclusive = [&](long long own) -> long long {
+        part[tid] = own;
+        __syncthreads();
+        for (int off = 1; off < NTH; off <<= 1) {
+            const long long x = tid >= off ? part[tid - off] : 0;
+            __syncthreads();
+            part[tid] += x;
+            __syncthreads();
+        }
+        const long long incl = part[tid];
+        __syncthreads();
+        return incl - own;
+    };
+    // sequences with more than c chunks: nseq - (inclusive prefix of the histogram at c)
+    long long acc = 0;
+    for (int i = b; i < e; ++i) acc += t.hist[i];
+    acc = block_exclusive(acc);
+    for (int i = b; i < e; ++i) { acc += t.hist[i]; t.U[i] = acc; }
+    __syncthreads();
+    for (int i = b; i < e; ++i) t.hist[i] = nseq - (int)t.U[i];
+    __syncthreads();
+    // U[c] = H x (units of the chunk levels below c)
+    acc = 0;
+    for (int i = b; i < e; ++i) acc += t.hist[i];
+    acc = block_exclusive(acc);
+    for (int i = b; i < e; ++i) { t.U[i] = (long long)H * acc; acc += t.hist[i]; }
+    __syncthreads();
+    // rank = sequences with more chunks + place among the equal ones
+    for (int q = tid; q < nseq; q += NTH) {
+        const int nc = min((__ldg(cu + q + 1) - __ldg(cu + q) + C - 1) / C, t.cmax);
+        const int r = t.hist[nc] + atomicAdd(t.fill + nc, 1);
+        t.pos[q] = r;
+        t.order[r] = q;
+    }
+}
+
 // ================================================================= host side
-size_t two_phase_workspace_bytes(long long nchains, long long nchunks_max) {
-    const long long units = nchains * nchunks_max;
-    return 256 + (size_t)units * 4 * DK * 8 + (size_t)units * Rec::BYTES;
+namespace {
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+size_t table_bytes(long long cmax, long long nseq) {
+    return round256((size_t)(cmax + 1) * 8) + 2 * round256((size_t)nseq * 4) + 2 * round256((size_t)(cmax + 1) * 4);
+}
+}  // namespace
+
+// units: upper bound of the number of units; cmax > 0 for packed problems (their unit table)
+size_t two_phase_workspace_bytes(long long units, long long cmax, long long nseq) {
+    const size_t table = cmax > 0 ? table_bytes(cmax, nseq) : 0;
+    return 256 + table + (size_t)units * 4 * DK * 8 + (size_t)units * Rec::BYTES;
 }
 
 template <int DVT>
@@ -892,31 +988,62 @@ cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long
                                    cudaStream_t st) {
     const long long nchains = (long long)a.nseq * a.H;
     if (nchains == 0) return cudaSuccess;
-    const long long units = nchains * nchunks_max;
+    const bool packed = a.cu != nullptr;
+    // packed: sum_s ceil(len_s / 64) <= T / 64 + nseq units per head
+    const long long cmax = packed ? (ntok + C - 1) / C : 0;
+    const long long units = packed ? (ntok / C + a.nseq) * a.H : nchains * nchunks_max;
     const size_t desc_bytes = (size_t)units * 4 * DK * 8;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint8_t *tab = ws + 256;
+    const size_t tbytes = packed ? table_bytes(cmax, a.nseq) : 0;
 
     PrepArgs pa;
     pa.a = a;
     pa.nchunks_max = nchunks_max;
     pa.nchains = (int)nchains;
     pa.counter = reinterpret_cast<unsigned *>(ws);
-    pa.desc = reinterpret_cast<unsigned long long *>(ws + 256);
-    pa.rec = ws + 256 + desc_bytes;
+    pa.desc = reinterpret_cast<unsigned long long *>(ws + 256 + tbytes);
+    pa.rec = ws + 256 + tbytes + desc_bytes;
+    pa.U = nullptr;
+    pa.order = nullptr;
+    pa.pos = nullptr;
+    pa.cmax = (int)cmax;
+    UnitTable t{};
+    if (packed) {
+        t.U = reinterpret_cast<long long *>(tab);
+        t.order = reinterpret_cast<int *>(tab + round256((size_t)(cmax + 1) * 8));
+        t.pos = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(t.order) + round256((size_t)a.nseq * 4));
+        t.hist = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(t.pos) + round256((size_t)a.nseq * 4));
+        t.fill = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(t.hist) + round256((size_t)(cmax + 1) * 4));
+        t.cmax = (int)cmax;
+        pa.U = t.U;
+        pa.order = t.order;
+        pa.pos = t.pos;
+    }
 
     StateArgs sa;
     sa.a = a;
     sa.rec = pa.rec;
     sa.nchunks_max = nchunks_max;
     sa.nchains = (int)nchains;
+    sa.U = pa.U;
+    sa.order = pa.order;
     if (!make_token_map(&sa.tv, a.v, a.dv, a.H, ntok)) return cudaErrorInvalidValue;
 
     cudaError_t e = cudaSuccess;
     if (units > 0) {
-        e = cudaMemsetAsync(ws, 0, 256 + desc_bytes, st);   // ticket counter and look-back words (untagged)
+        e = cudaMemsetAsync(ws, 0, 256, st);   // ticket counter
         if (e != cudaSuccess) return e;
+        e = cudaMemsetAsync(pa.desc, 0, desc_bytes, st);   // look-back words (untagged)
+        if (e != cudaSuccess) return e;
+        if (packed) {
+            unit_table_kernel<<<1, 1024, 0, st>>>(a.cu, a.nseq, a.H, t);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
         constexpr size_t psmem = PrepSmem::total + 1024;
-        auto prep = a.iso ? chunk_prep_kernel<true> : chunk_prep_kernel<false>;
+        auto prep = a.iso ? (packed ? chunk_prep_kernel<true, true> : chunk_prep_kernel<true, false>)
+                          : (packed ? chunk_prep_kernel<false, true> : chunk_prep_kernel<false, false>);
         e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
         if (e != cudaSuccess) return e;
         // all of the unified L1 / shared array as shared memory, so that two CTAs fit on an SM

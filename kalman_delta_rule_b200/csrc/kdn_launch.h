@@ -22,7 +22,8 @@ cudaError_t launch_chunk_tc(const TokenArgs &a, long long ntok, int dvt, cudaStr
 // the same algebra in two launches: a chunk-parallel prep kernel (uncertainty by decoupled
 // look-back, intra-chunk matrices, triangular inverse) writing per-chunk operand records to
 // the workspace, then the chunk-serial state kernel
-size_t two_phase_workspace_bytes(long long nchains, long long nchunks_max);
+// units: upper bound of the (chunk, sequence x head) units; cmax > 0 for packed problems
+size_t two_phase_workspace_bytes(long long units, long long cmax, long long nseq);
 cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long nchunks_max, void *workspace,
                                    cudaStream_t st);
 // [ntok, H, d] bf16 as a TMA tensor map with 64 x 1 x 64 boxes and 128-byte swizzle
