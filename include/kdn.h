@@ -84,14 +84,16 @@ typedef struct {
     float mu;                       /* information scaling, > 0 */
     int chunk;                      /* execution path, see above */
     int max_seqlen;                 /* varlen: upper bound on every sequence length (0 = unknown, taken as T);
-                                       sizes the gain scan's work list.  A sequence longer than it makes
-                                       kdn_gain_scan record KDN_ERR_INVALID_ARG in the device error word. */
+                                       sizes only the gain scan's work list (the forward needs no bound).  A
+                                       sequence longer than it makes kdn_gain_scan record KDN_ERR_INVALID_ARG
+                                       in the device error word. */
     int variant;                    /* kdn_variant_t; 0 (zero-initialised struct) = diagonal */
 } kdn_problem_t;
 
 /* Bytes of device workspace for `p`: the larger of what kdn_gain_scan() and the two-launch
- * tensor-core forward use (about 68 KB per 64-token chunk and head: per-chunk operand
- * records and look-back state; `max_seqlen` bounds it for packed sequences).  The forward
+ * tensor-core forward use.  The forward's part is about 70 KB per 64-token chunk and head
+ * (per-chunk operand records and look-back state); packed sequences hold at most
+ * T/64 + num_seqs chunks per head, so it does not depend on `max_seqlen`.  The forward
  * also accepts workspace = NULL and then runs the single-kernel paths.  Host-only. */
 kdn_status_t kdn_workspace_size(const kdn_problem_t *p, size_t *bytes);
 
