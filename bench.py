@@ -333,9 +333,53 @@ def bench_prefill(args, world, rank, dev, kdn):
         s_bytes = w.ntok * w.H * (3 * w.dk * esz + esz + w.dk * 4 + 4) + w.num_seqs * w.H * w.dk * 4
         scan = dict(value=world * w.ntok / (s_ms / 1e3), ms_step=s_ms, bytes=s_bytes, launches=args.steps)
 
+    # the backward pass (gradients of <o, d_o> with respect to every input, S0 and P0) on the
+    # same inputs, d_o drawn once on the device
+    bwd = None
+    if not args.no_backward:
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(1234 + rank)
+        d_o = torch.randn(o.shape, generator=gen, device=dev).to(o.dtype)
+        f32 = dict(dtype=torch.float32, device=dev)
+        grads = dict(dq=torch.empty(d["q"].shape, **f32), dk=torch.empty(d["k"].shape, **f32),
+                     dv=torch.empty(d["v"].shape, **f32), dalpha=torch.empty(d["alpha"].shape, **f32),
+                     dsigma=torch.empty(d["sigma"].shape, **f32), dr=torch.empty(d["r"].shape, **f32),
+                     dS0=torch.empty((w.num_seqs, w.H, w.dk, w.dv), **f32), dP0=torch.empty((w.num_seqs, w.H, w.dk), **f32))
+        bp = kdn.make_problem(d["q"], d["v"], cu_seqlens=cu, mu=w.mu, chunk=0)
+        ws_bwd = torch.empty(kdn.kdn_backward_workspace_size(bp), dtype=torch.uint8, device=dev)
+        bargs = [d[n].data_ptr() for n in names]
+        gptr = [grads[n].data_ptr() for n in ("dq", "dk", "dv", "dalpha", "dsigma", "dr", "dS0", "dP0")]
+        sh = stream.cuda_stream or None
+
+        def bwd_step():
+            st = kdn.kdn_backward(bp, *bargs, None, None, d_o.data_ptr(), None, None, *gptr,
+                                  ws_bwd.data_ptr(), ws_bwd.numel(), sh)
+            if st != kdn.KDN_OK:
+                raise kdn.KdnError(st, "kdn_backward")
+
+        for _ in range(2):
+            bwd_step()
+        kdn.last_device_error()
+        barrier(world)
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_bwd = 3
+        b0.record(stream)
+        for _ in range(n_bwd):
+            bwd_step()
+        b1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        kdn.last_device_error()
+        b_ms = max_over_ranks(b0.elapsed_time(b1), world) / n_bwd
+        esz = 2 if w.bf16 else 4
+        b_bytes = (w.ntok * w.H * ((4 * w.dk + 2 * w.dv + 1) * esz + (4 * w.dk + w.dv + 1) * 4)
+                   + w.num_seqs * w.H * (w.dk * w.dv + w.dk) * 4)
+        del ws_bwd
+        bwd = dict(value=world * w.ntok / (b_ms / 1e3), ms_step=b_ms, bytes=b_bytes, launches=3 * n_bwd)
+
     nbytes = algorithmic_bytes(w)
     return dict(w=w, value=value, ms_step=ms_step, per_step_ms=per_step_ms, clocks=clk.summary(), path=path, scan=scan,
-                single=single, iso=iso,
+                single=single, iso=iso, bwd=bwd,
                 e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                          steps=e_steps),
                 bytes=nbytes, launches=args.steps * launches_per_step)
@@ -501,6 +545,16 @@ def ours(args):
                                  "roofline": {"bound": "hbm", "achieved": sach, "peak": hbm, "unit": "GB/s",
                                               "frac": sach / hbm, "traffic": None,
                                               "algorithmic_bytes_per_launch": sc["bytes"]}}
+        if pre["bwd"] is not None:
+            bw = pre["bwd"]
+            bach = bw["bytes"] / (bw["ms_step"] / 1e3) / 1e9
+            line["backward"] = {"metric": "backward tokens/s (gradients of o w.r.t. q, k, v, alpha, sigma, r, S0, P0)",
+                                "value": bw["value"], "unit": "tokens/s", "ms_per_step": bw["ms_step"],
+                                "gpu_launches": bw["launches"], "dtype": "f32 (bf16 inputs widened)",
+                                "roofline": {"bound": "hbm", "achieved": bach, "peak": hbm, "unit": "GB/s",
+                                             "frac": bach / hbm, "traffic": None,
+                                             "algorithmic_bytes_per_launch": bw["bytes"],
+                                             "unit_of_measure": "one backward call = its three launches"}}
         if dec is not None:
             dach = dec["bytes"] / (dec["ms_step"] / 1e3) / 1e9
             line["decode"] = {"metric": "decode steps/s", "value": dec["value"], "unit": "steps/s",
@@ -583,6 +637,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-scan", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=1024)
     args = ap.parse_args()
     if args.warmup < 3:

@@ -191,6 +191,37 @@ kdn_status_t kdn_gain_scan_noalloc(const kdn_problem_t *p,
                                    const void *k, const void *alpha, const void *sigma, const void *r,
                                    const float *P0, float *g, float *beta_eff, float *P_out, void *stream);
 
+/* Backward pass of the diagonal KDN, for training (KDA article, "chunkwise" section: the
+ * chunkwise regime serves training; explainer "对角近似" for the recurrence differentiated).
+ * Computes the gradients of  L = <o, d_o> + <S_T, dS_T> + <P_T, dP_T>, where o, S_T and P_T are
+ * what kdn_forward_chunkwise() returns for the same problem and inputs, with respect to every
+ * input: the vector-Jacobian products of one training step.
+ *  p                  : as for the forward (variant must be KDN_VARIANT_DIAGONAL, else
+ *                       KDN_ERR_UNSUPPORTED; `chunk` and `max_seqlen` are ignored)
+ *  q ... P0           : the forward's inputs, same layouts (S0 / P0 NULL = 0 / 1)
+ *  d_o                : device [B, T, H, d_v] (in_dtype), gradient of L with respect to o
+ *  dS_T, dP_T         : device fp32 [N, H, d_k, d_v], [N, H, d_k], gradients with respect to the
+ *                       final S and P, or NULL (zero)
+ *  dq, dk, dalpha, dsigma : device fp32 [B, T, H, d_k];  dv : device fp32 [B, T, H, d_v]
+ *  dr                 : device fp32 [B, T, H]
+ *  dS0, dP0           : device fp32 [N, H, d_k, d_v], [N, H, d_k], or NULL (not written)
+ *  workspace          : device, >= kdn_backward_workspace_size() bytes, 256-byte aligned
+ *                       (contents on entry do not matter; distinct per concurrent call).
+ * Method: the uncertainty forward is taped (P before each token, den, g), the memory forward
+ * is checkpointed every 32 tokens, and the reverse sweep recomputes each chunk from its
+ * checkpoint (the state before every token is re-stepped forward, never reconstructed by
+ * dividing by alpha); fp32 CUDA-core arithmetic.  Every pointer 16-byte aligned.  Outputs may
+ * not alias inputs.  Asynchronous on `stream`; errors as for the forward. */
+kdn_status_t kdn_backward_workspace_size(const kdn_problem_t *p, size_t *bytes);
+kdn_status_t kdn_backward(const kdn_problem_t *p,
+                          const void *q, const void *k, const void *v,
+                          const void *alpha, const void *sigma, const void *r,
+                          const float *S0, const float *P0,
+                          const void *d_o, const float *dS_T, const float *dP_T,
+                          float *dq, float *dk, float *dv, float *dalpha, float *dsigma, float *dr,
+                          float *dS0, float *dP0,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
 /* Which execution path kdn_forward_chunkwise() takes for `p` (host-only; no CUDA call
  * besides resolving the driver's tensor-map encoder once): 0 token-serial recurrence,
  * 1 fp32 CUDA-core chunk kernel, 2 tcgen05 tensor-core chunk kernel, 3 the tcgen05 path in

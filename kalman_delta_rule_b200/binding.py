@@ -1,9 +1,9 @@
 """Thin Python binding of libkdn.so (the C ABI declared in include/kdn.h).
 
 The raw functions keep the C names (``kdn_forward_chunkwise``, ``kdn_decode_step``,
-``kdn_gain_scan``, ``kdn_workspace_size``, ``kdn_last_device_error``,
+``kdn_gain_scan``, ``kdn_backward``, ``kdn_workspace_size``, ``kdn_last_device_error``,
 ``kdn_status_string``, ``kdn_version``) and take plain integers for pointers.
-``forward``, ``decode_step`` and ``gain_scan`` marshal torch CUDA tensors into those
+``forward``, ``backward``, ``decode_step`` and ``gain_scan`` marshal torch CUDA tensors into those
 calls: they allocate outputs and workspace with torch and pass the current stream.
 Every step of the computation runs in the library's kernels; there is no CPU or
 PyTorch fallback -- a missing library or device raises.
@@ -53,6 +53,8 @@ _SIGS = {
     "kdn_version": (ctypes.c_char_p, []),
     "kdn_execution_path": (_i, [_PP]),
     "kdn_gain_scan_noalloc": (_i, [_PP] + [_vp] * 4 + [_vp] + [_vp] * 3 + [_vp]),
+    "kdn_backward_workspace_size": (_i, [_PP, ctypes.POINTER(_sz)]),
+    "kdn_backward": (_i, [_PP] + [_vp] * 6 + [_vp] * 2 + [_vp] * 3 + [_vp] * 6 + [_vp] * 2 + [_vp, _sz, _vp]),
 }
 
 
@@ -108,6 +110,20 @@ def kdn_gain_scan_noalloc(problem, k, alpha, sigma, r, P0, g, beta_eff, P_out, s
     """The gain scan on the library's fixed scratch array: for callers that cannot
     allocate device memory when they call (no workspace argument)."""
     return load().kdn_gain_scan_noalloc(ctypes.byref(problem), k, alpha, sigma, r, P0, g, beta_eff, P_out, stream)
+
+
+def kdn_backward_workspace_size(problem: kdn_problem_t) -> int:
+    n = ctypes.c_size_t(0)
+    st = load().kdn_backward_workspace_size(ctypes.byref(problem), ctypes.byref(n))
+    if st != KDN_OK:
+        raise KdnError(st, "kdn_backward_workspace_size")
+    return n.value
+
+
+def kdn_backward(problem, q, k, v, alpha, sigma, r, S0, P0, d_o, dS_T, dP_T, dq, dk, dv, dalpha, dsigma, dr,
+                 dS0, dP0, workspace, workspace_bytes, stream):
+    return load().kdn_backward(ctypes.byref(problem), q, k, v, alpha, sigma, r, S0, P0, d_o, dS_T, dP_T,
+                               dq, dk, dv, dalpha, dsigma, dr, dS0, dP0, workspace, workspace_bytes, stream)
 
 
 def kdn_last_device_error(stream=None) -> int:
@@ -208,6 +224,37 @@ def forward(q, k, v, alpha, sigma, r, cu_seqlens=None, S0=None, P0=None, mu: flo
                                _ptr(o), _ptr(S_out), _ptr(P_out), _ptr(workspace), wbytes, _stream_handle(stream))
     _check(st, "kdn_forward_chunkwise")
     return o, S_out, P_out
+
+
+def backward(q, k, v, alpha, sigma, r, d_o, cu_seqlens=None, S0=None, P0=None, dS=None, dP=None, mu: float = 1.0,
+             workspace=None, want_initial: bool = True, stream=None):
+    """Run kdn_backward on torch tensors laid out as for ``forward``.
+
+    Returns a dict of fp32 gradients of <o, d_o> + <S_T, dS> + <P_T, dP>: dq, dk, dv,
+    dalpha, dsigma ([B,T,H,d]), dr ([B,T,H]) and, with ``want_initial``, dS0 [N,H,dk,dv]
+    and dP0 [N,H,dk].  The workspace is allocated when not given."""
+    torch = _torch()
+    if d_o.dtype != q.dtype:
+        raise ValueError("d_o must have the dtype of the inputs")
+    p = make_problem(q, v, cu_seqlens=cu_seqlens, mu=mu, chunk=0)
+    N = p.num_seqs
+    dev = q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = dict(dq=torch.empty(q.shape, **f32), dk=torch.empty(k.shape, **f32), dv=torch.empty(v.shape, **f32),
+               dalpha=torch.empty(alpha.shape, **f32), dsigma=torch.empty(sigma.shape, **f32),
+               dr=torch.empty(r.shape, **f32))
+    if want_initial:
+        out["dS0"] = torch.empty((N, p.H, p.d_k, p.d_v), **f32)
+        out["dP0"] = torch.empty((N, p.H, p.d_k), **f32)
+    if workspace is None:
+        workspace = torch.empty(kdn_backward_workspace_size(p), dtype=torch.uint8, device=dev)
+    wbytes = workspace.numel() * workspace.element_size()
+    st = kdn_backward(p, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(sigma), _ptr(r), _ptr(S0), _ptr(P0),
+                      _ptr(d_o), _ptr(dS), _ptr(dP), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                      _ptr(out["dalpha"]), _ptr(out["dsigma"]), _ptr(out["dr"]), _ptr(out.get("dS0")),
+                      _ptr(out.get("dP0")), _ptr(workspace), wbytes, _stream_handle(stream))
+    _check(st, "kdn_backward")
+    return out
 
 
 def decode_step(q, k, v, alpha, sigma, r, S, P, mu: float = 1.0, o=None, stream=None, variant: str = "diagonal"):

@@ -235,6 +235,46 @@ kdn_status_t kdn_gain_scan_noalloc(const kdn_problem_t *p, const void *k, const 
     return cuda_status(kdn::launch_gain_scan_noalloc(a, rv.bf16, rv.ntok, static_cast<cudaStream_t>(stream)));
 }
 
+kdn_status_t kdn_backward_workspace_size(const kdn_problem_t *p, size_t *bytes) {
+    Resolved rv;
+    kdn_status_t st = check_problem(p, &rv);
+    if (st != KDN_OK) return st;
+    if (p->variant != KDN_VARIANT_DIAGONAL) return KDN_ERR_UNSUPPORTED;
+    if (!bytes) return KDN_ERR_INVALID_ARG;
+    *bytes = kdn::backward_workspace_bytes(rv.ntok, rv.nseq, p->H, p->d_k, p->d_v);
+    return KDN_OK;
+}
+
+kdn_status_t kdn_backward(const kdn_problem_t *p, const void *q, const void *k, const void *v, const void *alpha,
+                          const void *sigma, const void *r, const float *S0, const float *P0, const void *d_o,
+                          const float *dS_T, const float *dP_T, float *dq, float *dk, float *dv, float *dalpha,
+                          float *dsigma, float *dr, float *dS0, float *dP0, void *workspace, size_t workspace_bytes,
+                          void *stream) {
+    Resolved rv;
+    kdn_status_t st = check_problem(p, &rv);
+    if (st != KDN_OK) return st;
+    if (p->variant != KDN_VARIANT_DIAGONAL) return KDN_ERR_UNSUPPORTED;
+    if (rv.nseq == 0) return KDN_OK;
+    if (rv.ntok > 0 && (!q || !k || !v || !alpha || !sigma || !r || !d_o || !dq || !dk || !dv || !dalpha ||
+                        !dsigma || !dr))
+        return KDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, alpha, sigma, r, S0, P0, d_o, dS_T, dP_T, dq, dk, dv, dalpha, dsigma, dr, dS0, dP0};
+    for (const void *ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KDN_ERR_INVALID_ARG;
+    const size_t need = kdn::backward_workspace_bytes(rv.ntok, rv.nseq, p->H, p->d_k, p->d_v);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return KDN_ERR_WORKSPACE;
+
+    kdn::BwdArgs b{};
+    kdn::TokenArgs &a = b.a;
+    a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.sigma = sigma; a.r = r;
+    a.S0 = S0; a.P0 = P0;
+    a.cu = p->cu_seqlens; a.T = p->T; a.nseq = rv.nseq; a.H = p->H; a.dk = p->d_k; a.dv = p->d_v;
+    a.mu = p->mu; a.iso = 0; a.err = err_word();
+    b.d_o = d_o; b.dS_T = dS_T; b.dP_T = dP_T;
+    b.dq = dq; b.dk = dk; b.dv = dv; b.dalpha = dalpha; b.dsigma = dsigma; b.dr = dr; b.dS0 = dS0; b.dP0 = dP0;
+    return cuda_status(kdn::launch_backward(b, rv.bf16, rv.ntok, workspace, static_cast<cudaStream_t>(stream)));
+}
+
 kdn_status_t kdn_selftest_bounded_wait(long long limit_cycles, void *stream) {
     if (limit_cycles < 1000 || limit_cycles > 4000000000ll) return KDN_ERR_INVALID_ARG;
     unsigned *err = err_word();

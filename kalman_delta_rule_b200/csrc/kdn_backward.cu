@@ -1,0 +1,443 @@
+// Backward pass of the Diagonal KDN (the chunkwise regime is the training regime: KDA article,
+// "chunkwise" section; the recurrence is the explainer's diagonal approximation, "对角近似").
+//
+// Gradients of  L = <o, d_o> + <S_T, dS_T> + <P_T, dP_T>  with respect to q, k, v, alpha, sigma,
+// r, S0 and P0, by reverse-mode differentiation of the token recurrence
+//     P^- = alpha^2 P + sigma,  den = r + sum_i P^-_i k_i^2,  g = P^- k / den,
+//     W = diag(alpha) S,  u = v - W^T k,  S' = W + g u^T,  o = S'^T q,
+//     P' = P^- / (1 + c P^-),  c = mu k^2 / r.
+// Reverse step of one token (^ marks an adjoint; S^ arrives from the later tokens):
+//     S^ += q d_o^T;  dq = S' d_o;  g^ = S^ u;  u^ = S^T g;  dv = u^;
+//     W^ = S^ - k u^T;  k^ += -W u^;  alpha^ += rowsum(W^ o S);  S^ <- diag(alpha) W^;
+//     den^ = -(g^ . g) / den;  P^-^ = g^ k / den + den^ k^2 + P'^ z^2   (z = 1 / (1 + c P^-));
+//     c^ = -P'^ P'^2;  k^ += g^ P^- / den + 2 den^ P^- k + c^ 2 mu k / r;
+//     r^ = den^ - sum_i c^_i mu k_i^2 / r^2;  sigma^ = P^-^;  alpha^ += 2 alpha P P^-^;  P^ = alpha^2 P^-^.
+//
+// Three launches:
+//   tape  (one CTA per (sequence, head), thread = key channel): the uncertainty forward; writes
+//         P before each token, den and g per token;
+//   state (one CTA per (sequence, head, 16-column block of d_v), thread = key channel = row of S):
+//         the memory forward with S checkpoints every 32 tokens, then the reverse sweep chunk by
+//         chunk: the chunk's inputs are staged in shared memory, the chunk is recomputed from its
+//         checkpoint with shared-memory sub-checkpoints every 8 tokens (and u per token), and the
+//         state before each token is re-stepped from the nearest sub-checkpoint (never
+//         reconstructed by dividing by alpha, which loses it when alpha is small).  Writes dv and,
+//         per column block, partial sums over its columns of dq, g^, the S-part of k^ and the
+//         S-part of alpha^;
+//   prev  (one CTA per (sequence, head), thread = key channel): sums the partials and runs the
+//         uncertainty adjoint backwards; writes dq, dk, dalpha, dsigma, dr and dP0.
+// Everything is fp32 on the CUDA cores; inputs may be bf16 (widened exactly).
+#include "kdn_common.cuh"
+#include "kdn_launch.h"
+
+namespace kdn {
+
+namespace {
+constexpr int DB = 16;    // d_v columns per state CTA
+constexpr int CK = 32;    // tokens between the DRAM checkpoints of S
+constexpr int NS = 8;     // tokens between the shared-memory sub-checkpoints
+constexpr int GT = 32;    // tokens per group in the uncertainty kernels
+
+struct BwdWs {
+    float *Pprev, *g, *den, *ckpt, *part;
+    long long ntok;
+    int nblk;
+};
+
+// Sums 16 per-lane values over the 32 lanes of a warp (each step exchanges half of the
+// remaining values).  Lanes 2m and 2m+1 end with the total of value `which`.
+__device__ __forceinline__ float reduce16(float (&v)[16], int lane, int &which) {
+    const unsigned FULL = 0xffffffffu;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const bool up = lane & 16;
+        const float send = up ? v[i] : v[i + 8], keep = up ? v[i + 8] : v[i];
+        v[i] = keep + __shfl_xor_sync(FULL, send, 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const bool up = lane & 8;
+        const float send = up ? v[i] : v[i + 4], keep = up ? v[i + 4] : v[i];
+        v[i] = keep + __shfl_xor_sync(FULL, send, 8);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const bool up = lane & 4;
+        const float send = up ? v[i] : v[i + 2], keep = up ? v[i + 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(FULL, send, 4);
+    }
+    {
+        const bool up = lane & 2;
+        const float send = up ? v[0] : v[1], keep = up ? v[1] : v[0];
+        v[0] = keep + __shfl_xor_sync(FULL, send, 2);
+    }
+    v[0] += __shfl_xor_sync(FULL, v[0], 1);
+    which = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+    return v[0];
+}
+
+}  // namespace
+
+// ================================================================= tape
+// dynamic shared memory: alpha, sigma, k of a group [GT][dk] each, P^- and P^- k^2 [GT][dk], den [GT]
+template <typename T>
+__global__ void __launch_bounds__(128) bwd_tape_kernel(const BwdArgs b, const BwdWs w)
+{
+    extern __shared__ float smf[];
+    const TokenArgs &a = b.a;
+    const int dk = a.dk, H = a.H;
+    float *al_s = smf, *sg_s = al_s + GT * dk, *k_s = sg_s + GT * dk, *pm_s = k_s + GT * dk, *x_s = pm_s + GT * dk;
+    float *den_s = x_s + GT * dk, *r_s = den_s + GT;
+    const T *alpha = static_cast<const T *>(a.alpha), *sigma = static_cast<const T *>(a.sigma);
+    const T *k = static_cast<const T *>(a.k), *r = static_cast<const T *>(a.r);
+    const int chain = blockIdx.x, s = chain / H, h = chain % H;
+    const int i = threadIdx.x, warp = i >> 5, lane = i & 31, nw = dk >> 5;
+    int t0, t1;
+    seq_range(a, s, t0, t1);
+    float P = a.P0 ? a.P0[(size_t)chain * dk + i] : 1.f;
+    for (int tb = t0; tb < t1; tb += GT) {
+        const int n = min(GT, t1 - tb);
+        // stage the group's inputs (independent loads, all in flight together)
+#pragma unroll 8
+        for (int tt = 0; tt < n; ++tt) {
+            const size_t e = ((size_t)(tb + tt) * H + h) * dk + i;
+            al_s[tt * dk + i] = ldf(alpha + e);
+            sg_s[tt * dk + i] = ldf(sigma + e);
+            k_s[tt * dk + i] = ldf(k + e);
+        }
+        if (i < n) r_s[i] = ldf(r + (size_t)(tb + i) * H + h);
+        __syncthreads();
+        for (int tt = 0; tt < n; ++tt) {
+            const float al = al_s[tt * dk + i], kk = k_s[tt * dk + i];
+            w.Pprev[((size_t)(tb + tt) * H + h) * dk + i] = P;
+            const float pm = fmaf(al * al, P, sg_s[tt * dk + i]);
+            pm_s[tt * dk + i] = pm;
+            x_s[tt * dk + i] = pm * kk * kk;
+            P = pm / (1.f + a.mu * kk * kk * pm / r_s[tt]);
+        }
+        __syncthreads();
+        for (int tt = warp; tt < n; tt += nw) {
+            float x = 0.f;
+            for (int c = lane; c < dk; c += 32) x += x_s[tt * dk + c];
+            x = warp_sum(x);
+            if (lane == 0) {
+                den_s[tt] = r_s[tt] + x;
+                w.den[(size_t)(tb + tt) * H + h] = den_s[tt];
+            }
+        }
+        __syncthreads();
+        for (int tt = 0; tt < n; ++tt)
+            w.g[((size_t)(tb + tt) * H + h) * dk + i] = pm_s[tt * dk + i] * k_s[tt * dk + i] / den_s[tt];
+        __syncthreads();
+    }
+}
+
+// ================================================================= state
+// dynamic shared memory, per chunk of CK tokens: alpha, k, g, q [CK][dk]; v and d_o of the
+// column block [CK][DB]; sub-checkpoints [CK/NS][DB][dk]; u per token [CK][DB]; reduction
+// partials [4][DB]; u^ [DB]
+template <typename T>
+__global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, const BwdWs w)
+{
+    extern __shared__ float smf[];
+    const TokenArgs &a = b.a;
+    const int dk = a.dk, dv = a.dv, H = a.H;
+    float *al_s = smf, *k_s = al_s + CK * dk, *g_s = k_s + CK * dk, *q_s = g_s + CK * dk;
+    float *v_s = q_s + CK * dk, *do_s = v_s + CK * DB;
+    float *sub = do_s + CK * DB;              // [CK/NS][DB][dk]
+    float *us = sub + (CK / NS) * DB * dk;    // [CK][DB]
+    float *red = us + CK * DB;                // [4][DB]
+    float *uh = red + 4 * DB;                 // [DB]
+
+    const T *q = static_cast<const T *>(a.q), *k = static_cast<const T *>(a.k), *v = static_cast<const T *>(a.v);
+    const T *alpha = static_cast<const T *>(a.alpha), *d_o = static_cast<const T *>(b.d_o);
+    const int chain = blockIdx.x / w.nblk, blk = blockIdx.x % w.nblk, col0 = blk * DB;
+    const int s = chain / H, h = chain % H;
+    const int i = threadIdx.x, warp = i >> 5, lane = i & 31, nw = dk >> 5, nt = blockDim.x;
+    int t0, t1;
+    seq_range(a, s, t0, t1);
+    const long long slot0 = t0 / CK + s;      // checkpoint slots of this sequence: slot0 + chunk
+    const size_t tokstride = (size_t)w.ntok * H * dk;
+    auto ckpt_at = [&](int m) { return w.ckpt + (((size_t)(slot0 + m) * H + h) * w.nblk + blk) * DB * dk; };
+
+    // the chunk's per-token inputs into shared memory (reverse: also q and d_o)
+    auto stage = [&](int c0, int L, bool rev) {
+        __syncthreads();   // the previous chunk is done with the staged inputs
+#pragma unroll 8
+        for (int tt = 0; tt < L; ++tt) {
+            const size_t e = ((size_t)(c0 + tt) * H + h) * dk + i;
+            al_s[tt * dk + i] = ldf(alpha + e);
+            k_s[tt * dk + i] = ldf(k + e);
+            g_s[tt * dk + i] = w.g[e];
+            if (rev) q_s[tt * dk + i] = ldf(q + e);
+        }
+        for (int x = i; x < L * DB; x += nt) {
+            const int tt = x / DB, j = x % DB;
+            const size_t e = ((size_t)(c0 + tt) * H + h) * dv + col0 + j;
+            v_s[x] = ldf(v + e);
+            if (rev) do_s[x] = ldf(d_o + e);
+        }
+        __syncthreads();
+    };
+    // u_j = v_j - sum_i alpha_i k_i S_ij for staged token tt -> dst[DB] (shared), then into u
+    auto forward_u = [&](int tt, const float (&S)[16], float *dst, float (&u)[16]) {
+        const float ak = al_s[tt * dk + i] * k_s[tt * dk + i];
+        float p[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) p[j] = ak * S[j];
+        int which;
+        const float tot = reduce16(p, lane, which);
+        if ((lane & 1) == 0) red[warp * DB + which] = tot;
+        __syncthreads();
+        if (i < DB) {
+            float x = 0.f;
+            for (int ww = 0; ww < nw; ++ww) x += red[ww * DB + i];
+            dst[i] = v_s[tt * DB + i] - x;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) u[j] = dst[j];
+    };
+    auto step = [&](int tt, float (&S)[16], const float (&u)[16]) {
+        const float al = al_s[tt * dk + i], gg = g_s[tt * dk + i];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) S[j] = fmaf(gg, u[j], al * S[j]);
+    };
+
+    float S[16], Sh[16], u[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) S[j] = a.S0 ? a.S0[((size_t)chain * dk + i) * dv + col0 + j] : 0.f;
+
+    // ---- forward: checkpoints every CK tokens
+    const int nchk = (t1 - t0 + CK - 1) / CK;
+    for (int m = 0; m < nchk; ++m) {
+        const int c0 = t0 + m * CK, L = min(CK, t1 - c0);
+        float *ck = ckpt_at(m);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) ck[j * dk + i] = S[j];
+        stage(c0, L, false);
+        for (int tt = 0; tt < L; ++tt) {
+            forward_u(tt, S, uh, u);
+            step(tt, S, u);
+        }
+    }
+
+    // ---- reverse, chunk by chunk
+#pragma unroll
+    for (int j = 0; j < 16; ++j) Sh[j] = b.dS_T ? b.dS_T[((size_t)chain * dk + i) * dv + col0 + j] : 0.f;
+    for (int m = nchk - 1; m >= 0; --m) {
+        const int c0 = t0 + m * CK, L = min(CK, t1 - c0);
+        const float *ck = ckpt_at(m);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) S[j] = ck[j * dk + i];
+        stage(c0, L, true);
+        for (int tt = 0; tt < L; ++tt) {
+            if (tt % NS == 0) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) sub[((tt / NS) * DB + j) * dk + i] = S[j];
+            }
+            forward_u(tt, S, us + tt * DB, u);
+            step(tt, S, u);
+        }
+        for (int js = (L - 1) / NS; js >= 0; --js) {
+            for (int tt = min(L, js * NS + NS) - 1; tt >= js * NS; --tt) {
+                const int t = c0 + tt;
+                // state before token t, re-stepped from the sub-checkpoint
+                float Sp[16], uu[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) Sp[j] = sub[(js * DB + j) * dk + i];
+                for (int oo = js * NS; oo < tt; ++oo) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) uu[j] = us[oo * DB + j];
+                    step(oo, Sp, uu);
+                }
+                const float al = al_s[tt * dk + i], kk = k_s[tt * dk + i], gg = g_s[tt * dk + i], qq = q_s[tt * dk + i];
+                float dqp = 0.f, gp = 0.f, p[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float uj = us[tt * DB + j], doj = do_s[tt * DB + j];
+                    const float St = fmaf(gg, uj, al * Sp[j]);
+                    Sh[j] = fmaf(qq, doj, Sh[j]);
+                    dqp = fmaf(St, doj, dqp);
+                    gp = fmaf(Sh[j], uj, gp);
+                    p[j] = Sh[j] * gg;
+                }
+                int which;
+                const float tot = reduce16(p, lane, which);
+                if ((lane & 1) == 0) red[warp * DB + which] = tot;
+                __syncthreads();
+                if (i < DB) {
+                    float x = 0.f;
+                    for (int ww = 0; ww < nw; ++ww) x += red[ww * DB + i];
+                    uh[i] = x;
+                    b.dv[((size_t)t * H + h) * dv + col0 + i] = x;
+                }
+                __syncthreads();
+                float kp = 0.f, ap = 0.f;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float uhj = uh[j];
+                    const float Wh = fmaf(-kk, uhj, Sh[j]);
+                    kp = fmaf(al * Sp[j], uhj, kp);
+                    ap = fmaf(Wh, Sp[j], ap);
+                    Sh[j] = al * Wh;
+                }
+                float *pp = w.part + (size_t)blk * 4 * tokstride + ((size_t)t * H + h) * dk + i;
+                pp[0] = dqp;
+                pp[tokstride] = gp;
+                pp[2 * tokstride] = -kp;
+                pp[3 * tokstride] = ap;
+            }
+        }
+    }
+    if (b.dS0) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) b.dS0[((size_t)chain * dk + i) * dv + col0 + j] = Sh[j];
+    }
+}
+
+// ================================================================= prev
+// dynamic shared memory, per group of GT tokens: g^, k^ (S part), alpha^ (S part), scratch,
+// alpha, sigma, k, P before the token [GT][dk] each; den^, r, den [GT].  NB = number of
+// column blocks (d_v / 16), a template argument so that every partial load is issued at once.
+template <typename T, int NB>
+__global__ void __launch_bounds__(128) bwd_prev_kernel(const BwdArgs b, const BwdWs w)
+{
+    extern __shared__ float smf[];
+    const TokenArgs &a = b.a;
+    const int dk = a.dk, H = a.H;
+    float *gh_s = smf, *ks_s = gh_s + GT * dk, *as_s = ks_s + GT * dk, *x_s = as_s + GT * dk;
+    float *al_s = x_s + GT * dk, *sg_s = al_s + GT * dk, *k_s = sg_s + GT * dk, *pp_s = k_s + GT * dk;
+    float *dd_s = pp_s + GT * dk, *r_s = dd_s + GT, *den_s = r_s + GT;
+    const T *alpha = static_cast<const T *>(a.alpha), *sigma = static_cast<const T *>(a.sigma);
+    const T *k = static_cast<const T *>(a.k), *r = static_cast<const T *>(a.r);
+    const int chain = blockIdx.x, s = chain / H, h = chain % H;
+    const int i = threadIdx.x, warp = i >> 5, lane = i & 31, nw = dk >> 5;
+    const float mu = a.mu;
+    const size_t tokstride = (size_t)w.ntok * H * dk;
+    int t0, t1;
+    seq_range(a, s, t0, t1);
+    float Ph = b.dP_T ? b.dP_T[(size_t)chain * dk + i] : 0.f;
+    for (int te = t1; te > t0; te -= GT) {
+        const int tb = max(t0, te - GT), n = te - tb;
+        // stage the group: partial sums over the column blocks, the inputs, the tapes
+#pragma unroll 4
+        for (int tt = 0; tt < n; ++tt) {
+            const size_t e = ((size_t)(tb + tt) * H + h) * dk + i;
+            float p4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int bb = 0; bb < NB; ++bb) {
+                const float *pp = w.part + (size_t)bb * 4 * tokstride + e;
+                p4[0] += pp[0];
+                p4[1] += pp[tokstride];
+                p4[2] += pp[2 * tokstride];
+                p4[3] += pp[3 * tokstride];
+            }
+            b.dq[e] = p4[0];
+            gh_s[tt * dk + i] = p4[1];
+            ks_s[tt * dk + i] = p4[2];
+            as_s[tt * dk + i] = p4[3];
+            x_s[tt * dk + i] = p4[1] * w.g[e];
+            al_s[tt * dk + i] = ldf(alpha + e);
+            sg_s[tt * dk + i] = ldf(sigma + e);
+            k_s[tt * dk + i] = ldf(k + e);
+            pp_s[tt * dk + i] = w.Pprev[e];
+        }
+        if (i < n) {
+            r_s[i] = ldf(r + (size_t)(tb + i) * H + h);
+            den_s[i] = w.den[(size_t)(tb + i) * H + h];
+        }
+        __syncthreads();
+        for (int tt = warp; tt < n; tt += nw) {
+            float x = 0.f;
+            for (int c = lane; c < dk; c += 32) x += x_s[tt * dk + c];
+            x = warp_sum(x);
+            if (lane == 0) dd_s[tt] = -x / den_s[tt];
+        }
+        __syncthreads();
+        for (int tt = n - 1; tt >= 0; --tt) {
+            const size_t e = ((size_t)(tb + tt) * H + h) * dk + i;
+            const float al = al_s[tt * dk + i], kk = k_s[tt * dk + i], rr = r_s[tt], dn = den_s[tt];
+            const float Pp = pp_s[tt * dk + i];
+            const float pm = fmaf(al * al, Pp, sg_s[tt * dk + i]);
+            const float c = mu * kk * kk / rr;
+            const float z = 1.f / (1.f + c * pm);
+            const float Pt = pm * z;
+            const float gh = gh_s[tt * dk + i], dd = dd_s[tt];
+            const float pmh = gh * kk / dn + dd * kk * kk + Ph * z * z;
+            const float ch = -Ph * Pt * Pt;
+            b.dk[e] = ks_s[tt * dk + i] + gh * pm / dn + 2.f * dd * pm * kk + ch * 2.f * mu * kk / rr;
+            x_s[tt * dk + i] = -ch * mu * kk * kk / (rr * rr);
+            b.dsigma[e] = pmh;
+            b.dalpha[e] = as_s[tt * dk + i] + 2.f * al * Pp * pmh;
+            Ph = al * al * pmh;
+        }
+        __syncthreads();
+        for (int tt = warp; tt < n; tt += nw) {
+            float x = 0.f;
+            for (int c = lane; c < dk; c += 32) x += x_s[tt * dk + c];
+            x = warp_sum(x);
+            if (lane == 0) b.dr[(size_t)(tb + tt) * H + h] = dd_s[tt] + x;
+        }
+        __syncthreads();
+    }
+    if (b.dP0) b.dP0[(size_t)chain * dk + i] = Ph;
+}
+
+// ================================================================= host
+namespace {
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+long long ckpt_slots(long long ntok, int nseq) { return ntok / CK + nseq + 1; }
+}  // namespace
+
+size_t backward_workspace_bytes(long long ntok, int nseq, int H, int dk, int dv) {
+    const size_t th = (size_t)ntok * H;
+    size_t n = 0;
+    n += align256(th * dk * 4);                                     // P before each token
+    n += align256(th * dk * 4);                                     // g
+    n += align256(th * 4);                                          // den
+    n += align256((size_t)ckpt_slots(ntok, nseq) * H * dk * dv * 4);   // S checkpoints
+    n += align256((size_t)4 * (dv / DB) * th * dk * 4);             // per-column-block partials
+    return n;
+}
+
+template <typename T>
+static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, cudaStream_t st) {
+    const int chains = b.a.nseq * b.a.H, dk = b.a.dk;
+    const size_t tsm = ((size_t)5 * GT * dk + 2 * GT) * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(bwd_tape_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+    if (e != cudaSuccess) return e;
+    bwd_tape_kernel<T><<<chains, dk, tsm, st>>>(b, w);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t ssm = ((size_t)4 * CK * dk + 2 * CK * DB + (CK / NS) * DB * dk + CK * DB + 4 * DB + DB) * sizeof(float);
+    e = cudaFuncSetAttribute(bwd_state_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
+    if (e != cudaSuccess) return e;
+    bwd_state_kernel<T><<<(unsigned)chains * w.nblk, dk, ssm, st>>>(b, w);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t psm = ((size_t)8 * GT * dk + 3 * GT) * sizeof(float);
+    auto prev = w.nblk == 2 ? bwd_prev_kernel<T, 2> : w.nblk == 4 ? bwd_prev_kernel<T, 4>
+              : w.nblk == 8 ? bwd_prev_kernel<T, 8> : bwd_prev_kernel<T, 16>;
+    e = cudaFuncSetAttribute(prev, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
+    if (e != cudaSuccess) return e;
+    prev<<<chains, dk, psm, st>>>(b, w);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_backward(const BwdArgs &b, bool bf16_in, long long ntok, void *workspace, cudaStream_t st) {
+    const TokenArgs &a = b.a;
+    const size_t th = (size_t)ntok * a.H;
+    uint8_t *p = static_cast<uint8_t *>(workspace);
+    BwdWs w;
+    w.ntok = ntok;
+    w.nblk = a.dv / DB;
+    w.Pprev = reinterpret_cast<float *>(p); p += align256(th * a.dk * 4);
+    w.g = reinterpret_cast<float *>(p); p += align256(th * a.dk * 4);
+    w.den = reinterpret_cast<float *>(p); p += align256(th * 4);
+    w.ckpt = reinterpret_cast<float *>(p); p += align256((size_t)ckpt_slots(ntok, a.nseq) * a.H * a.dk * a.dv * 4);
+    w.part = reinterpret_cast<float *>(p);
+    return bf16_in ? launch_bwd_typed<bf16>(b, w, st) : launch_bwd_typed<float>(b, w, st);
+}
+
+}  // namespace kdn

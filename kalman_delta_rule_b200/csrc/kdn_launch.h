@@ -29,6 +29,18 @@ cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long
 // [ntok, H, d] bf16 as a TMA tensor map with 64 x 1 x 64 boxes and 128-byte swizzle
 bool make_token_map(CUtensorMap *m, const void *base, int d, int H, long long ntok);
 
+// backward of the diagonal KDN (three launches: uncertainty tape, memory state pass,
+// uncertainty adjoint); all gradients fp32
+struct BwdArgs {
+    TokenArgs a;                                 // forward inputs (o, S_out, P_out unused)
+    const void *d_o;                             // [ntok, H, dv], input dtype
+    const float *dS_T, *dP_T;                    // [N, H, dk, dv], [N, H, dk]; NULL = 0
+    float *dq, *dk, *dv, *dalpha, *dsigma, *dr;  // token layouts
+    float *dS0, *dP0;                            // may be NULL
+};
+size_t backward_workspace_bytes(long long ntok, int nseq, int H, int dk, int dv);
+cudaError_t launch_backward(const BwdArgs &b, bool bf16_in, long long ntok, void *workspace, cudaStream_t st);
+
 // failure-detection self-test: bounded waits that run out and record ERR_TIMEOUT
 cudaError_t launch_bounded_wait_selftest(long long limit_cycles, unsigned *err, cudaStream_t st);
 

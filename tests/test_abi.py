@@ -117,6 +117,31 @@ def test_forward_rejects_bad_pointers(lib):
     assert B.kdn_gain_scan_noalloc(piso, *k_a_s_r, None, FAKE, None, None, None) == B.KDN_ERR_UNSUPPORTED
 
 
+def test_backward_validates_before_any_cuda_call(lib):
+    p = problem(chunk=64)
+    need = B.kdn_backward_workspace_size(p)
+    # P tape, g, den, S checkpoints every 32 tokens and per-16-column partial sums
+    ntok, H, dk, dv = 2 * 128, 4, 128, 128
+    assert need >= 4 * (2 * ntok * H * dk + ntok * H + (ntok // 32 + 2 + 1) * H * dk * dv + 4 * (dv // 16) * ntok * H * dk)
+    assert need < 4 * (2 * ntok * H * dk + ntok * H + (ntok // 32 + 2 + 1) * H * dk * dv + 4 * (dv // 16) * ntok * H * dk) + 5 * 256
+    ins = [FAKE] * 6                 # q, k, v, alpha, sigma, r
+    outs = [FAKE + 4096 * (i + 1) for i in range(6)]   # dq, dk, dv, dalpha, dsigma, dr
+    args = lambda d_o=FAKE, o=outs, ws=FAKE, wb=need: [p, *ins, None, None, d_o, None, None, *o, None, None, ws, wb, None]
+    assert B.kdn_backward(*args(ws=None)) == B.KDN_ERR_WORKSPACE
+    assert B.kdn_backward(*args(wb=need - 1)) == B.KDN_ERR_WORKSPACE
+    assert B.kdn_backward(*args(ws=FAKE + 16)) == B.KDN_ERR_WORKSPACE
+    assert B.kdn_backward(*args(d_o=None)) == B.KDN_ERR_INVALID_ARG
+    assert B.kdn_backward(*args(d_o=FAKE + 2)) == B.KDN_ERR_INVALID_ARG
+    bad = list(outs); bad[5] = None
+    assert B.kdn_backward(*args(o=bad)) == B.KDN_ERR_INVALID_ARG
+    # diagonal uncertainty only; sizes as for the forward
+    piso = problem(chunk=64, variant=1)
+    assert lib.kdn_backward_workspace_size(ctypes.byref(piso), ctypes.byref(ctypes.c_size_t())) == B.KDN_ERR_UNSUPPORTED
+    assert B.kdn_backward(piso, *args()[1:]) == B.KDN_ERR_UNSUPPORTED
+    assert B.kdn_backward(problem(d_k=48), *args()[1:]) == B.KDN_ERR_UNSUPPORTED
+    assert B.kdn_backward(problem(num_seqs=0, B=0), *args()[1:]) == B.KDN_OK   # nothing to do
+
+
 def test_decode_rejects_bad_arguments(lib):
     ptrs = [FAKE] * 9
     assert B.kdn_decode_step(4, 2, 48, 64, B.KDN_DTYPE_BF16, 1.0, *ptrs, None) == B.KDN_ERR_UNSUPPORTED

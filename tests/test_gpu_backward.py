@@ -1,0 +1,113 @@
+"""GPU parity of the backward pass (kdn_backward) against the fp64 gradient oracle
+(oracle/kdn_grad.py): every gradient, element by element, for fp32 and bf16 inputs, ragged
+varlen batches with an empty sequence, initial states and final-state gradients, every d_k
+and the d_v extremes, and the full-size prefill workload (B4 H16 T4096 d128 bf16) on sampled
+(sequence, head) chains -- each chain's gradients depend on that chain's inputs only."""
+import numpy as np
+import pytest
+
+from kalman_delta_rule_b200 import inputs
+from oracle import kdn_grad
+from tests.kdn_testutil import dense_shape, max_rel_err, to_dev, to_host
+from tests.test_gpu_recurrent import ragged
+
+pytestmark = pytest.mark.gpu
+
+# fp32 arithmetic on exactly widened inputs (bf16 inputs are widened without rounding on both
+# sides), so bf16 and fp32 inputs share the fp32 tolerance
+TOL = 1e-4
+NAMES = ("dq", "dk", "dv", "dalpha", "dsigma", "dr", "dS0", "dP0")
+
+
+def cotangents(seed, w, with_final=True):
+    rng = np.random.default_rng(seed)
+    d_o = rng.standard_normal((w.ntok, w.H, w.dv)).astype(np.float32)
+    if w.bf16:
+        d_o = inputs.bf16_bits(d_o)
+    dS = dP = None
+    if with_final:
+        dS = rng.standard_normal((w.num_seqs, w.H, w.dk, w.dv)).astype(np.float32)
+        dP = rng.standard_normal((w.num_seqs, w.H, w.dk)).astype(np.float32)
+    return d_o, dS, dP
+
+
+def initial_state(seed, w):
+    rng = np.random.default_rng(seed)
+    S0 = (0.1 * rng.standard_normal((w.num_seqs, w.H, w.dk, w.dv))).astype(np.float32)
+    P0 = rng.uniform(0.3, 2.0, (w.num_seqs, w.H, w.dk)).astype(np.float32)
+    return S0, P0
+
+
+def run_backward(kdn, w, d_o, S0=None, P0=None, dS=None, dP=None, mu=1.0):
+    import torch
+    args = [to_dev(dense_shape(w, getattr(w, n))) for n in ("q", "k", "v", "alpha", "sigma", "r")]
+    cu = to_dev(w.cu_seqlens) if w.B == 1 and w.num_seqs > 1 else None
+    g = kdn.backward(*args, to_dev(dense_shape(w, d_o)), cu_seqlens=cu, S0=to_dev(S0), P0=to_dev(P0),
+                     dS=to_dev(dS), dP=to_dev(dP), mu=mu)
+    torch.cuda.synchronize()
+    kdn.last_device_error()
+    out = {n: to_host(g[n]) for n in NAMES}
+    for n in ("dq", "dk", "dv", "dalpha", "dsigma", "dr"):
+        out[n] = out[n].reshape((w.ntok,) + out[n].shape[2:])
+    return out
+
+
+def check(got, ref, tol=TOL):
+    for n in NAMES:
+        err = max_rel_err(got[n], ref[n])
+        assert err <= tol, f"{n}: max relative error {err:.3e} > {tol}"
+
+
+@pytest.mark.parametrize("mu", [1.0, 32.0])
+def test_backward_tiny_fp32(kdn, mu):
+    w = inputs.tiny_fp32()
+    S0, P0 = initial_state(1, w)
+    d_o, dS, dP = cotangents(2, w)
+    ref = kdn_grad.diag_grad(w.q, w.k, w.v, w.alpha, w.sigma, w.r, d_o, cu_seqlens=w.cu_seqlens,
+                             S0=S0, P0=P0, dS=dS, dP=dP, mu=mu)
+    check(run_backward(kdn, w, d_o, S0, P0, dS, dP, mu=mu), ref)
+
+
+@pytest.mark.parametrize("dk,dv", [(32, 32), (64, 256), (128, 128)])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_backward_ragged_varlen(kdn, dk, dv, bf16):
+    """Sequences of 1, 63, 64, 0, 65 and 130 tokens (one empty): partial checkpoint chunks,
+    partial sub-checkpoint groups and an empty chain, with S0/P0 and final-state gradients."""
+    w = ragged(400 + dk + dv, [1, 63, 64, 0, 65, 130], 2, dk, dv, bf16)
+    S0, P0 = initial_state(3, w)
+    d_o, dS, dP = cotangents(4, w)
+    ref = kdn_grad.diag_grad(w.q, w.k, w.v, w.alpha, w.sigma, w.r, d_o, cu_seqlens=w.cu_seqlens,
+                             S0=S0, P0=P0, dS=dS, dP=dP, mu=2.0)
+    got = run_backward(kdn, w, d_o, S0, P0, dS, dP, mu=2.0)
+    check(got, ref)
+    # the empty sequence passes the final-state gradients straight through
+    np.testing.assert_array_equal(got["dS0"][3], dS[3])
+    np.testing.assert_array_equal(got["dP0"][3], dP[3])
+
+
+def test_backward_dense_defaults(kdn):
+    """Dense batch, S0 = 0 and P0 = 1 by default, no final-state gradients."""
+    w = inputs.dense("bwd_dense", 12, 2, 3, 150, 128, 128, bf16=True)
+    d_o, _, _ = cotangents(5, w, with_final=False)
+    ref = kdn_grad.diag_grad(w.q, w.k, w.v, w.alpha, w.sigma, w.r, d_o, cu_seqlens=w.cu_seqlens)
+    check(run_backward(kdn, w, d_o), ref)
+
+
+def test_backward_full_size_sampled_chains(kdn):
+    """The prefill workload at full size (B4 H16 T4096 d128 bf16) through one backward call;
+    the oracle recomputes two (sequence, head) chains on their own."""
+    w = inputs.prefill_4x4096()
+    d_o, dS, dP = cotangents(6, w)
+    got = run_backward(kdn, w, d_o, dS=dS, dP=dP)
+    T = w.ntok // w.B
+    for s, h in ((0, 0), (3, 15)):
+        sl = slice(s * T, (s + 1) * T)
+        pick = lambda x: x[sl, h:h + 1]
+        ref = kdn_grad.diag_grad(pick(w.q), pick(w.k), pick(w.v), pick(w.alpha), pick(w.sigma), w.r[sl, h:h + 1],
+                                 d_o[sl, h:h + 1], dS=dS[s:s + 1, h:h + 1], dP=dP[s:s + 1, h:h + 1])
+        for n in ("dq", "dk", "dv", "dalpha", "dsigma"):
+            err = max_rel_err(got[n][sl, h], ref[n][:, 0])
+            assert err <= TOL, f"chain ({s},{h}) {n}: {err:.3e}"
+        assert max_rel_err(got["dr"][sl, h], ref["dr"][:, 0]) <= TOL
+        assert max_rel_err(got["dS0"][s, h], ref["dS0"][0, 0]) <= TOL
+        assert max_rel_err(got["dP0"][s, h], ref["dP0"][0, 0]) <= TOL
