@@ -13,20 +13,26 @@
 //     c^ = -P'^ P'^2;  k^ += g^ P^- / den + 2 den^ P^- k + c^ 2 mu k / r;
 //     r^ = den^ - sum_i c^_i mu k_i^2 / r^2;  sigma^ = P^-^;  alpha^ += 2 alpha P P^-^;  P^ = alpha^2 P^-^.
 //
-// Three launches:
+// Four launches:
 //   tape  (one CTA per (sequence, head), thread = key channel): the uncertainty forward; writes
 //         P before each token, den and g per token;
 //   state (one CTA per (sequence, head, 16-column block of d_v), thread = key channel = row of S):
-//         the memory forward with S checkpoints every 32 tokens, then the reverse sweep chunk by
-//         chunk: the chunk's inputs are staged in shared memory, the chunk is recomputed from its
-//         checkpoint with shared-memory sub-checkpoints every 8 tokens (and u per token), and the
+//         the memory forward with S checkpoints every 32 tokens and u of every token taped, then
+//         the reverse sweep chunk by chunk: the chunk's inputs are staged in shared memory, the
+//         chunk is re-stepped from its checkpoint (with the taped u, so without the cross-row
+//         reduction) into shared-memory sub-checkpoints every 8 tokens, and the
 //         state before each token is re-stepped from the nearest sub-checkpoint (never
 //         reconstructed by dividing by alpha, which loses it when alpha is small).  Writes dv and,
 //         per column block, partial sums over its columns of dq, g^, the S-part of k^ and the
 //         S-part of alpha^;
-//   prev  (one CTA per (sequence, head), thread = key channel): sums the partials and runs the
-//         uncertainty adjoint backwards; writes dq, dk, dalpha, dsigma, dr and dP0.
-// Everything is fp32 on the CUDA cores; inputs may be bf16 (widened exactly).
+//   local (one warp per (token, head), every token in parallel): sums the partials, writes dq and
+//         den^, and the parts of P^-^ and k^ that do not depend on the later tokens' P^;
+//   prev  (one CTA per (sequence, head), thread = key channel): the one serial part of the
+//         uncertainty adjoint, P^ <- alpha^2 (P^-^local + P^ z^2), and the outputs that need P^:
+//         dk, dalpha, dsigma, dr and dP0.
+// Token rows are staged into shared memory with 16-byte asynchronous copies, a group of tokens at
+// a time, so each group costs one memory round trip.  Everything is fp32 on the CUDA cores;
+// inputs may be bf16 (widened exactly).
 #include "kdn_common.cuh"
 #include "kdn_launch.h"
 
@@ -39,10 +45,32 @@ constexpr int NS = 8;     // tokens between the shared-memory sub-checkpoints
 constexpr int GT = 32;    // tokens per group in the uncertainty kernels
 
 struct BwdWs {
-    float *Pprev, *g, *den, *ckpt, *part;
+    float *Pprev, *g, *den, *dden, *utape, *ckpt, *part;
     long long ntok;
     int nblk;
 };
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
+}
+// n rows of row_bytes (a multiple of 16) from src + row * stride_bytes into dst, rows packed;
+// every thread of the block takes a share of the 16-byte pieces
+__device__ __forceinline__ void stage_rows(void *dst, const void *src, size_t stride_bytes, int n, int row_bytes) {
+    const int per = row_bytes >> 4, nt = blockDim.x;
+    for (int x = threadIdx.x; x < n * per; x += nt) {
+        const int rr = x / per, c = x - rr * per;
+        cp_async16(static_cast<char *>(dst) + (size_t)rr * row_bytes + c * 16,
+                   static_cast<const char *>(src) + (size_t)rr * stride_bytes + c * 16);
+    }
+}
+__device__ __forceinline__ float lds(const float *p) { return *p; }
+__device__ __forceinline__ float lds(const bf16 *p) {
+    return __uint_as_float(((unsigned)*reinterpret_cast<const unsigned short *>(p)) << 16);
+}
 
 // Sums 16 per-lane values over the 32 lanes of a warp (each step exchanges half of the
 // remaining values).  Lanes 2m and 2m+1 end with the total of value `which`.
@@ -79,38 +107,38 @@ __device__ __forceinline__ float reduce16(float (&v)[16], int lane, int &which) 
 }  // namespace
 
 // ================================================================= tape
-// dynamic shared memory: alpha, sigma, k of a group [GT][dk] each, P^- and P^- k^2 [GT][dk], den [GT]
+// dynamic shared memory: alpha, sigma, k rows of a group [GT][dk] (input type); P^- and P^- k^2
+// [GT][dk]; den, r [GT]
 template <typename T>
 __global__ void __launch_bounds__(128) bwd_tape_kernel(const BwdArgs b, const BwdWs w)
 {
     extern __shared__ float smf[];
     const TokenArgs &a = b.a;
     const int dk = a.dk, H = a.H;
-    float *al_s = smf, *sg_s = al_s + GT * dk, *k_s = sg_s + GT * dk, *pm_s = k_s + GT * dk, *x_s = pm_s + GT * dk;
-    float *den_s = x_s + GT * dk, *r_s = den_s + GT;
+    float *pm_s = smf, *x_s = pm_s + GT * dk, *den_s = x_s + GT * dk, *r_s = den_s + GT;
+    T *al_s = reinterpret_cast<T *>(r_s + GT), *sg_s = al_s + GT * dk, *k_s = sg_s + GT * dk;
     const T *alpha = static_cast<const T *>(a.alpha), *sigma = static_cast<const T *>(a.sigma);
     const T *k = static_cast<const T *>(a.k), *r = static_cast<const T *>(a.r);
     const int chain = blockIdx.x, s = chain / H, h = chain % H;
     const int i = threadIdx.x, warp = i >> 5, lane = i & 31, nw = dk >> 5;
+    const size_t rstride = (size_t)H * dk * sizeof(T);
+    const int rbytes = dk * (int)sizeof(T);
     int t0, t1;
     seq_range(a, s, t0, t1);
     float P = a.P0 ? a.P0[(size_t)chain * dk + i] : 1.f;
     for (int tb = t0; tb < t1; tb += GT) {
         const int n = min(GT, t1 - tb);
-        // stage the group's inputs (independent loads, all in flight together)
-#pragma unroll 8
-        for (int tt = 0; tt < n; ++tt) {
-            const size_t e = ((size_t)(tb + tt) * H + h) * dk + i;
-            al_s[tt * dk + i] = ldf(alpha + e);
-            sg_s[tt * dk + i] = ldf(sigma + e);
-            k_s[tt * dk + i] = ldf(k + e);
-        }
+        const size_t row0 = ((size_t)tb * H + h) * dk;
+        stage_rows(al_s, alpha + row0, rstride, n, rbytes);
+        stage_rows(sg_s, sigma + row0, rstride, n, rbytes);
+        stage_rows(k_s, k + row0, rstride, n, rbytes);
         if (i < n) r_s[i] = ldf(r + (size_t)(tb + i) * H + h);
+        cp_async_wait_all();
         __syncthreads();
         for (int tt = 0; tt < n; ++tt) {
-            const float al = al_s[tt * dk + i], kk = k_s[tt * dk + i];
+            const float al = lds(al_s + tt * dk + i), kk = lds(k_s + tt * dk + i);
             w.Pprev[((size_t)(tb + tt) * H + h) * dk + i] = P;
-            const float pm = fmaf(al * al, P, sg_s[tt * dk + i]);
+            const float pm = fmaf(al * al, P, lds(sg_s + tt * dk + i));
             pm_s[tt * dk + i] = pm;
             x_s[tt * dk + i] = pm * kk * kk;
             P = pm / (1.f + a.mu * kk * kk * pm / r_s[tt]);
@@ -127,61 +155,62 @@ __global__ void __launch_bounds__(128) bwd_tape_kernel(const BwdArgs b, const Bw
         }
         __syncthreads();
         for (int tt = 0; tt < n; ++tt)
-            w.g[((size_t)(tb + tt) * H + h) * dk + i] = pm_s[tt * dk + i] * k_s[tt * dk + i] / den_s[tt];
+            w.g[((size_t)(tb + tt) * H + h) * dk + i] = pm_s[tt * dk + i] * lds(k_s + tt * dk + i) / den_s[tt];
         __syncthreads();
     }
 }
 
 // ================================================================= state
-// dynamic shared memory, per chunk of CK tokens: alpha, k, g, q [CK][dk]; v and d_o of the
-// column block [CK][DB]; sub-checkpoints [CK/NS][DB][dk]; u per token [CK][DB]; reduction
-// partials [4][DB]; u^ [DB]
+// dynamic shared memory, per chunk of CK tokens: g rows [CK][dk] fp32; sub-checkpoints
+// [CK/NS][DB][dk]; u per token [CK][DB]; reduction partials [4][DB]; u^ [DB]; then alpha, k, q
+// rows [CK][dk] and the column block of v (forward) or d_o (reverse) [CK][DB] in the input type
 template <typename T>
 __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, const BwdWs w)
 {
     extern __shared__ float smf[];
     const TokenArgs &a = b.a;
     const int dk = a.dk, dv = a.dv, H = a.H;
-    float *al_s = smf, *k_s = al_s + CK * dk, *g_s = k_s + CK * dk, *q_s = g_s + CK * dk;
-    float *v_s = q_s + CK * dk, *do_s = v_s + CK * DB;
-    float *sub = do_s + CK * DB;              // [CK/NS][DB][dk]
+    float *g_s = smf;
+    float *sub = g_s + CK * dk;               // [CK/NS][DB][dk]
     float *us = sub + (CK / NS) * DB * dk;    // [CK][DB]
     float *red = us + CK * DB;                // [4][DB]
     float *uh = red + 4 * DB;                 // [DB]
+    T *al_s = reinterpret_cast<T *>(uh + DB), *k_s = al_s + CK * dk, *q_s = k_s + CK * dk;
+    T *v_s = q_s + CK * dk, *do_s = v_s;      // v in the forward, d_o in the reverse
 
     const T *q = static_cast<const T *>(a.q), *k = static_cast<const T *>(a.k), *v = static_cast<const T *>(a.v);
     const T *alpha = static_cast<const T *>(a.alpha), *d_o = static_cast<const T *>(b.d_o);
     const int chain = blockIdx.x / w.nblk, blk = blockIdx.x % w.nblk, col0 = blk * DB;
     const int s = chain / H, h = chain % H;
-    const int i = threadIdx.x, warp = i >> 5, lane = i & 31, nw = dk >> 5, nt = blockDim.x;
+    const int i = threadIdx.x, warp = i >> 5, lane = i & 31, nw = dk >> 5;
     int t0, t1;
     seq_range(a, s, t0, t1);
     const long long slot0 = t0 / CK + s;      // checkpoint slots of this sequence: slot0 + chunk
     const size_t tokstride = (size_t)w.ntok * H * dk;
     auto ckpt_at = [&](int m) { return w.ckpt + (((size_t)(slot0 + m) * H + h) * w.nblk + blk) * DB * dk; };
 
-    // the chunk's per-token inputs into shared memory (reverse: also q and d_o)
+    // the chunk's per-token inputs into shared memory (forward: v; reverse: q, d_o and the taped u)
     auto stage = [&](int c0, int L, bool rev) {
         __syncthreads();   // the previous chunk is done with the staged inputs
-#pragma unroll 8
-        for (int tt = 0; tt < L; ++tt) {
-            const size_t e = ((size_t)(c0 + tt) * H + h) * dk + i;
-            al_s[tt * dk + i] = ldf(alpha + e);
-            k_s[tt * dk + i] = ldf(k + e);
-            g_s[tt * dk + i] = w.g[e];
-            if (rev) q_s[tt * dk + i] = ldf(q + e);
+        const size_t row0 = ((size_t)c0 * H + h) * dk, vrow0 = ((size_t)c0 * H + h) * dv + col0;
+        const size_t rstride = (size_t)H * dk * sizeof(T), vstride = (size_t)H * dv * sizeof(T);
+        stage_rows(al_s, alpha + row0, rstride, L, dk * (int)sizeof(T));
+        stage_rows(k_s, k + row0, rstride, L, dk * (int)sizeof(T));
+        stage_rows(g_s, w.g + row0, (size_t)H * dk * 4, L, dk * 4);
+        if (rev) {
+            stage_rows(q_s, q + row0, rstride, L, dk * (int)sizeof(T));
+            stage_rows(do_s, d_o + vrow0, vstride, L, DB * (int)sizeof(T));
+            stage_rows(us, w.utape + vrow0, (size_t)H * dv * 4, L, DB * 4);
+        } else {
+            stage_rows(v_s, v + vrow0, vstride, L, DB * (int)sizeof(T));
         }
-        for (int x = i; x < L * DB; x += nt) {
-            const int tt = x / DB, j = x % DB;
-            const size_t e = ((size_t)(c0 + tt) * H + h) * dv + col0 + j;
-            v_s[x] = ldf(v + e);
-            if (rev) do_s[x] = ldf(d_o + e);
-        }
+        cp_async_wait_all();
         __syncthreads();
     };
-    // u_j = v_j - sum_i alpha_i k_i S_ij for staged token tt -> dst[DB] (shared), then into u
-    auto forward_u = [&](int tt, const float (&S)[16], float *dst, float (&u)[16]) {
-        const float ak = al_s[tt * dk + i] * k_s[tt * dk + i];
+    // u_j = v_j - sum_i alpha_i k_i S_ij for staged token tt of the chunk at c0 -> the u tape and
+    // dst[DB] (shared), then into u
+    auto forward_u = [&](int c0, int tt, const float (&S)[16], float *dst, float (&u)[16]) {
+        const float ak = lds(al_s + tt * dk + i) * lds(k_s + tt * dk + i);
         float p[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) p[j] = ak * S[j];
@@ -192,14 +221,15 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
         if (i < DB) {
             float x = 0.f;
             for (int ww = 0; ww < nw; ++ww) x += red[ww * DB + i];
-            dst[i] = v_s[tt * DB + i] - x;
+            dst[i] = lds(v_s + tt * DB + i) - x;
+            w.utape[((size_t)(c0 + tt) * H + h) * dv + col0 + i] = dst[i];
         }
         __syncthreads();
 #pragma unroll
         for (int j = 0; j < 16; ++j) u[j] = dst[j];
     };
     auto step = [&](int tt, float (&S)[16], const float (&u)[16]) {
-        const float al = al_s[tt * dk + i], gg = g_s[tt * dk + i];
+        const float al = lds(al_s + tt * dk + i), gg = g_s[tt * dk + i];
 #pragma unroll
         for (int j = 0; j < 16; ++j) S[j] = fmaf(gg, u[j], al * S[j]);
     };
@@ -217,7 +247,7 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
         for (int j = 0; j < 16; ++j) ck[j * dk + i] = S[j];
         stage(c0, L, false);
         for (int tt = 0; tt < L; ++tt) {
-            forward_u(tt, S, uh, u);
+            forward_u(c0, tt, S, uh, u);
             step(tt, S, u);
         }
     }
@@ -236,7 +266,8 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
 #pragma unroll
                 for (int j = 0; j < 16; ++j) sub[((tt / NS) * DB + j) * dk + i] = S[j];
             }
-            forward_u(tt, S, us + tt * DB, u);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) u[j] = us[tt * DB + j];
             step(tt, S, u);
         }
         for (int js = (L - 1) / NS; js >= 0; --js) {
@@ -251,11 +282,12 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
                     for (int j = 0; j < 16; ++j) uu[j] = us[oo * DB + j];
                     step(oo, Sp, uu);
                 }
-                const float al = al_s[tt * dk + i], kk = k_s[tt * dk + i], gg = g_s[tt * dk + i], qq = q_s[tt * dk + i];
+                const float al = lds(al_s + tt * dk + i), kk = lds(k_s + tt * dk + i), gg = g_s[tt * dk + i];
+                const float qq = lds(q_s + tt * dk + i);
                 float dqp = 0.f, gp = 0.f, p[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const float uj = us[tt * DB + j], doj = do_s[tt * DB + j];
+                    const float uj = us[tt * DB + j], doj = lds(do_s + tt * DB + j);
                     const float St = fmaf(gg, uj, al * Sp[j]);
                     Sh[j] = fmaf(qq, doj, Sh[j]);
                     dqp = fmaf(St, doj, dqp);
@@ -296,34 +328,31 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
     }
 }
 
-// ================================================================= prev
-// dynamic shared memory, per group of GT tokens: g^, k^ (S part), alpha^ (S part), scratch,
-// alpha, sigma, k, P before the token [GT][dk] each; den^, r, den [GT].  NB = number of
-// column blocks (d_v / 16), a template argument so that every partial load is issued at once.
+// ================================================================= local
+// One warp per (token, head), lanes over the key channels.  Sums the NB column-block partials;
+// writes dq and den^ = -(g^ . g) / den, and overwrites block 0's partial slots 1..3 with
+//   A  = g^ k / den + den^ k^2                      (P^-^ without the later tokens' part)
+//   Kl = k^_S + g^ P^- / den + 2 den^ P^- k         (k^ without the uncertainty-update part)
+//   alpha^_S                                        (summed)
 template <typename T, int NB>
-__global__ void __launch_bounds__(128) bwd_prev_kernel(const BwdArgs b, const BwdWs w)
+__global__ void __launch_bounds__(256) bwd_local_kernel(const BwdArgs b, const BwdWs w)
 {
-    extern __shared__ float smf[];
     const TokenArgs &a = b.a;
     const int dk = a.dk, H = a.H;
-    float *gh_s = smf, *ks_s = gh_s + GT * dk, *as_s = ks_s + GT * dk, *x_s = as_s + GT * dk;
-    float *al_s = x_s + GT * dk, *sg_s = al_s + GT * dk, *k_s = sg_s + GT * dk, *pp_s = k_s + GT * dk;
-    float *dd_s = pp_s + GT * dk, *r_s = dd_s + GT, *den_s = r_s + GT;
+    const long long th = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (th >= w.ntok * H) return;
     const T *alpha = static_cast<const T *>(a.alpha), *sigma = static_cast<const T *>(a.sigma);
-    const T *k = static_cast<const T *>(a.k), *r = static_cast<const T *>(a.r);
-    const int chain = blockIdx.x, s = chain / H, h = chain % H;
-    const int i = threadIdx.x, warp = i >> 5, lane = i & 31, nw = dk >> 5;
-    const float mu = a.mu;
+    const T *k = static_cast<const T *>(a.k);
     const size_t tokstride = (size_t)w.ntok * H * dk;
-    int t0, t1;
-    seq_range(a, s, t0, t1);
-    float Ph = b.dP_T ? b.dP_T[(size_t)chain * dk + i] : 0.f;
-    for (int te = t1; te > t0; te -= GT) {
-        const int tb = max(t0, te - GT), n = te - tb;
-        // stage the group: partial sums over the column blocks, the inputs, the tapes
-#pragma unroll 4
-        for (int tt = 0; tt < n; ++tt) {
-            const size_t e = ((size_t)(tb + tt) * H + h) * dk + i;
+    const float dn = w.den[th];
+    float gh[4], kS[4], aS[4], xg = 0.f;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int c = lane + 32 * m;
+        gh[m] = kS[m] = aS[m] = 0.f;
+        if (c < dk) {
+            const size_t e = (size_t)th * dk + c;
             float p4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int bb = 0; bb < NB; ++bb) {
@@ -334,42 +363,80 @@ __global__ void __launch_bounds__(128) bwd_prev_kernel(const BwdArgs b, const Bw
                 p4[3] += pp[3 * tokstride];
             }
             b.dq[e] = p4[0];
-            gh_s[tt * dk + i] = p4[1];
-            ks_s[tt * dk + i] = p4[2];
-            as_s[tt * dk + i] = p4[3];
-            x_s[tt * dk + i] = p4[1] * w.g[e];
-            al_s[tt * dk + i] = ldf(alpha + e);
-            sg_s[tt * dk + i] = ldf(sigma + e);
-            k_s[tt * dk + i] = ldf(k + e);
-            pp_s[tt * dk + i] = w.Pprev[e];
+            gh[m] = p4[1];
+            kS[m] = p4[2];
+            aS[m] = p4[3];
+            xg = fmaf(p4[1], w.g[e], xg);
         }
+    }
+    const float dd = -warp_sum(xg) / dn;
+    if (lane == 0) w.dden[th] = dd;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int c = lane + 32 * m;
+        if (c < dk) {
+            const size_t e = (size_t)th * dk + c;
+            const float al = ldf(alpha + e), kk = ldf(k + e);
+            const float pm = fmaf(al * al, w.Pprev[e], ldf(sigma + e));
+            float *pp = w.part + e;
+            pp[tokstride] = gh[m] * kk / dn + dd * kk * kk;
+            pp[2 * tokstride] = kS[m] + gh[m] * pm / dn + 2.f * dd * pm * kk;
+            pp[3 * tokstride] = aS[m];
+        }
+    }
+}
+
+// ================================================================= prev
+// dynamic shared memory, per group of GT tokens: A, Kl, alpha^_S, P before the token [GT][dk]
+// fp32; r-terms [GT][dk]; r, den^ [GT]; alpha, sigma, k rows [GT][dk] in the input type
+template <typename T>
+__global__ void __launch_bounds__(128) bwd_prev_kernel(const BwdArgs b, const BwdWs w)
+{
+    extern __shared__ float smf[];
+    const TokenArgs &a = b.a;
+    const int dk = a.dk, H = a.H;
+    float *A_s = smf, *K_s = A_s + GT * dk, *aS_s = K_s + GT * dk, *pp_s = aS_s + GT * dk, *x_s = pp_s + GT * dk;
+    float *r_s = x_s + GT * dk, *dd_s = r_s + GT;
+    T *al_s = reinterpret_cast<T *>(dd_s + GT), *sg_s = al_s + GT * dk, *k_s = sg_s + GT * dk;
+    const T *alpha = static_cast<const T *>(a.alpha), *sigma = static_cast<const T *>(a.sigma);
+    const T *k = static_cast<const T *>(a.k), *r = static_cast<const T *>(a.r);
+    const int chain = blockIdx.x, s = chain / H, h = chain % H;
+    const int i = threadIdx.x, warp = i >> 5, lane = i & 31, nw = dk >> 5;
+    const float mu = a.mu;
+    const size_t tokstride = (size_t)w.ntok * H * dk;
+    const size_t rstride = (size_t)H * dk * sizeof(T), fstride = (size_t)H * dk * 4;
+    int t0, t1;
+    seq_range(a, s, t0, t1);
+    float Ph = b.dP_T ? b.dP_T[(size_t)chain * dk + i] : 0.f;
+    for (int te = t1; te > t0; te -= GT) {
+        const int tb = max(t0, te - GT), n = te - tb;
+        const size_t row0 = ((size_t)tb * H + h) * dk;
+        stage_rows(A_s, w.part + tokstride + row0, fstride, n, dk * 4);
+        stage_rows(K_s, w.part + 2 * tokstride + row0, fstride, n, dk * 4);
+        stage_rows(aS_s, w.part + 3 * tokstride + row0, fstride, n, dk * 4);
+        stage_rows(pp_s, w.Pprev + row0, fstride, n, dk * 4);
+        stage_rows(al_s, alpha + row0, rstride, n, dk * (int)sizeof(T));
+        stage_rows(sg_s, sigma + row0, rstride, n, dk * (int)sizeof(T));
+        stage_rows(k_s, k + row0, rstride, n, dk * (int)sizeof(T));
         if (i < n) {
             r_s[i] = ldf(r + (size_t)(tb + i) * H + h);
-            den_s[i] = w.den[(size_t)(tb + i) * H + h];
+            dd_s[i] = w.dden[(size_t)(tb + i) * H + h];
         }
-        __syncthreads();
-        for (int tt = warp; tt < n; tt += nw) {
-            float x = 0.f;
-            for (int c = lane; c < dk; c += 32) x += x_s[tt * dk + c];
-            x = warp_sum(x);
-            if (lane == 0) dd_s[tt] = -x / den_s[tt];
-        }
+        cp_async_wait_all();
         __syncthreads();
         for (int tt = n - 1; tt >= 0; --tt) {
             const size_t e = ((size_t)(tb + tt) * H + h) * dk + i;
-            const float al = al_s[tt * dk + i], kk = k_s[tt * dk + i], rr = r_s[tt], dn = den_s[tt];
-            const float Pp = pp_s[tt * dk + i];
-            const float pm = fmaf(al * al, Pp, sg_s[tt * dk + i]);
-            const float c = mu * kk * kk / rr;
-            const float z = 1.f / (1.f + c * pm);
+            const int o = tt * dk + i;
+            const float al = lds(al_s + o), kk = lds(k_s + o), rr = r_s[tt], Pp = pp_s[o];
+            const float pm = fmaf(al * al, Pp, lds(sg_s + o));
+            const float z = 1.f / (1.f + mu * kk * kk / rr * pm);
             const float Pt = pm * z;
-            const float gh = gh_s[tt * dk + i], dd = dd_s[tt];
-            const float pmh = gh * kk / dn + dd * kk * kk + Ph * z * z;
+            const float pmh = A_s[o] + Ph * z * z;
             const float ch = -Ph * Pt * Pt;
-            b.dk[e] = ks_s[tt * dk + i] + gh * pm / dn + 2.f * dd * pm * kk + ch * 2.f * mu * kk / rr;
-            x_s[tt * dk + i] = -ch * mu * kk * kk / (rr * rr);
+            b.dk[e] = K_s[o] + ch * 2.f * mu * kk / rr;
+            x_s[o] = -ch * mu * kk * kk / (rr * rr);
             b.dsigma[e] = pmh;
-            b.dalpha[e] = as_s[tt * dk + i] + 2.f * al * Pp * pmh;
+            b.dalpha[e] = aS_s[o] + 2.f * al * Pp * pmh;
             Ph = al * al * pmh;
         }
         __syncthreads();
@@ -396,32 +463,44 @@ size_t backward_workspace_bytes(long long ntok, int nseq, int H, int dk, int dv)
     n += align256(th * dk * 4);                                     // P before each token
     n += align256(th * dk * 4);                                     // g
     n += align256(th * 4);                                          // den
+    n += align256(th * 4);                                          // den^
+    n += align256(th * dv * 4);                                     // u of every token
     n += align256((size_t)ckpt_slots(ntok, nseq) * H * dk * dv * 4);   // S checkpoints
     n += align256((size_t)4 * (dv / DB) * th * dk * 4);             // per-column-block partials
     return n;
 }
 
+template <typename T, int NB>
+static cudaError_t launch_local(const BwdArgs &b, const BwdWs &w, cudaStream_t st) {
+    const long long rows = w.ntok * b.a.H;
+    if (rows == 0) return cudaSuccess;
+    bwd_local_kernel<T, NB><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(b, w);
+    return cudaGetLastError();
+}
+
 template <typename T>
 static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, cudaStream_t st) {
     const int chains = b.a.nseq * b.a.H, dk = b.a.dk;
-    const size_t tsm = ((size_t)5 * GT * dk + 2 * GT) * sizeof(float);
+    const size_t tsm = ((size_t)2 * GT * dk + 2 * GT) * sizeof(float) + (size_t)3 * GT * dk * sizeof(T);
     cudaError_t e = cudaFuncSetAttribute(bwd_tape_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
     if (e != cudaSuccess) return e;
     bwd_tape_kernel<T><<<chains, dk, tsm, st>>>(b, w);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t ssm = ((size_t)4 * CK * dk + 2 * CK * DB + (CK / NS) * DB * dk + CK * DB + 4 * DB + DB) * sizeof(float);
+    const size_t ssm = ((size_t)CK * dk + (CK / NS) * DB * dk + CK * DB + 4 * DB + DB) * sizeof(float) +
+                       ((size_t)3 * CK * dk + CK * DB) * sizeof(T);
     e = cudaFuncSetAttribute(bwd_state_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
     if (e != cudaSuccess) return e;
     bwd_state_kernel<T><<<(unsigned)chains * w.nblk, dk, ssm, st>>>(b, w);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t psm = ((size_t)8 * GT * dk + 3 * GT) * sizeof(float);
-    auto prev = w.nblk == 2 ? bwd_prev_kernel<T, 2> : w.nblk == 4 ? bwd_prev_kernel<T, 4>
-              : w.nblk == 8 ? bwd_prev_kernel<T, 8> : bwd_prev_kernel<T, 16>;
-    e = cudaFuncSetAttribute(prev, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
+    e = w.nblk == 2 ? launch_local<T, 2>(b, w, st) : w.nblk == 4 ? launch_local<T, 4>(b, w, st)
+      : w.nblk == 8 ? launch_local<T, 8>(b, w, st) : launch_local<T, 16>(b, w, st);
     if (e != cudaSuccess) return e;
-    prev<<<chains, dk, psm, st>>>(b, w);
+    const size_t psm = ((size_t)5 * GT * dk + 2 * GT) * sizeof(float) + (size_t)3 * GT * dk * sizeof(T);
+    e = cudaFuncSetAttribute(bwd_prev_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
+    if (e != cudaSuccess) return e;
+    bwd_prev_kernel<T><<<chains, dk, psm, st>>>(b, w);
     return cudaGetLastError();
 }
 
@@ -435,6 +514,8 @@ cudaError_t launch_backward(const BwdArgs &b, bool bf16_in, long long ntok, void
     w.Pprev = reinterpret_cast<float *>(p); p += align256(th * a.dk * 4);
     w.g = reinterpret_cast<float *>(p); p += align256(th * a.dk * 4);
     w.den = reinterpret_cast<float *>(p); p += align256(th * 4);
+    w.dden = reinterpret_cast<float *>(p); p += align256(th * 4);
+    w.utape = reinterpret_cast<float *>(p); p += align256(th * a.dv * 4);
     w.ckpt = reinterpret_cast<float *>(p); p += align256((size_t)ckpt_slots(ntok, a.nseq) * a.H * a.dk * a.dv * 4);
     w.part = reinterpret_cast<float *>(p);
     return bf16_in ? launch_bwd_typed<bf16>(b, w, st) : launch_bwd_typed<float>(b, w, st);
