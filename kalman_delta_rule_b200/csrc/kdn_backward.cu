@@ -20,7 +20,7 @@
 //         the memory forward with S checkpoints every 32 tokens and u of every token taped, then
 //         the reverse sweep chunk by chunk: the chunk's inputs are staged in shared memory, the
 //         chunk is re-stepped from its checkpoint (with the taped u, so without the cross-row
-//         reduction) into shared-memory sub-checkpoints every 8 tokens, and the
+//         reduction) into shared-memory sub-checkpoints every 4 tokens, and the
 //         state before each token is re-stepped from the nearest sub-checkpoint (never
 //         reconstructed by dividing by alpha, which loses it when alpha is small).  Writes dv and,
 //         per column block, partial sums over its columns of dq, g^, the S-part of k^ and the
@@ -41,7 +41,7 @@ namespace kdn {
 namespace {
 constexpr int DB = 16;    // d_v columns per state CTA
 constexpr int CK = 32;    // tokens between the DRAM checkpoints of S
-constexpr int NS = 8;     // tokens between the shared-memory sub-checkpoints
+constexpr int NS = 4;     // tokens between the shared-memory sub-checkpoints
 constexpr int GT = 32;    // tokens per group in the uncertainty kernels
 
 struct BwdWs {
@@ -68,6 +68,14 @@ __device__ __forceinline__ void stage_rows(void *dst, const void *src, size_t st
     }
 }
 __device__ __forceinline__ float lds(const float *p) { return *p; }
+// 16 consecutive floats of shared memory (16-byte aligned) into registers
+__device__ __forceinline__ void lds16(const float *p, float (&x)[16]) {
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+        const float4 f = reinterpret_cast<const float4 *>(p)[q4];
+        x[4 * q4] = f.x; x[4 * q4 + 1] = f.y; x[4 * q4 + 2] = f.z; x[4 * q4 + 3] = f.w;
+    }
+}
 __device__ __forceinline__ float lds(const bf16 *p) {
     return __uint_as_float(((unsigned)*reinterpret_cast<const unsigned short *>(p)) << 16);
 }
@@ -162,7 +170,7 @@ __global__ void __launch_bounds__(128) bwd_tape_kernel(const BwdArgs b, const Bw
 
 // ================================================================= state
 // dynamic shared memory, per chunk of CK tokens: g rows [CK][dk] fp32; sub-checkpoints
-// [CK/NS][DB][dk]; u per token [CK][DB]; reduction partials [4][DB]; u^ [DB]; then alpha, k, q
+// [CK/NS][DB/4][dk] float4; u per token [CK][DB]; reduction partials [4][DB]; u^ [DB]; then alpha, k, q
 // rows [CK][dk] and the column block of v (forward) or d_o (reverse) [CK][DB] in the input type
 template <typename T>
 __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, const BwdWs w)
@@ -171,7 +179,7 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
     const TokenArgs &a = b.a;
     const int dk = a.dk, dv = a.dv, H = a.H;
     float *g_s = smf;
-    float *sub = g_s + CK * dk;               // [CK/NS][DB][dk]
+    float *sub = g_s + CK * dk;               // [CK/NS][DB/4][dk] float4 (thread i's 16 columns, conflict-free)
     float *us = sub + (CK / NS) * DB * dk;    // [CK][DB]
     float *red = us + CK * DB;                // [4][DB]
     float *uh = red + 4 * DB;                 // [DB]
@@ -225,8 +233,7 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
             w.utape[((size_t)(c0 + tt) * H + h) * dv + col0 + i] = dst[i];
         }
         __syncthreads();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) u[j] = dst[j];
+        lds16(dst, u);
     };
     auto step = [&](int tt, float (&S)[16], const float (&u)[16]) {
         const float al = lds(al_s + tt * dk + i), gg = g_s[tt * dk + i];
@@ -263,11 +270,12 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
         stage(c0, L, true);
         for (int tt = 0; tt < L; ++tt) {
             if (tt % NS == 0) {
+                float4 *sb = reinterpret_cast<float4 *>(sub) + (size_t)(tt / NS) * 4 * dk + i;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) sub[((tt / NS) * DB + j) * dk + i] = S[j];
+                for (int q4 = 0; q4 < 4; ++q4)
+                    sb[q4 * dk] = make_float4(S[4 * q4], S[4 * q4 + 1], S[4 * q4 + 2], S[4 * q4 + 3]);
             }
-#pragma unroll
-            for (int j = 0; j < 16; ++j) u[j] = us[tt * DB + j];
+            lds16(us + tt * DB, u);
             step(tt, S, u);
         }
         for (int js = (L - 1) / NS; js >= 0; --js) {
@@ -275,19 +283,25 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
                 const int t = c0 + tt;
                 // state before token t, re-stepped from the sub-checkpoint
                 float Sp[16], uu[16];
+                {
+                    const float4 *sb = reinterpret_cast<const float4 *>(sub) + (size_t)js * 4 * dk + i;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) Sp[j] = sub[(js * DB + j) * dk + i];
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float4 f = sb[q4 * dk];
+                        Sp[4 * q4] = f.x; Sp[4 * q4 + 1] = f.y; Sp[4 * q4 + 2] = f.z; Sp[4 * q4 + 3] = f.w;
+                    }
+                }
                 for (int oo = js * NS; oo < tt; ++oo) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) uu[j] = us[oo * DB + j];
+                    lds16(us + oo * DB, uu);
                     step(oo, Sp, uu);
                 }
                 const float al = lds(al_s + tt * dk + i), kk = lds(k_s + tt * dk + i), gg = g_s[tt * dk + i];
                 const float qq = lds(q_s + tt * dk + i);
                 float dqp = 0.f, gp = 0.f, p[16];
+                lds16(us + tt * DB, uu);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const float uj = us[tt * DB + j], doj = lds(do_s + tt * DB + j);
+                    const float uj = uu[j], doj = lds(do_s + tt * DB + j);
                     const float St = fmaf(gg, uj, al * Sp[j]);
                     Sh[j] = fmaf(qq, doj, Sh[j]);
                     dqp = fmaf(St, doj, dqp);
@@ -306,9 +320,10 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
                 }
                 __syncthreads();
                 float kp = 0.f, ap = 0.f;
+                lds16(uh, uu);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const float uhj = uh[j];
+                    const float uhj = uu[j];
                     const float Wh = fmaf(-kk, uhj, Sh[j]);
                     kp = fmaf(al * Sp[j], uhj, kp);
                     ap = fmaf(Wh, Sp[j], ap);
