@@ -115,16 +115,16 @@ __device__ __forceinline__ float reduce16(float (&v)[16], int lane, int &which) 
 }  // namespace
 
 // ================================================================= tape
-// dynamic shared memory: alpha, sigma, k rows of a group [GT][dk] (input type); P^- and P^- k^2
-// [GT][dk]; den, r [GT]
+// dynamic shared memory: P^- and P^- k^2 [GT][dk]; den, r, 1/r [GT]; alpha, sigma, k rows of a
+// group [GT][dk] (input type)
 template <typename T>
 __global__ void __launch_bounds__(128) bwd_tape_kernel(const BwdArgs b, const BwdWs w)
 {
     extern __shared__ float smf[];
     const TokenArgs &a = b.a;
     const int dk = a.dk, H = a.H;
-    float *pm_s = smf, *x_s = pm_s + GT * dk, *den_s = x_s + GT * dk, *r_s = den_s + GT;
-    T *al_s = reinterpret_cast<T *>(r_s + GT), *sg_s = al_s + GT * dk, *k_s = sg_s + GT * dk;
+    float *pm_s = smf, *x_s = pm_s + GT * dk, *den_s = x_s + GT * dk, *r_s = den_s + GT, *ir_s = r_s + GT;
+    T *al_s = reinterpret_cast<T *>(ir_s + 2 * GT), *sg_s = al_s + GT * dk, *k_s = sg_s + GT * dk;
     const T *alpha = static_cast<const T *>(a.alpha), *sigma = static_cast<const T *>(a.sigma);
     const T *k = static_cast<const T *>(a.k), *r = static_cast<const T *>(a.r);
     const int chain = blockIdx.x, s = chain / H, h = chain % H;
@@ -140,7 +140,11 @@ __global__ void __launch_bounds__(128) bwd_tape_kernel(const BwdArgs b, const Bw
         stage_rows(al_s, alpha + row0, rstride, n, rbytes);
         stage_rows(sg_s, sigma + row0, rstride, n, rbytes);
         stage_rows(k_s, k + row0, rstride, n, rbytes);
-        if (i < n) r_s[i] = ldf(r + (size_t)(tb + i) * H + h);
+        if (i < n) {
+            const float rr = ldf(r + (size_t)(tb + i) * H + h);
+            r_s[i] = rr;
+            ir_s[i] = 1.f / rr;
+        }
         cp_async_wait_all();
         __syncthreads();
         for (int tt = 0; tt < n; ++tt) {
@@ -149,7 +153,7 @@ __global__ void __launch_bounds__(128) bwd_tape_kernel(const BwdArgs b, const Bw
             const float pm = fmaf(al * al, P, lds(sg_s + tt * dk + i));
             pm_s[tt * dk + i] = pm;
             x_s[tt * dk + i] = pm * kk * kk;
-            P = pm / (1.f + a.mu * kk * kk * pm / r_s[tt]);
+            P = pm / fmaf(a.mu * kk * kk * ir_s[tt], pm, 1.f);
         }
         __syncthreads();
         for (int tt = warp; tt < n; tt += nw) {
@@ -403,7 +407,7 @@ __global__ void __launch_bounds__(256) bwd_local_kernel(const BwdArgs b, const B
 
 // ================================================================= prev
 // dynamic shared memory, per group of GT tokens: A, Kl, alpha^_S, P before the token [GT][dk]
-// fp32; r-terms [GT][dk]; r, den^ [GT]; alpha, sigma, k rows [GT][dk] in the input type
+// fp32; r-terms [GT][dk]; 1/r, den^ [GT]; alpha, sigma, k rows [GT][dk] in the input type
 template <typename T>
 __global__ void __launch_bounds__(128) bwd_prev_kernel(const BwdArgs b, const BwdWs w)
 {
@@ -434,7 +438,7 @@ __global__ void __launch_bounds__(128) bwd_prev_kernel(const BwdArgs b, const Bw
         stage_rows(sg_s, sigma + row0, rstride, n, dk * (int)sizeof(T));
         stage_rows(k_s, k + row0, rstride, n, dk * (int)sizeof(T));
         if (i < n) {
-            r_s[i] = ldf(r + (size_t)(tb + i) * H + h);
+            r_s[i] = 1.f / ldf(r + (size_t)(tb + i) * H + h);   // 1/r
             dd_s[i] = w.dden[(size_t)(tb + i) * H + h];
         }
         cp_async_wait_all();
@@ -442,14 +446,15 @@ __global__ void __launch_bounds__(128) bwd_prev_kernel(const BwdArgs b, const Bw
         for (int tt = n - 1; tt >= 0; --tt) {
             const size_t e = ((size_t)(tb + tt) * H + h) * dk + i;
             const int o = tt * dk + i;
-            const float al = lds(al_s + o), kk = lds(k_s + o), rr = r_s[tt], Pp = pp_s[o];
+            const float al = lds(al_s + o), kk = lds(k_s + o), ir = r_s[tt], Pp = pp_s[o];
             const float pm = fmaf(al * al, Pp, lds(sg_s + o));
-            const float z = 1.f / (1.f + mu * kk * kk / rr * pm);
+            const float mk = mu * kk * ir;                 // mu k / r
+            const float z = 1.f / fmaf(mk * kk, pm, 1.f);
             const float Pt = pm * z;
             const float pmh = A_s[o] + Ph * z * z;
             const float ch = -Ph * Pt * Pt;
-            b.dk[e] = K_s[o] + ch * 2.f * mu * kk / rr;
-            x_s[o] = -ch * mu * kk * kk / (rr * rr);
+            b.dk[e] = K_s[o] + ch * 2.f * mk;
+            x_s[o] = -ch * mk * kk * ir;
             b.dsigma[e] = pmh;
             b.dalpha[e] = aS_s[o] + 2.f * al * Pp * pmh;
             Ph = al * al * pmh;
@@ -496,7 +501,7 @@ static cudaError_t launch_local(const BwdArgs &b, const BwdWs &w, cudaStream_t s
 template <typename T>
 static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, cudaStream_t st) {
     const int chains = b.a.nseq * b.a.H, dk = b.a.dk;
-    const size_t tsm = ((size_t)2 * GT * dk + 2 * GT) * sizeof(float) + (size_t)3 * GT * dk * sizeof(T);
+    const size_t tsm = ((size_t)2 * GT * dk + 4 * GT) * sizeof(float) + (size_t)3 * GT * dk * sizeof(T);
     cudaError_t e = cudaFuncSetAttribute(bwd_tape_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
     if (e != cudaSuccess) return e;
     bwd_tape_kernel<T><<<chains, dk, tsm, st>>>(b, w);
