@@ -272,28 +272,57 @@ def bench_prefill(args, world, rank, dev, kdn):
         iso = dict(value=i_value, ms_per_step=i_ms / n_iso, gpu_launches=n_iso * launches_per_step,
                    path=kdn.execution_path(d["q"], d["v"], cu_seqlens=cu, chunk=w.chunk, variant="isotropic"))
 
-    # end to end through the C ABI: pinned host inputs -> device, forward, o -> host
+    # end to end through the C ABI: every step copies its inputs from pinned host memory to the
+    # device, runs the forward and copies o back to pinned host memory.  Steps are pipelined over
+    # three streams and two device buffer sets: the copy-in of step n+1 and the copy-out of step
+    # n-1 overlap the forward of step n (the two copy directions use separate copy engines).
     pinned = {n: torch.from_numpy(np.ascontiguousarray(host[n]).view(np.int16) if host[n].dtype == np.uint16
                                   else np.ascontiguousarray(host[n])).pin_memory() for n in names}
-    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    o_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
-    d2h = o_host.numel() * o_host.element_size()
+    d2h = o_host[0].numel() * o_host[0].element_size()
+    dd = [d, {n: torch.empty_like(d[n]) for n in names}]
+    oo = [o, torch.empty_like(o)]
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev = lambda: torch.cuda.Event()
+    fwd_done = [ev(), ev()]     # the forward of the slot's previous step has read its inputs
+    out_done = [ev(), ev()]     # the slot's previous o has reached the host
+    for sl in range(2):
+        fwd_done[sl].record(stream)
+        out_done[sl].record(stream)
 
-    def e2e_step():
-        for n in names:
-            dst = d[n].view(torch.int16) if d[n].dtype == torch.bfloat16 else d[n]
-            dst.copy_(pinned[n], non_blocking=True)
-        step()
-        o_host.copy_(o, non_blocking=True)
+    def e2e_step(n):
+        sl = n % 2
+        di, do_, in_ready, o_ready = dd[sl], oo[sl], ev(), ev()
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(fwd_done[sl])
+            for nm in names:
+                dst = di[nm].view(torch.int16) if di[nm].dtype == torch.bfloat16 else di[nm]
+                dst.copy_(pinned[nm], non_blocking=True)
+            in_ready.record(s_in)
+        stream.wait_event(in_ready)
+        stream.wait_event(out_done[sl])
+        kdn.forward(di["q"], di["k"], di["v"], di["alpha"], di["sigma"], di["r"], cu_seqlens=cu, mu=w.mu,
+                    chunk=w.chunk, o=do_, S_out=S_out, P_out=P_out, workspace=ws, max_seqlen=max_seqlen, stream=stream)
+        fwd_done[sl].record(stream)
+        o_ready.record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(o_ready)
+            o_host[sl].copy_(do_, non_blocking=True)
+            out_done[sl].record(s_out)
 
-    for _ in range(max(1, args.warmup // 2)):
-        e2e_step()
+    for i in range(max(2, args.warmup // 2)):
+        e2e_step(i)
+    torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_steps = max(3, min(args.steps, 10))
+    e_steps = max(4, min(args.steps, 10))
     e0.record(stream)
-    for _ in range(e_steps):
-        e2e_step()
+    s_in.wait_event(e0)
+    for i in range(e_steps):
+        e2e_step(i)
+    stream.wait_event(out_done[(e_steps - 1) % 2])
+    stream.wait_event(out_done[(e_steps - 2) % 2])
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
