@@ -1,8 +1,8 @@
 """Pins of the fp64 gradient oracle (oracle/kdn_grad.py) to things other than itself (CPU only).
 
-* its forward restatement equals the C oracle (an independent implementation, pinned on
+* its forward restatement equals the C oracle for both variants (an independent implementation, pinned on
   its own in test_oracle_pins.py);
-* every gradient equals central finite differences of the C oracle's forward;
+* every gradient equals central finite differences of the C oracle's forward (both variants);
 * single-token closed forms, derived by hand from the five steps of the recurrence;
 * a readout gradient at the first token does not depend on mu (mu scales only the
   uncertainty update, which acts from the next token on).
@@ -27,36 +27,41 @@ def rand_problem(rng, ntok, H, dk, dv):
     return q, k, v, alpha, sigma, r
 
 
-def c_loss(x, d_o, dS, dP, cu, mu):
+def c_loss(x, d_o, dS, dP, cu, mu, iso=False):
     q, k, v, alpha, sigma, r, S0, P0 = x
-    f = oracle.diag_forward(q, k, v, alpha, sigma, r, cu_seqlens=cu, S0=S0, P0=P0, mu=mu, threads=1)
+    fwd = oracle.iso_forward if iso else oracle.diag_forward
+    f = fwd(q, k, v, alpha, sigma, r, cu_seqlens=cu, S0=S0, P0=P0, mu=mu, threads=1)
     return float((f["o"] * d_o).sum() + (f["S"] * dS).sum() + (f["P"] * dP).sum())
 
 
-def test_restated_forward_equals_c_oracle():
+@pytest.mark.parametrize("iso", [False, True])
+def test_restated_forward_equals_c_oracle(iso):
     rng = np.random.default_rng(3)
     cu = np.array([0, 5, 12], dtype=np.int32)
     q, k, v, alpha, sigma, r = rand_problem(rng, 12, 2, 4, 3)
     S0 = 0.3 * rng.standard_normal((2, 2, 4, 3))
-    P0 = np.logaddexp(0, rng.standard_normal((2, 2, 4)))
-    ref = oracle.diag_forward(q, k, v, alpha, sigma, r, cu_seqlens=cu, S0=S0, P0=P0, mu=1.7)
-    g = kdn_grad.diag_grad(q, k, v, alpha, sigma, r, np.zeros((12, 2, 3)), cu_seqlens=cu, S0=S0, P0=P0, mu=1.7)
+    P0 = np.logaddexp(0, rng.standard_normal((2, 2) if iso else (2, 2, 4)))
+    fwd = oracle.iso_forward if iso else oracle.diag_forward
+    ref = fwd(q, k, v, alpha, sigma, r, cu_seqlens=cu, S0=S0, P0=P0, mu=1.7)
+    g = kdn_grad.diag_grad(q, k, v, alpha, sigma, r, np.zeros((12, 2, 3)), cu_seqlens=cu, S0=S0, P0=P0, mu=1.7,
+                           iso=iso)
     for n in ("o", "S", "P"):
         np.testing.assert_allclose(g[n], ref[n], rtol=1e-12, atol=1e-13)
 
 
-@pytest.mark.parametrize("mu", [1.0, 4.0])
-def test_gradients_equal_finite_differences_of_the_c_oracle(mu):
+@pytest.mark.parametrize("mu,iso", [(1.0, False), (4.0, False), (1.0, True), (4.0, True)])
+def test_gradients_equal_finite_differences_of_the_c_oracle(mu, iso):
     rng = np.random.default_rng(5)
     cu = np.array([0, 3, 7], dtype=np.int32)
     ntok, H, dk, dv = 7, 1, 3, 2
     q, k, v, alpha, sigma, r = rand_problem(rng, ntok, H, dk, dv)
+    pshape = (2, H) if iso else (2, H, dk)
     S0 = 0.5 * rng.standard_normal((2, H, dk, dv))
-    P0 = np.logaddexp(0, rng.standard_normal((2, H, dk)))
+    P0 = np.logaddexp(0, rng.standard_normal(pshape))
     d_o = rng.standard_normal((ntok, H, dv))
     dS = rng.standard_normal((2, H, dk, dv))
-    dP = rng.standard_normal((2, H, dk))
-    g = kdn_grad.diag_grad(q, k, v, alpha, sigma, r, d_o, cu_seqlens=cu, S0=S0, P0=P0, dS=dS, dP=dP, mu=mu)
+    dP = rng.standard_normal(pshape)
+    g = kdn_grad.diag_grad(q, k, v, alpha, sigma, r, d_o, cu_seqlens=cu, S0=S0, P0=P0, dS=dS, dP=dP, mu=mu, iso=iso)
     x = [q, k, v, alpha, sigma, r, S0, P0]
     names = ("dq", "dk", "dv", "dalpha", "dsigma", "dr", "dS0", "dP0")
     for i, name in enumerate(names):
@@ -67,7 +72,7 @@ def test_gradients_equal_finite_differences_of_the_c_oracle(mu):
             xm = [a.copy() for a in x]
             xp[i][idx] += h
             xm[i][idx] -= h
-            fd[idx] = (c_loss(xp, d_o, dS, dP, cu, mu) - c_loss(xm, d_o, dS, dP, cu, mu)) / (2 * h)
+            fd[idx] = (c_loss(xp, d_o, dS, dP, cu, mu, iso) - c_loss(xm, d_o, dS, dP, cu, mu, iso)) / (2 * h)
         np.testing.assert_allclose(g[name], fd, rtol=2e-6, atol=2e-7, err_msg=name)
 
 
