@@ -191,20 +191,20 @@ kdn_status_t kdn_gain_scan_noalloc(const kdn_problem_t *p,
                                    const void *k, const void *alpha, const void *sigma, const void *r,
                                    const float *P0, float *g, float *beta_eff, float *P_out, void *stream);
 
-/* Backward pass of the diagonal KDN, for training (KDA article, "chunkwise" section: the
- * chunkwise regime serves training; explainer "对角近似" for the recurrence differentiated).
+/* Backward pass of the KDN, for training (KDA article, "chunkwise" section: the chunkwise
+ * regime serves training; explainer "对角近似" and "各向同性近似" for the recurrences
+ * differentiated).
  * Computes the gradients of  L = <o, d_o> + <S_T, dS_T> + <P_T, dP_T>, where o, S_T and P_T are
  * what kdn_forward_chunkwise() returns for the same problem and inputs, with respect to every
  * input: the vector-Jacobian products of one training step.
- *  p                  : as for the forward (variant must be KDN_VARIANT_DIAGONAL, else
- *                       KDN_ERR_UNSUPPORTED; `chunk` and `max_seqlen` are ignored)
- *  q ... P0           : the forward's inputs, same layouts (S0 / P0 NULL = 0 / 1)
+ *  p                  : as for the forward, either variant (`chunk` and `max_seqlen` are ignored)
+ *  q ... P0           : the forward's inputs, same layouts (S0 / P0 NULL = 0 / 1; P0 [N, H] isotropic)
  *  d_o                : device [B, T, H, d_v] (in_dtype), gradient of L with respect to o
- *  dS_T, dP_T         : device fp32 [N, H, d_k, d_v], [N, H, d_k], gradients with respect to the
- *                       final S and P, or NULL (zero)
+ *  dS_T, dP_T         : device fp32 [N, H, d_k, d_v], [N, H, d_k] ([N, H] isotropic), gradients
+ *                       with respect to the final S and P, or NULL (zero)
  *  dq, dk, dalpha, dsigma : device fp32 [B, T, H, d_k];  dv : device fp32 [B, T, H, d_v]
  *  dr                 : device fp32 [B, T, H]
- *  dS0, dP0           : device fp32 [N, H, d_k, d_v], [N, H, d_k], or NULL (not written)
+ *  dS0, dP0           : device fp32 [N, H, d_k, d_v], [N, H, d_k] ([N, H] isotropic), or NULL (not written)
  *  workspace          : device, >= kdn_backward_workspace_size() bytes, 256-byte aligned
  *                       (contents on entry do not matter; distinct per concurrent call).
  * Method: the uncertainty forward is taped (P before each token, den, g), the memory forward

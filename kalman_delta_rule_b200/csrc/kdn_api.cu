@@ -239,7 +239,6 @@ kdn_status_t kdn_backward_workspace_size(const kdn_problem_t *p, size_t *bytes) 
     Resolved rv;
     kdn_status_t st = check_problem(p, &rv);
     if (st != KDN_OK) return st;
-    if (p->variant != KDN_VARIANT_DIAGONAL) return KDN_ERR_UNSUPPORTED;
     if (!bytes) return KDN_ERR_INVALID_ARG;
     *bytes = kdn::backward_workspace_bytes(rv.ntok, rv.nseq, p->H, p->d_k, p->d_v);
     return KDN_OK;
@@ -253,7 +252,6 @@ kdn_status_t kdn_backward(const kdn_problem_t *p, const void *q, const void *k, 
     Resolved rv;
     kdn_status_t st = check_problem(p, &rv);
     if (st != KDN_OK) return st;
-    if (p->variant != KDN_VARIANT_DIAGONAL) return KDN_ERR_UNSUPPORTED;
     if (rv.nseq == 0) return KDN_OK;
     if (rv.ntok > 0 && (!q || !k || !v || !alpha || !sigma || !r || !d_o || !dq || !dk || !dv || !dalpha ||
                         !dsigma || !dr))
@@ -269,7 +267,7 @@ kdn_status_t kdn_backward(const kdn_problem_t *p, const void *q, const void *k, 
     a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.sigma = sigma; a.r = r;
     a.S0 = S0; a.P0 = P0;
     a.cu = p->cu_seqlens; a.T = p->T; a.nseq = rv.nseq; a.H = p->H; a.dk = p->d_k; a.dv = p->d_v;
-    a.mu = p->mu; a.iso = 0; a.err = err_word();
+    a.mu = p->mu; a.iso = p->variant == KDN_VARIANT_ISOTROPIC; a.err = err_word();
     b.d_o = d_o; b.dS_T = dS_T; b.dP_T = dP_T;
     b.dq = dq; b.dk = dk; b.dv = dv; b.dalpha = dalpha; b.dsigma = dsigma; b.dr = dr; b.dS0 = dS0; b.dP0 = dP0;
     return cuda_status(kdn::launch_backward(b, rv.bf16, rv.ntok, workspace, static_cast<cudaStream_t>(stream)));

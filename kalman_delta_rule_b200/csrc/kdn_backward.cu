@@ -471,6 +471,194 @@ __global__ void __launch_bounds__(128) bwd_prev_kernel(const BwdArgs b, const Bw
     if (b.dP0) b.dP0[(size_t)chain * dk + i] = Ph;
 }
 
+// ================================================================= isotropic variant
+// One uncertainty p per head (explainer "各向同性近似"): p^- = a p + s with a = mean(alpha^2),
+// s = mean(sigma); g = p^- k / den, den = r + p^- K2, K2 = |k|^2; p' = p^- z, z = 1/(1 + c p^-),
+// c = mu K2 / (d_k r).  Adjoint of one token (p^ arrives from the later tokens):
+//     p^-^ = (g^.k - (g^.g) K2) / den + p^ z^2;   c^ = -p^ p'^2;   p^ <- a p^-^
+//     k^ = k^_S + g^ p^- / den - 2 (g^.g) p^- k / den + c^ 2 mu k / (d_k r)
+//     r^ = -(g^.g) / den - c^ mu K2 / (d_k r^2);  sigma^ = p^-^ / d_k;  alpha^ = alpha^_S + 2 alpha p p^-^ / d_k
+// The memory state pass is the diagonal one (it only needs g and alpha).  Per-token scalars
+// live in the first 8 floats of the (token, head) row of the P tape:
+//     [0] p before the token, [1] a, [3] K2, [4] the local part of p^-^, [5] the local part of r^, [6] p^-.
+namespace {
+constexpr int SC_P = 0, SC_A = 1, SC_K2 = 3, SC_AL = 4, SC_RL = 5, SC_PM = 6;
+}
+
+// dynamic shared memory: channel sums (alpha^2, sigma, k^2) [GT][4]; p^-, den, r [GT]; alpha,
+// sigma, k rows [GT][dk] in the input type
+template <typename T>
+__global__ void __launch_bounds__(128) bwd_tape_iso_kernel(const BwdArgs b, const BwdWs w)
+{
+    extern __shared__ float smf[];
+    const TokenArgs &a = b.a;
+    const int dk = a.dk, H = a.H;
+    float *sum_s = smf, *pm_s = sum_s + 4 * GT, *den_s = pm_s + GT, *r_s = den_s + GT;
+    T *al_s = reinterpret_cast<T *>(r_s + GT), *sg_s = al_s + GT * dk, *k_s = sg_s + GT * dk;
+    const T *alpha = static_cast<const T *>(a.alpha), *sigma = static_cast<const T *>(a.sigma);
+    const T *k = static_cast<const T *>(a.k), *r = static_cast<const T *>(a.r);
+    const int chain = blockIdx.x, s = chain / H, h = chain % H;
+    const int i = threadIdx.x, warp = i >> 5, lane = i & 31, nw = dk >> 5;
+    const size_t rstride = (size_t)H * dk * sizeof(T);
+    const int rbytes = dk * (int)sizeof(T);
+    const float inv_dk = 1.f / dk;
+    int t0, t1;
+    seq_range(a, s, t0, t1);
+    float p = a.P0 ? a.P0[chain] : 1.f;   // thread 0's running uncertainty
+    for (int tb = t0; tb < t1; tb += GT) {
+        const int n = min(GT, t1 - tb);
+        const size_t row0 = ((size_t)tb * H + h) * dk;
+        stage_rows(al_s, alpha + row0, rstride, n, rbytes);
+        stage_rows(sg_s, sigma + row0, rstride, n, rbytes);
+        stage_rows(k_s, k + row0, rstride, n, rbytes);
+        if (i < n) r_s[i] = ldf(r + (size_t)(tb + i) * H + h);
+        cp_async_wait_all();
+        __syncthreads();
+        for (int tt = warp; tt < n; tt += nw) {
+            float xa = 0.f, xs = 0.f, xk = 0.f;
+            for (int c = lane; c < dk; c += 32) {
+                const float al = lds(al_s + tt * dk + c), kk = lds(k_s + tt * dk + c);
+                xa = fmaf(al, al, xa);
+                xs += lds(sg_s + tt * dk + c);
+                xk = fmaf(kk, kk, xk);
+            }
+            xa = warp_sum(xa); xs = warp_sum(xs); xk = warp_sum(xk);
+            if (lane == 0) {
+                sum_s[tt * 4 + 0] = xa * inv_dk;
+                sum_s[tt * 4 + 1] = xs * inv_dk;
+                sum_s[tt * 4 + 2] = xk;
+            }
+        }
+        __syncthreads();
+        if (i == 0) {
+            for (int tt = 0; tt < n; ++tt) {
+                const size_t th = (size_t)(tb + tt) * H + h;
+                const float aa = sum_s[tt * 4 + 0], K2 = sum_s[tt * 4 + 2];
+                const float pm = fmaf(aa, p, sum_s[tt * 4 + 1]);
+                const float den = fmaf(pm, K2, r_s[tt]);
+                float *sc = w.Pprev + th * dk;
+                sc[SC_P] = p; sc[SC_A] = aa; sc[SC_K2] = K2; sc[SC_PM] = pm;
+                w.den[th] = den;
+                pm_s[tt] = pm;
+                den_s[tt] = den;
+                p = pm / fmaf(a.mu * K2 * inv_dk / r_s[tt], pm, 1.f);
+            }
+        }
+        __syncthreads();
+        for (int tt = 0; tt < n; ++tt)
+            w.g[((size_t)(tb + tt) * H + h) * dk + i] = pm_s[tt] * lds(k_s + tt * dk + i) / den_s[tt];
+        __syncthreads();
+    }
+}
+
+// one warp per (token, head): sums the column-block partials, writes dq, and the local parts
+// of k^ (block 0's slot 2), alpha^_S (slot 3), p^-^ and r^ (tape scalars)
+template <typename T, int NB>
+__global__ void __launch_bounds__(256) bwd_local_iso_kernel(const BwdArgs b, const BwdWs w)
+{
+    const TokenArgs &a = b.a;
+    const int dk = a.dk, H = a.H;
+    const long long th = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (th >= w.ntok * H) return;
+    const T *k = static_cast<const T *>(a.k);
+    const size_t tokstride = (size_t)w.ntok * H * dk;
+    float *sc = w.Pprev + (size_t)th * dk;
+    const float dn = w.den[th], pm = sc[SC_PM], K2 = sc[SC_K2];
+    float gh[4], kS[4], aS[4], kk[4], gk = 0.f, gg = 0.f;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int c = lane + 32 * m;
+        gh[m] = kS[m] = aS[m] = kk[m] = 0.f;
+        if (c < dk) {
+            const size_t e = (size_t)th * dk + c;
+            float p4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int bb = 0; bb < NB; ++bb) {
+                const float *pp = w.part + (size_t)bb * 4 * tokstride + e;
+                p4[0] += pp[0];
+                p4[1] += pp[tokstride];
+                p4[2] += pp[2 * tokstride];
+                p4[3] += pp[3 * tokstride];
+            }
+            b.dq[e] = p4[0];
+            gh[m] = p4[1];
+            kS[m] = p4[2];
+            aS[m] = p4[3];
+            kk[m] = ldf(k + e);
+            gk = fmaf(p4[1], kk[m], gk);
+            gg = fmaf(p4[1], w.g[e], gg);
+        }
+    }
+    gk = warp_sum(gk);
+    gg = warp_sum(gg);
+    if (lane == 0) {
+        sc[SC_AL] = (gk - gg * K2) / dn;
+        sc[SC_RL] = -gg / dn;
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int c = lane + 32 * m;
+        if (c < dk) {
+            float *pp = w.part + (size_t)th * dk + c;
+            pp[2 * tokstride] = kS[m] + gh[m] * pm / dn - 2.f * gg * pm * kk[m] / dn;
+            pp[3 * tokstride] = aS[m];
+        }
+    }
+}
+
+// dynamic shared memory, per group of GT tokens: local k^, alpha^_S [GT][dk] fp32; tape scalars
+// [GT][8]; 1/r [GT]; alpha, k rows [GT][dk] in the input type
+template <typename T>
+__global__ void __launch_bounds__(128) bwd_prev_iso_kernel(const BwdArgs b, const BwdWs w)
+{
+    extern __shared__ float smf[];
+    const TokenArgs &a = b.a;
+    const int dk = a.dk, H = a.H;
+    float *K_s = smf, *aS_s = K_s + GT * dk, *sc_s = aS_s + GT * dk, *ir_s = sc_s + 8 * GT;
+    T *al_s = reinterpret_cast<T *>(ir_s + GT), *k_s = al_s + GT * dk;
+    const T *alpha = static_cast<const T *>(a.alpha), *k = static_cast<const T *>(a.k);
+    const T *r = static_cast<const T *>(a.r);
+    const int chain = blockIdx.x, s = chain / H, h = chain % H;
+    const int i = threadIdx.x;
+    const float mu = a.mu, inv_dk = 1.f / dk;
+    const size_t tokstride = (size_t)w.ntok * H * dk;
+    const size_t rstride = (size_t)H * dk * sizeof(T), fstride = (size_t)H * dk * 4;
+    int t0, t1;
+    seq_range(a, s, t0, t1);
+    float ph = b.dP_T ? b.dP_T[chain] : 0.f;
+    for (int te = t1; te > t0; te -= GT) {
+        const int tb = max(t0, te - GT), n = te - tb;
+        const size_t row0 = ((size_t)tb * H + h) * dk;
+        stage_rows(K_s, w.part + 2 * tokstride + row0, fstride, n, dk * 4);
+        stage_rows(aS_s, w.part + 3 * tokstride + row0, fstride, n, dk * 4);
+        stage_rows(sc_s, w.Pprev + row0, fstride, n, 32);
+        stage_rows(al_s, alpha + row0, rstride, n, dk * (int)sizeof(T));
+        stage_rows(k_s, k + row0, rstride, n, dk * (int)sizeof(T));
+        if (i < n) ir_s[i] = 1.f / ldf(r + (size_t)(tb + i) * H + h);
+        cp_async_wait_all();
+        __syncthreads();
+        for (int tt = n - 1; tt >= 0; --tt) {
+            const size_t th = (size_t)(tb + tt) * H + h, e = th * dk + i;
+            const float *sc = sc_s + tt * 8;
+            const float pp = sc[SC_P], aa = sc[SC_A], K2 = sc[SC_K2], pm = sc[SC_PM], ir = ir_s[tt];
+            const float mk = mu * inv_dk * ir;            // mu / (d_k r)
+            const float z = 1.f / fmaf(mk * K2, pm, 1.f);
+            const float pt = pm * z;
+            const float pmh = sc[SC_AL] + ph * z * z;
+            const float ch = -ph * pt * pt;
+            const float al = lds(al_s + tt * dk + i), kk = lds(k_s + tt * dk + i);
+            b.dk[e] = K_s[tt * dk + i] + ch * 2.f * mk * kk;
+            b.dsigma[e] = pmh * inv_dk;
+            b.dalpha[e] = aS_s[tt * dk + i] + 2.f * al * pp * pmh * inv_dk;
+            if (i == 0) b.dr[th] = sc[SC_RL] - ch * mk * K2 * ir;
+            ph = aa * pmh;
+        }
+        __syncthreads();
+    }
+    if (b.dP0 && i == 0) b.dP0[chain] = ph;
+}
+
 // ================================================================= host
 namespace {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -494,17 +682,28 @@ template <typename T, int NB>
 static cudaError_t launch_local(const BwdArgs &b, const BwdWs &w, cudaStream_t st) {
     const long long rows = w.ntok * b.a.H;
     if (rows == 0) return cudaSuccess;
-    bwd_local_kernel<T, NB><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(b, w);
+    if (b.a.iso)
+        bwd_local_iso_kernel<T, NB><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(b, w);
+    else
+        bwd_local_kernel<T, NB><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(b, w);
     return cudaGetLastError();
 }
 
 template <typename T>
 static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, cudaStream_t st) {
     const int chains = b.a.nseq * b.a.H, dk = b.a.dk;
-    const size_t tsm = ((size_t)2 * GT * dk + 4 * GT) * sizeof(float) + (size_t)3 * GT * dk * sizeof(T);
-    cudaError_t e = cudaFuncSetAttribute(bwd_tape_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
-    if (e != cudaSuccess) return e;
-    bwd_tape_kernel<T><<<chains, dk, tsm, st>>>(b, w);
+    cudaError_t e;
+    if (b.a.iso) {
+        const size_t tsm = (size_t)7 * GT * sizeof(float) + (size_t)3 * GT * dk * sizeof(T);
+        e = cudaFuncSetAttribute(bwd_tape_iso_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+        if (e != cudaSuccess) return e;
+        bwd_tape_iso_kernel<T><<<chains, dk, tsm, st>>>(b, w);
+    } else {
+        const size_t tsm = ((size_t)2 * GT * dk + 4 * GT) * sizeof(float) + (size_t)3 * GT * dk * sizeof(T);
+        e = cudaFuncSetAttribute(bwd_tape_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+        if (e != cudaSuccess) return e;
+        bwd_tape_kernel<T><<<chains, dk, tsm, st>>>(b, w);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const size_t ssm = ((size_t)CK * dk + (CK / NS) * DB * dk + CK * DB + 4 * DB + DB) * sizeof(float) +
@@ -517,6 +716,13 @@ static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, cudaStream
     e = w.nblk == 2 ? launch_local<T, 2>(b, w, st) : w.nblk == 4 ? launch_local<T, 4>(b, w, st)
       : w.nblk == 8 ? launch_local<T, 8>(b, w, st) : launch_local<T, 16>(b, w, st);
     if (e != cudaSuccess) return e;
+    if (b.a.iso) {
+        const size_t psm = ((size_t)2 * GT * dk + 9 * GT) * sizeof(float) + (size_t)2 * GT * dk * sizeof(T);
+        e = cudaFuncSetAttribute(bwd_prev_iso_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
+        if (e != cudaSuccess) return e;
+        bwd_prev_iso_kernel<T><<<chains, dk, psm, st>>>(b, w);
+        return cudaGetLastError();
+    }
     const size_t psm = ((size_t)5 * GT * dk + 2 * GT) * sizeof(float) + (size_t)3 * GT * dk * sizeof(T);
     e = cudaFuncSetAttribute(bwd_prev_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
     if (e != cudaSuccess) return e;

@@ -134,10 +134,10 @@ def test_backward_validates_before_any_cuda_call(lib):
     assert B.kdn_backward(*args(d_o=FAKE + 2)) == B.KDN_ERR_INVALID_ARG
     bad = list(outs); bad[5] = None
     assert B.kdn_backward(*args(o=bad)) == B.KDN_ERR_INVALID_ARG
-    # diagonal uncertainty only; sizes as for the forward
+    # both variants, the same workspace; sizes as for the forward
     piso = problem(chunk=64, variant=1)
-    assert lib.kdn_backward_workspace_size(ctypes.byref(piso), ctypes.byref(ctypes.c_size_t())) == B.KDN_ERR_UNSUPPORTED
-    assert B.kdn_backward(piso, *args()[1:]) == B.KDN_ERR_UNSUPPORTED
+    assert B.kdn_backward_workspace_size(piso) == need
+    assert B.kdn_backward(piso, *args(ws=None)[1:]) == B.KDN_ERR_WORKSPACE
     assert B.kdn_backward(problem(d_k=48), *args()[1:]) == B.KDN_ERR_UNSUPPORTED
     assert B.kdn_backward(problem(num_seqs=0, B=0), *args()[1:]) == B.KDN_OK   # nothing to do
 

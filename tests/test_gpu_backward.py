@@ -1,8 +1,9 @@
 """GPU parity of the backward pass (kdn_backward) against the fp64 gradient oracle
 (oracle/kdn_grad.py): every gradient, element by element, for fp32 and bf16 inputs, ragged
 varlen batches with an empty sequence, initial states and final-state gradients, every d_k
-and the d_v extremes, and the full-size prefill workload (B4 H16 T4096 d128 bf16) on sampled
-(sequence, head) chains -- each chain's gradients depend on that chain's inputs only."""
+and the d_v extremes, both uncertainty variants, and the full-size prefill workload
+(B4 H16 T4096 d128 bf16) on sampled (sequence, head) chains -- each chain's gradients depend
+on that chain's inputs only."""
 import numpy as np
 import pytest
 
@@ -19,7 +20,7 @@ TOL = 1e-4
 NAMES = ("dq", "dk", "dv", "dalpha", "dsigma", "dr", "dS0", "dP0")
 
 
-def cotangents(seed, w, with_final=True):
+def cotangents(seed, w, with_final=True, iso=False):
     rng = np.random.default_rng(seed)
     d_o = rng.standard_normal((w.ntok, w.H, w.dv)).astype(np.float32)
     if w.bf16:
@@ -27,23 +28,23 @@ def cotangents(seed, w, with_final=True):
     dS = dP = None
     if with_final:
         dS = rng.standard_normal((w.num_seqs, w.H, w.dk, w.dv)).astype(np.float32)
-        dP = rng.standard_normal((w.num_seqs, w.H, w.dk)).astype(np.float32)
+        dP = rng.standard_normal((w.num_seqs, w.H) + (() if iso else (w.dk,))).astype(np.float32)
     return d_o, dS, dP
 
 
-def initial_state(seed, w):
+def initial_state(seed, w, iso=False):
     rng = np.random.default_rng(seed)
     S0 = (0.1 * rng.standard_normal((w.num_seqs, w.H, w.dk, w.dv))).astype(np.float32)
-    P0 = rng.uniform(0.3, 2.0, (w.num_seqs, w.H, w.dk)).astype(np.float32)
+    P0 = rng.uniform(0.3, 2.0, (w.num_seqs, w.H) + (() if iso else (w.dk,))).astype(np.float32)
     return S0, P0
 
 
-def run_backward(kdn, w, d_o, S0=None, P0=None, dS=None, dP=None, mu=1.0):
+def run_backward(kdn, w, d_o, S0=None, P0=None, dS=None, dP=None, mu=1.0, iso=False):
     import torch
     args = [to_dev(dense_shape(w, getattr(w, n))) for n in ("q", "k", "v", "alpha", "sigma", "r")]
     cu = to_dev(w.cu_seqlens) if w.B == 1 and w.num_seqs > 1 else None
     g = kdn.backward(*args, to_dev(dense_shape(w, d_o)), cu_seqlens=cu, S0=to_dev(S0), P0=to_dev(P0),
-                     dS=to_dev(dS), dP=to_dev(dP), mu=mu)
+                     dS=to_dev(dS), dP=to_dev(dP), mu=mu, variant="isotropic" if iso else "diagonal")
     torch.cuda.synchronize()
     kdn.last_device_error()
     out = {n: to_host(g[n]) for n in NAMES}
@@ -82,6 +83,20 @@ def test_backward_ragged_varlen(kdn, dk, dv, bf16):
     check(got, ref)
     # the empty sequence passes the final-state gradients straight through
     np.testing.assert_array_equal(got["dS0"][3], dS[3])
+    np.testing.assert_array_equal(got["dP0"][3], dP[3])
+
+
+@pytest.mark.parametrize("dk,dv,bf16", [(32, 32, False), (64, 256, True), (128, 128, True)])
+def test_backward_isotropic_ragged_varlen(kdn, dk, dv, bf16):
+    """The isotropic variant (one uncertainty per head): ragged sequences with an empty one,
+    S0/p0 and final-state gradients."""
+    w = ragged(500 + dk + dv, [1, 63, 64, 0, 65, 130], 2, dk, dv, bf16)
+    S0, P0 = initial_state(7, w, iso=True)
+    d_o, dS, dP = cotangents(8, w, iso=True)
+    ref = kdn_grad.diag_grad(w.q, w.k, w.v, w.alpha, w.sigma, w.r, d_o, cu_seqlens=w.cu_seqlens,
+                             S0=S0, P0=P0, dS=dS, dP=dP, mu=3.0, iso=True)
+    got = run_backward(kdn, w, d_o, S0, P0, dS, dP, mu=3.0, iso=True)
+    check(got, ref)
     np.testing.assert_array_equal(got["dP0"][3], dP[3])
 
 
