@@ -100,6 +100,32 @@ def test_backward_isotropic_ragged_varlen(kdn, dk, dv, bf16):
     np.testing.assert_array_equal(got["dP0"][3], dP[3])
 
 
+@pytest.mark.parametrize("regime", ["no_decay_noiseless_onehot", "strong_decay"])
+def test_backward_degenerate_regimes(kdn, regime):
+    """Edge regimes of the recurrence: (a) alpha = 1, sigma = 0, r = 1e-3 and one-hot keys on every
+    other token (the gain saturates, repeated confirmation drives P down); (b) alpha in [0.01, 0.1],
+    where the state before a token cannot be recovered by undoing the decay -- the state pass
+    re-steps it forward from checkpoints instead.  Many one-token sequences among longer ones."""
+    import dataclasses
+    w = ragged(600, [1, 1, 2, 33, 64, 97], 2, 32, 32, False)
+    rng = np.random.default_rng(11)
+    if regime == "no_decay_noiseless_onehot":
+        k = w.k.copy()
+        onehot = np.zeros_like(k[1::2])
+        idx = rng.integers(0, w.dk, size=onehot.shape[:2])
+        np.put_along_axis(onehot, idx[..., None], 1.0, axis=-1)
+        k[1::2] = onehot
+        w = dataclasses.replace(w, k=k.astype(np.float32), alpha=np.ones_like(w.alpha), sigma=np.zeros_like(w.sigma),
+                                r=np.full_like(w.r, 1e-3))
+    else:
+        w = dataclasses.replace(w, alpha=rng.uniform(0.01, 0.1, w.alpha.shape).astype(np.float32))
+    S0, P0 = initial_state(9, w)
+    d_o, dS, dP = cotangents(10, w)
+    ref = kdn_grad.diag_grad(w.q, w.k, w.v, w.alpha, w.sigma, w.r, d_o, cu_seqlens=w.cu_seqlens,
+                             S0=S0, P0=P0, dS=dS, dP=dP, mu=32.0)
+    check(run_backward(kdn, w, d_o, S0, P0, dS, dP, mu=32.0), ref)
+
+
 def test_backward_dense_defaults(kdn):
     """Dense batch, S0 = 0 and P0 = 1 by default, no final-state gradients."""
     w = inputs.dense("bwd_dense", 12, 2, 3, 150, 128, 128, bf16=True)
