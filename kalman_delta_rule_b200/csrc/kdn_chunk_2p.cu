@@ -131,6 +131,29 @@ __device__ __forceinline__ uint4 pack8(const float *v, float sc = 1.f) {
 
 __device__ __forceinline__ uint32_t ldg_u32(const bf16 *p) { return __ldg(reinterpret_cast<const unsigned *>(p)); }
 
+// Two fp32 lanes in one 64-bit register pair, for sm_100's packed f32x2 arithmetic: a thread of the
+// uncertainty passes carries the key channels ch and ch + 1 in lockstep (x = channel ch, y = ch + 1).
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 pk2(float x, float y) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+    return r;
+}
+__device__ __forceinline__ float x2(f32x2 r) { return __uint_as_float((unsigned)r); }
+__device__ __forceinline__ float y2(f32x2 r) { return __uint_as_float((unsigned)(r >> 32)); }
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+// a bf16 pair (low half = channel ch) widened to f32x2
+__device__ __forceinline__ f32x2 bf2(uint32_t w) { return pk2(tc::bf16_lo(w), tc::bf16_hi(w)); }
+
 // Look-back descriptors are 64-bit words (value, tag): each word carries its own status, so a
 // reader that sees a tag also sees that word's value, with no fence between writer and flag.
 enum : unsigned { TAG_NONE = 0, TAG_AGG = 1, TAG_INCL = 2 };
@@ -349,7 +372,22 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
             __syncthreads();
         }
         // ---- segment composites of the uncertainty maps (predict [[a, s],[0,1]], update [[1,0],[c,1]])
-        {
+        if constexpr (!ISO) {   // both channels of the pair at once (f32x2)
+            f32x2 m00 = pk2(1.f, 1.f), m01 = pk2(0.f, 0.f), m10 = m01, m11 = m00, gm = m00;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                if (tb + j < L) {
+                    const float mr = mur[tb + j];
+                    const f32x2 al = bf2(aw[j]), kk = bf2(kw[j]), sg = bf2(sw[j]);
+                    const f32x2 aa = mul2(al, al), cc = mul2(mul2(pk2(mr, mr), kk), kk);
+                    const f32x2 y00 = fma2(aa, m00, mul2(sg, m10)), y01 = fma2(aa, m01, mul2(sg, m11));
+                    m10 = fma2(cc, y00, m10); m11 = fma2(cc, y01, m11); m00 = y00; m01 = y01; gm = mul2(gm, al);
+                }
+            }
+            const float sa = 1.f / x2(m11), sbb = 1.f / y2(m11);
+            *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch) * 4) = make_float4(x2(m00) * sa, x2(m01) * sa, x2(m10) * sa, x2(gm));
+            *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch + 1) * 4) = make_float4(y2(m00) * sbb, y2(m01) * sbb, y2(m10) * sbb, y2(gm));
+        } else {
             float a00 = 1.f, a01 = 0.f, a10 = 0.f, a11 = 1.f, ga = 1.f;
             float b00 = 1.f, b01 = 0.f, b10 = 0.f, b11 = 1.f, gb = 1.f;
 #pragma unroll
@@ -483,22 +521,30 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
                 const int t = tb + j;
                 uint32_t kq = 0u, qq = 0u, gg = 0u;
                 xs[j] = 0.f;
-                if (t < L) {
+                if (!ISO && t < L) {   // both channels of the pair at once (f32x2)
+                    const f32x2 al = bf2(aw[j]), kk = bf2(kw[j]);
+                    const f32x2 pm = fma2(mul2(al, al), pk2(Pa, Pb), bf2(sw[j]));
+                    const float mr = mur[t];
+                    const f32x2 dn = fma2(mul2(mul2(pk2(mr, mr), kk), kk), pm, pk2(1.f, 1.f));
+                    Pa = __fdividef(x2(pm), x2(dn));
+                    Pb = __fdividef(y2(pm), y2(dn));
+                    gama *= x2(al);
+                    gamb *= y2(al);
+                    const f32x2 gm = pk2(gama, gamb), pk = mul2(pm, kk), kg = mul2(kk, gm), qg = mul2(bf2(qw[j]), gm);
+                    kq = pack_bf16x2(x2(kg), y2(kg));
+                    qq = pack_bf16x2(x2(qg), y2(qg));
+                    gg = pack_bf16x2(__fdividef(x2(pk), gama), __fdividef(y2(pk), gamb));
+                    xs[j] = fmaf(x2(pk), x2(kk), y2(pk) * y2(kk));
+                } else if (ISO && t < L) {
                     const float ala = bf16_lo(aw[j]), alb = bf16_hi(aw[j]);
                     const float ka = bf16_lo(kw[j]), kb = bf16_hi(kw[j]);
                     float pma, pmb;
-                    if constexpr (ISO) {   // the head's map, the same on every channel
+                    {   // the head's map, the same on every channel
                         const float4 iso = *reinterpret_cast<const float4 *>(tsum + t * 4);
                         pma = fmaf(iso.x, Pa, iso.y);
                         pmb = fmaf(iso.x, Pb, iso.y);
                         Pa = __fdividef(pma, fmaf(iso.z, pma, 1.f));
                         Pb = __fdividef(pmb, fmaf(iso.z, pmb, 1.f));
-                    } else {
-                        pma = fmaf(ala * ala, Pa, bf16_lo(sw[j]));
-                        pmb = fmaf(alb * alb, Pb, bf16_hi(sw[j]));
-                        const float mr = mur[t];
-                        Pa = __fdividef(pma, fmaf(mr * ka * ka, pma, 1.f));
-                        Pb = __fdividef(pmb, fmaf(mr * kb * kb, pmb, 1.f));
                     }
                     gama *= ala;
                     gamb *= alb;
