@@ -68,14 +68,6 @@ __device__ __forceinline__ void stage_rows(void *dst, const void *src, size_t st
     }
 }
 __device__ __forceinline__ float lds(const float *p) { return *p; }
-// 16 consecutive floats of shared memory (16-byte aligned) into registers
-__device__ __forceinline__ void lds16(const float *p, float (&x)[16]) {
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-        const float4 f = reinterpret_cast<const float4 *>(p)[q4];
-        x[4 * q4] = f.x; x[4 * q4 + 1] = f.y; x[4 * q4 + 2] = f.z; x[4 * q4 + 3] = f.w;
-    }
-}
 __device__ __forceinline__ float lds(const bf16 *p) {
     return __uint_as_float(((unsigned)*reinterpret_cast<const unsigned short *>(p)) << 16);
 }
@@ -219,13 +211,27 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
         cp_async_wait_all();
         __syncthreads();
     };
+    // 16 consecutive shared floats (16-byte aligned) as 8 column pairs
+    auto lds8x2 = [&](const float *p, f32x2 (&x)[8]) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const ulonglong2 v = reinterpret_cast<const ulonglong2 *>(p)[q];
+            x[2 * q] = v.x;
+            x[2 * q + 1] = v.y;
+        }
+    };
     // u_j = v_j - sum_i alpha_i k_i S_ij for staged token tt of the chunk at c0 -> the u tape and
     // dst[DB] (shared), then into u
-    auto forward_u = [&](int c0, int tt, const float (&S)[16], float *dst, float (&u)[16]) {
+    auto forward_u = [&](int c0, int tt, const f32x2 (&S)[8], float *dst, f32x2 (&u)[8]) {
         const float ak = lds(al_s + tt * dk + i) * lds(k_s + tt * dk + i);
+        const f32x2 ak2 = pk2(ak, ak);
         float p[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) p[j] = ak * S[j];
+        for (int jp = 0; jp < 8; ++jp) {
+            const f32x2 x = mul2(ak2, S[jp]);
+            p[2 * jp] = x2(x);
+            p[2 * jp + 1] = y2(x);
+        }
         int which;
         const float tot = reduce16(p, lane, which);
         if ((lane & 1) == 0) red[warp * DB + which] = tot;
@@ -237,17 +243,21 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
             w.utape[((size_t)(c0 + tt) * H + h) * dv + col0 + i] = dst[i];
         }
         __syncthreads();
-        lds16(dst, u);
+        lds8x2(dst, u);
     };
-    auto step = [&](int tt, float (&S)[16], const float (&u)[16]) {
+    auto step = [&](int tt, f32x2 (&S)[8], const f32x2 (&u)[8]) {
         const float al = lds(al_s + tt * dk + i), gg = g_s[tt * dk + i];
+        const f32x2 al2 = pk2(al, al), gg2 = pk2(gg, gg);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) S[j] = fmaf(gg, u[j], al * S[j]);
+        for (int jp = 0; jp < 8; ++jp) S[jp] = fma2(gg2, u[jp], mul2(al2, S[jp]));
     };
 
-    float S[16], Sh[16], u[16];
+    f32x2 S[8], Sh[8], u[8];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) S[j] = a.S0 ? a.S0[((size_t)chain * dk + i) * dv + col0 + j] : 0.f;
+    for (int jp = 0; jp < 8; ++jp) {
+        const size_t e = ((size_t)chain * dk + i) * dv + col0 + 2 * jp;
+        S[jp] = a.S0 ? pk2(a.S0[e], a.S0[e + 1]) : pk2(0.f, 0.f);
+    }
 
     // ---- forward: checkpoints every CK tokens
     const int nchk = (t1 - t0 + CK - 1) / CK;
@@ -255,7 +265,10 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
         const int c0 = t0 + m * CK, L = min(CK, t1 - c0);
         float *ck = ckpt_at(m);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) ck[j * dk + i] = S[j];
+        for (int jp = 0; jp < 8; ++jp) {
+            ck[(2 * jp) * dk + i] = x2(S[jp]);
+            ck[(2 * jp + 1) * dk + i] = y2(S[jp]);
+        }
         stage(c0, L, false);
         for (int tt = 0; tt < L; ++tt) {
             forward_u(c0, tt, S, uh, u);
@@ -265,52 +278,59 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
 
     // ---- reverse, chunk by chunk
 #pragma unroll
-    for (int j = 0; j < 16; ++j) Sh[j] = b.dS_T ? b.dS_T[((size_t)chain * dk + i) * dv + col0 + j] : 0.f;
+    for (int jp = 0; jp < 8; ++jp) {
+        const size_t e = ((size_t)chain * dk + i) * dv + col0 + 2 * jp;
+        Sh[jp] = b.dS_T ? pk2(b.dS_T[e], b.dS_T[e + 1]) : pk2(0.f, 0.f);
+    }
     for (int m = nchk - 1; m >= 0; --m) {
         const int c0 = t0 + m * CK, L = min(CK, t1 - c0);
         const float *ck = ckpt_at(m);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) S[j] = ck[j * dk + i];
+        for (int jp = 0; jp < 8; ++jp) S[jp] = pk2(ck[(2 * jp) * dk + i], ck[(2 * jp + 1) * dk + i]);
         stage(c0, L, true);
         for (int tt = 0; tt < L; ++tt) {
             if (tt % NS == 0) {
-                float4 *sb = reinterpret_cast<float4 *>(sub) + (size_t)(tt / NS) * 4 * dk + i;
+                ulonglong2 *sb = reinterpret_cast<ulonglong2 *>(sub) + (size_t)(tt / NS) * 4 * dk + i;
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    sb[q4 * dk] = make_float4(S[4 * q4], S[4 * q4 + 1], S[4 * q4 + 2], S[4 * q4 + 3]);
+                for (int q = 0; q < 4; ++q) sb[q * dk] = make_ulonglong2(S[2 * q], S[2 * q + 1]);
             }
-            lds16(us + tt * DB, u);
+            lds8x2(us + tt * DB, u);
             step(tt, S, u);
         }
         for (int js = (L - 1) / NS; js >= 0; --js) {
             for (int tt = min(L, js * NS + NS) - 1; tt >= js * NS; --tt) {
                 const int t = c0 + tt;
                 // state before token t, re-stepped from the sub-checkpoint
-                float Sp[16], uu[16];
+                f32x2 Sp[8], uu[8];
                 {
-                    const float4 *sb = reinterpret_cast<const float4 *>(sub) + (size_t)js * 4 * dk + i;
+                    const ulonglong2 *sb = reinterpret_cast<const ulonglong2 *>(sub) + (size_t)js * 4 * dk + i;
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const float4 f = sb[q4 * dk];
-                        Sp[4 * q4] = f.x; Sp[4 * q4 + 1] = f.y; Sp[4 * q4 + 2] = f.z; Sp[4 * q4 + 3] = f.w;
+                    for (int q = 0; q < 4; ++q) {
+                        const ulonglong2 v = sb[q * dk];
+                        Sp[2 * q] = v.x;
+                        Sp[2 * q + 1] = v.y;
                     }
                 }
                 for (int oo = js * NS; oo < tt; ++oo) {
-                    lds16(us + oo * DB, uu);
+                    lds8x2(us + oo * DB, uu);
                     step(oo, Sp, uu);
                 }
                 const float al = lds(al_s + tt * dk + i), kk = lds(k_s + tt * dk + i), gg = g_s[tt * dk + i];
                 const float qq = lds(q_s + tt * dk + i);
-                float dqp = 0.f, gp = 0.f, p[16];
-                lds16(us + tt * DB, uu);
+                const f32x2 al2 = pk2(al, al), gg2 = pk2(gg, gg), qq2 = pk2(qq, qq), nk2 = pk2(-kk, -kk);
+                f32x2 dq2 = pk2(0.f, 0.f), gp2 = dq2;
+                float p[16];
+                lds8x2(us + tt * DB, uu);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float uj = uu[j], doj = lds(do_s + tt * DB + j);
-                    const float St = fmaf(gg, uj, al * Sp[j]);
-                    Sh[j] = fmaf(qq, doj, Sh[j]);
-                    dqp = fmaf(St, doj, dqp);
-                    gp = fmaf(Sh[j], uj, gp);
-                    p[j] = Sh[j] * gg;
+                for (int jp = 0; jp < 8; ++jp) {
+                    const f32x2 do2 = pk2(lds(do_s + tt * DB + 2 * jp), lds(do_s + tt * DB + 2 * jp + 1));
+                    const f32x2 St = fma2(gg2, uu[jp], mul2(al2, Sp[jp]));
+                    Sh[jp] = fma2(qq2, do2, Sh[jp]);
+                    dq2 = fma2(St, do2, dq2);
+                    gp2 = fma2(Sh[jp], uu[jp], gp2);
+                    const f32x2 x = mul2(Sh[jp], gg2);
+                    p[2 * jp] = x2(x);
+                    p[2 * jp + 1] = y2(x);
                 }
                 int which;
                 const float tot = reduce16(p, lane, which);
@@ -323,27 +343,30 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
                     b.dv[((size_t)t * H + h) * dv + col0 + i] = x;
                 }
                 __syncthreads();
-                float kp = 0.f, ap = 0.f;
-                lds16(uh, uu);
+                f32x2 kp2 = pk2(0.f, 0.f), ap2 = kp2;
+                lds8x2(uh, uu);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float uhj = uu[j];
-                    const float Wh = fmaf(-kk, uhj, Sh[j]);
-                    kp = fmaf(al * Sp[j], uhj, kp);
-                    ap = fmaf(Wh, Sp[j], ap);
-                    Sh[j] = al * Wh;
+                for (int jp = 0; jp < 8; ++jp) {
+                    const f32x2 Wh = fma2(nk2, uu[jp], Sh[jp]);
+                    kp2 = fma2(mul2(al2, Sp[jp]), uu[jp], kp2);
+                    ap2 = fma2(Wh, Sp[jp], ap2);
+                    Sh[jp] = mul2(al2, Wh);
                 }
                 float *pp = w.part + (size_t)blk * 4 * tokstride + ((size_t)t * H + h) * dk + i;
-                pp[0] = dqp;
-                pp[tokstride] = gp;
-                pp[2 * tokstride] = -kp;
-                pp[3 * tokstride] = ap;
+                pp[0] = x2(dq2) + y2(dq2);
+                pp[tokstride] = x2(gp2) + y2(gp2);
+                pp[2 * tokstride] = -(x2(kp2) + y2(kp2));
+                pp[3 * tokstride] = x2(ap2) + y2(ap2);
             }
         }
     }
     if (b.dS0) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) b.dS0[((size_t)chain * dk + i) * dv + col0 + j] = Sh[j];
+        for (int jp = 0; jp < 8; ++jp) {
+            const size_t e = ((size_t)chain * dk + i) * dv + col0 + 2 * jp;
+            b.dS0[e] = x2(Sh[jp]);
+            b.dS0[e + 1] = y2(Sh[jp]);
+        }
     }
 }
 

@@ -131,26 +131,6 @@ __device__ __forceinline__ uint4 pack8(const float *v, float sc = 1.f) {
 
 __device__ __forceinline__ uint32_t ldg_u32(const bf16 *p) { return __ldg(reinterpret_cast<const unsigned *>(p)); }
 
-// Two fp32 lanes in one 64-bit register pair, for sm_100's packed f32x2 arithmetic: a thread of the
-// uncertainty passes carries the key channels ch and ch + 1 in lockstep (x = channel ch, y = ch + 1).
-typedef unsigned long long f32x2;
-__device__ __forceinline__ f32x2 pk2(float x, float y) {
-    f32x2 r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
-    return r;
-}
-__device__ __forceinline__ float x2(f32x2 r) { return __uint_as_float((unsigned)r); }
-__device__ __forceinline__ float y2(f32x2 r) { return __uint_as_float((unsigned)(r >> 32)); }
-__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
-    f32x2 d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
-    f32x2 d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
 // a bf16 pair (low half = channel ch) widened to f32x2
 __device__ __forceinline__ f32x2 bf2(uint32_t w) { return pk2(tc::bf16_lo(w), tc::bf16_hi(w)); }
 

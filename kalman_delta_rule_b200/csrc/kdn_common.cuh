@@ -45,6 +45,27 @@ __device__ __forceinline__ void stf4(bf16 *p, float4 v) {
 __device__ __forceinline__ void stf(float *p, float v) { *p = v; }
 __device__ __forceinline__ void stf(bf16 *p, float v) { *p = __float2bfloat16_rn(v); }
 
+// Two fp32 lanes in one 64-bit register pair, for sm_100's packed f32x2 arithmetic (x = the low
+// lane, y = the high one); mul2 / fma2 round each lane as the scalar instruction would.
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 pk2(float x, float y) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(x), "f"(y));
+    return r;
+}
+__device__ __forceinline__ float x2(f32x2 r) { return __uint_as_float((unsigned)r); }
+__device__ __forceinline__ float y2(f32x2 r) { return __uint_as_float((unsigned)(r >> 32)); }
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
