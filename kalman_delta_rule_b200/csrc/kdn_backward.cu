@@ -22,11 +22,12 @@
 //         chunk is re-stepped from its checkpoint (with the taped u, so without the cross-row
 //         reduction) into shared-memory sub-checkpoints every 4 tokens, and the
 //         state before each token is re-stepped from the nearest sub-checkpoint (never
-//         reconstructed by dividing by alpha, which loses it when alpha is small).  Writes dv and,
-//         per column block, partial sums over its columns of dq, g^, the S-part of k^ and the
-//         S-part of alpha^;
-//   local (one warp per (token, head), every token in parallel): sums the partials, writes dq and
-//         den^, and the parts of P^-^ and k^ that do not depend on the later tokens' P^;
+//         reconstructed by dividing by alpha, which loses it when alpha is small).  Writes dv and
+//         adds its column block's share of dq, g^, the S-part of k^ and the S-part of alpha^ into
+//         them with fire-and-forget atomic adds (dq into the output, the others into three token
+//         vectors that the tape kernel zeroed);
+//   local (one warp per (token, head), every token in parallel): writes den^ and the parts of P^-^
+//         and k^ that do not depend on the later tokens' P^;
 //   prev  (one CTA per (sequence, head), thread = key channel): the one serial part of the
 //         uncertainty adjoint, P^ <- alpha^2 (P^-^local + P^ z^2), and the outputs that need P^:
 //         dk, dalpha, dsigma, dr and dP0.
@@ -121,7 +122,7 @@ __global__ void __launch_bounds__(128) bwd_tape_kernel(const BwdArgs b, const Bw
     const T *k = static_cast<const T *>(a.k), *r = static_cast<const T *>(a.r);
     const int chain = blockIdx.x, s = chain / H, h = chain % H;
     const int i = threadIdx.x, warp = i >> 5, lane = i & 31, nw = dk >> 5;
-    const size_t rstride = (size_t)H * dk * sizeof(T);
+    const size_t rstride = (size_t)H * dk * sizeof(T), tokstride = (size_t)w.ntok * H * dk;
     const int rbytes = dk * (int)sizeof(T);
     int t0, t1;
     seq_range(a, s, t0, t1);
@@ -158,8 +159,14 @@ __global__ void __launch_bounds__(128) bwd_tape_kernel(const BwdArgs b, const Bw
             }
         }
         __syncthreads();
-        for (int tt = 0; tt < n; ++tt)
-            w.g[((size_t)(tb + tt) * H + h) * dk + i] = pm_s[tt * dk + i] * lds(k_s + tt * dk + i) / den_s[tt];
+        for (int tt = 0; tt < n; ++tt) {
+            const size_t e = ((size_t)(tb + tt) * H + h) * dk + i;
+            w.g[e] = pm_s[tt * dk + i] * lds(k_s + tt * dk + i) / den_s[tt];
+            b.dq[e] = 0.f;   // the state pass adds its column blocks' shares into these
+            w.part[e] = 0.f;
+            w.part[tokstride + e] = 0.f;
+            w.part[2 * tokstride + e] = 0.f;
+        }
         __syncthreads();
     }
 }
@@ -352,11 +359,11 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
                     ap2 = fma2(Wh, Sp[jp], ap2);
                     Sh[jp] = mul2(al2, Wh);
                 }
-                float *pp = w.part + (size_t)blk * 4 * tokstride + ((size_t)t * H + h) * dk + i;
-                pp[0] = x2(dq2) + y2(dq2);
-                pp[tokstride] = x2(gp2) + y2(gp2);
-                pp[2 * tokstride] = -(x2(kp2) + y2(kp2));
-                pp[3 * tokstride] = x2(ap2) + y2(ap2);
+                const size_t e = ((size_t)t * H + h) * dk + i;
+                atomicAdd(b.dq + e, x2(dq2) + y2(dq2));
+                atomicAdd(w.part + e, x2(gp2) + y2(gp2));
+                atomicAdd(w.part + tokstride + e, -(x2(kp2) + y2(kp2)));
+                atomicAdd(w.part + 2 * tokstride + e, x2(ap2) + y2(ap2));
             }
         }
     }
@@ -371,12 +378,11 @@ __global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, cons
 }
 
 // ================================================================= local
-// One warp per (token, head), lanes over the key channels.  Sums the NB column-block partials;
-// writes dq and den^ = -(g^ . g) / den, and overwrites block 0's partial slots 1..3 with
+// One warp per (token, head), lanes over the key channels.  Writes den^ = -(g^ . g) / den and
+// overwrites the sums of g^ and k^_S with
 //   A  = g^ k / den + den^ k^2                      (P^-^ without the later tokens' part)
 //   Kl = k^_S + g^ P^- / den + 2 den^ P^- k         (k^ without the uncertainty-update part)
-//   alpha^_S                                        (summed)
-template <typename T, int NB>
+template <typename T>
 __global__ void __launch_bounds__(256) bwd_local_kernel(const BwdArgs b, const BwdWs w)
 {
     const TokenArgs &a = b.a;
@@ -388,27 +394,16 @@ __global__ void __launch_bounds__(256) bwd_local_kernel(const BwdArgs b, const B
     const T *k = static_cast<const T *>(a.k);
     const size_t tokstride = (size_t)w.ntok * H * dk;
     const float dn = w.den[th];
-    float gh[4], kS[4], aS[4], xg = 0.f;
+    float gh[4], kS[4], xg = 0.f;
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
         const int c = lane + 32 * m;
-        gh[m] = kS[m] = aS[m] = 0.f;
+        gh[m] = kS[m] = 0.f;
         if (c < dk) {
             const size_t e = (size_t)th * dk + c;
-            float p4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int bb = 0; bb < NB; ++bb) {
-                const float *pp = w.part + (size_t)bb * 4 * tokstride + e;
-                p4[0] += pp[0];
-                p4[1] += pp[tokstride];
-                p4[2] += pp[2 * tokstride];
-                p4[3] += pp[3 * tokstride];
-            }
-            b.dq[e] = p4[0];
-            gh[m] = p4[1];
-            kS[m] = p4[2];
-            aS[m] = p4[3];
-            xg = fmaf(p4[1], w.g[e], xg);
+            gh[m] = w.part[e];
+            kS[m] = w.part[tokstride + e];
+            xg = fmaf(gh[m], w.g[e], xg);
         }
     }
     const float dd = -warp_sum(xg) / dn;
@@ -420,10 +415,8 @@ __global__ void __launch_bounds__(256) bwd_local_kernel(const BwdArgs b, const B
             const size_t e = (size_t)th * dk + c;
             const float al = ldf(alpha + e), kk = ldf(k + e);
             const float pm = fmaf(al * al, w.Pprev[e], ldf(sigma + e));
-            float *pp = w.part + e;
-            pp[tokstride] = gh[m] * kk / dn + dd * kk * kk;
-            pp[2 * tokstride] = kS[m] + gh[m] * pm / dn + 2.f * dd * pm * kk;
-            pp[3 * tokstride] = aS[m];
+            w.part[e] = gh[m] * kk / dn + dd * kk * kk;
+            w.part[tokstride + e] = kS[m] + gh[m] * pm / dn + 2.f * dd * pm * kk;
         }
     }
 }
@@ -453,9 +446,9 @@ __global__ void __launch_bounds__(128) bwd_prev_kernel(const BwdArgs b, const Bw
     for (int te = t1; te > t0; te -= GT) {
         const int tb = max(t0, te - GT), n = te - tb;
         const size_t row0 = ((size_t)tb * H + h) * dk;
-        stage_rows(A_s, w.part + tokstride + row0, fstride, n, dk * 4);
-        stage_rows(K_s, w.part + 2 * tokstride + row0, fstride, n, dk * 4);
-        stage_rows(aS_s, w.part + 3 * tokstride + row0, fstride, n, dk * 4);
+        stage_rows(A_s, w.part + row0, fstride, n, dk * 4);
+        stage_rows(K_s, w.part + tokstride + row0, fstride, n, dk * 4);
+        stage_rows(aS_s, w.part + 2 * tokstride + row0, fstride, n, dk * 4);
         stage_rows(pp_s, w.Pprev + row0, fstride, n, dk * 4);
         stage_rows(al_s, alpha + row0, rstride, n, dk * (int)sizeof(T));
         stage_rows(sg_s, sigma + row0, rstride, n, dk * (int)sizeof(T));
@@ -522,7 +515,7 @@ __global__ void __launch_bounds__(128) bwd_tape_iso_kernel(const BwdArgs b, cons
     const T *k = static_cast<const T *>(a.k), *r = static_cast<const T *>(a.r);
     const int chain = blockIdx.x, s = chain / H, h = chain % H;
     const int i = threadIdx.x, warp = i >> 5, lane = i & 31, nw = dk >> 5;
-    const size_t rstride = (size_t)H * dk * sizeof(T);
+    const size_t rstride = (size_t)H * dk * sizeof(T), tokstride = (size_t)w.ntok * H * dk;
     const int rbytes = dk * (int)sizeof(T);
     const float inv_dk = 1.f / dk;
     int t0, t1;
@@ -568,15 +561,20 @@ __global__ void __launch_bounds__(128) bwd_tape_iso_kernel(const BwdArgs b, cons
             }
         }
         __syncthreads();
-        for (int tt = 0; tt < n; ++tt)
-            w.g[((size_t)(tb + tt) * H + h) * dk + i] = pm_s[tt] * lds(k_s + tt * dk + i) / den_s[tt];
+        for (int tt = 0; tt < n; ++tt) {
+            const size_t e = ((size_t)(tb + tt) * H + h) * dk + i;
+            w.g[e] = pm_s[tt] * lds(k_s + tt * dk + i) / den_s[tt];
+            b.dq[e] = 0.f;   // the state pass adds its column blocks' shares into these
+            w.part[e] = 0.f;
+            w.part[tokstride + e] = 0.f;
+            w.part[2 * tokstride + e] = 0.f;
+        }
         __syncthreads();
     }
 }
 
-// one warp per (token, head): sums the column-block partials, writes dq, and the local parts
-// of k^ (block 0's slot 2), alpha^_S (slot 3), p^-^ and r^ (tape scalars)
-template <typename T, int NB>
+// one warp per (token, head): the local parts of k^ (over the k^_S sum), p^-^ and r^ (tape scalars)
+template <typename T>
 __global__ void __launch_bounds__(256) bwd_local_iso_kernel(const BwdArgs b, const BwdWs w)
 {
     const TokenArgs &a = b.a;
@@ -588,29 +586,18 @@ __global__ void __launch_bounds__(256) bwd_local_iso_kernel(const BwdArgs b, con
     const size_t tokstride = (size_t)w.ntok * H * dk;
     float *sc = w.Pprev + (size_t)th * dk;
     const float dn = w.den[th], pm = sc[SC_PM], K2 = sc[SC_K2];
-    float gh[4], kS[4], aS[4], kk[4], gk = 0.f, gg = 0.f;
+    float gh[4], kS[4], kk[4], gk = 0.f, gg = 0.f;
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
         const int c = lane + 32 * m;
-        gh[m] = kS[m] = aS[m] = kk[m] = 0.f;
+        gh[m] = kS[m] = kk[m] = 0.f;
         if (c < dk) {
             const size_t e = (size_t)th * dk + c;
-            float p4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int bb = 0; bb < NB; ++bb) {
-                const float *pp = w.part + (size_t)bb * 4 * tokstride + e;
-                p4[0] += pp[0];
-                p4[1] += pp[tokstride];
-                p4[2] += pp[2 * tokstride];
-                p4[3] += pp[3 * tokstride];
-            }
-            b.dq[e] = p4[0];
-            gh[m] = p4[1];
-            kS[m] = p4[2];
-            aS[m] = p4[3];
+            gh[m] = w.part[e];
+            kS[m] = w.part[tokstride + e];
             kk[m] = ldf(k + e);
-            gk = fmaf(p4[1], kk[m], gk);
-            gg = fmaf(p4[1], w.g[e], gg);
+            gk = fmaf(gh[m], kk[m], gk);
+            gg = fmaf(gh[m], w.g[e], gg);
         }
     }
     gk = warp_sum(gk);
@@ -623,9 +610,7 @@ __global__ void __launch_bounds__(256) bwd_local_iso_kernel(const BwdArgs b, con
     for (int m = 0; m < 4; ++m) {
         const int c = lane + 32 * m;
         if (c < dk) {
-            float *pp = w.part + (size_t)th * dk + c;
-            pp[2 * tokstride] = kS[m] + gh[m] * pm / dn - 2.f * gg * pm * kk[m] / dn;
-            pp[3 * tokstride] = aS[m];
+            w.part[tokstride + (size_t)th * dk + c] = kS[m] + gh[m] * pm / dn - 2.f * gg * pm * kk[m] / dn;
         }
     }
 }
@@ -653,8 +638,8 @@ __global__ void __launch_bounds__(128) bwd_prev_iso_kernel(const BwdArgs b, cons
     for (int te = t1; te > t0; te -= GT) {
         const int tb = max(t0, te - GT), n = te - tb;
         const size_t row0 = ((size_t)tb * H + h) * dk;
-        stage_rows(K_s, w.part + 2 * tokstride + row0, fstride, n, dk * 4);
-        stage_rows(aS_s, w.part + 3 * tokstride + row0, fstride, n, dk * 4);
+        stage_rows(K_s, w.part + tokstride + row0, fstride, n, dk * 4);
+        stage_rows(aS_s, w.part + 2 * tokstride + row0, fstride, n, dk * 4);
         stage_rows(sc_s, w.Pprev + row0, fstride, n, 32);
         stage_rows(al_s, alpha + row0, rstride, n, dk * (int)sizeof(T));
         stage_rows(k_s, k + row0, rstride, n, dk * (int)sizeof(T));
@@ -697,18 +682,18 @@ size_t backward_workspace_bytes(long long ntok, int nseq, int H, int dk, int dv)
     n += align256(th * 4);                                          // den^
     n += align256(th * dv * 4);                                     // u of every token
     n += align256((size_t)ckpt_slots(ntok, nseq) * H * dk * dv * 4);   // S checkpoints
-    n += align256((size_t)4 * (dv / DB) * th * dk * 4);             // per-column-block partials
+    n += align256((size_t)3 * th * dk * 4);                         // sums of g^, k^_S, alpha^_S
     return n;
 }
 
-template <typename T, int NB>
+template <typename T>
 static cudaError_t launch_local(const BwdArgs &b, const BwdWs &w, cudaStream_t st) {
     const long long rows = w.ntok * b.a.H;
     if (rows == 0) return cudaSuccess;
     if (b.a.iso)
-        bwd_local_iso_kernel<T, NB><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(b, w);
+        bwd_local_iso_kernel<T><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(b, w);
     else
-        bwd_local_kernel<T, NB><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(b, w);
+        bwd_local_kernel<T><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(b, w);
     return cudaGetLastError();
 }
 
@@ -736,8 +721,7 @@ static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, cudaStream
     bwd_state_kernel<T><<<(unsigned)chains * w.nblk, dk, ssm, st>>>(b, w);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    e = w.nblk == 2 ? launch_local<T, 2>(b, w, st) : w.nblk == 4 ? launch_local<T, 4>(b, w, st)
-      : w.nblk == 8 ? launch_local<T, 8>(b, w, st) : launch_local<T, 16>(b, w, st);
+    e = launch_local<T>(b, w, st);
     if (e != cudaSuccess) return e;
     if (b.a.iso) {
         const size_t psm = ((size_t)2 * GT * dk + 9 * GT) * sizeof(float) + (size_t)2 * GT * dk * sizeof(T);
