@@ -38,3 +38,13 @@ def test_reference_arm_other_ranks_exit_quietly():
     p = run_ref({"RANK": "1", "WORLD_SIZE": "2"})
     assert p.returncode == 0, p.stderr[-2000:]
     assert p.stdout.strip() == ""
+
+
+def test_prefill_roofline_numerator_matches_the_documented_bytes():
+    """The prefill roofline's algorithmic bytes: per token and head q, k, alpha, sigma (4 x 256 B),
+    v and o (2 x 256 B) and r (2 B), plus the final S and P of every (sequence, head), for
+    B4 H16 T4096 d128 bf16: 262144 x 1538 + 64 x (128 x 128 + 128) x 4 = 407,404,544 bytes."""
+    sys.path.insert(0, ROOT)
+    import bench
+    w = bench.workload("prefill")
+    assert bench.algorithmic_bytes(w) == 262144 * 1538 + 64 * (128 * 128 + 128) * 4 == 407404544
