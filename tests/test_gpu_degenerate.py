@@ -8,7 +8,7 @@ path's documented range limit.
   64-token chunk.  The token-serial and fp32 chunk paths (pairwise decay factors) still match the
   oracle; the tensor-core paths, which factor the decay through the chunk start, report
   KDN_ERR_RANGE through kdn_last_device_error (and the error word is cleared afterwards).
-Sequences of 1, 1, 2, 33, 64 and 130 tokens."""
+The gain scan is checked in both regimes as well.  Sequences of 1, 1, 2, 33, 64 and 130 tokens."""
 import dataclasses
 
 import numpy as np
@@ -100,3 +100,18 @@ def test_strong_decay_tensor_core_paths_report_range(kdn, path):
     ok = regime("no_decay_noiseless_onehot", dk, 64, bf16)
     forward(kdn, ok, chunk, ws)
     kdn.last_device_error()
+
+
+@pytest.mark.parametrize("name", ["no_decay_noiseless_onehot", "strong_decay"])
+@pytest.mark.parametrize("bf16,dk", [(False, 32), (True, 128)])
+def test_gain_scan_edge_regimes(kdn, name, bf16, dk):
+    """The Moebius gain scan (generic kernel for fp32, the TMA kernel for bf16 d_k = 128) in both
+    edge regimes: the gain, k^T g and the final uncertainty against the oracle's traces.  The scan
+    composes 2x2 maps and never factors the decay, so strong decay is in range."""
+    from tests.test_gpu_scan import TOL, run_scan
+    w = regime(name, dk, 64, bf16)
+    ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens, mu=4.0, trace=True)
+    g, be, P = run_scan(kdn, w, mu=4.0, max_seqlen=max(LENS))
+    assert max_rel_err(g, ref["trace_g"]) <= TOL[bf16]
+    assert max_rel_err(be, ref["trace_beta_eff"]) <= TOL[bf16]
+    assert max_rel_err(P, ref["P"]) <= TOL[bf16]
