@@ -9,9 +9,10 @@ workload (B=4, H=16, T=4096, d_k=d_v=128, bf16 inputs, fp32 state, chunk 64); a 
 is one forward over the whole batch (uncertainty/gain, chunk algebra, state carry and
 readout -- every step of the hot path), timed with CUDA events on the launching stream.
 The JSON line also carries the decode rate (steps/s on 256 sequences x 32 heads,
-d = 128, fp32 state, 1024 steps), each with its roofline fraction against the measured
-HBM copy bandwidth, the end-to-end rate through the C ABI with host buffers, and the
-fp64 oracle timed on the host cores.
+d = 128, fp32 state, 1024 steps), the long-context (B=1, H=32, T=65536, key pool) and
+packed-varlen (262144 tokens, d_v = 256) prefill rates, the gain scan and the backward,
+each with its roofline fraction against the measured HBM copy bandwidth, the end-to-end
+rate through the C ABI with host buffers, and the fp64 oracle timed on the host cores.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own independent batch
 (weak scaling, no data-path collective); timings are the max over ranks.
@@ -226,27 +227,6 @@ def bench_prefill(args, world, rank, dev, kdn):
     value, total_ms = whole_job_rate(tokens, args.steps, evs[0].elapsed_time(evs[-1]), world)
     ms_step = total_ms / args.steps
 
-    # the same forward without a workspace (the one-kernel tensor-core path), for comparison
-    single = None
-    if path == "chunk_tcgen05_two_phase":
-        def step_single():
-            kdn.forward(d["q"], d["k"], d["v"], d["alpha"], d["sigma"], d["r"], cu_seqlens=cu, mu=w.mu,
-                        chunk=w.chunk, o=o, S_out=S_out, P_out=P_out, workspace=False, max_seqlen=max_seqlen)
-        for _ in range(2):
-            step_single()
-        barrier(world)
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_single = max(3, min(args.steps, 5))
-        f0.record(stream)
-        for _ in range(n_single):
-            step_single()
-        f1.record(stream)
-        torch.cuda.synchronize()
-        barrier(world)
-        kdn.last_device_error()
-        s_value, s_ms = whole_job_rate(w.ntok, n_single, f0.elapsed_time(f1), world)
-        single = dict(value=s_value, ms_per_step=s_ms / n_single, path="chunk_tcgen05", gpu_launches=n_single)
-
     # the isotropic variant (one uncertainty per head) on the same inputs and path
     iso = None
     if path.startswith("chunk_tcgen05"):
@@ -408,26 +388,62 @@ def bench_prefill(args, world, rank, dev, kdn):
 
     nbytes = algorithmic_bytes(w)
     return dict(w=w, value=value, ms_step=ms_step, per_step_ms=per_step_ms, clocks=clk.summary(), path=path, scan=scan,
-                single=single, iso=iso, bwd=bwd,
+                iso=iso, bwd=bwd,
                 e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                          steps=e_steps),
                 bytes=nbytes, launches=args.steps * launches_per_step)
 
 
+def bench_prefill_other(args, world, rank, dev, kdn, name, steps=5):
+    """Another prefill workload (long context, packed varlen) timed like the headline one: inputs
+    resident in HBM, CUDA events around `steps` forwards after the warm-up."""
+    import torch
+    w = workload(name, seed_offset=rank)
+    B = w.B if w.B else 1
+    names = ("q", "k", "v", "alpha", "sigma", "r")
+    d = {n: to_dev(getattr(w, n).reshape((B, w.ntok // B) + getattr(w, n).shape[1:]), dev) for n in names}
+    cu = to_dev(w.cu_seqlens, dev) if (w.B == 1 and w.num_seqs > 1) else None
+    o = torch.empty(d["q"].shape[:3] + (w.dv,), dtype=d["q"].dtype, device=dev)
+    S_out = torch.empty((w.num_seqs, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+    P_out = torch.empty((w.num_seqs, w.H, w.dk), dtype=torch.float32, device=dev)
+    max_seqlen = int(np.diff(w.cu_seqlens).max()) if cu is not None else 0
+    prob = kdn.make_problem(d["q"], d["v"], cu_seqlens=cu, mu=w.mu, chunk=w.chunk, max_seqlen=max_seqlen)
+    ws = torch.empty(max(kdn.kdn_workspace_size(prob), 1), dtype=torch.uint8, device=dev)
+    path = kdn.PATH_NAMES[kdn.kdn_execution_path(prob)]
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kdn.forward(d["q"], d["k"], d["v"], d["alpha"], d["sigma"], d["r"], cu_seqlens=cu, mu=w.mu, chunk=w.chunk,
+                    o=o, S_out=S_out, P_out=P_out, workspace=ws, max_seqlen=max_seqlen)
+
+    for _ in range(args.warmup):
+        step()
+    kdn.last_device_error()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    kdn.last_device_error()
+    value, ms = whole_job_rate(w.ntok, steps, e0.elapsed_time(e1), world)
+    out = dict(workload=w.name, value=value, unit="tokens/s", ms_per_step=ms / steps, steps=steps,
+               gpu_launches=steps * (2 if path == "chunk_tcgen05_two_phase" else 1), path=path,
+               bytes=algorithmic_bytes(w))
+    del d, o, S_out, P_out, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def bench_decode(args, world, rank, dev, kdn, steps=1024, N=256, H=32, d=128):
     """1024 decode steps on 256 sequences x 32 heads (inputs resident, drawn on the device)."""
     import torch
-    g = torch.Generator(device=dev)
-    g.manual_seed(2_000 + rank)
-    S = 0.1 * torch.randn((N, H, d, d), generator=g, device=dev)
-    P = torch.nn.functional.softplus(torch.randn((N, H, d), generator=g, device=dev))
-    shape = (steps, N, H, d)
-    q = torch.nn.functional.normalize(torch.randn(shape, generator=g, device=dev), dim=-1).bfloat16()
-    k = torch.nn.functional.normalize(torch.randn(shape, generator=g, device=dev), dim=-1).bfloat16()
-    v = torch.randn(shape, generator=g, device=dev).bfloat16()
-    al = torch.sigmoid(torch.randn(shape, generator=g, device=dev) + 4.0).bfloat16()
-    r = (torch.nn.functional.softplus(torch.randn((steps, N, H), generator=g, device=dev)) + 1e-3).bfloat16()
-    sg = torch.nn.functional.softplus(torch.randn(shape, generator=g, device=dev) - 3.0).bfloat16()
+    from kalman_delta_rule_b200 import inputs
+    dv = inputs.decode_inputs_device(2_000 + rank, steps, N, H, d, device=dev)
+    S, P = dv["S0"], dv["P0"]
+    q, k, v, al, sg, r = (dv[n] for n in ("q", "k", "v", "alpha", "sigma", "r"))
     o = torch.empty((N, H, d), dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -527,6 +543,11 @@ def ours(args):
     pk, pk_kind = peaks()
     pre = bench_prefill(args, world, rank, dev, kdn)
     dec = bench_decode(args, world, rank, dev, kdn, steps=args.decode_steps) if not args.no_decode else None
+    others = []
+    if not args.no_other_workloads:
+        for name in ("long", "varlen"):
+            if name != args.workload:
+                others.append(bench_prefill_other(args, world, rank, dev, kdn, name))
     w = pre["w"]
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -562,10 +583,6 @@ def ours(args):
             it["unit"] = "tokens/s"
             it["roofline_frac"] = pre["bytes"] / (it["ms_per_step"] / 1e3) / 1e9 / hbm
             line["prefill_isotropic"] = it
-        if pre["single"] is not None:
-            sg = pre["single"]
-            sg["roofline_frac"] = pre["bytes"] / (sg["ms_per_step"] / 1e3) / 1e9 / hbm
-            line["prefill_single_kernel"] = sg
         if pre["scan"] is not None:
             sc = pre["scan"]
             sach = sc["bytes"] / (sc["ms_step"] / 1e3) / 1e9
@@ -584,6 +601,16 @@ def ours(args):
                                              "frac": bach / hbm, "traffic": None,
                                              "algorithmic_bytes_per_launch": bw["bytes"],
                                              "unit_of_measure": "one backward call = its four launches"}}
+        for ot in others:
+            oach = ot["bytes"] / (ot["ms_per_step"] / 1e3) / 1e9
+            key = "prefill_long" if ot["workload"].startswith("long") else "prefill_varlen"
+            line[key] = {"metric": "KDN prefill tokens/s", "workload": ot["workload"], "value": ot["value"],
+                         "unit": "tokens/s", "ms_per_step": ot["ms_per_step"], "steps": ot["steps"],
+                         "gpu_launches": ot["gpu_launches"], "kernel_path": ot["path"],
+                         "roofline": {"bound": "hbm", "achieved": oach, "peak": hbm, "unit": "GB/s",
+                                      "frac": oach / hbm, "traffic": None,
+                                      "algorithmic_bytes_per_launch": ot["bytes"],
+                                      "unit_of_measure": "one forward step (prep + state launch)"}}
         if dec is not None:
             dach = dec["bytes"] / (dec["ms_step"] / 1e3) / 1e9
             line["decode"] = {"metric": "decode steps/s", "value": dec["value"], "unit": "steps/s",
@@ -667,6 +694,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-scan", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the long-context and packed-varlen prefill lines")
     ap.add_argument("--decode-steps", type=int, default=1024)
     args = ap.parse_args()
     if args.warmup < 3:

@@ -38,9 +38,10 @@
  *  - Streams: every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream).  Argument validation is synchronous and returns an
  *    error before anything is launched.  A failed launch returns KDN_ERR_CUDA.
- *  - Device-side conditions (a bounded wait that gave up, an input outside the
- *    tensor-core path's range) are recorded in a device error word and reported,
- *    after a stream synchronisation, by kdn_last_device_error().
+ *  - Device-side conditions (a bounded wait that gave up, a packed sequence longer than
+ *    the gain scan's max_seqlen) are recorded in a device error word and reported, after
+ *    a stream synchronisation, by kdn_last_device_error().  The outputs of a call whose
+ *    kernels recorded such a condition are undefined.
  *  - Thread safety: calls may come from several host threads on different streams.
  *    Calls that share output or state buffers must be ordered by the caller.
  */
@@ -60,7 +61,7 @@ typedef enum {
     KDN_ERR_UNSUPPORTED = 2,   /* d_k / d_v / chunk / dtype combination not built */
     KDN_ERR_CUDA = 3,          /* a CUDA runtime call or a launch failed */
     KDN_ERR_TIMEOUT = 4,       /* a bounded device wait gave up (kernel returned early) */
-    KDN_ERR_RANGE = 5,         /* a chunk's cumulative decay left the tensor-core path's range */
+    KDN_ERR_RANGE = 5,         /* reserved: no path limits the decay range (every alpha in [0,1] is supported) */
     KDN_ERR_WORKSPACE = 6      /* workspace missing or smaller than kdn_workspace_size() */
 } kdn_status_t;
 
@@ -71,11 +72,13 @@ typedef enum { KDN_VARIANT_DIAGONAL = 0, KDN_VARIANT_ISOTROPIC = 1 } kdn_variant
 
 /* Execution paths of kdn_forward_chunkwise (the `chunk` field):
  *  0        token-serial fused recurrence (any dtype; exact fp32 arithmetic);
- *  16/32/64 chunkwise: for bf16 inputs, d_k = 128 and chunk 64 the tcgen05 tensor cores --
- *           in two launches (a chunk-parallel prep kernel, then the chunk-serial state
- *           kernel) when the call gets a workspace of kdn_workspace_size() bytes and the
- *           uncertainty is diagonal, else in one fused kernel; otherwise the fp32
- *           CUDA-core chunk kernel (same algebra, fp32 FMA). */
+ *  16/32/64 chunkwise: for bf16 inputs, d_k = 128 and chunk 64, when the call gets a
+ *           workspace of kdn_workspace_size() bytes, the tcgen05 tensor cores in two
+ *           launches (a chunk-parallel prep kernel, then the chunk-serial state kernel);
+ *           otherwise the fp32 CUDA-core chunk kernel (same algebra, fp32 FMA, exact but
+ *           several times slower).  Every path accepts any alpha in [0, 1], alpha = 0
+ *           resets included: the tensor-core path forms the intra-chunk decay factors on the
+ *           CUDA cores for a chunk whose decay falls below 2^-100 on some channel. */
 typedef struct {
     int B, T, H, d_k, d_v;          /* varlen: B == 1 and T = total tokens */
     const int32_t *cu_seqlens;      /* device int32 [num_seqs + 1], cu[0] = 0, cu[num_seqs] = T; NULL = dense batch */
@@ -94,7 +97,7 @@ typedef struct {
  * tensor-core forward use.  The forward's part is about 70 KB per 64-token chunk and head
  * (per-chunk operand records and look-back state); packed sequences hold at most
  * T/64 + num_seqs chunks per head, so it does not depend on `max_seqlen`.  The forward
- * also accepts workspace = NULL and then runs the single-kernel paths.  Host-only. */
+ * also accepts workspace = NULL and then runs the fp32 CUDA-core paths.  Host-only. */
 kdn_status_t kdn_workspace_size(const kdn_problem_t *p, size_t *bytes);
 
 /* Prefill / training forward over whole sequences (KDA article, "chunkwise" regime;
@@ -106,10 +109,11 @@ kdn_status_t kdn_workspace_size(const kdn_problem_t *p, size_t *bytes);
  *  o                  : device [B, T, H, d_v]        (in_dtype), written for every token
  *  S_out, P_out       : device fp32, final states per sequence (shapes as S0, P0); either may be NULL.
  *                       They may not alias S0 / P0.
- *  workspace          : device, 256-byte aligned, or NULL.  With >= kdn_workspace_size()
- *                       bytes the tensor-core path runs in two launches (faster); with less
- *                       or NULL it runs as one kernel.  Contents on entry do not matter;
- *                       concurrent calls must use distinct workspaces.
+ *  workspace          : device, 256-byte aligned, or NULL.  The tensor-core path (bf16,
+ *                       d_k = 128, chunk 64) runs only with >= kdn_workspace_size() bytes;
+ *                       with less or NULL the call takes the fp32 CUDA-core chunk kernel.
+ *                       Contents on entry do not matter; concurrent calls must use distinct
+ *                       workspaces.
  * Every sequence starts from its own S0/P0 (chunks restart at sequence starts). */
 kdn_status_t kdn_forward_chunkwise(const kdn_problem_t *p,
                                    const void *q, const void *k, const void *v,
@@ -227,9 +231,9 @@ kdn_status_t kdn_backward(const kdn_problem_t *p,
 
 /* Which execution path kdn_forward_chunkwise() takes for `p` (host-only; no CUDA call
  * besides resolving the driver's tensor-map encoder once): 0 token-serial recurrence,
- * 1 fp32 CUDA-core chunk kernel, 2 tcgen05 tensor-core chunk kernel, 3 the tcgen05 path in
- * two launches (taken when the call also gets a workspace of kdn_workspace_size() bytes;
- * without one such a problem runs path 2); -1 if `p` is invalid. */
+ * 1 fp32 CUDA-core chunk kernel, 3 the tcgen05 tensor-core path in two launches (taken when
+ * the call also gets a workspace of kdn_workspace_size() bytes; without one such a problem
+ * runs path 1); -1 if `p` is invalid.  (2 is not returned.) */
 int kdn_execution_path(const kdn_problem_t *p);
 
 /* Self-test of failure detection: launches one kernel whose two bounded waits -- a poll of a
@@ -241,7 +245,7 @@ int kdn_execution_path(const kdn_problem_t *p);
 kdn_status_t kdn_selftest_bounded_wait(long long limit_cycles, void *stream);
 
 /* Synchronises `stream`, then returns and clears the device error word
- * (KDN_ERR_TIMEOUT, KDN_ERR_RANGE or KDN_ERR_INVALID_ARG if a kernel recorded one, else KDN_OK). */
+ * (KDN_ERR_TIMEOUT or KDN_ERR_INVALID_ARG if a kernel recorded one, else KDN_OK). */
 kdn_status_t kdn_last_device_error(void *stream);
 
 /* Static description of a status code. */

@@ -203,7 +203,7 @@ def forward(q, k, v, alpha, sigma, r, cu_seqlens=None, S0=None, P0=None, mu: flo
 
     Returns (o, S_out, P_out); P is [N,H,dk] (diagonal) or [N,H] (isotropic).  Outputs are
     allocated when not given; so is the workspace when ``workspace`` is None (``False``
-    passes none, which selects the single-kernel paths)."""
+    passes none: the tensor-core path needs one, so such a call runs the fp32 chunk kernel)."""
     torch = _torch()
     p = make_problem(q, v, cu_seqlens=cu_seqlens, mu=mu, chunk=chunk, variant=variant, max_seqlen=max_seqlen)
     N = p.num_seqs
@@ -310,17 +310,18 @@ def gain_scan(k, alpha, sigma, r, cu_seqlens=None, P0=None, mu: float = 1.0, chu
     return g, be, P_out
 
 
-PATH_NAMES = {0: "recurrent", 1: "chunk_fp32", 2: "chunk_tcgen05", 3: "chunk_tcgen05_two_phase"}
+PATH_NAMES = {0: "recurrent", 1: "chunk_fp32", 3: "chunk_tcgen05_two_phase"}
 
 
 def execution_path(q, v, cu_seqlens=None, mu: float = 1.0, chunk: int = 64, variant: str = "diagonal",
                    workspace: bool = True) -> str:
     """Name of the kernel path kdn_forward_chunkwise takes for these tensors (``workspace``:
-    whether the call gets a workspace of kdn_workspace_size() bytes)."""
+    whether the call gets a workspace of kdn_workspace_size() bytes; the tensor-core path
+    needs one, and without it the call runs the fp32 chunk kernel)."""
     p = make_problem(q, v, cu_seqlens=cu_seqlens, mu=mu, chunk=chunk, variant=variant)
     code = kdn_execution_path(p)
     if code == 3 and not workspace:
-        code = 2
+        code = 1
     return PATH_NAMES.get(code, "invalid")
 
 

@@ -1,7 +1,6 @@
 // C ABI of libkdn.so: argument validation, workspace sizing, dispatch to the kernels,
 // and the device error word.  Declarations and the contract are in include/kdn.h.
 #include <math.h>
-#include <mutex>
 
 #include "kdn_common.cuh"
 #include "kdn_launch.h"
@@ -10,20 +9,11 @@ namespace {
 
 __device__ unsigned g_kdn_err;  // bits kdn::ERR_*; one copy per device
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-unsigned *g_err_ptr[kMaxDevices];
-
+// the current device's error word (address looked up once per device and context)
 unsigned *err_word() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_err_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_kdn_err) != cudaSuccess) return nullptr;
-        g_err_ptr[dev] = static_cast<unsigned *>(p);
-    }
-    return g_err_ptr[dev];
+    void *p = nullptr;
+    if (kdn::symbol_address(reinterpret_cast<const void *>(&g_kdn_err), &p) != cudaSuccess) return nullptr;
+    return static_cast<unsigned *>(p);
 }
 
 bool dk_ok(int d) { return d == 32 || d == 64 || d == 128; }
@@ -63,14 +53,11 @@ kdn_status_t check_problem(const kdn_problem_t *p, Resolved *out) {
 
 kdn_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? KDN_OK : KDN_ERR_CUDA; }
 
-// the tensor-core chunk kernels serve this problem (bf16, d_k = 128, chunk 64)
-bool tc_path(const kdn_problem_t *p, const Resolved &rv) {
-    return kdn::chunk_tc_supported(p->d_k, p->d_v, rv.bf16, p->chunk, rv.ntok);
-}
-// ... and the two-launch form applies (work list within 2^31 units)
+// the tensor-core chunk kernels serve this problem (bf16, d_k = 128, chunk 64, work list
+// within 2^31 units)
 bool two_phase_path(const kdn_problem_t *p, const Resolved &rv) {
     const long long units = p->cu_seqlens ? (rv.ntok / 64 + rv.nseq) * p->H : (long long)rv.nseq * p->H * rv.nchunks_max;
-    return tc_path(p, rv) && units < (1ll << 31);
+    return kdn::chunk_tc_supported(p->d_k, p->d_v, rv.bf16, p->chunk, rv.ntok) && units < (1ll << 31);
 }
 size_t two_phase_bytes(const kdn_problem_t *p, const Resolved &rv) {
     if (p->cu_seqlens) {   // packed: sum_s ceil(len_s / 64) <= T / 64 + num_seqs units per head
@@ -91,7 +78,7 @@ const char *kdn_status_string(kdn_status_t s) {
         case KDN_ERR_UNSUPPORTED: return "unsupported size, dtype or chunk";
         case KDN_ERR_CUDA: return "CUDA runtime or launch error";
         case KDN_ERR_TIMEOUT: return "a bounded device wait gave up";
-        case KDN_ERR_RANGE: return "chunk decay outside the tensor-core path's range";
+        case KDN_ERR_RANGE: return "value outside the supported range (reserved; no kernel reports it)";
         case KDN_ERR_WORKSPACE: return "workspace missing or too small";
     }
     return "unknown status";
@@ -141,11 +128,6 @@ kdn_status_t kdn_forward_chunkwise(const kdn_problem_t *p, const void *q, const 
     }
     if (two_phase_path(p, rv) && workspace && aligned256(workspace) && workspace_bytes >= two_phase_bytes(p, rv))
         return cuda_status(kdn::launch_chunk_two_phase(a, rv.ntok, rv.nchunks_max, workspace, cs));
-    if (tc_path(p, rv)) {
-        const long long ctas128 = (long long)rv.nseq * p->H * (p->d_v / 128);
-        const int dvt = (p->d_v == 64 || ctas128 < 148) ? 64 : 128;
-        return cuda_status(kdn::launch_chunk_tc(a, rv.ntok, dvt, cs));
-    }
     return cuda_status(kdn::launch_chunk_simt(a, rv.bf16, p->chunk, cs));
 }
 
@@ -284,8 +266,7 @@ int kdn_execution_path(const kdn_problem_t *p) {
     Resolved rv;
     if (check_problem(p, &rv) != KDN_OK) return -1;
     if (p->chunk == 0) return 0;
-    if (two_phase_path(p, rv)) return 3;
-    return tc_path(p, rv) ? 2 : 1;
+    return two_phase_path(p, rv) ? 3 : 1;
 }
 
 kdn_status_t kdn_last_device_error(void *stream) {

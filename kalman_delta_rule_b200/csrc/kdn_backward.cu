@@ -697,18 +697,24 @@ static cudaError_t launch_local(const BwdArgs &b, const BwdWs &w, cudaStream_t s
     return cudaGetLastError();
 }
 
+// the kernel's dynamic shared-memory limit, set once per device and context
+static cudaError_t set_smem(const void *kern, size_t smem) {
+    KernelSetup ks;
+    return kernel_setup(kern, smem, 128, false, &ks);
+}
+
 template <typename T>
 static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, cudaStream_t st) {
     const int chains = b.a.nseq * b.a.H, dk = b.a.dk;
     cudaError_t e;
     if (b.a.iso) {
         const size_t tsm = (size_t)7 * GT * sizeof(float) + (size_t)3 * GT * dk * sizeof(T);
-        e = cudaFuncSetAttribute(bwd_tape_iso_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+        e = set_smem(reinterpret_cast<const void *>(bwd_tape_iso_kernel<T>), tsm);
         if (e != cudaSuccess) return e;
         bwd_tape_iso_kernel<T><<<chains, dk, tsm, st>>>(b, w);
     } else {
         const size_t tsm = ((size_t)2 * GT * dk + 4 * GT) * sizeof(float) + (size_t)3 * GT * dk * sizeof(T);
-        e = cudaFuncSetAttribute(bwd_tape_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+        e = set_smem(reinterpret_cast<const void *>(bwd_tape_kernel<T>), tsm);
         if (e != cudaSuccess) return e;
         bwd_tape_kernel<T><<<chains, dk, tsm, st>>>(b, w);
     }
@@ -716,7 +722,7 @@ static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, cudaStream
     if (e != cudaSuccess) return e;
     const size_t ssm = ((size_t)CK * dk + (CK / NS) * DB * dk + CK * DB + 4 * DB + DB) * sizeof(float) +
                        ((size_t)3 * CK * dk + CK * DB) * sizeof(T);
-    e = cudaFuncSetAttribute(bwd_state_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssm);
+    e = set_smem(reinterpret_cast<const void *>(bwd_state_kernel<T>), ssm);
     if (e != cudaSuccess) return e;
     bwd_state_kernel<T><<<(unsigned)chains * w.nblk, dk, ssm, st>>>(b, w);
     e = cudaGetLastError();
@@ -725,13 +731,13 @@ static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, cudaStream
     if (e != cudaSuccess) return e;
     if (b.a.iso) {
         const size_t psm = ((size_t)2 * GT * dk + 9 * GT) * sizeof(float) + (size_t)2 * GT * dk * sizeof(T);
-        e = cudaFuncSetAttribute(bwd_prev_iso_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
+        e = set_smem(reinterpret_cast<const void *>(bwd_prev_iso_kernel<T>), psm);
         if (e != cudaSuccess) return e;
         bwd_prev_iso_kernel<T><<<chains, dk, psm, st>>>(b, w);
         return cudaGetLastError();
     }
     const size_t psm = ((size_t)5 * GT * dk + 2 * GT) * sizeof(float) + (size_t)3 * GT * dk * sizeof(T);
-    e = cudaFuncSetAttribute(bwd_prev_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
+    e = set_smem(reinterpret_cast<const void *>(bwd_prev_kernel<T>), psm);
     if (e != cudaSuccess) return e;
     bwd_prev_kernel<T><<<chains, dk, psm, st>>>(b, w);
     return cudaGetLastError();

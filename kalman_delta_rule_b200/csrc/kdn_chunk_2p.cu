@@ -8,12 +8,17 @@
 //
 //   prep  (one unit = one 64-token chunk of one (sequence, head); every unit in parallel):
 //         compose the chunk's 2x2 uncertainty maps, take the starting uncertainty from the
-//         chunk's predecessors by decoupled look-back, re-expand P^- per token, form
-//         K~ = k Gam, Q~ = q Gam, G^ = P^- k / Gam and 1/den, then on the tensor cores
-//         [A; Aq] = [K~; Q~] G^^T, T = (I + A)^{-1}, X = Aq T, [w; X K~] = [T; X] K~, and
-//         write one record per unit: [-w; Q'] (Q' = Q~ - X K~), [T; X], G^, 1/den, Gam_{L-1};
+//         chunk's predecessors by decoupled look-back, re-expand P^- per token, form the
+//         decayed operands and 1/den, then [A; Aq] (the intra-chunk interaction matrices with
+//         their pairwise decay), T = (I + A)^{-1}, X = Aq T, [w; X K~] = [T; X] K~, and write
+//         one record per unit: [-w; Q'] (Q' = Q~ - X K~), [T; X], G', 1/den, Gam_L;
 //   state (one CTA per (sequence, head, d_v tile); chunks in order):
-//         [U; O] = [-w; Q'] S + [T; X] V,   S <- Gam_{L-1} (S + G^^T (U / den)).
+//         [U; O] = [-w; Q'] S + [T; X] V,   S <- Gam_L S + G'^T (U / den).
+// Here Gam_t is the decay from the chunk start through token t (per channel), Gam_L the whole
+// chunk's, K~ = k Gam_t, Q~ = q Gam_t and G' = P^- k Gam_L / Gam_t: every operand of the state
+// kernel is at most its undecayed value, whatever the decay.  A and Aq are formed on the tensor
+// cores from operands referenced to the chunk end when every channel's Gam_L >= 2^-100, else on
+// the CUDA cores from log-space pairwise decay factors, so any alpha in [0, 1] is in range.
 //
 // Records are stored exactly in the state kernel's shared-memory operand layout (128-byte
 // swizzled atoms), so the state kernel fetches each with one bulk copy, double-buffered,
@@ -26,6 +31,8 @@
 // The prep kernel runs two 256-thread CTAs per SM; work is handed out by a ticket counter
 // in chunk-major order, so every predecessor of a unit belongs to a CTA that is already
 // running, and every wait is bounded (a wait that gives up records KDN_ERR_TIMEOUT).
+#include <mutex>
+
 #include "kdn_common.cuh"
 #include "kdn_launch.h"
 #include "kdn_tc.cuh"
@@ -35,19 +42,23 @@ namespace kdn {
 namespace {
 constexpr int C = 64, DK = 128, PNT = 256, SNT = 256;
 constexpr int ADS = 36;   // padded fp32 row stride of the diagonal blocks (conflict-free row-wise float4 access)
+constexpr int XLD = 65;   // padded row stride (words) of the out-of-range path's [channel][token] staging
+// A chunk whose decay Gam_L (product of its alphas) is at least this on every channel takes the
+// factored tensor-core form (operands up to 1 / Gam_L); below it, the pairwise CUDA-core form.
+constexpr float kMinChunkDecay = 0x1p-100f;
 
 // one unit's record; each part in the state kernel's operand layout
 struct Rec {
     static constexpr uint32_t A4 = 0;          // [-w; Q'] bf16: 2 channel atoms x 128 rows x 128 B
     static constexpr uint32_t Y = 32768;       // [T; X] bf16: 128 rows x 64 tokens
-    static constexpr uint32_t G = 49152;       // G^ bf16: 2 channel atoms x 64 token rows
-    static constexpr uint32_t MISC = 65536;    // 1/den [64] fp32, then Gam_{L-1} [128] fp32
+    static constexpr uint32_t G = 49152;       // G' bf16: 2 channel atoms x 64 token rows
+    static constexpr uint32_t MISC = 65536;    // 1/den [64] fp32, then Gam_L [128] fp32
     static constexpr uint32_t BYTES = MISC + 768;
 };
 
 struct PrepSmem {
-    static constexpr uint32_t KQ = 0;                  // [K~; Q~] bf16, 2 channel atoms x 128 rows
-    static constexpr uint32_t G = 32768;               // G^ bf16 (record part)
+    static constexpr uint32_t KQ = 0;                  // [K; Q] decayed bf16, 2 channel atoms x 128 rows
+    static constexpr uint32_t G = 32768;               // G' bf16 (record part)
     static constexpr uint32_t W = 49152;               // work region, reused phase by phase:
     static constexpr uint32_t COMP = W;                //   segment composites fp32 [4][128][4]
     static constexpr uint32_t AQ = W;                  //   Aq bf16 64 x 64
@@ -57,7 +68,7 @@ struct PrepSmem {
     static constexpr uint32_t ADG = W + 32768;         //   fp32 [2][32][ADS]: A's diagonal blocks, then D's
     static constexpr uint32_t A4 = W;                  //   [-w; Q'] (record part), once the inverse is done
     static constexpr uint32_t Y = W + 43008;           //   [T; X] (record part)
-    static constexpr uint32_t MISC = W + 59392;        // 1/den [64], Gam_{L-1} [128] (record tail)
+    static constexpr uint32_t MISC = W + 59392;        // 1/den [64], Gam_L [128] (record tail)
     static constexpr uint32_t RS = MISC + 768;         // r [64]
     static constexpr uint32_t MUR = RS + 256;          // mu / r [64]
     static constexpr uint32_t PST = MUR + 256;         // uncertainty at the chunk start [128]
@@ -65,8 +76,16 @@ struct PrepSmem {
     static constexpr uint32_t TSUM = DSUM + 256;       // isotropic: per-token sums of alpha^2, sigma, k^2 [64][4]
     static constexpr uint32_t CTL = TSUM + 1024;       // mbarrier, ticket, TMEM slot, look-back flag, abort
     static constexpr uint32_t total = CTL + 64;
+    // out-of-range units (pairwise decay on the CUDA cores), staged one half of the channels at a time
+    static constexpr uint32_t XKQ = 0;                 // (k, q) bf16 pairs [64][XLD], over K~/Q~
+    static constexpr uint32_t XPK = XKQ + 64 * XLD * 4;  // P^- k fp32 [64][XLD]
+    static constexpr uint32_t XLG = W + 8192;          // log2 decay from the chunk start fp32 [64][XLD]
+    static constexpr uint32_t LSUM = W + 26624;        // per-segment log2 decay sums [4][128]
+    static constexpr uint32_t XAA = W + 8192;          // A (rows 0..63) and Aq fp32 [128][XLD], once staged
     static_assert(COMP + 4 * 128 * 16 <= DB, "composites overlap D");
     static_assert(ADG + 64 * ADS * 4 <= Y && Y + 16384 <= MISC && A4 + 32768 <= Y, "work region");
+    static_assert(XPK + 64 * XLD * 4 <= W && XLG + 64 * XLD * 4 <= LSUM && LSUM + 2048 <= Y, "staging");
+    static_assert(XAA + 128 * XLD * 4 <= Y, "A staging");
 };
 
 template <int DVT>
@@ -202,12 +221,13 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
     float *pst = reinterpret_cast<float *>(sm + L_::PST);
     float *dsum = reinterpret_cast<float *>(sm + L_::DSUM);
     float *tsum = reinterpret_cast<float *>(sm + L_::TSUM);
+    float *lsum = reinterpret_cast<float *>(sm + L_::LSUM);
     float *comp = reinterpret_cast<float *>(sm + L_::COMP);
     float *adg = reinterpret_cast<float *>(sm + L_::ADG);
     uint64_t *bar_mma = reinterpret_cast<uint64_t *>(sm + L_::CTL);
     long long *ticket = reinterpret_cast<long long *>(sm + L_::CTL + 8);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L_::CTL + 16);
-    int *ctl = reinterpret_cast<int *>(sm + L_::CTL + 20);   // [0] look-back flag, [1] abort
+    int *ctl = reinterpret_cast<int *>(sm + L_::CTL + 20);   // [0] look-back flag, [1] abort, [2] out-of-range unit
 
     const TokenArgs &a = pa.a;
     const bf16 *__restrict__ qin = static_cast<const bf16 *>(a.q);
@@ -273,7 +293,10 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
     };
 
     for (;;) {
-        if (tid == 0) *ticket = (long long)atomicAdd(pa.counter, 1u);
+        if (tid == 0) {
+            *ticket = (long long)atomicAdd(pa.counter, 1u);
+            ctl[2] = 0;   // the unit's decay-range class (set below when it leaves the factored range)
+        }
         __syncthreads();
         const long long u = *ticket;
         if (u >= units || ctl[1]) break;
@@ -428,6 +451,12 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
                 const float sc = 1.f / n11;
                 g00 = n00 * sc; g01 = n01 * sc; g10 = n10 * sc; g11 = 1.f;
             }
+            {   // the chunk's decay Gam_{L-1} per channel, from the segments' decay products
+                const float gl = comp[cc * 4 + 3] * comp[(128 + cc) * 4 + 3] * comp[(256 + cc) * 4 + 3] *
+                                 comp[(384 + cc) * 4 + 3];
+                gamc[cc] = gl;
+                if (!(gl >= kMinChunkDecay)) ctl[2] = 1;
+            }
             if (c > 0) {   // publish the aggregate
                 st_relaxed(desc + 0 * DK, tagged(g00, TAG_AGG));
                 st_relaxed(desc + 1 * DK, tagged(g01, TAG_AGG));
@@ -484,91 +513,215 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
         __syncthreads();
 
         // ---- re-expansion fused with the chunk operands: P^- per token (from the chunk-start
-        //      uncertainty through the earlier segments' composites), Gam (inclusive decay from
-        //      the chunk start), K~ = k Gam, Q~ = q Gam, G^ = P^- k / Gam, den partial sums
-        {
-            float Pa = pst[ch], Pb = pst[ch + 1], gama, gamb;
-            gamma_start(gama, gamb);
-            for (int q2 = 0; q2 < sgi; ++q2) {
-                const float4 ca = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch) * 4);
-                const float4 cb = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch + 1) * 4);
-                Pa = mob(ca.x, ca.y, ca.z, 1.f, Pa);
-                Pb = mob(cb.x, cb.y, cb.z, 1.f, Pb);
+        //      uncertainty through the earlier segments' composites), the gain denominators'
+        //      partial sums, and the decayed operands.
+        //      In range (every channel's chunk decay Gam_L >= kMinChunkDecay) the operands are
+        //      referenced to the chunk END: K' = k Gam_t / Gam_L and Q' = q Gam_t / Gam_L (between
+        //      k and k / Gam_L), G' = P^- k Gam_L / Gam_t (at most P^- k), so MMA1's A = K' G'^T
+        //      carries the pairwise decay Gam_t / Gam_s of every pair exactly, and MMA2 takes
+        //      Gam_L back as a column scale.
+        //      Out of range (an alpha = 0 reset, or strong decay) A and Aq are formed on the CUDA
+        //      cores with every pairwise factor 2^(lg_t - lg_s) <= 1 taken from log-space decay
+        //      sums, and the operands are referenced to the chunk START: K~ = k Gam_t, Q~ = q Gam_t,
+        //      G' = P^- k 2^(lg_L - lg_t); every factor is at most 1, so nothing overflows.
+        const bool out_of_range = ctl[2] != 0;   // CTA-uniform
+        float Ps_a = pst[ch], Ps_b = pst[ch + 1];   // uncertainty at the segment start
+        for (int q2 = 0; q2 < sgi; ++q2) {
+            const float4 ca = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch) * 4);
+            const float4 cb = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch + 1) * 4);
+            Ps_a = mob(ca.x, ca.y, ca.z, 1.f, Ps_a);
+            Ps_b = mob(cb.x, cb.y, cb.z, 1.f, Ps_b);
+        }
+        // one token of the uncertainty walk on the channel pair's bf16 words (alpha, sigma, k):
+        // returns P^- of the pair and advances P
+        auto predict_update = [&](int t, uint32_t aa, uint32_t ss, uint32_t kk2, float &Pa, float &Pb) -> f32x2 {
+            if constexpr (!ISO) {   // both channels of the pair at once (f32x2)
+                const f32x2 al = bf2(aa), kk = bf2(kk2);
+                const f32x2 pm = fma2(mul2(al, al), pk2(Pa, Pb), bf2(ss));
+                const float mr = mur[t];
+                const f32x2 dn = fma2(mul2(mul2(pk2(mr, mr), kk), kk), pm, pk2(1.f, 1.f));
+                Pa = __fdividef(x2(pm), x2(dn));
+                Pb = __fdividef(y2(pm), y2(dn));
+                return pm;
+            } else {   // the head's map, the same on every channel
+                const float4 iso = *reinterpret_cast<const float4 *>(tsum + t * 4);
+                const float pma = fmaf(iso.x, Pa, iso.y), pmb = fmaf(iso.x, Pb, iso.y);
+                Pa = __fdividef(pma, fmaf(iso.z, pma, 1.f));
+                Pb = __fdividef(pmb, fmaf(iso.z, pmb, 1.f));
+                return pk2(pma, pmb);
             }
+        };
+        auto store_operands = [&](int t, uint32_t kq, uint32_t qq, uint32_t gg) {
+            *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(t, bch)) = kq;
+            *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(64 + t, bch)) = qq;
+            *reinterpret_cast<uint32_t *>(sm + L_::G + atom8 + swz(t, bch)) = gg;
+        };
+        if (!out_of_range) {
+            float Pa = Ps_a, Pb = Ps_b, gama, gamb;
+            gamma_start(gama, gamb);
+            // up = Gam_t / Gam_L, in [1, 2^100]: K' = k up, Q' = q up, G' = P^- k / up
+            f32x2 up = pk2(gama / gamc[ch], gamb / gamc[ch + 1]);
             float xs[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const int t = tb + j;
                 uint32_t kq = 0u, qq = 0u, gg = 0u;
                 xs[j] = 0.f;
-                if (!ISO && t < L) {   // both channels of the pair at once (f32x2)
-                    const f32x2 al = bf2(aw[j]), kk = bf2(kw[j]);
-                    const f32x2 pm = fma2(mul2(al, al), pk2(Pa, Pb), bf2(sw[j]));
-                    const float mr = mur[t];
-                    const f32x2 dn = fma2(mul2(mul2(pk2(mr, mr), kk), kk), pm, pk2(1.f, 1.f));
-                    Pa = __fdividef(x2(pm), x2(dn));
-                    Pb = __fdividef(y2(pm), y2(dn));
-                    gama *= x2(al);
-                    gamb *= y2(al);
-                    const f32x2 gm = pk2(gama, gamb), pk = mul2(pm, kk), kg = mul2(kk, gm), qg = mul2(bf2(qw[j]), gm);
+                if (t < L) {
+                    const f32x2 pm = predict_update(t, aw[j], sw[j], kw[j], Pa, Pb);
+                    const f32x2 kk = bf2(kw[j]);
+                    up = mul2(up, bf2(aw[j]));
+                    const f32x2 pk = mul2(pm, kk), kg = mul2(kk, up), qg = mul2(bf2(qw[j]), up);
                     kq = pack_bf16x2(x2(kg), y2(kg));
                     qq = pack_bf16x2(x2(qg), y2(qg));
-                    gg = pack_bf16x2(__fdividef(x2(pk), gama), __fdividef(y2(pk), gamb));
+                    gg = pack_bf16x2(__fdividef(x2(pk), x2(up)), __fdividef(y2(pk), y2(up)));
                     xs[j] = fmaf(x2(pk), x2(kk), y2(pk) * y2(kk));
-                } else if (ISO && t < L) {
-                    const float ala = bf16_lo(aw[j]), alb = bf16_hi(aw[j]);
-                    const float ka = bf16_lo(kw[j]), kb = bf16_hi(kw[j]);
-                    float pma, pmb;
-                    {   // the head's map, the same on every channel
-                        const float4 iso = *reinterpret_cast<const float4 *>(tsum + t * 4);
-                        pma = fmaf(iso.x, Pa, iso.y);
-                        pmb = fmaf(iso.x, Pb, iso.y);
-                        Pa = __fdividef(pma, fmaf(iso.z, pma, 1.f));
-                        Pb = __fdividef(pmb, fmaf(iso.z, pmb, 1.f));
-                    }
-                    gama *= ala;
-                    gamb *= alb;
-                    const float pka = pma * ka, pkb = pmb * kb;
-                    kq = pack_bf16x2(ka * gama, kb * gamb);
-                    qq = pack_bf16x2(bf16_lo(qw[j]) * gama, bf16_hi(qw[j]) * gamb);
-                    gg = pack_bf16x2(__fdividef(pka, gama), __fdividef(pkb, gamb));
-                    xs[j] = fmaf(pka, ka, pkb * kb);
                 }
-                *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(t, bch)) = kq;
-                *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(64 + t, bch)) = qq;
-                *reinterpret_cast<uint32_t *>(sm + L_::G + atom8 + swz(t, bch)) = gg;
-            }
-            if (tb < L && tb + 16 >= L) {   // this segment holds the chunk's last token
-                gamc[ch] = gama;
-                gamc[ch + 1] = gamb;
-                if (!(gama >= 1e-30f) || !(gamb >= 1e-30f)) raise_error(a.err, ERR_RANGE);
+                store_operands(t, kq, qq, gg);
             }
             int which;
             const float tot = warp_reduce16(xs, lane, which);
             if ((lane & 1) == 0 && tb + which < L) atomicAdd(dsum + tb + which, tot);
+        } else {
+            // Rare path: the unit's tokens are re-read from global memory (L2) where needed, so
+            // that the fast path's input registers are dead here.
+            // log2 of the decay, floored at 2^-126 (a zero decay acts as 2^-126: every pairwise
+            // factor across it is then below 2^-126); per-segment sums first
+            auto lg2 = [](float al) { return __log2f(fmaxf(al, 0x1p-126f)); };
+            auto tok = [&](const bf16 *base, int t) { return ldg_u32(base + ((size_t)(c0 + t) * H + h) * DK + ch); };
+            {
+                float la = 0.f, lb = 0.f;
+                for (int j = 0; j < 16; ++j)
+                    if (tb + j < L) {
+                        const uint32_t aa = tok(ain, tb + j);
+                        la += lg2(bf16_lo(aa));
+                        lb += lg2(bf16_hi(aa));
+                    }
+                lsum[sgi * 128 + ch] = la;
+                lsum[sgi * 128 + ch + 1] = lb;
+            }
+            __syncthreads();
+            float lga = 0.f, lgb = 0.f, lLa = 0.f, lLb = 0.f;   // at the segment start; over the chunk
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+                const float xa = lsum[q2 * 128 + ch], xb = lsum[q2 * 128 + ch + 1];
+                if (q2 < sgi) { lga += xa; lgb += xb; }
+                lLa += xa;
+                lLb += xb;
+            }
+            // A_ts = sum_i k_ti pk_si 2^(lg_ti - lg_si) (s < t), Aq_ts likewise with q (s <= t), one
+            // half of the channels at a time staged as [channel][token]: (k, q) bf16 pairs, P^- k and
+            // lg in fp32.  Thread = token row tr x column set {sgc + 4 j}.
+            uint32_t *kqr = reinterpret_cast<uint32_t *>(sm + L_::XKQ);
+            float *pks = reinterpret_cast<float *>(sm + L_::XPK);
+            float *lgs = reinterpret_cast<float *>(sm + L_::XLG);
+            const int tr = tid & 63, sgc = tid >> 6;
+            float accA[16], accQ[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) { accA[j] = 0.f; accQ[j] = 0.f; }
+            for (int half = 0; half < 2; ++half) {
+                if ((warp & 1) == half) {   // the owners of this half's channels stage their tokens
+                    float Pa = Ps_a, Pb = Ps_b, lta = lga, ltb = lgb;
+                    const int c2 = ch - 64 * half;
+                    for (int j = 0; j < 16; ++j) {
+                        const int t = tb + j;
+                        uint32_t kqa = 0u, kqb = 0u;
+                        float pka = 0.f, pkb = 0.f;
+                        if (t < L) {
+                            const uint32_t aa = tok(ain, t), kk2 = tok(kin, t), qq2 = tok(qin, t);
+                            const f32x2 pm = predict_update(t, aa, tok(sin_, t), kk2, Pa, Pb);
+                            lta += lg2(bf16_lo(aa));
+                            ltb += lg2(bf16_hi(aa));
+                            pka = x2(pm) * bf16_lo(kk2);
+                            pkb = y2(pm) * bf16_hi(kk2);
+                            kqa = (kk2 & 0xffffu) | (qq2 << 16);
+                            kqb = (kk2 >> 16) | (qq2 & 0xffff0000u);
+                        }
+                        kqr[c2 * XLD + t] = kqa;
+                        kqr[(c2 + 1) * XLD + t] = kqb;
+                        pks[c2 * XLD + t] = pka;
+                        pks[(c2 + 1) * XLD + t] = pkb;
+                        lgs[c2 * XLD + t] = lta;
+                        lgs[(c2 + 1) * XLD + t] = ltb;
+                    }
+                }
+                __syncthreads();
+                if (tid < C) {   // this half's share of the gain denominators sum_i P^-_i k_i^2
+                    float acc = 0.f;
+                    for (int c2 = 0; c2 < 64; ++c2) acc = fmaf(pks[c2 * XLD + tid], bf16_lo(kqr[c2 * XLD + tid]), acc);
+                    dsum[tid] += acc;
+                }
+                for (int c2 = 0; c2 < 64; ++c2) {
+                    const uint32_t kq = kqr[c2 * XLD + tr];
+                    const float kt = bf16_lo(kq), qt = bf16_hi(kq), lt = lgs[c2 * XLD + tr];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int s_ = sgc + 4 * j;
+                        if (s_ <= tr) {
+                            const float w = pks[c2 * XLD + s_] * exp2f(lt - lgs[c2 * XLD + s_]);
+                            accA[j] = fmaf(kt, w, accA[j]);
+                            accQ[j] = fmaf(qt, w, accQ[j]);
+                        }
+                    }
+                }
+                __syncthreads();
+            }
+            float *aaf = reinterpret_cast<float *>(sm + L_::XAA);   // rows 0..63 A, 64..127 Aq
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                aaf[tr * XLD + sgc + 4 * j] = accA[j];
+                aaf[(64 + tr) * XLD + sgc + 4 * j] = accQ[j];
+            }
+            // the operands of the rest of the unit, referenced to the chunk start
+            float Pa = Ps_a, Pb = Ps_b, lta = lga, ltb = lgb;
+            for (int j = 0; j < 16; ++j) {
+                const int t = tb + j;
+                uint32_t kq = 0u, qq = 0u, gg = 0u;
+                if (t < L) {
+                    const uint32_t aa = tok(ain, t), kk2 = tok(kin, t);
+                    const f32x2 pm = predict_update(t, aa, tok(sin_, t), kk2, Pa, Pb);
+                    const f32x2 kk = bf2(kk2), qk = bf2(tok(qin, t));
+                    lta += lg2(bf16_lo(aa));
+                    ltb += lg2(bf16_hi(aa));
+                    const float ga = exp2f(lta), gb = exp2f(ltb);
+                    kq = pack_bf16x2(x2(kk) * ga, y2(kk) * gb);
+                    qq = pack_bf16x2(x2(qk) * ga, y2(qk) * gb);
+                    gg = pack_bf16x2(x2(pm) * x2(kk) * exp2f(lLa - lta), y2(pm) * y2(kk) * exp2f(lLb - ltb));
+                }
+                store_operands(t, kq, qq, gg);
+            }
         }
         __syncthreads();
         if (tid < C) invden[tid] = tid < L ? __fdividef(1.f, r_s[tid] + dsum[tid]) : 0.f;
         sync_tc();
 
-        // ---- MMA1: [A; Aq] = [K~; Q~] G^^T   (M=128, N=64 tokens, K=128 channels)
-        if (tid == 0) {
-            tc_fence_after();
+        // ---- MMA1 (in range): [A; Aq] = [K'; Q'] G'^T   (M=128, N=64 tokens, K=128 channels)
+        if (!out_of_range) {
+            if (tid == 0) {
+                tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t ka = (uint32_t)(ks >> 2), ko = (uint32_t)(ks & 3) * 32u;
-                mma_bf16(T_A, sdesc(sb + L_::KQ + ka * 16384u + ko, 16, 1024), sdesc(sb + L_::G + ka * 8192u + ko, 16, 1024),
-                         ID_M128_N64_KK, ks > 0);
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t ka = (uint32_t)(ks >> 2), ko = (uint32_t)(ks & 3) * 32u;
+                    mma_bf16(T_A, sdesc(sb + L_::KQ + ka * 16384u + ko, 16, 1024),
+                             sdesc(sb + L_::G + ka * 8192u + ko, 16, 1024), ID_M128_N64_KK, ks > 0);
+                }
+                mma_commit(bar_mma);
             }
-            mma_commit(bar_mma);
+            wait_mma();
         }
-        wait_mma();
         // rows 0..63: A (strictly lower) -> its lower-left 32x32 block L (bf16) and its two
         // diagonal blocks (fp32); rows 64..127: Aq (lower incl. diagonal, bf16); columns / den
         {
             const int s0 = cg * 32;
             float v[32];
-            tmem_ld32(T_A + lane_off + s0, v);
+            if (!out_of_range) {
+                tmem_ld32(T_A + lane_off + s0, v);
+            } else {
+                const float *src = reinterpret_cast<const float *>(sm + L_::XAA) + row * XLD + s0;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = src[j];
+                __syncthreads();   // every row is read before the epilogue reuses the region
+            }
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
                 const float4 d4 = *reinterpret_cast<const float4 *>(invden + s0 + j);
@@ -681,28 +834,36 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
             mma_commit(bar_mma);
         }
         wait_mma();
-        // rows 0..63 -> -w ; rows 64..127 -> Q' = Q~ - X K~   (bf16, record layout), 16 columns at a time
+        // rows 0..63 -> -w ; rows 64..127 -> Q' = Q~ - X K~   (bf16, record layout), 16 columns at a
+        // time; operands referenced to the chunk end take the chunk decay Gam_L back per column
 #pragma unroll
         for (int hh = 0; hh < 4; ++hh) {
-            float v[16];
+            float v[16], gl[16];
             tmem_ld16(T_A + 128 + lane_off + cg * 64 + hh * 16, v);
+#pragma unroll
+            for (int e = 0; e < 16; e += 4) {
+                const float4 g4 = out_of_range ? make_float4(1.f, 1.f, 1.f, 1.f)
+                                               : *reinterpret_cast<const float4 *>(gamc + cg * 64 + hh * 16 + e);
+                gl[e] = g4.x; gl[e + 1] = g4.y; gl[e + 2] = g4.z; gl[e + 3] = g4.w;
+            }
             const uint32_t atom = (uint32_t)cg * 16384u;
 #pragma unroll
             for (int chn = 0; chn < 2; ++chn) {
                 const uint32_t boff = atom + swz(row, (hh * 2 + chn) * 16);
+                float w8[8];
                 if (row < 64) {
-                    *reinterpret_cast<uint4 *>(sm + L_::A4 + boff) = pack8(v + chn * 8, -1.f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) w8[e] = -v[chn * 8 + e] * gl[chn * 8 + e];
                 } else {
                     const uint4 q4 = *reinterpret_cast<const uint4 *>(sm + L_::KQ + boff);
                     const uint32_t *qp = reinterpret_cast<const uint32_t *>(&q4);
-                    float w8[8];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        w8[2 * e] = bf16_lo(qp[e]) - v[chn * 8 + 2 * e];
-                        w8[2 * e + 1] = bf16_hi(qp[e]) - v[chn * 8 + 2 * e + 1];
+                        w8[2 * e] = (bf16_lo(qp[e]) - v[chn * 8 + 2 * e]) * gl[chn * 8 + 2 * e];
+                        w8[2 * e + 1] = (bf16_hi(qp[e]) - v[chn * 8 + 2 * e + 1]) * gl[chn * 8 + 2 * e + 1];
                     }
-                    *reinterpret_cast<uint4 *>(sm + L_::A4 + boff) = pack8(w8);
                 }
+                *reinterpret_cast<uint4 *>(sm + L_::A4 + boff) = pack8(w8);
             }
         }
         sync_tc();
@@ -849,6 +1010,20 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
                          sdesc(sb + L_::V0 + st * L_::V_BYTES + ks * 2048u + voff, 8192, 1024), ID_M128_NV_KM, 1);
             mma_commit(bar_mma);
         }
+        // ---- the memory's rows decayed by the chunk's Gam_L while MMA4 (which reads the bf16
+        //      copy) runs: S <- Gam_L S, before MMA5 adds G'^T (U / den), G' = P^- k Gam_L / Gam_s
+        {
+            const float gC = gamc[row];
+#pragma unroll
+            for (int p = 0; p < NC / CW; ++p) {
+                float v[CW];
+                const int col = cb0 + p * CW;
+                tmem_ld<CW>(T_S + lane_off + col, v);
+#pragma unroll
+                for (int j = 0; j < CW; ++j) v[j] *= gC;
+                tmem_st<CW>(T_S + lane_off + col, v);
+            }
+        }
         wait_mma();
         // rows 0..63 -> U / den (bf16); rows 64..127 -> o (global, tokens of the chunk)
 #pragma unroll
@@ -872,7 +1047,7 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        // ---- MMA5: S += G^^T (U / den)   (M=128 channels, N=DVT, K=64 tokens; both MN-major)
+        // ---- MMA5: S += G'^T (U / den)   (M=128 channels, N=DVT, K=64 tokens; both MN-major)
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
@@ -882,17 +1057,13 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
             mma_commit(bar_mma);
         }
         wait_mma();
-        // ---- rows decayed by the chunk's Gam_{L-1}; refresh the bf16 operand copy
+        // ---- refresh the bf16 operand copy of the memory
         {
-            const float gC = gamc[row];
 #pragma unroll
             for (int p = 0; p < NC / CW; ++p) {
                 float v[CW];
                 const int col = cb0 + p * CW;
                 tmem_ld<CW>(T_S + lane_off + col, v);
-#pragma unroll
-                for (int j = 0; j < CW; ++j) v[j] *= gC;
-                tmem_st<CW>(T_S + lane_off + col, v);
                 const uint32_t atom = (uint32_t)(col >> 6) * 16384u;
 #pragma unroll
                 for (int chn = 0; chn < CW / 8; ++chn)
@@ -987,6 +1158,41 @@ __global__ void __launch_bounds__(1024) unit_table_kernel(const int32_t *__restr
 }
 
 // ================================================================= host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// the driver's tensor-map encoder, resolved once through the runtime (no link against libcuda)
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [ntok, H, d] bf16 viewed as a 3-D tensor {d, H, ntok}; box = 64 channels x 1 head x 64 tokens, 128B swizzle
+bool make_token_map(CUtensorMap *m, const void *base, int d, int H, long long ntok) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)ntok};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
+    cuuint32_t box[3] = {64, 1, 64};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool chunk_tc_supported(int dk, int dv, bool bf16_in, int chunk, long long ntok) {
+    return bf16_in && chunk == C && dk == DK && (dv == 64 || dv == 128 || dv == 256) && ntok > 0 && encode_fn() != nullptr;
+}
+
 namespace {
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 size_t table_bytes(long long cmax, long long nseq) {
@@ -1004,7 +1210,8 @@ template <int DVT>
 static cudaError_t launch_state(const StateArgs &sa, unsigned grid, cudaStream_t st) {
     constexpr size_t smem = StateSmem<DVT>::total + 1024;
     auto kern = chunk_state_kernel<DVT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    KernelSetup ks;
+    cudaError_t e = kernel_setup(reinterpret_cast<const void *>(kern), smem, SNT, false, &ks);
     if (e != cudaSuccess) return e;
     kern<<<grid, SNT, smem, st>>>(sa);
     return cudaGetLastError();
@@ -1070,18 +1277,13 @@ cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long
         constexpr size_t psmem = PrepSmem::total + 1024;
         auto prep = a.iso ? (packed ? chunk_prep_kernel<true, true> : chunk_prep_kernel<true, false>)
                           : (packed ? chunk_prep_kernel<false, true> : chunk_prep_kernel<false, false>);
-        e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
-        if (e != cudaSuccess) return e;
         // all of the unified L1 / shared array as shared memory, so that two CTAs fit on an SM
-        e = cudaFuncSetAttribute(prep, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        KernelSetup ks;
+        e = kernel_setup(reinterpret_cast<const void *>(prep), psmem, PNT, true, &ks);
         if (e != cudaSuccess) return e;
-        int dev = 0, sms = 148, per = 1;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, prep, PNT, psmem);
         // two CTAs fit on an SM (registers and shared memory); the occupancy query can report
         // fewer.  Extra CTAs are harmless: units go out by ticket to resident CTAs only.
-        long long grid = (long long)sms * (per > 2 ? per : 2);
+        long long grid = (long long)ks.sms * (ks.blocks_per_sm > 2 ? ks.blocks_per_sm : 2);
         if (grid > units) grid = units;
         prep<<<(unsigned)grid, PNT, psmem, st>>>(pa);
         e = cudaGetLastError();
@@ -1091,9 +1293,11 @@ cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long
     // shorter MMAs and epilogues); with more chains than that, the widest
     int sms = 148;
     {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        KernelSetup ks;
+        e = kernel_setup(reinterpret_cast<const void *>(chunk_state_kernel<128>), StateSmem<128>::total + 1024, SNT,
+                         false, &ks);
+        if (e != cudaSuccess) return e;
+        sms = ks.sms;
     }
     int dvt = a.dv < 128 ? a.dv : 128;
     for (int w = 32; w <= dvt; w *= 2)

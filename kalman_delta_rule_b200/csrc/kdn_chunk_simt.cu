@@ -266,7 +266,8 @@ template <int DK, int DVT, typename Tin>
 static cudaError_t launch_simt(const TokenArgs &a, int C, cudaStream_t st) {
     constexpr size_t smem = SimtSmem<DK, DVT>::bytes;
     auto kern = chunk_simt_kernel<DK, DVT, Tin>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    KernelSetup ks;
+    cudaError_t e = kernel_setup(reinterpret_cast<const void *>(kern), smem, NT, false, &ks);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((size_t)a.nseq * a.H * (a.dv / DVT));
     kern<<<grid, NT, smem, st>>>(a, C);

@@ -9,19 +9,29 @@
 
 namespace kdn {
 
+// Launch set-up of a kernel on the current device and context, done once and cached: the
+// dynamic shared-memory limit set to `smem` (and the whole unified L1/shared array as shared
+// memory when `max_carveout`), the SM count and the occupancy at `threads` per CTA.
+struct KernelSetup {
+    int sms;            // multiprocessors of the device
+    int blocks_per_sm;  // resident CTAs per SM at this shared memory and block size
+};
+cudaError_t kernel_setup(const void *kern, size_t smem, int threads, bool max_carveout, KernelSetup *out);
+// Device address of a __device__ symbol on the current device and context, looked up once
+// (with that device current) and cached; looked up again after the context changes.
+cudaError_t symbol_address(const void *symbol, void **out);
+
 // token-serial fused recurrence; dvt = d_v tile per CTA (32/64/128/256, divides d_v)
 cudaError_t launch_recurrent(const TokenArgs &a, bool bf16_in, int dvt, cudaStream_t st);
 
 // chunkwise forward on CUDA cores in fp32 (chunk C <= 64); any dtype
 cudaError_t launch_chunk_simt(const TokenArgs &a, bool bf16_in, int C, cudaStream_t st);
 
-// chunkwise forward on tcgen05 tensor cores (bf16 inputs, d_k = 128, chunk 64)
+// chunkwise forward on tcgen05 tensor cores (bf16 inputs, d_k = 128, chunk 64) in two launches:
+// a chunk-parallel prep kernel (uncertainty by decoupled look-back, intra-chunk matrices,
+// triangular inverse) writing per-chunk operand records to the workspace, then the
+// chunk-serial state kernel
 bool chunk_tc_supported(int dk, int dv, bool bf16_in, int chunk, long long ntok);
-cudaError_t launch_chunk_tc(const TokenArgs &a, long long ntok, int dvt, cudaStream_t st);
-
-// the same algebra in two launches: a chunk-parallel prep kernel (uncertainty by decoupled
-// look-back, intra-chunk matrices, triangular inverse) writing per-chunk operand records to
-// the workspace, then the chunk-serial state kernel
 // units: upper bound of the (chunk, sequence x head) units; cmax > 0 for packed problems
 size_t two_phase_workspace_bytes(long long units, long long cmax, long long nseq);
 cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long nchunks_max, void *workspace,

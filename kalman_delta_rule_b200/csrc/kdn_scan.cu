@@ -264,14 +264,11 @@ template <int DK, typename Tin>
 static cudaError_t launch_scan_t(const ScanArgs &a, cudaStream_t st) {
     constexpr size_t smem = ScanSmem<DK, Tin>::total;
     auto kern = gain_scan_kernel<DK, Tin>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    KernelSetup ks;
+    cudaError_t e = kernel_setup(reinterpret_cast<const void *>(kern), smem, SNT, false, &ks);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 148, per = 1;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kern, SNT, smem);
     const long long units = (long long)a.nchunks_max * a.nchains;
-    long long grid = (long long)sms * (per > 0 ? per : 1);
+    long long grid = (long long)ks.sms * (ks.blocks_per_sm > 0 ? ks.blocks_per_sm : 1);
     if (grid > units) grid = units;
     if (grid < 1) grid = 1;
     kern<<<(unsigned)grid, SNT, smem, st>>>(a);
@@ -314,29 +311,11 @@ cudaError_t launch_gain_scan(ScanArgs a, bool bf16_in, long long ntok, void *wor
 constexpr size_t kNoAllocScratchBytes = (size_t)32 << 20;
 static __device__ __align__(256) unsigned char g_scan_scratch[kNoAllocScratchBytes];
 
-namespace {
-constexpr int kMaxScratchDevices = 64;
-std::mutex g_scratch_mu;
-void *g_scratch_addr[kMaxScratchDevices];
-}  // namespace
-
 // Device address of the current GPU's scratch array.  In host code the array's name only
-// stands for the symbol, so the address is looked up once per device (with that device
-// current) and cached.
+// stands for the symbol, so the address is looked up once per device and context (with that
+// device current) and cached.
 static cudaError_t scratch_address(void **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_scan_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
-    return cudaSuccess;
+    return symbol_address(reinterpret_cast<const void *>(&g_scan_scratch), out);
 }
 
 size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }

@@ -170,13 +170,17 @@ __global__ void __launch_bounds__(NT, 2) gain_scan_tma_kernel(const __grid_const
             dsum[tid] = 0.f;
         }
         if (!mbar_wait(bar_full + st, (uint32_t)((it >> 1) & 1))) abort = true;   // k-th use of a stage: parity k & 1
-        // the next unit's tiles go to the other stage while this one is processed
-        nx = claim();
-        if (nx.u < units) fetch(nx, st ^ 1);
         if (__syncthreads_or(abort)) {
+            // nothing new is issued; the stage that timed out is the only copy that can still be in
+            // flight (the other one was consumed), so give it one more bounded wait before the CTA
+            // exits and its shared memory goes away
+            if (tid == 0) mbar_wait(bar_full + st, (uint32_t)((it >> 1) & 1));
             raise_error(a.err, ERR_TIMEOUT);
             break;
         }
+        // the next unit's tiles go to the other stage while this one is processed
+        nx = claim();
+        if (nx.u < units) fetch(nx, st ^ 1);
         const uint8_t *tile = sm + st * L_::STAGE;
 
         // ---- segment composites of the uncertainty maps (predict [[a, s],[0,1]], update [[1,0],[c,1]])
@@ -353,15 +357,11 @@ cudaError_t launch_gain_scan_tma(const ScanArgs &a, long long ntok, void *worksp
     cudaError_t e = cudaMemsetAsync(ws, 0, scan_tma_workspace_bytes(a.nchains, a.nchunks_max), st);
     if (e != cudaSuccess) return e;
     constexpr size_t smem = ScanTmaSmem::total + 1024;
-    e = cudaFuncSetAttribute(gain_scan_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    KernelSetup ks;
+    e = kernel_setup(reinterpret_cast<const void *>(gain_scan_tma_kernel), smem, NT, true, &ks);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gain_scan_tma_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return e;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     // two CTAs per SM; units go out by ticket to resident CTAs only, so extra CTAs are harmless
-    long long grid = (long long)sms * 2;
+    long long grid = (long long)ks.sms * 2;
     if (grid > units) grid = units;
     gain_scan_tma_kernel<<<(unsigned)grid, NT, smem, st>>>(sa);
     return cudaGetLastError();

@@ -267,3 +267,27 @@ def decode_256x32(seed: int = 2, with_state: bool = True, N: int = 256, H: int =
 
 
 WORKLOADS = {0: tiny_fp32, 1: prefill_4x4096, 2: decode_256x32, 3: long_context_65536, 4: varlen_262144}
+
+
+def decode_inputs_device(seed: int, steps: int, N: int = 256, H: int = 32, d: int = 128, device="cuda"):
+    """The fused-decode workload drawn on a device with a seeded torch generator, for runs too long
+    to draw and copy from the host (1024 steps of 256 x 32 heads are 10.7 GB of bf16 inputs).
+
+    Same distributions as the host workload: S0 ~ N(0, std 0.1) and P0 = softplus(N(0, 1)) in fp32;
+    per step q, k ~ N(0, 1) L2-normalised per (sequence, head), v ~ N(0, 1), alpha = sigmoid(N(4, 1)),
+    r = softplus(N(0, 1)) + 1e-3, sigma = softplus(N(-3, 1)), each rounded to bf16.  Returns a dict:
+    S0 [N, H, d, d], P0 [N, H, d], and q, k, v, alpha, sigma [steps, N, H, d], r [steps, N, H]."""
+    import torch
+    import torch.nn.functional as F
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    rn = lambda *shape: torch.randn(shape, generator=g, device=device)
+    out = {"S0": 0.1 * rn(N, H, d, d), "P0": F.softplus(rn(N, H, d))}
+    shape = (steps, N, H, d)
+    out["q"] = F.normalize(rn(*shape), dim=-1).bfloat16()
+    out["k"] = F.normalize(rn(*shape), dim=-1).bfloat16()
+    out["v"] = rn(*shape).bfloat16()
+    out["alpha"] = torch.sigmoid(rn(*shape) + 4.0).bfloat16()
+    out["r"] = (F.softplus(rn(steps, N, H)) + 1e-3).bfloat16()
+    out["sigma"] = F.softplus(rn(*shape) - 3.0).bfloat16()
+    return out

@@ -27,3 +27,15 @@ def kdn():
     assert torch.cuda.is_available(), "GPU test run without a CUDA device"
     from kalman_delta_rule_b200 import binding
     return binding
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """Write every parity check's achieved error to $KDN_PARITY_LOG (JSON), if set."""
+    path = os.environ.get("KDN_PARITY_LOG")
+    if not path:
+        return
+    import json
+    from tests.kdn_testutil import MARGINS
+    os.makedirs(os.path.dirname(os.path.abspath(path)), exist_ok=True)
+    with open(path, "w") as f:
+        json.dump(MARGINS, f, indent=0)

@@ -1,5 +1,7 @@
 """Helpers shared by the tests: host->device marshalling, the error metric, and
 running the oracle on sampled (sequence, head) chains of a workload."""
+import os
+
 import numpy as np
 
 import oracle
@@ -12,6 +14,20 @@ def max_rel_err(x, y):
     if y.size == 0:
         return 0.0
     return float(np.max(np.abs(x - y)) / max(float(np.max(np.abs(y))), 1e-6))
+
+
+# every parity check's achieved error: (test id, what, error, tolerance); conftest writes them
+# to the JSON file named by $KDN_PARITY_LOG at the end of the session
+MARGINS = []
+
+
+def assert_rel(got, want, tol, what=""):
+    """Assert max_rel_err(got, want) <= tol and record the achieved error."""
+    err = max_rel_err(got, want)
+    test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
+    MARGINS.append({"test": test, "what": str(what), "err": err, "tol": float(tol)})
+    assert err <= tol, f"{what}: max relative error {err:.3e} > {tol:.1e}"
+    return err
 
 
 def to_dev(a, device="cuda"):

@@ -9,7 +9,7 @@ import pytest
 
 from kalman_delta_rule_b200 import inputs
 from oracle import kdn_grad
-from tests.kdn_testutil import dense_shape, max_rel_err, to_dev, to_host
+from tests.kdn_testutil import dense_shape, assert_rel, max_rel_err, to_dev, to_host
 from tests.test_gpu_recurrent import ragged
 
 pytestmark = pytest.mark.gpu
@@ -55,8 +55,7 @@ def run_backward(kdn, w, d_o, S0=None, P0=None, dS=None, dP=None, mu=1.0, iso=Fa
 
 def check(got, ref, tol=TOL):
     for n in NAMES:
-        err = max_rel_err(got[n], ref[n])
-        assert err <= tol, f"{n}: max relative error {err:.3e} > {tol}"
+        assert_rel(got[n], ref[n], tol, n)
 
 
 @pytest.mark.parametrize("mu", [1.0, 32.0])
@@ -147,8 +146,7 @@ def test_backward_full_size_sampled_chains(kdn):
         ref = kdn_grad.diag_grad(pick(w.q), pick(w.k), pick(w.v), pick(w.alpha), pick(w.sigma), w.r[sl, h:h + 1],
                                  d_o[sl, h:h + 1], dS=dS[s:s + 1, h:h + 1], dP=dP[s:s + 1, h:h + 1])
         for n in ("dq", "dk", "dv", "dalpha", "dsigma"):
-            err = max_rel_err(got[n][sl, h], ref[n][:, 0])
-            assert err <= TOL, f"chain ({s},{h}) {n}: {err:.3e}"
-        assert max_rel_err(got["dr"][sl, h], ref["dr"][:, 0]) <= TOL
-        assert max_rel_err(got["dS0"][s, h], ref["dS0"][0, 0]) <= TOL
-        assert max_rel_err(got["dP0"][s, h], ref["dP0"][0, 0]) <= TOL
+            assert_rel(got[n][sl, h], ref[n][:, 0], TOL, f"chain ({s},{h}) {n}")
+        assert_rel(got["dr"][sl, h], ref["dr"][:, 0], TOL, 'got["dr"][sl, h]')
+        assert_rel(got["dS0"][s, h], ref["dS0"][0, 0], TOL, 'got["dS0"][s, h]')
+        assert_rel(got["dP0"][s, h], ref["dP0"][0, 0], TOL, 'got["dP0"][s, h]')

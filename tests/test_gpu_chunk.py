@@ -5,7 +5,7 @@ import pytest
 
 import oracle
 from kalman_delta_rule_b200 import inputs
-from tests.kdn_testutil import max_rel_err
+from tests.kdn_testutil import assert_rel, max_rel_err
 from tests.test_gpu_recurrent import TOL_BF16, TOL_F32, ragged, run_forward
 
 pytestmark = pytest.mark.gpu
@@ -17,9 +17,9 @@ def test_tiny_fp32_chunkwise_matches_oracle(kdn, chunk, mu):
     w = inputs.tiny_fp32()
     ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens, mu=mu)
     o, S, P = run_forward(kdn, w, chunk=chunk, mu=mu)
-    assert max_rel_err(o, ref["o"]) <= TOL_F32
-    assert max_rel_err(S, ref["S"]) <= TOL_F32
-    assert max_rel_err(P, ref["P"]) <= TOL_F32
+    assert_rel(o, ref["o"], TOL_F32, 'o')
+    assert_rel(S, ref["S"], TOL_F32, 'S')
+    assert_rel(P, ref["P"], TOL_F32, 'P')
 
 
 @pytest.mark.parametrize("chunk", [16, 32, 64])
@@ -33,9 +33,9 @@ def test_ragged_varlen_chunkwise(kdn, chunk, dk, dv, bf16):
     ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens, S0=S0, P0=P0, mu=3.0)
     o, S, P = run_forward(kdn, w, chunk=chunk, mu=3.0, S0=S0, P0=P0)
     tol = TOL_BF16 if bf16 else TOL_F32
-    assert max_rel_err(o, ref["o"]) <= tol
-    assert max_rel_err(S, ref["S"]) <= tol
-    assert max_rel_err(P, ref["P"]) <= tol
+    assert_rel(o, ref["o"], tol, 'o')
+    assert_rel(S, ref["S"], tol, 'S')
+    assert_rel(P, ref["P"], tol, 'P')
 
 
 def test_extreme_decays_fp32(kdn):
@@ -51,9 +51,9 @@ def test_extreme_decays_fp32(kdn):
     ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens)
     for chunk in (0, 16, 64):
         o, S, P = run_forward(kdn, w, chunk=chunk)
-        assert max_rel_err(o, ref["o"]) <= TOL_F32, chunk
-        assert max_rel_err(S, ref["S"]) <= TOL_F32, chunk
-        assert max_rel_err(P, ref["P"]) <= TOL_F32, chunk
+        assert_rel(o, ref["o"], TOL_F32, ('o', chunk))
+        assert_rel(S, ref["S"], TOL_F32, ('S', chunk))
+        assert_rel(P, ref["P"], TOL_F32, ('P', chunk))
 
 
 def test_split_sequence_carry_on_gpu(kdn):
@@ -69,6 +69,6 @@ def test_split_sequence_carry_on_gpu(kdn):
                                alpha=w.alpha[lo:hi], sigma=w.sigma[lo:hi], r=w.r[lo:hi])
     o1, S1, P1 = run_forward(kdn, part(0, cut), chunk=64)
     o2, S2, P2 = run_forward(kdn, part(cut, w.ntok), chunk=64, S0=S1, P0=P1)
-    assert max_rel_err(np.concatenate([o1, o2]), full_o) <= TOL_F32
-    assert max_rel_err(S2, full_S) <= TOL_F32
-    assert max_rel_err(P2, full_P) <= TOL_F32
+    assert_rel(np.concatenate([o1, o2]), full_o, TOL_F32, 'np.concatenate([o1, o2])')
+    assert_rel(S2, full_S, TOL_F32, 'S2')
+    assert_rel(P2, full_P, TOL_F32, 'P2')

@@ -5,7 +5,7 @@ import pytest
 
 import oracle
 from kalman_delta_rule_b200 import inputs
-from tests.kdn_testutil import max_rel_err
+from tests.kdn_testutil import assert_rel, max_rel_err
 from tests.test_gpu_recurrent import TOL_F32, run_forward
 
 pytestmark = pytest.mark.gpu
@@ -21,4 +21,4 @@ def test_bounded_waits_report_timeout_and_the_context_survives(kdn):
     w = inputs.tiny_fp32()                        # and the device still computes correctly
     ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens)
     o, S, P = run_forward(kdn, w, chunk=0)
-    assert max_rel_err(o, ref["o"]) <= TOL_F32
+    assert_rel(o, ref["o"], TOL_F32, 'o')

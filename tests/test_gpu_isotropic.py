@@ -6,7 +6,7 @@ import pytest
 
 import oracle
 from kalman_delta_rule_b200 import inputs
-from tests.kdn_testutil import dense_shape, max_rel_err, to_dev, to_host
+from tests.kdn_testutil import dense_shape, assert_rel, max_rel_err, to_dev, to_host
 from tests.test_gpu_recurrent import ragged
 
 pytestmark = pytest.mark.gpu
@@ -16,7 +16,7 @@ TOL_F32, TOL_BF16 = 1e-4, 2e-2
 
 def run_iso(kdn, w, chunk, mu=1.0, S0=None, P0=None, workspace=None):
     """Isotropic forward; ``workspace`` None allocates one (two-launch tensor-core path where
-    it applies), False passes none (the fused tensor-core kernel)."""
+    it applies), False passes none (the fp32 chunk kernel)."""
     import torch
     args = [to_dev(dense_shape(w, getattr(w, n))) for n in ("q", "k", "v", "alpha", "sigma", "r")]
     cu = to_dev(w.cu_seqlens) if w.B == 1 and w.num_seqs > 1 else None
@@ -38,14 +38,14 @@ def test_iso_tiny_fp32_every_chunk(kdn, chunk, mu):
     path, o, S, P = run_iso(kdn, w, chunk, mu=mu)
     assert path == ("recurrent" if chunk == 0 else "chunk_fp32")
     assert P.shape == ref["P"].shape
-    assert max_rel_err(o, ref["o"]) <= TOL_F32
-    assert max_rel_err(S, ref["S"]) <= TOL_F32
-    assert max_rel_err(P, ref["P"]) <= TOL_F32
+    assert_rel(o, ref["o"], TOL_F32, 'o')
+    assert_rel(S, ref["S"], TOL_F32, 'S')
+    assert_rel(P, ref["P"], TOL_F32, 'P')
 
 
 @pytest.mark.parametrize("dk,dv,chunk,form", [(128, 64, 64, "two_phase"), (128, 128, 64, "two_phase"),
-                                              (128, 256, 64, "two_phase"), (128, 128, 64, "fused"),
-                                              (128, 256, 64, "fused"), (64, 128, 64, "two_phase"),
+                                              (128, 256, 64, "two_phase"), (128, 128, 64, "no_workspace"),
+                                              (128, 256, 64, "no_workspace"), (64, 128, 64, "two_phase"),
                                               (128, 128, 0, "two_phase"), (32, 32, 32, "two_phase")])
 def test_iso_ragged_varlen_bf16_with_initial_state(kdn, dk, dv, chunk, form):
     """Ragged sequences (1 token, chunk-1, chunk, chunk+1, several chunks and a tail),
@@ -57,27 +57,27 @@ def test_iso_ragged_varlen_bf16_with_initial_state(kdn, dk, dv, chunk, form):
     ref = oracle.iso_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens, S0=S0, P0=P0, mu=4.0)
     path, o, S, P = run_iso(kdn, w, chunk, mu=4.0, S0=S0, P0=P0, workspace=None if form == "two_phase" else False)
     if chunk == 64 and dk == 128:
-        assert path == ("chunk_tcgen05_two_phase" if form == "two_phase" else "chunk_tcgen05")
-    assert max_rel_err(o, ref["o"]) <= TOL_BF16
-    assert max_rel_err(S, ref["S"]) <= TOL_BF16
-    assert max_rel_err(P, ref["P"]) <= TOL_BF16
+        assert path == ("chunk_tcgen05_two_phase" if form == "two_phase" else "chunk_fp32")
+    assert_rel(o, ref["o"], TOL_BF16, 'o')
+    assert_rel(S, ref["S"], TOL_BF16, 'S')
+    assert_rel(P, ref["P"], TOL_BF16, 'P')
     np.testing.assert_array_equal(P[3], P0[3])      # the empty sequence keeps its uncertainty
 
 
 def test_iso_prefill_full_size_sampled(kdn):
-    """The prefill workload (4 x 4096 tokens, 16 heads, d = 128, bf16) on the tcgen05 path
-    in both forms; sampled chains against the oracle element by element."""
+    """The prefill workload (4 x 4096 tokens, 16 heads, d = 128, bf16) on the tcgen05 path;
+    sampled chains against the oracle element by element."""
     w = inputs.prefill_4x4096()
     ref = oracle.diag_chains(w, [(0, 0), (2, 7), (3, 15)], iso=True)
-    for workspace, name in ((None, "chunk_tcgen05_two_phase"), (False, "chunk_tcgen05")):
+    for workspace, name in ((None, "chunk_tcgen05_two_phase"),):
         path, o, S, P = run_iso(kdn, w, 64, workspace=workspace)
         assert path == name
         o = o.reshape(w.B * w.T, w.H, -1)
         for (s, h), rr in ref.items():
             sl = slice(int(w.cu_seqlens[s]), int(w.cu_seqlens[s + 1]))
-            assert max_rel_err(o[sl, h], rr["o"]) <= TOL_BF16, (name, s, h)
-            assert max_rel_err(S[s, h], rr["S"]) <= TOL_BF16, (name, s, h)
-            assert max_rel_err(P[s, h], rr["P"]) <= TOL_BF16, (name, s, h)
+            assert_rel(o[sl, h], rr["o"], TOL_BF16, ('o[sl, h]', (name, s, h)))
+            assert_rel(S[s, h], rr["S"], TOL_BF16, ('S[s, h]', (name, s, h)))
+            assert_rel(P[s, h], rr["P"], TOL_BF16, ('P[s, h]', (name, s, h)))
 
 
 @pytest.mark.parametrize("n", [1, 5])
@@ -96,9 +96,9 @@ def test_iso_decode_tokens_matches_oracle(kdn, n, dk, dv):
     torch.cuda.synchronize()
     kdn.last_device_error()
     ref = oracle.run_decode(S0, P0, steps, mu=3.0, iso=True)
-    assert max_rel_err(to_host(o).transpose(1, 0, 2, 3), ref["o"]) <= TOL_BF16
-    assert max_rel_err(to_host(S), ref["S"]) <= TOL_BF16
-    assert max_rel_err(to_host(P), ref["P"]) <= TOL_BF16
+    assert_rel(to_host(o).transpose(1, 0, 2, 3), ref["o"], TOL_BF16, 'to_host(o).transpose(1, 0, 2, 3)')
+    assert_rel(to_host(S), ref["S"], TOL_BF16, 'to_host(S)')
+    assert_rel(to_host(P), ref["P"], TOL_BF16, 'to_host(P)')
     if n == 1:   # the single-step wrapper takes the same path
         S2, P2 = to_dev(S0).clone(), to_dev(P0).clone()
         o2 = kdn.decode_step(*[to_dev(steps[0][nm]) for nm in ("q", "k", "v", "alpha", "sigma", "r")], S2, P2,

@@ -5,7 +5,7 @@ import pytest
 
 import oracle
 from kalman_delta_rule_b200 import inputs
-from tests.kdn_testutil import dense_shape, max_rel_err, to_dev, to_host
+from tests.kdn_testutil import dense_shape, assert_rel, max_rel_err, to_dev, to_host
 from tests.test_gpu_recurrent import ragged
 
 pytestmark = pytest.mark.gpu
@@ -28,9 +28,9 @@ def test_scan_tiny_fp32(kdn, mu):
     w = inputs.tiny_fp32()
     ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens, mu=mu, trace=True)
     g, be, P = run_scan(kdn, w, mu=mu)
-    assert max_rel_err(g, ref["trace_g"]) <= TOL[False]
-    assert max_rel_err(be, ref["trace_beta_eff"]) <= TOL[False]
-    assert max_rel_err(P, ref["P"]) <= TOL[False]
+    assert_rel(g, ref["trace_g"], TOL[False], 'g')
+    assert_rel(be, ref["trace_beta_eff"], TOL[False], 'be')
+    assert_rel(P, ref["P"], TOL[False], 'P')
 
 
 @pytest.mark.parametrize("dk", [32, 64, 128])
@@ -44,9 +44,9 @@ def test_scan_ragged_varlen(kdn, dk, bf16):
                               trace=True)
     for ms in (0, max(lens)):
         g, be, P = run_scan(kdn, w, mu=4.0, P0=P0, max_seqlen=ms)
-        assert max_rel_err(g, ref["trace_g"]) <= TOL[bf16]
-        assert max_rel_err(be, ref["trace_beta_eff"]) <= TOL[bf16]
-        assert max_rel_err(P, ref["P"]) <= TOL[bf16]
+        assert_rel(g, ref["trace_g"], TOL[bf16], 'g')
+        assert_rel(be, ref["trace_beta_eff"], TOL[bf16], 'be')
+        assert_rel(P, ref["P"], TOL[bf16], 'P')
 
 
 def test_scan_long_context_full_size_sampled(kdn):
@@ -55,9 +55,9 @@ def test_scan_long_context_full_size_sampled(kdn):
     g, be, P = run_scan(kdn, w)
     ref = oracle.diag_chains(w, [(0, 0), (0, 17)], trace=True)
     for (s, h), rr in ref.items():
-        assert max_rel_err(g[:, h], rr["g"]) <= TOL[True]
-        assert max_rel_err(be[:, h], rr["beta_eff"]) <= TOL[True]
-        assert max_rel_err(P[s, h], rr["P"]) <= TOL[True]
+        assert_rel(g[:, h], rr["g"], TOL[True], 'g[:, h]')
+        assert_rel(be[:, h], rr["beta_eff"], TOL[True], 'be[:, h]')
+        assert_rel(P[s, h], rr["P"], TOL[True], 'P[s, h]')
 
 
 def test_scan_prefill_full_size_sampled(kdn):
@@ -67,9 +67,9 @@ def test_scan_prefill_full_size_sampled(kdn):
     ref = oracle.diag_chains(w, picks, trace=True)
     for (s, h), rr in ref.items():
         sl = slice(int(w.cu_seqlens[s]), int(w.cu_seqlens[s + 1]))
-        assert max_rel_err(g[sl, h], rr["g"]) <= TOL[True]
-        assert max_rel_err(be[sl, h], rr["beta_eff"]) <= TOL[True]
-        assert max_rel_err(P[s, h], rr["P"]) <= TOL[True]
+        assert_rel(g[sl, h], rr["g"], TOL[True], 'g[sl, h]')
+        assert_rel(be[sl, h], rr["beta_eff"], TOL[True], 'be[sl, h]')
+        assert_rel(P[s, h], rr["P"], TOL[True], 'P[s, h]')
 
 
 def test_scan_reports_a_too_small_max_seqlen(kdn):
@@ -97,7 +97,7 @@ def test_information_scaling_weakens_the_effective_write_strength(kdn):
     for mu in (1.0, 128.0):
         g, be, P = run_scan(kdn, w, mu=mu)
         ref = oracle.diag_chains(w, [(0, 3)], mu=mu, trace=True)[(0, 3)]
-        assert max_rel_err(be[:4096, 3], ref["beta_eff"]) <= TOL[True]
+        assert_rel(be[:4096, 3], ref["beta_eff"], TOL[True], 'be[:4096, 3]')
         means[mu] = be
     assert np.all(means[128.0] <= means[1.0] * (1 + 1e-5) + 1e-7)
     assert float(np.mean(means[128.0])) < float(np.mean(means[1.0]))

@@ -1,20 +1,20 @@
-"""GPU parity of the tcgen05 tensor-core chunk path (bf16 inputs, d_k = 128, chunk 64)
-in both its forms -- two launches (chunk-parallel prep, chunk-serial state; with a
-workspace) and one fused kernel (without) -- against the fp64 oracle: ragged tails,
+"""GPU parity of the tcgen05 tensor-core chunk path (bf16 inputs, d_k = 128, chunk 64; two
+launches: chunk-parallel prep, chunk-serial state) against the fp64 oracle: ragged tails,
 varlen, every d_v tile width, initial states, and the full-size workloads on sampled
-(sequence, head) chains."""
+(sequence, head) chains.  The same calls without a workspace take the fp32 chunk kernel and
+are checked too."""
 import numpy as np
 import pytest
 
 import oracle
 from kalman_delta_rule_b200 import inputs
-from tests.kdn_testutil import dense_shape, max_rel_err, oracle_chains, to_dev, to_host
+from tests.kdn_testutil import dense_shape, assert_rel, max_rel_err, oracle_chains, to_dev, to_host
 from tests.test_gpu_recurrent import TOL_BF16, ragged, run_forward
 
 pytestmark = pytest.mark.gpu
 
 
-FORMS = {"two_phase": None, "fused": False}   # workspace argument of run_forward
+FORMS = {"two_phase": None, "no_workspace": False}   # workspace argument of run_forward
 
 
 def path_of(kdn, w, chunk=64):
@@ -33,9 +33,9 @@ def test_tc_dense_ragged_tail(kdn, dv, form):
     assert path_of(kdn, w) == "chunk_tcgen05_two_phase"
     ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens)
     o, S, P = run_forward(kdn, w, chunk=64, workspace=FORMS[form])
-    assert max_rel_err(o, ref["o"]) <= TOL_BF16
-    assert max_rel_err(S, ref["S"]) <= TOL_BF16
-    assert max_rel_err(P, ref["P"]) <= TOL_BF16
+    assert_rel(o, ref["o"], TOL_BF16, 'o')
+    assert_rel(S, ref["S"], TOL_BF16, 'S')
+    assert_rel(P, ref["P"], TOL_BF16, 'P')
 
 
 @pytest.mark.parametrize("H", [20, 80])
@@ -45,9 +45,9 @@ def test_tc_two_phase_wider_dv_tiles(kdn, H):
     w = inputs.dense("tc_tiles", 40 + H, 2, H, 136, 128, 128, bf16=True)   # 136 = 2 chunks + 8
     ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens, mu=2.0)
     o, S, P = run_forward(kdn, w, chunk=64, mu=2.0)
-    assert max_rel_err(o, ref["o"]) <= TOL_BF16
-    assert max_rel_err(S, ref["S"]) <= TOL_BF16
-    assert max_rel_err(P, ref["P"]) <= TOL_BF16
+    assert_rel(o, ref["o"], TOL_BF16, 'o')
+    assert_rel(S, ref["S"], TOL_BF16, 'S')
+    assert_rel(P, ref["P"], TOL_BF16, 'P')
 
 
 @pytest.mark.parametrize("form", sorted(FORMS))
@@ -60,9 +60,9 @@ def test_tc_varlen_with_initial_state(kdn, mu, form):
     P0 = rng.uniform(0.3, 2.0, (w.num_seqs, w.H, 128)).astype(np.float32)
     ref = oracle.diag_forward(w.q, w.k, w.v, w.alpha, w.sigma, w.r, cu_seqlens=w.cu_seqlens, S0=S0, P0=P0, mu=mu)
     o, S, P = run_forward(kdn, w, chunk=64, mu=mu, S0=S0, P0=P0, workspace=FORMS[form])
-    assert max_rel_err(o, ref["o"]) <= TOL_BF16
-    assert max_rel_err(S, ref["S"]) <= TOL_BF16
-    assert max_rel_err(P, ref["P"]) <= TOL_BF16
+    assert_rel(o, ref["o"], TOL_BF16, 'o')
+    assert_rel(S, ref["S"], TOL_BF16, 'S')
+    assert_rel(P, ref["P"], TOL_BF16, 'P')
     np.testing.assert_array_equal(S[3], S0[3])     # the empty sequence passes its state through
     np.testing.assert_array_equal(P[3], P0[3])
 
@@ -74,25 +74,24 @@ def sampled_check(kdn, w, picks, tol=TOL_BF16, forms=("two_phase",)):
         o, S, P = run_forward(kdn, w, chunk=64, workspace=FORMS[form])
         for (s, h), rr in ref.items():
             sl = slice(int(cu[s]), int(cu[s + 1]))
-            assert max_rel_err(o[sl, h], rr["o"]) <= tol, (form, s, h)
-            assert max_rel_err(S[s, h], rr["S"]) <= tol, (form, s, h)
-            assert max_rel_err(P[s, h], rr["P"]) <= tol, (form, s, h)
+            assert_rel(o[sl, h], rr["o"], tol, ('o[sl, h]', (form, s, h)))
+            assert_rel(S[s, h], rr["S"], tol, ('S[s, h]', (form, s, h)))
+            assert_rel(P[s, h], rr["P"], tol, ('P[s, h]', (form, s, h)))
 
 
 def test_prefill_4x4096_full_size_sampled(kdn):
-    """B=4, H=16, T=4096, d=128, bf16, chunk 64 -- the benchmark's launch configuration
-    (both forms)."""
+    """B=4, H=16, T=4096, d=128, bf16, chunk 64 -- the benchmark's launch configuration."""
     w = inputs.prefill_4x4096()
     assert path_of(kdn, w) == "chunk_tcgen05_two_phase"
     rng = np.random.default_rng(1)
     picks = [(0, 0), (3, 15)] + [(int(a), int(b)) for a, b in zip(rng.integers(0, 4, 6), rng.integers(0, 16, 6))]
-    sampled_check(kdn, w, sorted(set(picks)), forms=("two_phase", "fused"))
+    sampled_check(kdn, w, sorted(set(picks)))
 
 
 def test_long_context_65536_full_size_sampled(kdn):
     """B=1, H=32, T=65536 with repeated-key segments; two whole heads checked."""
     w = inputs.long_context_65536()
-    sampled_check(kdn, w, [(0, 0), (0, 31)], forms=("two_phase", "fused"))
+    sampled_check(kdn, w, [(0, 0), (0, 31)])
 
 
 def test_varlen_262144_full_size_sampled(kdn):
