@@ -74,7 +74,8 @@ struct PrepSmem {
     static constexpr uint32_t PST = MUR + 256;         // uncertainty at the chunk start [128]
     static constexpr uint32_t DSUM = PST + 512;        // sum_i P^- k^2 per token [64]
     static constexpr uint32_t TSUM = DSUM + 256;       // isotropic: per-token sums of alpha^2, sigma, k^2 [64][4]
-    static constexpr uint32_t CTL = TSUM + 1024;       // mbarrier, ticket, TMEM slot, look-back flag, abort
+    static constexpr uint32_t HCOMP = TSUM + 1024;     // isotropic: the head map's segment composites [4][4]
+    static constexpr uint32_t CTL = HCOMP + 64;        // mbarrier, ticket, TMEM slot, flags
     static constexpr uint32_t total = CTL + 64;
     // out-of-range units (pairwise decay on the CUDA cores), staged one half of the channels at a time
     static constexpr uint32_t XKQ = 0;                 // (k, q) bf16 pairs [64][XLD], over K~/Q~
@@ -203,6 +204,160 @@ __device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane, int &wh
 }
 }  // namespace
 
+// one token of the uncertainty walk on a key-channel pair's bf16 words (alpha, sigma, k):
+// returns P^- of the pair and advances P (isotropic: the head's map from the token sums)
+template <bool ISO>
+__device__ __forceinline__ f32x2 uncertainty_step(const float *mur, const float *tsum, int t, uint32_t aa,
+                                                  uint32_t ss, uint32_t kk2, float &Pa, float &Pb) {
+    if constexpr (!ISO) {   // both channels of the pair at once (f32x2)
+        const f32x2 al = bf2(aa), kk = bf2(kk2);
+        const f32x2 pm = fma2(mul2(al, al), pk2(Pa, Pb), bf2(ss));
+        const float mr = mur[t];
+        const f32x2 dn = fma2(mul2(mul2(pk2(mr, mr), kk), kk), pm, pk2(1.f, 1.f));
+        Pa = __fdividef(x2(pm), x2(dn));
+        Pb = __fdividef(y2(pm), y2(dn));
+        return pm;
+    } else {   // the head's map, the same on every channel
+        const float4 iso = *reinterpret_cast<const float4 *>(tsum + t * 4);
+        const float pma = fmaf(iso.x, Pa, iso.y), pmb = fmaf(iso.x, Pb, iso.y);
+        Pa = __fdividef(pma, fmaf(iso.z, pma, 1.f));
+        Pb = __fdividef(pmb, fmaf(iso.z, pmb, 1.f));
+        return pk2(pma, pmb);
+    }
+}
+
+// What the out-of-range form of a prep unit needs from the kernel (thread = key-channel pair
+// ch, ch + 1 x 16-token segment sgi starting at token tb of the chunk).
+struct PairwiseCtx {
+    uint8_t *sm;
+    const bf16 *q, *k, *alpha, *sigma;
+    const float *mur, *tsum;
+    float *lsum, *dsum;
+    int tid, warp, ch, tb, sgi, L, c0, h, H;
+    uint32_t atom16, atom8, bch;
+    float Ps_a, Ps_b;   // uncertainty of the pair at the segment start
+};
+
+// A unit whose chunk decay leaves the factored range (some channel's Gam_L < 2^-100: an alpha = 0
+// reset, or strong decay): A and Aq are formed on the CUDA cores with every pairwise decay factor
+// 2^(lg_t - lg_s) <= 1 from log-space sums lg_t = sum log2 max(alpha, 2^-126) (a zero decay acts as
+// 2^-126, so a factor across it is below 2^-126 instead of 0), written fp32 to XAA (rows 0..63 A,
+// 64..127 Aq, before the 1/den column scale); then the operands referenced to the chunk start, K~ =
+// k Gam_t, Q~ = q Gam_t and G' = P^- k 2^(lg_L - lg_t), and the gain denominators' sums.  Kept out
+// of line (rare path): the unit's tokens are re-read from global memory, and its registers do not
+// weigh on the factored path's.
+template <bool ISO>
+__device__ __noinline__ void pairwise_unit(const PairwiseCtx &x) {
+    using L_ = PrepSmem;
+    using namespace tc;
+    const int tid = x.tid, ch = x.ch, tb = x.tb, sgi = x.sgi, L = x.L, c0 = x.c0, h = x.h, H = x.H;
+    auto lg2 = [](float al) { return __log2f(fmaxf(al, 0x1p-126f)); };
+    auto tok = [&](const bf16 *base, int t) { return ldg_u32(base + ((size_t)(c0 + t) * H + h) * DK + ch); };
+    {   // per-segment sums of log2 alpha
+        float la = 0.f, lb = 0.f;
+        for (int j = 0; j < 16; ++j)
+            if (tb + j < L) {
+                const uint32_t aa = tok(x.alpha, tb + j);
+                la += lg2(bf16_lo(aa));
+                lb += lg2(bf16_hi(aa));
+            }
+        x.lsum[sgi * 128 + ch] = la;
+        x.lsum[sgi * 128 + ch + 1] = lb;
+    }
+    __syncthreads();
+    float lga = 0.f, lgb = 0.f, lLa = 0.f, lLb = 0.f;   // at the segment start; over the chunk
+#pragma unroll
+    for (int q2 = 0; q2 < 4; ++q2) {
+        const float xa = x.lsum[q2 * 128 + ch], xb = x.lsum[q2 * 128 + ch + 1];
+        if (q2 < sgi) { lga += xa; lgb += xb; }
+        lLa += xa;
+        lLb += xb;
+    }
+    // A_ts = sum_i k_ti pk_si 2^(lg_ti - lg_si) (s < t), Aq_ts likewise with q (s <= t), one half of
+    // the channels at a time staged as [channel][token]: (k, q) bf16 pairs, P^- k and lg in fp32.
+    // Thread = token row tr x column set {sgc + 4 j}.
+    uint32_t *kqr = reinterpret_cast<uint32_t *>(x.sm + L_::XKQ);
+    float *pks = reinterpret_cast<float *>(x.sm + L_::XPK);
+    float *lgs = reinterpret_cast<float *>(x.sm + L_::XLG);
+    const int tr = tid & 63, sgc = tid >> 6;
+    float accA[16], accQ[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) { accA[j] = 0.f; accQ[j] = 0.f; }
+    for (int half = 0; half < 2; ++half) {
+        if ((x.warp & 1) == half) {   // the owners of this half's channels stage their tokens
+            float Pa = x.Ps_a, Pb = x.Ps_b, lta = lga, ltb = lgb;
+            const int c2 = ch - 64 * half;
+            for (int j = 0; j < 16; ++j) {
+                const int t = tb + j;
+                uint32_t kqa = 0u, kqb = 0u;
+                float pka = 0.f, pkb = 0.f;
+                if (t < L) {
+                    const uint32_t aa = tok(x.alpha, t), kk2 = tok(x.k, t), qq2 = tok(x.q, t);
+                    const f32x2 pm = uncertainty_step<ISO>(x.mur, x.tsum, t, aa, tok(x.sigma, t), kk2, Pa, Pb);
+                    lta += lg2(bf16_lo(aa));
+                    ltb += lg2(bf16_hi(aa));
+                    pka = x2(pm) * bf16_lo(kk2);
+                    pkb = y2(pm) * bf16_hi(kk2);
+                    kqa = (kk2 & 0xffffu) | (qq2 << 16);
+                    kqb = (kk2 >> 16) | (qq2 & 0xffff0000u);
+                }
+                kqr[c2 * XLD + t] = kqa;
+                kqr[(c2 + 1) * XLD + t] = kqb;
+                pks[c2 * XLD + t] = pka;
+                pks[(c2 + 1) * XLD + t] = pkb;
+                lgs[c2 * XLD + t] = lta;
+                lgs[(c2 + 1) * XLD + t] = ltb;
+            }
+        }
+        __syncthreads();
+        if (tid < C) {   // this half's share of the gain denominators sum_i P^-_i k_i^2
+            float acc = 0.f;
+            for (int c2 = 0; c2 < 64; ++c2) acc = fmaf(pks[c2 * XLD + tid], bf16_lo(kqr[c2 * XLD + tid]), acc);
+            x.dsum[tid] += acc;
+        }
+        for (int c2 = 0; c2 < 64; ++c2) {
+            const uint32_t kq = kqr[c2 * XLD + tr];
+            const float kt = bf16_lo(kq), qt = bf16_hi(kq), lt = lgs[c2 * XLD + tr];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int s_ = sgc + 4 * j;
+                if (s_ <= tr) {
+                    const float w = pks[c2 * XLD + s_] * exp2f(lt - lgs[c2 * XLD + s_]);
+                    accA[j] = fmaf(kt, w, accA[j]);
+                    accQ[j] = fmaf(qt, w, accQ[j]);
+                }
+            }
+        }
+        __syncthreads();
+    }
+    float *aaf = reinterpret_cast<float *>(x.sm + L_::XAA);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        aaf[tr * XLD + sgc + 4 * j] = accA[j];
+        aaf[(64 + tr) * XLD + sgc + 4 * j] = accQ[j];
+    }
+    // the operands of the rest of the unit, referenced to the chunk start
+    float Pa = x.Ps_a, Pb = x.Ps_b, lta = lga, ltb = lgb;
+    for (int j = 0; j < 16; ++j) {
+        const int t = tb + j;
+        uint32_t kq = 0u, qq = 0u, gg = 0u;
+        if (t < L) {
+            const uint32_t aa = tok(x.alpha, t), kk2 = tok(x.k, t);
+            const f32x2 pm = uncertainty_step<ISO>(x.mur, x.tsum, t, aa, tok(x.sigma, t), kk2, Pa, Pb);
+            const f32x2 kk = bf2(kk2), qk = bf2(tok(x.q, t));
+            lta += lg2(bf16_lo(aa));
+            ltb += lg2(bf16_hi(aa));
+            const float ga = exp2f(lta), gb = exp2f(ltb);
+            kq = pack_bf16x2(x2(kk) * ga, y2(kk) * gb);
+            qq = pack_bf16x2(x2(qk) * ga, y2(qk) * gb);
+            gg = pack_bf16x2(x2(pm) * x2(kk) * exp2f(lLa - lta), y2(pm) * y2(kk) * exp2f(lLb - ltb));
+        }
+        *reinterpret_cast<uint32_t *>(x.sm + L_::KQ + x.atom16 + swz(t, x.bch)) = kq;
+        *reinterpret_cast<uint32_t *>(x.sm + L_::KQ + x.atom16 + swz(64 + t, x.bch)) = qq;
+        *reinterpret_cast<uint32_t *>(x.sm + L_::G + x.atom8 + swz(t, x.bch)) = gg;
+    }
+}
+
 // ================================================================= prep
 template <bool ISO, bool PACKED>
 __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constant__ PrepArgs pa)
@@ -222,6 +377,7 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
     float *dsum = reinterpret_cast<float *>(sm + L_::DSUM);
     float *tsum = reinterpret_cast<float *>(sm + L_::TSUM);
     float *lsum = reinterpret_cast<float *>(sm + L_::LSUM);
+    float *hcomp = reinterpret_cast<float *>(sm + L_::HCOMP);
     float *comp = reinterpret_cast<float *>(sm + L_::COMP);
     float *adg = reinterpret_cast<float *>(sm + L_::ADG);
     uint64_t *bar_mma = reinterpret_cast<uint64_t *>(sm + L_::CTL);
@@ -242,6 +398,8 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
     const long long units = packed ? pa.U[pa.cmax] : pa.nchunks_max * pa.nchains;
     int level = 0;   // packed: this CTA's chunk level (its tickets only grow)
 
+    // the state kernel (launched next, as a programmatic dependent) may start its prologue
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (tid == 0) {
         mbar_init(bar_mma, 1);
         mbar_fence_init();
@@ -292,6 +450,21 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
         }
     };
 
+    // unit u -> its chunk c, chain, rank among the packed sequences, and the chain's token range
+    auto decode = [&](long long u, int &lvl, int &c, int &chain, int &rank, int &t0, int &t1) {
+        rank = 0;
+        if constexpr (PACKED) {
+            while (lvl < pa.cmax && pa.U[lvl + 1] <= u) ++lvl;
+            c = lvl;
+            const int idx = (int)(u - pa.U[c]);
+            rank = idx / H;
+            chain = pa.order[rank] * H + idx % H;
+        } else {
+            c = (int)(u / pa.nchains);
+            chain = (int)(u % pa.nchains);
+        }
+        seq_range(a, chain / H, t0, t1);
+    };
     for (;;) {
         if (tid == 0) {
             *ticket = (long long)atomicAdd(pa.counter, 1u);
@@ -300,20 +473,9 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
         __syncthreads();
         const long long u = *ticket;
         if (u >= units || ctl[1]) break;
-        int c, chain, rank = 0;
-        if constexpr (PACKED) {
-            while (level < pa.cmax && pa.U[level + 1] <= u) ++level;
-            c = level;
-            const int idx = (int)(u - pa.U[c]);
-            rank = idx / H;
-            chain = pa.order[rank] * H + idx % H;
-        } else {
-            c = (int)(u / pa.nchains);
-            chain = (int)(u % pa.nchains);
-        }
+        int c, chain, rank, t0, t1;
+        decode(u, level, c, chain, rank, t0, t1);
         const int s = chain / H, h = chain % H;
-        int t0, t1;
-        seq_range(a, s, t0, t1);
         const int nch = (t1 - t0 + C - 1) / C;
         if (!packed && c == 0 && tid == 0 && nch > pa.nchunks_max) raise_error(a.err, ERR_ARG);
         if (c >= nch) {
@@ -331,6 +493,7 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
         }
         // thread = key-channel pair cp x 16-token segment sgi; alpha, sigma, k of its tokens
         const int cp = (warp & 1) * 32 + lane, sgi = warp >> 1, ch = cp * 2, tb = sgi * 16;
+        float hexcl[4];   // isotropic, warp 0: the head map composed over the tokens before 2 lane
         uint32_t aw[16], sw[16], kw[16], qw[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -370,7 +533,7 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
                 constexpr float inv_dk = 1.f / DK;
                 const float4 x = *reinterpret_cast<const float4 *>(tsum + tid * 4);
                 *reinterpret_cast<float4 *>(tsum + tid * 4) =
-                    make_float4(x.x * inv_dk, x.y * inv_dk, mur[tid] * x.z * inv_dk, 0.f);
+                    make_float4(x.x * inv_dk, x.y * inv_dk, mur[tid] * x.z * inv_dk, x.z);
             }
             __syncthreads();
         }
@@ -391,33 +554,52 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
             *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch) * 4) = make_float4(x2(m00) * sa, x2(m01) * sa, x2(m10) * sa, x2(gm));
             *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch + 1) * 4) = make_float4(y2(m00) * sbb, y2(m01) * sbb, y2(m10) * sbb, y2(gm));
         } else {
-            float a00 = 1.f, a01 = 0.f, a10 = 0.f, a11 = 1.f, ga = 1.f;
-            float b00 = 1.f, b01 = 0.f, b10 = 0.f, b11 = 1.f, gb = 1.f;
+            // isotropic: the per-channel decay products, and (one thread per segment) the head map's
+            // composite -- the same map on every channel, so it is composed once
+            float ga = 1.f, gb = 1.f;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                if (tb + j < L) {
-                    const float mr = mur[tb + j];
-                    float4 iso = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if constexpr (ISO) iso = *reinterpret_cast<const float4 *>(tsum + (tb + j) * 4);
-                    {
-                        const float al = bf16_lo(aw[j]), kk = bf16_lo(kw[j]);
-                        const float aa = ISO ? iso.x : al * al, sg = ISO ? iso.y : bf16_lo(sw[j]);
-                        const float cc = ISO ? iso.z : mr * kk * kk;
-                        const float y00 = fmaf(aa, a00, sg * a10), y01 = fmaf(aa, a01, sg * a11);
-                        a10 = fmaf(cc, y00, a10); a11 = fmaf(cc, y01, a11); a00 = y00; a01 = y01; ga *= al;
+            for (int j = 0; j < 16; ++j)
+                if (tb + j < L) { ga *= bf16_lo(aw[j]); gb *= bf16_hi(aw[j]); }
+            comp[(sgi * 128 + ch) * 4 + 3] = ga;
+            comp[(sgi * 128 + ch + 1) * 4 + 3] = gb;
+            if (warp == 0) {   // the head map's prefix composites over the chunk: lane l = tokens 2l, 2l + 1
+                // map of token t: x -> (a x + s) / (c (a x + s) + 1), the matrix [[a, s], [c a, c s + 1]]
+                auto tmap = [&](int t, float (&m)[4]) {
+                    if (t < L) {
+                        const float4 iso = *reinterpret_cast<const float4 *>(tsum + t * 4);
+                        m[0] = iso.x; m[1] = iso.y; m[2] = iso.z * iso.x; m[3] = fmaf(iso.z, iso.y, 1.f);
+                    } else {
+                        m[0] = 1.f; m[1] = 0.f; m[2] = 0.f; m[3] = 1.f;
                     }
-                    {
-                        const float al = bf16_hi(aw[j]), kk = bf16_hi(kw[j]);
-                        const float aa = ISO ? iso.x : al * al, sg = ISO ? iso.y : bf16_hi(sw[j]);
-                        const float cc = ISO ? iso.z : mr * kk * kk;
-                        const float y00 = fmaf(aa, b00, sg * b10), y01 = fmaf(aa, b01, sg * b11);
-                        b10 = fmaf(cc, y00, b10); b11 = fmaf(cc, y01, b11); b00 = y00; b01 = y01; gb *= al;
+                };
+                // x <- y after x (2x2 product y x), normalised so that (1,1) = 1
+                auto after = [](float (&x)[4], const float (&y)[4]) {
+                    const float n00 = fmaf(y[0], x[0], y[1] * x[2]), n01 = fmaf(y[0], x[1], y[1] * x[3]);
+                    const float n10 = fmaf(y[2], x[0], y[3] * x[2]), n11 = fmaf(y[2], x[1], y[3] * x[3]);
+                    const float sc = 1.f / n11;
+                    x[0] = n00 * sc; x[1] = n01 * sc; x[2] = n10 * sc; x[3] = 1.f;
+                };
+                float m[4], m1[4];
+                tmap(2 * lane, m);
+                tmap(2 * lane + 1, m1);
+                after(m, m1);   // the lane's two tokens
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {   // inclusive scan over the lanes
+                    float o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o[e] = __shfl_up_sync(0xffffffffu, m[e], off);
+                    if (lane >= off) {
+                        float y[4] = {m[0], m[1], m[2], m[3]};
+                        m[0] = o[0]; m[1] = o[1]; m[2] = o[2]; m[3] = o[3];
+                        after(m, y);   // this lane's part after the earlier lanes'
                     }
                 }
+                // the lane's exclusive prefix (tokens before 2l), kept for the per-token pass below
+#pragma unroll
+                for (int e = 0; e < 4; ++e) hexcl[e] = __shfl_up_sync(0xffffffffu, m[e], 1);
+                if (lane == 0) { hexcl[0] = 1.f; hexcl[1] = 0.f; hexcl[2] = 0.f; hexcl[3] = 1.f; }
+                if (lane == 31) *reinterpret_cast<float4 *>(hcomp) = make_float4(m[0], m[1], m[2], m[3]);
             }
-            const float sa = 1.f / a11, sbb = 1.f / b11;
-            *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch) * 4) = make_float4(a00 * sa, a01 * sa, a10 * sa, ga);
-            *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch + 1) * 4) = make_float4(b00 * sbb, b01 * sbb, b10 * sbb, gb);
         }
         // q of the thread's tokens (consumed after the look-back)
 #pragma unroll
@@ -441,21 +623,28 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
         };
         if (warp < 4) {
             const int cc = tid;   // key channel
-            unsigned long long *desc = pa.desc + (size_t)u * 4 * DK + cc;
-            float g00 = 1.f, g01 = 0.f, g10 = 0.f, g11 = 1.f;
-#pragma unroll
-            for (int q2 = 0; q2 < 4; ++q2) {
-                const float4 cm = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + cc) * 4);
-                const float n00 = fmaf(cm.x, g00, cm.y * g10), n01 = fmaf(cm.x, g01, cm.y * g11);
-                const float n10 = fmaf(cm.z, g00, g10), n11 = fmaf(cm.z, g01, g11);
-                const float sc = 1.f / n11;
-                g00 = n00 * sc; g01 = n01 * sc; g10 = n10 * sc; g11 = 1.f;
-            }
-            {   // the chunk's decay Gam_{L-1} per channel, from the segments' decay products
+            {   // the chunk's decay Gam_L per channel, from the segments' decay products
                 const float gl = comp[cc * 4 + 3] * comp[(128 + cc) * 4 + 3] * comp[(256 + cc) * 4 + 3] *
                                  comp[(384 + cc) * 4 + 3];
                 gamc[cc] = gl;
                 if (!(gl >= kMinChunkDecay)) ctl[2] = 1;
+            }
+        }
+        if (warp < 4 && (!ISO || tid == 0)) {   // isotropic: one uncertainty per head, one walk
+            const int cc = tid;   // key channel
+            unsigned long long *desc = pa.desc + (size_t)u * 4 * DK + cc;
+            float g00 = 1.f, g01 = 0.f, g10 = 0.f, g11 = 1.f;
+            if constexpr (ISO) {   // the whole chunk's head map, from the scan
+                g00 = hcomp[0]; g01 = hcomp[1]; g10 = hcomp[2];
+            } else {
+#pragma unroll
+                for (int q2 = 0; q2 < 4; ++q2) {
+                    const float4 cm = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + cc) * 4);
+                    const float n00 = fmaf(cm.x, g00, cm.y * g10), n01 = fmaf(cm.x, g01, cm.y * g11);
+                    const float n10 = fmaf(cm.z, g00, g10), n11 = fmaf(cm.z, g01, g11);
+                    const float sc = 1.f / n11;
+                    g00 = n00 * sc; g01 = n01 * sc; g10 = n10 * sc; g11 = 1.f;
+                }
             }
             if (c > 0) {   // publish the aggregate
                 st_relaxed(desc + 0 * DK, tagged(g00, TAG_AGG));
@@ -525,38 +714,66 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
         //      sums, and the operands are referenced to the chunk START: K~ = k Gam_t, Q~ = q Gam_t,
         //      G' = P^- k 2^(lg_L - lg_t); every factor is at most 1, so nothing overflows.
         const bool out_of_range = ctl[2] != 0;   // CTA-uniform
-        float Ps_a = pst[ch], Ps_b = pst[ch + 1];   // uncertainty at the segment start
-        for (int q2 = 0; q2 < sgi; ++q2) {
-            const float4 ca = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch) * 4);
-            const float4 cb = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch + 1) * 4);
-            Ps_a = mob(ca.x, ca.y, ca.z, 1.f, Ps_a);
-            Ps_b = mob(cb.x, cb.y, cb.z, 1.f, Ps_b);
-        }
-        // one token of the uncertainty walk on the channel pair's bf16 words (alpha, sigma, k):
-        // returns P^- of the pair and advances P
-        auto predict_update = [&](int t, uint32_t aa, uint32_t ss, uint32_t kk2, float &Pa, float &Pb) -> f32x2 {
-            if constexpr (!ISO) {   // both channels of the pair at once (f32x2)
-                const f32x2 al = bf2(aa), kk = bf2(kk2);
-                const f32x2 pm = fma2(mul2(al, al), pk2(Pa, Pb), bf2(ss));
-                const float mr = mur[t];
-                const f32x2 dn = fma2(mul2(mul2(pk2(mr, mr), kk), kk), pm, pk2(1.f, 1.f));
-                Pa = __fdividef(x2(pm), x2(dn));
-                Pb = __fdividef(y2(pm), y2(dn));
-                return pm;
-            } else {   // the head's map, the same on every channel
-                const float4 iso = *reinterpret_cast<const float4 *>(tsum + t * 4);
-                const float pma = fmaf(iso.x, Pa, iso.y), pmb = fmaf(iso.x, Pb, iso.y);
-                Pa = __fdividef(pma, fmaf(iso.z, pma, 1.f));
-                Pb = __fdividef(pmb, fmaf(iso.z, pmb, 1.f));
-                return pk2(pma, pmb);
+        float Ps_a, Ps_b;   // uncertainty at the segment start
+        if constexpr (ISO) {
+            // warp 0: the head's P^- of every token from the chunk-start uncertainty and the exclusive
+            // prefix maps, the gain denominators r + p^- |k|^2, and the uncertainty after each token
+            float *ppost = lsum;   // [64]
+            if (warp == 0) {
+                float P = mob(hexcl[0], hexcl[1], hexcl[2], hexcl[3], pst[0]);
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int t = 2 * lane + e;
+                    if (t < L) {
+                        const float4 iso = *reinterpret_cast<const float4 *>(tsum + t * 4);
+                        const float pm = fmaf(iso.x, P, iso.y);
+                        P = __fdividef(pm, fmaf(iso.z, pm, 1.f));
+                        dsum[t] = pm;
+                        invden[t] = __fdividef(1.f, fmaf(pm, iso.w, r_s[t]));
+                    } else {
+                        invden[t] = 0.f;
+                    }
+                    ppost[t] = P;
+                }
             }
-        };
+            __syncthreads();
+            Ps_a = sgi == 0 ? pst[0] : ppost[tb - 1];
+            Ps_b = Ps_a;
+        } else {
+            Ps_a = pst[ch];
+            Ps_b = pst[ch + 1];
+            for (int q2 = 0; q2 < sgi; ++q2) {
+                const float4 ca = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch) * 4);
+                const float4 cb = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch + 1) * 4);
+                Ps_a = mob(ca.x, ca.y, ca.z, 1.f, Ps_a);
+                Ps_b = mob(cb.x, cb.y, cb.z, 1.f, Ps_b);
+            }
+        }
         auto store_operands = [&](int t, uint32_t kq, uint32_t qq, uint32_t gg) {
             *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(t, bch)) = kq;
             *reinterpret_cast<uint32_t *>(sm + L_::KQ + atom16 + swz(64 + t, bch)) = qq;
             *reinterpret_cast<uint32_t *>(sm + L_::G + atom8 + swz(t, bch)) = gg;
         };
-        if (!out_of_range) {
+        if (ISO && !out_of_range) {   // P^- of the head per token (dsum) and 1/den are ready
+            float gama, gamb;
+            gamma_start(gama, gamb);
+            f32x2 up = pk2(__fdividef(gama, gamc[ch]), __fdividef(gamb, gamc[ch + 1]));
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int t = tb + j;
+                uint32_t kq = 0u, qq = 0u, gg = 0u;
+                if (t < L) {
+                    const float pm = dsum[t];
+                    const f32x2 kk = bf2(kw[j]);
+                    up = mul2(up, bf2(aw[j]));
+                    const f32x2 kg = mul2(kk, up), qg = mul2(bf2(qw[j]), up);
+                    kq = pack_bf16x2(x2(kg), y2(kg));
+                    qq = pack_bf16x2(x2(qg), y2(qg));
+                    gg = pack_bf16x2(__fdividef(pm * x2(kk), x2(up)), __fdividef(pm * y2(kk), y2(up)));
+                }
+                store_operands(t, kq, qq, gg);
+            }
+        } else if (!out_of_range) {
             float Pa = Ps_a, Pb = Ps_b, gama, gamb;
             gamma_start(gama, gamb);
             // up = Gam_t / Gam_L, in [1, 2^100]: K' = k up, Q' = q up, G' = P^- k / up
@@ -568,7 +785,7 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
                 uint32_t kq = 0u, qq = 0u, gg = 0u;
                 xs[j] = 0.f;
                 if (t < L) {
-                    const f32x2 pm = predict_update(t, aw[j], sw[j], kw[j], Pa, Pb);
+                    const f32x2 pm = uncertainty_step<ISO>(mur, tsum, t, aw[j], sw[j], kw[j], Pa, Pb);
                     const f32x2 kk = bf2(kw[j]);
                     up = mul2(up, bf2(aw[j]));
                     const f32x2 pk = mul2(pm, kk), kg = mul2(kk, up), qg = mul2(bf2(qw[j]), up);
@@ -583,116 +800,15 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
             const float tot = warp_reduce16(xs, lane, which);
             if ((lane & 1) == 0 && tb + which < L) atomicAdd(dsum + tb + which, tot);
         } else {
-            // Rare path: the unit's tokens are re-read from global memory (L2) where needed, so
-            // that the fast path's input registers are dead here.
-            // log2 of the decay, floored at 2^-126 (a zero decay acts as 2^-126: every pairwise
-            // factor across it is then below 2^-126); per-segment sums first
-            auto lg2 = [](float al) { return __log2f(fmaxf(al, 0x1p-126f)); };
-            auto tok = [&](const bf16 *base, int t) { return ldg_u32(base + ((size_t)(c0 + t) * H + h) * DK + ch); };
-            {
-                float la = 0.f, lb = 0.f;
-                for (int j = 0; j < 16; ++j)
-                    if (tb + j < L) {
-                        const uint32_t aa = tok(ain, tb + j);
-                        la += lg2(bf16_lo(aa));
-                        lb += lg2(bf16_hi(aa));
-                    }
-                lsum[sgi * 128 + ch] = la;
-                lsum[sgi * 128 + ch + 1] = lb;
-            }
-            __syncthreads();
-            float lga = 0.f, lgb = 0.f, lLa = 0.f, lLb = 0.f;   // at the segment start; over the chunk
-#pragma unroll
-            for (int q2 = 0; q2 < 4; ++q2) {
-                const float xa = lsum[q2 * 128 + ch], xb = lsum[q2 * 128 + ch + 1];
-                if (q2 < sgi) { lga += xa; lgb += xb; }
-                lLa += xa;
-                lLb += xb;
-            }
-            // A_ts = sum_i k_ti pk_si 2^(lg_ti - lg_si) (s < t), Aq_ts likewise with q (s <= t), one
-            // half of the channels at a time staged as [channel][token]: (k, q) bf16 pairs, P^- k and
-            // lg in fp32.  Thread = token row tr x column set {sgc + 4 j}.
-            uint32_t *kqr = reinterpret_cast<uint32_t *>(sm + L_::XKQ);
-            float *pks = reinterpret_cast<float *>(sm + L_::XPK);
-            float *lgs = reinterpret_cast<float *>(sm + L_::XLG);
-            const int tr = tid & 63, sgc = tid >> 6;
-            float accA[16], accQ[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) { accA[j] = 0.f; accQ[j] = 0.f; }
-            for (int half = 0; half < 2; ++half) {
-                if ((warp & 1) == half) {   // the owners of this half's channels stage their tokens
-                    float Pa = Ps_a, Pb = Ps_b, lta = lga, ltb = lgb;
-                    const int c2 = ch - 64 * half;
-                    for (int j = 0; j < 16; ++j) {
-                        const int t = tb + j;
-                        uint32_t kqa = 0u, kqb = 0u;
-                        float pka = 0.f, pkb = 0.f;
-                        if (t < L) {
-                            const uint32_t aa = tok(ain, t), kk2 = tok(kin, t), qq2 = tok(qin, t);
-                            const f32x2 pm = predict_update(t, aa, tok(sin_, t), kk2, Pa, Pb);
-                            lta += lg2(bf16_lo(aa));
-                            ltb += lg2(bf16_hi(aa));
-                            pka = x2(pm) * bf16_lo(kk2);
-                            pkb = y2(pm) * bf16_hi(kk2);
-                            kqa = (kk2 & 0xffffu) | (qq2 << 16);
-                            kqb = (kk2 >> 16) | (qq2 & 0xffff0000u);
-                        }
-                        kqr[c2 * XLD + t] = kqa;
-                        kqr[(c2 + 1) * XLD + t] = kqb;
-                        pks[c2 * XLD + t] = pka;
-                        pks[(c2 + 1) * XLD + t] = pkb;
-                        lgs[c2 * XLD + t] = lta;
-                        lgs[(c2 + 1) * XLD + t] = ltb;
-                    }
-                }
-                __syncthreads();
-                if (tid < C) {   // this half's share of the gain denominators sum_i P^-_i k_i^2
-                    float acc = 0.f;
-                    for (int c2 = 0; c2 < 64; ++c2) acc = fmaf(pks[c2 * XLD + tid], bf16_lo(kqr[c2 * XLD + tid]), acc);
-                    dsum[tid] += acc;
-                }
-                for (int c2 = 0; c2 < 64; ++c2) {
-                    const uint32_t kq = kqr[c2 * XLD + tr];
-                    const float kt = bf16_lo(kq), qt = bf16_hi(kq), lt = lgs[c2 * XLD + tr];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int s_ = sgc + 4 * j;
-                        if (s_ <= tr) {
-                            const float w = pks[c2 * XLD + s_] * exp2f(lt - lgs[c2 * XLD + s_]);
-                            accA[j] = fmaf(kt, w, accA[j]);
-                            accQ[j] = fmaf(qt, w, accQ[j]);
-                        }
-                    }
-                }
-                __syncthreads();
-            }
-            float *aaf = reinterpret_cast<float *>(sm + L_::XAA);   // rows 0..63 A, 64..127 Aq
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                aaf[tr * XLD + sgc + 4 * j] = accA[j];
-                aaf[(64 + tr) * XLD + sgc + 4 * j] = accQ[j];
-            }
-            // the operands of the rest of the unit, referenced to the chunk start
-            float Pa = Ps_a, Pb = Ps_b, lta = lga, ltb = lgb;
-            for (int j = 0; j < 16; ++j) {
-                const int t = tb + j;
-                uint32_t kq = 0u, qq = 0u, gg = 0u;
-                if (t < L) {
-                    const uint32_t aa = tok(ain, t), kk2 = tok(kin, t);
-                    const f32x2 pm = predict_update(t, aa, tok(sin_, t), kk2, Pa, Pb);
-                    const f32x2 kk = bf2(kk2), qk = bf2(tok(qin, t));
-                    lta += lg2(bf16_lo(aa));
-                    ltb += lg2(bf16_hi(aa));
-                    const float ga = exp2f(lta), gb = exp2f(ltb);
-                    kq = pack_bf16x2(x2(kk) * ga, y2(kk) * gb);
-                    qq = pack_bf16x2(x2(qk) * ga, y2(qk) * gb);
-                    gg = pack_bf16x2(x2(pm) * x2(kk) * exp2f(lLa - lta), y2(pm) * y2(kk) * exp2f(lLb - ltb));
-                }
-                store_operands(t, kq, qq, gg);
-            }
+            PairwiseCtx x;
+            x.sm = sm; x.q = qin; x.k = kin; x.alpha = ain; x.sigma = sin_;
+            x.mur = mur; x.tsum = tsum; x.lsum = lsum; x.dsum = dsum;
+            x.tid = tid; x.warp = warp; x.ch = ch; x.tb = tb; x.sgi = sgi; x.L = L; x.c0 = c0; x.h = h; x.H = H;
+            x.atom16 = atom16; x.atom8 = atom8; x.bch = bch; x.Ps_a = Ps_a; x.Ps_b = Ps_b;
+            pairwise_unit<ISO>(x);
         }
         __syncthreads();
-        if (tid < C) invden[tid] = tid < L ? __fdividef(1.f, r_s[tid] + dsum[tid]) : 0.f;
+        if (tid < C && !(ISO && !out_of_range)) invden[tid] = tid < L ? __fdividef(1.f, r_s[tid] + dsum[tid]) : 0.f;
         sync_tc();
 
         // ---- MMA1 (in range): [A; Aq] = [K'; Q'] G'^T   (M=128, N=64 tokens, K=128 channels)
@@ -969,6 +1085,9 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
         for (int chn = 0; chn < CW / 8; ++chn)
             *reinterpret_cast<uint4 *>(sm + L_::S + atom + swz(row, (((col & 63) >> 3) + chn) * 16)) = pack8(v + chn * 8);
     }
+    // launched as a programmatic dependent of the prep kernel: everything above overlaps the
+    // prep's tail; the records are read only once the whole prep grid has completed
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (tid == 0 && nch > 0) issue(0, 0);
     fence_async_smem();
     tc_fence_before();
@@ -1213,8 +1332,18 @@ static cudaError_t launch_state(const StateArgs &sa, unsigned grid, cudaStream_t
     KernelSetup ks;
     cudaError_t e = kernel_setup(reinterpret_cast<const void *>(kern), smem, SNT, false, &ks);
     if (e != cudaSuccess) return e;
-    kern<<<grid, SNT, smem, st>>>(sa);
-    return cudaGetLastError();
+    // programmatic dependent launch: the CTAs may start while the prep kernel finishes
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(SNT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, sa);
 }
 
 cudaError_t launch_chunk_two_phase(const TokenArgs &a, long long ntok, long long nchunks_max, void *workspace,
