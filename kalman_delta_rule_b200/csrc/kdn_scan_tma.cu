@@ -1,8 +1,8 @@
 // The uncertainty / gain scan for bf16 inputs with d_k = 128: the same single pass with a
 // decoupled look-back as the generic scan (explainer, closing paragraph of "各向同性近似": the
 // uncertainty recursion is a Moebius map whose 2x2 matrices compose), with
-//  - the chunk's alpha, sigma and k tiles fetched by TMA one unit ahead (two stages), so the
-//    loads of the next unit overlap the current one;
+//  - the chunk's alpha, sigma and k tiles fetched by TMA into one stage per CTA, three CTAs per
+//    SM, so the loads of one CTA overlap the arithmetic of the others;
 //  - look-back words that carry their own tag (64-bit (value, tag) per key channel), so a
 //    reader never needs a fence or a flag, and every channel walks back on its own;
 //  - thread = key-channel pair x 16-token segment in the composite and re-expansion passes.
@@ -19,7 +19,7 @@ enum : unsigned { TAG_AGG = 1, TAG_INCL = 2 };
 
 struct ScanTmaSmem {
     static constexpr uint32_t STAGE = 3 * 16384;          // alpha, sigma, k tiles of one chunk
-    static constexpr uint32_t COMP = 2 * STAGE;           // segment composites fp32 [4][128][4]
+    static constexpr uint32_t COMP = STAGE;               // segment composites fp32 [4][128][4]
     static constexpr uint32_t MISC = COMP + 4 * 128 * 16;  // r [64], mu / r [64], P at chunk start [128], sum P^- k^2 [64]
     static constexpr uint32_t CTL = MISC + 1280;           // 2 mbarriers, ticket
     static constexpr uint32_t total = CTL + 64;
@@ -81,7 +81,7 @@ __device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane, int &wh
 }
 }  // namespace
 
-__global__ void __launch_bounds__(NT, 2) gain_scan_tma_kernel(const __grid_constant__ ScanTmaArgs sa)
+__global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_constant__ ScanTmaArgs sa)
 {
     using L_ = ScanTmaSmem;
     using namespace tc;
@@ -155,13 +155,12 @@ __global__ void __launch_bounds__(NT, 2) gain_scan_tma_kernel(const __grid_const
         r_next = (tid < n.L) ? ldf(rin + (size_t)(n.c0 + tid) * H + n.h) : 1.f;
     };
 
-    Unit nx = claim();
-    if (nx.u < units) fetch(nx, 0);
-    bool abort = false;
+    // One stage: a unit's tiles are fetched when the unit is claimed; three CTAs per SM keep the
+    // loads of one CTA under the arithmetic of the others.
     for (int it = 0;; ++it) {
-        const Unit cur = nx;
-        if (cur.u >= units || abort) break;
-        const int st = it & 1;
+        const Unit cur = claim();
+        if (cur.u >= units) break;
+        fetch(cur, 0);
         const long long u = cur.u;
         const int c = cur.c, chain = cur.chain, h = cur.h, c0 = cur.c0, L = cur.L, nch = cur.nch;
         if (tid < C) {
@@ -169,19 +168,15 @@ __global__ void __launch_bounds__(NT, 2) gain_scan_tma_kernel(const __grid_const
             mur[tid] = a.mu / r_next;
             dsum[tid] = 0.f;
         }
-        if (!mbar_wait(bar_full + st, (uint32_t)((it >> 1) & 1))) abort = true;   // k-th use of a stage: parity k & 1
+        const bool abort = !mbar_wait(bar_full, (uint32_t)(it & 1));   // the stage's it-th use: parity it & 1
         if (__syncthreads_or(abort)) {
-            // nothing new is issued; the stage that timed out is the only copy that can still be in
-            // flight (the other one was consumed), so give it one more bounded wait before the CTA
-            // exits and its shared memory goes away
-            if (tid == 0) mbar_wait(bar_full + st, (uint32_t)((it >> 1) & 1));
+            // the copy that timed out is the only one in flight: one more bounded wait for it
+            // before the CTA exits and its shared memory goes away
+            if (tid == 0) mbar_wait(bar_full, (uint32_t)(it & 1));
             raise_error(a.err, ERR_TIMEOUT);
             break;
         }
-        // the next unit's tiles go to the other stage while this one is processed
-        nx = claim();
-        if (nx.u < units) fetch(nx, st ^ 1);
-        const uint8_t *tile = sm + st * L_::STAGE;
+        uint8_t *tile = sm;
 
         // ---- segment composites of the uncertainty maps (predict [[a, s],[0,1]], update [[1,0],[c,1]])
         {
@@ -279,8 +274,8 @@ __global__ void __launch_bounds__(NT, 2) gain_scan_tma_kernel(const __grid_const
         }
         __syncthreads();
 
-        // ---- re-expansion: P^- k per token and channel, the gain denominators, g and k^T g
-        float pk[32];
+        // ---- re-expansion: P^- k per token and channel (written fp32 over the token's alpha and
+        //      sigma words, which only this thread reads), the gain denominators, g and k^T g
         {
             float Pa = pst[ch], Pb = pst[ch + 1];
             for (int q2 = 0; q2 < sgi; ++q2) {
@@ -292,8 +287,6 @@ __global__ void __launch_bounds__(NT, 2) gain_scan_tma_kernel(const __grid_const
             float xs[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                pk[2 * j] = 0.f;
-                pk[2 * j + 1] = 0.f;
                 xs[j] = 0.f;
                 if (tb + j < L) {
                     const uint32_t off = catom + swz(tb + j, bch);
@@ -306,8 +299,8 @@ __global__ void __launch_bounds__(NT, 2) gain_scan_tma_kernel(const __grid_const
                     const float mr = mur[tb + j];
                     Pa = __fdividef(pma, fmaf(mr * ka, pka, 1.f));
                     Pb = __fdividef(pmb, fmaf(mr * kb, pkb, 1.f));
-                    pk[2 * j] = pka;
-                    pk[2 * j + 1] = pkb;
+                    *reinterpret_cast<float *>(tile + off) = pka;
+                    *reinterpret_cast<float *>(tile + 16384 + off) = pkb;
                     xs[j] = fmaf(pka, ka, pkb * kb);
                 }
             }
@@ -328,8 +321,10 @@ __global__ void __launch_bounds__(NT, 2) gain_scan_tma_kernel(const __grid_const
             for (int j = 0; j < 16; ++j) {
                 if (tb + j < L) {
                     const float inv = dsum[tb + j];
+                    const uint32_t off = catom + swz(tb + j, bch);
                     *reinterpret_cast<float2 *>(a.g + ((size_t)(c0 + tb + j) * H + h) * DK + ch) =
-                        make_float2(pk[2 * j] * inv, pk[2 * j + 1] * inv);
+                        make_float2(*reinterpret_cast<const float *>(tile + off) * inv,
+                                    *reinterpret_cast<const float *>(tile + 16384 + off) * inv);
                 }
             }
         }
@@ -360,8 +355,8 @@ cudaError_t launch_gain_scan_tma(const ScanArgs &a, long long ntok, void *worksp
     KernelSetup ks;
     e = kernel_setup(reinterpret_cast<const void *>(gain_scan_tma_kernel), smem, NT, true, &ks);
     if (e != cudaSuccess) return e;
-    // two CTAs per SM; units go out by ticket to resident CTAs only, so extra CTAs are harmless
-    long long grid = (long long)ks.sms * 2;
+    // three CTAs per SM; units go out by ticket to resident CTAs only, so extra CTAs are harmless
+    long long grid = (long long)ks.sms * 3;
     if (grid > units) grid = units;
     gain_scan_tma_kernel<<<(unsigned)grid, NT, smem, st>>>(sa);
     return cudaGetLastError();
