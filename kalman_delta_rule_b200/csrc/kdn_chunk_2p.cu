@@ -870,17 +870,20 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
             }
         }
         __syncthreads();
-        // ---- T = (I + A)^{-1}: D = the two 32x32 diagonal-block inverses (forward substitution,
-        //      thread = one column of one block), N = D L (N^2 = 0), T = (I - N) D
+        // ---- T = (I + A)^{-1}: D = the two 32x32 diagonal-block inverses, each from the inverses
+        //      D1, D2 of its two 16x16 diagonal blocks (forward substitution, thread = one column of
+        //      one 16-block) and its lower-left block -D2 A21 D1 (two 16x16 products on every thread);
+        //      then N = D L (N^2 = 0), T = (I - N) D
         {
-            float x[32];
-            const int b = tid >> 5, j = tid & 31;
             if (tid < 64) {
+                float x[16];
+                const int b16 = tid >> 4, j = tid & 15, o = (b16 & 1) * 16;
+                float *blk = adg + ((b16 >> 1) * 32 + o) * ADS + o;   // the 16-block's first entry
 #pragma unroll
-                for (int r = 0; r < 32; ++r) x[r] = (r == j) ? 1.f : 0.f;
+                for (int r = 0; r < 16; ++r) x[r] = (r == j) ? 1.f : 0.f;
 #pragma unroll
-                for (int r = 1; r < 32; ++r) {   // A's row r is zero from column r on
-                    const float4 *arow = reinterpret_cast<const float4 *>(adg + (b * 32 + r) * ADS);
+                for (int r = 1; r < 16; ++r) {   // A's row r is zero from column r on
+                    const float4 *arow = reinterpret_cast<const float4 *>(blk + r * ADS);
                     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int q4 = 0; q4 < (r + 3) / 4; ++q4) {
@@ -892,11 +895,36 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
                     }
                     if (r > j) x[r] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
                 }
+                __syncwarp();   // the 16-block's rows are read (its columns belong to this warp's half)
+#pragma unroll
+                for (int r = 0; r < 16; ++r) blk[r * ADS + j] = x[r];
             }
             __syncthreads();
-            if (tid < 64) {
+            // Y = A21 D1 (fp32 [2][16][16] in the N tile, written later), then the lower-left block
+            // -D2 Y over A21; thread = two entries (32-block, row, column)
+            float *yt = reinterpret_cast<float *>(sm + L_::NB);
 #pragma unroll
-                for (int r = 0; r < 32; ++r) adg[(b * 32 + r) * ADS + j] = x[r];
+            for (int e = 0; e < 2; ++e) {
+                const int idx = tid * 2 + e, b = idx >> 8, r = (idx >> 4) & 15, cc = idx & 15;
+                const float *a21 = adg + (b * 32 + 16 + r) * ADS, *d1 = adg + (b * 32) * ADS + cc;
+                float acc = 0.f;
+                for (int m = cc; m < 16; ++m) acc = fmaf(a21[m], d1[m * ADS], acc);   // D1 is lower triangular
+                yt[idx] = acc;
+            }
+            __syncthreads();
+            float z[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int idx = tid * 2 + e, b = idx >> 8, r = (idx >> 4) & 15, cc = idx & 15;
+                const float *d2 = adg + (b * 32 + 16 + r) * ADS + 16;
+                float acc = 0.f;
+                for (int m = 0; m <= r; ++m) acc = fmaf(d2[m], yt[(b * 16 + m) * 16 + cc], acc);   // D2 too
+                z[e] = -acc;
+            }
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {   // over A21: every read of it was before the last barrier
+                const int idx = tid * 2 + e, b = idx >> 8, r = (idx >> 4) & 15, cc = idx & 15;
+                adg[(b * 32 + 16 + r) * ADS + cc] = z[e];
             }
             __syncthreads();
             // bf16 D: 64 rows x 8 chunks of 16 B, two chunks per thread
