@@ -21,7 +21,7 @@ struct ScanTmaSmem {
     static constexpr uint32_t STAGE = 3 * 16384;          // alpha, sigma, k tiles of one chunk
     static constexpr uint32_t COMP = STAGE;               // segment composites fp32 [4][128][4]
     static constexpr uint32_t MISC = COMP + 4 * 128 * 16;  // r [64], mu / r [64], P at chunk start [128], sum P^- k^2 [64]
-    static constexpr uint32_t CTL = MISC + 1280;           // 2 mbarriers, ticket
+    static constexpr uint32_t CTL = MISC + 1280;           // 2 mbarriers, the claimed unit
     static constexpr uint32_t total = CTL + 64;
 };
 
@@ -31,6 +31,7 @@ struct ScanTmaArgs {
     unsigned long long *words;   // per unit [4][128]: aggregate (m00, m01, m10), end-of-chunk P
 };
 
+__device__ __forceinline__ f32x2 bf2(uint32_t w) { return pk2(tc::bf16_lo(w), tc::bf16_hi(w)); }
 __device__ __forceinline__ float mob(float m00, float m01, float m10, float m11, float x) {
     return fmaf(m00, x, m01) / fmaf(m10, x, m11);
 }
@@ -95,7 +96,6 @@ __global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_const
     float *pst = mur + 64;
     float *dsum = pst + 128;
     uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + L_::CTL);   // [2]
-    long long *ticket = reinterpret_cast<long long *>(sm + L_::CTL + 16);
 
     const ScanArgs &a = sa.a;
     const bf16 *__restrict__ rin = static_cast<const bf16 *>(a.r);
@@ -116,29 +116,36 @@ __global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_const
     __syncthreads();
 
     struct Unit { long long u; int c, chain, h, c0, L, nch; };
-    // next unit with tokens (all threads; tickets of chunks past a sequence's end are skipped)
+    static_assert(sizeof(Unit) <= 48, "claimed unit slot");
+    Unit *claimed = reinterpret_cast<Unit *>(sm + L_::CTL + 16);
+    // next unit with tokens: thread 0 takes tickets (skipping chunks past a sequence's end) and
+    // decodes the unit once for the block
     auto claim = [&]() -> Unit {
-        Unit n;
-        for (;;) {
-            if (tid == 0) *ticket = (long long)atomicAdd(a.counter, 1u);
-            __syncthreads();
-            n.u = *ticket;
-            __syncthreads();
-            if (n.u >= units) return n;
-            n.c = (int)(n.u / a.nchains);
-            n.chain = (int)(n.u % a.nchains);
-            n.h = n.chain % H;
-            int t0, t1;
-            if (a.cu) { t0 = __ldg(a.cu + n.chain / H); t1 = __ldg(a.cu + n.chain / H + 1); }
-            else { t0 = (n.chain / H) * a.T; t1 = t0 + a.T; }
-            n.nch = (t1 - t0 + C - 1) / C;
-            if (n.c == 0 && tid == 0 && n.nch > a.nchunks_max) raise_error(a.err, ERR_ARG);
-            if (n.c < n.nch) {
-                n.c0 = t0 + n.c * C;
-                n.L = min(C, t1 - n.c0);
-                return n;
+        if (tid == 0) {
+            Unit n;
+            for (;;) {
+                n.u = (long long)atomicAdd(a.counter, 1u);
+                if (n.u >= units) break;
+                const unsigned uu = (unsigned)n.u, nc = (unsigned)a.nchains;
+                n.c = (int)(uu / nc);
+                n.chain = (int)(uu - (unsigned)n.c * nc);
+                const int s = n.chain / H;
+                n.h = n.chain - s * H;
+                int t0, t1;
+                if (a.cu) { t0 = __ldg(a.cu + s); t1 = __ldg(a.cu + s + 1); }
+                else { t0 = s * a.T; t1 = t0 + a.T; }
+                n.nch = (t1 - t0 + C - 1) / C;
+                if (n.c == 0 && n.nch > a.nchunks_max) raise_error(a.err, ERR_ARG);
+                if (n.c < n.nch) {
+                    n.c0 = t0 + n.c * C;
+                    n.L = min(C, t1 - n.c0);
+                    break;
+                }
             }
+            *claimed = n;
         }
+        __syncthreads();
+        return *claimed;
     };
     // the unit's tiles into stage st (thread 0), its r into r_next (threads < 64)
     float r_next = 1.f;
@@ -178,35 +185,32 @@ __global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_const
         }
         uint8_t *tile = sm;
 
-        // ---- segment composites of the uncertainty maps (predict [[a, s],[0,1]], update [[1,0],[c,1]])
+        // ---- segment composites of the uncertainty maps (predict [[a, s],[0,1]], update [[1,0],[c,1]]);
+        //      channels ch and ch + 1 in the two lanes of packed f32x2 arithmetic
         {
-            float a00 = 1.f, a01 = 0.f, a10 = 0.f, a11 = 1.f, ga = 1.f;
-            float b00 = 1.f, b01 = 0.f, b10 = 0.f, b11 = 1.f, gb = 1.f;
+            f32x2 m00 = pk2(1.f, 1.f), m01 = pk2(0.f, 0.f), m10 = m01, m11 = m00, gm = m00;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 if (tb + j < L) {
                     const uint32_t off = catom + swz(tb + j, bch);
-                    const uint32_t aw = *reinterpret_cast<const uint32_t *>(tile + off);
-                    const uint32_t sw = *reinterpret_cast<const uint32_t *>(tile + 16384 + off);
-                    const uint32_t kw = *reinterpret_cast<const uint32_t *>(tile + 32768 + off);
+                    const f32x2 al = bf2(*reinterpret_cast<const uint32_t *>(tile + off));
+                    const f32x2 sg = bf2(*reinterpret_cast<const uint32_t *>(tile + 16384 + off));
+                    const f32x2 kk = bf2(*reinterpret_cast<const uint32_t *>(tile + 32768 + off));
                     const float mr = mur[tb + j];
-                    {
-                        const float al = bf16_lo(aw), sg = bf16_lo(sw), kk = bf16_lo(kw);
-                        const float aa = al * al, cc = mr * kk * kk;
-                        const float y00 = fmaf(aa, a00, sg * a10), y01 = fmaf(aa, a01, sg * a11);
-                        a10 = fmaf(cc, y00, a10); a11 = fmaf(cc, y01, a11); a00 = y00; a01 = y01; ga *= al;
-                    }
-                    {
-                        const float al = bf16_hi(aw), sg = bf16_hi(sw), kk = bf16_hi(kw);
-                        const float aa = al * al, cc = mr * kk * kk;
-                        const float y00 = fmaf(aa, b00, sg * b10), y01 = fmaf(aa, b01, sg * b11);
-                        b10 = fmaf(cc, y00, b10); b11 = fmaf(cc, y01, b11); b00 = y00; b01 = y01; gb *= al;
-                    }
+                    const f32x2 aa = mul2(al, al), cc = mul2(mul2(pk2(mr, mr), kk), kk);
+                    const f32x2 y00 = fma2(aa, m00, mul2(sg, m10)), y01 = fma2(aa, m01, mul2(sg, m11));
+                    m10 = fma2(cc, y00, m10);
+                    m11 = fma2(cc, y01, m11);
+                    m00 = y00;
+                    m01 = y01;
+                    gm = mul2(gm, al);
                 }
             }
-            const float sa_ = 1.f / a11, sb_ = 1.f / b11;
-            *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch) * 4) = make_float4(a00 * sa_, a01 * sa_, a10 * sa_, ga);
-            *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch + 1) * 4) = make_float4(b00 * sb_, b01 * sb_, b10 * sb_, gb);
+            const float sa_ = 1.f / x2(m11), sb_ = 1.f / y2(m11);
+            *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch) * 4) =
+                make_float4(x2(m00) * sa_, x2(m01) * sa_, x2(m10) * sa_, x2(gm));
+            *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch + 1) * 4) =
+                make_float4(y2(m00) * sb_, y2(m01) * sb_, y2(m10) * sb_, y2(gm));
         }
         __syncthreads();
 
@@ -290,18 +294,18 @@ __global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_const
                 xs[j] = 0.f;
                 if (tb + j < L) {
                     const uint32_t off = catom + swz(tb + j, bch);
-                    const uint32_t aw = *reinterpret_cast<const uint32_t *>(tile + off);
-                    const uint32_t sw = *reinterpret_cast<const uint32_t *>(tile + 16384 + off);
-                    const uint32_t kw = *reinterpret_cast<const uint32_t *>(tile + 32768 + off);
-                    const float ala = bf16_lo(aw), alb = bf16_hi(aw), ka = bf16_lo(kw), kb = bf16_hi(kw);
-                    const float pma = fmaf(ala * ala, Pa, bf16_lo(sw)), pmb = fmaf(alb * alb, Pb, bf16_hi(sw));
-                    const float pka = pma * ka, pkb = pmb * kb;
+                    const f32x2 al = bf2(*reinterpret_cast<const uint32_t *>(tile + off));
+                    const f32x2 sg = bf2(*reinterpret_cast<const uint32_t *>(tile + 16384 + off));
+                    const f32x2 kk = bf2(*reinterpret_cast<const uint32_t *>(tile + 32768 + off));
                     const float mr = mur[tb + j];
-                    Pa = __fdividef(pma, fmaf(mr * ka, pka, 1.f));
-                    Pb = __fdividef(pmb, fmaf(mr * kb, pkb, 1.f));
-                    *reinterpret_cast<float *>(tile + off) = pka;
-                    *reinterpret_cast<float *>(tile + 16384 + off) = pkb;
-                    xs[j] = fmaf(pka, ka, pkb * kb);
+                    const f32x2 pm = fma2(mul2(al, al), pk2(Pa, Pb), sg);
+                    const f32x2 pk = mul2(pm, kk);
+                    const f32x2 dn = fma2(mul2(pk2(mr, mr), kk), pk, pk2(1.f, 1.f));
+                    Pa = __fdividef(x2(pm), x2(dn));
+                    Pb = __fdividef(y2(pm), y2(dn));
+                    *reinterpret_cast<float *>(tile + off) = x2(pk);
+                    *reinterpret_cast<float *>(tile + 16384 + off) = y2(pk);
+                    xs[j] = fmaf(x2(pk), x2(kk), y2(pk) * y2(kk));
                 }
             }
             int which;
