@@ -212,11 +212,11 @@ kdn_status_t kdn_gain_scan_noalloc(const kdn_problem_t *p,
  *  workspace          : device, >= kdn_backward_workspace_size() bytes, 256-byte aligned
  *                       (contents on entry do not matter; distinct per concurrent call).
  * Method: the uncertainty forward is taped (P before each token, den, g), the memory forward
- * is checkpointed every 32 tokens, and the reverse sweep recomputes each chunk from its
+ * is checkpointed every 16 tokens, and the reverse sweep recomputes each chunk from its
  * checkpoint (the state before every token is re-stepped forward, never reconstructed by
  * dividing by alpha); fp32 CUDA-core arithmetic.  The d_v column blocks of a (sequence, head)
  * add their shares of the sums over d_v with atomic adds, so the last bits of every gradient
- * except dv and dS0 can differ from run to run.  Workspace: about 5.1 KB per token and head
+ * except dv and dS0 can differ from run to run.  Workspace: about 7.0 KB per token and head
  * at d_k = d_v = 128.  Every pointer 16-byte aligned.  Outputs may not alias inputs.
  * Asynchronous on `stream`; errors as for the forward. */
 kdn_status_t kdn_backward_workspace_size(const kdn_problem_t *p, size_t *bytes);

@@ -252,7 +252,8 @@ kdn_status_t kdn_backward(const kdn_problem_t *p, const void *q, const void *k, 
     a.mu = p->mu; a.iso = p->variant == KDN_VARIANT_ISOTROPIC; a.err = err_word();
     b.d_o = d_o; b.dS_T = dS_T; b.dP_T = dP_T;
     b.dq = dq; b.dk = dk; b.dv = dv; b.dalpha = dalpha; b.dsigma = dsigma; b.dr = dr; b.dS0 = dS0; b.dP0 = dP0;
-    return cuda_status(kdn::launch_backward(b, rv.bf16, rv.ntok, workspace, static_cast<cudaStream_t>(stream)));
+    return cuda_status(kdn::launch_backward(b, rv.bf16, rv.ntok, rv.nchunks_max, workspace,
+                                            static_cast<cudaStream_t>(stream)));
 }
 
 kdn_status_t kdn_selftest_bounded_wait(long long limit_cycles, void *stream) {

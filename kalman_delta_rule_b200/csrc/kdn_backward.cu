@@ -17,7 +17,7 @@
 //   tape  (one CTA per (sequence, head), thread = key channel): the uncertainty forward; writes
 //         P before each token, den and g per token;
 //   state (one CTA per (sequence, head, 16-column block of d_v), thread = key channel = row of S):
-//         the memory forward with S checkpoints every 32 tokens and u of every token taped, then
+//         the memory forward with S checkpoints every 16 tokens and u of every token taped, then
 //         the reverse sweep chunk by chunk: the chunk's inputs are staged in shared memory, the
 //         chunk is re-stepped from its checkpoint (with the taped u, so without the cross-row
 //         reduction) into shared-memory sub-checkpoints every 4 tokens, and the
@@ -41,7 +41,7 @@ namespace kdn {
 
 namespace {
 constexpr int DB = 16;    // d_v columns per state CTA
-constexpr int CK = 32;    // tokens between the DRAM checkpoints of S
+constexpr int CK = 16;    // tokens between the DRAM checkpoints of S (four CTAs per SM fit)
 constexpr int NS = 4;     // tokens between the shared-memory sub-checkpoints
 constexpr int GT = 32;    // tokens per group in the uncertainty kernels
 
@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(128) bwd_tape_kernel(const BwdArgs b, const Bw
 // [CK/NS][DB/4][dk] float4; u per token [CK][DB]; reduction partials [4][DB]; u^ [DB]; then alpha, k, q
 // rows [CK][dk] and the column block of v (forward) or d_o (reverse) [CK][DB] in the input type
 template <typename T>
-__global__ void __launch_bounds__(128, 2) bwd_state_kernel(const BwdArgs b, const BwdWs w)
+__global__ void __launch_bounds__(128, 4) bwd_state_kernel(const BwdArgs b, const BwdWs w)
 {
     extern __shared__ float smf[];
     const TokenArgs &a = b.a;
@@ -700,14 +700,35 @@ static cudaError_t launch_local(const BwdArgs &b, const BwdWs &w, cudaStream_t s
 // the kernel's dynamic shared-memory limit, set once per device and context
 static cudaError_t set_smem(const void *kern, size_t smem) {
     KernelSetup ks;
-    return kernel_setup(kern, smem, 128, false, &ks);
+    return kernel_setup(kern, smem, 128, true, &ks);
+}
+
+// The uncertainty forward as the chunk-parallel gain scan (bf16, d_k = 128, diagonal): P before
+// each token, g and den, with its look-back words in the checkpoint region (written by the
+// state pass only later); then the four sums the state pass adds into are cleared.
+static cudaError_t launch_tape_scan(const BwdArgs &b, const BwdWs &w, int nchunks_max, cudaStream_t st) {
+    const TokenArgs &a = b.a;
+    ScanArgs sa{};
+    sa.k = a.k; sa.alpha = a.alpha; sa.sigma = a.sigma; sa.r = a.r; sa.P0 = a.P0;
+    sa.g = w.g; sa.P_prev = w.Pprev; sa.den = w.den;
+    sa.cu = a.cu; sa.T = a.T; sa.nseq = a.nseq; sa.H = a.H; sa.dk = a.dk; sa.mu = a.mu;
+    sa.nchunks_max = nchunks_max; sa.nchains = a.nseq * a.H; sa.err = a.err;
+    const size_t th = (size_t)w.ntok * a.H;
+    cudaError_t e = cudaMemsetAsync(b.dq, 0, th * a.dk * 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(w.part, 0, 3 * th * a.dk * 4, st);
+    if (e != cudaSuccess) return e;
+    return launch_gain_scan_tma(sa, w.ntok, w.ckpt, st);
 }
 
 template <typename T>
-static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, cudaStream_t st) {
+static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, bool tape_scan, int nchunks_max,
+                                    cudaStream_t st) {
     const int chains = b.a.nseq * b.a.H, dk = b.a.dk;
     cudaError_t e;
-    if (b.a.iso) {
+    if (tape_scan) {
+        e = launch_tape_scan(b, w, nchunks_max, st);
+        if (e != cudaSuccess) return e;
+    } else if (b.a.iso) {
         const size_t tsm = (size_t)7 * GT * sizeof(float) + (size_t)3 * GT * dk * sizeof(T);
         e = set_smem(reinterpret_cast<const void *>(bwd_tape_iso_kernel<T>), tsm);
         if (e != cudaSuccess) return e;
@@ -743,7 +764,8 @@ static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, cudaStream
     return cudaGetLastError();
 }
 
-cudaError_t launch_backward(const BwdArgs &b, bool bf16_in, long long ntok, void *workspace, cudaStream_t st) {
+cudaError_t launch_backward(const BwdArgs &b, bool bf16_in, long long ntok, long long nchunks_max, void *workspace,
+                            cudaStream_t st) {
     const TokenArgs &a = b.a;
     const size_t th = (size_t)ntok * a.H;
     uint8_t *p = static_cast<uint8_t *>(workspace);
@@ -755,9 +777,15 @@ cudaError_t launch_backward(const BwdArgs &b, bool bf16_in, long long ntok, void
     w.den = reinterpret_cast<float *>(p); p += align256(th * 4);
     w.dden = reinterpret_cast<float *>(p); p += align256(th * 4);
     w.utape = reinterpret_cast<float *>(p); p += align256(th * a.dv * 4);
-    w.ckpt = reinterpret_cast<float *>(p); p += align256((size_t)ckpt_slots(ntok, a.nseq) * a.H * a.dk * a.dv * 4);
+    const size_t ckpt_bytes = (size_t)ckpt_slots(ntok, a.nseq) * a.H * a.dk * a.dv * 4;
+    w.ckpt = reinterpret_cast<float *>(p); p += align256(ckpt_bytes);
     w.part = reinterpret_cast<float *>(p);
-    return bf16_in ? launch_bwd_typed<bf16>(b, w, st) : launch_bwd_typed<float>(b, w, st);
+    // the scan's look-back words must fit the checkpoint region (they may not for packed
+    // sequences of very different lengths, whose work list is nseq x H x the longest's chunks)
+    const bool tape_scan = !a.iso && ntok > 0 && gain_scan_tma_supported(a.dk, bf16_in) &&
+                           scan_tma_workspace_bytes((long long)a.nseq * a.H, nchunks_max) <= ckpt_bytes;
+    const int ncm = (int)(nchunks_max < (1ll << 30) ? nchunks_max : (1ll << 30));
+    return bf16_in ? launch_bwd_typed<bf16>(b, w, tape_scan, ncm, st) : launch_bwd_typed<float>(b, w, tape_scan, ncm, st);
 }
 
 }  // namespace kdn

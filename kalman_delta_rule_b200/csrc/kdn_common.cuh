@@ -90,6 +90,8 @@ struct ScanArgs {
     const void *k, *alpha, *sigma, *r;          // [ntok, H, dk] / [ntok, H]
     const float *P0;                            // [N, H, dk] or NULL (ones)
     float *g, *beta, *P_out;                    // [ntok, H, dk], [ntok, H], [N, H, dk]; each may be NULL
+    float *P_prev, *den;                        // [ntok, H, dk], [ntok, H]: P before each token and the gain
+                                                // denominator (the backward's tape); NULL = not written
     const int32_t *cu;                          // device [N+1] or NULL
     int T, nseq, H, dk;
     float mu;

@@ -49,7 +49,8 @@ struct BwdArgs {
     float *dS0, *dP0;                            // may be NULL
 };
 size_t backward_workspace_bytes(long long ntok, int nseq, int H, int dk, int dv);
-cudaError_t launch_backward(const BwdArgs &b, bool bf16_in, long long ntok, void *workspace, cudaStream_t st);
+cudaError_t launch_backward(const BwdArgs &b, bool bf16_in, long long ntok, long long nchunks_max, void *workspace,
+                            cudaStream_t st);
 
 // failure-detection self-test: bounded waits that run out and record ERR_TIMEOUT
 cudaError_t launch_bounded_wait_selftest(long long limit_cycles, unsigned *err, cudaStream_t st);

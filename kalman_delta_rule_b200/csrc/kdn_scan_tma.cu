@@ -6,7 +6,8 @@
 //  - look-back words that carry their own tag (64-bit (value, tag) per key channel), so a
 //    reader never needs a fence or a flag, and every channel walks back on its own;
 //  - thread = key-channel pair x 16-token segment in the composite and re-expansion passes.
-// Outputs: g_t = P^-_t k_t / den_t (fp32), k_t^T g_t, and the uncertainty after each sequence.
+// Outputs: g_t = P^-_t k_t / den_t (fp32), k_t^T g_t, and the uncertainty after each sequence;
+// for the backward also P before each token and den_t.
 #include "kdn_common.cuh"
 #include "kdn_launch.h"
 #include "kdn_tc.cuh"
@@ -298,6 +299,9 @@ __global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_const
                     const f32x2 sg = bf2(*reinterpret_cast<const uint32_t *>(tile + 16384 + off));
                     const f32x2 kk = bf2(*reinterpret_cast<const uint32_t *>(tile + 32768 + off));
                     const float mr = mur[tb + j];
+                    if (a.P_prev)
+                        *reinterpret_cast<float2 *>(a.P_prev + ((size_t)(c0 + tb + j) * H + h) * DK + ch) =
+                            make_float2(Pa, Pb);
                     const f32x2 pm = fma2(mul2(al, al), pk2(Pa, Pb), sg);
                     const f32x2 pk = mul2(pm, kk);
                     const f32x2 dn = fma2(mul2(pk2(mr, mr), kk), pk, pk2(1.f, 1.f));
@@ -315,8 +319,9 @@ __global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_const
         __syncthreads();
         if (tid < C && tid < L) {
             const float x = dsum[tid];
-            const float inv = 1.f / (r_s[tid] + x);
+            const float dn = r_s[tid] + x, inv = 1.f / dn;
             dsum[tid] = inv;
+            if (a.den) a.den[(size_t)(c0 + tid) * H + h] = dn;
             if (a.beta) a.beta[(size_t)(c0 + tid) * H + h] = x * inv;
         }
         __syncthreads();

@@ -120,10 +120,10 @@ def test_forward_rejects_bad_pointers(lib):
 def test_backward_validates_before_any_cuda_call(lib):
     p = problem(chunk=64)
     need = B.kdn_backward_workspace_size(p)
-    # P tape, g, den, den^, u tape, S checkpoints every 32 tokens and the sums of g^, k^_S, alpha^_S
+    # P tape, g, den, den^, u tape, S checkpoints every 16 tokens and the sums of g^, k^_S, alpha^_S
     ntok, H, dk, dv = 2 * 128, 4, 128, 128
-    assert need >= 4 * (2 * ntok * H * dk + 2 * ntok * H + ntok * H * dv + (ntok // 32 + 2 + 1) * H * dk * dv + 3 * ntok * H * dk)
-    assert need < 4 * (2 * ntok * H * dk + 2 * ntok * H + ntok * H * dv + (ntok // 32 + 2 + 1) * H * dk * dv + 3 * ntok * H * dk) + 7 * 256
+    assert need >= 4 * (2 * ntok * H * dk + 2 * ntok * H + ntok * H * dv + (ntok // 16 + 2 + 1) * H * dk * dv + 3 * ntok * H * dk)
+    assert need < 4 * (2 * ntok * H * dk + 2 * ntok * H + ntok * H * dv + (ntok // 16 + 2 + 1) * H * dk * dv + 3 * ntok * H * dk) + 7 * 256
     ins = [FAKE] * 6                 # q, k, v, alpha, sigma, r
     outs = [FAKE + 4096 * (i + 1) for i in range(6)]   # dq, dk, dv, dalpha, dsigma, dr
     args = lambda d_o=FAKE, o=outs, ws=FAKE, wb=need: [p, *ins, None, None, d_o, None, None, *o, None, None, ws, wb, None]
