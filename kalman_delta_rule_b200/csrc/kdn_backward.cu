@@ -487,6 +487,175 @@ __global__ void __launch_bounds__(128) bwd_prev_kernel(const BwdArgs b, const Bw
     if (b.dP0) b.dP0[(size_t)chain * dk + i] = Ph;
 }
 
+// ================================================================= prev, chunk-parallel
+// The serial part of the uncertainty adjoint, P^ <- alpha^2 (P^-^local + P^ z^2), is affine in P^
+// per key channel (P^_before = a P^_after + b, a = alpha^2 z^2, b = alpha^2 P^-^local), so it is
+// scanned like the forward uncertainty, over chunks of PC tokens counted from the sequence end:
+// a unit (chunk, chain) composes its chunk's maps (thread = key channel), publishes the
+// aggregate as tagged 64-bit words, walks over the later chunks' words to the last published
+// chunk-start value (decoupled look-back, bounded waits), publishes its own, and walks its
+// tokens again with the incoming P^ to write dk, dsigma, dalpha and dr.  Tickets go out
+// chunk-major in that order, so every unit a look-back waits for was taken earlier by a running
+// CTA.  A sequence without tokens gets one empty unit, which passes dP_T through to dP0.
+namespace {
+constexpr int PC = 64;
+enum : unsigned { TAG_AGG = 1, TAG_INCL = 2 };
+struct PrevWs {
+    unsigned *counter;
+    unsigned long long *words;   // per unit [3][dk]: aggregate (a, b), chunk-start P^
+    long long nchunks_max;
+};
+__device__ __forceinline__ unsigned long long tagged(float x, unsigned tag) {
+    return ((unsigned long long)tag << 32) | __float_as_uint(x);
+}
+__device__ __forceinline__ unsigned tag_of(unsigned long long v) { return (unsigned)(v >> 32); }
+__device__ __forceinline__ float value_of(unsigned long long v) { return __uint_as_float((unsigned)v); }
+__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+struct PrevUnit { long long u; int j, chain, h, lo, hi, nch; };
+}  // namespace
+
+// dynamic shared memory: dr terms [PC][dk]; 1/r, den^ [PC]; the claimed unit
+template <typename T>
+__global__ void __launch_bounds__(128) bwd_prev_scan_kernel(const BwdArgs b, const BwdWs w, const PrevWs pw)
+{
+    extern __shared__ float smf[];
+    const TokenArgs &a = b.a;
+    const int dk = a.dk, H = a.H;
+    float *x_s = smf, *ir_s = x_s + PC * dk, *dd_s = ir_s + PC;
+    PrevUnit *claimed = reinterpret_cast<PrevUnit *>(dd_s + PC);
+    const T *alpha = static_cast<const T *>(a.alpha), *sigma = static_cast<const T *>(a.sigma);
+    const T *k = static_cast<const T *>(a.k), *r = static_cast<const T *>(a.r);
+    const int i = threadIdx.x, warp = i >> 5, lane = i & 31, nw = dk >> 5;
+    const float mu = a.mu;
+    const size_t tokstride = (size_t)w.ntok * H * dk;
+    const int nchains = a.nseq * H;
+    const long long units = pw.nchunks_max * nchains;
+    for (;;) {
+        if (i == 0) {
+            PrevUnit n;
+            for (;;) {
+                n.u = (long long)atomicAdd(pw.counter, 1u);
+                if (n.u >= units) break;
+                n.j = (int)(n.u / nchains);
+                n.chain = (int)(n.u - (long long)n.j * nchains);
+                const int s = n.chain / H;
+                n.h = n.chain - s * H;
+                int t0, t1;
+                seq_range(a, s, t0, t1);
+                n.nch = (t1 - t0 + PC - 1) / PC;
+                if (n.j < n.nch || n.j == 0) {
+                    n.hi = t1 - n.j * PC;
+                    n.lo = max(t0, n.hi - PC);
+                    break;
+                }
+            }
+            *claimed = n;
+        }
+        __syncthreads();
+        const PrevUnit cu = *claimed;
+        if (cu.u >= units) break;
+        const int L = cu.hi - cu.lo;
+        for (int tt = i; tt < L; tt += dk) {
+            const size_t th = (size_t)(cu.lo + tt) * H + cu.h;
+            ir_s[tt] = 1.f / ldf(r + th);
+            dd_s[tt] = w.dden[th];
+        }
+        __syncthreads();
+
+        // pass 1: the chunk's composite map, P^ at the chunk start = ra P^_end + rb
+        float ra = 1.f, rb = 0.f;
+#pragma unroll 4
+        for (int tt = L - 1; tt >= 0; --tt) {
+            const size_t e = ((size_t)(cu.lo + tt) * H + cu.h) * dk + i;
+            const float al = ldf(alpha + e), kk = ldf(k + e);
+            const float pm = fmaf(al * al, w.Pprev[e], ldf(sigma + e));
+            const float mk = mu * kk * ir_s[tt];
+            const float z = 1.f / fmaf(mk * kk, pm, 1.f);
+            const float aa = al * al, at = aa * z * z;
+            rb = fmaf(at, rb, aa * w.part[e]);
+            ra *= at;
+        }
+
+        // the incoming P^ at the chunk end: dP_T for the last chunk, else the later chunks' words.
+        // The last chunk publishes no aggregate, so every walk ends at a start value.
+        unsigned long long *wd = pw.words + (size_t)cu.u * 3 * dk + i;
+        if (cu.j > 0 && cu.j + 1 < cu.nch) {
+            st_relaxed(wd, tagged(ra, TAG_AGG));
+            st_relaxed(wd + dk, tagged(rb, TAG_AGG));
+        }
+        float ph_end = 0.f;
+        if (cu.j == 0) {
+            ph_end = b.dP_T ? b.dP_T[(size_t)cu.chain * dk + i] : 0.f;
+        } else {
+            float qa = 1.f, qb = 0.f;   // P^_end = qa x + qb, x = the start value of chunk jj
+            for (int jj = cu.j - 1;; --jj) {
+                const unsigned long long *dj = pw.words + ((size_t)jj * nchains + cu.chain) * 3 * dk + i;
+                unsigned long long w0 = 0ull, w1 = 0ull, w2 = ld_relaxed(dj + 2 * dk);
+                const long long ts = clock64();
+                bool timed_out = false;
+                while (tag_of(w2) != TAG_INCL) {
+                    w0 = ld_relaxed(dj);
+                    w1 = ld_relaxed(dj + dk);
+                    if (jj > 0 && tag_of(w0) == TAG_AGG && tag_of(w1) == TAG_AGG) break;
+                    // give up after ~1 s, or at once when another wait already gave up
+                    if (clock64() - ts > 2000000000ll || (a.err && (*(volatile unsigned *)a.err & ERR_TIMEOUT))) {
+                        timed_out = true;
+                        break;
+                    }
+                    __nanosleep(32);
+                    w2 = ld_relaxed(dj + 2 * dk);
+                }
+                if (timed_out) {
+                    raise_error(a.err, ERR_TIMEOUT);
+                    break;
+                }
+                if (tag_of(w2) == TAG_INCL || jj == 0) {
+                    ph_end = fmaf(qa, value_of(w2), qb);
+                    break;
+                }
+                qb = fmaf(qa, value_of(w1), qb);
+                qa *= value_of(w0);
+            }
+        }
+        st_relaxed(wd + 2 * dk, tagged(fmaf(ra, ph_end, rb), TAG_INCL));
+
+        // pass 2: the token adjoints with the incoming P^ (the serial kernel's arithmetic)
+        float ph = ph_end;
+#pragma unroll 2
+        for (int tt = L - 1; tt >= 0; --tt) {
+            const size_t e = ((size_t)(cu.lo + tt) * H + cu.h) * dk + i;
+            const float al = ldf(alpha + e), kk = ldf(k + e), ir = ir_s[tt], Pp = w.Pprev[e];
+            const float pm = fmaf(al * al, Pp, ldf(sigma + e));
+            const float mk = mu * kk * ir;
+            const float z = 1.f / fmaf(mk * kk, pm, 1.f);
+            const float Pt = pm * z;
+            const float pmh = w.part[e] + ph * z * z;
+            const float ch = -ph * Pt * Pt;
+            b.dk[e] = w.part[tokstride + e] + ch * 2.f * mk;
+            x_s[tt * dk + i] = -ch * mk * kk * ir;
+            b.dsigma[e] = pmh;
+            b.dalpha[e] = w.part[2 * tokstride + e] + 2.f * al * Pp * pmh;
+            ph = al * al * pmh;
+        }
+        if (cu.j >= cu.nch - 1 && b.dP0) b.dP0[(size_t)cu.chain * dk + i] = ph;
+        __syncthreads();
+        for (int tt = warp; tt < L; tt += nw) {
+            float x = 0.f;
+            for (int c = lane; c < dk; c += 32) x += x_s[tt * dk + c];
+            x = warp_sum(x);
+            if (lane == 0) b.dr[(size_t)(cu.lo + tt) * H + cu.h] = dd_s[tt] + x;
+        }
+        __syncthreads();   // the staged values and the claimed unit are free for the next unit
+    }
+}
+
 // ================================================================= isotropic variant
 // One uncertainty p per head (explainer "各向同性近似"): p^- = a p + s with a = mean(alpha^2),
 // s = mean(sigma); g = p^- k / den, den = r + p^- K2, K2 = |k|^2; p' = p^- z, z = 1/(1 + c p^-),
@@ -720,9 +889,38 @@ static cudaError_t launch_tape_scan(const BwdArgs &b, const BwdWs &w, int nchunk
     return launch_gain_scan_tma(sa, w.ntok, w.ckpt, st);
 }
 
+// bytes of the chunk-parallel adjoint's ticket counter and look-back words
+static size_t prev_scan_bytes(long long nchains, long long nchunks_max, int dk) {
+    return 256 + (size_t)nchains * (size_t)(nchunks_max > 0 ? nchunks_max : 1) * 3 * dk * 8;
+}
+
+// The serial uncertainty adjoint as the chunk-parallel scan, its words in the checkpoint
+// region (the state pass is done with it)
 template <typename T>
-static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, bool tape_scan, int nchunks_max,
-                                    cudaStream_t st) {
+static cudaError_t launch_prev_scan(const BwdArgs &b, const BwdWs &w, long long nchunks_max, cudaStream_t st) {
+    const int dk = b.a.dk;
+    const long long nchains = (long long)b.a.nseq * b.a.H;
+    PrevWs pw;
+    pw.counter = reinterpret_cast<unsigned *>(w.ckpt);
+    pw.words = reinterpret_cast<unsigned long long *>(reinterpret_cast<uint8_t *>(w.ckpt) + 256);
+    pw.nchunks_max = nchunks_max > 0 ? nchunks_max : 1;
+    cudaError_t e = cudaMemsetAsync(w.ckpt, 0, prev_scan_bytes(nchains, nchunks_max, dk), st);
+    if (e != cudaSuccess) return e;
+    const size_t smem = ((size_t)PC * dk + 2 * PC) * sizeof(float) + sizeof(PrevUnit);
+    KernelSetup ks;
+    e = kernel_setup(reinterpret_cast<const void *>(bwd_prev_scan_kernel<T>), smem, dk, true, &ks);
+    if (e != cudaSuccess) return e;
+    // persistent CTAs; units go out by ticket to resident CTAs only
+    long long grid = (long long)ks.sms * (ks.blocks_per_sm > 0 ? ks.blocks_per_sm : 1);
+    const long long units = pw.nchunks_max * nchains;
+    if (grid > units) grid = units;
+    bwd_prev_scan_kernel<T><<<(unsigned)grid, dk, smem, st>>>(b, w, pw);
+    return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, bool tape_scan, bool prev_scan,
+                                    int nchunks_max, cudaStream_t st) {
     const int chains = b.a.nseq * b.a.H, dk = b.a.dk;
     cudaError_t e;
     if (tape_scan) {
@@ -757,6 +955,7 @@ static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, bool tape_
         bwd_prev_iso_kernel<T><<<chains, dk, psm, st>>>(b, w);
         return cudaGetLastError();
     }
+    if (prev_scan) return launch_prev_scan<T>(b, w, nchunks_max, st);
     const size_t psm = ((size_t)5 * GT * dk + 2 * GT) * sizeof(float) + (size_t)3 * GT * dk * sizeof(T);
     e = set_smem(reinterpret_cast<const void *>(bwd_prev_kernel<T>), psm);
     if (e != cudaSuccess) return e;
@@ -784,8 +983,10 @@ cudaError_t launch_backward(const BwdArgs &b, bool bf16_in, long long ntok, long
     // sequences of very different lengths, whose work list is nseq x H x the longest's chunks)
     const bool tape_scan = !a.iso && ntok > 0 && gain_scan_tma_supported(a.dk, bf16_in) &&
                            scan_tma_workspace_bytes((long long)a.nseq * a.H, nchunks_max) <= ckpt_bytes;
+    const bool prev_scan = !a.iso && prev_scan_bytes((long long)a.nseq * a.H, nchunks_max, a.dk) <= ckpt_bytes;
     const int ncm = (int)(nchunks_max < (1ll << 30) ? nchunks_max : (1ll << 30));
-    return bf16_in ? launch_bwd_typed<bf16>(b, w, tape_scan, ncm, st) : launch_bwd_typed<float>(b, w, tape_scan, ncm, st);
+    return bf16_in ? launch_bwd_typed<bf16>(b, w, tape_scan, prev_scan, ncm, st)
+                   : launch_bwd_typed<float>(b, w, tape_scan, prev_scan, ncm, st);
 }
 
 }  // namespace kdn
