@@ -575,11 +575,11 @@ __global__ void __launch_bounds__(128) bwd_prev_scan_kernel(const BwdArgs b, con
         for (int tt = L - 1; tt >= 0; --tt) {
             const size_t e = ((size_t)(cu.lo + tt) * H + cu.h) * dk + i;
             const float al = ldf(alpha + e), kk = ldf(k + e);
-            const float pm = fmaf(al * al, w.Pprev[e], ldf(sigma + e));
+            const float pm = fmaf(al * al, ldf(w.Pprev + e), ldf(sigma + e));
             const float mk = mu * kk * ir_s[tt];
             const float z = 1.f / fmaf(mk * kk, pm, 1.f);
             const float aa = al * al, at = aa * z * z;
-            rb = fmaf(at, rb, aa * w.part[e]);
+            rb = fmaf(at, rb, aa * ldf(w.part + e));
             ra *= at;
         }
 
@@ -628,20 +628,20 @@ __global__ void __launch_bounds__(128) bwd_prev_scan_kernel(const BwdArgs b, con
 
         // pass 2: the token adjoints with the incoming P^ (the serial kernel's arithmetic)
         float ph = ph_end;
-#pragma unroll 2
+#pragma unroll 4
         for (int tt = L - 1; tt >= 0; --tt) {
             const size_t e = ((size_t)(cu.lo + tt) * H + cu.h) * dk + i;
-            const float al = ldf(alpha + e), kk = ldf(k + e), ir = ir_s[tt], Pp = w.Pprev[e];
+            const float al = ldf(alpha + e), kk = ldf(k + e), ir = ir_s[tt], Pp = ldf(w.Pprev + e);
             const float pm = fmaf(al * al, Pp, ldf(sigma + e));
             const float mk = mu * kk * ir;
             const float z = 1.f / fmaf(mk * kk, pm, 1.f);
             const float Pt = pm * z;
-            const float pmh = w.part[e] + ph * z * z;
+            const float pmh = ldf(w.part + e) + ph * z * z;
             const float ch = -ph * Pt * Pt;
-            b.dk[e] = w.part[tokstride + e] + ch * 2.f * mk;
+            b.dk[e] = ldf(w.part + tokstride + e) + ch * 2.f * mk;
             x_s[tt * dk + i] = -ch * mk * kk * ir;
             b.dsigma[e] = pmh;
-            b.dalpha[e] = w.part[2 * tokstride + e] + 2.f * al * Pp * pmh;
+            b.dalpha[e] = ldf(w.part + 2 * tokstride + e) + 2.f * al * Pp * pmh;
             ph = al * al * pmh;
         }
         if (cu.j >= cu.nch - 1 && b.dP0) b.dP0[(size_t)cu.chain * dk + i] = ph;
