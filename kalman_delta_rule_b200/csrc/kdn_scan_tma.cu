@@ -1,7 +1,7 @@
 // The uncertainty / gain scan for bf16 inputs with d_k = 128: the same single pass with a
 // decoupled look-back as the generic scan (explainer, closing paragraph of "各向同性近似": the
 // uncertainty recursion is a Moebius map whose 2x2 matrices compose), with
-//  - the chunk's alpha, sigma and k tiles fetched by TMA into one stage per CTA, three CTAs per
+//  - the chunk's alpha, sigma and k tiles fetched by TMA into one stage per CTA, four CTAs per
 //    SM, so the loads of one CTA overlap the arithmetic of the others;
 //  - look-back words that carry their own tag (64-bit (value, tag) per key channel), so a
 //    reader never needs a fence or a flag, and every channel walks back on its own;
@@ -20,10 +20,14 @@ enum : unsigned { TAG_AGG = 1, TAG_INCL = 2 };
 
 struct ScanTmaSmem {
     static constexpr uint32_t STAGE = 3 * 16384;          // alpha, sigma, k tiles of one chunk
-    static constexpr uint32_t COMP = STAGE;               // segment composites fp32 [4][128][4]
-    static constexpr uint32_t MISC = COMP + 4 * 128 * 16;  // r [64], mu / r [64], P at chunk start [128], sum P^- k^2 [64]
-    static constexpr uint32_t CTL = MISC + 1280;           // 2 mbarriers, the claimed unit
-    static constexpr uint32_t total = CTL + 64;
+    // segment composites fp32 (normalised maps [[m00, m01], [m10, 1]]): (m00, m01) [4][128] and
+    // m10 [4][128]; the last segment's m10 slots then hold the uncertainty at the chunk start
+    // (the re-expansion never reads that segment's composite)
+    static constexpr uint32_t COMP01 = STAGE;
+    static constexpr uint32_t COMP10 = COMP01 + 4 * 128 * 8;
+    static constexpr uint32_t MISC = COMP10 + 4 * 128 * 4;  // mu / r [64], sum P^- k^2 [64]
+    static constexpr uint32_t CTL = MISC + 512;             // 2 mbarriers, the claimed unit
+    static constexpr uint32_t total = CTL + 64;             // four CTAs per SM: <= 56 KB with the alignment pad
 };
 
 struct ScanTmaArgs {
@@ -83,7 +87,7 @@ __device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane, int &wh
 }
 }  // namespace
 
-__global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_constant__ ScanTmaArgs sa)
+__global__ void __launch_bounds__(NT, 4) gain_scan_tma_kernel(const __grid_constant__ ScanTmaArgs sa)
 {
     using L_ = ScanTmaSmem;
     using namespace tc;
@@ -91,11 +95,11 @@ __global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_const
     const uint32_t raw_u32 = smem_u32(smraw);
     const uint32_t sb = (raw_u32 + 1023u) & ~1023u;
     uint8_t *sm = smraw + (sb - raw_u32);
-    float *comp = reinterpret_cast<float *>(sm + L_::COMP);
-    float *r_s = reinterpret_cast<float *>(sm + L_::MISC);
-    float *mur = r_s + 64;
-    float *pst = mur + 64;
-    float *dsum = pst + 128;
+    float *comp01 = reinterpret_cast<float *>(sm + L_::COMP01);
+    float *comp10 = reinterpret_cast<float *>(sm + L_::COMP10);
+    float *pst = comp10 + 3 * 128;
+    float *mur = reinterpret_cast<float *>(sm + L_::MISC);
+    float *dsum = mur + 64;
     uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + L_::CTL);   // [2]
 
     const ScanArgs &a = sa.a;
@@ -118,6 +122,7 @@ __global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_const
 
     struct Unit { long long u; int c, chain, h, c0, L, nch; };
     static_assert(sizeof(Unit) <= 48, "claimed unit slot");
+    static_assert(L_::total + 1024 <= 57344, "four CTAs per SM");
     Unit *claimed = reinterpret_cast<Unit *>(sm + L_::CTL + 16);
     // next unit with tokens: thread 0 takes tickets (skipping chunks past a sequence's end) and
     // decodes the unit once for the block
@@ -163,7 +168,7 @@ __global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_const
         r_next = (tid < n.L) ? ldf(rin + (size_t)(n.c0 + tid) * H + n.h) : 1.f;
     };
 
-    // One stage: a unit's tiles are fetched when the unit is claimed; three CTAs per SM keep the
+    // One stage: a unit's tiles are fetched when the unit is claimed; four CTAs per SM keep the
     // loads of one CTA under the arithmetic of the others.
     for (int it = 0;; ++it) {
         const Unit cur = claim();
@@ -171,8 +176,8 @@ __global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_const
         fetch(cur, 0);
         const long long u = cur.u;
         const int c = cur.c, chain = cur.chain, h = cur.h, c0 = cur.c0, L = cur.L, nch = cur.nch;
+        const float r_cur = r_next;   // threads < 64: r of token tid
         if (tid < C) {
-            r_s[tid] = r_next;
             mur[tid] = a.mu / r_next;
             dsum[tid] = 0.f;
         }
@@ -189,7 +194,7 @@ __global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_const
         // ---- segment composites of the uncertainty maps (predict [[a, s],[0,1]], update [[1,0],[c,1]]);
         //      channels ch and ch + 1 in the two lanes of packed f32x2 arithmetic
         {
-            f32x2 m00 = pk2(1.f, 1.f), m01 = pk2(0.f, 0.f), m10 = m01, m11 = m00, gm = m00;
+            f32x2 m00 = pk2(1.f, 1.f), m01 = pk2(0.f, 0.f), m10 = m01, m11 = m00;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 if (tb + j < L) {
@@ -204,14 +209,12 @@ __global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_const
                     m11 = fma2(cc, y01, m11);
                     m00 = y00;
                     m01 = y01;
-                    gm = mul2(gm, al);
                 }
             }
             const float sa_ = 1.f / x2(m11), sb_ = 1.f / y2(m11);
-            *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch) * 4) =
-                make_float4(x2(m00) * sa_, x2(m01) * sa_, x2(m10) * sa_, x2(gm));
-            *reinterpret_cast<float4 *>(comp + (sgi * 128 + ch + 1) * 4) =
-                make_float4(y2(m00) * sb_, y2(m01) * sb_, y2(m10) * sb_, y2(gm));
+            *reinterpret_cast<float4 *>(comp01 + (sgi * 128 + ch) * 2) =
+                make_float4(x2(m00) * sa_, x2(m01) * sa_, y2(m00) * sb_, y2(m01) * sb_);
+            *reinterpret_cast<float2 *>(comp10 + sgi * 128 + ch) = make_float2(x2(m10) * sa_, y2(m10) * sb_);
         }
         __syncthreads();
 
@@ -222,7 +225,8 @@ __global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_const
             float g00 = 1.f, g01 = 0.f, g10 = 0.f, g11 = 1.f;
 #pragma unroll
             for (int q2 = 0; q2 < 4; ++q2) {
-                const float4 cm = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + cc) * 4);
+                const float2 c01 = *reinterpret_cast<const float2 *>(comp01 + (q2 * 128 + cc) * 2);
+                const float4 cm = make_float4(c01.x, c01.y, comp10[q2 * 128 + cc], 0.f);
                 const float n00 = fmaf(cm.x, g00, cm.y * g10), n01 = fmaf(cm.x, g01, cm.y * g11);
                 const float n10 = fmaf(cm.z, g00, g10), n11 = fmaf(cm.z, g01, g11);
                 const float sc = 1.f / n11;
@@ -284,8 +288,9 @@ __global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_const
         {
             float Pa = pst[ch], Pb = pst[ch + 1];
             for (int q2 = 0; q2 < sgi; ++q2) {
-                const float4 ca = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch) * 4);
-                const float4 cb = *reinterpret_cast<const float4 *>(comp + (q2 * 128 + ch + 1) * 4);
+                const float4 c01 = *reinterpret_cast<const float4 *>(comp01 + (q2 * 128 + ch) * 2);
+                const float2 c10 = *reinterpret_cast<const float2 *>(comp10 + q2 * 128 + ch);
+                const float4 ca = make_float4(c01.x, c01.y, c10.x, 0.f), cb = make_float4(c01.z, c01.w, c10.y, 0.f);
                 Pa = mob(ca.x, ca.y, ca.z, 1.f, Pa);
                 Pb = mob(cb.x, cb.y, cb.z, 1.f, Pb);
             }
@@ -319,7 +324,7 @@ __global__ void __launch_bounds__(NT, 3) gain_scan_tma_kernel(const __grid_const
         __syncthreads();
         if (tid < C && tid < L) {
             const float x = dsum[tid];
-            const float dn = r_s[tid] + x, inv = 1.f / dn;
+            const float dn = r_cur + x, inv = 1.f / dn;
             dsum[tid] = inv;
             if (a.den) a.den[(size_t)(c0 + tid) * H + h] = dn;
             if (a.beta) a.beta[(size_t)(c0 + tid) * H + h] = x * inv;
@@ -364,8 +369,8 @@ cudaError_t launch_gain_scan_tma(const ScanArgs &a, long long ntok, void *worksp
     KernelSetup ks;
     e = kernel_setup(reinterpret_cast<const void *>(gain_scan_tma_kernel), smem, NT, true, &ks);
     if (e != cudaSuccess) return e;
-    // three CTAs per SM; units go out by ticket to resident CTAs only, so extra CTAs are harmless
-    long long grid = (long long)ks.sms * 3;
+    // four CTAs per SM; units go out by ticket to resident CTAs only, so extra CTAs are harmless
+    long long grid = (long long)ks.sms * 4;
     if (grid > units) grid = units;
     gain_scan_tma_kernel<<<(unsigned)grid, NT, smem, st>>>(sa);
     return cudaGetLastError();
