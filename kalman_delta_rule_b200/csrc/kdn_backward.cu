@@ -499,6 +499,7 @@ __global__ void __launch_bounds__(128) bwd_prev_kernel(const BwdArgs b, const Bw
 // CTA.  A sequence without tokens gets one empty unit, which passes dP_T through to dP0.
 namespace {
 constexpr int PC = 64;
+constexpr int PSEG = 4;   // segments of PC / PSEG tokens per chunk
 enum : unsigned { TAG_AGG = 1, TAG_INCL = 2 };
 struct PrevWs {
     unsigned *counter;
@@ -521,24 +522,28 @@ __device__ __forceinline__ void st_relaxed(unsigned long long *p, unsigned long 
 struct PrevUnit { long long u; int j, chain, h, lo, hi, nch; };
 }  // namespace
 
-// dynamic shared memory: dr terms [PC][dk]; 1/r, den^ [PC]; the claimed unit
+// dynamic shared memory: dr terms [PC][dk]; 1/r, den^ [PC]; segment maps and incoming P^
+// [PSEG][dk] float2; the claimed unit.  Thread = key channel x segment of PC / PSEG tokens
+// (segment 0 holds the latest tokens).
 template <typename T>
-__global__ void __launch_bounds__(128) bwd_prev_scan_kernel(const BwdArgs b, const BwdWs w, const PrevWs pw)
+__global__ void __launch_bounds__(512) bwd_prev_scan_kernel(const BwdArgs b, const BwdWs w, const PrevWs pw)
 {
     extern __shared__ float smf[];
     const TokenArgs &a = b.a;
     const int dk = a.dk, H = a.H;
     float *x_s = smf, *ir_s = x_s + PC * dk, *dd_s = ir_s + PC;
-    PrevUnit *claimed = reinterpret_cast<PrevUnit *>(dd_s + PC);
+    float2 *seg_s = reinterpret_cast<float2 *>(dd_s + PC);       // [PSEG][dk]: (a, b), then (P^_in, -)
+    PrevUnit *claimed = reinterpret_cast<PrevUnit *>(seg_s + PSEG * dk);
     const T *alpha = static_cast<const T *>(a.alpha), *sigma = static_cast<const T *>(a.sigma);
     const T *k = static_cast<const T *>(a.k), *r = static_cast<const T *>(a.r);
-    const int i = threadIdx.x, warp = i >> 5, lane = i & 31, nw = dk >> 5;
+    const int tid = threadIdx.x, nt = blockDim.x, warp = tid >> 5, lane = tid & 31, nw = nt >> 5;
+    const int i = tid % dk, sg = tid / dk;
     const float mu = a.mu;
     const size_t tokstride = (size_t)w.ntok * H * dk;
     const int nchains = a.nseq * H;
     const long long units = pw.nchunks_max * nchains;
     for (;;) {
-        if (i == 0) {
+        if (tid == 0) {
             PrevUnit n;
             for (;;) {
                 n.u = (long long)atomicAdd(pw.counter, 1u);
@@ -562,17 +567,19 @@ __global__ void __launch_bounds__(128) bwd_prev_scan_kernel(const BwdArgs b, con
         const PrevUnit cu = *claimed;
         if (cu.u >= units) break;
         const int L = cu.hi - cu.lo;
-        for (int tt = i; tt < L; tt += dk) {
+        for (int tt = tid; tt < L; tt += nt) {
             const size_t th = (size_t)(cu.lo + tt) * H + cu.h;
             ir_s[tt] = 1.f / ldf(r + th);
             dd_s[tt] = w.dden[th];
         }
         __syncthreads();
+        // this thread's tokens (chunk offsets), walked from the latest
+        const int seg_hi = L - sg * (PC / PSEG), seg_lo = max(0, seg_hi - PC / PSEG);
 
-        // pass 1: the chunk's composite map, P^ at the chunk start = ra P^_end + rb
+        // pass 1: the segment's composite map, P^ at its start = ra P^ at its end + rb
         float ra = 1.f, rb = 0.f;
 #pragma unroll 4
-        for (int tt = L - 1; tt >= 0; --tt) {
+        for (int tt = seg_hi - 1; tt >= seg_lo; --tt) {
             const size_t e = ((size_t)(cu.lo + tt) * H + cu.h) * dk + i;
             const float al = ldf(alpha + e), kk = ldf(k + e);
             const float pm = fmaf(al * al, ldf(w.Pprev + e), ldf(sigma + e));
@@ -582,54 +589,75 @@ __global__ void __launch_bounds__(128) bwd_prev_scan_kernel(const BwdArgs b, con
             rb = fmaf(at, rb, aa * ldf(w.part + e));
             ra *= at;
         }
+        seg_s[sg * dk + i] = make_float2(ra, rb);
+        __syncthreads();
 
-        // the incoming P^ at the chunk end: dP_T for the last chunk, else the later chunks' words.
-        // The last chunk publishes no aggregate, so every walk ends at a start value.
-        unsigned long long *wd = pw.words + (size_t)cu.u * 3 * dk + i;
-        if (cu.j > 0 && cu.j + 1 < cu.nch) {
-            st_relaxed(wd, tagged(ra, TAG_AGG));
-            st_relaxed(wd + dk, tagged(rb, TAG_AGG));
-        }
-        float ph_end = 0.f;
-        if (cu.j == 0) {
-            ph_end = b.dP_T ? b.dP_T[(size_t)cu.chain * dk + i] : 0.f;
-        } else {
-            float qa = 1.f, qb = 0.f;   // P^_end = qa x + qb, x = the start value of chunk jj
-            for (int jj = cu.j - 1;; --jj) {
-                const unsigned long long *dj = pw.words + ((size_t)jj * nchains + cu.chain) * 3 * dk + i;
-                unsigned long long w0 = 0ull, w1 = 0ull, w2 = ld_relaxed(dj + 2 * dk);
-                const long long ts = clock64();
-                bool timed_out = false;
-                while (tag_of(w2) != TAG_INCL) {
-                    w0 = ld_relaxed(dj);
-                    w1 = ld_relaxed(dj + dk);
-                    if (jj > 0 && tag_of(w0) == TAG_AGG && tag_of(w1) == TAG_AGG) break;
-                    // give up after ~1 s, or at once when another wait already gave up
-                    if (clock64() - ts > 2000000000ll || (a.err && (*(volatile unsigned *)a.err & ERR_TIMEOUT))) {
-                        timed_out = true;
+        // segment-0 threads (one per key channel): the chunk's map, its publication, the
+        // incoming P^ at the chunk end (dP_T for the last chunk, else the later chunks' words),
+        // and the incoming P^ of every segment.  The last chunk publishes no aggregate, so every
+        // walk ends at a start value.
+        if (sg == 0) {
+            float ca = 1.f, cb = 0.f;
+#pragma unroll
+            for (int q = 0; q < PSEG; ++q) {
+                const float2 m = seg_s[q * dk + i];
+                cb = fmaf(m.x, cb, m.y);
+                ca *= m.x;
+            }
+            unsigned long long *wd = pw.words + (size_t)cu.u * 3 * dk + i;
+            if (cu.j > 0 && cu.j + 1 < cu.nch) {
+                st_relaxed(wd, tagged(ca, TAG_AGG));
+                st_relaxed(wd + dk, tagged(cb, TAG_AGG));
+            }
+            float ph_end = 0.f;
+            if (cu.j == 0) {
+                ph_end = b.dP_T ? b.dP_T[(size_t)cu.chain * dk + i] : 0.f;
+            } else {
+                float qa = 1.f, qb = 0.f;   // P^_end = qa x + qb, x = the start value of chunk jj
+                for (int jj = cu.j - 1;; --jj) {
+                    const unsigned long long *dj = pw.words + ((size_t)jj * nchains + cu.chain) * 3 * dk + i;
+                    unsigned long long w0 = 0ull, w1 = 0ull, w2 = ld_relaxed(dj + 2 * dk);
+                    const long long ts = clock64();
+                    bool timed_out = false;
+                    while (tag_of(w2) != TAG_INCL) {
+                        w0 = ld_relaxed(dj);
+                        w1 = ld_relaxed(dj + dk);
+                        if (jj > 0 && tag_of(w0) == TAG_AGG && tag_of(w1) == TAG_AGG) break;
+                        // give up after ~1 s, or at once when another wait already gave up
+                        if (clock64() - ts > 2000000000ll || (a.err && (*(volatile unsigned *)a.err & ERR_TIMEOUT))) {
+                            timed_out = true;
+                            break;
+                        }
+                        __nanosleep(32);
+                        w2 = ld_relaxed(dj + 2 * dk);
+                    }
+                    if (timed_out) {
+                        raise_error(a.err, ERR_TIMEOUT);
                         break;
                     }
-                    __nanosleep(32);
-                    w2 = ld_relaxed(dj + 2 * dk);
+                    if (tag_of(w2) == TAG_INCL || jj == 0) {
+                        ph_end = fmaf(qa, value_of(w2), qb);
+                        break;
+                    }
+                    qb = fmaf(qa, value_of(w1), qb);
+                    qa *= value_of(w0);
                 }
-                if (timed_out) {
-                    raise_error(a.err, ERR_TIMEOUT);
-                    break;
-                }
-                if (tag_of(w2) == TAG_INCL || jj == 0) {
-                    ph_end = fmaf(qa, value_of(w2), qb);
-                    break;
-                }
-                qb = fmaf(qa, value_of(w1), qb);
-                qa *= value_of(w0);
+            }
+            st_relaxed(wd + 2 * dk, tagged(fmaf(ca, ph_end, cb), TAG_INCL));
+            float in = ph_end;
+#pragma unroll
+            for (int q = 0; q < PSEG; ++q) {
+                const float2 m = seg_s[q * dk + i];
+                seg_s[q * dk + i] = make_float2(in, 0.f);
+                in = fmaf(m.x, in, m.y);
             }
         }
-        st_relaxed(wd + 2 * dk, tagged(fmaf(ra, ph_end, rb), TAG_INCL));
+        __syncthreads();
 
         // pass 2: the token adjoints with the incoming P^ (the serial kernel's arithmetic)
-        float ph = ph_end;
+        float ph = seg_s[sg * dk + i].x;
 #pragma unroll 4
-        for (int tt = L - 1; tt >= 0; --tt) {
+        for (int tt = seg_hi - 1; tt >= seg_lo; --tt) {
             const size_t e = ((size_t)(cu.lo + tt) * H + cu.h) * dk + i;
             const float al = ldf(alpha + e), kk = ldf(k + e), ir = ir_s[tt], Pp = ldf(w.Pprev + e);
             const float pm = fmaf(al * al, Pp, ldf(sigma + e));
@@ -644,7 +672,7 @@ __global__ void __launch_bounds__(128) bwd_prev_scan_kernel(const BwdArgs b, con
             b.dalpha[e] = ldf(w.part + 2 * tokstride + e) + 2.f * al * Pp * pmh;
             ph = al * al * pmh;
         }
-        if (cu.j >= cu.nch - 1 && b.dP0) b.dP0[(size_t)cu.chain * dk + i] = ph;
+        if (sg == PSEG - 1 && cu.j >= cu.nch - 1 && b.dP0) b.dP0[(size_t)cu.chain * dk + i] = ph;
         __syncthreads();
         for (int tt = warp; tt < L; tt += nw) {
             float x = 0.f;
@@ -906,15 +934,16 @@ static cudaError_t launch_prev_scan(const BwdArgs &b, const BwdWs &w, long long 
     pw.nchunks_max = nchunks_max > 0 ? nchunks_max : 1;
     cudaError_t e = cudaMemsetAsync(w.ckpt, 0, prev_scan_bytes(nchains, nchunks_max, dk), st);
     if (e != cudaSuccess) return e;
-    const size_t smem = ((size_t)PC * dk + 2 * PC) * sizeof(float) + sizeof(PrevUnit);
+    const size_t smem = ((size_t)PC * dk + 2 * PC) * sizeof(float) + (size_t)PSEG * dk * sizeof(float2) + sizeof(PrevUnit);
+    const int nt = dk * PSEG;
     KernelSetup ks;
-    e = kernel_setup(reinterpret_cast<const void *>(bwd_prev_scan_kernel<T>), smem, dk, true, &ks);
+    e = kernel_setup(reinterpret_cast<const void *>(bwd_prev_scan_kernel<T>), smem, nt, true, &ks);
     if (e != cudaSuccess) return e;
     // persistent CTAs; units go out by ticket to resident CTAs only
     long long grid = (long long)ks.sms * (ks.blocks_per_sm > 0 ? ks.blocks_per_sm : 1);
     const long long units = pw.nchunks_max * nchains;
     if (grid > units) grid = units;
-    bwd_prev_scan_kernel<T><<<(unsigned)grid, dk, smem, st>>>(b, w, pw);
+    bwd_prev_scan_kernel<T><<<(unsigned)grid, nt, smem, st>>>(b, w, pw);
     return cudaGetLastError();
 }
 
