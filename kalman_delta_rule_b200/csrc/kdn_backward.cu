@@ -69,6 +69,25 @@ __device__ __forceinline__ void stage_rows(void *dst, const void *src, size_t st
     }
 }
 __device__ __forceinline__ float lds(const float *p) { return *p; }
+// 16 consecutive staged values (16-byte aligned) as 8 column pairs, in 128-bit shared loads
+__device__ __forceinline__ void lds16x2(const float *p, f32x2 (&x)[8]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const ulonglong2 v = reinterpret_cast<const ulonglong2 *>(p)[q];
+        x[2 * q] = v.x;
+        x[2 * q + 1] = v.y;
+    }
+}
+__device__ __forceinline__ void lds16x2(const bf16 *p, f32x2 (&x)[8]) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const uint4 v = reinterpret_cast<const uint4 *>(p)[q];
+        const unsigned w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+            x[4 * q + m] = pk2(__uint_as_float(w[m] << 16), __uint_as_float(w[m] & 0xffff0000u));
+    }
+}
 __device__ __forceinline__ float lds(const bf16 *p) {
     return __uint_as_float(((unsigned)*reinterpret_cast<const unsigned short *>(p)) << 16);
 }
@@ -327,10 +346,12 @@ __global__ void __launch_bounds__(128, 4) bwd_state_kernel(const BwdArgs b, cons
                 const f32x2 al2 = pk2(al, al), gg2 = pk2(gg, gg), qq2 = pk2(qq, qq), nk2 = pk2(-kk, -kk);
                 f32x2 dq2 = pk2(0.f, 0.f), gp2 = dq2;
                 float p[16];
+                f32x2 dov[8];
                 lds8x2(us + tt * DB, uu);
+                lds16x2(do_s + tt * DB, dov);
 #pragma unroll
                 for (int jp = 0; jp < 8; ++jp) {
-                    const f32x2 do2 = pk2(lds(do_s + tt * DB + 2 * jp), lds(do_s + tt * DB + 2 * jp + 1));
+                    const f32x2 do2 = dov[jp];
                     const f32x2 St = fma2(gg2, uu[jp], mul2(al2, Sp[jp]));
                     Sh[jp] = fma2(qq2, do2, Sh[jp]);
                     dq2 = fma2(St, do2, dq2);
