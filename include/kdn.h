@@ -201,7 +201,8 @@ kdn_status_t kdn_gain_scan_noalloc(const kdn_problem_t *p,
  * Computes the gradients of  L = <o, d_o> + <S_T, dS_T> + <P_T, dP_T>, where o, S_T and P_T are
  * what kdn_forward_chunkwise() returns for the same problem and inputs, with respect to every
  * input: the vector-Jacobian products of one training step.
- *  p                  : as for the forward, either variant (`chunk` and `max_seqlen` are ignored)
+ *  p                  : as for the forward, either variant (`chunk` is ignored; `max_seqlen`, for
+ *                       packed sequences, bounds the chunk-parallel work lists as for the forward)
  *  q ... P0           : the forward's inputs, same layouts (S0 / P0 NULL = 0 / 1; P0 [N, H] isotropic)
  *  d_o                : device [B, T, H, d_v] (in_dtype), gradient of L with respect to o
  *  dS_T, dP_T         : device fp32 [N, H, d_k, d_v], [N, H, d_k] ([N, H] isotropic), gradients
@@ -214,7 +215,11 @@ kdn_status_t kdn_gain_scan_noalloc(const kdn_problem_t *p,
  * Method: the uncertainty forward is taped (P before each token, den, g), the memory forward
  * is checkpointed every 16 tokens, and the reverse sweep recomputes each chunk from its
  * checkpoint (the state before every token is re-stepped forward, never reconstructed by
- * dividing by alpha); fp32 CUDA-core arithmetic.  The d_v column blocks of a (sequence, head)
+ * dividing by alpha); fp32 CUDA-core arithmetic.  The uncertainty tape (bf16, d_k = 128) and
+ * the uncertainty adjoint (diagonal variant) run as chunk-parallel scans with decoupled
+ * look-back whenever their work lists (N x H x the chunks of the longest sequence) fit the
+ * checkpoint region, else as one serial walk per (sequence, head); both give the same result
+ * to fp32 rounding.  The d_v column blocks of a (sequence, head)
  * add their shares of the sums over d_v with atomic adds, so the last bits of every gradient
  * except dv and dS0 can differ from run to run.  Workspace: about 7.0 KB per token and head
  * at d_k = d_v = 128.  Every pointer 16-byte aligned.  Outputs may not alias inputs.

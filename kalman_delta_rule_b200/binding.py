@@ -227,16 +227,17 @@ def forward(q, k, v, alpha, sigma, r, cu_seqlens=None, S0=None, P0=None, mu: flo
 
 
 def backward(q, k, v, alpha, sigma, r, d_o, cu_seqlens=None, S0=None, P0=None, dS=None, dP=None, mu: float = 1.0,
-             workspace=None, want_initial: bool = True, stream=None, variant: str = "diagonal"):
+             workspace=None, want_initial: bool = True, stream=None, variant: str = "diagonal", max_seqlen: int = 0):
     """Run kdn_backward on torch tensors laid out as for ``forward``.
 
     Returns a dict of fp32 gradients of <o, d_o> + <S_T, dS> + <P_T, dP>: dq, dk, dv,
     dalpha, dsigma ([B,T,H,d]), dr ([B,T,H]) and, with ``want_initial``, dS0 [N,H,dk,dv]
-    and dP0 ([N,H,dk] diagonal, [N,H] isotropic).  The workspace is allocated when not given."""
+    and dP0 ([N,H,dk] diagonal, [N,H] isotropic).  The workspace is allocated when not given.
+    ``max_seqlen`` (packed sequences; 0 = unknown) bounds the chunk-parallel work lists."""
     torch = _torch()
     if d_o.dtype != q.dtype:
         raise ValueError("d_o must have the dtype of the inputs")
-    p = make_problem(q, v, cu_seqlens=cu_seqlens, mu=mu, chunk=0, variant=variant)
+    p = make_problem(q, v, cu_seqlens=cu_seqlens, mu=mu, chunk=0, variant=variant, max_seqlen=max_seqlen)
     N = p.num_seqs
     dev = q.device
     f32 = dict(dtype=torch.float32, device=dev)

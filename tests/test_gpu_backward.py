@@ -4,6 +4,8 @@ varlen batches with an empty sequence, initial states and final-state gradients,
 and the d_v extremes, both uncertainty variants, and the full-size prefill workload
 (B4 H16 T4096 d128 bf16) on sampled (sequence, head) chains -- each chain's gradients depend
 on that chain's inputs only."""
+import functools
+
 import numpy as np
 import pytest
 
@@ -150,3 +152,33 @@ def test_backward_full_size_sampled_chains(kdn):
         assert_rel(got["dr"][sl, h], ref["dr"][:, 0], TOL, 'got["dr"][sl, h]')
         assert_rel(got["dS0"][s, h], ref["dS0"][0, 0], TOL, 'got["dS0"][s, h]')
         assert_rel(got["dP0"][s, h], ref["dP0"][0, 0], TOL, 'got["dP0"][s, h]')
+
+
+@functools.lru_cache(maxsize=1)
+def _many_short_case():
+    lens = np.random.default_rng(31).integers(1, 25, 200)
+    w = ragged(950, list(lens), 2, 128, 128, True)
+    S0, P0 = initial_state(33, w)
+    d_o, dS, dP = cotangents(34, w)
+    ref = kdn_grad.diag_grad(w.q, w.k, w.v, w.alpha, w.sigma, w.r, d_o, cu_seqlens=w.cu_seqlens,
+                             S0=S0, P0=P0, dS=dS, dP=dP, mu=1.5)
+    return w, S0, P0, d_o, dS, dP, ref
+
+
+@pytest.mark.parametrize("max_seqlen", [0, 24])
+def test_backward_many_short_sequences_both_work_lists(kdn, max_seqlen):
+    """200 packed sequences of 1-24 tokens, bf16, d = 128.  Without max_seqlen the chunk-parallel
+    work lists (nseq x H x the chunks of the whole packed length) do not fit the checkpoint
+    region, so the uncertainty tape and its adjoint take the serial per-chain kernels; with it
+    they take the chunk-parallel scans.  Both against the gradient oracle."""
+    import torch
+    w, S0, P0, d_o, dS, dP, ref = _many_short_case()
+    args = [to_dev(dense_shape(w, getattr(w, n))) for n in ("q", "k", "v", "alpha", "sigma", "r")]
+    g = kdn.backward(*args, to_dev(dense_shape(w, d_o)), cu_seqlens=to_dev(w.cu_seqlens), S0=to_dev(S0),
+                     P0=to_dev(P0), dS=to_dev(dS), dP=to_dev(dP), mu=1.5, max_seqlen=max_seqlen)
+    torch.cuda.synchronize()
+    kdn.last_device_error()
+    got = {n: to_host(g[n]) for n in NAMES}
+    for n in ("dq", "dk", "dv", "dalpha", "dsigma", "dr"):
+        got[n] = got[n].reshape((w.ntok,) + got[n].shape[2:])
+    check(got, ref)
