@@ -39,7 +39,8 @@
  *    legacy default stream).  Argument validation is synchronous and returns an
  *    error before anything is launched.  A failed launch returns KDN_ERR_CUDA.
  *  - Device-side conditions (a bounded wait that gave up, a packed sequence longer than
- *    the gain scan's max_seqlen) are recorded in a device error word and reported, after
+ *    the max_seqlen given to the gain scan or the backward) are recorded in a device error
+ *    word and reported, after
  *    a stream synchronisation, by kdn_last_device_error().  The outputs of a call whose
  *    kernels recorded such a condition are undefined.
  *  - Thread safety: calls may come from several host threads on different streams.
@@ -87,9 +88,10 @@ typedef struct {
     float mu;                       /* information scaling, > 0 */
     int chunk;                      /* execution path, see above */
     int max_seqlen;                 /* varlen: upper bound on every sequence length (0 = unknown, taken as T);
-                                       sizes only the gain scan's work list (the forward needs no bound).  A
-                                       sequence longer than it makes kdn_gain_scan record KDN_ERR_INVALID_ARG
-                                       in the device error word. */
+                                       sizes the gain scan's work list and the backward's chunk-parallel
+                                       uncertainty work lists (the forward needs no bound).  A sequence
+                                       longer than it makes kdn_gain_scan / kdn_backward record
+                                       KDN_ERR_INVALID_ARG in the device error word. */
     int variant;                    /* kdn_variant_t; 0 (zero-initialised struct) = diagonal */
 } kdn_problem_t;
 

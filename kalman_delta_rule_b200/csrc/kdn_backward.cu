@@ -576,6 +576,8 @@ __global__ void __launch_bounds__(512) bwd_prev_scan_kernel(const BwdArgs b, con
                 int t0, t1;
                 seq_range(a, s, t0, t1);
                 n.nch = (t1 - t0 + PC - 1) / PC;
+                // a sequence longer than max_seqlen has chunks past the work list
+                if (n.j == 0 && n.nch > pw.nchunks_max) raise_error(a.err, ERR_ARG);
                 if (n.j < n.nch || n.j == 0) {
                     n.hi = t1 - n.j * PC;
                     n.lo = max(t0, n.hi - PC);

@@ -182,3 +182,25 @@ def test_backward_many_short_sequences_both_work_lists(kdn, max_seqlen):
     for n in ("dq", "dk", "dv", "dalpha", "dsigma", "dr"):
         got[n] = got[n].reshape((w.ntok,) + got[n].shape[2:])
     check(got, ref)
+
+
+def test_backward_reports_a_sequence_longer_than_max_seqlen(kdn):
+    """The chunk-parallel uncertainty work lists are sized by max_seqlen (64-token chunks); a
+    longer packed sequence is reported by kdn_last_device_error, and the context stays usable:
+    the same call with a sufficient bound then matches the gradient oracle."""
+    import torch
+    w = ragged(977, [1, 63, 64, 0, 65, 130], 2, 128, 128, True)
+    d_o, dS, dP = cotangents(5, w)
+    args = [to_dev(dense_shape(w, getattr(w, n))) for n in ("q", "k", "v", "alpha", "sigma", "r")]
+    cu = to_dev(w.cu_seqlens)
+    kdn.backward(*args, to_dev(dense_shape(w, d_o)), cu_seqlens=cu, max_seqlen=64)
+    with pytest.raises(kdn.KdnError):
+        kdn.last_device_error()
+    ref = kdn_grad.diag_grad(w.q, w.k, w.v, w.alpha, w.sigma, w.r, d_o, cu_seqlens=w.cu_seqlens, dS=dS, dP=dP)
+    g = kdn.backward(*args, to_dev(dense_shape(w, d_o)), cu_seqlens=cu, dS=to_dev(dS), dP=to_dev(dP), max_seqlen=130)
+    torch.cuda.synchronize()
+    kdn.last_device_error()
+    got = {n: to_host(g[n]) for n in NAMES}
+    for n in ("dq", "dk", "dv", "dalpha", "dsigma", "dr"):
+        got[n] = got[n].reshape((w.ntok,) + got[n].shape[2:])
+    check(got, ref)
