@@ -154,6 +154,15 @@ __device__ __forceinline__ uint32_t ldg_u32(const bf16 *p) { return __ldg(reinte
 // a bf16 pair (low half = channel ch) widened to f32x2
 __device__ __forceinline__ f32x2 bf2(uint32_t w) { return pk2(tc::bf16_lo(w), tc::bf16_hi(w)); }
 
+// Failure paths: after a bounded wait gave up, one more bounded wait for the tcgen05 operations
+// (a fresh commit covers every earlier one) or the copy a CTA issued, before its tensor and shared
+// memory are released.  Out of line, so the kernels' register allocation does not carry them.
+__device__ __noinline__ void drain_mma(uint64_t *bar, uint32_t phase) {
+    tc::mma_commit(bar);
+    tc::mbar_wait(bar, phase);
+}
+__device__ __noinline__ void drain_copy(uint64_t *bar, uint32_t parity) { tc::mbar_wait(bar, parity); }
+
 // Look-back descriptors are 64-bit words (value, tag): each word carries its own status, so a
 // reader that sees a tag also sees that word's value, with no fence between writer and flag.
 enum : unsigned { TAG_NONE = 0, TAG_AGG = 1, TAG_INCL = 2 };
@@ -1021,7 +1030,12 @@ __global__ void __launch_bounds__(PNT, 2) chunk_prep_kernel(const __grid_constan
             bulk_commit();
         }
     }
-    if (ctl[1]) raise_error(a.err, ERR_TIMEOUT);
+    if (ctl[1]) {
+        raise_error(a.err, ERR_TIMEOUT);
+        // an MMA wait gave up: one more bounded wait for everything this CTA issued before its
+        // tensor memory is released
+        if (tid == 0) drain_mma(bar_mma, mma_phase);
+    }
     if (tid == 0) bulk_wait0();
     tc_fence_before();
     __syncthreads();
@@ -1086,7 +1100,9 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
     // the v tile: whole 64-column boxes; a 32-column tile is one half of its box
     const int vx0 = (tile * DVT) & ~63;
     const uint32_t voff = (uint32_t)((tile * DVT) & 63) * 2u;
+    int last0 = -1, last1 = -1;         // thread 0: the chunk last fetched into stage 0 / 1
     auto issue = [&](int c, int st) {   // record and v tile of chunk c into stage st
+        if (st == 0) last0 = c; else last1 = c;
         const long long uc = packed ? sa.U[c] + (long long)rank * H + h : (long long)c * sa.nchains + chain;
         const uint8_t *src = sa.rec + (size_t)uc * Rec::BYTES;
         mbar_expect_tx(bar_full + st, Rec::BYTES + L_::V_BYTES);
@@ -1244,6 +1260,13 @@ __global__ void __launch_bounds__(SNT, 1) chunk_state_kernel(const __grid_consta
         }
     } else {
         raise_error(a.err, ERR_TIMEOUT);
+        // a wait gave up: one more bounded wait for the MMAs and copies this CTA issued before
+        // its tensor and shared memory are released
+        if (tid == 0) {
+            drain_mma(bar_mma, mma_phase);
+            if (last0 >= 0) drain_copy(bar_full, (uint32_t)((last0 >> 1) & 1));
+            if (last1 >= 0) drain_copy(bar_full + 1, (uint32_t)((last1 >> 1) & 1));
+        }
     }
     tc_fence_before();
     __syncthreads();
