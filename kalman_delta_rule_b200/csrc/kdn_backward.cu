@@ -636,12 +636,17 @@ __global__ void __launch_bounds__(512) bwd_prev_scan_kernel(const BwdArgs b, con
             if (cu.j == 0) {
                 ph_end = b.dP_T ? b.dP_T[(size_t)cu.chain * dk + i] : 0.f;
             } else {
-                float qa = 1.f, qb = 0.f;   // P^_end = qa x + qb, x = the start value of chunk jj
-                for (int jj = cu.j - 1;; --jj) {
-                    const unsigned long long *dj = pw.words + ((size_t)jj * nchains + cu.chain) * 3 * dk + i;
+                // walk to the nearest later chunk whose start value is published, then back through
+                // the aggregates of the chunks in between, each applied as its owner applies it:
+                // the result does not depend on which words were published when (bit-reproducible)
+                auto words_of = [&](int jj) { return pw.words + ((size_t)jj * nchains + cu.chain) * 3 * dk + i; };
+                bool timed_out = false;
+                int jj = cu.j - 1;
+                float x = 0.f;
+                for (;; --jj) {
+                    const unsigned long long *dj = words_of(jj);
                     unsigned long long w0 = 0ull, w1 = 0ull, w2 = ld_relaxed(dj + 2 * dk);
                     const long long ts = clock64();
-                    bool timed_out = false;
                     while (tag_of(w2) != TAG_INCL) {
                         w0 = ld_relaxed(dj);
                         w1 = ld_relaxed(dj + dk);
@@ -659,12 +664,17 @@ __global__ void __launch_bounds__(512) bwd_prev_scan_kernel(const BwdArgs b, con
                         break;
                     }
                     if (tag_of(w2) == TAG_INCL || jj == 0) {
-                        ph_end = fmaf(qa, value_of(w2), qb);
+                        x = value_of(w2);
                         break;
                     }
-                    qb = fmaf(qa, value_of(w1), qb);
-                    qa *= value_of(w0);
                 }
+                if (!timed_out) {
+                    for (int k2 = jj + 1; k2 < cu.j; ++k2) {   // aggregates seen published by the walk
+                        const unsigned long long *dq = words_of(k2);
+                        x = fmaf(value_of(ld_relaxed(dq)), x, value_of(ld_relaxed(dq + dk)));
+                    }
+                }
+                ph_end = timed_out ? 0.f : x;
             }
             st_relaxed(wd + 2 * dk, tagged(fmaf(ca, ph_end, cb), TAG_INCL));
             float in = ph_end;

@@ -159,44 +159,42 @@ __global__ void __launch_bounds__(SNT) gain_scan_kernel(ScanArgs a)
         if (c == 0) {
             if (tid < DK) pst[tid] = a.P0 ? a.P0[(size_t)chain * DK + tid] : 1.f;
         } else {
-            float r00 = 1.f, r01 = 0.f, r10 = 0.f, r11 = 1.f;   // composite of the chunks walked over
-            int j = c - 1;
+            // walk back to the nearest chunk whose end-of-chunk uncertainty is published, then
+            // forward through the aggregates of the chunks in between, each applied as its owner
+            // applies it: the start value does not depend on which flags were set when
+            int j = c - 1, f = FLAG_NONE;
             for (;;) {
                 const long long uj = (long long)j * a.nchains + chain;
                 if (tid == 0) {
                     volatile int *fp = a.flags + uj;
-                    int f = *fp;
+                    int fl = *fp;
                     const long long tstart = clock64();
-                    while (f == FLAG_NONE) {
+                    while (fl == FLAG_NONE) {
                         // give up after ~1 s, or at once when another wait already gave up
                         if (clock64() - tstart > 2000000000ll || (a.err && (*(volatile unsigned *)a.err & ERR_TIMEOUT))) break;
                         __nanosleep(64);
-                        f = *fp;
+                        fl = *fp;
                     }
-                    if (f == FLAG_NONE) { raise_error(a.err, ERR_TIMEOUT); f = -1; }
-                    ctl[1] = f;
+                    if (fl == FLAG_NONE) { raise_error(a.err, ERR_TIMEOUT); fl = -1; }
+                    ctl[1] = fl;
                 }
                 __syncthreads();
-                const int f = ctl[1];
-                __threadfence();
-                const float *dj = a.desc + (size_t)uj * 4 * DK;
-                if (f == FLAG_INCL || f < 0) {
-                    if (tid < DK) {
-                        const float pe = f < 0 ? 1.f : __ldcg(dj + 3 * DK + tid);
-                        pst[tid] = mob(r00, r01, r10, r11, pe);
-                    }
-                    __syncthreads();
-                    break;
-                }
-                if (tid < DK) {   // R <- R * A_j (A_j acts first)
-                    const float m00 = __ldcg(dj + tid), m01 = __ldcg(dj + DK + tid), m10 = __ldcg(dj + 2 * DK + tid);
-                    const float n00 = fmaf(r00, m00, r01 * m10), n01 = fmaf(r00, m01, r01);
-                    const float n10 = fmaf(r10, m00, r11 * m10), n11 = fmaf(r10, m01, r11);
-                    const float sc = 1.f / n11;
-                    r00 = n00 * sc; r01 = n01 * sc; r10 = n10 * sc; r11 = 1.f;
-                }
-                __syncthreads();
+                f = ctl[1];
+                __syncthreads();   // ctl[1] is read by every thread before it is replaced
+                if (f == FLAG_INCL || f < 0) break;
                 --j;
+            }
+            __threadfence();
+            if (tid < DK) {
+                float x = 1.f;
+                if (f >= 0) {
+                    x = __ldcg(a.desc + ((size_t)((long long)j * a.nchains + chain) * 4 + 3) * DK + tid);
+                    for (int jj = j + 1; jj < c; ++jj) {   // aggregates whose flags the walk saw
+                        const float *dq = a.desc + (size_t)((long long)jj * a.nchains + chain) * 4 * DK;
+                        x = mob(__ldcg(dq + tid), __ldcg(dq + DK + tid), __ldcg(dq + 2 * DK + tid), 1.f, x);
+                    }
+                }
+                pst[tid] = x;
             }
         }
         __syncthreads();

@@ -241,10 +241,15 @@ __global__ void __launch_bounds__(NT, 4) gain_scan_tma_kernel(const __grid_const
             if (c == 0) {
                 p0 = a.P0 ? a.P0[(size_t)chain * DK + cc] : 1.f;
             } else {
-                float r00 = 1.f, r01 = 0.f, r10 = 0.f;   // composite of the chunks walked over ((1,1) kept at 1)
+                // walk back to the nearest published end-of-chunk uncertainty, then forward through the
+                // aggregates of the chunks in between, each applied as its owner applies it: the start
+                // value does not depend on which words were published when (bit-reproducible)
+                auto words_of = [&](int j) { return sa.words + ((size_t)j * a.nchains + chain) * 4 * DK + cc; };
                 bool timed_out = false;
-                for (int j = c - 1;; --j) {
-                    const unsigned long long *dj = sa.words + ((size_t)j * a.nchains + chain) * 4 * DK + cc;
+                int j = c - 1;
+                float x = 1.f;
+                for (;; --j) {
+                    const unsigned long long *dj = words_of(j);
                     unsigned long long w0 = 0ull, w1 = 0ull, w2 = 0ull, w3 = ld_relaxed(dj + 3 * DK);
                     const long long ts = clock64();
                     while (tag_of(w3) != TAG_INCL) {
@@ -262,19 +267,20 @@ __global__ void __launch_bounds__(NT, 4) gain_scan_tma_kernel(const __grid_const
                     }
                     if (timed_out) {
                         raise_error(a.err, ERR_TIMEOUT);
-                        p0 = 1.f;
                         break;
                     }
                     if (tag_of(w3) == TAG_INCL) {
-                        p0 = mob(r00, r01, r10, 1.f, value_of(w3));
+                        x = value_of(w3);
                         break;
                     }
-                    const float m00 = value_of(w0), m01 = value_of(w1), m10 = value_of(w2);
-                    const float n00 = fmaf(r00, m00, r01 * m10), n01 = fmaf(r00, m01, r01);
-                    const float n10 = fmaf(r10, m00, m10), n11 = fmaf(r10, m01, 1.f);
-                    const float sc = 1.f / n11;
-                    r00 = n00 * sc; r01 = n01 * sc; r10 = n10 * sc;
                 }
+                if (!timed_out) {
+                    for (int jj = j + 1; jj < c; ++jj) {   // aggregates seen published by the walk
+                        const unsigned long long *dq = words_of(jj);
+                        x = mob(value_of(ld_relaxed(dq)), value_of(ld_relaxed(dq + DK)), value_of(ld_relaxed(dq + 2 * DK)), 1.f, x);
+                    }
+                }
+                p0 = timed_out ? 1.f : x;
             }
             pst[cc] = p0;
             const float pe = mob(g00, g01, g10, 1.f, p0);

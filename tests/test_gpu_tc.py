@@ -102,3 +102,32 @@ def test_varlen_262144_full_size_sampled(kdn):
     shortest = int(np.argmin(lens))
     picks = [(longest, 3), (shortest, 0), (w.num_seqs - 1, 15), (0, 7)]
     sampled_check(kdn, w, picks)
+
+
+@pytest.mark.parametrize("variant", ["diagonal", "isotropic"])
+def test_prefill_and_gain_scan_are_bit_reproducible(kdn, variant):
+    """The decoupled look-backs form each chunk's starting uncertainty by the same operations
+    whichever predecessors had published, so two calls on the prefill workload (4096 units on
+    every SM, the look-back paths taken differing from run to run) give identical bits: o, S, P of
+    the two-launch forward, and g, k^T g, P of the gain scan."""
+    import torch
+    w = inputs.prefill_4x4096()
+    args = [to_dev(dense_shape(w, getattr(w, n))) for n in ("q", "k", "v", "alpha", "sigma", "r")]
+    outs = []
+    for _ in range(2):
+        o, S, P = kdn.forward(*args, mu=1.0, chunk=64, variant=variant)
+        torch.cuda.synchronize()
+        kdn.last_device_error()
+        outs.append((to_host(o), to_host(S), to_host(P)))
+    for a_, b_, n in zip(outs[0], outs[1], ("o", "S", "P")):
+        np.testing.assert_array_equal(a_, b_, err_msg=n)
+    if variant == "diagonal":
+        k, al, sg, r = args[1], args[3], args[4], args[5]
+        scans = []
+        for _ in range(2):
+            g, be, P = kdn.gain_scan(k, al, sg, r, mu=1.0)
+            torch.cuda.synchronize()
+            kdn.last_device_error()
+            scans.append((to_host(g), to_host(be), to_host(P)))
+        for a_, b_, n in zip(scans[0], scans[1], ("g", "k^T g", "P")):
+            np.testing.assert_array_equal(a_, b_, err_msg=n)

@@ -7,20 +7,19 @@ scratch in the library's fixed device array.  Two calls in a row with different 
 second call finds the first one's leftovers in the shared array, and any of them read as its
 own would change its result), each compared with the workspace call on the same problem, for
 both scan kernels: the TMA kernel (bf16, d_k = 128) and the generic one (fp32, d_k = 64, a
-ragged tail).  The decoupled look-back takes a chunk's starting uncertainty from whichever
-predecessors have published by then, so the last bits may differ between any two calls (two
-workspace calls included); the comparison is therefore at 1e-6 relative, a thousand times
-tighter than the scan's parity tolerance.  The device's free memory must not change across a
+ragged tail).  The decoupled look-back forms a chunk's starting uncertainty by the same
+operations whichever predecessors have published by then, so the scan is bit-reproducible and
+the two entry points must agree bit for bit.  The device's free memory must not change across a
 call.  This file is collected last, so a stop-at-first-failure run has run every other test.
 """
+import numpy as np
 import pytest
 
 from kalman_delta_rule_b200 import inputs
-from tests.kdn_testutil import assert_rel, dense_shape, to_dev, to_host
+from tests.kdn_testutil import dense_shape, to_dev, to_host
 
 pytestmark = pytest.mark.gpu
 
-TOL = 1e-6
 
 CASES = {
     # 64 chunks x 64 (sequence, head) pairs: fits the fixed scratch
@@ -53,9 +52,9 @@ def test_noalloc_gain_scan_matches_the_workspace_version_twice(kdn, case):
         kdn.last_device_error()
         if call == 1:   # the first call on a device may load the library's module with its fixed array
             assert free_after == free_before, (free_before, free_after)
-        assert_rel(to_host(g), to_host(g_ref), TOL, f"g, call {call}")
-        assert_rel(to_host(be), to_host(be_ref), TOL, f"k^T g, call {call}")
-        assert_rel(to_host(P), to_host(P_ref), TOL, f"P, call {call}")
+        np.testing.assert_array_equal(to_host(g), to_host(g_ref), err_msg=f"g, call {call}")
+        np.testing.assert_array_equal(to_host(be), to_host(be_ref), err_msg=f"k^T g, call {call}")
+        np.testing.assert_array_equal(to_host(P), to_host(P_ref), err_msg=f"P, call {call}")
 
 
 def test_noalloc_gain_scan_rejects_a_problem_larger_than_its_scratch(kdn):
