@@ -14,8 +14,9 @@
 //     r^ = den^ - sum_i c^_i mu k_i^2 / r^2;  sigma^ = P^-^;  alpha^ += 2 alpha P P^-^;  P^ = alpha^2 P^-^.
 //
 // Four launches:
-//   tape  (one CTA per (sequence, head), thread = key channel): the uncertainty forward; writes
-//         P before each token, den and g per token;
+//   tape  the uncertainty forward; writes P before each token, den and g per token: the
+//         chunk-parallel gain scan (bf16, d_k = 128, diagonal), else one CTA per (sequence, head),
+//         thread = key channel;
 //   state (one CTA per (sequence, head, 16-column block of d_v), thread = key channel = row of S):
 //         the memory forward with S checkpoints every 16 tokens and u of every token taped, then
 //         the reverse sweep chunk by chunk: the chunk's inputs are staged in shared memory, the
@@ -25,12 +26,12 @@
 //         reconstructed by dividing by alpha, which loses it when alpha is small).  Writes dv and
 //         adds its column block's share of dq, g^, the S-part of k^ and the S-part of alpha^ into
 //         them with fire-and-forget atomic adds (dq into the output, the others into three token
-//         vectors that the tape kernel zeroed);
+//         vectors cleared before the tape);
 //   local (one warp per (token, head), every token in parallel): writes den^ and the parts of P^-^
 //         and k^ that do not depend on the later tokens' P^;
-//   prev  (one CTA per (sequence, head), thread = key channel): the one serial part of the
-//         uncertainty adjoint, P^ <- alpha^2 (P^-^local + P^ z^2), and the outputs that need P^:
-//         dk, dalpha, dsigma, dr and dP0.
+//   prev  the one serial part of the uncertainty adjoint, P^ <- alpha^2 (P^-^local + P^ z^2), and
+//         the outputs that need P^: dk, dalpha, dsigma, dr and dP0 -- for the diagonal variant a
+//         chunk-parallel reverse affine scan, else one CTA per (sequence, head).
 // Token rows are staged into shared memory with 16-byte asynchronous copies, a group of tokens at
 // a time, so each group costs one memory round trip.  Everything is fp32 on the CUDA cores;
 // inputs may be bf16 (widened exactly).
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(128) bwd_tape_kernel(const BwdArgs b, const Bw
     const T *k = static_cast<const T *>(a.k), *r = static_cast<const T *>(a.r);
     const int chain = blockIdx.x, s = chain / H, h = chain % H;
     const int i = threadIdx.x, warp = i >> 5, lane = i & 31, nw = dk >> 5;
-    const size_t rstride = (size_t)H * dk * sizeof(T), tokstride = (size_t)w.ntok * H * dk;
+    const size_t rstride = (size_t)H * dk * sizeof(T);
     const int rbytes = dk * (int)sizeof(T);
     int t0, t1;
     seq_range(a, s, t0, t1);
@@ -181,10 +182,6 @@ __global__ void __launch_bounds__(128) bwd_tape_kernel(const BwdArgs b, const Bw
         for (int tt = 0; tt < n; ++tt) {
             const size_t e = ((size_t)(tb + tt) * H + h) * dk + i;
             w.g[e] = pm_s[tt * dk + i] * lds(k_s + tt * dk + i) / den_s[tt];
-            b.dq[e] = 0.f;   // the state pass adds its column blocks' shares into these
-            w.part[e] = 0.f;
-            w.part[tokstride + e] = 0.f;
-            w.part[2 * tokstride + e] = 0.f;
         }
         __syncthreads();
     }
@@ -726,80 +723,106 @@ __global__ void __launch_bounds__(512) bwd_prev_scan_kernel(const BwdArgs b, con
 //     r^ = -(g^.g) / den - c^ mu K2 / (d_k r^2);  sigma^ = p^-^ / d_k;  alpha^ = alpha^_S + 2 alpha p p^-^ / d_k
 // The memory state pass is the diagonal one (it only needs g and alpha).  Per-token scalars
 // live in the first 8 floats of the (token, head) row of the P tape:
-//     [0] p before the token, [1] a, [3] K2, [4] the local part of p^-^, [5] the local part of r^, [6] p^-.
+//     [0] p before the token, [1] a, [2] mean sigma (forward), then p^-^ (adjoint), [3] K2,
+//     [4] the local part of p^-^, [5] the local part of r^, [6] p^-, [7] c^ (adjoint).
 namespace {
 constexpr int SC_P = 0, SC_A = 1, SC_K2 = 3, SC_AL = 4, SC_RL = 5, SC_PM = 6;
 }
 
-// dynamic shared memory: channel sums (alpha^2, sigma, k^2) [GT][4]; p^-, den, r [GT]; alpha,
-// sigma, k rows [GT][dk] in the input type
+// The isotropic uncertainty forward in three launches, with the expressions of a serial walk:
+// the channel sums of every (token, head) (one warp each: mean alpha^2, mean sigma and |k|^2 into
+// the token's scalar row); the scalar recursion of each head (one warp per (sequence, head): the
+// lanes load 32 tokens' sums at a time and lane 0 carries p through them), which writes p before
+// the token, p^- and den; then g = p^- k / den for every channel (one warp per (token, head)).
+namespace {
+constexpr int SC_S = 2;   // mean sigma of the token, until SC_PMH takes the slot in the adjoint
+}
+
 template <typename T>
-__global__ void __launch_bounds__(128) bwd_tape_iso_kernel(const BwdArgs b, const BwdWs w)
+__global__ void __launch_bounds__(256) bwd_tape_iso_sums_kernel(const BwdArgs b, const BwdWs w)
 {
-    extern __shared__ float smf[];
     const TokenArgs &a = b.a;
     const int dk = a.dk, H = a.H;
-    float *sum_s = smf, *pm_s = sum_s + 4 * GT, *den_s = pm_s + GT, *r_s = den_s + GT;
-    T *al_s = reinterpret_cast<T *>(r_s + GT), *sg_s = al_s + GT * dk, *k_s = sg_s + GT * dk;
+    const long long th = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (th >= w.ntok * H) return;
     const T *alpha = static_cast<const T *>(a.alpha), *sigma = static_cast<const T *>(a.sigma);
-    const T *k = static_cast<const T *>(a.k), *r = static_cast<const T *>(a.r);
+    const T *k = static_cast<const T *>(a.k);
+    const float inv_dk = 1.f / dk;
+    float xa = 0.f, xs = 0.f, xk = 0.f;
+    for (int c = lane; c < dk; c += 32) {
+        const size_t e = (size_t)th * dk + c;
+        const float al = ldf(alpha + e), kk = ldf(k + e);
+        xa = fmaf(al, al, xa);
+        xs += ldf(sigma + e);
+        xk = fmaf(kk, kk, xk);
+    }
+    xa = warp_sum(xa); xs = warp_sum(xs); xk = warp_sum(xk);
+    if (lane == 0) {
+        float *sc = w.Pprev + (size_t)th * dk;
+        sc[SC_A] = xa * inv_dk;
+        sc[SC_S] = xs * inv_dk;
+        sc[SC_K2] = xk;
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(32) bwd_tape_iso_chain_kernel(const BwdArgs b, const BwdWs w)
+{
+    __shared__ float aa_s[32], s_s[32], k2_s[32], r_s[32], p_s[32];
+    const TokenArgs &a = b.a;
+    const int dk = a.dk, H = a.H;
+    const T *r = static_cast<const T *>(a.r);
     const int chain = blockIdx.x, s = chain / H, h = chain % H;
-    const int i = threadIdx.x, warp = i >> 5, lane = i & 31, nw = dk >> 5;
-    const size_t rstride = (size_t)H * dk * sizeof(T), tokstride = (size_t)w.ntok * H * dk;
-    const int rbytes = dk * (int)sizeof(T);
+    const int lane = threadIdx.x;
     const float inv_dk = 1.f / dk;
     int t0, t1;
     seq_range(a, s, t0, t1);
-    float p = a.P0 ? a.P0[chain] : 1.f;   // thread 0's running uncertainty
-    for (int tb = t0; tb < t1; tb += GT) {
-        const int n = min(GT, t1 - tb);
-        const size_t row0 = ((size_t)tb * H + h) * dk;
-        stage_rows(al_s, alpha + row0, rstride, n, rbytes);
-        stage_rows(sg_s, sigma + row0, rstride, n, rbytes);
-        stage_rows(k_s, k + row0, rstride, n, rbytes);
-        if (i < n) r_s[i] = ldf(r + (size_t)(tb + i) * H + h);
-        cp_async_wait_all();
-        __syncthreads();
-        for (int tt = warp; tt < n; tt += nw) {
-            float xa = 0.f, xs = 0.f, xk = 0.f;
-            for (int c = lane; c < dk; c += 32) {
-                const float al = lds(al_s + tt * dk + c), kk = lds(k_s + tt * dk + c);
-                xa = fmaf(al, al, xa);
-                xs += lds(sg_s + tt * dk + c);
-                xk = fmaf(kk, kk, xk);
-            }
-            xa = warp_sum(xa); xs = warp_sum(xs); xk = warp_sum(xk);
-            if (lane == 0) {
-                sum_s[tt * 4 + 0] = xa * inv_dk;
-                sum_s[tt * 4 + 1] = xs * inv_dk;
-                sum_s[tt * 4 + 2] = xk;
-            }
+    float p = a.P0 ? a.P0[chain] : 1.f;   // lane 0's running uncertainty
+    for (int tb = t0; tb < t1; tb += 32) {
+        const int n = min(32, t1 - tb);
+        if (lane < n) {
+            const size_t th = (size_t)(tb + lane) * H + h;
+            const float *sc = w.Pprev + th * dk;
+            aa_s[lane] = sc[SC_A];
+            s_s[lane] = sc[SC_S];
+            k2_s[lane] = sc[SC_K2];
+            r_s[lane] = ldf(r + th);
         }
-        __syncthreads();
-        if (i == 0) {
+        __syncwarp();
+        if (lane == 0) {
             for (int tt = 0; tt < n; ++tt) {
-                const size_t th = (size_t)(tb + tt) * H + h;
-                const float aa = sum_s[tt * 4 + 0], K2 = sum_s[tt * 4 + 2];
-                const float pm = fmaf(aa, p, sum_s[tt * 4 + 1]);
-                const float den = fmaf(pm, K2, r_s[tt]);
-                float *sc = w.Pprev + th * dk;
-                sc[SC_P] = p; sc[SC_A] = aa; sc[SC_K2] = K2; sc[SC_PM] = pm;
-                w.den[th] = den;
-                pm_s[tt] = pm;
-                den_s[tt] = den;
-                p = pm / fmaf(a.mu * K2 * inv_dk / r_s[tt], pm, 1.f);
+                p_s[tt] = p;
+                const float pm = fmaf(aa_s[tt], p, s_s[tt]);
+                p = pm / fmaf(a.mu * k2_s[tt] * inv_dk / r_s[tt], pm, 1.f);
             }
         }
-        __syncthreads();
-        for (int tt = 0; tt < n; ++tt) {
-            const size_t e = ((size_t)(tb + tt) * H + h) * dk + i;
-            w.g[e] = pm_s[tt] * lds(k_s + tt * dk + i) / den_s[tt];
-            b.dq[e] = 0.f;   // the state pass adds its column blocks' shares into these
-            w.part[e] = 0.f;
-            w.part[tokstride + e] = 0.f;
-            w.part[2 * tokstride + e] = 0.f;
+        __syncwarp();
+        if (lane < n) {
+            const size_t th = (size_t)(tb + lane) * H + h;
+            float *sc = w.Pprev + th * dk;
+            const float pm = fmaf(aa_s[lane], p_s[lane], s_s[lane]);
+            sc[SC_P] = p_s[lane];
+            sc[SC_PM] = pm;
+            w.den[th] = fmaf(pm, k2_s[lane], r_s[lane]);
         }
-        __syncthreads();
+        __syncwarp();
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_tape_iso_gain_kernel(const BwdArgs b, const BwdWs w)
+{
+    const TokenArgs &a = b.a;
+    const int dk = a.dk, H = a.H;
+    const long long th = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (th >= w.ntok * H) return;
+    const T *k = static_cast<const T *>(a.k);
+    const float pm = w.Pprev[(size_t)th * dk + SC_PM], den = w.den[th];
+    for (int c = lane; c < dk; c += 32) {
+        const size_t e = (size_t)th * dk + c;
+        w.g[e] = pm * ldf(k + e) / den;
     }
 }
 
@@ -845,56 +868,96 @@ __global__ void __launch_bounds__(256) bwd_local_iso_kernel(const BwdArgs b, con
     }
 }
 
-// dynamic shared memory, per group of GT tokens: local k^, alpha^_S [GT][dk] fp32; tape scalars
-// [GT][8]; 1/r [GT]; alpha, k rows [GT][dk] in the input type
+// The isotropic uncertainty adjoint in two launches.  Its serial part is a scalar per head, so
+// one warp per (sequence, head) walks it: the lanes form the per-token terms of 32 tokens at a
+// time (z, the head's a, the local part of p^-^), lane 0 carries p^ through them (two dependent
+// operations per token), and the lanes then write p^-^ and c^ of their tokens (slots SC_PMH,
+// SC_CH of the token's scalar row) and dr.  A second launch, one warp per (token, head), forms
+// dk, dsigma and dalpha of every channel.  The expressions are the one-CTA-per-head kernel's.
+namespace {
+constexpr int SC_PMH = 2, SC_CH = 7;
+}
+
 template <typename T>
-__global__ void __launch_bounds__(128) bwd_prev_iso_kernel(const BwdArgs b, const BwdWs w)
+__global__ void __launch_bounds__(32) bwd_prev_iso_chain_kernel(const BwdArgs b, const BwdWs w)
 {
-    extern __shared__ float smf[];
+    __shared__ float z_s[32], aa_s[32], al_s[32], ph_s[32];
     const TokenArgs &a = b.a;
     const int dk = a.dk, H = a.H;
-    float *K_s = smf, *aS_s = K_s + GT * dk, *sc_s = aS_s + GT * dk, *ir_s = sc_s + 8 * GT;
-    T *al_s = reinterpret_cast<T *>(ir_s + GT), *k_s = al_s + GT * dk;
-    const T *alpha = static_cast<const T *>(a.alpha), *k = static_cast<const T *>(a.k);
     const T *r = static_cast<const T *>(a.r);
     const int chain = blockIdx.x, s = chain / H, h = chain % H;
-    const int i = threadIdx.x;
+    const int lane = threadIdx.x;
     const float mu = a.mu, inv_dk = 1.f / dk;
-    const size_t tokstride = (size_t)w.ntok * H * dk;
-    const size_t rstride = (size_t)H * dk * sizeof(T), fstride = (size_t)H * dk * 4;
     int t0, t1;
     seq_range(a, s, t0, t1);
-    float ph = b.dP_T ? b.dP_T[chain] : 0.f;
-    for (int te = t1; te > t0; te -= GT) {
-        const int tb = max(t0, te - GT), n = te - tb;
-        const size_t row0 = ((size_t)tb * H + h) * dk;
-        stage_rows(K_s, w.part + tokstride + row0, fstride, n, dk * 4);
-        stage_rows(aS_s, w.part + 2 * tokstride + row0, fstride, n, dk * 4);
-        stage_rows(sc_s, w.Pprev + row0, fstride, n, 32);
-        stage_rows(al_s, alpha + row0, rstride, n, dk * (int)sizeof(T));
-        stage_rows(k_s, k + row0, rstride, n, dk * (int)sizeof(T));
-        if (i < n) ir_s[i] = 1.f / ldf(r + (size_t)(tb + i) * H + h);
-        cp_async_wait_all();
-        __syncthreads();
-        for (int tt = n - 1; tt >= 0; --tt) {
-            const size_t th = (size_t)(tb + tt) * H + h, e = th * dk + i;
-            const float *sc = sc_s + tt * 8;
-            const float pp = sc[SC_P], aa = sc[SC_A], K2 = sc[SC_K2], pm = sc[SC_PM], ir = ir_s[tt];
-            const float mk = mu * inv_dk * ir;            // mu / (d_k r)
+    float ph = b.dP_T ? b.dP_T[chain] : 0.f;   // lane 0's running p^
+    for (int te = t1; te > t0; te -= 32) {
+        const int tb = max(t0, te - 32), n = te - tb;
+        float pt = 0.f, mk = 0.f, K2 = 0.f, ir = 0.f;
+        float *sc = nullptr;
+        if (lane < n) {
+            const size_t th = (size_t)(tb + lane) * H + h;
+            sc = w.Pprev + th * dk;
+            const float aa = sc[SC_A], pm = sc[SC_PM];
+            K2 = sc[SC_K2];
+            ir = 1.f / ldf(r + th);
+            mk = mu * inv_dk * ir;
             const float z = 1.f / fmaf(mk * K2, pm, 1.f);
-            const float pt = pm * z;
-            const float pmh = sc[SC_AL] + ph * z * z;
-            const float ch = -ph * pt * pt;
-            const float al = lds(al_s + tt * dk + i), kk = lds(k_s + tt * dk + i);
-            b.dk[e] = K_s[tt * dk + i] + ch * 2.f * mk * kk;
-            b.dsigma[e] = pmh * inv_dk;
-            b.dalpha[e] = aS_s[tt * dk + i] + 2.f * al * pp * pmh * inv_dk;
-            if (i == 0) b.dr[th] = sc[SC_RL] - ch * mk * K2 * ir;
-            ph = aa * pmh;
+            pt = pm * z;
+            z_s[lane] = z;
+            aa_s[lane] = aa;
+            al_s[lane] = sc[SC_AL];
         }
-        __syncthreads();
+        __syncwarp();
+        if (lane == 0) {
+            for (int tt = n - 1; tt >= 0; --tt) {
+                ph_s[tt] = ph;
+                const float z = z_s[tt];
+                const float pmh = al_s[tt] + ph * z * z;
+                ph = aa_s[tt] * pmh;
+            }
+        }
+        __syncwarp();
+        if (lane < n) {
+            const float p_in = ph_s[lane], z = z_s[lane];
+            const float pmh = al_s[lane] + p_in * z * z;
+            const float ch = -p_in * pt * pt;
+            sc[SC_PMH] = pmh;
+            sc[SC_CH] = ch;
+            b.dr[(size_t)(tb + lane) * H + h] = sc[SC_RL] - ch * mk * K2 * ir;
+        }
+        __syncwarp();
     }
-    if (b.dP0 && i == 0) b.dP0[chain] = ph;
+    if (b.dP0 && lane == 0) b.dP0[chain] = ph;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_prev_iso_out_kernel(const BwdArgs b, const BwdWs w)
+{
+    const TokenArgs &a = b.a;
+    const int dk = a.dk, H = a.H;
+    const long long th = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (th >= w.ntok * H) return;
+    const T *alpha = static_cast<const T *>(a.alpha), *k = static_cast<const T *>(a.k);
+    const T *r = static_cast<const T *>(a.r);
+    const size_t tokstride = (size_t)w.ntok * H * dk;
+    const float *sc = w.Pprev + (size_t)th * dk;
+    const float mu = a.mu, inv_dk = 1.f / dk;
+    const float pp = sc[SC_P], pmh = sc[SC_PMH], ch = sc[SC_CH];
+    const float ir = 1.f / ldf(r + th);
+    const float mk = mu * inv_dk * ir;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int c = lane + 32 * m;
+        if (c < dk) {
+            const size_t e = (size_t)th * dk + c;
+            const float al = ldf(alpha + e), kk = ldf(k + e);
+            b.dk[e] = w.part[tokstride + e] + ch * 2.f * mk * kk;
+            b.dsigma[e] = pmh * inv_dk;
+            b.dalpha[e] = w.part[2 * tokstride + e] + 2.f * al * pp * pmh * inv_dk;
+        }
+    }
 }
 
 // ================================================================= host
@@ -935,7 +998,7 @@ static cudaError_t set_smem(const void *kern, size_t smem) {
 
 // The uncertainty forward as the chunk-parallel gain scan (bf16, d_k = 128, diagonal): P before
 // each token, g and den, with its look-back words in the checkpoint region (written by the
-// state pass only later); then the four sums the state pass adds into are cleared.
+// state pass only later).
 static cudaError_t launch_tape_scan(const BwdArgs &b, const BwdWs &w, int nchunks_max, cudaStream_t st) {
     const TokenArgs &a = b.a;
     ScanArgs sa{};
@@ -943,10 +1006,6 @@ static cudaError_t launch_tape_scan(const BwdArgs &b, const BwdWs &w, int nchunk
     sa.g = w.g; sa.P_prev = w.Pprev; sa.den = w.den;
     sa.cu = a.cu; sa.T = a.T; sa.nseq = a.nseq; sa.H = a.H; sa.dk = a.dk; sa.mu = a.mu;
     sa.nchunks_max = nchunks_max; sa.nchains = a.nseq * a.H; sa.err = a.err;
-    const size_t th = (size_t)w.ntok * a.H;
-    cudaError_t e = cudaMemsetAsync(b.dq, 0, th * a.dk * 4, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(w.part, 0, 3 * th * a.dk * 4, st);
-    if (e != cudaSuccess) return e;
     return launch_gain_scan_tma(sa, w.ntok, w.ckpt, st);
 }
 
@@ -984,15 +1043,25 @@ template <typename T>
 static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, bool tape_scan, bool prev_scan,
                                     int nchunks_max, cudaStream_t st) {
     const int chains = b.a.nseq * b.a.H, dk = b.a.dk;
-    cudaError_t e;
+    // the state pass adds its column blocks' shares into dq and the three sums
+    const size_t thd = (size_t)w.ntok * b.a.H * dk * 4;
+    cudaError_t e = cudaMemsetAsync(b.dq, 0, thd, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(w.part, 0, 3 * thd, st);
+    if (e != cudaSuccess) return e;
     if (tape_scan) {
         e = launch_tape_scan(b, w, nchunks_max, st);
         if (e != cudaSuccess) return e;
     } else if (b.a.iso) {
-        const size_t tsm = (size_t)7 * GT * sizeof(float) + (size_t)3 * GT * dk * sizeof(T);
-        e = set_smem(reinterpret_cast<const void *>(bwd_tape_iso_kernel<T>), tsm);
-        if (e != cudaSuccess) return e;
-        bwd_tape_iso_kernel<T><<<chains, dk, tsm, st>>>(b, w);
+        const long long rows = w.ntok * b.a.H;
+        if (rows > 0) {
+            bwd_tape_iso_sums_kernel<T><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(b, w);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+            bwd_tape_iso_chain_kernel<T><<<chains, 32, 0, st>>>(b, w);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+            bwd_tape_iso_gain_kernel<T><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(b, w);
+        }
     } else {
         const size_t tsm = ((size_t)2 * GT * dk + 4 * GT) * sizeof(float) + (size_t)3 * GT * dk * sizeof(T);
         e = set_smem(reinterpret_cast<const void *>(bwd_tape_kernel<T>), tsm);
@@ -1011,10 +1080,11 @@ static cudaError_t launch_bwd_typed(const BwdArgs &b, const BwdWs &w, bool tape_
     e = launch_local<T>(b, w, st);
     if (e != cudaSuccess) return e;
     if (b.a.iso) {
-        const size_t psm = ((size_t)2 * GT * dk + 9 * GT) * sizeof(float) + (size_t)2 * GT * dk * sizeof(T);
-        e = set_smem(reinterpret_cast<const void *>(bwd_prev_iso_kernel<T>), psm);
+        bwd_prev_iso_chain_kernel<T><<<chains, 32, 0, st>>>(b, w);
+        e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        bwd_prev_iso_kernel<T><<<chains, dk, psm, st>>>(b, w);
+        const long long rows = w.ntok * b.a.H;
+        if (rows > 0) bwd_prev_iso_out_kernel<T><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(b, w);
         return cudaGetLastError();
     }
     if (prev_scan) return launch_prev_scan<T>(b, w, nchunks_max, st);
