@@ -221,7 +221,8 @@ kdn_status_t kdn_gain_scan_noalloc(const kdn_problem_t *p,
  * the uncertainty adjoint (diagonal variant) run as chunk-parallel scans with decoupled
  * look-back whenever their work lists (N x H x the chunks of the longest sequence) fit the
  * checkpoint region, else as one serial walk per (sequence, head); both give the same result
- * to fp32 rounding.  The d_v column blocks of a (sequence, head)
+ * to fp32 rounding.  The isotropic variant's scalar uncertainty walks run one warp per
+ * (sequence, head) between per-token parallel launches.  The d_v column blocks of a (sequence, head)
  * add their shares of the sums over d_v with atomic adds, so the last bits of every gradient
  * except dv and dS0 can differ from run to run.  Workspace: about 7.0 KB per token and head
  * at d_k = d_v = 128.  Every pointer 16-byte aligned.  Outputs may not alias inputs.
