@@ -343,18 +343,18 @@ def bench_prefill(args, world, rank, dev, kdn):
         scan = dict(value=world * w.ntok / (s_ms / 1e3), ms_step=s_ms, bytes=s_bytes, launches=args.steps)
 
     # the backward pass (gradients of <o, d_o> with respect to every input, S0 and P0) on the
-    # same inputs, d_o drawn once on the device
-    bwd = None
-    if not args.no_backward:
+    # same inputs, d_o drawn once on the device; both uncertainty variants
+    def bwd_leg(variant):
         gen = torch.Generator(device=dev)
         gen.manual_seed(1234 + rank)
         d_o = torch.randn(o.shape, generator=gen, device=dev).to(o.dtype)
         f32 = dict(dtype=torch.float32, device=dev)
+        p_shape = (w.num_seqs, w.H) + ((w.dk,) if variant == "diagonal" else ())
         grads = dict(dq=torch.empty(d["q"].shape, **f32), dk=torch.empty(d["k"].shape, **f32),
                      dv=torch.empty(d["v"].shape, **f32), dalpha=torch.empty(d["alpha"].shape, **f32),
                      dsigma=torch.empty(d["sigma"].shape, **f32), dr=torch.empty(d["r"].shape, **f32),
-                     dS0=torch.empty((w.num_seqs, w.H, w.dk, w.dv), **f32), dP0=torch.empty((w.num_seqs, w.H, w.dk), **f32))
-        bp = kdn.make_problem(d["q"], d["v"], cu_seqlens=cu, mu=w.mu, chunk=0)
+                     dS0=torch.empty((w.num_seqs, w.H, w.dk, w.dv), **f32), dP0=torch.empty(p_shape, **f32))
+        bp = kdn.make_problem(d["q"], d["v"], cu_seqlens=cu, mu=w.mu, chunk=0, max_seqlen=max_seqlen, variant=variant)
         ws_bwd = torch.empty(kdn.kdn_backward_workspace_size(bp), dtype=torch.uint8, device=dev)
         bargs = [d[n].data_ptr() for n in names]
         gptr = [grads[n].data_ptr() for n in ("dq", "dk", "dv", "dalpha", "dsigma", "dr", "dS0", "dP0")]
@@ -382,13 +382,18 @@ def bench_prefill(args, world, rank, dev, kdn):
         b_ms = max_over_ranks(b0.elapsed_time(b1), world) / n_bwd
         esz = 2 if w.bf16 else 4
         b_bytes = (w.ntok * w.H * ((4 * w.dk + 2 * w.dv + 1) * esz + (4 * w.dk + w.dv + 1) * 4)
-                   + w.num_seqs * w.H * (w.dk * w.dv + w.dk) * 4)
+                   + w.num_seqs * w.H * (w.dk * w.dv + (w.dk if variant == "diagonal" else 1)) * 4)
         del ws_bwd
-        bwd = dict(value=world * w.ntok / (b_ms / 1e3), ms_step=b_ms, bytes=b_bytes, launches=4 * n_bwd)
+        return dict(value=world * w.ntok / (b_ms / 1e3), ms_step=b_ms, bytes=b_bytes, variant=variant)
+
+    bwd = bwd_iso = None
+    if not args.no_backward:
+        bwd = bwd_leg("diagonal")
+        bwd_iso = bwd_leg("isotropic")
 
     nbytes = algorithmic_bytes(w)
     return dict(w=w, value=value, ms_step=ms_step, per_step_ms=per_step_ms, clocks=clk.summary(), path=path, scan=scan,
-                iso=iso, bwd=bwd,
+                iso=iso, bwd=bwd, bwd_iso=bwd_iso,
                 e2e=dict(value=e2e_value, unit="tokens/s", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
                          steps=e_steps),
                 bytes=nbytes, launches=args.steps * launches_per_step)
@@ -591,16 +596,17 @@ def ours(args):
                                  "roofline": {"bound": "hbm", "achieved": sach, "peak": hbm, "unit": "GB/s",
                                               "frac": sach / hbm, "traffic": None,
                                               "algorithmic_bytes_per_launch": sc["bytes"]}}
-        if pre["bwd"] is not None:
-            bw = pre["bwd"]
+        for key, bw, launches in (("backward", pre["bwd"], 4), ("backward_isotropic", pre["bwd_iso"], 7)):
+            if bw is None:
+                continue
             bach = bw["bytes"] / (bw["ms_step"] / 1e3) / 1e9
-            line["backward"] = {"metric": "backward tokens/s (gradients of o w.r.t. q, k, v, alpha, sigma, r, S0, P0)",
-                                "value": bw["value"], "unit": "tokens/s", "ms_per_step": bw["ms_step"],
-                                "gpu_launches": bw["launches"], "dtype": "f32 (bf16 inputs widened)",
-                                "roofline": {"bound": "hbm", "achieved": bach, "peak": hbm, "unit": "GB/s",
-                                             "frac": bach / hbm, "traffic": None,
-                                             "algorithmic_bytes_per_launch": bw["bytes"],
-                                             "unit_of_measure": "one backward call = its four launches"}}
+            line[key] = {"metric": f"{bw['variant']} backward tokens/s (gradients of o w.r.t. q, k, v, alpha, sigma, r, S0, P0)",
+                         "value": bw["value"], "unit": "tokens/s", "ms_per_step": bw["ms_step"],
+                         "gpu_launches": 3 * launches, "dtype": "f32 (bf16 inputs widened)",
+                         "roofline": {"bound": "hbm", "achieved": bach, "peak": hbm, "unit": "GB/s",
+                                      "frac": bach / hbm, "traffic": None,
+                                      "algorithmic_bytes_per_launch": bw["bytes"],
+                                      "unit_of_measure": f"one backward call = its {launches} launches"}}
         for ot in others:
             oach = ot["bytes"] / (ot["ms_per_step"] / 1e3) / 1e9
             key = "prefill_long" if ot["workload"].startswith("long") else "prefill_varlen"
